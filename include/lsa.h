@@ -1,0 +1,230 @@
+/*
+ * lsa.h -- C-ABI of liblsa: the D-LSA Flat hot path (content index, bucket
+ * retrieval, exact sparse attention) as hand-written CUDA kernels for B200
+ * (sm_100a).
+ *
+ * Method sources (web pages about arXiv 2610.42147):
+ *   "Latent Sparse Attention: un indice gerarchico per contesti lunghi",
+ *     paragraph on index construction: consecutive keys are pooled in small
+ *     groups, the pooled sequence is split into blocks, each block groups
+ *     similar representations into buckets that keep a centroid and the
+ *     indices of the original keys;
+ *     paragraph on retrieval: the query is compared with the centroids to
+ *     choose buckets; attention then runs over the selected keys and values;
+ *     paragraph on the read budget: a 64-dimensional index; each query reads
+ *     4096 long-range keys outside the recent window, the 512 most recent keys
+ *     and 4 sink keys (2048 long-range keys for GLM below position 1M).
+ *   "Prefrontal's Latent Sparse Attention speeds up one attention layer 72x at
+ *     10M tokens; end to end, the gain is 9x", section "What it changes": the
+ *     attention kernel itself is unchanged; LSA only decides which keys are
+ *     read.  Section "The numbers, and which ones to quote": the timed unit is
+ *     the last 32k query chunk of a 10M-token context.
+ *
+ * Conventions for every call
+ *   - Status: every call returns lsa_status; nothing is thrown or aborted
+ *     across the ABI.  lsa_last_error() returns a thread-local description of
+ *     the last failure on the calling thread.
+ *   - Arguments are checked on the host before any launch.  A failed check
+ *     launches nothing and returns LSA_ERR_INVALID_ARG (or LSA_ERR_ALIGNMENT /
+ *     LSA_ERR_WORKSPACE).
+ *   - Memory: every tensor pointer is a DEVICE pointer owned by the caller.
+ *     The library never allocates device memory: index storage and scratch
+ *     are caller buffers sized by lsa_index_bytes / lsa_*_workspace_bytes.
+ *     Device pointers must be 16-byte aligned.
+ *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *     default stream).  All work is enqueued asynchronously; outputs are
+ *     valid once the stream has been synchronised.  No call synchronises the
+ *     stream, so every call can be captured in a CUDA graph (except
+ *     lsa_index_check, which reads back a status word).
+ *   - Layouts (row-major, innermost last):
+ *       latent keys   latent_K [B][T_cap][64]
+ *       keys, values  K, V     [B][T_cap][Hkv][d]   (token-major: one key of
+ *                                                   all KV heads is contiguous)
+ *       latent query  latent_Q [B][Nq][64]
+ *       query         Q        [B][Nq][Hq][d]
+ *       output        O        [B][Nq][Hq][d]       (same dtype as Q)
+ *       selection     indices  [B][Nq][s_max] int32, -1 padded
+ *                     counts   [B][Nq] int32
+ *     T_cap is the per-sequence capacity given to lsa_index_init; every
+ *     per-sequence cache uses it as its sequence stride.
+ *   - Dtypes: LSA_F32 or LSA_BF16, uniform for the index and the call.
+ *     Positions and indices are int32 (T_cap <= 2^31 - 1); device offsets are
+ *     64-bit internally.
+ *   - Shapes supported by the kernels: latent dim 64; d in {64, 128};
+ *     Hq % Hkv == 0 with Hq / Hkv in {1, 2, 4, 8}.
+ */
+#ifndef LSA_H
+#define LSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LSA_OK = 0,
+    LSA_ERR_INVALID_ARG = 1, /* a size, shape, pointer or parameter is invalid */
+    LSA_ERR_ALIGNMENT = 2,   /* a pointer is not 16-byte aligned */
+    LSA_ERR_WORKSPACE = 3,   /* a caller buffer is smaller than required */
+    LSA_ERR_CUDA = 4,        /* a CUDA runtime call failed (message in lsa_last_error) */
+    LSA_ERR_TIMEOUT = 5,     /* a bounded device wait gave up (status word) */
+    LSA_ERR_INTERNAL = 6,    /* a device-side consistency check failed (status word) */
+    LSA_ERR_UNSUPPORTED = 7  /* valid request outside what the kernels implement */
+} lsa_status;
+
+typedef enum { LSA_F32 = 0, LSA_BF16 = 1 } lsa_dtype;
+
+/* Index parameters.  p: keys per pooled group; block: pooled groups per block
+ * (G); n_buckets: buckets per block (k); lloyd_iters: Lloyd iterations (L). */
+typedef struct {
+    int p;
+    int block;
+    int n_buckets;
+    int lloyd_iters;
+} lsa_index_params;
+
+/* Read budget.  budget: long-range keys R; window: recent keys W; sinks: S. */
+typedef struct {
+    int budget;
+    int window;
+    int sinks;
+} lsa_select_params;
+
+/* Opaque host handle over caller-owned index storage. */
+typedef struct lsa_index lsa_index;
+
+/* Thread-local text of the last failure on this thread ("" if none). */
+const char* lsa_last_error(void);
+
+/* Library version string. */
+const char* lsa_version(void);
+
+/* ---------------------------------------------------------------------------
+ * Content index  ("un indice gerarchico", paragraph on index construction)
+ *
+ * Per sequence: pooled groups j = 0 .. T/p - 1 (keys jp .. jp+p-1, mean of
+ * their latent keys, summed left to right in binary32 then divided by p);
+ * unit vectors u_j = x_j / ||x_j|| (norm from a binary64 sum of squares);
+ * block b = pooled groups [bG, (b+1)G); inside each block spherical k-means
+ * into k buckets: c_m initialised to u[bG + floor(m*G/k)], then L times
+ * {assign each u to the bucket of largest <u, c_m> (exact products summed in
+ * binary64 in ascending dimension; ties to the lowest m); c_m = normalised
+ * binary64 sum of its members in ascending order, an empty bucket keeps its
+ * centroid}.  Bucket records: global bucket g = b*k + m, CSR offsets and
+ * members (pooled ids, ascending).  Retrieval copy of the centroids: bf16
+ * (round to nearest even) for LSA_BF16 indices, fp32 otherwise.
+ * Completed pooled groups after the last whole block ("open block") are
+ * assigned to the bucket of their nearest closed centroid (decode append).
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of device storage for an index of B sequences with capacity T_cap
+ * keys each.  Returns 0 on invalid arguments (see lsa_last_error). */
+size_t lsa_index_bytes(int64_t B, int64_t T_cap, lsa_index_params ip, lsa_dtype dtype);
+
+/* Creates a host handle over `buf` (device, >= lsa_index_bytes, 256-byte
+ * aligned) and records the parameters.  The index starts empty (0 blocks);
+ * storage is not touched until the first build/extend.  *out must be released
+ * with lsa_index_release; the device buffer stays owned by the caller. */
+lsa_status lsa_index_init(void* buf, size_t bytes, int64_t B, int64_t T_cap, lsa_index_params ip,
+                          lsa_dtype dtype, lsa_index** out);
+
+/* Frees the host handle only. */
+void lsa_index_release(lsa_index* idx);
+
+/* Builds the index over keys [0, T) of every sequence: same as
+ * lsa_index_extend(idx, latent_K, 0, T, stream). */
+lsa_status lsa_build_index(lsa_index* idx, const void* latent_K, int64_t T, void* stream);
+
+/* (Re)clusters every whole block overlapping [T_old, T_new) (blocks
+ * floor(T_old/(pG)) .. floor(T_new/(pG)) - 1), then resets the open block and
+ * assigns its completed pooled groups below T_new.  Requires
+ * floor(T_old/(pG)) <= current block count (no gap) and T_new <= T_cap.
+ * Rebuilding a block from the same keys reproduces it bit for bit. */
+lsa_status lsa_index_extend(lsa_index* idx, const void* latent_K, int64_t T_old, int64_t T_new,
+                            void* stream);
+
+/* Number of closed blocks currently indexed (host-side counter). */
+int64_t lsa_index_num_blocks(const lsa_index* idx);
+
+/* Copies the index state to caller DEVICE buffers (any may be NULL):
+ * pooled/unit [B][T_cap/p][64] f32, cent [B][nblk_max*k][64] f32,
+ * cent_rt [B][nblk_max*k][64] (dtype of the index), offsets
+ * [B][nblk_max*k + 1] i32, members [B][T_cap/p] i32, assign [B][T_cap/p] i16,
+ * open_bucket [B][G] i32 (-1 = not assigned). */
+lsa_status lsa_index_export(const lsa_index* idx, float* pooled, float* unit, float* cent,
+                            void* cent_rt, int32_t* offsets, int32_t* members, int16_t* assign,
+                            int32_t* open_bucket, void* stream);
+
+/* Reads and clears the index's device status word (synchronises `stream`).
+ * Returns LSA_OK, or the error recorded by a kernel since the last check
+ * (for example LSA_ERR_INTERNAL when a decode step found its open block full);
+ * *fallbacks (nullable) receives the number of queries that took the exact
+ * selection fallback since the last check. */
+lsa_status lsa_index_check(lsa_index* idx, int64_t* fallbacks, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Retrieval  ("un indice gerarchico", paragraphs on retrieval and on the
+ * read budget)
+ *
+ * Query at position pos with latent q: s_g = <q, c~_g> over every closed
+ * bucket; buckets ranked by (s desc, g asc); key t of bucket g is available
+ * iff S <= t <= pos - W; long-range keys are filled greedily up to R: whole
+ * buckets' available keys while they fit, then the first `rem` available keys
+ * of the next bucket in ascending position.  Emitted row: sinks
+ * [0, min(S, pos+1)), long-range keys in take order, window
+ * [max(pos-W+1, min(S,pos+1)), pos]; the rest -1.  The scores are those of
+ * exact products summed in binary64, so the selection is reproducible bit
+ * for bit (approximate tensor-core scores only nominate candidates; a query
+ * whose candidates cannot prove the exact ranking takes an exact fallback).
+ * ------------------------------------------------------------------------- */
+
+/* Workspace bytes for lsa_select on Nq queries per sequence. */
+size_t lsa_select_workspace_bytes(const lsa_index* idx, int64_t Nq);
+
+/* latent_Q [B][Nq][64] (index dtype), positions [B][Nq] int32 device (each
+ * 0 <= pos < T_cap; keys below pos-W+1 must be indexed or in the open lists),
+ * indices [B][Nq][s_max] with s_max >= budget+window+sinks, counts [B][Nq]. */
+lsa_status lsa_select(const lsa_index* idx, const void* latent_Q, const int32_t* positions,
+                      int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
+                      int s_max, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Exact sparse attention ("Prefrontal's ...", section "What it changes")
+ *
+ * For query (b, i) and head h with KV head kh = h / (Hq/Hkv):
+ *   o = softmax_t(scale * <Q_h, K_{t,kh}>) V_{t,kh}
+ * over t = indices[b][i][0 .. counts[b][i]).  fp32 softmax and accumulation;
+ * bf16 inputs use tensor-core MMA.  lse (nullable) [B][Nq][Hq] f32 receives
+ * max + ln(sum) of the scaled logits.  counts must be >= 1 and every listed
+ * index in [0, T_cap).
+ * ------------------------------------------------------------------------- */
+lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtype dtype,
+                           int64_t B, int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
+                           const int32_t* indices, const int32_t* counts, int s_max, float scale,
+                           void* O, float* lse, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Fused entries
+ * ------------------------------------------------------------------------- */
+
+/* Workspace bytes for lsa_prefill_chunk with Nq = T_new - T_old queries. */
+size_t lsa_prefill_workspace_bytes(const lsa_index* idx, int64_t Nq, lsa_select_params sp);
+
+/* One prefill chunk ("Prefrontal's ...", section "The numbers, and which ones
+ * to quote": prefilling the last query chunk of a long context).  Queries are
+ * the positions [T_old, T_new) of every sequence.  Steps: lsa_index_extend
+ * over [T_old, T_new), selection for every chunk query, sparse attention with
+ * scale 1/sqrt(d).  latent_Q [B][Nq][64], Q and O [B][Nq][Hq][d]; the caches
+ * already hold keys [0, T_new).  The selection is written to the workspace. */
+lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* latent_Q,
+                             const void* Q, const void* K, const void* V, int64_t T_old,
+                             int64_t T_new, int Hq, int Hkv, int d, lsa_select_params sp,
+                             void* workspace, size_t ws_bytes, void* O, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H */

@@ -1,0 +1,281 @@
+"""Python binding of liblsa, the D-LSA Flat hot path for B200 (sm_100a).
+
+Argument marshalling only: every step of the path runs in liblsa's CUDA
+kernels.  PyTorch provides device memory and streams.  The names mirror the
+C-ABI in include/lsa.h; see that header for the semantics of every call.
+
+Method: Latent Sparse Attention in its D-LSA Flat form ("Latent Sparse
+Attention: un indice gerarchico per contesti lunghi", paragraphs on index
+construction, retrieval and the read budget; "Prefrontal's Latent Sparse
+Attention speeds up one attention layer 72x at 10M tokens ...", section
+"What it changes").
+"""
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "LsaError", "LsaIndex", "lsa_index_bytes", "lsa_build_index", "lsa_select",
+    "lsa_sparse_attn", "lsa_prefill_chunk", "lsa_prefill_workspace_bytes",
+    "library_path", "F32", "BF16",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liblsa.so")
+
+F32, BF16 = 0, 1
+_STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID_ARG", 2: "LSA_ERR_ALIGNMENT", 3: "LSA_ERR_WORKSPACE",
+           4: "LSA_ERR_CUDA", 5: "LSA_ERR_TIMEOUT", 6: "LSA_ERR_INTERNAL",
+           7: "LSA_ERR_UNSUPPORTED"}
+
+
+class LsaError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__("%s: %s" % (_STATUS.get(code, str(code)), msg))
+        self.code = code
+
+
+class IndexParams(ctypes.Structure):
+    _fields_ = [("p", ctypes.c_int), ("block", ctypes.c_int), ("n_buckets", ctypes.c_int),
+                ("lloyd_iters", ctypes.c_int)]
+
+
+class SelectParams(ctypes.Structure):
+    _fields_ = [("budget", ctypes.c_int), ("window", ctypes.c_int), ("sinks", ctypes.c_int)]
+
+
+def _declare(lib):
+    P, I, I64, SZ, F = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t,
+                        ctypes.c_float)
+    sigs = {
+        "lsa_last_error": ([], ctypes.c_char_p),
+        "lsa_version": ([], ctypes.c_char_p),
+        "lsa_index_bytes": ([I64, I64, IndexParams, I], SZ),
+        "lsa_index_init": ([P, SZ, I64, I64, IndexParams, I, ctypes.POINTER(P)], I),
+        "lsa_index_release": ([P], None),
+        "lsa_build_index": ([P, P, I64, P], I),
+        "lsa_index_extend": ([P, P, I64, I64, P], I),
+        "lsa_index_num_blocks": ([P], I64),
+        "lsa_index_export": ([P, P, P, P, P, P, P, P, P, P], I),
+        "lsa_index_check": ([P, ctypes.POINTER(I64), P], I),
+        "lsa_select_workspace_bytes": ([P, I64], SZ),
+        "lsa_select": ([P, P, P, I64, SelectParams, P, P, I, P, SZ, P], I),
+        "lsa_sparse_attn": ([P, P, P, I, I64, I64, I64, I, I, I, P, P, I, F, P, P, P], I),
+        "lsa_prefill_workspace_bytes": ([P, I64, SelectParams], SZ),
+        "lsa_prefill_chunk": ([P, P, P, P, P, P, I64, I64, I, I, I, SelectParams, P, SZ, P, P],
+                              I),
+    }
+    for name, (args, res) in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError("liblsa.so is not built; run `python -m long_context_indexing_b200._build`"
+                          " (or __graft_entry__.build())")
+    return _declare(ctypes.CDLL(_LIB_PATH))
+
+
+_lib = _load()
+
+
+def library_path():
+    return _LIB_PATH
+
+
+def _check(rc):
+    if rc != 0:
+        raise LsaError(rc, _lib.lsa_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError("tensors must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def lsa_index_bytes(B, T_cap, p, block, n_buckets, lloyd_iters, dtype=BF16):
+    n = _lib.lsa_index_bytes(B, T_cap, IndexParams(p, block, n_buckets, lloyd_iters), dtype)
+    if n == 0:
+        raise LsaError(1, _lib.lsa_last_error().decode())
+    return n
+
+
+class LsaIndex:
+    """A D-LSA Flat content index over B sequences of capacity T_cap keys.
+
+    The device storage is one torch uint8 buffer owned by this object; the
+    library only records pointers into it."""
+
+    def __init__(self, B, T_cap, p, block, n_buckets, lloyd_iters, dtype=BF16, device="cuda"):
+        self.B, self.T_cap = int(B), int(T_cap)
+        self.p, self.G, self.k, self.L = int(p), int(block), int(n_buckets), int(lloyd_iters)
+        self.dtype = dtype
+        self.params = IndexParams(self.p, self.G, self.k, self.L)
+        nbytes = lsa_index_bytes(self.B, self.T_cap, self.p, self.G, self.k, self.L, dtype)
+        self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        h = ctypes.c_void_p()
+        _check(_lib.lsa_index_init(_ptr(self.buffer), nbytes, self.B, self.T_cap, self.params,
+                                   dtype, ctypes.byref(h)))
+        self._h = h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            _lib.lsa_index_release(h)
+            self._h = None
+
+    @property
+    def handle(self):
+        return self._h
+
+    @property
+    def num_blocks(self):
+        return int(_lib.lsa_index_num_blocks(self._h))
+
+    @property
+    def n_pooled(self):
+        return self.T_cap // self.p
+
+    @property
+    def n_buckets_max(self):
+        return (self.n_pooled // self.G) * self.k
+
+    def build(self, latent_K, T, stream=None):
+        _cuda(latent_K)
+        _check(_lib.lsa_build_index(self._h, _ptr(latent_K), int(T), _stream(stream)))
+        return self
+
+    def extend(self, latent_K, T_old, T_new, stream=None):
+        _cuda(latent_K)
+        _check(_lib.lsa_index_extend(self._h, _ptr(latent_K), int(T_old), int(T_new),
+                                     _stream(stream)))
+        return self
+
+    def export(self, stream=None):
+        """Copies of the index state as torch tensors on the index's device."""
+        dev = self.buffer.device
+        B, NP, NBK = self.B, self.n_pooled, self.n_buckets_max
+        rt = torch.bfloat16 if self.dtype == BF16 else torch.float32
+        out = dict(
+            pooled=torch.empty(B, NP, 64, dtype=torch.float32, device=dev),
+            unit=torch.empty(B, NP, 64, dtype=torch.float32, device=dev),
+            cent=torch.empty(B, NBK, 64, dtype=torch.float32, device=dev),
+            cent_rt=torch.empty(B, NBK, 64, dtype=rt, device=dev),
+            offsets=torch.empty(B, NBK + 1, dtype=torch.int32, device=dev),
+            members=torch.empty(B, NP, dtype=torch.int32, device=dev),
+            assign=torch.empty(B, NP, dtype=torch.int16, device=dev),
+            open_bucket=torch.empty(B, self.G, dtype=torch.int32, device=dev),
+        )
+        _check(_lib.lsa_index_export(self._h, *[_ptr(out[k]) for k in (
+            "pooled", "unit", "cent", "cent_rt", "offsets", "members", "assign", "open_bucket")],
+            _stream(stream)))
+        return out
+
+    def check(self, stream=None):
+        """Raises LsaError if a kernel recorded an error; returns the number of
+        queries that took the exact selection fallback since the last check."""
+        fb = ctypes.c_int64(0)
+        _check(_lib.lsa_index_check(self._h, ctypes.byref(fb), _stream(stream)))
+        return int(fb.value)
+
+
+def lsa_build_index(latent_K, T, p, block, n_buckets, lloyd_iters=3, T_cap=None, stream=None):
+    """Builds an index over keys [0, T) of latent_K [B][T_cap][64]."""
+    _cuda(latent_K)
+    B, cap = latent_K.shape[0], latent_K.shape[1]
+    idx = LsaIndex(B, T_cap or cap, p, block, n_buckets, lloyd_iters, _dtype_code(latent_K),
+                   latent_K.device)
+    return idx.build(latent_K, T, stream)
+
+
+def lsa_select(index, latent_Q, positions, budget, window, sinks, s_max=None, workspace=None,
+               stream=None):
+    """Per-query selection: returns (indices [B][Nq][s_max] int32, counts [B][Nq] int32)."""
+    _cuda(latent_Q, positions)
+    if positions.dtype != torch.int32:
+        raise TypeError("positions must be int32")
+    B, Nq = latent_Q.shape[0], latent_Q.shape[1]
+    s_max = s_max or (budget + window + sinks)
+    dev = latent_Q.device
+    indices = torch.empty(B, Nq, s_max, dtype=torch.int32, device=dev)
+    counts = torch.empty(B, Nq, dtype=torch.int32, device=dev)
+    need = _lib.lsa_select_workspace_bytes(index.handle, Nq)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check(_lib.lsa_select(index.handle, _ptr(latent_Q), _ptr(positions), Nq,
+                           SelectParams(budget, window, sinks), _ptr(indices), _ptr(counts),
+                           s_max, _ptr(workspace), workspace.numel(), _stream(stream)))
+    return indices, counts
+
+
+def lsa_sparse_attn(Q, K, V, indices, counts, scale=None, return_lse=False, out=None,
+                    stream=None):
+    """Exact attention of Q [B][Nq][Hq][d] over the selected rows of K, V [B][T_cap][Hkv][d]."""
+    _cuda(Q, K, V, indices, counts, out)
+    B, Nq, Hq, d = Q.shape
+    T_cap, Hkv = K.shape[1], K.shape[2]
+    if scale is None:
+        scale = float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))
+    O = out if out is not None else torch.empty_like(Q)
+    lse = torch.empty(B, Nq, Hq, dtype=torch.float32, device=Q.device) if return_lse else None
+    _check(_lib.lsa_sparse_attn(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), B, Nq, T_cap, Hq, Hkv,
+                                d, _ptr(indices), _ptr(counts), indices.shape[-1], scale, _ptr(O),
+                                _ptr(lse), _stream(stream)))
+    return (O, lse) if return_lse else O
+
+
+def lsa_prefill_workspace_bytes(index, Nq, budget, window, sinks):
+    return int(_lib.lsa_prefill_workspace_bytes(index.handle, Nq,
+                                                SelectParams(budget, window, sinks)))
+
+
+def lsa_prefill_chunk(index, latent_K, latent_Q, Q, K, V, T_old, T_new, budget, window, sinks,
+                      workspace=None, out=None, stream=None):
+    """One fused prefill chunk (queries at positions [T_old, T_new)); returns O.
+
+    The chunk's selection (indices [B][Nq][R+W+S] then counts [B][Nq]) is left
+    at the start of `workspace`."""
+    _cuda(latent_K, latent_Q, Q, K, V, out)
+    B, Nq, Hq, d = Q.shape
+    Hkv = K.shape[2]
+    need = lsa_prefill_workspace_bytes(index, Nq, budget, window, sinks)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    O = out if out is not None else torch.empty_like(Q)
+    _check(_lib.lsa_prefill_chunk(index.handle, _ptr(latent_K), _ptr(latent_Q), _ptr(Q), _ptr(K),
+                                  _ptr(V), int(T_old), int(T_new), Hq, Hkv, d,
+                                  SelectParams(budget, window, sinks), _ptr(workspace),
+                                  workspace.numel(), _ptr(O), _stream(stream)))
+    return O
+
+
+def prefill_selection_views(workspace, B, Nq, s_max):
+    """(indices, counts) views of the selection a prefill chunk left in `workspace`."""
+    n_idx = B * Nq * s_max
+    al = (n_idx * 4 + 255) // 256 * 256
+    indices = workspace[: n_idx * 4].view(torch.int32).view(B, Nq, s_max)
+    counts = workspace[al: al + B * Nq * 4].view(torch.int32).view(B, Nq)
+    return indices, counts

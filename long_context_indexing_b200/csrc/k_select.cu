@@ -1,0 +1,565 @@
+// k_select.cu -- per-query bucket retrieval: candidate nomination, exact
+// ranking, greedy budget fill, sinks + window, exact fallback.
+//
+// Method: "Latent Sparse Attention: un indice gerarchico per contesti
+// lunghi", paragraph on retrieval (the query is compared with the centroids
+// to choose the buckets whose keys are read) and paragraph on the read budget
+// (a fixed number of long-range keys outside the recent window, the most
+// recent keys, and sink keys at the start of the sequence).
+//
+// Exactness.  The ranking that decides the selection uses exact binary64
+// scores (exact products of the binary32/bf16 inputs summed in ascending
+// dimension), identical bit for bit to a sequential evaluation.  A cheaper
+// binary32 (or tensor-core) pass only nominates KC candidate buckets per
+// query together with tau, an upper bound of the approximate score of every
+// bucket it did not nominate.  With |approx - exact| <= eps for every bucket,
+// the candidates' exact ranking is the true ranking up to the bucket c at
+// which the fill stops whenever exact(c) > tau + eps; otherwise (or when the
+// candidates run out while more keys are available) the query is sent to an
+// exact fallback that ranks every bucket.
+#include <float.h>
+
+#include "lsa_internal.cuh"
+
+namespace lsa {
+
+// Buckets of the closed blocks whose first key lies at or below pos - W (the
+// only ones that can hold an available key).
+__device__ __forceinline__ int64_t eligible_buckets(const IndexView& ix, int64_t n_blk, int64_t pos,
+                                                    int W)
+{
+    const int64_t hi = pos - W;
+    if (hi < 0) return 0;
+    const int64_t span = (int64_t)ix.p * ix.G;
+    int64_t nb = hi / span + 1;
+    if (nb > n_blk) nb = n_blk;
+    return nb * ix.k;
+}
+
+// Keys of pooled group j inside [S, hi].
+__device__ __forceinline__ int group_avail(int64_t j, int p, int64_t S, int64_t hi)
+{
+    int64_t lo = j * p, up = lo + p - 1;
+    if (lo < S) lo = S;
+    if (up > hi) up = hi;
+    return (up >= lo) ? (int)(up - lo + 1) : 0;
+}
+
+__device__ __forceinline__ float rt_load(const IndexView& ix, int64_t bseq, int64_t g, int i)
+{
+    const int64_t x = (bseq * ix.NBK + g) * DL + i;
+    if (ix.dtype == LSA_BF16) return __bfloat162float(((const __nv_bfloat16*)ix.cent_rt)[x]);
+    return ((const float*)ix.cent_rt)[x];
+}
+
+__device__ __forceinline__ bool rank_before(double s, int g, double s2, int g2)
+{
+    return s > s2 || (s == s2 && g < g2);  // score descending, then lowest bucket id
+}
+
+__device__ __forceinline__ uint32_t ord_key(float f)
+{
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_to_float(uint32_t k)
+{
+    const uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+    return __uint_as_float(u);
+}
+
+template <typename T>
+__device__ __forceinline__ void load_query(float* q_s, const T* lq, int64_t row)
+{
+    if (threadIdx.x < DL) q_s[threadIdx.x] = load_elt(lq + row * DL + threadIdx.x);
+}
+
+// ---------------------------------------------------------------------------
+// Candidate nomination, SIMT: one CTA per query.  Binary32 FMA scores of the
+// eligible buckets into shared memory, then an MSB-first radix select of the
+// KC-th largest score (4 passes of 8 bits).  Candidates: every bucket above
+// that score plus enough of those equal to it.  tau = that score.
+// ---------------------------------------------------------------------------
+constexpr int SIMT_THREADS = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(SIMT_THREADS) score_topk_simt_kernel(IndexView ix, int64_t n_blk,
+                                                                       const T* lq, PosSrc pos,
+                                                                       int64_t Nq, int W,
+                                                                       SelectWs ws)
+{
+    extern __shared__ float sc[];
+    __shared__ float q_s[DL];
+    __shared__ unsigned hist[256];
+    __shared__ uint32_t sh_prefix, sh_want;
+    __shared__ int sh_gt, sh_eq;
+    const int64_t b = blockIdx.y, i = blockIdx.x;
+    const int64_t row = b * Nq + i;
+    if (row == 0 && threadIdx.x == 0) *ws.fb_count = 0;
+    const int64_t pq = pos.at(b, Nq, i);
+    const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
+    load_query(q_s, lq, row);
+    __syncthreads();
+    int32_t* cand = ws.cand + row * KC;
+    if (nb <= KC) {
+        for (int x = threadIdx.x; x < KC; x += SIMT_THREADS) cand[x] = (x < nb) ? x : -1;
+        if (threadIdx.x == 0) {
+            ws.ncand[row] = (int32_t)nb;
+            ws.tau[row] = -INFINITY;
+        }
+        return;
+    }
+    for (int64_t g = threadIdx.x; g < nb; g += SIMT_THREADS) {
+        float s = 0.f;
+#pragma unroll 16
+        for (int d = 0; d < DL; ++d) s = fmaf(q_s[d], rt_load(ix, b, g, d), s);
+        sc[g] = s;
+    }
+    if (threadIdx.x == 0) {
+        sh_prefix = 0;
+        sh_want = KC;
+        sh_gt = 0;
+        sh_eq = 0;
+    }
+    __syncthreads();
+    uint32_t mask = 0;
+    for (int pass = 3; pass >= 0; --pass) {
+        const int sh = 8 * pass;
+        for (int x = threadIdx.x; x < 256; x += SIMT_THREADS) hist[x] = 0;
+        __syncthreads();
+        const uint32_t prefix = sh_prefix;
+        for (int64_t g = threadIdx.x; g < nb; g += SIMT_THREADS) {
+            const uint32_t kk = ord_key(sc[g]);
+            if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> sh) & 255u], 1u);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t want = sh_want, cum = 0;
+            for (int bin = 255; bin >= 0; --bin) {
+                const uint32_t h = hist[bin];
+                if (cum + h >= want) {
+                    sh_prefix = prefix | ((uint32_t)bin << sh);
+                    sh_want = want - cum;
+                    break;
+                }
+                cum += h;
+            }
+        }
+        mask |= 255u << sh;
+        __syncthreads();
+    }
+    const uint32_t thr = sh_prefix;      // key of the KC-th largest score
+    const int need_eq = (int)sh_want;    // how many of the ties at thr to take
+    for (int64_t g = threadIdx.x; g < nb; g += SIMT_THREADS) {
+        const uint32_t kk = ord_key(sc[g]);
+        if (kk > thr) {
+            const int s = atomicAdd(&sh_gt, 1);
+            cand[s] = (int32_t)g;
+        } else if (kk == thr) {
+            const int s = atomicAdd(&sh_eq, 1);
+            if (s < need_eq) cand[KC - need_eq + s] = (int32_t)g;
+        }
+    }
+    if (threadIdx.x == 0) {
+        ws.ncand[row] = KC;
+        ws.tau[row] = key_to_float(thr);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Availability and emission helpers (closed CSR members, then open members).
+// ---------------------------------------------------------------------------
+struct FillCtx {
+    IndexView ix;
+    int64_t bseq;
+    int64_t n_blk;
+    int64_t pos;
+    int64_t hi;     // pos - W
+    int64_t S;
+    bool open_live; // the open block has keys at or below hi
+};
+
+// Warp-cooperative count of available keys of bucket g.
+__device__ int64_t warp_avail(const FillCtx& f, int64_t g)
+{
+    const int lane = threadIdx.x & 31;
+    const IndexView& ix = f.ix;
+    const int32_t* off = ix.offsets + f.bseq * (ix.NBK + 1);
+    const int32_t* mem = ix.members + f.bseq * ix.NP;
+    const int p = ix.p;
+    const int64_t span = (int64_t)p * ix.G;
+    const int64_t blk = g / ix.k;
+    const int64_t bstart = blk * span, bend = bstart + span;
+    const int32_t o0 = off[g], o1 = off[g + 1];
+    int64_t a = 0;
+    if (bstart >= f.S && bend - 1 <= f.hi) {
+        a = (int64_t)(o1 - o0) * p;
+    } else if (bstart <= f.hi) {
+        int64_t c = 0;
+        for (int32_t x = o0 + lane; x < o1; x += 32) c += group_avail(mem[x], p, f.S, f.hi);
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        a = c;
+    }
+    if (f.open_live) {
+        const int32_t* open = ix.open_bucket + f.bseq * ix.G;
+        const int64_t j0 = f.n_blk * ix.G;
+        int64_t c = 0;
+        for (int o = lane; o < ix.G; o += 32)
+            if (open[o] == g) c += group_avail(j0 + o, p, f.S, f.hi);
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        a += c;
+    }
+    return a;
+}
+
+// Writes the first `take` available keys of bucket g (ascending) to out.
+// Called by every thread of the CTA; uses warp 0 for partial buckets.
+__device__ void cta_emit(const FillCtx& f, int64_t g, int64_t take, int32_t* out)
+{
+    const IndexView& ix = f.ix;
+    const int32_t* off = ix.offsets + f.bseq * (ix.NBK + 1);
+    const int32_t* mem = ix.members + f.bseq * ix.NP;
+    const int p = ix.p;
+    const int64_t span = (int64_t)p * ix.G;
+    const int64_t blk = g / ix.k;
+    const int64_t bstart = blk * span, bend = bstart + span;
+    const int32_t o0 = off[g], o1 = off[g + 1];
+    const bool full = (bstart >= f.S && bend - 1 <= f.hi) && !f.open_live;
+    if (full) {
+        for (int64_t x = threadIdx.x; x < take; x += blockDim.x)
+            out[x] = mem[o0 + x / p] * p + (int32_t)(x % p);
+        return;
+    }
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    int64_t cur = 0;
+    const int64_t nkeys = (int64_t)(o1 - o0) * p;
+    for (int64_t x0 = 0; x0 < nkeys && cur < take; x0 += 32) {
+        const int64_t x = x0 + lane;
+        int64_t t = -1;
+        if (x < nkeys) t = (int64_t)mem[o0 + x / p] * p + x % p;
+        const bool ok = (t >= f.S) && (t <= f.hi);
+        const unsigned bal = __ballot_sync(0xffffffffu, ok);
+        const int64_t at = cur + __popc(bal & ((1u << lane) - 1u));
+        if (ok && at < take) out[at] = (int32_t)t;
+        cur += __popc(bal);
+    }
+    if (f.open_live) {
+        const int32_t* open = ix.open_bucket + f.bseq * ix.G;
+        const int64_t j0 = f.n_blk * ix.G;
+        const int64_t nk = (int64_t)ix.G * p;
+        for (int64_t x0 = 0; x0 < nk && cur < take; x0 += 32) {
+            const int64_t x = x0 + lane;
+            int64_t t = -1;
+            if (x < nk && open[x / p] == g) t = (j0 + x / p) * p + x % p;
+            const bool ok = (t >= f.S) && (t <= f.hi);
+            const unsigned bal = __ballot_sync(0xffffffffu, ok);
+            const int64_t at = cur + __popc(bal & ((1u << lane) - 1u));
+            if (ok && at < take) out[at] = (int32_t)t;
+            cur += __popc(bal);
+        }
+    }
+}
+
+__device__ void cta_emit_tail(int64_t pq, int W, int64_t n_s, int64_t off, int s_max, int32_t* out,
+                              int32_t* count)
+{
+    int64_t w0 = pq - W + 1;
+    if (w0 < n_s) w0 = n_s;
+    const int64_t n_w = pq + 1 - w0;
+    for (int64_t x = threadIdx.x; x < n_w; x += blockDim.x) out[off + x] = (int32_t)(w0 + x);
+    for (int64_t x = off + n_w + threadIdx.x; x < s_max; x += blockDim.x) out[x] = -1;
+    if (threadIdx.x == 0) *count = (int32_t)(off + n_w);
+}
+
+// ---------------------------------------------------------------------------
+// Exact ranking + greedy fill + emission.  One CTA (128 threads) per query.
+// ---------------------------------------------------------------------------
+constexpr int FILL_THREADS = 128;
+
+template <typename T>
+__global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix, int64_t n_blk,
+                                                                   const T* lq, PosSrc pos,
+                                                                   int64_t Nq, int R, int W, int S,
+                                                                   int s_max, int32_t* indices,
+                                                                   int32_t* counts, SelectWs ws)
+{
+    __shared__ float q_s[DL];
+    __shared__ int cg[KC];
+    __shared__ double es[KC];
+    __shared__ int order[KC];
+    __shared__ int64_t av[KC];
+    __shared__ int take_g[KC];
+    __shared__ int64_t take_n[KC];
+    __shared__ int sh_ntake, sh_exact;
+    __shared__ float sh_l1;
+    const int64_t b = blockIdx.y, i = blockIdx.x;
+    const int64_t row = b * Nq + i;
+    const int64_t pq = pos.at(b, Nq, i);
+    load_query(q_s, lq, row);
+    const int nc = ws.ncand[row];
+    if (threadIdx.x < KC) cg[threadIdx.x] = ws.cand[row * KC + threadIdx.x];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float l1 = 0.f;
+        for (int d = 0; d < DL; ++d) l1 += fabsf(q_s[d]);
+        sh_l1 = l1;
+    }
+    if ((int)threadIdx.x < nc) {
+        const int g = cg[threadIdx.x];
+        double s = 0.0;
+#pragma unroll 16
+        for (int d = 0; d < DL; ++d) s = __fma_rn((double)q_s[d], (double)rt_load(ix, b, g, d), s);
+        es[threadIdx.x] = s;
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < nc) {
+        const int c = threadIdx.x;
+        int r = 0;
+        for (int c2 = 0; c2 < nc; ++c2) r += rank_before(es[c2], cg[c2], es[c], cg[c]);
+        order[r] = c;
+    }
+    FillCtx f;
+    f.ix = ix;
+    f.bseq = b;
+    f.n_blk = n_blk;
+    f.pos = pq;
+    f.hi = pq - W;
+    f.S = S;
+    f.open_live = (n_blk < ix.nblk_max) && (n_blk > 0) && (n_blk * (int64_t)ix.p * ix.G <= f.hi);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int c = warp; c < nc; c += FILL_THREADS / 32) {
+        const int64_t a = warp_avail(f, cg[c]);
+        if (lane == 0) av[c] = a;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int64_t rem = R;
+        int nt = 0, cut = -1;
+        for (int r = 0; r < nc && rem > 0; ++r) {
+            const int c = order[r];
+            const int64_t a = av[c];
+            if (a == 0) continue;
+            const int64_t t = (a <= rem) ? a : rem;
+            take_g[nt] = cg[c];
+            take_n[nt] = t;
+            ++nt;
+            rem -= t;
+            if (rem == 0) cut = c;
+        }
+        int exact = 1;
+        if (nc == KC) {
+            const double eps = ldexp((double)sh_l1, -12);
+            if (rem > 0) {
+                int64_t total = f.hi - S + 1;  // keys in [S, pos - W]
+                if (total < 0) total = 0;
+                exact = ((int64_t)R - rem) >= total;
+            } else if (cut >= 0) {
+                exact = es[cut] > (double)ws.tau[row] + eps;
+            }
+        }
+        sh_ntake = nt;
+        sh_exact = exact;
+    }
+    __syncthreads();
+    if (!sh_exact) {
+        if (threadIdx.x == 0) {
+            const int slot = atomicAdd(ws.fb_count, 1);
+            ws.fb_list[slot] = (int32_t)row;
+            atomicAdd(ix.status + 1, 1u);
+        }
+        return;
+    }
+    int32_t* out = indices + row * (int64_t)s_max;
+    const int64_t n_s = (S < pq + 1) ? S : pq + 1;
+    for (int64_t x = threadIdx.x; x < n_s; x += FILL_THREADS) out[x] = (int32_t)x;
+    int64_t o = n_s;
+    for (int t = 0; t < sh_ntake; ++t) {
+        cta_emit(f, take_g[t], take_n[t], out + o);
+        o += take_n[t];
+    }
+    __syncthreads();
+    cta_emit_tail(pq, W, n_s, o, s_max, out, counts + row);
+}
+
+// ---------------------------------------------------------------------------
+// Exact fallback: persistent CTAs walk the list of flagged queries.  Every
+// eligible bucket gets its exact binary64 score; the fill repeatedly takes the
+// best remaining bucket (score desc, lowest id) until the budget is met.
+// ---------------------------------------------------------------------------
+constexpr int FB_THREADS = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(FB_THREADS) select_fallback_kernel(IndexView ix, int64_t n_blk,
+                                                                     const T* lq, PosSrc pos,
+                                                                     int64_t Nq, int R, int W,
+                                                                     int S, int s_max,
+                                                                     int32_t* indices,
+                                                                     int32_t* counts, SelectWs ws)
+{
+    __shared__ float q_s[DL];
+    __shared__ double rs[FB_THREADS / 32];
+    __shared__ int64_t rg[FB_THREADS / 32];
+    __shared__ int64_t sh_best;
+    __shared__ int64_t sh_avail;
+    const int n = *ws.fb_count;
+    double* sc = ws.fb_scores + (int64_t)blockIdx.x * ix.NBK;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = blockIdx.x; e < n; e += gridDim.x) {
+        const int64_t row = ws.fb_list[e];
+        const int64_t b = row / Nq, i = row % Nq;
+        const int64_t pq = pos.at(b, Nq, i);
+        const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
+        __syncthreads();
+        load_query(q_s, lq, row);
+        __syncthreads();
+        for (int64_t g = threadIdx.x; g < nb; g += FB_THREADS) {
+            double s = 0.0;
+            for (int d = 0; d < DL; ++d) s = __fma_rn((double)q_s[d], (double)rt_load(ix, b, g, d), s);
+            sc[g] = s;
+        }
+        FillCtx f;
+        f.ix = ix;
+        f.bseq = b;
+        f.n_blk = n_blk;
+        f.pos = pq;
+        f.hi = pq - W;
+        f.S = S;
+        f.open_live = (n_blk < ix.nblk_max) && (n_blk > 0) && (n_blk * (int64_t)ix.p * ix.G <= f.hi);
+        int32_t* out = indices + row * (int64_t)s_max;
+        const int64_t n_s = (S < pq + 1) ? S : pq + 1;
+        for (int64_t x = threadIdx.x; x < n_s; x += FB_THREADS) out[x] = (int32_t)x;
+        int64_t o = n_s, rem = R;
+        __syncthreads();
+        while (rem > 0) {
+            double bs = -INFINITY;
+            int64_t bg = INT64_MAX;
+            for (int64_t g = threadIdx.x; g < nb; g += FB_THREADS) {
+                const double s = sc[g];
+                if (s != -INFINITY && (bs == -INFINITY || s > bs || (s == bs && g < bg))) {
+                    bs = s;
+                    bg = g;
+                }
+            }
+            for (int off = 16; off > 0; off >>= 1) {
+                const double os = __shfl_xor_sync(0xffffffffu, bs, off);
+                const int64_t og = __shfl_xor_sync(0xffffffffu, bg, off);
+                if (os != -INFINITY && (bs == -INFINITY || os > bs || (os == bs && og < bg))) {
+                    bs = os;
+                    bg = og;
+                }
+            }
+            if (lane == 0) {
+                rs[warp] = bs;
+                rg[warp] = bg;
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                for (int w = 1; w < FB_THREADS / 32; ++w)
+                    if (rs[w] != -INFINITY && (bs == -INFINITY || rs[w] > bs || (rs[w] == bs && rg[w] < bg))) {
+                        bs = rs[w];
+                        bg = rg[w];
+                    }
+                sh_best = (bs == -INFINITY) ? -1 : bg;
+            }
+            __syncthreads();
+            const int64_t g = sh_best;
+            if (g < 0) break;
+            if (warp == 0) {
+                const int64_t a = warp_avail(f, g);
+                if (lane == 0) sh_avail = a;
+            }
+            __syncthreads();
+            const int64_t a = sh_avail;
+            if (a > 0) {
+                const int64_t t = (a <= rem) ? a : rem;
+                cta_emit(f, g, t, out + o);
+                o += t;
+                rem -= t;
+            }
+            if (threadIdx.x == 0) sc[g] = -INFINITY;
+            __syncthreads();
+        }
+        cta_emit_tail(pq, W, n_s, o, s_max, out, counts + row);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Workspace and launch.
+// ---------------------------------------------------------------------------
+static inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t select_ws_bytes(const IndexView& ix, int64_t Nq)
+{
+    const size_t rows = (size_t)ix.B * (size_t)Nq;
+    return al256(rows * KC * 4) + al256(rows * 4) + al256(rows * 4) + al256(rows * 4) + al256(4) +
+           al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
+}
+
+SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
+{
+    const size_t rows = (size_t)ix.B * (size_t)Nq;
+    char* p = (char*)ws;
+    SelectWs w;
+    w.cand = (int32_t*)p;
+    p += al256(rows * KC * 4);
+    w.tau = (float*)p;
+    p += al256(rows * 4);
+    w.ncand = (int32_t*)p;
+    p += al256(rows * 4);
+    w.fb_list = (int32_t*)p;
+    p += al256(rows * 4);
+    w.fb_count = (int32_t*)p;
+    p += al256(4);
+    w.fb_scores = (double*)p;
+    return w;
+}
+
+cudaError_t launch_score_topk_tc(const IndexView& ix, int64_t n_blk, const void* latent_Q,
+                                 PosSrc pos, int64_t Nq, int W, const SelectWs& ws,
+                                 cudaStream_t st);
+
+template <typename T>
+static cudaError_t launch_select_t(const IndexView& ix, int64_t n_blk, const T* lq, PosSrc pos,
+                                   int64_t Nq, lsa_select_params sp, int32_t* indices,
+                                   int32_t* counts, int s_max, const SelectWs& ws, bool use_tc,
+                                   cudaStream_t st)
+{
+    dim3 grid((unsigned)Nq, (unsigned)ix.B);
+    cudaError_t e;
+    if (use_tc) {
+        e = launch_score_topk_tc(ix, n_blk, lq, pos, Nq, sp.window, ws, st);
+        if (e != cudaSuccess) return e;
+    } else {
+        const size_t smem = (size_t)n_blk * ix.k * sizeof(float);
+        e = cudaFuncSetAttribute(score_topk_simt_kernel<T>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        score_topk_simt_kernel<T><<<grid, SIMT_THREADS, smem, st>>>(ix, n_blk, lq, pos, Nq,
+                                                                    sp.window, ws);
+    }
+    select_fill_kernel<T><<<grid, FILL_THREADS, 0, st>>>(ix, n_blk, lq, pos, Nq, sp.budget,
+                                                         sp.window, sp.sinks, s_max, indices,
+                                                         counts, ws);
+    int64_t rows = ix.B * Nq;
+    const unsigned fb_grid = (unsigned)(rows < FB_CTAS ? rows : FB_CTAS);
+    select_fallback_kernel<T><<<fb_grid, FB_THREADS, 0, st>>>(ix, n_blk, lq, pos, Nq, sp.budget,
+                                                              sp.window, sp.sinks, s_max,
+                                                              indices, counts, ws);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select(const IndexView& ix, int64_t n_blk, const void* latent_Q, PosSrc pos,
+                          int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
+                          int s_max, const SelectWs& ws, bool use_tc, cudaStream_t st)
+{
+    if (Nq <= 0) return cudaSuccess;
+    if (ix.dtype == LSA_BF16)
+        return launch_select_t(ix, n_blk, (const __nv_bfloat16*)latent_Q, pos, Nq, sp, indices,
+                               counts, s_max, ws, use_tc, st);
+    return launch_select_t(ix, n_blk, (const float*)latent_Q, pos, Nq, sp, indices, counts, s_max,
+                           ws, false, st);
+}
+
+}  // namespace lsa

@@ -1,0 +1,381 @@
+// lsa_api.cu -- host side of the liblsa C-ABI: argument checks, index
+// storage layout, stream-ordered orchestration of the kernels, status words.
+// Every entry point is declared and documented in include/lsa.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <math.h>
+
+#include <new>
+
+#include "lsa_internal.cuh"
+
+using namespace lsa;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+lsa_status fail(lsa_status s, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+lsa_status cuda_fail(cudaError_t e, const char* where)
+{
+    return fail(LSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+lsa_status check_index_params(int64_t B, int64_t T_cap, lsa_index_params ip)
+{
+    if (B < 1 || B > 65535) return fail(LSA_ERR_INVALID_ARG, "B=%lld outside [1, 65535]", (long long)B);
+    if (T_cap < 1 || T_cap > 2147483647LL)
+        return fail(LSA_ERR_INVALID_ARG, "T_cap=%lld outside [1, 2^31-1]", (long long)T_cap);
+    if (ip.p < 1 || ip.block < 1 || ip.n_buckets < 1 || ip.lloyd_iters < 1)
+        return fail(LSA_ERR_INVALID_ARG, "index parameters must be >= 1");
+    if (ip.n_buckets > ip.block)
+        return fail(LSA_ERR_INVALID_ARG, "n_buckets=%d > block=%d", ip.n_buckets, ip.block);
+    if (ip.n_buckets > MAX_K)
+        return fail(LSA_ERR_UNSUPPORTED, "n_buckets=%d > %d", ip.n_buckets, MAX_K);
+    if (ip.block > 4096) return fail(LSA_ERR_UNSUPPORTED, "block=%d > 4096", ip.block);
+    if (ip.lloyd_iters > 1000) return fail(LSA_ERR_INVALID_ARG, "lloyd_iters > 1000");
+    if ((int64_t)ip.p * ip.block > T_cap)
+        return fail(LSA_ERR_INVALID_ARG, "T_cap=%lld holds no whole block", (long long)T_cap);
+    return LSA_OK;
+}
+
+struct Layout {
+    size_t pooled, unit, cent, cent_rt, offsets, members, assign, open, status, total;
+};
+
+Layout layout(int64_t B, int64_t T_cap, lsa_index_params ip, lsa_dtype dt)
+{
+    const int64_t NP = T_cap / ip.p;
+    const int64_t nblk = NP / ip.block;
+    const int64_t NBK = nblk * ip.n_buckets;
+    const size_t rt = (dt == LSA_BF16) ? 2 : 4;
+    Layout L;
+    size_t o = 0;
+    L.pooled = o;  o += al256((size_t)B * NP * DL * 4);
+    L.unit = o;    o += al256((size_t)B * NP * DL * 4);
+    L.cent = o;    o += al256((size_t)B * NBK * DL * 4);
+    L.cent_rt = o; o += al256((size_t)B * NBK * DL * rt);
+    L.offsets = o; o += al256((size_t)B * (NBK + 1) * 4);
+    L.members = o; o += al256((size_t)B * NP * 4);
+    L.assign = o;  o += al256((size_t)B * NP * 2);
+    L.open = o;    o += al256((size_t)B * ip.block * 4);
+    L.status = o;  o += al256(8 * 4);
+    L.total = o;
+    return L;
+}
+
+lsa_status check_select(const lsa_index* idx, lsa_select_params sp, int s_max)
+{
+    if (sp.budget < 0 || sp.window < 0 || sp.sinks < 0)
+        return fail(LSA_ERR_INVALID_ARG, "budget/window/sinks must be >= 0");
+    if ((int64_t)sp.budget + sp.window + sp.sinks > s_max)
+        return fail(LSA_ERR_INVALID_ARG, "s_max=%d < budget+window+sinks=%lld", s_max,
+                    (long long)sp.budget + sp.window + sp.sinks);
+    if (sp.window < idx->v.p - 1)
+        return fail(LSA_ERR_UNSUPPORTED,
+                    "window=%d < p-1: keys of an incomplete pooled group would be unreachable",
+                    sp.window);
+    return LSA_OK;
+}
+
+// The SIMT nominator keeps every eligible score in shared memory.
+constexpr int64_t SIMT_MAX_BUCKETS = (220 * 1024) / 4;
+
+bool use_tc_path(const lsa_index* idx, int64_t Nq)
+{
+    return idx->v.dtype == LSA_BF16 && Nq >= 128 && tc_scoring_available();
+}
+
+lsa_status run_select(const lsa_index* idx, const void* lq, PosSrc pos, int64_t Nq,
+                      lsa_select_params sp, int32_t* indices, int32_t* counts, int s_max, void* ws,
+                      cudaStream_t st)
+{
+    const bool tc = use_tc_path(idx, Nq);
+    if (!tc && idx->n_blk * idx->v.k > SIMT_MAX_BUCKETS)
+        return fail(LSA_ERR_UNSUPPORTED, "%lld buckets exceed the SIMT scorer's %lld",
+                    (long long)(idx->n_blk * idx->v.k), (long long)SIMT_MAX_BUCKETS);
+    SelectWs w = select_ws_carve(ws, idx->v, Nq);
+    cudaError_t e = launch_select(idx->v, idx->n_blk, lq, pos, Nq, sp, indices, counts, s_max, w,
+                                  tc, st);
+    if (e != cudaSuccess) return cuda_fail(e, "select");
+    return LSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lsa_last_error(void) { return g_err; }
+
+const char* lsa_version(void) { return "liblsa 0.1 (D-LSA Flat, sm_100a)"; }
+
+size_t lsa_index_bytes(int64_t B, int64_t T_cap, lsa_index_params ip, lsa_dtype dtype)
+{
+    if (check_index_params(B, T_cap, ip) != LSA_OK) return 0;
+    if (dtype != LSA_F32 && dtype != LSA_BF16) {
+        fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+        return 0;
+    }
+    return layout(B, T_cap, ip, dtype).total;
+}
+
+lsa_status lsa_index_init(void* buf, size_t bytes, int64_t B, int64_t T_cap, lsa_index_params ip,
+                          lsa_dtype dtype, lsa_index** out)
+{
+    if (!out) return fail(LSA_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    lsa_status s = check_index_params(B, T_cap, ip);
+    if (s != LSA_OK) return s;
+    if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
+    if (!buf) return fail(LSA_ERR_INVALID_ARG, "buf is NULL");
+    if (((uintptr_t)buf & 255u) != 0) return fail(LSA_ERR_ALIGNMENT, "buf not 256-byte aligned");
+    const Layout L = layout(B, T_cap, ip, dtype);
+    if (bytes < L.total)
+        return fail(LSA_ERR_WORKSPACE, "index buffer %zu < %zu bytes", bytes, L.total);
+    lsa_index* h = new (std::nothrow) lsa_index;
+    if (!h) return fail(LSA_ERR_INTERNAL, "host allocation failed");
+    char* base = (char*)buf;
+    IndexView& v = h->v;
+    v.B = B;
+    v.T_cap = T_cap;
+    v.NP = T_cap / ip.p;
+    v.nblk_max = (int)(v.NP / ip.block);
+    v.NBK = (int64_t)v.nblk_max * ip.n_buckets;
+    v.p = ip.p;
+    v.G = ip.block;
+    v.k = ip.n_buckets;
+    v.L = ip.lloyd_iters;
+    v.dtype = dtype;
+    v.pooled = (float*)(base + L.pooled);
+    v.unit = (float*)(base + L.unit);
+    v.cent = (float*)(base + L.cent);
+    v.cent_rt = (void*)(base + L.cent_rt);
+    v.offsets = (int32_t*)(base + L.offsets);
+    v.members = (int32_t*)(base + L.members);
+    v.assign = (int16_t*)(base + L.assign);
+    v.open_bucket = (int32_t*)(base + L.open);
+    v.status = (uint32_t*)(base + L.status);
+    h->n_blk = 0;
+    h->buf = buf;
+    h->bytes = bytes;
+    h->status_clean = false;
+    *out = h;
+    return LSA_OK;
+}
+
+void lsa_index_release(lsa_index* idx) { delete idx; }
+
+int64_t lsa_index_num_blocks(const lsa_index* idx) { return idx ? idx->n_blk : -1; }
+
+lsa_status lsa_index_extend(lsa_index* idx, const void* latent_K, int64_t T_old, int64_t T_new,
+                            void* stream)
+{
+    if (!idx || !latent_K) return fail(LSA_ERR_INVALID_ARG, "NULL index or latent_K");
+    if (!aligned16(latent_K)) return fail(LSA_ERR_ALIGNMENT, "latent_K not 16-byte aligned");
+    const IndexView& v = idx->v;
+    if (T_old < 0 || T_new < T_old || T_new > v.T_cap)
+        return fail(LSA_ERR_INVALID_ARG, "need 0 <= T_old <= T_new <= T_cap (%lld, %lld, %lld)",
+                    (long long)T_old, (long long)T_new, (long long)v.T_cap);
+    const int64_t span = (int64_t)v.p * v.G;
+    const int64_t b0 = T_old / span, b1 = T_new / span;
+    if (b0 > idx->n_blk)
+        return fail(LSA_ERR_INVALID_ARG, "extend from block %lld leaves a gap after %lld blocks",
+                    (long long)b0, (long long)idx->n_blk);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e;
+    if (!idx->status_clean) {
+        e = cudaMemsetAsync(v.status, 0, 8 * sizeof(uint32_t), st);
+        if (e != cudaSuccess) return cuda_fail(e, "status clear");
+        idx->status_clean = true;
+    }
+    const int64_t j_end = T_new / v.p;
+    e = launch_pool_unit(v, latent_K, b0 * v.G, j_end, st);
+    if (e != cudaSuccess) return cuda_fail(e, "pool");
+    e = launch_kmeans(v, b0, b1, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kmeans");
+    if (b1 > b0 || b1 > idx->n_blk) {
+        if (b1 > idx->n_blk) idx->n_blk = b1;
+        e = launch_open_assign(v, idx->n_blk, j_end, st);
+        if (e != cudaSuccess) return cuda_fail(e, "open assign");
+    } else if (j_end > idx->n_blk * v.G) {
+        e = launch_open_assign(v, idx->n_blk, j_end, st);
+        if (e != cudaSuccess) return cuda_fail(e, "open assign");
+    }
+    return LSA_OK;
+}
+
+lsa_status lsa_build_index(lsa_index* idx, const void* latent_K, int64_t T, void* stream)
+{
+    return lsa_index_extend(idx, latent_K, 0, T, stream);
+}
+
+lsa_status lsa_index_export(const lsa_index* idx, float* pooled, float* unit, float* cent,
+                            void* cent_rt, int32_t* offsets, int32_t* members, int16_t* assign,
+                            int32_t* open_bucket, void* stream)
+{
+    if (!idx) return fail(LSA_ERR_INVALID_ARG, "NULL index");
+    const IndexView& v = idx->v;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t rt = (v.dtype == LSA_BF16) ? 2 : 4;
+    struct {
+        void* dst;
+        const void* src;
+        size_t n;
+    } items[] = {
+        {pooled, v.pooled, (size_t)v.B * v.NP * DL * 4},
+        {unit, v.unit, (size_t)v.B * v.NP * DL * 4},
+        {cent, v.cent, (size_t)v.B * v.NBK * DL * 4},
+        {cent_rt, v.cent_rt, (size_t)v.B * v.NBK * DL * rt},
+        {offsets, v.offsets, (size_t)v.B * (v.NBK + 1) * 4},
+        {members, v.members, (size_t)v.B * v.NP * 4},
+        {assign, v.assign, (size_t)v.B * v.NP * 2},
+        {open_bucket, v.open_bucket, (size_t)v.B * v.G * 4},
+    };
+    for (auto& it : items) {
+        if (!it.dst) continue;
+        cudaError_t e = cudaMemcpyAsync(it.dst, it.src, it.n, cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(e, "export");
+    }
+    return LSA_OK;
+}
+
+lsa_status lsa_index_check(lsa_index* idx, int64_t* fallbacks, void* stream)
+{
+    if (!idx) return fail(LSA_ERR_INVALID_ARG, "NULL index");
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t h[8] = {0};
+    cudaError_t e = cudaMemcpyAsync(h, idx->v.status, sizeof(h), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(idx->v.status, 0, sizeof(h), st);
+    if (e != cudaSuccess) return cuda_fail(e, "index check");
+    if (fallbacks) *fallbacks = (int64_t)h[1];
+    switch (h[0]) {
+    case DEV_OK: return LSA_OK;
+    case DEV_OPEN_FULL:
+        return fail(LSA_ERR_INTERNAL, "decode append found the open block full (sequence %u)", h[2]);
+    case DEV_BAD_INDEX:
+        return fail(LSA_ERR_INVALID_ARG, "a selected index (%d) was outside [0, T_cap)", (int)h[2]);
+    case DEV_TIMEOUT:
+        return fail(LSA_ERR_TIMEOUT, "a bounded wait gave up (row %u)", h[2]);
+    default: return fail(LSA_ERR_INTERNAL, "device status %u (detail %u)", h[0], h[2]);
+    }
+}
+
+size_t lsa_select_workspace_bytes(const lsa_index* idx, int64_t Nq)
+{
+    if (!idx || Nq < 0) return 0;
+    return select_ws_bytes(idx->v, Nq);
+}
+
+lsa_status lsa_select(const lsa_index* idx, const void* latent_Q, const int32_t* positions,
+                      int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
+                      int s_max, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!idx || !latent_Q || !positions || !indices || !counts || !workspace)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    if (Nq < 0 || Nq > 2147483647LL) return fail(LSA_ERR_INVALID_ARG, "Nq out of range");
+    lsa_status s = check_select(idx, sp, s_max);
+    if (s != LSA_OK) return s;
+    if (!aligned16(latent_Q) || !aligned16(positions) || !aligned16(indices) ||
+        !aligned16(counts) || !aligned16(workspace))
+        return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    if (ws_bytes < select_ws_bytes(idx->v, Nq))
+        return fail(LSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes,
+                    select_ws_bytes(idx->v, Nq));
+    PosSrc pos{positions, 0};
+    return run_select(idx, latent_Q, pos, Nq, sp, indices, counts, s_max, workspace,
+                      (cudaStream_t)stream);
+}
+
+lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtype dtype, int64_t B,
+                           int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
+                           const int32_t* indices, const int32_t* counts, int s_max, float scale,
+                           void* O, float* lse, void* stream)
+{
+    if (!Q || !K || !V || !indices || !counts || !O)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
+    if (B < 1 || Nq < 0 || T_cap < 1 || T_cap > 2147483647LL || s_max < 1)
+        return fail(LSA_ERR_INVALID_ARG, "bad sizes");
+    if (Hkv < 1 || Hq < 1 || Hq % Hkv != 0) return fail(LSA_ERR_INVALID_ARG, "Hq %% Hkv != 0");
+    const int hpg = Hq / Hkv;
+    if (hpg != 1 && hpg != 2 && hpg != 4 && hpg != 8)
+        return fail(LSA_ERR_UNSUPPORTED, "Hq/Hkv=%d not in {1,2,4,8}", hpg);
+    if (d != 64 && d != 128) return fail(LSA_ERR_UNSUPPORTED, "d=%d not in {64,128}", d);
+    if (B * Nq * Hkv > 2147483647LL) return fail(LSA_ERR_UNSUPPORTED, "too many (query, head) pairs");
+    if (!(scale > 0.f)) return fail(LSA_ERR_INVALID_ARG, "scale must be > 0");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(indices) ||
+        !aligned16(counts) || !aligned16(O) || (lse && !aligned16(lse)))
+        return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    cudaError_t e = launch_attn(Q, K, V, dtype, B, Nq, T_cap, Hq, Hkv, d, indices, counts, s_max,
+                                scale, O, lse, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "sparse attention");
+    return LSA_OK;
+}
+
+size_t lsa_prefill_workspace_bytes(const lsa_index* idx, int64_t Nq, lsa_select_params sp)
+{
+    if (!idx || Nq < 0 || sp.budget < 0 || sp.window < 0 || sp.sinks < 0) return 0;
+    const int64_t s_max = (int64_t)sp.budget + sp.window + sp.sinks;
+    const size_t rows = (size_t)idx->v.B * (size_t)Nq;
+    return al256(rows * (size_t)s_max * 4) + al256(rows * 4) + select_ws_bytes(idx->v, Nq);
+}
+
+lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* latent_Q,
+                             const void* Q, const void* K, const void* V, int64_t T_old,
+                             int64_t T_new, int Hq, int Hkv, int d, lsa_select_params sp,
+                             void* workspace, size_t ws_bytes, void* O, void* stream)
+{
+    if (!idx || !latent_K || !latent_Q || !Q || !K || !V || !workspace || !O)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    const int64_t Nq = T_new - T_old;
+    if (Nq < 1) return fail(LSA_ERR_INVALID_ARG, "empty chunk");
+    const int s_max = sp.budget + sp.window + sp.sinks;
+    lsa_status s = check_select(idx, sp, s_max);
+    if (s != LSA_OK) return s;
+    if (ws_bytes < lsa_prefill_workspace_bytes(idx, Nq, sp))
+        return fail(LSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes,
+                    lsa_prefill_workspace_bytes(idx, Nq, sp));
+    if (!aligned16(workspace) || !aligned16(latent_Q) || !aligned16(Q) || !aligned16(O))
+        return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    // attention shape checks up front so that nothing launches on bad input
+    const int hpg = (Hkv > 0) ? Hq / Hkv : 0;
+    if (Hkv < 1 || Hq % Hkv != 0 || (hpg != 1 && hpg != 2 && hpg != 4 && hpg != 8))
+        return fail(LSA_ERR_UNSUPPORTED, "Hq/Hkv must be 1, 2, 4 or 8");
+    if (d != 64 && d != 128) return fail(LSA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    cudaStream_t st = (cudaStream_t)stream;
+    s = lsa_index_extend(idx, latent_K, T_old, T_new, stream);
+    if (s != LSA_OK) return s;
+    const size_t rows = (size_t)idx->v.B * (size_t)Nq;
+    char* p = (char*)workspace;
+    int32_t* indices = (int32_t*)p;
+    p += al256(rows * (size_t)s_max * 4);
+    int32_t* counts = (int32_t*)p;
+    p += al256(rows * 4);
+    PosSrc pos{nullptr, T_old};
+    s = run_select(idx, latent_Q, pos, Nq, sp, indices, counts, s_max, p, st);
+    if (s != LSA_OK) return s;
+    const float scale = (float)(1.0 / sqrt((double)d));
+    cudaError_t e = launch_attn_status(Q, K, V, idx->v.dtype, idx->v.B, Nq, idx->v.T_cap, Hq, Hkv,
+                                       d, indices, counts, s_max, scale, O, nullptr,
+                                       idx->v.status, st);
+    if (e != cudaSuccess) return cuda_fail(e, "sparse attention");
+    return LSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,133 @@
+// lsa_internal.cuh -- shared declarations of liblsa's CUDA sources.
+//
+// Index layout in the caller's device buffer (per array, B sequences
+// back to back; every array starts on a 256-byte boundary):
+//   pooled   f32 [B][NP][64]     x_j, mean of p consecutive latent keys
+//   unit     f32 [B][NP][64]     u_j = x_j / ||x_j||
+//   cent     f32 [B][NBK][64]    centroids, g = b*k + m
+//   cent_rt  T   [B][NBK][64]    retrieval copy (bf16 or f32)
+//   offsets  i32 [B][NBK+1]      CSR offsets (global pooled positions)
+//   members  i32 [B][NP]         pooled ids, ascending inside a bucket
+//   assign   i16 [B][NP]         bucket m inside the block
+//   open     i32 [B][G]          bucket of each completed open-block group, -1 if none
+//   status   u32 [8]             [0] first error code, [1] fallback count,
+//                                [2] error detail
+// with NP = T_cap / p pooled groups and NBK = (NP / G) * k buckets.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lsa.h"
+
+namespace lsa {
+
+constexpr int DL = 64;         // latent dimension (the pages' 64-d index)
+constexpr int KC = 64;         // candidate buckets nominated per query
+constexpr int MAX_K = 32;      // buckets per block supported by the kernels
+
+// Device-visible view of an index (passed by value to kernels).
+struct IndexView {
+    int64_t B;
+    int64_t T_cap;
+    int64_t NP;        // pooled groups per sequence (capacity)
+    int64_t NBK;       // buckets per sequence (capacity)
+    int p, G, k, L;
+    int nblk_max;
+    lsa_dtype dtype;
+    float* pooled;
+    float* unit;
+    float* cent;
+    void* cent_rt;
+    int32_t* offsets;
+    int32_t* members;
+    int16_t* assign;
+    int32_t* open_bucket;
+    uint32_t* status;
+};
+
+// Where a query's position comes from: an int32 array [B][Nq] or base + i.
+struct PosSrc {
+    const int32_t* arr;
+    int64_t base;
+    __host__ __device__ int64_t at(int64_t b, int64_t nq, int64_t i) const
+    {
+        return arr ? (int64_t)arr[b * nq + i] : base + i;
+    }
+};
+
+// Status codes written by kernels (first one wins).
+enum DevErr : uint32_t {
+    DEV_OK = 0,
+    DEV_OPEN_FULL = 1,     // decode append found the open block full
+    DEV_BAD_INDEX = 2,     // an index outside [0, T_cap) reached a gather
+    DEV_FALLBACK_OVF = 3,  // fallback list overflow (cannot happen by sizing)
+    DEV_TIMEOUT = 4,       // a bounded wait on a copy gave up
+};
+
+__device__ __forceinline__ void dev_error(uint32_t* status, uint32_t code, uint32_t detail)
+{
+    if (atomicCAS(status, 0u, code) == 0u) status[2] = detail;
+}
+
+__device__ __forceinline__ float load_elt(const float* p) { return *p; }
+__device__ __forceinline__ float load_elt(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+// ---------------------------------------------------------------------------
+// Launchers (each enqueues on `st`; returns cudaGetLastError()).
+// ---------------------------------------------------------------------------
+
+// Pool + normalise pooled groups [j0, j1) of every sequence.
+cudaError_t launch_pool_unit(const IndexView& ix, const void* latent_K, int64_t j0, int64_t j1,
+                             cudaStream_t st);
+
+// Spherical k-means of blocks [b0, b1) of every sequence (L Lloyd iterations),
+// CSR records and the retrieval copy.  Needs `unit` of those blocks.
+cudaError_t launch_kmeans(const IndexView& ix, int64_t b0, int64_t b1, cudaStream_t st);
+
+// Reset the open block (every slot -1) and assign its completed groups
+// [n_blk*G, j_end) to their nearest closed centroid.  Needs `unit` rows.
+cudaError_t launch_open_assign(const IndexView& ix, int64_t n_blk, int64_t j_end,
+                               cudaStream_t st);
+
+// Selection workspace carve-up.
+struct SelectWs {
+    int32_t* cand;       // [B][Nq][KC] candidate bucket ids (-1 padded)
+    float* tau;          // [B][Nq]     approximate score bound of non-candidates
+    int32_t* ncand;      // [B][Nq]
+    int32_t* fb_list;    // [B*Nq]      queries that need the exact fallback
+    int32_t* fb_count;   // [1]
+    double* fb_scores;   // [FB_CTAS][NBK] scratch of the fallback
+};
+constexpr int FB_CTAS = 148;
+size_t select_ws_bytes(const IndexView& ix, int64_t Nq);
+SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq);
+
+cudaError_t launch_select(const IndexView& ix, int64_t n_blk, const void* latent_Q, PosSrc pos,
+                          int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
+                          int s_max, const SelectWs& ws, bool use_tc, cudaStream_t st);
+
+// Sparse attention (status nullable: receives DEV_BAD_INDEX / DEV_TIMEOUT).
+cudaError_t launch_attn_status(const void* Q, const void* K, const void* V, lsa_dtype dt,
+                               int64_t B, int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
+                               const int32_t* indices, const int32_t* counts, int s_max,
+                               float scale, void* O, float* lse, uint32_t* status,
+                               cudaStream_t st);
+// True when the tensor-core candidate scorer is compiled in.
+bool tc_scoring_available();
+
+cudaError_t launch_attn(const void* Q, const void* K, const void* V, lsa_dtype dt, int64_t B,
+                        int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
+                        const int32_t* indices, const int32_t* counts, int s_max, float scale,
+                        void* O, float* lse, cudaStream_t st);
+
+}  // namespace lsa
+
+struct lsa_index {
+    lsa::IndexView v;
+    int64_t n_blk;       // closed blocks (host-side counter)
+    void* buf;
+    size_t bytes;
+    bool status_clean;   // status words cleared on the device
+};

@@ -1,0 +1,116 @@
+"""The C-ABI library loads on a host without a GPU, exports every entry point
+that include/lsa.h declares, and rejects bad arguments on the host before any
+launch.  No call here reaches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_indexing_b200 as lsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(lsa_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported():
+    lib = ctypes.CDLL(lsa.library_path())
+    names = _declared()
+    assert len(names) >= 15
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_version_and_empty_error():
+    assert b"D-LSA" in lsa._lib.lsa_version()
+
+
+def test_index_bytes_validation():
+    P = lsa.IndexParams
+    good = P(4, 1024, 16, 3)
+    n = lsa._lib.lsa_index_bytes(1, 1 << 20, good, lsa.BF16)
+    # pooled + unit (2 * NP * 64 * 4) dominate; everything 256-byte aligned
+    NP = (1 << 20) // 4
+    assert n >= 2 * NP * 64 * 4 and n % 256 == 0
+    for bad in [P(0, 1024, 16, 3), P(4, 1024, 0, 3), P(4, 16, 32, 3), P(4, 1024, 16, 0),
+                P(4, 1024, 64, 3)]:
+        assert lsa._lib.lsa_index_bytes(1, 1 << 20, bad, lsa.BF16) == 0
+        assert lsa._lib.lsa_last_error() != b""
+    assert lsa._lib.lsa_index_bytes(0, 1 << 20, good, lsa.BF16) == 0
+    assert lsa._lib.lsa_index_bytes(1, 100, good, lsa.BF16) == 0        # no whole block
+    assert lsa._lib.lsa_index_bytes(1, 1 << 20, good, 7) == 0           # bad dtype
+
+
+def test_index_init_checks_buffer():
+    P = lsa.IndexParams(4, 256, 8, 3)
+    need = lsa._lib.lsa_index_bytes(1, 8192, P, lsa.F32)
+    h = ctypes.c_void_p()
+    # NULL buffer, misaligned buffer, short buffer: all rejected on the host
+    assert lsa._lib.lsa_index_init(None, need, 1, 8192, P, lsa.F32, ctypes.byref(h)) == 1
+    assert lsa._lib.lsa_index_init(ctypes.c_void_p(4096 + 16), need, 1, 8192, P, lsa.F32,
+                                   ctypes.byref(h)) == 2
+    assert lsa._lib.lsa_index_init(ctypes.c_void_p(4096), need - 1, 1, 8192, P, lsa.F32,
+                                   ctypes.byref(h)) == 3
+    # a fake (never dereferenced on the host) aligned address is accepted
+    assert lsa._lib.lsa_index_init(ctypes.c_void_p(1 << 20), need, 1, 8192, P, lsa.F32,
+                                   ctypes.byref(h)) == 0
+    assert lsa._lib.lsa_index_num_blocks(h) == 0
+    # select / prefill argument checks fire before any launch
+    fake = ctypes.c_void_p(1 << 21)
+    S = lsa.SelectParams
+    ws = lsa._lib.lsa_select_workspace_bytes(h, 16)
+    assert ws > 0
+    rc = lsa._lib.lsa_select(h, fake, fake, 16, S(512, 64, 4), fake, fake, 100, fake, ws, None)
+    assert rc == 1 and b"s_max" in lsa._lib.lsa_last_error()
+    rc = lsa._lib.lsa_select(h, fake, fake, 16, S(512, 2, 4), fake, fake, 600, fake, ws, None)
+    assert rc == 7                                                      # window < p - 1
+    rc = lsa._lib.lsa_select(h, fake, fake, 16, S(-1, 64, 4), fake, fake, 600, fake, ws, None)
+    assert rc == 1
+    rc = lsa._lib.lsa_select(h, fake, fake, 16, S(512, 64, 4), fake, fake, 580, fake, ws - 1, None)
+    assert rc == 3
+    rc = lsa._lib.lsa_select(h, ctypes.c_void_p((1 << 21) + 4), fake, 16, S(512, 64, 4), fake, fake,
+                             580, fake, ws, None)
+    assert rc == 2
+    # extend: gap and range checks
+    assert lsa._lib.lsa_index_extend(h, fake, 2048, 4096, None) == 1      # block 2 > 0 blocks
+    assert lsa._lib.lsa_index_extend(h, fake, 0, 9000, None) == 1         # beyond T_cap
+    lsa._lib.lsa_index_release(h)
+
+
+def test_sparse_attn_argument_checks():
+    fake = ctypes.c_void_p(1 << 22)
+    f = lsa._lib.lsa_sparse_attn
+    assert f(fake, fake, fake, lsa.BF16, 1, 4, 100, 12, 4, 128, fake, fake, 8, 0.1, fake, None,
+             None) == 7                                                 # Hq/Hkv = 3
+    assert f(fake, fake, fake, lsa.BF16, 1, 4, 100, 8, 3, 128, fake, fake, 8, 0.1, fake, None,
+             None) == 1                                                 # Hq % Hkv
+    assert f(fake, fake, fake, lsa.BF16, 1, 4, 100, 8, 1, 96, fake, fake, 8, 0.1, fake, None,
+             None) == 7                                                 # d = 96
+    assert f(fake, fake, fake, lsa.BF16, 1, 4, 100, 8, 1, 64, fake, fake, 8, 0.0, fake, None,
+             None) == 1                                                 # scale
+    assert f(None, fake, fake, lsa.BF16, 1, 4, 100, 8, 1, 64, fake, fake, 8, 0.1, fake, None,
+             None) == 1
+    assert f(ctypes.c_void_p((1 << 22) + 8), fake, fake, lsa.BF16, 1, 4, 100, 8, 1, 64, fake, fake,
+             8, 0.1, fake, None, None) == 2
+
+
+def test_calls_without_gpu_fail_cleanly():
+    # With no device, a well-formed call reaches the CUDA runtime and must come
+    # back with LSA_ERR_CUDA rather than crash.  (Skipped where a GPU exists.)
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    fake = ctypes.c_void_p(1 << 22)
+    rc = lsa._lib.lsa_sparse_attn(fake, fake, fake, lsa.BF16, 1, 4, 100, 8, 1, 64, fake, fake, 8,
+                                  0.125, fake, None, None)
+    assert rc == 4
