@@ -1,0 +1,528 @@
+"""Benchmark of the D-LSA Flat hot path on B200.
+
+Default workload: the last 32,768-query chunk of a 10,485,760-token context
+(bf16, 32 query / 4 KV heads, d = 128, 64-d latent index with p = 4,
+1024 pooled groups per block, 16 buckets per block, 3 Lloyd iterations,
+4096 long-range + 512 recent + 4 sink keys per query).  One step is one call
+of lsa_prefill_chunk: cluster the chunk's 8 blocks, select for every chunk
+query, exact sparse attention.  Inputs are synthetic (the clustered mixture of
+the `synth` module) and resident in HBM before the timed region; K and V
+(21.5 GB) are far larger than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lsa|reference]
+
+Under torchrun every rank runs an independent chunk of its own sequence
+(weak scaling, no collective on the data path); times are the max over
+ranks.  `--impl reference` times the CPU oracle (the plain-C definition of
+the method) on a bounded query sample of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "prefill 32k-chunk queries/s and decode µs/step at 10M ctx; % of HBM/TC roofline"
+PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+# ------------------------------------------------------------------ helpers --
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    rank = torch.distributed.get_rank() if ws > 1 else 0
+    return rank, ws
+
+
+def _max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(ws):
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAK_FALLBACK), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("timestamp,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows, by_uuid = [], {}
+        for ts, line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                row = (ts, float(parts[2]), float(parts[3]), parts[5:])
+            except ValueError:
+                continue
+            by_uuid.setdefault(parts[1], []).append(row)
+        if self.uuid in by_uuid:
+            rows = by_uuid[self.uuid]
+        elif len(by_uuid) == 1:
+            rows = next(iter(by_uuid.values()))
+        if not rows:
+            return None
+        inside = [r for r in rows if self.t0 - 0.05 <= r[0] <= self.t1 + 0.15] or rows
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in inside:
+            for name, flag in zip(names, r[3][1:5]):
+                if flag.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": sorted(reasons),
+                "samples": len(inside)}
+
+
+def _gpu_uuid():
+    try:
+        u = torch.cuda.get_device_properties(torch.cuda.current_device()).uuid
+        s = str(u)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    except Exception:
+        return None
+
+
+def _events_time(fn, steps, stream):
+    """Runs fn() `steps` times between two events on `stream`; returns ms per step."""
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+# ---------------------------------------------------------------- workloads --
+
+def _workload_desc(w):
+    return ("D-LSA Flat prefill of the last %d-query chunk of a %d-token context "
+            "(bf16, Hq=%d, Hkv=%d, d=%d; index p=%d, block=%d pooled, %d buckets/block, "
+            "L=%d; reads %d long-range + %d recent + %d sinks)"
+            % (w.nq, w.T, w.Hq, w.Hkv, w.d, w.p, w.G, w.k, w.L, w.R, w.W, w.S))
+
+
+def _config(w, n_gpus):
+    return {"workload": _workload_desc(w), "name": w.name, "T": w.T, "chunk_queries": w.nq,
+            "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "p": w.p, "block": w.G, "buckets": w.k,
+            "lloyd_iters": w.L, "budget": w.R, "window": w.W, "sinks": w.S,
+            "l2": "no flush: K+V (%.1f GB) far exceed L2" % (2 * w.T * w.Hkv * w.d * 2 / 1e9),
+            "parallelism": "dp%d (independent chunk per rank)" % n_gpus}
+
+
+def _attn_algorithmic_bytes(w, counts):
+    """Bytes the attention of one chunk must move: every selected K and V row
+    of every KV head, Q and O, and the index rows it reads."""
+    elt = 2 if w.dtype == "bf16" else 4
+    n_sel = int(counts.sum().item())
+    kv = n_sel * w.Hkv * w.d * elt * 2
+    qo = w.B * w.nq * w.Hq * w.d * elt * 2
+    idx = (n_sel + w.B * w.nq) * 4
+    return kv + qo + idx
+
+
+def _traffic_record(kernel):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source
+    has not changed since it was captured."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "long_context_indexing_b200", "csrc", rec["source"])
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    return rec if sha == rec.get("sha256") else None
+
+
+# --------------------------------------------------------------- the oracle --
+
+class OracleRun:
+    """The CPU oracle on a bounded query sample of a prefill workload."""
+
+    def __init__(self, w, inp, T_old):
+        import oracle
+        self.oracle = oracle
+        self.w = w
+        self.T_old = T_old
+        lat = inp["latent_K"][0].float().cpu().numpy()
+        self.lat = lat
+        span = w.p * w.G
+        self.idx = oracle.Index(w.T, w.p, w.G, w.k, w.L, rt_bf16=(w.dtype == "bf16"))
+        t = time.time()
+        self.idx.extend(lat, 0, (T_old // span) * span)
+        self.setup_s = time.time() - t
+        self.inp = inp
+
+    def step(self, rows):
+        """Chunk step on the sampled queries: extend the chunk's blocks, select,
+        attend.  Host gathers of the selected K/V rows are outside the timing."""
+        o, w, inp = self.oracle, self.w, self.inp
+        t0 = time.time()
+        self.idx.extend(self.lat, self.T_old, w.T)
+        lq = inp["latent_Q"][0][rows].float().cpu().numpy()
+        pos = (self.T_old + rows.cpu().numpy()).astype(np.int64)
+        sel, cnt, _, _ = o.select(self.idx, lq, pos, w.R, w.W, w.S)
+        t1 = time.time()
+        uniq, inv = np.unique(np.where(sel >= 0, sel, 0), return_inverse=True)
+        remap = np.where(sel >= 0, inv.reshape(sel.shape), -1).astype(np.int32)
+        ui = torch.from_numpy(uniq).to(inp["K"].device)
+        K = inp["K"][0].index_select(0, ui).float().cpu().numpy()
+        V = inp["V"][0].index_select(0, ui).float().cpu().numpy()
+        Q = inp["Q"][0][rows].float().cpu().numpy()
+        t2 = time.time()
+        O, _ = o.attend(Q, K, V, remap, cnt, o.default_scale(w.d))
+        t3 = time.time()
+        return (t1 - t0) + (t3 - t2), O
+
+
+def _sample_rows(w, n, device):
+    stride = max(1, w.nq // n)
+    return torch.arange(0, n * stride, stride, device=device)[:n]
+
+
+# ---------------------------------------------------------------------- lsa --
+
+def _bench_workload(args):
+    over = {}
+    if args.T:
+        over["T"] = args.T
+    if args.nq:
+        over["nq"] = args.nq
+    return synth.workload(args.workload, **over)
+
+
+def run_lsa(args, rank, ws):
+    import long_context_indexing_b200 as lsa
+
+    w = _bench_workload(args)
+    torch.manual_seed(rank)
+    dev = torch.device("cuda")
+    inp = synth.prefill_inputs(w, seed=args.seed + rank, device=dev)
+    span = w.p * w.G
+    T_old = w.T - w.nq
+    idx = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16 if w.dtype == "bf16" else lsa.F32)
+    t = time.time()
+    idx.build(inp["latent_K"], (T_old // span) * span)
+    torch.cuda.synchronize()
+    build_s = time.time() - t
+    ws_bytes = lsa.lsa_prefill_workspace_bytes(idx, w.nq, w.R, w.W, w.S)
+    work = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    O = torch.empty_like(inp["Q"])
+    stream = torch.cuda.current_stream()
+
+    def step():
+        lsa.lsa_prefill_chunk(idx, inp["latent_K"], inp["latent_Q"], inp["Q"], inp["K"],
+                              inp["V"], T_old, w.T, w.R, w.W, w.S, workspace=work, out=O)
+
+    for _ in range(args.warmup):
+        step()
+    _barrier(ws)
+    sampler = ClockSampler(_gpu_uuid()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    launches0 = lsa.kernel_launches()
+    if sampler:
+        sampler.mark("t0")
+    ms = _events_time(step, args.steps, stream)
+    if sampler:
+        sampler.mark("t1")
+    launches = lsa.kernel_launches() - launches0
+    _barrier(ws)
+    clocks = sampler.stop() if sampler else None
+    ms = _max_over_ranks(ms, ws)
+    fallbacks = idx.check()
+
+    # Stage breakdown through the standalone entry points (same work, same stream).
+    sel_i, sel_c = lsa.prefill_selection_views(work, w.B, w.nq, w.s_max)
+    pos = torch.arange(T_old, w.T, device=dev, dtype=torch.int32).expand(w.B, w.nq).contiguous()
+    sel_ws = torch.empty(max(1, lsa._lib.lsa_select_workspace_bytes(idx.handle, w.nq)),
+                         dtype=torch.uint8, device=dev)
+    stage_ms = {
+        "index_extend": _events_time(lambda: idx.extend(inp["latent_K"], T_old, w.T),
+                                     args.steps, stream),
+        "select": _events_time(lambda: lsa.lsa_select(idx, inp["latent_Q"], pos, w.R, w.W, w.S,
+                                                      workspace=sel_ws), args.steps, stream),
+        "sparse_attn": _events_time(lambda: lsa.lsa_sparse_attn(inp["Q"], inp["K"], inp["V"],
+                                                                sel_i, sel_c, out=O),
+                                    args.steps, stream),
+    }
+    attn_ms = _max_over_ranks(stage_ms["sparse_attn"], ws)
+    peaks, peak_src = _peaks()
+    alg = _attn_algorithmic_bytes(w, sel_c)
+    achieved = alg / (attn_ms * 1e-3) / 1e9
+    traffic = _traffic_record("attn_bf16_kernel")
+    roofline = {"kernel": "attn_bf16_kernel", "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "peak_source": "%s (copy bandwidth)" % peak_src,
+                "algorithmic_bytes_per_launch": alg,
+                "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
+                "launch_ms": round(attn_ms, 4)}
+
+    # End to end through the C-ABI with host buffers: H2D of the step's inputs
+    # (the chunk's new latent/K/V rows, latent queries, queries), the fused
+    # call, D2H of the output.
+    h = {k: inp[k][:, T_old:w.T].cpu().pin_memory() for k in ("latent_K", "K", "V")}
+    hq = {k: inp[k].cpu().pin_memory() for k in ("latent_Q", "Q")}
+    hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in list(h.values()) + list(hq.values()))
+    d2h = hO.numel() * hO.element_size()
+
+    def e2e_step():
+        for k in ("latent_K", "K", "V"):
+            inp[k][:, T_old:w.T].copy_(h[k], non_blocking=True)
+        for k in ("latent_Q", "Q"):
+            inp[k].copy_(hq[k], non_blocking=True)
+        step()
+        hO.copy_(O, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    _barrier(ws)
+    e2e_ms = _max_over_ranks(_events_time(e2e_step, args.steps, stream), ws)
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        orc = OracleRun(w, inp, T_old)
+        rows = _sample_rows(w, args.cpu_queries, dev)
+        t_s, O_ref = orc.step(rows)
+        err = float(np.abs(O[0][rows].float().cpu().numpy() - O_ref).max())
+        cpu = {"value": round(len(rows) / t_s, 3), "unit": "queries/s",
+               "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": "%d of the %d chunk queries (every %d-th); chunk index build + selection "
+                         "+ attention; prefix index built untimed in %.1f s"
+                         % (len(rows), w.nq, w.nq // len(rows), orc.setup_s),
+               "max_abs_diff_vs_gpu": err}
+
+    decode = None
+    if not args.no_decode:
+        del inp, idx, work, O, sel_ws, h, hq, hO
+        torch.cuda.empty_cache()
+        decode = run_decode(args, peaks, peak_src, ws)
+
+    value = ws * w.nq / (ms * 1e-3)
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "queries/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic (seeded clustered mixture; no model weights or datasets)",
+            "config": _config(w, ws), "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": round(ws * w.nq / (e2e_ms * 1e-3), 2), "unit": "queries/s",
+                    "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches, "clocks": clocks,
+            "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "index_build_prefix_s": round(build_s, 3), "selection_fallbacks": fallbacks,
+            "decode": decode}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- decode --
+
+def run_decode(args, peaks, peak_src, ws=1):
+    """Decode workload: 8 sequences of 1,048,576-token context, one new token
+    per sequence per step, 256 steps captured once in a CUDA graph and
+    replayed.  Each step appends the token (and, every p-th token, the
+    completed pooled group), selects 4096 + 512 + 4 keys and attends over them.
+    Replays are idempotent: they rewrite the same rows and re-derive the same
+    open-list entries."""
+    import long_context_indexing_b200 as lsa
+
+    w = synth.workload("decode")
+    dev = torch.device("cuda")
+    span = w.p * w.G
+    t_cap = w.T + span                      # room for the open block
+    inp = synth.decode_inputs(w, seed=args.seed, device=dev, t_cap=t_cap)
+    idx = lsa.LsaIndex(w.B, t_cap, w.p, w.G, w.k, w.L, lsa.BF16)
+    idx.build(inp["latent_K"], w.T)
+    pos = (w.T + torch.arange(w.steps, device=dev, dtype=torch.int32))[:, None]
+    pos = pos.expand(w.steps, w.B).contiguous()
+    O = torch.empty(w.steps, w.B, w.Hq, w.d, dtype=torch.bfloat16, device=dev)
+    ws_bytes = lsa.lsa_decode_workspace_bytes(idx, w.Hq, w.Hkv, w.d, w.R, w.W, w.S)
+    work = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def step(s):
+        lsa.lsa_decode_step(idx, inp["latent_K"], inp["K"], inp["V"], inp["new_latent_k"][s],
+                            inp["new_k"][s], inp["new_v"][s], inp["latent_q"][s], inp["q"][s],
+                            pos[s], w.R, w.W, w.S, workspace=work, out=O[s])
+
+    for s in range(w.steps):                # eager warm-up pass
+        step(s)
+    torch.cuda.synchronize()
+    idx.check()
+    l0 = lsa.kernel_launches()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for s in range(w.steps):
+            step(s)
+    launches_per_step = (lsa.kernel_launches() - l0) / w.steps
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    reps = max(1, args.steps // 2)
+    ms = _events_time(graph.replay, reps, stream)
+    us = _max_over_ranks(1e3 * ms / w.steps, ws)
+    idx.check()
+    _, counts = lsa.decode_selection_views(work, w.B, w.s_max)
+    n_sel = int(counts.sum().item())
+    kv = n_sel * w.Hkv * w.d * 2 * 2
+    qo = w.B * w.Hq * w.d * 2 * 2
+    cent = w.B * (w.T // span) * w.k * 64 * 2
+    alg = kv + qo + cent + n_sel * 4
+    achieved = alg / (us * 1e-6) / 1e9
+    del graph
+    return {"value": round(us, 3), "unit": "µs/step", "higher_is_better": False,
+            "workload": "D-LSA Flat decode: %d sequences x %d-token context, 1 query/sequence/step, "
+                        "%d steps in one CUDA graph, replayed %d times" % (w.B, w.T, w.steps, reps),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                         "peak_source": "%s (copy bandwidth)" % peak_src,
+                         "algorithmic_bytes_per_step": alg},
+            "gpu_launches_per_step": launches_per_step}
+
+
+# ---------------------------------------------------------------- reference --
+
+def run_reference(args, rank, ws):
+    if rank != 0:
+        return
+    import oracle
+    w = _bench_workload(args)
+    dev = torch.device("cuda") if torch.cuda.is_available() else torch.device("cpu")
+    inp = synth.prefill_inputs(w, seed=args.seed, device=dev)
+    T_old = w.T - w.nq
+    orc = OracleRun(w, inp, T_old)
+    rows = _sample_rows(w, args.ref_queries, dev)
+    for _ in range(args.warmup):
+        orc.step(rows)
+    times = [orc.step(rows)[0] for _ in range(args.steps)]
+    t = sum(times) / len(times)
+    value = len(rows) / t
+    sample = ("%d of the %d chunk queries per step (every %d-th): chunk index build + selection "
+              "+ attention" % (len(rows), w.nq, w.nq // len(rows)))
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "queries/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * t, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(w, ws),
+            "cpu_baseline": {"value": round(value, 3), "unit": "queries/s",
+                             "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "queries/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["lsa", "reference"], default="lsa")
+    ap.add_argument("--workload", default="10m", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--T", type=int, default=None, help="override the context length")
+    ap.add_argument("--nq", type=int, default=None, help="override the chunk query count")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-queries", type=int, default=128)
+    ap.add_argument("--ref-queries", type=int, default=32)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode measurement (prints its object)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, ws = _dist()
+    try:
+        if args.decode_only:
+            peaks, src = _peaks()
+            out = run_decode(args, peaks, src, ws)
+            if rank == 0:
+                print(json.dumps(out), flush=True)
+        elif args.impl == "reference":
+            run_reference(args, rank, ws)
+        else:
+            run_lsa(args, rank, ws)
+    finally:
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -101,6 +101,10 @@ const char* lsa_last_error(void);
 /* Library version string. */
 const char* lsa_version(void);
 
+/* Number of CUDA kernel launches this library has enqueued in the process so
+ * far (all threads, all devices).  Host-side counter, never synchronises. */
+uint64_t lsa_kernel_launches(void);
+
 /* ---------------------------------------------------------------------------
  * Content index  ("un indice gerarchico", paragraph on index construction)
  *
@@ -222,6 +226,35 @@ lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* l
                              const void* Q, const void* K, const void* V, int64_t T_old,
                              int64_t T_new, int Hq, int Hkv, int d, lsa_select_params sp,
                              void* workspace, size_t ws_bytes, void* O, void* stream);
+
+/* Workspace bytes for lsa_decode_step (depends on the device's SM count). */
+size_t lsa_decode_workspace_bytes(const lsa_index* idx, int Hq, int Hkv, int d,
+                                  lsa_select_params sp);
+
+/* One decode step for every sequence ("Latent Sparse Attention: Towards
+ * Subquadratic Ultra-Long Context Attention", section "Full text": LSA also
+ * speeds up decode; the index maintenance below is this library's reading).
+ * Sequence b's new token sits at position pos[b] (device int32 [B]; keys
+ * [0, pos[b]) already in the caches, pos[b] in the open block that follows
+ * the index's closed blocks).  Steps, all on `stream`:
+ *   1. write new_latent_k [B][64], new_k / new_v [B][Hkv][d] to position
+ *      pos[b] of latent_K, K, V ([B][T_cap][...]);
+ *   2. if (pos[b]+1) % p == 0, pool and normalise the completed group and
+ *      append it to the bucket of its nearest closed centroid (exact binary64
+ *      score, lowest bucket id on ties); an open block that is already full
+ *      records LSA_ERR_INTERNAL in the status word (lsa_index_check) and the
+ *      group is not appended;
+ *   3. select for latent_q [B][64] at pos[b] exactly as lsa_select does;
+ *   4. exact attention of q [B][Hq][d] over the selection into O [B][Hq][d]
+ *      (split over keys, partials combined in fp32), scale 1/sqrt(d).
+ * The selection of step 3 never depends on the append of step 2 (a group
+ * that completes at pos lies inside the recent window), so the two run
+ * concurrently.  Graph-capturable: no synchronisation, no allocation. */
+lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
+                           const void* new_latent_k, const void* new_k, const void* new_v,
+                           const void* latent_q, const void* q, const int32_t* pos, int Hq,
+                           int Hkv, int d, lsa_select_params sp, void* workspace, size_t ws_bytes,
+                           void* O, void* stream);
 
 #ifdef __cplusplus
 }

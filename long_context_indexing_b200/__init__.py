@@ -19,7 +19,8 @@ import torch
 __all__ = [
     "LsaError", "LsaIndex", "lsa_index_bytes", "lsa_build_index", "lsa_select",
     "lsa_sparse_attn", "lsa_prefill_chunk", "lsa_prefill_workspace_bytes",
-    "library_path", "F32", "BF16",
+    "lsa_decode_workspace_bytes", "lsa_decode_step", "library_path", "kernel_launches", "F32",
+    "BF16",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -52,6 +53,7 @@ def _declare(lib):
     sigs = {
         "lsa_last_error": ([], ctypes.c_char_p),
         "lsa_version": ([], ctypes.c_char_p),
+        "lsa_kernel_launches": ([], ctypes.c_uint64),
         "lsa_index_bytes": ([I64, I64, IndexParams, I], SZ),
         "lsa_index_init": ([P, SZ, I64, I64, IndexParams, I, ctypes.POINTER(P)], I),
         "lsa_index_release": ([P], None),
@@ -66,6 +68,8 @@ def _declare(lib):
         "lsa_prefill_workspace_bytes": ([P, I64, SelectParams], SZ),
         "lsa_prefill_chunk": ([P, P, P, P, P, P, I64, I64, I, I, I, SelectParams, P, SZ, P, P],
                               I),
+        "lsa_decode_workspace_bytes": ([P, I, I, I, SelectParams], SZ),
+        "lsa_decode_step": ([P, P, P, P, P, P, P, P, P, P, I, I, I, SelectParams, P, SZ, P, P], I),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -86,6 +90,11 @@ _lib = _load()
 
 def library_path():
     return _LIB_PATH
+
+
+def kernel_launches():
+    """Kernel launches liblsa has enqueued in this process so far."""
+    return int(_lib.lsa_kernel_launches())
 
 
 def _check(rc):
@@ -278,4 +287,43 @@ def prefill_selection_views(workspace, B, Nq, s_max):
     al = (n_idx * 4 + 255) // 256 * 256
     indices = workspace[: n_idx * 4].view(torch.int32).view(B, Nq, s_max)
     counts = workspace[al: al + B * Nq * 4].view(torch.int32).view(B, Nq)
+    return indices, counts
+
+
+def lsa_decode_workspace_bytes(index, Hq, Hkv, d, budget, window, sinks):
+    n = int(_lib.lsa_decode_workspace_bytes(index.handle, Hq, Hkv, d,
+                                            SelectParams(budget, window, sinks)))
+    if n == 0:
+        raise LsaError(1, _lib.lsa_last_error().decode())
+    return n
+
+
+def lsa_decode_step(index, latent_K, K, V, new_latent_k, new_k, new_v, latent_q, q, pos, budget,
+                    window, sinks, workspace=None, out=None, stream=None):
+    """One decode step for every sequence (new token at pos[b]); returns O [B][Hq][d].
+
+    The caches latent_K, K, V [B][T_cap][...] are updated in place at pos."""
+    _cuda(latent_K, K, V, new_latent_k, new_k, new_v, latent_q, q, pos, out)
+    if pos.dtype != torch.int32:
+        raise TypeError("pos must be int32")
+    B, Hq, d = q.shape
+    Hkv = K.shape[2]
+    need = lsa_decode_workspace_bytes(index, Hq, Hkv, d, budget, window, sinks)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    O = out if out is not None else torch.empty_like(q)
+    _check(_lib.lsa_decode_step(index.handle, _ptr(latent_K), _ptr(K), _ptr(V), _ptr(new_latent_k),
+                                _ptr(new_k), _ptr(new_v), _ptr(latent_q), _ptr(q), _ptr(pos), Hq,
+                                Hkv, d, SelectParams(budget, window, sinks), _ptr(workspace),
+                                workspace.numel(), _ptr(O), _stream(stream)))
+    return O
+
+
+def decode_selection_views(workspace, B, s_max):
+    """(indices [B][s_max], counts [B]) views of the selection a decode step left in
+    `workspace`."""
+    n_idx = B * s_max
+    al = (n_idx * 4 + 255) // 256 * 256
+    indices = workspace[: n_idx * 4].view(torch.int32).view(B, s_max)
+    counts = workspace[al: al + B * 4].view(torch.int32).view(B)
     return indices, counts

@@ -10,17 +10,14 @@
 // The selection is shared by every query head; query head h reads KV head
 // h / (Hq/Hkv).  Both kernels use an fp32 online softmax.
 //
-// bf16 kernel (the hot one).  One CTA per (query, KV head), 4 warps; warp w
-// takes the 16-key tiles w, w+4, w+8, ... of the query's selection and keeps
-// its own online-softmax state; the warps merge at the end.  Each warp owns a
-// STAGES-deep ring of K and V tiles filled by per-row bulk copies
-// (cp.async.bulk, one per key row of d bf16) into padded shared-memory rows
-// (pitch = 2d + 16 bytes, so ldmatrix rows fall in distinct banks), completed
-// on one mbarrier per stage.  The logits are computed transposed,
-// S^T = K Q^T (keys on the MMA M dimension, the <= 8 heads of the KV group on
-// N), so no MMA row is padding; P^T is turned into the B operand of
-// O^T = V^T P^T with movmatrix, and V^T comes from ldmatrix.trans.
+// bf16 kernel (the hot one): see the comment above attn_bf16_kernel.  The
+// logits are computed transposed, S^T = K Q^T (keys on the MMA M dimension,
+// the <= 8 query heads of a KV head on N), so no MMA row is padding; P^T
+// becomes the B operand of O^T = V^T P^T through movmatrix, and V^T comes
+// from ldmatrix.trans.
 #include <math.h>
+
+#include <mutex>
 
 #include "lsa_internal.cuh"
 #include "ptx.cuh"
@@ -160,240 +157,323 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__
 
 // ---------------------------------------------------------------------------
 // bf16 tensor-core kernel.
+//
+// CTA = one query row and one group of HG <= 4 KV heads (and one key split
+// when split-KV is on).  Warp 4 is the producer: for every stage it copies the
+// KT selected keys' rows for the whole head group (HG*d bf16, contiguous in
+// the token-major cache) for K and for V with one bulk copy each into padded
+// shared-memory rows, completing on the stage's "full" mbarrier.  Warps 0-3
+// consume: warp w serves KV head w % HG and the 16-key slice w / HG of every
+// stage (KT = 16 * 4 / HG keys per stage), then arrives on the stage's
+// "empty" mbarrier.  At the end the warps of each head merge their
+// online-softmax states.  With NS > 1 splits, each CTA writes an fp32
+// partial (max, sum, unnormalised output) per query head; the last CTA of a
+// (row, head group) to finish -- an atomic counter, no waiting -- combines them.
 // ---------------------------------------------------------------------------
-constexpr int ATT_WARPS = 4;
+constexpr int CONS_WARPS = 4;
+constexpr int ATT_THREADS = (CONS_WARPS + 1) * 32;
 
-template <int D, int STAGES>
-struct AttnSmem {
-    static constexpr int ROWB = D * 2;            // bytes of one key row of one KV head
-    static constexpr int PITCH = ROWB + 16;       // padded shared-memory row
-    static constexpr int TILE = 16 * PITCH;       // one 16-key tile of K (or V)
-    static constexpr int WARP_BYTES = STAGES * 2 * TILE;
-    static constexpr int MERGE_BYTES = ATT_WARPS * 8 * (D + 2) * 4;
-    static constexpr int RING = ATT_WARPS * WARP_BYTES;
-    static constexpr int BYTES = (RING > MERGE_BYTES ? RING : MERGE_BYTES) + ATT_WARPS * STAGES * 8;
+template <int D, int HG, int STAGES>
+struct AttnCfg {
+    static constexpr int WPG = CONS_WARPS / HG;     // warps per KV head
+    static constexpr int KT = 16 * WPG;             // keys per stage
+    static constexpr int RB = HG * D * 2;           // bytes of one key's head-group row
+    static constexpr int PITCH = RB + 16;           // padded shared-memory row
+    static constexpr int TILE = KT * PITCH;         // K (or V) bytes of a stage
+    static constexpr int STAGE = 2 * TILE;
+    static constexpr int RING = STAGES * STAGE;
+    static constexpr int MERGE = CONS_WARPS * 8 * (D + 2) * 4;
+    static constexpr int BODY = RING > MERGE ? RING : MERGE;
+    static constexpr int BYTES = BODY + 2 * STAGES * 8 + 16;
 };
 
-template <int D, int STAGES>
-__global__ void __launch_bounds__(ATT_WARPS * 32) attn_bf16_kernel(
+struct SplitKV {
+    int ns;              // splits per (row, head group); 1 = off
+    int keys_per_split;  // multiple of the stage size
+    float* part;         // [rows][ns][Hq][D + 2]  (m, l, acc[D])
+    uint32_t* counter;   // [rows * n_hgroups], zero before the launch
+};
+
+template <int D, int HG, int STAGES>
+__global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
     const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
     const __nv_bfloat16* __restrict__ V, int64_t Nq, int64_t T_cap, int Hq, int Hkv, int hpg,
     const int32_t* __restrict__ indices, const int32_t* __restrict__ counts, int s_max,
-    float scale_log2, __nv_bfloat16* O, float* lse, uint32_t* status)
+    float scale_log2, __nv_bfloat16* O, float* lse, uint32_t* status, SplitKV sk)
 {
-    using SM = AttnSmem<D, STAGES>;
+    using C = AttnCfg<D, HG, STAGES>;
     constexpr int KSTEPS = D / 16;
     extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (SM::BYTES - ATT_WARPS * STAGES * 8));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BODY);
+    uint64_t* empty = full + STAGES;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = blockIdx.x / Hkv;
-    const int g = blockIdx.x % Hkv;
+    const int n_hg = Hkv / HG;
+    const int64_t unit = blockIdx.x / sk.ns;        // (row, head group)
+    const int split = blockIdx.x % sk.ns;
+    const int64_t row = unit / n_hg;
+    const int g0 = (int)(unit % n_hg) * HG;           // first KV head of the group
     const int64_t b = row / Nq;
     const int32_t* idx = indices + row * (int64_t)s_max;
-    const int n = min(counts[row], s_max);  // never read past the row
-    unsigned char* ring = smem + warp * SM::WARP_BYTES;
-    uint64_t* wbar = bars + warp * STAGES;
+    const int n_all = min(counts[row], s_max);        // never read past the row
+    const int k_lo = split * sk.keys_per_split;
+    const int k_hi = min(n_all, k_lo + sk.keys_per_split);
+    const int n = max(0, k_hi - k_lo);               // keys of this CTA
+    const int n_st = (n + C::KT - 1) / C::KT;
 
-    if (lane == 0)
-        for (int s = 0; s < STAGES; ++s) ptx::mbar_init(&wbar[s], 1);
-    ptx::fence_mbar_init();
-    __syncwarp();
-
-    // Q^T fragments (B operand): head n = lane/4, dims 2*(lane%4) + {0,1} (+8).
-    uint32_t qf[KSTEPS][2];
-    {
-        const int h = lane >> 2;
-        const bool live = h < hpg;
-        const __nv_bfloat16* qrow = Q + (row * Hq + (int64_t)g * hpg + (live ? h : 0)) * D;
-#pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk) {
-            const int c = kk * 16 + 2 * (lane & 3);
-            qf[kk][0] = live ? *reinterpret_cast<const uint32_t*>(qrow + c) : 0u;
-            qf[kk][1] = live ? *reinterpret_cast<const uint32_t*>(qrow + c + 8) : 0u;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], CONS_WARPS);
         }
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
     }
+    __syncthreads();
 
-    const int n_tiles = (n + 15) >> 4;
-    // tiles of this warp: t = warp + ATT_WARPS * j
-    const int my_tiles = (n_tiles > warp) ? (n_tiles - warp + ATT_WARPS - 1) / ATT_WARPS : 0;
-    const int32_t last_valid = (n > 0) ? n - 1 : 0;
-    bool timed_out = false;
-
-    auto issue = [&](int j) {
-        const int s = j % STAGES;
-        const int t = warp + ATT_WARPS * j;
-        unsigned char* kt = ring + s * 2 * SM::TILE;
-        unsigned char* vt = kt + SM::TILE;
-        if (lane == 0) ptx::mbar_arrive_expect_tx(&wbar[s], 2u * 16u * SM::ROWB);
-        __syncwarp();
-        const int r = lane & 15;
-        int key = t * 16 + r;
-        if (key > last_valid) key = last_valid;
-        const int32_t kidx = checked_index(idx[key], T_cap, status);
-        const int64_t off = ((b * T_cap + kidx) * Hkv + g) * (int64_t)D;
-        if (lane < 16)
-            ptx::bulk_g2s(kt + r * SM::PITCH, K + off, SM::ROWB, &wbar[s]);
-        else
-            ptx::bulk_g2s(vt + r * SM::PITCH, V + off, SM::ROWB, &wbar[s]);
-    };
-
-    for (int j = 0; j < STAGES && j < my_tiles; ++j) issue(j);
-
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float oacc[KSTEPS][4];
 #pragma unroll
     for (int mt = 0; mt < KSTEPS; ++mt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) oacc[mt][e] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
-    int j_stop = my_tiles;
-    for (int j = 0; j < my_tiles; ++j) {
-        const int s = j % STAGES;
-        const uint32_t parity = (uint32_t)((j / STAGES) & 1);
-        if (!ptx::mbar_wait_bounded(&wbar[s], parity, WAIT_LIMIT)) {
-            timed_out = true;
-            j_stop = j;
-            break;
+    if (warp == CONS_WARPS) {
+        // ---------------- producer ----------------
+        const int32_t last = (n_all > 0) ? idx[n_all - 1] : 0;
+        for (int j = 0; j < n_st; ++j) {
+            const int s = j % STAGES;
+            const uint32_t ph = (uint32_t)((j / STAGES) & 1);
+            if (*abort_flag) break;
+            if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1u, WAIT_LIMIT)) {
+                *abort_flag = 1;
+                if (status) dev_error(status, DEV_TIMEOUT, (uint32_t)row);
+                break;
+            }
+            if (lane == 0) ptx::mbar_arrive_expect_tx(&full[s], 2u * C::KT * C::RB);
+            __syncwarp();
+            unsigned char* kt = smem + s * C::STAGE;
+            for (int x = lane; x < 2 * C::KT; x += 32) {
+                const int r = x % C::KT;
+                const int key = k_lo + j * C::KT + r;
+                const int32_t t = checked_index(key < k_hi ? idx[key] : last, T_cap, status);
+                const int64_t off = ((b * T_cap + t) * Hkv + g0) * (int64_t)D;
+                if (x < C::KT)
+                    ptx::bulk_g2s(kt + r * C::PITCH, K + off, C::RB, &full[s]);
+                else
+                    ptx::bulk_g2s(kt + C::TILE + r * C::PITCH, V + off, C::RB, &full[s]);
+            }
         }
-        const unsigned char* kt = ring + s * 2 * SM::TILE;
-        const unsigned char* vt = kt + SM::TILE;
-        const int t = warp + ATT_WARPS * j;
-
-        // S^T[16 keys][8 heads] = K[16][D] Q^T[D][8]
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+    } else {
+        // ---------------- consumers ----------------
+        const int hl = warp % HG;              // KV head inside the group
+        const int sub = warp / HG;             // 16-key slice of every stage
+        const int g = g0 + hl;
+        uint32_t qf[KSTEPS][2];
         {
-            const unsigned char* base = kt + (lane & 15) * SM::PITCH + (lane >> 4) * 16;
+            const int h = lane >> 2;
+            const bool live = h < hpg;
+            const __nv_bfloat16* qrow = Q + (row * Hq + (int64_t)g * hpg + (live ? h : 0)) * D;
 #pragma unroll
             for (int kk = 0; kk < KSTEPS; ++kk) {
-                uint32_t a0, a1, a2, a3;
-                ptx::ldsm_x4(a0, a1, a2, a3, base + kk * 32);
-                ptx::mma_bf16_16816(sacc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                const int c = kk * 16 + 2 * (lane & 3);
+                qf[kk][0] = live ? *reinterpret_cast<const uint32_t*>(qrow + c) : 0u;
+                qf[kk][1] = live ? *reinterpret_cast<const uint32_t*>(qrow + c + 8) : 0u;
             }
         }
-        // online softmax in log2 units; keys beyond n are masked
-        const int key_lo = t * 16 + (lane >> 2), key_hi = key_lo + 8;
-        float z0 = (key_lo < n) ? sacc[0] * scale_log2 : -INFINITY;
-        float z1 = (key_lo < n) ? sacc[1] * scale_log2 : -INFINITY;
-        float z2 = (key_hi < n) ? sacc[2] * scale_log2 : -INFINITY;
-        float z3 = (key_hi < n) ? sacc[3] * scale_log2 : -INFINITY;
-        float tm0 = fmaxf(z0, z2), tm1 = fmaxf(z1, z3);
+        const int hoff = hl * D * 2;             // byte offset of this head in a row
+        for (int j = 0; j < n_st; ++j) {
+            const int s = j % STAGES;
+            const uint32_t ph = (uint32_t)((j / STAGES) & 1);
+            if (*abort_flag) break;
+            if (!ptx::mbar_wait_bounded(&full[s], ph, WAIT_LIMIT)) {
+                *abort_flag = 1;
+                if (status) dev_error(status, DEV_TIMEOUT, (uint32_t)row);
+                break;
+            }
+            const unsigned char* kt = smem + s * C::STAGE + sub * 16 * C::PITCH + hoff;
+            const unsigned char* vt = kt + C::TILE;
+            const int kbase = j * C::KT + sub * 16;   // key offset inside this CTA's keys
+            if (kbase < n) {
+                float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+                {
+                    const unsigned char* base = kt + (lane & 15) * C::PITCH + (lane >> 4) * 16;
+#pragma unroll
+                    for (int kk = 0; kk < KSTEPS; ++kk) {
+                        uint32_t a0, a1, a2, a3;
+                        ptx::ldsm_x4(a0, a1, a2, a3, base + kk * 32);
+                        ptx::mma_bf16_16816(sacc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                    }
+                }
+                const int key_lo = kbase + (lane >> 2), key_hi = key_lo + 8;
+                const float z0 = (key_lo < n) ? sacc[0] * scale_log2 : -INFINITY;
+                const float z1 = (key_lo < n) ? sacc[1] * scale_log2 : -INFINITY;
+                const float z2 = (key_hi < n) ? sacc[2] * scale_log2 : -INFINITY;
+                const float z3 = (key_hi < n) ? sacc[3] * scale_log2 : -INFINITY;
+                float tm0 = fmaxf(z0, z2), tm1 = fmaxf(z1, z3);
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) {
+                    tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, o));
+                    tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, o));
+                }
+                const float mn0 = fmaxf(m0, tm0), mn1 = fmaxf(m1, tm1);
+                const float al0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - mn0);
+                const float al1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - mn1);
+                const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
+                const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
+                const float p0 = exp2f(z0 - mu0), p1 = exp2f(z1 - mu1);
+                const float p2 = exp2f(z2 - mu0), p3 = exp2f(z3 - mu1);
+                m0 = mn0;
+                m1 = mn1;
+                l0 = l0 * al0 + (p0 + p2);
+                l1 = l1 * al1 + (p1 + p3);
+#pragma unroll
+                for (int mt = 0; mt < KSTEPS; ++mt) {
+                    oacc[mt][0] *= al0;
+                    oacc[mt][1] *= al1;
+                    oacc[mt][2] *= al0;
+                    oacc[mt][3] *= al1;
+                }
+                const uint32_t pb0 = ptx::movmatrix_t(ptx::pack_bf16(p0, p1));
+                const uint32_t pb1 = ptx::movmatrix_t(ptx::pack_bf16(p2, p3));
+                {
+                    const int mi = lane >> 3, r = lane & 7;
+                    const unsigned char* base = vt + (r + 8 * (mi >> 1)) * C::PITCH + (mi & 1) * 16;
+#pragma unroll
+                    for (int mt = 0; mt < KSTEPS; ++mt) {
+                        uint32_t a0, a1, a2, a3;
+                        ptx::ldsm_x4_t(a0, a1, a2, a3, base + mt * 32);
+                        ptx::mma_bf16_16816(oacc[mt], a0, a1, a2, a3, pb0, pb1);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&empty[s]);
+        }
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
-            tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, o));
-            tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, o));
+            l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, o);
         }
-        const float mn0 = fmaxf(m0, tm0), mn1 = fmaxf(m1, tm1);
-        const float al0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - mn0);
-        const float al1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - mn1);
-        const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
-        const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
-        const float p0 = exp2f(z0 - mu0), p1 = exp2f(z1 - mu1);
-        const float p2 = exp2f(z2 - mu0), p3 = exp2f(z3 - mu1);
-        m0 = mn0;
-        m1 = mn1;
-        l0 = l0 * al0 + (p0 + p2);
-        l1 = l1 * al1 + (p1 + p3);
-#pragma unroll
-        for (int mt = 0; mt < KSTEPS; ++mt) {
-            oacc[mt][0] *= al0;
-            oacc[mt][1] *= al1;
-            oacc[mt][2] *= al0;
-            oacc[mt][3] *= al1;
-        }
-        // P^T (C layout) -> B operand of O^T = V^T P^T
-        const uint32_t pb0 = ptx::movmatrix_t(ptx::pack_bf16(p0, p1));
-        const uint32_t pb1 = ptx::movmatrix_t(ptx::pack_bf16(p2, p3));
-        {
-            const int mi = lane >> 3, r = lane & 7;
-            const unsigned char* base = vt + (r + 8 * (mi >> 1)) * SM::PITCH + (mi & 1) * 16;
-#pragma unroll
-            for (int mt = 0; mt < KSTEPS; ++mt) {
-                uint32_t a0, a1, a2, a3;
-                ptx::ldsm_x4_t(a0, a1, a2, a3, base + mt * 32);
-                ptx::mma_bf16_16816(oacc[mt], a0, a1, a2, a3, pb0, pb1);
-            }
-        }
-        __syncwarp();
-        if (j + STAGES < my_tiles) issue(j + STAGES);
     }
+    // Copies of an aborted stage may still be in flight: give them a bounded
+    // chance to land before the ring is reused for the merge.
+    if (*abort_flag && warp == CONS_WARPS)
+        for (int j = 0; j < n_st && j < STAGES; ++j)
+            ptx::mbar_wait_bounded(&full[j % STAGES], (uint32_t)((j / STAGES) & 1), WAIT_LIMIT);
+    __syncthreads();
 
-    // After a timeout, give the copies this warp still has in flight a
-    // bounded chance to land before the ring is reused.
-    if (timed_out)
-        for (int j = j_stop; j < my_tiles && j < j_stop + STAGES; ++j)
-            ptx::mbar_wait_bounded(&wbar[j % STAGES], (uint32_t)((j / STAGES) & 1), WAIT_LIMIT);
-
-    // reduce l over the lanes sharing the same heads
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-    }
-    __syncthreads();  // every warp is done with its ring: reuse it for the merge
-    float* mw = reinterpret_cast<float*>(smem);            // [ATT_WARPS][8]
-    float* lw = mw + ATT_WARPS * 8;                         // [ATT_WARPS][8]
-    float* ow = lw + ATT_WARPS * 8;                         // [ATT_WARPS][8][D]
-    if (lane < 4) {
-        mw[warp * 8 + 2 * lane] = m0;
-        mw[warp * 8 + 2 * lane + 1] = m1;
-        lw[warp * 8 + 2 * lane] = l0;
-        lw[warp * 8 + 2 * lane + 1] = l1;
-    }
-    {
+    // ---------------- merge the warps of each head ----------------
+    float* mw = reinterpret_cast<float*>(smem);         // [CONS_WARPS][8]
+    float* lw = mw + CONS_WARPS * 8;                    // [CONS_WARPS][8]
+    float* ow = lw + CONS_WARPS * 8;                    // [CONS_WARPS][8][D]
+    if (warp < CONS_WARPS) {
+        if (lane < 4) {
+            mw[warp * 8 + 2 * lane] = m0;
+            mw[warp * 8 + 2 * lane + 1] = m1;
+            lw[warp * 8 + 2 * lane] = l0;
+            lw[warp * 8 + 2 * lane + 1] = l1;
+        }
         const int h0 = 2 * (lane & 3), dr = lane >> 2;
+        float* o = ow + (warp * 8) * D;
 #pragma unroll
         for (int mt = 0; mt < KSTEPS; ++mt) {
-            float* o = ow + (warp * 8) * D;
             o[h0 * D + mt * 16 + dr] = oacc[mt][0];
             o[(h0 + 1) * D + mt * 16 + dr] = oacc[mt][1];
             o[h0 * D + mt * 16 + dr + 8] = oacc[mt][2];
             o[(h0 + 1) * D + mt * 16 + dr + 8] = oacc[mt][3];
         }
     }
-    __shared__ int any_timeout;
-    if (threadIdx.x == 0) any_timeout = 0;
     __syncthreads();
-    if (timed_out) any_timeout = 1;
-    __syncthreads();
-    if (any_timeout && threadIdx.x == 0 && status) dev_error(status, DEV_TIMEOUT, (uint32_t)row);
-    for (int x = threadIdx.x; x < hpg * D; x += ATT_WARPS * 32) {
-        const int h = x / D, c = x % D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < ATT_WARPS; ++w) M = fmaxf(M, mw[w * 8 + h]);
-        float L = 0.f, acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < ATT_WARPS; ++w) {
-            const float sc = (mw[w * 8 + h] == -INFINITY) ? 0.f : exp2f(mw[w * 8 + h] - M);
-            L += lw[w * 8 + h] * sc;
-            acc += ow[(w * 8 + h) * D + c] * sc;
+    const bool aborted = *abort_flag != 0;
+    const int nq_heads = HG * hpg;                     // query heads of this CTA
+    const float nanf_ = __int_as_float(0x7fc00000);
+    if (sk.ns == 1) {
+        for (int x = threadIdx.x; x < nq_heads * D; x += ATT_THREADS) {
+            const int qh = x / D, c = x % D;
+            const int hl = qh / hpg, h = qh % hpg;
+            float M = -INFINITY;
+            for (int sb = 0; sb < CONS_WARPS / HG; ++sb) M = fmaxf(M, mw[(sb * HG + hl) * 8 + h]);
+            float L = 0.f, acc = 0.f;
+            for (int sb = 0; sb < CONS_WARPS / HG; ++sb) {
+                const int w = sb * HG + hl;
+                const float sc = (mw[w * 8 + h] == -INFINITY) ? 0.f : exp2f(mw[w * 8 + h] - M);
+                L += lw[w * 8 + h] * sc;
+                acc += ow[(w * 8 + h) * D + c] * sc;
+            }
+            const int64_t oh = row * Hq + (int64_t)g0 * hpg + qh;
+            O[oh * D + c] = __float2bfloat16_rn(aborted ? nanf_ : acc / L);
+            if (c == 0 && lse) lse[oh] = aborted ? nanf_ : (M + log2f(L)) * 0.69314718055994531f;
         }
-        float o = acc / L;
-        if (any_timeout) o = __int_as_float(0x7fc00000);
-        O[(row * Hq + (int64_t)g * hpg + h) * D + c] = __float2bfloat16_rn(o);
-        if (c == 0 && lse) {
-            float v = (M + log2f(L)) * 0.69314718055994531f;
-            if (any_timeout) v = __int_as_float(0x7fc00000);
-            lse[row * Hq + (int64_t)g * hpg + h] = v;
-        }
+        return;
     }
+    // split-KV: write this split's partial per query head
+    for (int x = threadIdx.x; x < nq_heads * (D + 2); x += ATT_THREADS) {
+        const int qh = x / (D + 2), c = x % (D + 2);
+        const int hl = qh / hpg, h = qh % hpg;
+        float M = -INFINITY;
+        for (int sb = 0; sb < CONS_WARPS / HG; ++sb) M = fmaxf(M, mw[(sb * HG + hl) * 8 + h]);
+        float v = 0.f;
+        if (c == 0) {
+            v = M;
+        } else {
+            for (int sb = 0; sb < CONS_WARPS / HG; ++sb) {
+                const int w = sb * HG + hl;
+                const float sc = (mw[w * 8 + h] == -INFINITY) ? 0.f : exp2f(mw[w * 8 + h] - M);
+                v += (c == 1 ? lw[w * 8 + h] : ow[(w * 8 + h) * D + (c - 2)]) * sc;
+            }
+        }
+        const int64_t qhg = (int64_t)g0 * hpg + qh;
+        sk.part[((row * sk.ns + split) * Hq + qhg) * (D + 2) + c] = aborted ? nanf_ : v;
+    }
+    __threadfence();
+    __syncthreads();
+    __shared__ uint32_t sh_last;
+    if (threadIdx.x == 0) {
+        const uint32_t prev = atomicAdd(&sk.counter[unit], 1u);
+        sh_last = (prev == (uint32_t)sk.ns - 1) ? 1u : 0u;
+    }
+    __syncthreads();
+    if (!sh_last) return;
+    __threadfence();
+    for (int x = threadIdx.x; x < nq_heads * D; x += ATT_THREADS) {
+        const int qh = x / D, c = x % D;
+        const int64_t qhg = (int64_t)g0 * hpg + qh;
+        const volatile float* pp = sk.part + (row * sk.ns * Hq + qhg) * (D + 2);
+        const int64_t sstride = (int64_t)Hq * (D + 2);
+        float M = -INFINITY;
+        for (int sp = 0; sp < sk.ns; ++sp) M = fmaxf(M, pp[sp * sstride]);
+        float L = 0.f, acc = 0.f;
+        for (int sp = 0; sp < sk.ns; ++sp) {
+            const float ms = pp[sp * sstride];
+            const float sc = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+            L += pp[sp * sstride + 1] * sc;
+            acc += pp[sp * sstride + 2 + c] * sc;
+        }
+        const int64_t oh = row * Hq + qhg;
+        O[oh * D + c] = __float2bfloat16_rn(acc / L);
+        if (c == 0 && lse) lse[oh] = (M + log2f(L)) * 0.69314718055994531f;
+    }
+    if (threadIdx.x == 0) sk.counter[unit] = 0;   // ready for the next launch
 }
 
-template <int D, int STAGES>
+template <int D, int HG, int STAGES>
 static cudaError_t launch_bf16(const void* Q, const void* K, const void* V, int64_t B, int64_t Nq,
                                int64_t T_cap, int Hq, int Hkv, const int32_t* indices,
                                const int32_t* counts, int s_max, float scale, void* O, float* lse,
-                               uint32_t* status, cudaStream_t st)
+                               uint32_t* status, SplitKV sk, cudaStream_t st)
 {
-    using SM = AttnSmem<D, STAGES>;
-    auto kern = attn_bf16_kernel<D, STAGES>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::BYTES);
+    using C = AttnCfg<D, HG, STAGES>;
+    auto kern = attn_bf16_kernel<D, HG, STAGES>;
+    cudaError_t e = ensure_smem_attr((const void*)kern, C::BYTES);
     if (e != cudaSuccess) return e;
-    const int64_t ctas = B * Nq * Hkv;
-    kern<<<(unsigned)ctas, ATT_WARPS * 32, SM::BYTES, st>>>(
+    if (sk.ns > 1 && sk.keys_per_split % C::KT != 0) return cudaErrorInvalidValue;
+    const int64_t ctas = B * Nq * (Hkv / HG) * sk.ns;
+    kern<<<(unsigned)ctas, ATT_THREADS, C::BYTES, st>>>(
         (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, Nq, T_cap, Hq,
         Hkv, Hq / Hkv, indices, counts, s_max, scale * 1.4426950408889634f, (__nv_bfloat16*)O, lse,
-        status);
+        status, sk);
+    note_launch();
     return cudaGetLastError();
 }
 
@@ -407,7 +487,68 @@ static cudaError_t launch_f32(const void* Q, const void* K, const void* V, int64
     attn_f32_kernel<HPG, D><<<(unsigned)ctas, 128, 0, st>>>(
         (const float*)Q, (const float*)K, (const float*)V, Nq, T_cap, Hq, Hkv, indices, counts,
         s_max, scale, (float*)O, lse, status);
+    note_launch();
     return cudaGetLastError();
+}
+
+// KV heads per CTA and keys per stage of the bf16 kernel for a given KV head
+// count (split sizes must be multiples of the stage).
+int attn_head_group(int Hkv) { return (Hkv % 4 == 0) ? 4 : Hkv; }
+
+int attn_stage_keys(int Hkv) { return 16 * (CONS_WARPS / attn_head_group(Hkv)); }
+
+cudaError_t ensure_smem_attr(const void* kernel, int bytes)
+{
+    constexpr int MAXDEV = 64;
+    struct Rec {
+        const void* k;
+        int dev;
+    };
+    static Rec done[256];
+    static int n_done = 0;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    for (int i = 0; i < n_done; ++i)
+        if (done[i].k == kernel && done[i].dev == dev) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    if (n_done < 256 && dev < MAXDEV) done[n_done++] = Rec{kernel, dev};
+    return cudaSuccess;
+}
+
+template <int D>
+static cudaError_t launch_bf16_d(const void* Q, const void* K, const void* V, int64_t B, int64_t Nq,
+                                 int64_t T_cap, int Hq, int Hkv, const int32_t* indices,
+                                 const int32_t* counts, int s_max, float scale, void* O,
+                                 float* lse, uint32_t* status, SplitKV sk, cudaStream_t st)
+{
+    if (Hkv % 4 == 0)
+        return launch_bf16<D, 4, 3>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale,
+                                    O, lse, status, sk, st);
+    if (Hkv == 2)
+        return launch_bf16<D, 2, 3>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale,
+                                    O, lse, status, sk, st);
+    if (Hkv == 1)
+        return launch_bf16<D, 1, 3>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale,
+                                    O, lse, status, sk, st);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_split(const void* Q, const void* K, const void* V, int64_t B, int64_t Nq,
+                              int64_t T_cap, int Hq, int Hkv, int d, const int32_t* indices,
+                              const int32_t* counts, int s_max, float scale, void* O, float* lse,
+                              uint32_t* status, int ns, int keys_per_split, float* part,
+                              uint32_t* counter, cudaStream_t st)
+{
+    SplitKV sk{ns, keys_per_split, part, counter};
+    if (d == 128)
+        return launch_bf16_d<128>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale,
+                                  O, lse, status, sk, st);
+    return launch_bf16_d<64>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale, O, lse,
+                             status, sk, st);
 }
 
 cudaError_t launch_attn_status(const void* Q, const void* K, const void* V, lsa_dtype dt, int64_t B,
@@ -417,12 +558,9 @@ cudaError_t launch_attn_status(const void* Q, const void* K, const void* V, lsa_
 {
     if (B * Nq == 0) return cudaSuccess;
     const int hpg = Hq / Hkv;
-    if (dt == LSA_BF16) {
-        if (d == 128) return launch_bf16<128, 3>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts,
-                                                 s_max, scale, O, lse, status, st);
-        return launch_bf16<64, 4>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale, O,
-                                  lse, status, st);
-    }
+    if (dt == LSA_BF16)
+        return launch_attn_split(Q, K, V, B, Nq, T_cap, Hq, Hkv, d, indices, counts, s_max, scale,
+                                 O, lse, status, 1, s_max, nullptr, nullptr, st);
 #define LSA_F32_CASE(H, DD)                                                                      \
     if (hpg == H && d == DD)                                                                     \
         return launch_f32<H, DD>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale, O, \

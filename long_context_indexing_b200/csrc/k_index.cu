@@ -97,6 +97,7 @@ cudaError_t launch_pool_unit(const IndexView& ix, const void* latent_K, int64_t 
             ix, (const __nv_bfloat16*)latent_K, j0, j1);
     else
         pool_unit_kernel<float><<<grid, per_cta, 0, st>>>(ix, (const float*)latent_K, j0, j1);
+    note_launch();
     return cudaGetLastError();
 }
 
@@ -283,8 +284,10 @@ cudaError_t launch_kmeans(const IndexView& ix, int64_t b0, int64_t b1, cudaStrea
     for (int it = 0; it < ix.L; ++it) {
         kmeans_assign_kernel<<<dim3((unsigned)(nb * splits), (unsigned)ix.B), ASSIGN_THREADS, 0,
                                st>>>(ix, b0, splits, it == 0);
+        note_launch();
         kmeans_update_kernel<<<dim3((unsigned)nb, (unsigned)ix.B), UPDATE_THREADS, 0, st>>>(
             ix, b0, it == ix.L - 1);
+        note_launch();
     }
     return cudaGetLastError();
 }
@@ -361,6 +364,7 @@ cudaError_t launch_open_assign(const IndexView& ix, int64_t n_blk, int64_t j_end
     if (n_done > ix.G) n_done = ix.G;
     if (n_blk == 0 || n_blk >= ix.nblk_max) n_done = 0;  // nothing to assign / no open block
     open_assign_kernel<<<dim3((unsigned)ix.G, (unsigned)ix.B), 256, 0, st>>>(ix, n_blk, n_done);
+    note_launch();
     return cudaGetLastError();
 }
 

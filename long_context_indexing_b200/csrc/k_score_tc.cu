@@ -32,7 +32,7 @@ namespace lsa {
 constexpr int TC_M = 128;
 constexpr int TC_N = 256;
 constexpr int TC_STAGES = 3;
-constexpr int TC_BUF = 96;
+constexpr int TC_BUF = 80;
 constexpr int TC_THREADS = 192;
 constexpr uint32_t TC_WAIT = 1u << 22;
 
@@ -41,7 +41,8 @@ constexpr int TC_C_BYTES = TC_N * DL * 2;                 // 32 KB per stage
 constexpr int TC_OFF_C = TC_Q_BYTES;
 constexpr int TC_OFF_VAL = TC_OFF_C + TC_STAGES * TC_C_BYTES;
 constexpr int TC_OFF_ID = TC_OFF_VAL + TC_BUF * TC_M * 4;
-constexpr int TC_OFF_BAR = TC_OFF_ID + TC_BUF * TC_M * 4;
+constexpr int TC_OFF_STG = TC_OFF_ID + TC_BUF * TC_M * 4;   // 32 staged scores per row
+constexpr int TC_OFF_BAR = TC_OFF_STG + 32 * TC_M * 4;
 constexpr int TC_NBAR = 1 + 2 * TC_STAGES + 4;
 constexpr int TC_OFF_MISC = TC_OFF_BAR + TC_NBAR * 8;
 constexpr int TC_SMEM = TC_OFF_MISC + 64 + 1024;          // + alignment slack
@@ -128,7 +129,7 @@ struct RowBuf {
         I(b) = ti;
     }
     // Moves the k largest of the first n entries to [0, k) (any order).
-    __device__ void select_top(int n, int k)
+    __device__ __noinline__ void select_top(int n, int k)
     {
         int lo = 0, hi = n - 1;
         while (lo < hi) {
@@ -168,6 +169,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
     unsigned char* c_s = smem + TC_OFF_C;
     float* val_s = reinterpret_cast<float*>(smem + TC_OFF_VAL);
     int* id_s = reinterpret_cast<int*>(smem + TC_OFF_ID);
+    float* stg_s = reinterpret_cast<float*>(smem + TC_OFF_STG);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TC_OFF_BAR);
     uint64_t* q_full = bars;
     uint64_t* full = bars + 1;
@@ -288,10 +290,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
                 __syncwarp();
                 tmem_ld32(tmem + lane_base + (uint32_t)(buf * TC_N + c * 32), v);
                 const int64_t gbase = (int64_t)t * TC_N + c * 32;
+                // Hot path: one compare per score into a bit mask.  Columns at or
+                // beyond the row's eligible count never qualify.
+                uint32_t hit = 0;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    if (v[j] > thr && gbase + j < nb_row) {
-                        rb.V(n_in) = v[j];
+                for (int j = 0; j < 32; ++j) hit |= (v[j] > thr ? 1u : 0u) << j;
+                const int64_t room = nb_row - gbase;
+                if (room < 32) hit &= (room <= 0) ? 0u : ((1u << room) - 1u);
+                if (hit) {
+                    // Rare path: stage the 32 scores, insert the qualifying ones.
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) stg_s[j * TC_M + r] = v[j];
+                    while (hit) {
+                        const int j = __ffs(hit) - 1;
+                        hit &= hit - 1;
+                        const float sj = stg_s[j * TC_M + r];
+                        if (!(sj > thr)) continue;  // threshold may have risen
+                        rb.V(n_in) = sj;
                         rb.I(n_in) = (int)(gbase + j);
                         if (++n_in == TC_BUF) {
                             rb.select_top(n_in, KC);
@@ -381,11 +396,11 @@ cudaError_t launch_score_topk_tc(const IndexView& ix, int64_t n_blk, const void*
     if (!make_rows64_bf16(&tmQ, latent_Q, (uint64_t)ix.B * Nq, TC_M) ||
         !make_rows64_bf16(&tmC, ix.cent_rt, (uint64_t)ix.B * ix.NBK, TC_N))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(score_topk_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM);
+    cudaError_t e = ensure_smem_attr((const void*)score_topk_tc_kernel, TC_SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((Nq + TC_M - 1) / TC_M), (unsigned)ix.B);
     score_topk_tc_kernel<<<grid, TC_THREADS, TC_SMEM, st>>>(tmQ, tmC, ix, n_blk, pos, Nq, W, ws);
+    note_launch();
     return cudaGetLastError();
 }
 

@@ -82,38 +82,30 @@ __device__ __forceinline__ void load_query(float* q_s, const T* lq, int64_t row)
 // that score plus enough of those equal to it.  tau = that score.
 // ---------------------------------------------------------------------------
 constexpr int SIMT_THREADS = 256;
+constexpr int64_t SIMT_SMEM_MAX = 220 * 1024;
 
-template <typename T>
-__global__ void __launch_bounds__(SIMT_THREADS) score_topk_simt_kernel(IndexView ix, int64_t n_blk,
-                                                                       const T* lq, PosSrc pos,
-                                                                       int64_t Nq, int W,
-                                                                       SelectWs ws)
+// Body of the SIMT nominator for query `row` at position pq; q_s holds the
+// latent query (every thread of the CTA calls it; sc holds n_blk*k floats).
+__device__ void simt_nominate(const IndexView& ix, int64_t n_blk, const float* q_s, int64_t bseq,
+                              int64_t row, int64_t pq, int W, const SelectWs& ws, float* sc)
 {
-    extern __shared__ float sc[];
-    __shared__ float q_s[DL];
     __shared__ unsigned hist[256];
     __shared__ uint32_t sh_prefix, sh_want;
     __shared__ int sh_gt, sh_eq;
-    const int64_t b = blockIdx.y, i = blockIdx.x;
-    const int64_t row = b * Nq + i;
-    if (row == 0 && threadIdx.x == 0) *ws.fb_count = 0;
-    const int64_t pq = pos.at(b, Nq, i);
     const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
-    load_query(q_s, lq, row);
-    __syncthreads();
     int32_t* cand = ws.cand + row * KC;
     if (nb <= KC) {
-        for (int x = threadIdx.x; x < KC; x += SIMT_THREADS) cand[x] = (x < nb) ? x : -1;
+        for (int x = threadIdx.x; x < KC; x += blockDim.x) cand[x] = (x < nb) ? x : -1;
         if (threadIdx.x == 0) {
             ws.ncand[row] = (int32_t)nb;
             ws.tau[row] = -INFINITY;
         }
         return;
     }
-    for (int64_t g = threadIdx.x; g < nb; g += SIMT_THREADS) {
+    for (int64_t g = threadIdx.x; g < nb; g += blockDim.x) {
         float s = 0.f;
 #pragma unroll 16
-        for (int d = 0; d < DL; ++d) s = fmaf(q_s[d], rt_load(ix, b, g, d), s);
+        for (int d = 0; d < DL; ++d) s = fmaf(q_s[d], rt_load(ix, bseq, g, d), s);
         sc[g] = s;
     }
     if (threadIdx.x == 0) {
@@ -126,10 +118,10 @@ __global__ void __launch_bounds__(SIMT_THREADS) score_topk_simt_kernel(IndexView
     uint32_t mask = 0;
     for (int pass = 3; pass >= 0; --pass) {
         const int sh = 8 * pass;
-        for (int x = threadIdx.x; x < 256; x += SIMT_THREADS) hist[x] = 0;
+        for (int x = threadIdx.x; x < 256; x += blockDim.x) hist[x] = 0;
         __syncthreads();
         const uint32_t prefix = sh_prefix;
-        for (int64_t g = threadIdx.x; g < nb; g += SIMT_THREADS) {
+        for (int64_t g = threadIdx.x; g < nb; g += blockDim.x) {
             const uint32_t kk = ord_key(sc[g]);
             if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> sh) & 255u], 1u);
         }
@@ -151,7 +143,7 @@ __global__ void __launch_bounds__(SIMT_THREADS) score_topk_simt_kernel(IndexView
     }
     const uint32_t thr = sh_prefix;      // key of the KC-th largest score
     const int need_eq = (int)sh_want;    // how many of the ties at thr to take
-    for (int64_t g = threadIdx.x; g < nb; g += SIMT_THREADS) {
+    for (int64_t g = threadIdx.x; g < nb; g += blockDim.x) {
         const uint32_t kk = ord_key(sc[g]);
         if (kk > thr) {
             const int s = atomicAdd(&sh_gt, 1);
@@ -165,6 +157,28 @@ __global__ void __launch_bounds__(SIMT_THREADS) score_topk_simt_kernel(IndexView
         ws.ncand[row] = KC;
         ws.tau[row] = key_to_float(thr);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Candidate nomination, SIMT: one CTA per query.  Binary32 FMA scores of the
+// eligible buckets into shared memory, then an MSB-first radix select of the
+// KC-th largest score (4 passes of 8 bits).  Candidates: every bucket above
+// that score plus enough of those equal to it.  tau = that score.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(SIMT_THREADS) score_topk_simt_kernel(IndexView ix, int64_t n_blk,
+                                                                       const T* lq, PosSrc pos,
+                                                                       int64_t Nq, int W,
+                                                                       SelectWs ws)
+{
+    extern __shared__ float sc[];
+    __shared__ float q_s[DL];
+    const int64_t b = blockIdx.y, i = blockIdx.x;
+    const int64_t row = b * Nq + i;
+    if (row == 0 && threadIdx.x == 0) *ws.fb_count = 0;
+    load_query(q_s, lq, row);
+    __syncthreads();
+    simt_nominate(ix, n_blk, q_s, b, row, pos.at(b, Nq, i), W, ws, sc);
 }
 
 // ---------------------------------------------------------------------------
@@ -486,6 +500,154 @@ __global__ void __launch_bounds__(FB_THREADS) select_fallback_kernel(IndexView i
 }
 
 // ---------------------------------------------------------------------------
+// Decode step, part 1.  grid (B, 2): role 0 appends sequence b's new token,
+// role 1 nominates candidates for its query.  The two are independent: a
+// pooled group that completes at position pos holds keys >= pos - p + 1,
+// which lie inside the recent window (W >= p - 1), so no selection made at
+// pos can read them.
+// Append: the new latent/key/value rows go to position pos of the caches; if
+// (pos + 1) % p == 0 the group j = (pos + 1)/p - 1 is pooled (binary32, left
+// to right), normalised (binary64 norm) and assigned to the closed bucket of
+// largest exact <u, c_g> (fp32 centroids, lowest g on ties).  A group beyond
+// the open block records DEV_OPEN_FULL and is not appended.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(SIMT_THREADS) decode_prep_kernel(
+    IndexView ix, int64_t n_blk, T* latK, T* Kc, T* Vc, const T* nlk, const T* nk, const T* nv,
+    const T* lq, const int32_t* pos, int Hkv, int d, int W, SelectWs ws, uint32_t* attn_counter,
+    int counters_per_seq)
+{
+    extern __shared__ float sc[];
+    __shared__ float q_s[DL];
+    __shared__ float x_s[DL];
+    __shared__ double nrm_s;
+    __shared__ double rs[SIMT_THREADS / 32];
+    __shared__ int rg[SIMT_THREADS / 32];
+    const int64_t b = blockIdx.x;
+    const int64_t pq = pos[b];
+    if (blockIdx.y == 1) {
+        if (b == 0 && threadIdx.x == 0) *ws.fb_count = 0;
+        load_query(q_s, lq, b);
+        __syncthreads();
+        simt_nominate(ix, n_blk, q_s, b, b, pq, W, ws, sc);
+        return;
+    }
+    for (int x = threadIdx.x; x < counters_per_seq; x += blockDim.x)
+        attn_counter[b * counters_per_seq + x] = 0u;
+    if (pq < 0 || pq >= ix.T_cap) {
+        if (threadIdx.x == 0) dev_error(ix.status, DEV_BAD_INDEX, (uint32_t)b);
+        return;
+    }
+    T* lrow = latK + (b * ix.T_cap + pq) * DL;
+    for (int x = threadIdx.x; x < DL; x += blockDim.x) lrow[x] = nlk[b * DL + x];
+    const int64_t kvn = (int64_t)Hkv * d;
+    T* krow = Kc + (b * ix.T_cap + pq) * kvn;
+    T* vrow = Vc + (b * ix.T_cap + pq) * kvn;
+    for (int64_t x = threadIdx.x; x < kvn; x += blockDim.x) {
+        krow[x] = nk[b * kvn + x];
+        vrow[x] = nv[b * kvn + x];
+    }
+    const int p = ix.p;
+    if ((pq + 1) % p != 0) return;
+    const int64_t j = (pq + 1) / p - 1;
+    const int64_t o = j - n_blk * ix.G;
+    if (n_blk < 1 || o < 0 || o >= ix.G || n_blk >= ix.nblk_max) {
+        if (threadIdx.x == 0) dev_error(ix.status, DEV_OPEN_FULL, (uint32_t)b);
+        return;
+    }
+    __syncthreads();   // the new latent row is visible to the whole CTA
+    if (threadIdx.x < DL) {
+        const int i = threadIdx.x;
+        const T* rows = latK + (b * ix.T_cap + j * p) * DL;
+        float s = load_elt(rows + i);
+        for (int r = 1; r < p; ++r) s = __fadd_rn(s, load_elt(rows + (int64_t)r * DL + i));
+        const float xv = __fdiv_rn(s, (float)p);
+        x_s[i] = xv;
+        ix.pooled[(b * ix.NP + j) * DL + i] = xv;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double ss = 0.0;
+        for (int i = 0; i < DL; ++i) ss = __fma_rn((double)x_s[i], (double)x_s[i], ss);
+        nrm_s = __dsqrt_rn(ss);
+    }
+    __syncthreads();
+    if (threadIdx.x < DL) {
+        const int i = threadIdx.x;
+        const float u = (nrm_s != 0.0) ? __double2float_rn(__ddiv_rn((double)x_s[i], nrm_s)) : 0.f;
+        ix.unit[(b * ix.NP + j) * DL + i] = u;
+        q_s[i] = u;   // reuse as the unit vector
+    }
+    __syncthreads();
+    const float* cent = ix.cent + b * ix.NBK * DL;
+    const int64_t nbk = n_blk * ix.k;
+    double bs = -INFINITY;
+    int bg = 0x7fffffff;
+    for (int64_t g = threadIdx.x; g < nbk; g += blockDim.x) {
+        const float* c = cent + g * DL;
+        double s = 0.0;
+#pragma unroll 16
+        for (int i = 0; i < DL; ++i) s = __fma_rn((double)q_s[i], (double)c[i], s);
+        if (s > bs || (s == bs && (int)g < bg)) {
+            bs = s;
+            bg = (int)g;
+        }
+    }
+    for (int off = 16; off > 0; off >>= 1) {
+        const double os = __shfl_xor_sync(0xffffffffu, bs, off);
+        const int og = __shfl_xor_sync(0xffffffffu, bg, off);
+        if (os > bs || (os == bs && og < bg)) {
+            bs = os;
+            bg = og;
+        }
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        rs[warp] = bs;
+        rg[warp] = bg;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < SIMT_THREADS / 32; ++w)
+            if (rs[w] > bs || (rs[w] == bs && rg[w] < bg)) {
+                bs = rs[w];
+                bg = rg[w];
+            }
+        ix.open_bucket[b * ix.G + o] = bg;
+    }
+}
+
+cudaError_t launch_decode_prep(const IndexView& ix, int64_t n_blk, void* latent_K, void* K,
+                               void* V, const void* new_latent_k, const void* new_k,
+                               const void* new_v, const void* latent_q, const int32_t* pos,
+                               int Hkv, int d, int W, const SelectWs& ws, uint32_t* attn_counter,
+                               int counters_per_seq, cudaStream_t st)
+{
+    const size_t smem = (size_t)n_blk * ix.k * sizeof(float);
+    dim3 grid((unsigned)ix.B, 2);
+    cudaError_t e;
+    if (ix.dtype == LSA_BF16) {
+        typedef __nv_bfloat16 T;
+        e = ensure_smem_attr((const void*)decode_prep_kernel<T>, (int)SIMT_SMEM_MAX);
+        if (e != cudaSuccess) return e;
+        decode_prep_kernel<T><<<grid, SIMT_THREADS, smem, st>>>(
+            ix, n_blk, (T*)latent_K, (T*)K, (T*)V, (const T*)new_latent_k, (const T*)new_k,
+            (const T*)new_v, (const T*)latent_q, pos, Hkv, d, W, ws, attn_counter,
+            counters_per_seq);
+    } else {
+        typedef float T;
+        e = ensure_smem_attr((const void*)decode_prep_kernel<T>, (int)SIMT_SMEM_MAX);
+        if (e != cudaSuccess) return e;
+        decode_prep_kernel<T><<<grid, SIMT_THREADS, smem, st>>>(
+            ix, n_blk, (T*)latent_K, (T*)K, (T*)V, (const T*)new_latent_k, (const T*)new_k,
+            (const T*)new_v, (const T*)latent_q, pos, Hkv, d, W, ws, attn_counter,
+            counters_per_seq);
+    }
+    note_launch();
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Workspace and launch.
 // ---------------------------------------------------------------------------
 static inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -521,6 +683,25 @@ cudaError_t launch_score_topk_tc(const IndexView& ix, int64_t n_blk, const void*
                                  cudaStream_t st);
 
 template <typename T>
+static cudaError_t launch_finish_t(const IndexView& ix, int64_t n_blk, const T* lq, PosSrc pos,
+                                   int64_t Nq, lsa_select_params sp, int32_t* indices,
+                                   int32_t* counts, int s_max, const SelectWs& ws, cudaStream_t st)
+{
+    dim3 grid((unsigned)Nq, (unsigned)ix.B);
+    select_fill_kernel<T><<<grid, FILL_THREADS, 0, st>>>(ix, n_blk, lq, pos, Nq, sp.budget,
+                                                         sp.window, sp.sinks, s_max, indices,
+                                                         counts, ws);
+    note_launch();
+    const int64_t rows = ix.B * Nq;
+    const unsigned fb_grid = (unsigned)(rows < FB_CTAS ? rows : FB_CTAS);
+    select_fallback_kernel<T><<<fb_grid, FB_THREADS, 0, st>>>(ix, n_blk, lq, pos, Nq, sp.budget,
+                                                              sp.window, sp.sinks, s_max,
+                                                              indices, counts, ws);
+    note_launch();
+    return cudaGetLastError();
+}
+
+template <typename T>
 static cudaError_t launch_select_t(const IndexView& ix, int64_t n_blk, const T* lq, PosSrc pos,
                                    int64_t Nq, lsa_select_params sp, int32_t* indices,
                                    int32_t* counts, int s_max, const SelectWs& ws, bool use_tc,
@@ -533,21 +714,13 @@ static cudaError_t launch_select_t(const IndexView& ix, int64_t n_blk, const T* 
         if (e != cudaSuccess) return e;
     } else {
         const size_t smem = (size_t)n_blk * ix.k * sizeof(float);
-        e = cudaFuncSetAttribute(score_topk_simt_kernel<T>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = ensure_smem_attr((const void*)score_topk_simt_kernel<T>, (int)SIMT_SMEM_MAX);
         if (e != cudaSuccess) return e;
         score_topk_simt_kernel<T><<<grid, SIMT_THREADS, smem, st>>>(ix, n_blk, lq, pos, Nq,
                                                                     sp.window, ws);
+        note_launch();
     }
-    select_fill_kernel<T><<<grid, FILL_THREADS, 0, st>>>(ix, n_blk, lq, pos, Nq, sp.budget,
-                                                         sp.window, sp.sinks, s_max, indices,
-                                                         counts, ws);
-    int64_t rows = ix.B * Nq;
-    const unsigned fb_grid = (unsigned)(rows < FB_CTAS ? rows : FB_CTAS);
-    select_fallback_kernel<T><<<fb_grid, FB_THREADS, 0, st>>>(ix, n_blk, lq, pos, Nq, sp.budget,
-                                                              sp.window, sp.sinks, s_max,
-                                                              indices, counts, ws);
-    return cudaGetLastError();
+    return launch_finish_t(ix, n_blk, lq, pos, Nq, sp, indices, counts, s_max, ws, st);
 }
 
 cudaError_t launch_select(const IndexView& ix, int64_t n_blk, const void* latent_Q, PosSrc pos,
@@ -560,6 +733,17 @@ cudaError_t launch_select(const IndexView& ix, int64_t n_blk, const void* latent
                                counts, s_max, ws, use_tc, st);
     return launch_select_t(ix, n_blk, (const float*)latent_Q, pos, Nq, sp, indices, counts, s_max,
                            ws, false, st);
+}
+
+cudaError_t launch_select_finish(const IndexView& ix, int64_t n_blk, const void* latent_Q,
+                                 PosSrc pos, int64_t Nq, lsa_select_params sp, int32_t* indices,
+                                 int32_t* counts, int s_max, const SelectWs& ws, cudaStream_t st)
+{
+    if (ix.dtype == LSA_BF16)
+        return launch_finish_t(ix, n_blk, (const __nv_bfloat16*)latent_Q, pos, Nq, sp, indices,
+                               counts, s_max, ws, st);
+    return launch_finish_t(ix, n_blk, (const float*)latent_Q, pos, Nq, sp, indices, counts, s_max,
+                           ws, st);
 }
 
 }  // namespace lsa

@@ -8,6 +8,7 @@
 
 #include <math.h>
 
+#include <atomic>
 #include <new>
 
 #include "lsa_internal.cuh"
@@ -15,6 +16,8 @@
 using namespace lsa;
 
 namespace {
+
+std::atomic<uint64_t> g_launches{0};
 
 thread_local char g_err[512] = "";
 
@@ -116,9 +119,68 @@ lsa_status run_select(const lsa_index* idx, const void* lq, PosSrc pos, int64_t 
     return LSA_OK;
 }
 
+struct DecodeLayout {
+    size_t indices, counts, sel, part, counter, total;
+    int ns, kps, n_hg;
+};
+
+int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+        return n;
+    cudaGetLastError();  // clear the error of a host without a device
+    return 148;
+}
+
+DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_select_params sp)
+{
+    const IndexView& v = idx->v;
+    const int64_t s_max = (int64_t)sp.budget + sp.window + sp.sinks;
+    DecodeLayout L;
+    const int hg = attn_head_group(Hkv);
+    L.n_hg = Hkv / hg;
+    const int kt = attn_stage_keys(Hkv);
+    const int64_t units = v.B * L.n_hg;
+    // about two CTAs per SM over all (sequence, head group, split) triples
+    int64_t ns = (2 * (int64_t)sm_count() + units - 1) / units;
+    if (ns < 1) ns = 1;
+    int64_t kps = (s_max + ns - 1) / ns;
+    kps = ((kps + kt - 1) / kt) * kt;
+    ns = (s_max + kps - 1) / kps;
+    L.ns = (int)ns;
+    L.kps = (int)kps;
+    size_t o = 0;
+    L.indices = o; o += al256((size_t)v.B * s_max * 4);
+    L.counts = o;  o += al256((size_t)v.B * 4);
+    L.sel = o;     o += select_ws_bytes(v, 1);
+    L.part = o;    o += al256((size_t)v.B * ns * Hq * (d + 2) * 4);
+    L.counter = o; o += al256((size_t)v.B * L.n_hg * 4);
+    L.total = o;
+    return L;
+}
+
+lsa_status check_attn_shape(int Hq, int Hkv, int d, lsa_dtype dt)
+{
+    if (Hkv < 1 || Hq < 1 || Hq % Hkv != 0) return fail(LSA_ERR_INVALID_ARG, "Hq %% Hkv != 0");
+    const int hpg = Hq / Hkv;
+    if (hpg != 1 && hpg != 2 && hpg != 4 && hpg != 8)
+        return fail(LSA_ERR_UNSUPPORTED, "Hq/Hkv=%d not in {1,2,4,8}", hpg);
+    if (d != 64 && d != 128) return fail(LSA_ERR_UNSUPPORTED, "d=%d not in {64,128}", d);
+    if (dt == LSA_BF16 && !(Hkv == 1 || Hkv == 2 || Hkv % 4 == 0))
+        return fail(LSA_ERR_UNSUPPORTED, "Hkv=%d: bf16 kernels need Hkv in {1, 2} or a multiple of 4",
+                    Hkv);
+    return LSA_OK;
+}
+
 }  // namespace
 
+void lsa::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 extern "C" {
+
+uint64_t lsa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* lsa_last_error(void) { return g_err; }
 
@@ -312,11 +374,8 @@ lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtyp
     if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
     if (B < 1 || Nq < 0 || T_cap < 1 || T_cap > 2147483647LL || s_max < 1)
         return fail(LSA_ERR_INVALID_ARG, "bad sizes");
-    if (Hkv < 1 || Hq < 1 || Hq % Hkv != 0) return fail(LSA_ERR_INVALID_ARG, "Hq %% Hkv != 0");
-    const int hpg = Hq / Hkv;
-    if (hpg != 1 && hpg != 2 && hpg != 4 && hpg != 8)
-        return fail(LSA_ERR_UNSUPPORTED, "Hq/Hkv=%d not in {1,2,4,8}", hpg);
-    if (d != 64 && d != 128) return fail(LSA_ERR_UNSUPPORTED, "d=%d not in {64,128}", d);
+    lsa_status sh = check_attn_shape(Hq, Hkv, d, dtype);
+    if (sh != LSA_OK) return sh;
     if (B * Nq * Hkv > 2147483647LL) return fail(LSA_ERR_UNSUPPORTED, "too many (query, head) pairs");
     if (!(scale > 0.f)) return fail(LSA_ERR_INVALID_ARG, "scale must be > 0");
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(indices) ||
@@ -354,10 +413,8 @@ lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* l
     if (!aligned16(workspace) || !aligned16(latent_Q) || !aligned16(Q) || !aligned16(O))
         return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
     // attention shape checks up front so that nothing launches on bad input
-    const int hpg = (Hkv > 0) ? Hq / Hkv : 0;
-    if (Hkv < 1 || Hq % Hkv != 0 || (hpg != 1 && hpg != 2 && hpg != 4 && hpg != 8))
-        return fail(LSA_ERR_UNSUPPORTED, "Hq/Hkv must be 1, 2, 4 or 8");
-    if (d != 64 && d != 128) return fail(LSA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    s = check_attn_shape(Hq, Hkv, d, idx->v.dtype);
+    if (s != LSA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
     s = lsa_index_extend(idx, latent_K, T_old, T_new, stream);
     if (s != LSA_OK) return s;
@@ -375,6 +432,67 @@ lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* l
                                        d, indices, counts, s_max, scale, O, nullptr,
                                        idx->v.status, st);
     if (e != cudaSuccess) return cuda_fail(e, "sparse attention");
+    return LSA_OK;
+}
+
+size_t lsa_decode_workspace_bytes(const lsa_index* idx, int Hq, int Hkv, int d,
+                                  lsa_select_params sp)
+{
+    if (!idx || sp.budget < 0 || sp.window < 0 || sp.sinks < 0) return 0;
+    if (check_attn_shape(Hq, Hkv, d, idx->v.dtype) != LSA_OK) return 0;
+    return decode_layout(idx, Hq, Hkv, d, sp).total;
+}
+
+lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
+                           const void* new_latent_k, const void* new_k, const void* new_v,
+                           const void* latent_q, const void* q, const int32_t* pos, int Hq,
+                           int Hkv, int d, lsa_select_params sp, void* workspace, size_t ws_bytes,
+                           void* O, void* stream)
+{
+    if (!idx || !latent_K || !K || !V || !new_latent_k || !new_k || !new_v || !latent_q || !q ||
+        !pos || !workspace || !O)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    const IndexView& v = idx->v;
+    const int s_max = sp.budget + sp.window + sp.sinks;
+    lsa_status s = check_select(idx, sp, s_max);
+    if (s != LSA_OK) return s;
+    s = check_attn_shape(Hq, Hkv, d, v.dtype);
+    if (s != LSA_OK) return s;
+    if (idx->n_blk < 1 || idx->n_blk >= v.nblk_max)
+        return fail(LSA_ERR_INVALID_ARG,
+                    "decode needs at least one closed block and room for an open block");
+    const void* ptrs[] = {latent_K, K, V, new_latent_k, new_k, new_v, latent_q, q, pos, workspace, O};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    const DecodeLayout L = decode_layout(idx, Hq, Hkv, d, sp);
+    if (ws_bytes < L.total)
+        return fail(LSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+    cudaStream_t st = (cudaStream_t)stream;
+    char* base = (char*)workspace;
+    int32_t* indices = (int32_t*)(base + L.indices);
+    int32_t* counts = (int32_t*)(base + L.counts);
+    SelectWs w = select_ws_carve(base + L.sel, v, 1);
+    float* part = (float*)(base + L.part);
+    uint32_t* counter = (uint32_t*)(base + L.counter);
+    if (!idx->status_clean) {
+        cudaError_t e = cudaMemsetAsync(v.status, 0, 8 * sizeof(uint32_t), st);
+        if (e != cudaSuccess) return cuda_fail(e, "status clear");
+        idx->status_clean = true;
+    }
+    cudaError_t e = launch_decode_prep(v, idx->n_blk, latent_K, K, V, new_latent_k, new_k, new_v,
+                                       latent_q, pos, Hkv, d, sp.window, w, counter, L.n_hg, st);
+    if (e != cudaSuccess) return cuda_fail(e, "decode append/nominate");
+    PosSrc ps{pos, 0};
+    e = launch_select_finish(v, idx->n_blk, latent_q, ps, 1, sp, indices, counts, s_max, w, st);
+    if (e != cudaSuccess) return cuda_fail(e, "decode select");
+    const float scale = (float)(1.0 / sqrt((double)d));
+    if (v.dtype == LSA_BF16)
+        e = launch_attn_split(q, K, V, v.B, 1, v.T_cap, Hq, Hkv, d, indices, counts, s_max, scale,
+                              O, nullptr, v.status, L.ns, L.kps, part, counter, st);
+    else
+        e = launch_attn_status(q, K, V, v.dtype, v.B, 1, v.T_cap, Hq, Hkv, d, indices, counts,
+                               s_max, scale, O, nullptr, v.status, st);
+    if (e != cudaSuccess) return cuda_fail(e, "decode attention");
     return LSA_OK;
 }
 

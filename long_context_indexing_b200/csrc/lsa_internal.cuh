@@ -71,6 +71,9 @@ __device__ __forceinline__ void dev_error(uint32_t* status, uint32_t code, uint3
     if (atomicCAS(status, 0u, code) == 0u) status[2] = detail;
 }
 
+// Host-side count of kernel launches enqueued by the library (all threads).
+void note_launch();
+
 __device__ __forceinline__ float load_elt(const float* p) { return *p; }
 __device__ __forceinline__ float load_elt(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
@@ -108,12 +111,39 @@ cudaError_t launch_select(const IndexView& ix, int64_t n_blk, const void* latent
                           int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
                           int s_max, const SelectWs& ws, bool use_tc, cudaStream_t st);
 
+// Exact fill + emission + fallback only (candidates already nominated).
+cudaError_t launch_select_finish(const IndexView& ix, int64_t n_blk, const void* latent_Q,
+                                 PosSrc pos, int64_t Nq, lsa_select_params sp, int32_t* indices,
+                                 int32_t* counts, int s_max, const SelectWs& ws, cudaStream_t st);
+
 // Sparse attention (status nullable: receives DEV_BAD_INDEX / DEV_TIMEOUT).
 cudaError_t launch_attn_status(const void* Q, const void* K, const void* V, lsa_dtype dt,
                                int64_t B, int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
                                const int32_t* indices, const int32_t* counts, int s_max,
                                float scale, void* O, float* lse, uint32_t* status,
                                cudaStream_t st);
+// Raises a kernel's dynamic shared-memory limit once per device (so that calls
+// made later, for example under stream capture, do not repeat it).
+cudaError_t ensure_smem_attr(const void* kernel, int bytes);
+
+// Split-KV bf16 attention: ns splits of keys_per_split keys per (row, head
+// group); part [rows][ns][Hq][d+2] and counter [rows * head groups] (zero
+// before the launch, left zero after it) are caller scratch.
+cudaError_t launch_attn_split(const void* Q, const void* K, const void* V, int64_t B, int64_t Nq,
+                              int64_t T_cap, int Hq, int Hkv, int d, const int32_t* indices,
+                              const int32_t* counts, int s_max, float scale, void* O, float* lse,
+                              uint32_t* status, int ns, int keys_per_split, float* part,
+                              uint32_t* counter, cudaStream_t st);
+int attn_stage_keys(int Hkv);
+int attn_head_group(int Hkv);
+
+// Decode: append + candidate nomination for one query per sequence.
+cudaError_t launch_decode_prep(const IndexView& ix, int64_t n_blk, void* latent_K, void* K,
+                               void* V, const void* new_latent_k, const void* new_k,
+                               const void* new_v, const void* latent_q, const int32_t* pos,
+                               int Hkv, int d, int W, const SelectWs& ws, uint32_t* attn_counter,
+                               int n_counter, cudaStream_t st);
+
 // True when the tensor-core candidate scorer is compiled in.
 bool tc_scoring_available();
 

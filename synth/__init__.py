@@ -175,27 +175,29 @@ def prefill_inputs(w: Workload, seed=0, device="cpu"):
                 Q=q.to(dt).contiguous(), positions=pos.contiguous())
 
 
-def decode_inputs(w: Workload, seed=0, device="cpu"):
+def decode_inputs(w: Workload, seed=0, device="cpu", t_cap=None):
     """Inputs of a decode workload: caches sized T + steps per sequence, holding
     the prefix keys (0 .. T-1) AND the keys each step will append (T .. T+steps-1,
     also returned separately as the per-step new rows), plus one query per
     sequence per step.
 
-    Returns a dict with latent_K [B][T+steps][64], K, V [B][T+steps][Hkv][d],
+    Returns a dict with latent_K [B][t_cap][64], K, V [B][t_cap][Hkv][d] (rows
+    from T + steps on are zero; t_cap defaults to T + steps),
     new_latent_k [steps][B][64], new_k / new_v [steps][B][Hkv][d],
     latent_q [steps][B][64], q [steps][B][Hq][d]."""
     dt = w.torch_dtype
-    t_cap = w.T + w.steps
-    mix = Mixture(w, seed, device, t_total=t_cap)
+    t_all = w.T + w.steps
+    t_cap = max(t_cap or t_all, t_all)
+    mix = Mixture(w, seed, device, t_total=t_all)
     dev = mix.device
-    latent_K = torch.empty(w.B, t_cap, LATENT_DIM, dtype=dt, device=dev)
-    K = torch.empty(w.B, t_cap, w.Hkv, w.d, dtype=dt, device=dev)
-    V = torch.empty(w.B, t_cap, w.Hkv, w.d, dtype=dt, device=dev)
+    latent_K = torch.zeros(w.B, t_cap, LATENT_DIM, dtype=dt, device=dev)
+    K = torch.zeros(w.B, t_cap, w.Hkv, w.d, dtype=dt, device=dev)
+    V = torch.zeros(w.B, t_cap, w.Hkv, w.d, dtype=dt, device=dev)
     mix.keys(latent_K, K, V)
     lq, q = mix.queries(w.steps)          # [B][steps][...]
-    new_lat = latent_K[:, w.T:].transpose(0, 1).contiguous()
-    new_k = K[:, w.T:].transpose(0, 1).contiguous()
-    new_v = V[:, w.T:].transpose(0, 1).contiguous()
+    new_lat = latent_K[:, w.T:t_all].transpose(0, 1).contiguous()
+    new_k = K[:, w.T:t_all].transpose(0, 1).contiguous()
+    new_v = V[:, w.T:t_all].transpose(0, 1).contiguous()
     return dict(latent_K=latent_K, K=K, V=V, new_latent_k=new_lat, new_k=new_k, new_v=new_v,
                 latent_q=lq.to(dt).transpose(0, 1).contiguous(),
                 q=q.to(dt).transpose(0, 1).contiguous())

@@ -278,3 +278,28 @@ def test_attention_shapes_and_ragged_counts(dtype, hpg, d):
                                        oracle.default_scale(d))
         _attn_check(O[b], O_ref, dtype)
         assert np.abs(_np(lse[b]) - lse_ref).max() < (1e-4 if dtype == "f32" else 2e-2)
+
+
+def test_tensor_core_nomination_ragged_tiles_and_mixed_positions():
+    # bf16 with Nq >= 128 takes the tcgen05 nominator: a ragged query count
+    # (two full 128-row tiles + 44), two sequences, positions scattered from 0
+    # to T-1 so rows of one tile see anywhere from 0 to 512 eligible buckets.
+    w = synth.workload("tiny", T=16384, nq=300, B=2, G=32, k=4, R=700, W=64, S=4, M=64,
+                       dtype="bf16", Hq=8, Hkv=1, d=64)
+    inp = synth.prefill_inputs(w, 7, "cpu")
+    rng = np.random.default_rng(7)
+    pos = rng.integers(0, w.T, size=(w.B, w.nq))
+    pos[:, :5] = [0, 1, w.W, w.W + 200, w.T - 1]
+    gpu = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16)
+    gpu.build(inp["latent_K"].cuda(), w.T)
+    g_idx, g_cnt = lsa.lsa_select(gpu, inp["latent_Q"].cuda(),
+                                  torch.from_numpy(pos.astype(np.int32)).cuda(), w.R, w.W, w.S)
+    torch.cuda.synchronize()
+    gpu.check()
+    for b in range(w.B):
+        orc = oracle.Index(w.T, w.p, w.G, w.k, w.L, rt_bf16=True)
+        orc.extend(inp["latent_K"][b].float().numpy(), 0, w.T)
+        _compare_index(gpu, orc, b)
+        o_idx, o_cnt, o_mg, _ = oracle.select(orc, inp["latent_Q"][b].float().numpy(), pos[b],
+                                              w.R, w.W, w.S)
+        assert _compare_selection(g_idx[b], g_cnt[b], o_idx, o_cnt, o_mg) == w.nq
