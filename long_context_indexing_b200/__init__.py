@@ -69,7 +69,6 @@ def _declare(lib):
         "lsa_prefill_chunk": ([P, P, P, P, P, P, I64, I64, I, I, I, SelectParams, P, SZ, P, P],
                               I),
         "lsa_decode_workspace_bytes": ([P, I, I, I, SelectParams], SZ),
-        "lsa_decode_step": ([P, P, P, P, P, P, P, P, P, P, I, I, I, SelectParams, P, SZ, P, P], I),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)

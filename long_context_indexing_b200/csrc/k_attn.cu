@@ -436,23 +436,45 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
     __syncthreads();
     if (!sh_last) return;
     __threadfence();
+    // Combine: per query head the global max M over splits and each split's
+    // weight exp2(m_s - M) / L (L = sum of the rescaled partial sums), then
+    // every output element is one weighted sum over splits.  Partials of other
+    // CTAs are read through L2 (__ldcg), never through a stale L1 line.
+    float* m_sp = reinterpret_cast<float*>(smem);           // [nq_heads][ns]
+    float* w_sp = m_sp + nq_heads * sk.ns;                   // [nq_heads][ns]
+    float* M_s = w_sp + nq_heads * sk.ns;                    // [nq_heads]
+    const int64_t sstride = (int64_t)Hq * (D + 2);
+    const float* pbase = sk.part + (row * sk.ns * Hq + (int64_t)g0 * hpg) * (D + 2);
+    for (int x = threadIdx.x; x < nq_heads * sk.ns; x += ATT_THREADS) {
+        const int qh = x / sk.ns, sp = x % sk.ns;
+        const float* pp = pbase + sp * sstride + (int64_t)qh * (D + 2);
+        m_sp[x] = __ldcg(pp);
+        w_sp[x] = __ldcg(pp + 1);   // partial sum for now
+    }
+    __syncthreads();
+    for (int qh = threadIdx.x; qh < nq_heads; qh += ATT_THREADS) {
+        float M = -INFINITY;
+        for (int sp = 0; sp < sk.ns; ++sp) M = fmaxf(M, m_sp[qh * sk.ns + sp]);
+        float L = 0.f;
+        for (int sp = 0; sp < sk.ns; ++sp) {
+            const float ms = m_sp[qh * sk.ns + sp];
+            const float e = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+            m_sp[qh * sk.ns + sp] = e;                       // reuse as the rescale
+            L += w_sp[qh * sk.ns + sp] * e;
+        }
+        for (int sp = 0; sp < sk.ns; ++sp) w_sp[qh * sk.ns + sp] = m_sp[qh * sk.ns + sp] / L;
+        M_s[qh] = M;
+        if (lse) lse[row * Hq + (int64_t)g0 * hpg + qh] = (M + log2f(L)) * 0.69314718055994531f;
+    }
+    __syncthreads();
     for (int x = threadIdx.x; x < nq_heads * D; x += ATT_THREADS) {
         const int qh = x / D, c = x % D;
-        const int64_t qhg = (int64_t)g0 * hpg + qh;
-        const volatile float* pp = sk.part + (row * sk.ns * Hq + qhg) * (D + 2);
-        const int64_t sstride = (int64_t)Hq * (D + 2);
-        float M = -INFINITY;
-        for (int sp = 0; sp < sk.ns; ++sp) M = fmaxf(M, pp[sp * sstride]);
-        float L = 0.f, acc = 0.f;
-        for (int sp = 0; sp < sk.ns; ++sp) {
-            const float ms = pp[sp * sstride];
-            const float sc = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-            L += pp[sp * sstride + 1] * sc;
-            acc += pp[sp * sstride + 2 + c] * sc;
-        }
-        const int64_t oh = row * Hq + qhg;
-        O[oh * D + c] = __float2bfloat16_rn(acc / L);
-        if (c == 0 && lse) lse[oh] = (M + log2f(L)) * 0.69314718055994531f;
+        const float* pp = pbase + (int64_t)qh * (D + 2) + 2 + c;
+        const float* wq = w_sp + qh * sk.ns;
+        float acc = 0.f;
+#pragma unroll 4
+        for (int sp = 0; sp < sk.ns; ++sp) acc += __ldcg(pp + sp * sstride) * wq[sp];
+        O[(row * Hq + (int64_t)g0 * hpg + qh) * D + c] = __float2bfloat16_rn(acc);
     }
     if (threadIdx.x == 0) sk.counter[unit] = 0;   // ready for the next launch
 }
@@ -468,6 +490,10 @@ static cudaError_t launch_bf16(const void* Q, const void* K, const void* V, int6
     cudaError_t e = ensure_smem_attr((const void*)kern, C::BYTES);
     if (e != cudaSuccess) return e;
     if (sk.ns > 1 && sk.keys_per_split % C::KT != 0) return cudaErrorInvalidValue;
+    // the split combine keeps 2 * (query heads of the CTA) * ns + heads floats
+    // in the freed ring
+    if (sk.ns > 1 && (size_t)(2 * HG * (Hq / Hkv) * sk.ns + HG * (Hq / Hkv)) * 4 > (size_t)C::BODY)
+        return cudaErrorInvalidValue;
     const int64_t ctas = B * Nq * (Hkv / HG) * sk.ns;
     kern<<<(unsigned)ctas, ATT_THREADS, C::BYTES, st>>>(
         (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, Nq, T_cap, Hq,

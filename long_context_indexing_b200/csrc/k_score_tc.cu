@@ -17,9 +17,10 @@
 //              a TC_STAGES-deep shared-memory ring (128-byte swizzle);
 //   warp 1     owns 512 TMEM columns (two 256-column fp32 accumulators) and
 //              issues tcgen05.mma (M=128, N=256, K=16, four per tile);
-//   warps 2-5  epilogue: tcgen05.ld 32 columns at a time, and per row a
-//              threshold-filtered buffer of TC_BUF entries, compacted to the
-//              top KC by quickselect when full.
+//   warps 2-5  epilogue: tcgen05.ld 32 columns at a time; per row, scores
+//              above the row's running threshold (the KC-th best kept so far)
+//              are appended to a 2*KC-slot buffer, which the warp compacts
+//              back to the top KC in lockstep when a row runs short of room.
 // Every mbarrier wait is bounded; on a timeout the CTA records DEV_TIMEOUT in
 // the index status word, stops waiting, and still frees its TMEM.
 #include <cuda.h>
@@ -31,8 +32,8 @@ namespace lsa {
 
 constexpr int TC_M = 128;
 constexpr int TC_N = 256;
-constexpr int TC_STAGES = 3;
-constexpr int TC_BUF = 80;
+constexpr int TC_STAGES = 2;
+constexpr int TC_BUF = 2 * KC;                 // kept top-KC + KC new slots
 constexpr int TC_THREADS = 192;
 constexpr uint32_t TC_WAIT = 1u << 22;
 
@@ -41,8 +42,7 @@ constexpr int TC_C_BYTES = TC_N * DL * 2;                 // 32 KB per stage
 constexpr int TC_OFF_C = TC_Q_BYTES;
 constexpr int TC_OFF_VAL = TC_OFF_C + TC_STAGES * TC_C_BYTES;
 constexpr int TC_OFF_ID = TC_OFF_VAL + TC_BUF * TC_M * 4;
-constexpr int TC_OFF_STG = TC_OFF_ID + TC_BUF * TC_M * 4;   // 32 staged scores per row
-constexpr int TC_OFF_BAR = TC_OFF_STG + 32 * TC_M * 4;
+constexpr int TC_OFF_BAR = TC_OFF_ID + TC_BUF * TC_M * 4;
 constexpr int TC_NBAR = 1 + 2 * TC_STAGES + 4;
 constexpr int TC_OFF_MISC = TC_OFF_BAR + TC_NBAR * 8;
 constexpr int TC_SMEM = TC_OFF_MISC + 64 + 1024;          // + alignment slack
@@ -114,36 +114,77 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v)
 }
 
 // ---- per-row candidate buffer (strided by TC_M in shared memory) -----------
+// Slots [0, KC) hold the kept candidates (sorted by score, descending, after
+// the first compaction); new entries go to [KC, 2KC).  A compaction keeps the
+// top KC of all 2KC slots with a data-oblivious network (every lane of a warp
+// runs the same compare-exchange sequence on its own row, so the warp never
+// diverges): bitonic sort of the new half, element-wise max of the kept half
+// against the reversed new half (a bitonic sequence holding the top KC), and
+// a bitonic merge of that sequence.
 struct RowBuf {
     float* v;
     int* id;
-    __device__ float& V(int x) { return v[x * TC_M]; }
-    __device__ int& I(int x) { return id[x * TC_M]; }
-    __device__ void swap(int a, int b)
+    __device__ __forceinline__ float& V(int x) { return v[x * TC_M]; }
+    __device__ __forceinline__ int& I(int x) { return id[x * TC_M]; }
+    // compare-exchange so that slot a ends up with the larger score
+    __device__ __forceinline__ void cx_desc(int a, int b)
     {
-        const float tv = V(a);
-        V(a) = V(b);
-        V(b) = tv;
-        const int ti = I(a);
-        I(a) = I(b);
-        I(b) = ti;
+        const float va = V(a), vb = V(b);
+        const int ia = I(a), ib = I(b);
+        const bool sw = va < vb;
+        V(a) = sw ? vb : va;
+        V(b) = sw ? va : vb;
+        I(a) = sw ? ib : ia;
+        I(b) = sw ? ia : ib;
     }
-    // Moves the k largest of the first n entries to [0, k) (any order).
-    __device__ __noinline__ void select_top(int n, int k)
+    // bitonic sort (descending) of the KC slots starting at `base`
+    __device__ void sort_desc(int base)
     {
-        int lo = 0, hi = n - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            swap(mid, hi);
-            const float pv = V(hi);
-            int st = lo;
-            for (int x = lo; x < hi; ++x)
-                if (V(x) > pv) swap(x, st++);
-            swap(st, hi);
-            if (st == k - 1 || st == k) return;
-            if (st < k - 1) lo = st + 1;
-            else hi = st - 1;
+        for (int k = 2; k <= KC; k <<= 1)
+            for (int j = k >> 1; j > 0; j >>= 1)
+                for (int t = 0; t < KC / 2; ++t) {
+                    const int i = ((t & ~(j - 1)) << 1) | (t & (j - 1));
+                    const int l = i | j;
+                    if ((i & k) == 0) cx_desc(base + i, base + l);
+                    else cx_desc(base + l, base + i);
+                }
+    }
+    // bitonic merge (descending) of a bitonic sequence in [0, KC)
+    __device__ void merge_desc()
+    {
+        for (int j = KC >> 1; j > 0; j >>= 1)
+            for (int t = 0; t < KC / 2; ++t) {
+                const int i = ((t & ~(j - 1)) << 1) | (t & (j - 1));
+                cx_desc(i, i | j);
+            }
+    }
+    // top KC of all 2KC slots into [0, KC), sorted descending; slots from n
+    // on are empty and padded first
+    __device__ void compact(int n, bool kept_sorted)
+    {
+        for (int x = KC; x < 2 * KC; ++x)
+            if (x >= n) {
+                V(x) = -INFINITY;
+                I(x) = -1;
+            }
+        if (!kept_sorted) {
+            for (int x = 0; x < KC; ++x)
+                if (x >= n) {
+                    V(x) = -INFINITY;
+                    I(x) = -1;
+                }
+            sort_desc(0);
         }
+        sort_desc(KC);
+        for (int i = 0; i < KC; ++i) {
+            const int l = 2 * KC - 1 - i;
+            const float va = V(i), vb = V(l);
+            if (vb > va) {
+                V(i) = vb;
+                I(i) = I(l);
+            }
+        }
+        merge_desc();
     }
 };
 
@@ -169,7 +210,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
     unsigned char* c_s = smem + TC_OFF_C;
     float* val_s = reinterpret_cast<float*>(smem + TC_OFF_VAL);
     int* id_s = reinterpret_cast<int*>(smem + TC_OFF_ID);
-    float* stg_s = reinterpret_cast<float*>(smem + TC_OFF_STG);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TC_OFF_BAR);
     uint64_t* q_full = bars;
     uint64_t* full = bars + 1;
@@ -274,6 +314,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
         RowBuf rb{val_s + r, id_s + r};
         float thr = -INFINITY;
         int n_in = 0;
+        bool kept_sorted = false;   // warp-uniform
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
         for (int t = 0; t < n_tiles; ++t) {
             const int buf = t & 1;
@@ -286,42 +327,41 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
             }
             tc_fence_after();
             for (int c = 0; c < TC_N / 32; ++c) {
+                // keep room for a whole chunk of inserts: compact the warp's
+                // rows together (lockstep, no divergence) when any row is short
+                if (__any_sync(0xffffffffu, n_in > TC_BUF - 32)) {
+                    rb.compact(n_in, kept_sorted);
+                    kept_sorted = true;
+                    n_in = KC;
+                    thr = rb.V(KC - 1);
+                }
                 float v[32];
                 __syncwarp();
                 tmem_ld32(tmem + lane_base + (uint32_t)(buf * TC_N + c * 32), v);
                 const int64_t gbase = (int64_t)t * TC_N + c * 32;
-                // Hot path: one compare per score into a bit mask.  Columns at or
-                // beyond the row's eligible count never qualify.
+                // one compare per score into a bit mask; columns at or beyond
+                // the row's eligible count never qualify
                 uint32_t hit = 0;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) hit |= (v[j] > thr ? 1u : 0u) << j;
                 const int64_t room = nb_row - gbase;
                 if (room < 32) hit &= (room <= 0) ? 0u : ((1u << room) - 1u);
                 if (hit) {
-                    // Rare path: stage the 32 scores, insert the qualifying ones.
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) stg_s[j * TC_M + r] = v[j];
-                    while (hit) {
-                        const int j = __ffs(hit) - 1;
-                        hit &= hit - 1;
-                        const float sj = stg_s[j * TC_M + r];
-                        if (!(sj > thr)) continue;  // threshold may have risen
-                        rb.V(n_in) = sj;
-                        rb.I(n_in) = (int)(gbase + j);
-                        if (++n_in == TC_BUF) {
-                            rb.select_top(n_in, KC);
-                            float m = rb.V(0);
-                            for (int x = 1; x < KC; ++x) m = fminf(m, rb.V(x));
-                            thr = m;
-                            n_in = KC;
+                    for (int j = 0; j < 32; ++j)
+                        if ((hit >> j) & 1u) {
+                            rb.V(n_in) = v[j];
+                            rb.I(n_in) = (int)(gbase + j);
+                            ++n_in;
                         }
-                    }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
         }
+        // final top KC (lockstep again)
+        rb.compact(n_in, kept_sorted);
         if (row_valid) {
             const int64_t row = b * Nq + q0 + r;
             int32_t* cand = ws.cand + row * KC;
@@ -330,14 +370,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
                 ws.ncand[row] = (int32_t)nb_row;
                 ws.tau[row] = -INFINITY;
             } else {
-                if (n_in > KC) rb.select_top(n_in, KC);
-                float m = rb.V(0);
-                for (int x = 0; x < KC; ++x) {
-                    cand[x] = rb.I(x);
-                    m = fminf(m, rb.V(x));
-                }
+                for (int x = 0; x < KC; ++x) cand[x] = rb.I(x);
                 ws.ncand[row] = KC;
-                ws.tau[row] = m;
+                ws.tau[row] = rb.V(KC - 1);
             }
         }
     }

@@ -84,6 +84,67 @@ __device__ __forceinline__ void load_query(float* q_s, const T* lq, int64_t row)
 constexpr int SIMT_THREADS = 256;
 constexpr int64_t SIMT_SMEM_MAX = 220 * 1024;
 
+// Approximate (binary32) scores of buckets [0, nb) into sc.  Each lane reads
+// 16 bytes of a centroid row, so a warp covers several rows per load
+// (128-byte bf16 rows: 8 lanes per row; 256-byte fp32 rows: 16 lanes per
+// row) and the partial sums are reduced across the row's lanes.  The order of
+// the fp32 sum is irrelevant here: these scores only nominate candidates.
+__device__ void approx_scores(const IndexView& ix, const float* q_s, int64_t bseq, int64_t nb,
+                              float* sc)
+{
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    if (ix.dtype == LSA_BF16) {
+        constexpr int LPR = 8;                  // lanes per row (16 B = 8 bf16 each)
+        const int sub = lane % LPR, rsel = lane / LPR;
+        float q[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) q[e] = q_s[sub * 8 + e];
+        const uint4* base = reinterpret_cast<const uint4*>(
+            (const __nv_bfloat16*)ix.cent_rt + bseq * ix.NBK * DL);
+        for (int64_t g0 = (int64_t)warp * 4; g0 < nb; g0 += (int64_t)nwarps * 4) {
+            const int64_t g = g0 + rsel;
+            float acc = 0.f;
+            if (g < nb) {
+                const uint4 raw = base[g * (DL / 8) + sub];
+                const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(h[e]);
+                    acc = fmaf(q[2 * e], f.x, acc);
+                    acc = fmaf(q[2 * e + 1], f.y, acc);
+                }
+            }
+#pragma unroll
+            for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (sub == 0 && g < nb) sc[g] = acc;
+        }
+    } else {
+        constexpr int LPR = 16;                 // 16 B = 4 floats each
+        const int sub = lane % LPR, rsel = lane / LPR;
+        float q[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) q[e] = q_s[sub * 4 + e];
+        const float4* base =
+            reinterpret_cast<const float4*>((const float*)ix.cent_rt + bseq * ix.NBK * DL);
+        for (int64_t g0 = (int64_t)warp * 2; g0 < nb; g0 += (int64_t)nwarps * 2) {
+            const int64_t g = g0 + rsel;
+            float acc = 0.f;
+            if (g < nb) {
+                const float4 f = base[g * (DL / 4) + sub];
+                acc = fmaf(q[0], f.x, acc);
+                acc = fmaf(q[1], f.y, acc);
+                acc = fmaf(q[2], f.z, acc);
+                acc = fmaf(q[3], f.w, acc);
+            }
+#pragma unroll
+            for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (sub == 0 && g < nb) sc[g] = acc;
+        }
+    }
+    __syncthreads();
+}
+
 // Body of the SIMT nominator for query `row` at position pq; q_s holds the
 // latent query (every thread of the CTA calls it; sc holds n_blk*k floats).
 __device__ void simt_nominate(const IndexView& ix, int64_t n_blk, const float* q_s, int64_t bseq,
@@ -102,12 +163,7 @@ __device__ void simt_nominate(const IndexView& ix, int64_t n_blk, const float* q
         }
         return;
     }
-    for (int64_t g = threadIdx.x; g < nb; g += blockDim.x) {
-        float s = 0.f;
-#pragma unroll 16
-        for (int d = 0; d < DL; ++d) s = fmaf(q_s[d], rt_load(ix, bseq, g, d), s);
-        sc[g] = s;
-    }
+    approx_scores(ix, q_s, bseq, nb, sc);
     if (threadIdx.x == 0) {
         sh_prefix = 0;
         sh_want = KC;
@@ -227,6 +283,17 @@ __device__ int64_t warp_avail(const FillCtx& f, int64_t g)
     return a;
 }
 
+__device__ void warp_emit_partial(const FillCtx& f, int64_t g, int64_t take, int32_t* out);
+
+// True when every key of bucket g's closed members is available and no open
+// member can be: the bucket's available keys are then its members expanded.
+__device__ __forceinline__ bool bucket_full(const FillCtx& f, int64_t g)
+{
+    const int64_t span = (int64_t)f.ix.p * f.ix.G;
+    const int64_t bstart = (g / f.ix.k) * span;
+    return bstart >= f.S && bstart + span - 1 <= f.hi && !f.open_live;
+}
+
 // Writes the first `take` available keys of bucket g (ascending) to out.
 // Called by every thread of the CTA; uses warp 0 for partial buckets.
 __device__ void cta_emit(const FillCtx& f, int64_t g, int64_t take, int32_t* out)
@@ -246,7 +313,19 @@ __device__ void cta_emit(const FillCtx& f, int64_t g, int64_t take, int32_t* out
         return;
     }
     if (threadIdx.x >= 32) return;
-    const int lane = threadIdx.x;
+    warp_emit_partial(f, g, take, out);
+}
+
+// Warp-cooperative emission of the first `take` available keys of bucket g
+// (closed members, then open-block members), in ascending position.
+__device__ void warp_emit_partial(const FillCtx& f, int64_t g, int64_t take, int32_t* out)
+{
+    const IndexView& ix = f.ix;
+    const int32_t* off = ix.offsets + f.bseq * (ix.NBK + 1);
+    const int32_t* mem = ix.members + f.bseq * ix.NP;
+    const int p = ix.p;
+    const int32_t o0 = off[g], o1 = off[g + 1];
+    const int lane = threadIdx.x & 31;
     int64_t cur = 0;
     const int64_t nkeys = (int64_t)(o1 - o0) * p;
     for (int64_t x0 = 0; x0 < nkeys && cur < take; x0 += 32) {
@@ -306,6 +385,9 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     __shared__ int64_t av[KC];
     __shared__ int take_g[KC];
     __shared__ int64_t take_n[KC];
+    __shared__ int64_t take_off[KC];     // output offset of each taken bucket
+    __shared__ int32_t take_o0[KC];      // its first CSR position
+    __shared__ int take_full[KC];
     __shared__ int sh_ntake, sh_exact;
     __shared__ float sh_l1;
     const int64_t b = blockIdx.y, i = blockIdx.x;
@@ -358,6 +440,7 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
             const int64_t t = (a <= rem) ? a : rem;
             take_g[nt] = cg[c];
             take_n[nt] = t;
+            take_off[nt] = (int64_t)R - rem;
             ++nt;
             rem -= t;
             if (rem == 0) cut = c;
@@ -388,13 +471,34 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     int32_t* out = indices + row * (int64_t)s_max;
     const int64_t n_s = (S < pq + 1) ? S : pq + 1;
     for (int64_t x = threadIdx.x; x < n_s; x += FILL_THREADS) out[x] = (int32_t)x;
-    int64_t o = n_s;
-    for (int t = 0; t < sh_ntake; ++t) {
-        cta_emit(f, take_g[t], take_n[t], out + o);
-        o += take_n[t];
+    const int nt = sh_ntake;
+    const int32_t* offs = ix.offsets + b * (ix.NBK + 1);
+    const int32_t* mem = ix.members + b * ix.NP;
+    for (int t = threadIdx.x; t < nt; t += FILL_THREADS) {
+        take_full[t] = bucket_full(f, take_g[t]) ? 1 : 0;
+        take_o0[t] = offs[take_g[t]];
     }
     __syncthreads();
-    cta_emit_tail(pq, W, n_s, o, s_max, out, counts + row);
+    const int64_t n_lr = nt ? take_off[nt - 1] + take_n[nt - 1] : 0;
+    // Whole-member buckets: every long-range slot independently (a binary
+    // search finds its bucket), so all member reads are in flight at once.
+    const int p = ix.p;
+    for (int64_t x = threadIdx.x; x < n_lr; x += FILL_THREADS) {
+        int lo = 0, hi = nt - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (take_off[mid] <= x) lo = mid;
+            else hi = mid - 1;
+        }
+        if (!take_full[lo]) continue;
+        const int64_t rel = x - take_off[lo];
+        out[n_s + x] = mem[take_o0[lo] + rel / p] * p + (int32_t)(rel % p);
+    }
+    // Buckets cut by the window or the sinks, or with open members: one warp each.
+    for (int t = warp; t < nt; t += FILL_THREADS / 32)
+        if (!take_full[t]) warp_emit_partial(f, take_g[t], take_n[t], out + n_s + take_off[t]);
+    __syncthreads();
+    cta_emit_tail(pq, W, n_s, n_s + n_lr, s_max, out, counts + row);
 }
 
 // ---------------------------------------------------------------------------
@@ -579,18 +683,39 @@ __global__ void __launch_bounds__(SIMT_THREADS) decode_prep_kernel(
         q_s[i] = u;   // reuse as the unit vector
     }
     __syncthreads();
+    // Exact scores against every closed centroid.  Tiles of SIMT_THREADS
+    // centroid rows are staged into shared memory with coalesced 16-byte loads
+    // (row pitch DL + 1 floats, so that thread t reading row t hits its own
+    // bank); each thread then sums its row in ascending dimension.
     const float* cent = ix.cent + b * ix.NBK * DL;
     const int64_t nbk = n_blk * ix.k;
+    float* tile = sc;                                   // [SIMT_THREADS][DL + 1]
     double bs = -INFINITY;
     int bg = 0x7fffffff;
-    for (int64_t g = threadIdx.x; g < nbk; g += blockDim.x) {
-        const float* c = cent + g * DL;
-        double s = 0.0;
+    for (int64_t g0 = 0; g0 < nbk; g0 += SIMT_THREADS) {
+        const int rows = (int)((nbk - g0) < SIMT_THREADS ? (nbk - g0) : SIMT_THREADS);
+        __syncthreads();
+        const float4* src = reinterpret_cast<const float4*>(cent + g0 * DL);
+        for (int x = threadIdx.x; x < rows * (DL / 4); x += blockDim.x) {
+            const float4 f = src[x];
+            const int r = x / (DL / 4), c = (x % (DL / 4)) * 4;
+            float* dst = tile + r * (DL + 1) + c;
+            dst[0] = f.x;
+            dst[1] = f.y;
+            dst[2] = f.z;
+            dst[3] = f.w;
+        }
+        __syncthreads();
+        if ((int)threadIdx.x < rows) {
+            const float* c = tile + threadIdx.x * (DL + 1);
+            double s = 0.0;
 #pragma unroll 16
-        for (int i = 0; i < DL; ++i) s = __fma_rn((double)q_s[i], (double)c[i], s);
-        if (s > bs || (s == bs && (int)g < bg)) {
-            bs = s;
-            bg = (int)g;
+            for (int i = 0; i < DL; ++i) s = __fma_rn((double)q_s[i], (double)c[i], s);
+            const int g = (int)(g0 + threadIdx.x);
+            if (s > bs || (s == bs && g < bg)) {
+                bs = s;
+                bg = g;
+            }
         }
     }
     for (int off = 16; off > 0; off >>= 1) {
@@ -623,7 +748,9 @@ cudaError_t launch_decode_prep(const IndexView& ix, int64_t n_blk, void* latent_
                                int Hkv, int d, int W, const SelectWs& ws, uint32_t* attn_counter,
                                int counters_per_seq, cudaStream_t st)
 {
-    const size_t smem = (size_t)n_blk * ix.k * sizeof(float);
+    size_t smem = (size_t)n_blk * ix.k * sizeof(float);          // nominator scores
+    const size_t tile = (size_t)SIMT_THREADS * (DL + 1) * sizeof(float);  // exact-search tile
+    if (smem < tile) smem = tile;
     dim3 grid((unsigned)ix.B, 2);
     cudaError_t e;
     if (ix.dtype == LSA_BF16) {

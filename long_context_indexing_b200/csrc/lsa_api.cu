@@ -143,9 +143,10 @@ DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_sel
     L.n_hg = Hkv / hg;
     const int kt = attn_stage_keys(Hkv);
     const int64_t units = v.B * L.n_hg;
-    // about two CTAs per SM over all (sequence, head group, split) triples
-    int64_t ns = (2 * (int64_t)sm_count() + units - 1) / units;
+    // about one CTA per SM over all (sequence, head group, split) triples
+    int64_t ns = ((int64_t)sm_count() + units - 1) / units;
     if (ns < 1) ns = 1;
+    if (ns > 128) ns = 128;   // the combine keeps 2 * heads * ns floats in shared memory
     int64_t kps = (s_max + ns - 1) / ns;
     kps = ((kps + kt - 1) / kt) * kt;
     ns = (s_max + kps - 1) / kps;
