@@ -194,6 +194,23 @@ lsa_status lsa_select(const lsa_index* idx, const void* latent_Q, const int32_t*
                       int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
                       int s_max, void* workspace, size_t ws_bytes, void* stream);
 
+/* Same as lsa_select, for callers that cannot allocate device memory (a
+ * plug-in whose host hands it only input and output buffers, a serving loop
+ * whose device memory was divided up at start-up, a program with no device
+ * allocator): no workspace argument and no allocation.  The pages describe no
+ * such call; it exists for those callers.  Its scratch is one built-in 8 MiB
+ * device array that every GPU loading the library keeps until the process
+ * exits; a request needing more (lsa_select_workspace_bytes(idx, Nq) >
+ * 8 MiB, roughly Nq * 272 B + 148 * buckets * 8 B) returns
+ * LSA_ERR_WORKSPACE and launches nothing.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress); make that first
+ * call before any stream capture.  All calls share the array: calls that
+ * overlap on the GPU (other streams, other threads) race and must be
+ * serialised by the caller.  Results are identical to lsa_select's. */
+lsa_status lsa_select_noalloc(const lsa_index* idx, const void* latent_Q,
+                              const int32_t* positions, int64_t Nq, lsa_select_params sp,
+                              int32_t* indices, int32_t* counts, int s_max, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Exact sparse attention ("Prefrontal's ...", section "What it changes")
  *

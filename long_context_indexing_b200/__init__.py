@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "LsaError", "LsaIndex", "lsa_index_bytes", "lsa_build_index", "lsa_select",
     "lsa_sparse_attn", "lsa_prefill_chunk", "lsa_prefill_workspace_bytes",
-    "lsa_decode_workspace_bytes", "lsa_decode_step", "library_path", "kernel_launches", "F32",
+    "lsa_decode_workspace_bytes", "lsa_decode_step", "lsa_select_noalloc", "library_path", "kernel_launches", "F32",
     "BF16",
 ]
 
@@ -69,6 +69,8 @@ def _declare(lib):
         "lsa_prefill_chunk": ([P, P, P, P, P, P, I64, I64, I, I, I, SelectParams, P, SZ, P, P],
                               I),
         "lsa_decode_workspace_bytes": ([P, I, I, I, SelectParams], SZ),
+        "lsa_select_noalloc": ([P, P, P, I64, SelectParams, P, P, I, P], I),
+        "lsa_decode_step": ([P, P, P, P, P, P, P, P, P, P, I, I, I, SelectParams, P, SZ, P, P], I),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -236,6 +238,21 @@ def lsa_select(index, latent_Q, positions, budget, window, sinks, s_max=None, wo
     _check(_lib.lsa_select(index.handle, _ptr(latent_Q), _ptr(positions), Nq,
                            SelectParams(budget, window, sinks), _ptr(indices), _ptr(counts),
                            s_max, _ptr(workspace), workspace.numel(), _stream(stream)))
+    return indices, counts
+
+
+def lsa_select_noalloc(index, latent_Q, positions, budget, window, sinks, indices, counts,
+                       stream=None):
+    """lsa_select without a workspace, for callers that cannot allocate device
+    memory: the outputs `indices` [B][Nq][s_max] and `counts` [B][Nq] (int32)
+    are caller buffers and the scratch is the library's built-in device array
+    (see include/lsa.h for its limit and for the race between overlapping
+    calls)."""
+    _cuda(latent_Q, positions, indices, counts)
+    Nq = latent_Q.shape[1]
+    _check(_lib.lsa_select_noalloc(index.handle, _ptr(latent_Q), _ptr(positions), Nq,
+                                   SelectParams(budget, window, sinks), _ptr(indices),
+                                   _ptr(counts), indices.shape[-1], _stream(stream)))
     return indices, counts
 
 

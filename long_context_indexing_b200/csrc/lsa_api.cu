@@ -497,4 +497,32 @@ lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
     return LSA_OK;
 }
 
+lsa_status lsa_select_noalloc(const lsa_index* idx, const void* latent_Q,
+                              const int32_t* positions, int64_t Nq, lsa_select_params sp,
+                              int32_t* indices, int32_t* counts, int s_max, void* stream)
+{
+    if (!idx || !latent_Q || !positions || !indices || !counts)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    if (Nq < 0 || Nq > 2147483647LL) return fail(LSA_ERR_INVALID_ARG, "Nq out of range");
+    lsa_status s = check_select(idx, sp, s_max);
+    if (s != LSA_OK) return s;
+    if (!aligned16(latent_Q) || !aligned16(positions) || !aligned16(indices) || !aligned16(counts))
+        return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    const size_t need = select_ws_bytes(idx->v, Nq);
+    if (need > noalloc_scratch_bytes())
+        return fail(LSA_ERR_WORKSPACE,
+                    "selection of %lld queries over this index needs %zu bytes of scratch; the "
+                    "built-in array holds %zu: use lsa_select with a caller workspace",
+                    (long long)Nq, need, noalloc_scratch_bytes());
+    const bool tc = use_tc_path(idx, Nq);
+    if (!tc && idx->n_blk * idx->v.k > SIMT_MAX_BUCKETS)
+        return fail(LSA_ERR_UNSUPPORTED, "%lld buckets exceed the SIMT scorer's %lld",
+                    (long long)(idx->n_blk * idx->v.k), (long long)SIMT_MAX_BUCKETS);
+    if (Nq == 0) return LSA_OK;
+    cudaError_t e = noalloc_select(idx->v, idx->n_blk, latent_Q, positions, Nq, sp, indices,
+                                   counts, s_max, tc, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "select (built-in scratch)");
+    return LSA_OK;
+}
+
 }  // extern "C"

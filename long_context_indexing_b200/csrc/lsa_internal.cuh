@@ -144,6 +144,14 @@ cudaError_t launch_decode_prep(const IndexView& ix, int64_t n_blk, void* latent_
                                int Hkv, int d, int W, const SelectWs& ws, uint32_t* attn_counter,
                                int n_counter, cudaStream_t st);
 
+// Selection with scratch in a built-in device array (no caller workspace);
+// see k_select_noalloc.cu.
+size_t noalloc_scratch_bytes();
+cudaError_t noalloc_select(const IndexView& ix, int64_t n_blk, const void* latent_Q,
+                           const int32_t* positions, int64_t Nq, lsa_select_params sp,
+                           int32_t* indices, int32_t* counts, int s_max, bool use_tc,
+                           cudaStream_t st);
+
 // True when the tensor-core candidate scorer is compiled in.
 bool tc_scoring_available();
 
