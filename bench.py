@@ -404,7 +404,7 @@ def run_decode(args, peaks, peak_src, ws=1):
     open-list entries."""
     import long_context_indexing_b200 as lsa
 
-    w = synth.workload("decode")
+    w = synth.workload("decode", **({"T": args.decode_T} if args.decode_T else {}))
     dev = torch.device("cuda")
     span = w.p * w.G
     t_cap = w.T + span                      # room for the open block
@@ -503,6 +503,8 @@ def main():
     ap.add_argument("--ref-queries", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-T", type=int, default=None,
+                    help="override the decode context length (a multiple of p * block)")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the decode measurement (prints its object)")
     args = ap.parse_args()

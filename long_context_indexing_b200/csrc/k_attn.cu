@@ -190,7 +190,7 @@ struct AttnCfg {
 struct SplitKV {
     int ns;              // splits per (row, head group); 1 = off
     int keys_per_split;  // multiple of the stage size
-    float* part;         // [rows][ns][Hq][D + 2]  (m, l, acc[D])
+    float* part;         // [rows][ns][Hq][D + 4]  (acc[D], max, sum, pad)
     uint32_t* counter;   // [rows * n_hgroups], zero before the launch
 };
 
@@ -407,25 +407,28 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
         }
         return;
     }
-    // split-KV: write this split's partial per query head
+    // split-KV: write this split's partial per query head as
+    // [acc[0..D) | max | sum | 2 pad] (stride D + 4 floats, 16-byte aligned)
+    constexpr int PS = D + 4;
     for (int x = threadIdx.x; x < nq_heads * (D + 2); x += ATT_THREADS) {
         const int qh = x / (D + 2), c = x % (D + 2);
         const int hl = qh / hpg, h = qh % hpg;
         float M = -INFINITY;
         for (int sb = 0; sb < CONS_WARPS / HG; ++sb) M = fmaxf(M, mw[(sb * HG + hl) * 8 + h]);
         float v = 0.f;
-        if (c == 0) {
+        if (c == D) {
             v = M;
         } else {
             for (int sb = 0; sb < CONS_WARPS / HG; ++sb) {
                 const int w = sb * HG + hl;
                 const float sc = (mw[w * 8 + h] == -INFINITY) ? 0.f : exp2f(mw[w * 8 + h] - M);
-                v += (c == 1 ? lw[w * 8 + h] : ow[(w * 8 + h) * D + (c - 2)]) * sc;
+                v += (c == D + 1 ? lw[w * 8 + h] : ow[(w * 8 + h) * D + c]) * sc;
             }
         }
         const int64_t qhg = (int64_t)g0 * hpg + qh;
-        sk.part[((row * sk.ns + split) * Hq + qhg) * (D + 2) + c] = aborted ? nanf_ : v;
+        sk.part[((row * sk.ns + split) * Hq + qhg) * PS + c] = aborted ? nanf_ : v;
     }
+    if (!sk.counter) return;   // partials only: attn_combine_kernel merges them
     __threadfence();
     __syncthreads();
     __shared__ uint32_t sh_last;
@@ -442,14 +445,14 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
     // CTAs are read through L2 (__ldcg), never through a stale L1 line.
     float* m_sp = reinterpret_cast<float*>(smem);           // [nq_heads][ns]
     float* w_sp = m_sp + nq_heads * sk.ns;                   // [nq_heads][ns]
-    float* M_s = w_sp + nq_heads * sk.ns;                    // [nq_heads]
-    const int64_t sstride = (int64_t)Hq * (D + 2);
-    const float* pbase = sk.part + (row * sk.ns * Hq + (int64_t)g0 * hpg) * (D + 2);
+    const int64_t sstride = (int64_t)Hq * PS;
+    const float* pbase = sk.part + (row * sk.ns * Hq + (int64_t)g0 * hpg) * PS;
     for (int x = threadIdx.x; x < nq_heads * sk.ns; x += ATT_THREADS) {
         const int qh = x / sk.ns, sp = x % sk.ns;
-        const float* pp = pbase + sp * sstride + (int64_t)qh * (D + 2);
-        m_sp[x] = __ldcg(pp);
-        w_sp[x] = __ldcg(pp + 1);   // partial sum for now
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(pbase + sp * sstride +
+                                                                 (int64_t)qh * PS + D));
+        m_sp[x] = ml.x;
+        w_sp[x] = ml.y;   // partial sum for now
     }
     __syncthreads();
     for (int qh = threadIdx.x; qh < nq_heads; qh += ATT_THREADS) {
@@ -463,20 +466,102 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
             L += w_sp[qh * sk.ns + sp] * e;
         }
         for (int sp = 0; sp < sk.ns; ++sp) w_sp[qh * sk.ns + sp] = m_sp[qh * sk.ns + sp] / L;
-        M_s[qh] = M;
         if (lse) lse[row * Hq + (int64_t)g0 * hpg + qh] = (M + log2f(L)) * 0.69314718055994531f;
     }
     __syncthreads();
-    for (int x = threadIdx.x; x < nq_heads * D; x += ATT_THREADS) {
-        const int qh = x / D, c = x % D;
-        const float* pp = pbase + (int64_t)qh * (D + 2) + 2 + c;
+    // every output element is one weighted sum over splits; 4 dims per thread,
+    // several splits' loads in flight at once
+    for (int x = threadIdx.x; x < nq_heads * (D / 4); x += ATT_THREADS) {
+        const int qh = x / (D / 4), c = (x % (D / 4)) * 4;
+        const float* pp = pbase + (int64_t)qh * PS + c;
         const float* wq = w_sp + qh * sk.ns;
-        float acc = 0.f;
-#pragma unroll 4
-        for (int sp = 0; sp < sk.ns; ++sp) acc += __ldcg(pp + sp * sstride) * wq[sp];
-        O[(row * Hq + (int64_t)g0 * hpg + qh) * D + c] = __float2bfloat16_rn(acc);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int sp = 0; sp < sk.ns; ++sp) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(pp + sp * sstride));
+            const float w = wq[sp];
+            acc.x += v.x * w;
+            acc.y += v.y * w;
+            acc.z += v.z * w;
+            acc.w += v.w * w;
+        }
+        __nv_bfloat16* o = O + (row * Hq + (int64_t)g0 * hpg + qh) * D + c;
+        o[0] = __float2bfloat16_rn(acc.x);
+        o[1] = __float2bfloat16_rn(acc.y);
+        o[2] = __float2bfloat16_rn(acc.z);
+        o[3] = __float2bfloat16_rn(acc.w);
     }
     if (threadIdx.x == 0) sk.counter[unit] = 0;   // ready for the next launch
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV combine: one warp per (query row, query head).  Lane s holds split
+// s's (max, sum) (32 splits at a time); weights exp2(m_s - M) / L are
+// broadcast by shuffles and every lane accumulates 4 output dimensions with
+// 16-byte loads of each split's partial.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restrict__ part, int ns,
+                                                           int64_t n_heads_total, int Hq,
+                                                           __nv_bfloat16* O, float* lse)
+{
+    constexpr int PS = D + 4;
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);   // (row, head)
+    if (wid >= n_heads_total) return;
+    const int64_t row = wid / Hq, h = wid % Hq;
+    const float* base = part + (row * ns * Hq + h) * PS;
+    const int64_t sstride = (int64_t)Hq * PS;
+    float M = -INFINITY;
+    for (int s0 = 0; s0 < ns; s0 += 32)
+        if (s0 + lane < ns) M = fmaxf(M, __ldcg(base + (s0 + lane) * sstride + D));
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const bool live = lane < D / 4;
+    for (int s0 = 0; s0 < ns; s0 += 32) {
+        float w = 0.f;
+        if (s0 + lane < ns) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(base + (s0 + lane) * sstride + D));
+            w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
+            L += ml.y * w;
+        }
+        const int n = min(32, ns - s0);
+        for (int j = 0; j < n; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, w, j);
+            if (live) {
+                const float4 v =
+                    __ldcg(reinterpret_cast<const float4*>(base + (s0 + j) * sstride) + lane);
+                acc.x += v.x * wj;
+                acc.y += v.y * wj;
+                acc.z += v.z * wj;
+                acc.w += v.w * wj;
+            }
+        }
+    }
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (live) {
+        const float inv = 1.f / L;
+        __nv_bfloat16* op = O + wid * D + 4 * lane;
+        op[0] = __float2bfloat16_rn(acc.x * inv);
+        op[1] = __float2bfloat16_rn(acc.y * inv);
+        op[2] = __float2bfloat16_rn(acc.z * inv);
+        op[3] = __float2bfloat16_rn(acc.w * inv);
+    }
+    if (lane == 0 && lse) lse[wid] = (M + log2f(L)) * 0.69314718055994531f;
+}
+
+cudaError_t launch_attn_combine(const float* part, int ns, int64_t rows, int Hq, int d, void* O,
+                                float* lse, cudaStream_t st)
+{
+    const int64_t n = rows * Hq;
+    const unsigned grid = (unsigned)((n + 3) / 4);
+    if (d == 128)
+        attn_combine_kernel<128><<<grid, 128, 0, st>>>(part, ns, n, Hq, (__nv_bfloat16*)O, lse);
+    else
+        attn_combine_kernel<64><<<grid, 128, 0, st>>>(part, ns, n, Hq, (__nv_bfloat16*)O, lse);
+    note_launch();
+    return cudaGetLastError();
 }
 
 template <int D, int HG, int STAGES>
@@ -492,7 +577,7 @@ static cudaError_t launch_bf16(const void* Q, const void* K, const void* V, int6
     if (sk.ns > 1 && sk.keys_per_split % C::KT != 0) return cudaErrorInvalidValue;
     // the split combine keeps 2 * (query heads of the CTA) * ns + heads floats
     // in the freed ring
-    if (sk.ns > 1 && (size_t)(2 * HG * (Hq / Hkv) * sk.ns + HG * (Hq / Hkv)) * 4 > (size_t)C::BODY)
+    if (sk.ns > 1 && (size_t)(2 * HG * (Hq / Hkv) * sk.ns) * 4 > (size_t)C::BODY)
         return cudaErrorInvalidValue;
     const int64_t ctas = B * Nq * (Hkv / HG) * sk.ns;
     kern<<<(unsigned)ctas, ATT_THREADS, C::BYTES, st>>>(
@@ -549,8 +634,11 @@ template <int D>
 static cudaError_t launch_bf16_d(const void* Q, const void* K, const void* V, int64_t B, int64_t Nq,
                                  int64_t T_cap, int Hq, int Hkv, const int32_t* indices,
                                  const int32_t* counts, int s_max, float scale, void* O,
-                                 float* lse, uint32_t* status, SplitKV sk, cudaStream_t st)
+                                 float* lse, uint32_t* status, SplitKV sk, int hg, cudaStream_t st)
 {
+    if (hg == 1)
+        return launch_bf16<D, 1, 3>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale,
+                                    O, lse, status, sk, st);
     if (Hkv % 4 == 0)
         return launch_bf16<D, 4, 3>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale,
                                     O, lse, status, sk, st);
@@ -567,14 +655,14 @@ cudaError_t launch_attn_split(const void* Q, const void* K, const void* V, int64
                               int64_t T_cap, int Hq, int Hkv, int d, const int32_t* indices,
                               const int32_t* counts, int s_max, float scale, void* O, float* lse,
                               uint32_t* status, int ns, int keys_per_split, float* part,
-                              uint32_t* counter, cudaStream_t st)
+                              uint32_t* counter, int hg, cudaStream_t st)
 {
     SplitKV sk{ns, keys_per_split, part, counter};
     if (d == 128)
         return launch_bf16_d<128>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale,
-                                  O, lse, status, sk, st);
+                                  O, lse, status, sk, hg, st);
     return launch_bf16_d<64>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale, O, lse,
-                             status, sk, st);
+                             status, sk, hg, st);
 }
 
 cudaError_t launch_attn_status(const void* Q, const void* K, const void* V, lsa_dtype dt, int64_t B,
@@ -586,7 +674,7 @@ cudaError_t launch_attn_status(const void* Q, const void* K, const void* V, lsa_
     const int hpg = Hq / Hkv;
     if (dt == LSA_BF16)
         return launch_attn_split(Q, K, V, B, Nq, T_cap, Hq, Hkv, d, indices, counts, s_max, scale,
-                                 O, lse, status, 1, s_max, nullptr, nullptr, st);
+                                 O, lse, status, 1, s_max, nullptr, nullptr, 0, st);
 #define LSA_F32_CASE(H, DD)                                                                      \
     if (hpg == H && d == DD)                                                                     \
         return launch_f32<H, DD>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale, O, \

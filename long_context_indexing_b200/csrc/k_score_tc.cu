@@ -7,23 +7,24 @@
 // path: scores S = Q C^T with Q [queries][64] and C [buckets][64], both bf16,
 // accumulated in fp32.
 //
-// These approximate scores only nominate KC candidate buckets per query (its
-// running top-KC) together with tau, the KC-th largest approximate score: every
-// bucket left out scored at most tau.  The exact ranking and the fill happen
-// in select_fill_kernel (k_select.cu), which re-scores the candidates exactly.
+// These approximate scores are written as fp16 to a [queries][buckets] matrix
+// in the selection workspace; select_fill_kernel (k_select.cu) nominates each
+// query's candidates from its row and then ranks them with exact binary64
+// scores.  At 10M context the matrix is 32768 x 40960 fp16 (2.7 GB), written
+// once and read once.
 //
 // CTA = 128 queries of one sequence (one TMEM lane each), 6 warps:
 //   warp 0     TMA producer: the query tile once, then 256-centroid tiles into
 //              a TC_STAGES-deep shared-memory ring (128-byte swizzle);
 //   warp 1     owns 512 TMEM columns (two 256-column fp32 accumulators) and
 //              issues tcgen05.mma (M=128, N=256, K=16, four per tile);
-//   warps 2-5  epilogue: tcgen05.ld 32 columns at a time; per row, scores
-//              above the row's running threshold (the KC-th best kept so far)
-//              are appended to a 2*KC-slot buffer, which the warp compacts
-//              back to the top KC in lockstep when a row runs short of room.
+//   warps 2-5  epilogue: tcgen05.ld 32 columns at a time, fp32 -> fp16, and
+//              64-byte row segments straight to the score matrix.
 // Every mbarrier wait is bounded; on a timeout the CTA records DEV_TIMEOUT in
 // the index status word, stops waiting, and still frees its TMEM.
 #include <cuda.h>
+
+#include <cuda_fp16.h>
 
 #include "lsa_internal.cuh"
 #include "ptx.cuh"
@@ -32,22 +33,18 @@ namespace lsa {
 
 constexpr int TC_M = 128;
 constexpr int TC_N = 256;
-constexpr int TC_STAGES = 2;
-constexpr int TC_BUF = 2 * KC;                 // kept top-KC + KC new slots
+constexpr int TC_STAGES = 4;
 constexpr int TC_THREADS = 192;
 constexpr uint32_t TC_WAIT = 1u << 22;
 
 constexpr int TC_Q_BYTES = TC_M * DL * 2;                 // 16 KB
 constexpr int TC_C_BYTES = TC_N * DL * 2;                 // 32 KB per stage
 constexpr int TC_OFF_C = TC_Q_BYTES;
-constexpr int TC_OFF_VAL = TC_OFF_C + TC_STAGES * TC_C_BYTES;
-constexpr int TC_OFF_ID = TC_OFF_VAL + TC_BUF * TC_M * 4;
-constexpr int TC_OFF_BAR = TC_OFF_ID + TC_BUF * TC_M * 4;
+constexpr int TC_OFF_BAR = TC_OFF_C + TC_STAGES * TC_C_BYTES;
 constexpr int TC_NBAR = 1 + 2 * TC_STAGES + 4;
 constexpr int TC_OFF_MISC = TC_OFF_BAR + TC_NBAR * 8;
 constexpr int TC_SMEM = TC_OFF_MISC + 64 + 1024;          // + alignment slack
 
-static_assert(KC <= TC_BUF, "buffer must hold KC candidates");
 
 // ---- tcgen05 / TMA wrappers -------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
@@ -113,81 +110,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v)
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
-// ---- per-row candidate buffer (strided by TC_M in shared memory) -----------
-// Slots [0, KC) hold the kept candidates (sorted by score, descending, after
-// the first compaction); new entries go to [KC, 2KC).  A compaction keeps the
-// top KC of all 2KC slots with a data-oblivious network (every lane of a warp
-// runs the same compare-exchange sequence on its own row, so the warp never
-// diverges): bitonic sort of the new half, element-wise max of the kept half
-// against the reversed new half (a bitonic sequence holding the top KC), and
-// a bitonic merge of that sequence.
-struct RowBuf {
-    float* v;
-    int* id;
-    __device__ __forceinline__ float& V(int x) { return v[x * TC_M]; }
-    __device__ __forceinline__ int& I(int x) { return id[x * TC_M]; }
-    // compare-exchange so that slot a ends up with the larger score
-    __device__ __forceinline__ void cx_desc(int a, int b)
-    {
-        const float va = V(a), vb = V(b);
-        const int ia = I(a), ib = I(b);
-        const bool sw = va < vb;
-        V(a) = sw ? vb : va;
-        V(b) = sw ? va : vb;
-        I(a) = sw ? ib : ia;
-        I(b) = sw ? ia : ib;
-    }
-    // bitonic sort (descending) of the KC slots starting at `base`
-    __device__ void sort_desc(int base)
-    {
-        for (int k = 2; k <= KC; k <<= 1)
-            for (int j = k >> 1; j > 0; j >>= 1)
-                for (int t = 0; t < KC / 2; ++t) {
-                    const int i = ((t & ~(j - 1)) << 1) | (t & (j - 1));
-                    const int l = i | j;
-                    if ((i & k) == 0) cx_desc(base + i, base + l);
-                    else cx_desc(base + l, base + i);
-                }
-    }
-    // bitonic merge (descending) of a bitonic sequence in [0, KC)
-    __device__ void merge_desc()
-    {
-        for (int j = KC >> 1; j > 0; j >>= 1)
-            for (int t = 0; t < KC / 2; ++t) {
-                const int i = ((t & ~(j - 1)) << 1) | (t & (j - 1));
-                cx_desc(i, i | j);
-            }
-    }
-    // top KC of all 2KC slots into [0, KC), sorted descending; slots from n
-    // on are empty and padded first
-    __device__ void compact(int n, bool kept_sorted)
-    {
-        for (int x = KC; x < 2 * KC; ++x)
-            if (x >= n) {
-                V(x) = -INFINITY;
-                I(x) = -1;
-            }
-        if (!kept_sorted) {
-            for (int x = 0; x < KC; ++x)
-                if (x >= n) {
-                    V(x) = -INFINITY;
-                    I(x) = -1;
-                }
-            sort_desc(0);
-        }
-        sort_desc(KC);
-        for (int i = 0; i < KC; ++i) {
-            const int l = 2 * KC - 1 - i;
-            const float va = V(i), vb = V(l);
-            if (vb > va) {
-                V(i) = vb;
-                I(i) = I(l);
-            }
-        }
-        merge_desc();
-    }
-};
-
 __device__ __forceinline__ int64_t tc_eligible(const IndexView& ix, int64_t n_blk, int64_t pos,
                                                int W)
 {
@@ -208,8 +130,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
         (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);  // 1 KB aligned
     unsigned char* q_s = smem;
     unsigned char* c_s = smem + TC_OFF_C;
-    float* val_s = reinterpret_cast<float*>(smem + TC_OFF_VAL);
-    int* id_s = reinterpret_cast<int*>(smem + TC_OFF_ID);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TC_OFF_BAR);
     uint64_t* q_full = bars;
     uint64_t* full = bars + 1;
@@ -311,11 +231,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
         }
     } else if (warp >= 2) {
         // ---------------- epilogue ----------------
-        RowBuf rb{val_s + r, id_s + r};
-        float thr = -INFINITY;
-        int n_in = 0;
-        bool kept_sorted = false;   // warp-uniform
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        __half* srow = ws.scores + (b * Nq + q0 + r) * ws.score_ld;
+        __half* crow = ws.cmax + (b * Nq + q0 + r) * (ws.score_ld / 32);
         for (int t = 0; t < n_tiles; ++t) {
             const int buf = t & 1;
             const uint32_t ph = (uint32_t)((t >> 1) & 1);
@@ -327,53 +245,30 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
             }
             tc_fence_after();
             for (int c = 0; c < TC_N / 32; ++c) {
-                // keep room for a whole chunk of inserts: compact the warp's
-                // rows together (lockstep, no divergence) when any row is short
-                if (__any_sync(0xffffffffu, n_in > TC_BUF - 32)) {
-                    rb.compact(n_in, kept_sorted);
-                    kept_sorted = true;
-                    n_in = KC;
-                    thr = rb.V(KC - 1);
-                }
                 float v[32];
                 __syncwarp();
                 tmem_ld32(tmem + lane_base + (uint32_t)(buf * TC_N + c * 32), v);
-                const int64_t gbase = (int64_t)t * TC_N + c * 32;
-                // one compare per score into a bit mask; columns at or beyond
-                // the row's eligible count never qualify
-                uint32_t hit = 0;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) hit |= (v[j] > thr ? 1u : 0u) << j;
-                const int64_t room = nb_row - gbase;
-                if (room < 32) hit &= (room <= 0) ? 0u : ((1u << room) - 1u);
-                if (hit) {
+                const int64_t g0 = (int64_t)t * TC_N + c * 32;
+                if (row_valid && g0 < nb_row) {
+                    uint4 pk[4];
+                    __half2* h = reinterpret_cast<__half2*>(pk);
+                    float mx = -INFINITY;
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if ((hit >> j) & 1u) {
-                            rb.V(n_in) = v[j];
-                            rb.I(n_in) = (int)(gbase + j);
-                            ++n_in;
-                        }
+                        if (g0 + j < nb_row) mx = fmaxf(mx, v[j]);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) h[j] = __floats2half2_rn(v[2 * j], v[2 * j + 1]);
+                    uint4* dst = reinterpret_cast<uint4*>(srow + g0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) dst[j] = pk[j];
+                    // fp16 rounding is monotone: the rounded maximum is the
+                    // maximum of the rounded scores of the chunk
+                    crow[g0 / 32] = __float2half_rn(mx);
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
-        }
-        // final top KC (lockstep again)
-        rb.compact(n_in, kept_sorted);
-        if (row_valid) {
-            const int64_t row = b * Nq + q0 + r;
-            int32_t* cand = ws.cand + row * KC;
-            if (nb_row <= KC) {
-                for (int x = 0; x < KC; ++x) cand[x] = (x < nb_row) ? x : -1;
-                ws.ncand[row] = (int32_t)nb_row;
-                ws.tau[row] = -INFINITY;
-            } else {
-                for (int x = 0; x < KC; ++x) cand[x] = rb.I(x);
-                ws.ncand[row] = KC;
-                ws.tau[row] = rb.V(KC - 1);
-            }
         }
     }
     tc_fence_before();

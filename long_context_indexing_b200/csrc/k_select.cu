@@ -92,57 +92,109 @@ constexpr int64_t SIMT_SMEM_MAX = 220 * 1024;
 __device__ void approx_scores(const IndexView& ix, const float* q_s, int64_t bseq, int64_t nb,
                               float* sc)
 {
+    // Each warp handles a contiguous range of rows; the loads of UNR
+    // iterations are issued before any of them is consumed, so a warp keeps
+    // UNR * 512 bytes in flight instead of waiting on one load at a time.
+    constexpr int UNR = 8;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     if (ix.dtype == LSA_BF16) {
-        constexpr int LPR = 8;                  // lanes per row (16 B = 8 bf16 each)
+        constexpr int LPR = 8, RPI = 32 / LPR;  // lanes per row, rows per iteration
         const int sub = lane % LPR, rsel = lane / LPR;
         float q[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) q[e] = q_s[sub * 8 + e];
         const uint4* base = reinterpret_cast<const uint4*>(
             (const __nv_bfloat16*)ix.cent_rt + bseq * ix.NBK * DL);
-        for (int64_t g0 = (int64_t)warp * 4; g0 < nb; g0 += (int64_t)nwarps * 4) {
-            const int64_t g = g0 + rsel;
-            float acc = 0.f;
-            if (g < nb) {
-                const uint4 raw = base[g * (DL / 8) + sub];
-                const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        for (int64_t g0 = (int64_t)warp * RPI * UNR; g0 < nb; g0 += (int64_t)nwarps * RPI * UNR) {
+            uint4 raw[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int64_t g = g0 + u * RPI + rsel;
+                raw[u] = (g < nb) ? __ldg(base + g * (DL / 8) + sub) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+                float acc = 0.f;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 f = __bfloat1622float2(h[e]);
                     acc = fmaf(q[2 * e], f.x, acc);
                     acc = fmaf(q[2 * e + 1], f.y, acc);
                 }
-            }
 #pragma unroll
-            for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (sub == 0 && g < nb) sc[g] = acc;
+                for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                const int64_t g = g0 + u * RPI + rsel;
+                if (sub == 0 && g < nb) sc[g] = acc;
+            }
         }
     } else {
-        constexpr int LPR = 16;                 // 16 B = 4 floats each
+        constexpr int LPR = 16, RPI = 32 / LPR;
         const int sub = lane % LPR, rsel = lane / LPR;
         float q[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) q[e] = q_s[sub * 4 + e];
         const float4* base =
             reinterpret_cast<const float4*>((const float*)ix.cent_rt + bseq * ix.NBK * DL);
-        for (int64_t g0 = (int64_t)warp * 2; g0 < nb; g0 += (int64_t)nwarps * 2) {
-            const int64_t g = g0 + rsel;
-            float acc = 0.f;
-            if (g < nb) {
-                const float4 f = base[g * (DL / 4) + sub];
-                acc = fmaf(q[0], f.x, acc);
-                acc = fmaf(q[1], f.y, acc);
-                acc = fmaf(q[2], f.z, acc);
-                acc = fmaf(q[3], f.w, acc);
+        for (int64_t g0 = (int64_t)warp * RPI * UNR; g0 < nb; g0 += (int64_t)nwarps * RPI * UNR) {
+            float4 f[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int64_t g = g0 + u * RPI + rsel;
+                f[u] = (g < nb) ? __ldg(base + g * (DL / 4) + sub) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
-            for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (sub == 0 && g < nb) sc[g] = acc;
+            for (int u = 0; u < UNR; ++u) {
+                float acc = fmaf(q[0], f[u].x, 0.f);
+                acc = fmaf(q[1], f[u].y, acc);
+                acc = fmaf(q[2], f[u].z, acc);
+                acc = fmaf(q[3], f[u].w, acc);
+#pragma unroll
+                for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                const int64_t g = g0 + u * RPI + rsel;
+                if (sub == 0 && g < nb) sc[g] = acc;
+            }
         }
     }
     __syncthreads();
+}
+
+// Exact score of one bucket: the retrieval centroid's row is read with 16-byte
+// loads (all in flight together), then summed in ascending dimension as exact
+// binary64 products.
+__device__ __forceinline__ double exact_score(const IndexView& ix, int64_t bseq, int64_t g,
+                                              const float* q_s)
+{
+    double s = 0.0;
+    if (ix.dtype == LSA_BF16) {
+        const uint4* row = reinterpret_cast<const uint4*>((const __nv_bfloat16*)ix.cent_rt +
+                                                          (bseq * ix.NBK + g) * DL);
+        uint4 raw[DL / 8];
+#pragma unroll
+        for (int x = 0; x < DL / 8; ++x) raw[x] = __ldg(row + x);
+#pragma unroll
+        for (int x = 0; x < DL / 8; ++x) {
+            const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw[x]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                s = __fma_rn((double)q_s[x * 8 + e], (double)__bfloat162float(h[e]), s);
+        }
+    } else {
+        const float4* row =
+            reinterpret_cast<const float4*>((const float*)ix.cent_rt + (bseq * ix.NBK + g) * DL);
+        float4 f[DL / 4];
+#pragma unroll
+        for (int x = 0; x < DL / 4; ++x) f[x] = __ldg(row + x);
+#pragma unroll
+        for (int x = 0; x < DL / 4; ++x) {
+            s = __fma_rn((double)q_s[4 * x + 0], (double)f[x].x, s);
+            s = __fma_rn((double)q_s[4 * x + 1], (double)f[x].y, s);
+            s = __fma_rn((double)q_s[4 * x + 2], (double)f[x].z, s);
+            s = __fma_rn((double)q_s[4 * x + 3], (double)f[x].w, s);
+        }
+    }
+    return s;
 }
 
 // Body of the SIMT nominator for query `row` at position pq; q_s holds the
@@ -182,16 +234,36 @@ __device__ void simt_nominate(const IndexView& ix, int64_t n_blk, const float* q
             if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> sh) & 255u], 1u);
         }
         __syncthreads();
-        if (threadIdx.x == 0) {
-            uint32_t want = sh_want, cum = 0;
-            for (int bin = 255; bin >= 0; --bin) {
-                const uint32_t h = hist[bin];
-                if (cum + h >= want) {
-                    sh_prefix = prefix | ((uint32_t)bin << sh);
-                    sh_want = want - cum;
-                    break;
+        if (threadIdx.x < 32) {
+            // warp 0 finds the bin holding the want-th largest key: lane l owns
+            // bins 255-8l .. 248-8l (high to low); an exclusive scan of the lane
+            // totals gives each lane the count above its bins.
+            const int l = threadIdx.x;
+            uint32_t hb[8], tot = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                hb[e] = hist[255 - 8 * l - e];
+                tot += hb[e];
+            }
+            uint32_t incl = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (l >= o) incl += y;
+            }
+            const uint32_t want = sh_want;
+            uint32_t cum = incl - tot;
+            const bool mine = cum < want && incl >= want;
+            if (mine) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if (cum + hb[e] >= want) {
+                        sh_prefix = prefix | ((uint32_t)(255 - 8 * l - e) << sh);
+                        sh_want = want - cum;
+                        break;
+                    }
+                    cum += hb[e];
                 }
-                cum += h;
             }
         }
         mask |= 255u << sh;
@@ -367,11 +439,194 @@ __device__ void cta_emit_tail(int64_t pq, int W, int64_t n_s, int64_t off, int s
 }
 
 // ---------------------------------------------------------------------------
+// Candidate nomination from a query's fp16 tensor-core scores.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t half_key(uint32_t u)
+{
+    u &= 0xFFFFu;
+    return (u & 0x8000u) ? (~u & 0xFFFFu) : (u | 0x8000u);
+}
+
+__device__ __forceinline__ float key_half_value(uint32_t k)
+{
+    const uint16_t u = (k & 0x8000u) ? (uint16_t)(k & 0x7FFFu) : (uint16_t)(~k & 0xFFFFu);
+    return __half2float(__ushort_as_half(u));
+}
+
+constexpr int FILL_THREADS = 128;
+// Radix select (two 8-bit passes over 16-bit keys) shared by the nominator:
+// every thread offers up to NK keys (0 = none); returns the key of the
+// want-th largest and, in *need_eq, how many keys equal to it are needed to
+// make up `want`.
+template <int NK>
+__device__ uint32_t radix16_kth(const uint32_t (&key)[NK], uint32_t want, int* need_eq)
+{
+    __shared__ unsigned hist[256];
+    __shared__ uint32_t sh_prefix, sh_want;
+    if (threadIdx.x == 0) {
+        sh_prefix = 0;
+        sh_want = want;
+    }
+    uint32_t mask = 0;
+    for (int pass = 1; pass >= 0; --pass) {
+        const int sh = 8 * pass;
+        for (int x = threadIdx.x; x < 256; x += blockDim.x) hist[x] = 0;
+        __syncthreads();
+        const uint32_t prefix = sh_prefix;
+#pragma unroll
+        for (int i = 0; i < NK; ++i)
+            if (key[i] != 0u && (key[i] & mask) == prefix) atomicAdd(&hist[(key[i] >> sh) & 255u], 1u);
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            const int l = threadIdx.x;
+            uint32_t hb[8], tot = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                hb[e] = hist[255 - 8 * l - e];
+                tot += hb[e];
+            }
+            uint32_t incl = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (l >= o) incl += y;
+            }
+            const uint32_t w = sh_want;
+            uint32_t cum = incl - tot;
+            if (cum < w && incl >= w) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if (cum + hb[e] >= w) {
+                        sh_prefix = prefix | ((uint32_t)(255 - 8 * l - e) << sh);
+                        sh_want = w - cum;
+                        break;
+                    }
+                    cum += hb[e];
+                }
+            }
+        }
+        mask |= 255u << sh;
+        __syncthreads();
+    }
+    *need_eq = (int)sh_want;
+    const uint32_t T = sh_prefix;
+    __syncthreads();
+    return T;
+}
+
+constexpr int NOM_CHUNK_MAX = 2048;   // chunk maxima held in registers: up to 65536 buckets
+
+// Candidate nomination from a query's fp16 tensor-core scores (CTA of
+// FILL_THREADS threads, nb > KC eligible buckets).  The scores come in chunks
+// of 32 with each chunk's maximum stored beside them.  The KC chunks with the
+// largest maxima hold the KC largest scores (each of those scores is at least
+// the KC-th largest chunk maximum, so it lies in a chunk whose maximum is at
+// least that), so only those chunks are read: the KC largest of their scores
+// are the candidates.  Every bucket left out scored at most
+// tau16 = max(the KC-th largest key among the read scores, the largest
+// maximum of a chunk that was not read).  Returns the fp32 upper bound of the
+// approximate binary32 score of every bucket left out: the midpoint between
+// tau16 and the next fp16 value above it (round to nearest put every such
+// score at or below it).
+__device__ float nominate_from_scores(const __half* srow, const __half* crow, int64_t nb,
+                                      int* cg)
+{
+    __shared__ int chunk_sel[KC];
+    __shared__ uint8_t in_sel[NOM_CHUNK_MAX];
+    __shared__ uint32_t sh_rest;
+    __shared__ int sh_gt, sh_eq;
+    const int nch = (int)((nb + 31) / 32);
+    constexpr int CPT = NOM_CHUNK_MAX / FILL_THREADS;       // chunk keys per thread
+    if (threadIdx.x == 0) {
+        sh_rest = 0;
+        sh_gt = 0;
+        sh_eq = 0;
+    }
+    for (int c = threadIdx.x; c < nch; c += FILL_THREADS) in_sel[c] = 0;
+    // 1. the KC chunks with the largest maxima (all of them when nch <= KC)
+    uint32_t ck[CPT];
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = threadIdx.x + i * FILL_THREADS;
+        ck[i] = (c < nch) ? half_key(__half_as_ushort(crow[c])) : 0u;
+    }
+    int n_read;
+    if (nch <= KC) {
+        for (int c = threadIdx.x; c < nch; c += FILL_THREADS) chunk_sel[c] = c;
+        n_read = nch;
+        __syncthreads();
+    } else {
+        int need;
+        const uint32_t Tc = radix16_kth<CPT>(ck, KC, &need);
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = threadIdx.x + i * FILL_THREADS;
+            if (ck[i] > Tc) {
+                const int q = atomicAdd(&sh_gt, 1);
+                chunk_sel[q] = c;
+                in_sel[c] = 1;
+            } else if (ck[i] == Tc && ck[i] != 0u) {
+                const int q = atomicAdd(&sh_eq, 1);
+                if (q < need) {
+                    chunk_sel[KC - need + q] = c;
+                    in_sel[c] = 1;
+                }
+            }
+        }
+        __syncthreads();
+        // the largest maximum among chunks not read bounds every score in them
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = threadIdx.x + i * FILL_THREADS;
+            if (c < nch && !in_sel[c]) atomicMax(&sh_rest, ck[i]);
+        }
+        n_read = KC;
+    }
+    // 2. the read chunks' scores: KC chunks x 32 = 2048 keys, 16 per thread
+    constexpr int EPT = KC * 32 / FILL_THREADS;
+    uint32_t ek[EPT];
+    int eg[EPT];
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+        const int slot = threadIdx.x + i * FILL_THREADS;      // slot = chunk rank * 32 + lane
+        const int ci = slot >> 5, j = slot & 31;
+        ek[i] = 0u;
+        eg[i] = -1;
+        if (ci < n_read) {
+            const int64_t g = (int64_t)chunk_sel[ci] * 32 + j;
+            if (g < nb) {
+                ek[i] = half_key(__half_as_ushort(srow[g]));
+                eg[i] = (int)g;
+            }
+        }
+    }
+    if (threadIdx.x == 0) {
+        sh_gt = 0;
+        sh_eq = 0;
+    }
+    int need;
+    const uint32_t T = radix16_kth<EPT>(ek, KC, &need);
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+        if (ek[i] == 0u) continue;
+        if (ek[i] > T) {
+            cg[atomicAdd(&sh_gt, 1)] = eg[i];
+        } else if (ek[i] == T) {
+            const int q = atomicAdd(&sh_eq, 1);
+            if (q < need) cg[KC - need + q] = eg[i];
+        }
+    }
+    __syncthreads();
+    const uint32_t k = T > sh_rest ? T : sh_rest;
+    const float tv = key_half_value(k);
+    const float above = (k >= 0xFFFFu) ? INFINITY : key_half_value(k + 1);
+    return tv + 0.5f * (above - tv);
+}
+
+// ---------------------------------------------------------------------------
 // Exact ranking + greedy fill + emission.  One CTA (128 threads) per query.
 // ---------------------------------------------------------------------------
-constexpr int FILL_THREADS = 128;
-
-template <typename T>
+template <typename T, bool FROM_SCORES>
 __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix, int64_t n_blk,
                                                                    const T* lq, PosSrc pos,
                                                                    int64_t Nq, int R, int W, int S,
@@ -394,21 +649,31 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     const int64_t row = b * Nq + i;
     const int64_t pq = pos.at(b, Nq, i);
     load_query(q_s, lq, row);
-    const int nc = ws.ncand[row];
-    if (threadIdx.x < KC) cg[threadIdx.x] = ws.cand[row * KC + threadIdx.x];
+    int nc;
+    float tau;
+    if (FROM_SCORES) {
+        const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
+        if (nb <= KC) {
+            if (threadIdx.x < KC) cg[threadIdx.x] = (threadIdx.x < nb) ? (int)threadIdx.x : -1;
+            nc = (int)nb;
+            tau = -INFINITY;
+        } else {
+            tau = nominate_from_scores(ws.scores + row * ws.score_ld,
+                                       ws.cmax + row * (ws.score_ld / 32), nb, cg);
+            nc = KC;
+        }
+    } else {
+        nc = ws.ncand[row];
+        tau = ws.tau[row];
+        if (threadIdx.x < KC) cg[threadIdx.x] = ws.cand[row * KC + threadIdx.x];
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
         float l1 = 0.f;
         for (int d = 0; d < DL; ++d) l1 += fabsf(q_s[d]);
         sh_l1 = l1;
     }
-    if ((int)threadIdx.x < nc) {
-        const int g = cg[threadIdx.x];
-        double s = 0.0;
-#pragma unroll 16
-        for (int d = 0; d < DL; ++d) s = __fma_rn((double)q_s[d], (double)rt_load(ix, b, g, d), s);
-        es[threadIdx.x] = s;
-    }
+    if ((int)threadIdx.x < nc) es[threadIdx.x] = exact_score(ix, b, cg[threadIdx.x], q_s);
     __syncthreads();
     if ((int)threadIdx.x < nc) {
         const int c = threadIdx.x;
@@ -425,7 +690,25 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     f.S = S;
     f.open_live = (n_blk < ix.nblk_max) && (n_blk > 0) && (n_blk * (int64_t)ix.p * ix.G <= f.hi);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int c = warp; c < nc; c += FILL_THREADS / 32) {
+    __shared__ int slow[KC];
+    __shared__ int n_slow;
+    if (threadIdx.x == 0) n_slow = 0;
+    __syncthreads();
+    if ((int)threadIdx.x < nc) {
+        // buckets whose keys are all available: count = p * members, one
+        // round trip for every candidate at once
+        const int c = threadIdx.x;
+        const int g = cg[c];
+        if (bucket_full(f, g)) {
+            const int32_t* off = ix.offsets + b * (ix.NBK + 1);
+            av[c] = (int64_t)(off[g + 1] - off[g]) * ix.p;
+        } else {
+            slow[atomicAdd(&n_slow, 1)] = c;
+        }
+    }
+    __syncthreads();
+    for (int e = warp; e < n_slow; e += FILL_THREADS / 32) {
+        const int c = slow[e];
         const int64_t a = warp_avail(f, cg[c]);
         if (lane == 0) av[c] = a;
     }
@@ -453,7 +736,7 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
                 if (total < 0) total = 0;
                 exact = ((int64_t)R - rem) >= total;
             } else if (cut >= 0) {
-                exact = es[cut] > (double)ws.tau[row] + eps;
+                exact = es[cut] > (double)tau + eps;
             }
         }
         sh_ntake = nt;
@@ -483,16 +766,35 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     // Whole-member buckets: every long-range slot independently (a binary
     // search finds its bucket), so all member reads are in flight at once.
     const int p = ix.p;
-    for (int64_t x = threadIdx.x; x < n_lr; x += FILL_THREADS) {
-        int lo = 0, hi = nt - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (take_off[mid] <= x) lo = mid;
-            else hi = mid - 1;
+    constexpr int EU = 8;   // slots per thread per batch: EU member loads in flight
+    for (int64_t x0 = threadIdx.x; x0 < n_lr; x0 += (int64_t)FILL_THREADS * EU) {
+        int64_t src[EU];
+        int rem_[EU];
+#pragma unroll
+        for (int u = 0; u < EU; ++u) {
+            const int64_t x = x0 + (int64_t)u * FILL_THREADS;
+            src[u] = -1;
+            rem_[u] = 0;
+            if (x < n_lr) {
+                int lo = 0, hi = nt - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (take_off[mid] <= x) lo = mid;
+                    else hi = mid - 1;
+                }
+                if (take_full[lo]) {
+                    const int64_t rel = x - take_off[lo];
+                    src[u] = take_o0[lo] + rel / p;
+                    rem_[u] = (int)(rel % p);
+                }
+            }
         }
-        if (!take_full[lo]) continue;
-        const int64_t rel = x - take_off[lo];
-        out[n_s + x] = mem[take_o0[lo] + rel / p] * p + (int32_t)(rel % p);
+        int32_t m[EU];
+#pragma unroll
+        for (int u = 0; u < EU; ++u) m[u] = (src[u] >= 0) ? __ldg(mem + src[u]) : 0;
+#pragma unroll
+        for (int u = 0; u < EU; ++u)
+            if (src[u] >= 0) out[n_s + x0 + (int64_t)u * FILL_THREADS] = m[u] * p + rem_[u];
     }
     // Buckets cut by the window or the sinks, or with open members: one warp each.
     for (int t = warp; t < nt; t += FILL_THREADS / 32)
@@ -532,11 +834,7 @@ __global__ void __launch_bounds__(FB_THREADS) select_fallback_kernel(IndexView i
         __syncthreads();
         load_query(q_s, lq, row);
         __syncthreads();
-        for (int64_t g = threadIdx.x; g < nb; g += FB_THREADS) {
-            double s = 0.0;
-            for (int d = 0; d < DL; ++d) s = __fma_rn((double)q_s[d], (double)rt_load(ix, b, g, d), s);
-            sc[g] = s;
-        }
+        for (int64_t g = threadIdx.x; g < nb; g += FB_THREADS) sc[g] = exact_score(ix, b, g, q_s);
         FillCtx f;
         f.ix = ix;
         f.bseq = b;
@@ -779,11 +1077,22 @@ cudaError_t launch_decode_prep(const IndexView& ix, int64_t n_blk, void* latent_
 // ---------------------------------------------------------------------------
 static inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+bool select_uses_tc(const IndexView& ix, int64_t Nq)
+{
+    return ix.dtype == LSA_BF16 && Nq >= 128 && ix.NBK <= (int64_t)NOM_CHUNK_MAX * 32 &&
+           tc_scoring_available();
+}
+
+static int64_t score_ld_of(const IndexView& ix) { return ((ix.NBK + 255) / 256) * 256; }
+
 size_t select_ws_bytes(const IndexView& ix, int64_t Nq)
 {
     const size_t rows = (size_t)ix.B * (size_t)Nq;
-    return al256(rows * KC * 4) + al256(rows * 4) + al256(rows * 4) + al256(rows * 4) + al256(4) +
-           al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
+    size_t n = al256(rows * KC * 4) + al256(rows * 4) + al256(rows * 4) + al256(rows * 4) + al256(4) +
+               al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
+    if (select_uses_tc(ix, Nq))
+        n += al256(rows * (size_t)score_ld_of(ix) * 2) + al256(rows * (size_t)score_ld_of(ix) / 16);
+    return n;
 }
 
 SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
@@ -802,6 +1111,15 @@ SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
     w.fb_count = (int32_t*)p;
     p += al256(4);
     w.fb_scores = (double*)p;
+    p += al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
+    w.score_ld = score_ld_of(ix);
+    w.scores = nullptr;
+    w.cmax = nullptr;
+    if (select_uses_tc(ix, Nq)) {
+        w.scores = (__half*)p;
+        p += al256(rows * (size_t)w.score_ld * 2);
+        w.cmax = (__half*)p;
+    }
     return w;
 }
 
@@ -815,9 +1133,12 @@ static cudaError_t launch_finish_t(const IndexView& ix, int64_t n_blk, const T* 
                                    int32_t* counts, int s_max, const SelectWs& ws, cudaStream_t st)
 {
     dim3 grid((unsigned)Nq, (unsigned)ix.B);
-    select_fill_kernel<T><<<grid, FILL_THREADS, 0, st>>>(ix, n_blk, lq, pos, Nq, sp.budget,
-                                                         sp.window, sp.sinks, s_max, indices,
-                                                         counts, ws);
+    if (ws.scores)
+        select_fill_kernel<T, true><<<grid, FILL_THREADS, 0, st>>>(
+            ix, n_blk, lq, pos, Nq, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
+    else
+        select_fill_kernel<T, false><<<grid, FILL_THREADS, 0, st>>>(
+            ix, n_blk, lq, pos, Nq, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
     note_launch();
     const int64_t rows = ix.B * Nq;
     const unsigned fb_grid = (unsigned)(rows < FB_CTAS ? rows : FB_CTAS);

@@ -99,10 +99,7 @@ lsa_status check_select(const lsa_index* idx, lsa_select_params sp, int s_max)
 // The SIMT nominator keeps every eligible score in shared memory.
 constexpr int64_t SIMT_MAX_BUCKETS = (220 * 1024) / 4;
 
-bool use_tc_path(const lsa_index* idx, int64_t Nq)
-{
-    return idx->v.dtype == LSA_BF16 && Nq >= 128 && tc_scoring_available();
-}
+bool use_tc_path(const lsa_index* idx, int64_t Nq) { return select_uses_tc(idx->v, Nq); }
 
 lsa_status run_select(const lsa_index* idx, const void* lq, PosSrc pos, int64_t Nq,
                       lsa_select_params sp, int32_t* indices, int32_t* counts, int s_max, void* ws,
@@ -139,6 +136,9 @@ DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_sel
     const IndexView& v = idx->v;
     const int64_t s_max = (int64_t)sp.budget + sp.window + sp.sinks;
     DecodeLayout L;
+    // decode attends one query per sequence: each CTA gathers whole head-group
+    // rows (1 KB at Hkv=4, d=128: few large bulk copies) over one key split;
+    // a separate combine kernel merges the splits
     const int hg = attn_head_group(Hkv);
     L.n_hg = Hkv / hg;
     const int kt = attn_stage_keys(Hkv);
@@ -156,7 +156,7 @@ DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_sel
     L.indices = o; o += al256((size_t)v.B * s_max * 4);
     L.counts = o;  o += al256((size_t)v.B * 4);
     L.sel = o;     o += select_ws_bytes(v, 1);
-    L.part = o;    o += al256((size_t)v.B * ns * Hq * (d + 2) * 4);
+    L.part = o;    o += al256((size_t)v.B * ns * Hq * (d + 4) * 4);
     L.counter = o; o += al256((size_t)v.B * L.n_hg * 4);
     L.total = o;
     return L;
@@ -488,8 +488,12 @@ lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
     if (e != cudaSuccess) return cuda_fail(e, "decode select");
     const float scale = (float)(1.0 / sqrt((double)d));
     if (v.dtype == LSA_BF16)
+    {
         e = launch_attn_split(q, K, V, v.B, 1, v.T_cap, Hq, Hkv, d, indices, counts, s_max, scale,
-                              O, nullptr, v.status, L.ns, L.kps, part, counter, st);
+                              O, nullptr, v.status, L.ns, L.kps, part, nullptr, 0, st);
+        if (e == cudaSuccess && L.ns > 1)
+            e = launch_attn_combine(part, L.ns, v.B, Hq, d, O, nullptr, st);
+    }
     else
         e = launch_attn_status(q, K, V, v.dtype, v.B, 1, v.T_cap, Hq, Hkv, d, indices, counts,
                                s_max, scale, O, nullptr, v.status, st);

@@ -16,6 +16,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -102,8 +103,13 @@ struct SelectWs {
     int32_t* fb_list;    // [B*Nq]      queries that need the exact fallback
     int32_t* fb_count;   // [1]
     double* fb_scores;   // [FB_CTAS][NBK] scratch of the fallback
+    __half* scores;      // [B*Nq][score_ld] tensor-core scores (tensor-core path only)
+    __half* cmax;        // [B*Nq][score_ld/32] maximum of every 32-score chunk
+    int64_t score_ld;
 };
 constexpr int FB_CTAS = 148;
+// The tensor-core scorer serves bf16 indices and at least one 128-query tile.
+bool select_uses_tc(const IndexView& ix, int64_t Nq);
 size_t select_ws_bytes(const IndexView& ix, int64_t Nq);
 SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq);
 
@@ -127,14 +133,18 @@ cudaError_t launch_attn_status(const void* Q, const void* K, const void* V, lsa_
 cudaError_t ensure_smem_attr(const void* kernel, int bytes);
 
 // Split-KV bf16 attention: ns splits of keys_per_split keys per (row, head
-// group); part [rows][ns][Hq][d+2] and counter [rows * head groups] (zero
-// before the launch, left zero after it) are caller scratch.
+// group); part [rows][ns][Hq][d+4] and counter [rows * head groups] (zero
+// before the launch, left zero after it) are caller scratch.  hg = 1 forces
+// one KV head per CTA (smaller partials), 0 picks the default head group.
 cudaError_t launch_attn_split(const void* Q, const void* K, const void* V, int64_t B, int64_t Nq,
                               int64_t T_cap, int Hq, int Hkv, int d, const int32_t* indices,
                               const int32_t* counts, int s_max, float scale, void* O, float* lse,
                               uint32_t* status, int ns, int keys_per_split, float* part,
-                              uint32_t* counter, cudaStream_t st);
+                              uint32_t* counter, int hg, cudaStream_t st);
 int attn_stage_keys(int Hkv);
+// Merges the ns split partials of every (row, query head) into O (bf16) and lse.
+cudaError_t launch_attn_combine(const float* part, int ns, int64_t rows, int Hq, int d, void* O,
+                                float* lse, cudaStream_t st);
 int attn_head_group(int Hkv);
 
 // Decode: append + candidate nomination for one query per sequence.
