@@ -182,31 +182,38 @@ def _config(w, n_gpus):
             "parallelism": "dp%d (independent chunk per rank)" % n_gpus}
 
 
-def _attn_algorithmic_bytes(w, counts):
-    """Bytes the attention of one chunk must move: every selected K and V row
-    of every KV head, Q and O, and the index rows it reads."""
+def _attn_floor_bytes(w, indices, counts, T_cap):
+    """Compulsory bytes of one chunk's attention: every K and V row (all KV
+    heads) that at least one query selected, read once, plus Q read and O
+    written.  Counted from the chunk's selection."""
     elt = 2 if w.dtype == "bf16" else 4
-    n_sel = int(counts.sum().item())
-    kv = n_sel * w.Hkv * w.d * elt * 2
+    rows = 0
+    for b in range(w.B):
+        sel = indices[b]
+        mask = torch.zeros(T_cap, dtype=torch.bool, device=sel.device)
+        mask[sel[sel >= 0].long()] = True
+        rows += int(mask.sum().item())
+    kv = rows * w.Hkv * w.d * elt * 2
     qo = w.B * w.nq * w.Hq * w.d * elt * 2
-    idx = (n_sel + w.B * w.nq) * 4
-    return kv + qo + idx
+    gather = int(counts.sum().item()) * w.Hkv * w.d * elt * 2 + qo
+    return kv + qo, rows, gather
 
 
-def _traffic_record(kernel):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source
-    has not changed since it was captured."""
+def _traffic_record(name):
+    """DRAM bytes per call from a committed ncu summary, if none of the sources
+    it was measured with has changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        rec = json.load(f).get(kernel)
+        rec = json.load(f).get(name)
     if not rec:
         return None
-    src = os.path.join(ROOT, "long_context_indexing_b200", "csrc", rec["source"])
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    return rec if sha == rec.get("sha256") else None
+    for src, want in rec["sources"].items():
+        with open(os.path.join(ROOT, "long_context_indexing_b200", "csrc", src), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != want:
+                return None
+    return rec
 
 
 # --------------------------------------------------------------- the oracle --
@@ -280,7 +287,7 @@ def run_lsa(args, rank, ws):
     idx.build(inp["latent_K"], (T_old // span) * span)
     torch.cuda.synchronize()
     build_s = time.time() - t
-    ws_bytes = lsa.lsa_prefill_workspace_bytes(idx, w.nq, w.R, w.W, w.S)
+    ws_bytes = lsa.lsa_prefill_workspace_bytes(idx, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S)
     work = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     O = torch.empty_like(inp["Q"])
     stream = torch.cuda.current_stream()
@@ -307,31 +314,38 @@ def run_lsa(args, rank, ws):
     ms = _max_over_ranks(ms, ws)
     fallbacks = idx.check()
 
-    # Stage breakdown through the standalone entry points (same work, same stream).
+    # Stage breakdown: the chunk's two halves through their own entry points
+    # (same work, same stream, same workspace), and the index extension alone.
     sel_i, sel_c = lsa.prefill_selection_views(work, w.B, w.nq, w.s_max)
-    pos = torch.arange(T_old, w.T, device=dev, dtype=torch.int32).expand(w.B, w.nq).contiguous()
-    sel_ws = torch.empty(max(1, lsa._lib.lsa_select_workspace_bytes(idx.handle, w.nq)),
-                         dtype=torch.uint8, device=dev)
     stage_ms = {
         "index_extend": _events_time(lambda: idx.extend(inp["latent_K"], T_old, w.T),
                                      args.steps, stream),
-        "select": _events_time(lambda: lsa.lsa_select(idx, inp["latent_Q"], pos, w.R, w.W, w.S,
-                                                      workspace=sel_ws), args.steps, stream),
-        "sparse_attn": _events_time(lambda: lsa.lsa_sparse_attn(inp["Q"], inp["K"], inp["V"],
-                                                                sel_i, sel_c, out=O),
-                                    args.steps, stream),
+        "extend_and_select": _events_time(
+            lambda: lsa.lsa_prefill_select(idx, inp["latent_K"], inp["latent_Q"], T_old, w.T,
+                                           w.Hq, w.Hkv, w.d, w.R, w.W, w.S, work),
+            args.steps, stream),
+        "attend": _events_time(
+            lambda: lsa.lsa_prefill_attend(idx, inp["Q"], inp["K"], inp["V"], T_old, w.T, w.R,
+                                           w.W, w.S, work, out=O),
+            args.steps, stream),
     }
-    attn_ms = _max_over_ranks(stage_ms["sparse_attn"], ws)
+    attn_ms = _max_over_ranks(stage_ms["attend"], ws)
     peaks, peak_src = _peaks()
-    alg = _attn_algorithmic_bytes(w, sel_c)
-    achieved = alg / (attn_ms * 1e-3) / 1e9
-    traffic = _traffic_record("attn_bf16_kernel")
-    roofline = {"kernel": "attn_bf16_kernel", "bound": "hbm", "achieved": round(achieved, 1),
+    floor, uniq_rows, gather = _attn_floor_bytes(w, sel_i, sel_c, w.T)
+    achieved = floor / (attn_ms * 1e-3) / 1e9
+    bucket = w.dtype == "bf16"
+    traffic = _traffic_record("prefill_attend_" + args.workload)
+    roofline = {"kernel": ("lsa_prefill_attend: bucket_attn_kernel + plan, scatter, merge"
+                           if bucket else "lsa_prefill_attend: attn_f32_kernel"),
+                "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": "%s (copy bandwidth)" % peak_src,
-                "algorithmic_bytes_per_launch": alg,
-                "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
+                "algorithmic_bytes_per_launch": floor,
+                "algorithmic_bytes": "compulsory floor: %d distinct selected K/V rows x Hkv x d "
+                                     "x 2 B x 2, plus Q and O" % uniq_rows,
+                "per_query_gather_bytes": gather,
+                "traffic": traffic["dram_bytes_per_call"] if traffic else None,
                 "launch_ms": round(attn_ms, 4)}
 
     # End to end through the C-ABI with host buffers: H2D of the step's inputs
@@ -372,7 +386,7 @@ def run_lsa(args, rank, ws):
 
     decode = None
     if not args.no_decode:
-        del inp, idx, work, O, sel_ws, h, hq, hO
+        del inp, idx, work, O, h, hq, hO, sel_i, sel_c
         torch.cuda.empty_cache()
         decode = run_decode(args, peaks, peak_src, ws)
 

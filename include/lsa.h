@@ -230,19 +230,65 @@ lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtyp
  * Fused entries
  * ------------------------------------------------------------------------- */
 
-/* Workspace bytes for lsa_prefill_chunk with Nq = T_new - T_old queries. */
-size_t lsa_prefill_workspace_bytes(const lsa_index* idx, int64_t Nq, lsa_select_params sp);
+/* Recommended workspace bytes for lsa_prefill_chunk with Nq = T_new - T_old
+ * queries of Hq query heads, Hkv KV heads and head size d (0 on bad
+ * arguments).  For a bf16 index it includes the bucket-major attention lists
+ * with room for the chunk's expected softmax partials: about
+ * 1.5 * budget / (p * block / n_buckets) + 2 slots of Hq * (d + 4) floats per
+ * query (14.4 GB for 32768 queries, Hq = 32, d = 128, budget 4096, 256-key
+ * buckets).  A smaller workspace also works; see lsa_prefill_partial_slots. */
+size_t lsa_prefill_workspace_bytes(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d,
+                                   lsa_select_params sp);
+
+/* Softmax partial slots that a workspace of ws_bytes gives lsa_prefill_chunk
+ * (this library's own quantity; the pages have no counterpart): -1 when
+ * ws_bytes is below the minimum, 0 for the fp32 path or a minimal bf16
+ * workspace.  Each query row of a bf16 chunk needs (buckets it took + 1) slots;
+ * rows that find no free slot are attended key by key instead, which gives
+ * the same result up to fp32 summation order, only slower. */
+int64_t lsa_prefill_partial_slots(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d,
+                                  lsa_select_params sp, size_t ws_bytes);
 
 /* One prefill chunk ("Prefrontal's ...", section "The numbers, and which ones
  * to quote": prefilling the last query chunk of a long context).  Queries are
  * the positions [T_old, T_new) of every sequence.  Steps: lsa_index_extend
  * over [T_old, T_new), selection for every chunk query, sparse attention with
  * scale 1/sqrt(d).  latent_Q [B][Nq][64], Q and O [B][Nq][Hq][d]; the caches
- * already hold keys [0, T_new).  The selection is written to the workspace. */
+ * already hold keys [0, T_new).  The selection is written to the workspace
+ * (read it back as indices [B][Nq][s_max] int32 at offset 0 and counts
+ * [B][Nq] int32 at the next 256-byte boundary).
+ * bf16 attention runs bucket-major ("Latent Sparse Attention: un indice
+ * gerarchico per contesti lunghi", paragraph on retrieval: the selected keys
+ * are whole buckets plus sinks and window): the key rows of every bucket that
+ * chunk queries took are read once per KV head for up to 16 of those queries,
+ * each query's softmax partials (one per bucket, one for sinks and window)
+ * are merged in fp32.  Rows listed as exact-selection fallbacks, or that find
+ * no partial slot, are attended key by key from their index list.
+ * ws_bytes may be anything from the minimum (lsa_prefill_partial_slots >= 0)
+ * up; less than that returns LSA_ERR_WORKSPACE. */
 lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* latent_Q,
                              const void* Q, const void* K, const void* V, int64_t T_old,
                              int64_t T_new, int Hq, int Hkv, int d, lsa_select_params sp,
                              void* workspace, size_t ws_bytes, void* O, void* stream);
+
+/* The two halves of lsa_prefill_chunk, for callers that overlap or time them
+ * separately (this library's split; the pages describe the chunk as one
+ * step).  lsa_prefill_select extends the index over [T_old, T_new) and
+ * selects for every chunk query, leaving the selection and (bf16) the bucket
+ * lists in the workspace.  lsa_prefill_attend then attends from that
+ * workspace into O; it must get the same T_old, T_new, Hq, Hkv, d, sp,
+ * workspace and ws_bytes, and the caches must hold keys [0, T_new).  It
+ * changes only the attention part of the workspace, so it may be repeated.
+ * Both check every argument before any launch and fail like
+ * lsa_prefill_chunk. */
+lsa_status lsa_prefill_select(lsa_index* idx, const void* latent_K, const void* latent_Q,
+                              int64_t T_old, int64_t T_new, int Hq, int Hkv, int d,
+                              lsa_select_params sp, void* workspace, size_t ws_bytes,
+                              void* stream);
+lsa_status lsa_prefill_attend(const lsa_index* idx, const void* Q, const void* K, const void* V,
+                              int64_t T_old, int64_t T_new, int Hq, int Hkv, int d,
+                              lsa_select_params sp, void* workspace, size_t ws_bytes, void* O,
+                              void* stream);
 
 /* Workspace bytes for lsa_decode_step (depends on the device's SM count). */
 size_t lsa_decode_workspace_bytes(const lsa_index* idx, int Hq, int Hkv, int d,

@@ -19,6 +19,7 @@ import torch
 __all__ = [
     "LsaError", "LsaIndex", "lsa_index_bytes", "lsa_build_index", "lsa_select",
     "lsa_sparse_attn", "lsa_prefill_chunk", "lsa_prefill_workspace_bytes",
+    "lsa_prefill_partial_slots", "lsa_prefill_select", "lsa_prefill_attend",
     "lsa_decode_workspace_bytes", "lsa_decode_step", "lsa_select_noalloc", "library_path", "kernel_launches", "F32",
     "BF16",
 ]
@@ -65,9 +66,12 @@ def _declare(lib):
         "lsa_select_workspace_bytes": ([P, I64], SZ),
         "lsa_select": ([P, P, P, I64, SelectParams, P, P, I, P, SZ, P], I),
         "lsa_sparse_attn": ([P, P, P, I, I64, I64, I64, I, I, I, P, P, I, F, P, P, P], I),
-        "lsa_prefill_workspace_bytes": ([P, I64, SelectParams], SZ),
+        "lsa_prefill_workspace_bytes": ([P, I64, I, I, I, SelectParams], SZ),
+        "lsa_prefill_partial_slots": ([P, I64, I, I, I, SelectParams, SZ], I64),
         "lsa_prefill_chunk": ([P, P, P, P, P, P, I64, I64, I, I, I, SelectParams, P, SZ, P, P],
                               I),
+        "lsa_prefill_select": ([P, P, P, I64, I64, I, I, I, SelectParams, P, SZ, P], I),
+        "lsa_prefill_attend": ([P, P, P, P, I64, I64, I, I, I, SelectParams, P, SZ, P, P], I),
         "lsa_decode_workspace_bytes": ([P, I, I, I, SelectParams], SZ),
         "lsa_select_noalloc": ([P, P, P, I64, SelectParams, P, P, I, P], I),
         "lsa_decode_step": ([P, P, P, P, P, P, P, P, P, P, I, I, I, SelectParams, P, SZ, P, P], I),
@@ -272,9 +276,19 @@ def lsa_sparse_attn(Q, K, V, indices, counts, scale=None, return_lse=False, out=
     return (O, lse) if return_lse else O
 
 
-def lsa_prefill_workspace_bytes(index, Nq, budget, window, sinks):
-    return int(_lib.lsa_prefill_workspace_bytes(index.handle, Nq,
-                                                SelectParams(budget, window, sinks)))
+def lsa_prefill_workspace_bytes(index, Nq, Hq, Hkv, d, budget, window, sinks):
+    """Recommended workspace bytes of lsa_prefill_chunk."""
+    n = int(_lib.lsa_prefill_workspace_bytes(index.handle, Nq, Hq, Hkv, d,
+                                             SelectParams(budget, window, sinks)))
+    if n == 0:
+        raise LsaError(1, "bad arguments")
+    return n
+
+
+def lsa_prefill_partial_slots(index, Nq, Hq, Hkv, d, budget, window, sinks, ws_bytes):
+    """Softmax partial slots a workspace of ws_bytes gives (-1: below the minimum)."""
+    return int(_lib.lsa_prefill_partial_slots(index.handle, Nq, Hq, Hkv, d,
+                                              SelectParams(budget, window, sinks), ws_bytes))
 
 
 def lsa_prefill_chunk(index, latent_K, latent_Q, Q, K, V, T_old, T_new, budget, window, sinks,
@@ -286,14 +300,36 @@ def lsa_prefill_chunk(index, latent_K, latent_Q, Q, K, V, T_old, T_new, budget, 
     _cuda(latent_K, latent_Q, Q, K, V, out)
     B, Nq, Hq, d = Q.shape
     Hkv = K.shape[2]
-    need = lsa_prefill_workspace_bytes(index, Nq, budget, window, sinks)
-    if workspace is None or workspace.numel() < need:
+    if workspace is None:
+        need = lsa_prefill_workspace_bytes(index, Nq, Hq, Hkv, d, budget, window, sinks)
         workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
     O = out if out is not None else torch.empty_like(Q)
     _check(_lib.lsa_prefill_chunk(index.handle, _ptr(latent_K), _ptr(latent_Q), _ptr(Q), _ptr(K),
                                   _ptr(V), int(T_old), int(T_new), Hq, Hkv, d,
                                   SelectParams(budget, window, sinks), _ptr(workspace),
                                   workspace.numel(), _ptr(O), _stream(stream)))
+    return O
+
+
+def lsa_prefill_select(index, latent_K, latent_Q, T_old, T_new, Hq, Hkv, d, budget, window,
+                       sinks, workspace, stream=None):
+    """First half of a prefill chunk: index extension and selection into `workspace`."""
+    _cuda(latent_K, latent_Q, workspace)
+    _check(_lib.lsa_prefill_select(index.handle, _ptr(latent_K), _ptr(latent_Q), int(T_old),
+                                   int(T_new), Hq, Hkv, d, SelectParams(budget, window, sinks),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def lsa_prefill_attend(index, Q, K, V, T_old, T_new, budget, window, sinks, workspace, out=None,
+                       stream=None):
+    """Second half of a prefill chunk: attention from the selection in `workspace`."""
+    _cuda(Q, K, V, workspace, out)
+    B, Nq, Hq, d = Q.shape
+    Hkv = K.shape[2]
+    O = out if out is not None else torch.empty_like(Q)
+    _check(_lib.lsa_prefill_attend(index.handle, _ptr(Q), _ptr(K), _ptr(V), int(T_old),
+                                   int(T_new), Hq, Hkv, d, SelectParams(budget, window, sinks),
+                                   _ptr(workspace), workspace.numel(), _ptr(O), _stream(stream)))
     return O
 
 

@@ -192,6 +192,8 @@ struct SplitKV {
     int keys_per_split;  // multiple of the stage size
     float* part;         // [rows][ns][Hq][D + 4]  (acc[D], max, sum, pad)
     uint32_t* counter;   // [rows * n_hgroups], zero before the launch
+    const int32_t* row_list;   // optional: CTA i serves row row_list[i] ...
+    const int32_t* row_count;  // ... for i < *row_count (the rest exit)
 };
 
 template <int D, int HG, int STAGES>
@@ -211,7 +213,11 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
     const int n_hg = Hkv / HG;
     const int64_t unit = blockIdx.x / sk.ns;        // (row, head group)
     const int split = blockIdx.x % sk.ns;
-    const int64_t row = unit / n_hg;
+    int64_t row = unit / n_hg;
+    if (sk.row_list) {
+        if (row >= *sk.row_count) return;   // the whole CTA leaves before any barrier
+        row = sk.row_list[row];
+    }
     const int g0 = (int)(unit % n_hg) * HG;           // first KV head of the group
     const int64_t b = row / Nq;
     const int32_t* idx = indices + row * (int64_t)s_max;
@@ -663,6 +669,21 @@ cudaError_t launch_attn_split(const void* Q, const void* K, const void* V, int64
                                   O, lse, status, sk, hg, st);
     return launch_bf16_d<64>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale, O, lse,
                              status, sk, hg, st);
+}
+
+cudaError_t launch_attn_rows(const void* Q, const void* K, const void* V, int64_t B, int64_t Nq,
+                             int64_t T_cap, int Hq, int Hkv, int d, const int32_t* indices,
+                             const int32_t* counts, int s_max, float scale, void* O,
+                             uint32_t* status, const int32_t* row_list, const int32_t* row_count,
+                             cudaStream_t st)
+{
+    if (B * Nq == 0) return cudaSuccess;
+    SplitKV sk{1, s_max, nullptr, nullptr, row_list, row_count};
+    if (d == 128)
+        return launch_bf16_d<128>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale,
+                                  O, nullptr, status, sk, 0, st);
+    return launch_bf16_d<64>(Q, K, V, B, Nq, T_cap, Hq, Hkv, indices, counts, s_max, scale, O,
+                             nullptr, status, sk, 0, st);
 }
 
 cudaError_t launch_attn_status(const void* Q, const void* K, const void* V, lsa_dtype dt, int64_t B,

@@ -1,0 +1,562 @@
+// k_attn_bucket_tc.cu -- bucket-major attention tiles on the 5th-generation
+// tensor cores (tcgen05 MMA with TMEM accumulators; sm_100a).
+//
+// Same tiles and results as bucket_attn_kernel (k_attn_bucket.cu; method
+// citations there): a tile is one bucket, or one run of consecutive queries'
+// sinks and windows, with up to 16 queries and one KV head.  Here the tile's
+// 16 queries x 8 query heads are the 128 rows of one MMA (a row per TMEM
+// lane), and the tile's keys stream through in 64-key stages:
+//
+//   S  = Q K^T   M = 128, N = 64 keys, K = d      (TMEM, double-buffered)
+//   P  = exp2(S * scale * log2 e - m)            (softmax warps, bf16 to smem)
+//   O += P V     M = 128, N = d, K = 64 keys      (TMEM, one accumulator)
+//
+// Warp roles (8 warps):
+//   warp 0     planner: claims work items and copies each tile's description
+//              (written by bucket_tile_records_kernel) and the bucket's member
+//              lists into shared memory, one item ahead;
+//   warps 1-2  loaders: gather the tile's Q rows and every stage's K and V rows
+//              of the KV head with 16-byte cp.async into 128-byte-swizzled
+//              planes (the layout the MMA descriptors name); completion lands
+//              on mbarriers;
+//   warp 3     allocates TMEM; lane 0 issues all MMAs and commits;
+//   warps 4-7  softmax: thread = row = TMEM lane; reads its 64 scores of a
+//              stage, masks keys outside its query's ranges, keeps the
+//              running max (raised lazily: O and the sum are rescaled only
+//              when the max grows by more than 2^8), writes its P row, and at
+//              the end of the tile writes the row's partial (acc, max, sum).
+// Q and tile descriptions are double-buffered across work items and the K/V
+// ring continues across them, so loads of the next tile overlap this one.
+// Every wait is bounded; on a timeout the CTA records DEV_TIMEOUT, all roles
+// leave, outstanding copies and MMAs are waited for, and TMEM is freed.
+#include <limits.h>
+#include <math.h>
+
+#include "attn_bucket.cuh"
+#include "lsa_internal.cuh"
+#include "ptx.cuh"
+
+namespace lsa {
+
+constexpr int TB_M = 128;            // MMA rows: BA_Q queries x 8 query heads
+constexpr int TB_N = 64;             // keys per stage
+constexpr int TB_NS = 3;             // K/V stages in the ring
+constexpr int TB_OPEN_MAX = 2048;    // open-block members one tile can hold
+constexpr int TB_THREADS = 256;      // 8 warps
+constexpr uint32_t TB_WAIT = 1u << 22;
+
+template <int D>
+struct TbCfg {
+    static constexpr int CH = D / 8;                    // 16-byte chunks per row
+    static constexpr int Q_PLANE = TB_M * 128;          // 64 dims of 128 rows
+    static constexpr int Q_BYTES = (D / 64) * Q_PLANE;
+    static constexpr int KV_PLANE = TB_N * 128;         // 64 dims of 64 keys
+    static constexpr int K_BYTES = (D / 64) * KV_PLANE;
+    static constexpr int STAGE = 2 * K_BYTES;           // K then V
+    static constexpr int P_BYTES = TB_M * TB_N * 2;
+    static constexpr int OFF_Q = 0;                     // two buffers
+    static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
+    static constexpr int OFF_P = OFF_KV + TB_NS * STAGE;
+    static constexpr int OFF_OPEN = OFF_P + P_BYTES;    // two open-member lists
+    static constexpr int OFF_MEM = OFF_OPEN + 2 * TB_OPEN_MAX * 4;   // two closed-member lists
+    static constexpr int OFF_BAR = OFF_MEM + 2 * TB_OPEN_MAX * 4;
+    static constexpr int NBAR = 16 + 2 * TB_NS;
+    static constexpr int BYTES = OFF_BAR + NBAR * 8 + 1024;   // + alignment slack
+    static constexpr uint32_t KSTEPS = D / 16;
+    // kind::f16, fp32 accumulate, bf16 A and B, M = 128
+    static constexpr uint32_t IDESC_S =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TB_N >> 3) << 17) | ((uint32_t)(TB_M >> 4) << 24);
+    static constexpr uint32_t IDESC_PV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) /* B MN-major */ |
+                                         ((uint32_t)(D >> 3) << 17) | ((uint32_t)(TB_M >> 4) << 24);
+};
+
+// ---- tcgen05 wrappers --------------------------------------------------------
+__device__ __forceinline__ uint64_t tb_desc(uint32_t smem_addr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) /* tcgen05 descriptor */ |
+           (2ull << 61) /* 128-byte swizzle */;
+}
+
+__device__ __forceinline__ void tb_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void tb_commit(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     ptx::smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tb_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tb_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tb_ld32(uint32_t taddr, float* v)
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+        "%29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+__device__ __forceinline__ void tb_st32(uint32_t taddr, const float* v)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
+{
+    using C = TbCfg<D>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* info_full = bars;          // [2]
+    uint64_t* info_empty = bars + 2;     // [2]
+    uint64_t* q_full = bars + 4;         // [2]
+    uint64_t* q_empty = bars + 6;        // [2]
+    uint64_t* s_full = bars + 8;         // [2]
+    uint64_t* s_empty = bars + 10;       // [2]
+    uint64_t* p_full = bars + 12;
+    uint64_t* p_empty = bars + 13;
+    uint64_t* o_full = bars + 14;
+    uint64_t* o_empty = bars + 15;
+    uint64_t* kv_full = bars + 16;       // [TB_NS]
+    uint64_t* kv_empty = kv_full + TB_NS;
+    __shared__ TileInfo ti[2];
+    __shared__ uint32_t tmem_slot;
+    __shared__ volatile int abort_flag;
+    __shared__ int cnt_s[1];
+    __shared__ uint64_t fin_bar;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const IndexView& ix = a.ix;
+    const int p = ix.p;
+    const int lp = ((p & (p - 1)) == 0) ? __ffs(p) - 1 : -1;
+    const int64_t n_work = (a.n_wt + a.P.ctr[CTR_TILES]) * a.Hkv;
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&info_full[i], 1);
+            ptx::mbar_init(&info_empty[i], 7);     // 4 softmax warps, the MMA thread, 2 loader warps
+            ptx::mbar_init(&q_full[i], 64);        // every producer thread's cp.async arrival
+            ptx::mbar_init(&q_empty[i], 1);
+            ptx::mbar_init(&s_full[i], 1);
+            ptx::mbar_init(&s_empty[i], 4);
+        }
+        ptx::mbar_init(p_full, 4);
+        ptx::mbar_init(p_empty, 1);
+        ptx::mbar_init(o_full, 1);
+        ptx::mbar_init(o_empty, 4);
+        for (int s = 0; s < TB_NS; ++s) {
+            ptx::mbar_init(&kv_full[s], 64);
+            ptx::mbar_init(&kv_empty[s], 1);
+        }
+        ptx::mbar_init(&fin_bar, 1);
+        abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 3) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+                         ptx::smem_addr(&tmem_slot))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tb_fence_before();
+    __syncthreads();
+    tb_fence_after();
+    const uint32_t tmem = tmem_slot;
+
+    // Bounded waits.  wait1: one thread.  waitw: every lane of a warp polls
+    // (each gets the barrier's acquire) and the warp agrees on the outcome,
+    // so that warp-collective instructions after it are never divergent.
+    auto fail = [&](uint32_t where) {
+        abort_flag = 1;
+        dev_error(ix.status, DEV_TIMEOUT, where);
+    };
+    auto wait1 = [&](uint64_t* bar, uint32_t parity, uint32_t where) -> bool {
+        if (abort_flag) return false;
+        if (ptx::mbar_wait_bounded(bar, parity, TB_WAIT)) return true;
+        fail(where);
+        return false;
+    };
+    auto waitw = [&](uint64_t* bar, uint32_t parity, uint32_t where) -> bool {
+        bool ok = !abort_flag && ptx::mbar_wait_bounded(bar, parity, TB_WAIT);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok && lane == 0) fail(where);
+        return ok;
+    };
+
+    if (warp == 0) {
+        // ============================ planner ============================
+        // Claims work items and brings each tile's description and member
+        // lists into shared memory, one item ahead of the loaders.
+        int w_next = 0;
+        if (lane == 0) w_next = atomicAdd(a.P.ctr + CTR_WORK, 1);
+        const TileInfo* recs = reinterpret_cast<const TileInfo*>(a.P.recs);
+        for (int i = 0;; ++i) {
+            const int ib = i & 1;
+            const uint32_t iph = (uint32_t)((i >> 1) & 1);
+            TileInfo& T = ti[ib];
+            if (!waitw(&info_empty[ib], iph ^ 1u, 100u)) break;
+            const int64_t w = __shfl_sync(0xffffffffu, w_next, 0);
+            if (lane == 0) w_next = atomicAdd(a.P.ctr + CTR_WORK, 1);
+            if (w >= n_work) {
+                if (lane == 0) {
+                    T.n_st = -1;
+                    ptx::mbar_arrive(&info_full[ib]);
+                }
+                break;
+            }
+            const int64_t t = w / a.Hkv;
+            {
+                const uint4* src = reinterpret_cast<const uint4*>(recs + t);
+                uint4* dst = reinterpret_cast<uint4*>(&T);
+                for (int x = lane; x < TILE_REC_BYTES / 16; x += 32) dst[x] = src[x];
+            }
+            __syncwarp();
+            if (lane == 0) T.h = (int)(w % a.Hkv);
+            if (T.kind == 1) {
+                int32_t* mem_l = reinterpret_cast<int32_t*>(smem + C::OFF_MEM) + ib * TB_OPEN_MAX;
+                const int32_t* mem_g = ix.members + T.b * ix.NP + T.o0;
+                for (int x = lane; x < T.nclosed / p; x += 32) mem_l[x] = mem_g[x];
+                if (T.any_open) {
+                    int32_t* open_l = reinterpret_cast<int32_t*>(smem + C::OFF_OPEN) + ib * TB_OPEN_MAX;
+                    ba_open_list(ix, a.n_blk, T.b, T.g, lane, 32, cnt_s, open_l, [] { __syncwarp(); });
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&info_full[ib]);
+        }
+    } else if (warp < 3) {
+        // ============================ loaders ============================
+        // Gather the tile's Q rows and every stage's K and V rows of the KV
+        // head (tokens from the shared-memory member lists).
+        const int ltid = tid - 32;   // 0 .. 63
+        const int lw = warp - 1;
+        int64_t gs = 0;
+        for (int i = 0;; ++i) {
+            const int ib = i & 1;
+            const uint32_t iph = (uint32_t)((i >> 1) & 1);
+            const TileInfo& T = ti[ib];
+            if (!waitw(&info_full[ib], iph, 105u)) break;
+            const int n_st = T.n_st;
+            if (n_st < 0) break;
+            const int32_t* mem_l = reinterpret_cast<const int32_t*>(smem + C::OFF_MEM) + ib * TB_OPEN_MAX;
+            const int32_t* open_l = reinterpret_cast<const int32_t*>(smem + C::OFF_OPEN) + ib * TB_OPEN_MAX;
+
+            // ---- the tile's Q rows: row r = query r / hpg, head r % hpg ----
+            if (!waitw(&q_empty[ib], iph ^ 1u, 110u)) break;
+            unsigned char* qs = smem + C::OFF_Q + ib * C::Q_BYTES;
+            for (int x = ltid; x < TB_M * C::CH; x += 64) {
+                const int r = x / C::CH, c = x % C::CH;
+                const int q = r / a.hpg, hh = r % a.hpg;
+                const bool live = q < BA_Q && T.slot[q] >= 0;
+                const __nv_bfloat16* src =
+                    a.Q + ((size_t)(live ? T.row[q] : 0) * a.Hq + (size_t)T.h * a.hpg + hh) * D + c * 8;
+                unsigned char* dst = qs + (c >> 3) * C::Q_PLANE + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+                ptx::cp_async16_zfill(dst, live ? (const void*)src : (const void*)a.Q, live ? 16u : 0u);
+            }
+            ptx::cp_async_mbar_arrive(&q_full[ib]);
+
+            // ---- K / V stages ----
+            const size_t tstride = (size_t)a.Hkv * D;
+            const __nv_bfloat16* Kb = a.K + ((size_t)T.b * ix.T_cap * a.Hkv + T.h) * D;
+            const __nv_bfloat16* Vb = a.V + ((size_t)T.b * ix.T_cap * a.Hkv + T.h) * D;
+            bool stop = false;
+            for (int s = 0; s < n_st; ++s, ++gs) {
+                const int slot = (int)(gs % TB_NS);
+                if (!waitw(&kv_empty[slot], (uint32_t)(((gs / TB_NS) & 1) ^ 1), 120u)) {
+                    stop = true;
+                    break;
+                }
+                // this lane's key of the stage: one token per lane, shared by shuffles
+                int k = T.kbeg + s * TB_N + 32 * lw + lane;
+                if (k >= T.kend) k = T.kend - 1;   // padding rows repeat a real key (masked)
+                const int64_t t64 = ba_token(T, k, p, lp, mem_l, open_l);
+                int32_t tok = (int32_t)t64;
+                if (t64 < 0 || t64 >= ix.T_cap) {
+                    dev_error(ix.status, DEV_BAD_INDEX, (uint32_t)t64);
+                    tok = 0;
+                }
+                unsigned char* ks = smem + C::OFF_KV + slot * C::STAGE;
+                constexpr int KPI = 32 / C::CH;       // keys per warp instruction
+#pragma unroll 4
+                for (int j = 0; j < 32 / KPI; ++j) {
+                    const int kl = KPI * j + lane / C::CH;        // key inside this warp's 32
+                    const int c = lane % C::CH;
+                    const int32_t tk = __shfl_sync(0xffffffffu, tok, kl);
+                    const int kr = 32 * lw + kl;                  // row inside the stage
+                    const int soff = (c >> 3) * C::KV_PLANE + kr * 128 + (((c & 7) ^ (kr & 7)) << 4);
+                    const size_t goff = (size_t)tk * tstride + c * 8;
+                    ptx::cp_async16(ks + soff, Kb + goff);
+                    ptx::cp_async16(ks + C::K_BYTES + soff, Vb + goff);
+                }
+                ptx::cp_async_mbar_arrive(&kv_full[slot]);
+            }
+            if (stop) break;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&info_empty[ib]);   // done with ti[ib]
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == 3) {
+        // =========================== MMA issuer ===========================
+        if (lane == 0) {
+            int64_t gs = 0, pv = 0;
+            bool stop = false;
+            const uint32_t q_base = ptx::smem_addr(smem + C::OFF_Q);
+            const uint32_t kv_base = ptx::smem_addr(smem + C::OFF_KV);
+            const uint32_t p_base = ptx::smem_addr(smem + C::OFF_P);
+            const uint32_t t_o = tmem + 128;
+            for (int i = 0; !stop; ++i) {
+                const int ib = i & 1;
+                const uint32_t iph = (uint32_t)((i >> 1) & 1);
+                if (!wait1(&info_full[ib], iph, 200u)) break;
+                const int n_st = ti[ib].n_st;
+                ptx::mbar_arrive(&info_empty[ib]);
+                if (n_st < 0) break;
+                if (!wait1(&q_full[ib], iph, 210u)) break;
+                const uint32_t qa = q_base + ib * C::Q_BYTES;
+                int prev_slot = 0;
+                auto do_pv = [&](int s, int slot) -> bool {
+                    if (!wait1(p_full, (uint32_t)(pv & 1), 220u)) return false;
+                    if (s == 0 && !wait1(o_empty, (uint32_t)((i & 1) ^ 1), 230u)) return false;
+                    tb_fence_after();
+                    ptx::fence_proxy_async();
+                    const uint32_t va = kv_base + slot * C::STAGE + C::K_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < TB_N / 16; ++kk)
+                        tb_mma(t_o, tb_desc(p_base + kk * 32, 16, 1024),
+                               tb_desc(va + kk * 2048, C::KV_PLANE, 1024), C::IDESC_PV,
+                               (s > 0 || kk > 0) ? 1u : 0u);
+                    tb_commit(&kv_empty[slot]);
+                    tb_commit(p_empty);
+                    ++pv;
+                    return true;
+                };
+                for (int s = 0; s < n_st; ++s, ++gs) {
+                    const int slot = (int)(gs % TB_NS);
+                    const int sb = (int)(gs & 1);
+                    if (!wait1(&kv_full[slot], (uint32_t)((gs / TB_NS) & 1), 240u) ||
+                        !wait1(&s_empty[sb], (uint32_t)(((gs >> 1) & 1) ^ 1), 250u)) {
+                        stop = true;
+                        break;
+                    }
+                    tb_fence_after();
+                    ptx::fence_proxy_async();
+                    const uint32_t ka = kv_base + slot * C::STAGE;
+#pragma unroll
+                    for (int kk = 0; kk < (int)C::KSTEPS; ++kk) {
+                        const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
+                        tb_mma(tmem + sb * TB_N,
+                               tb_desc(qa + (kk >> 2) * C::Q_PLANE + off, 16, 1024),
+                               tb_desc(ka + (kk >> 2) * C::KV_PLANE + off, 16, 1024), C::IDESC_S,
+                               kk > 0 ? 1u : 0u);
+                    }
+                    tb_commit(&s_full[sb]);
+                    if (s == n_st - 1) tb_commit(&q_empty[ib]);
+                    if (s > 0 && !do_pv(s - 1, prev_slot)) {
+                        stop = true;
+                        break;
+                    }
+                    prev_slot = slot;
+                }
+                if (stop || !do_pv(n_st - 1, prev_slot)) break;
+                tb_commit(o_full);
+            }
+            // nothing of this CTA may still run on the tensor cores at exit
+            tb_commit(&fin_bar);
+            ptx::mbar_wait_bounded(&fin_bar, 0, TB_WAIT);
+        }
+    } else {
+        // ============================ softmax ============================
+        const int r = 32 * (warp & 3) + lane;               // row = TMEM lane
+        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        int64_t gs = 0, pv = 0;
+        unsigned char* prow = smem + C::OFF_P + r * 128;
+        for (int i = 0;; ++i) {
+            const int ib = i & 1;
+            const uint32_t iph = (uint32_t)((i >> 1) & 1);
+            if (!waitw(&info_full[ib], iph, 300u)) break;
+            const TileInfo& T = ti[ib];
+            const int n_st = T.n_st;
+            if (n_st < 0) {
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&info_empty[ib]);
+                break;
+            }
+            const int q = r / a.hpg, hh = r % a.hpg;
+            const bool live = q < BA_Q && T.slot[q] >= 0;
+            const QRange rg = live ? T.rng[q] : QRange{0, 0, 0, 0};
+            const int kbeg = T.kbeg;
+            float m_run = -INFINITY, l = 0.f;
+            bool stop = false;
+            for (int s = 0; s < n_st; ++s, ++gs) {
+                const int sb = (int)(gs & 1);
+                if (!waitw(&s_full[sb], (uint32_t)((gs >> 1) & 1), 310u)) {
+                    stop = true;
+                    break;
+                }
+                tb_fence_after();
+                float v[TB_N];
+                tb_ld32(tmem + lane_base + sb * TB_N, v);
+                tb_ld32(tmem + lane_base + sb * TB_N + 32, v + 32);
+                tb_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&s_empty[sb]);
+
+                const int kb = kbeg + s * TB_N;
+                const bool all_in = live && rg.covers(kb, kb + TB_N);
+                float mx = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < TB_N; ++j) {
+                    const bool ok = all_in || (live && rg.has(kb + j));
+                    v[j] = ok ? v[j] * a.scale_log2 : -INFINITY;
+                    mx = fmaxf(mx, v[j]);
+                }
+                // Lazy running max: raised only on the item's first stage, from
+                // nothing, or by more than 8 (a factor 2^8), so that O needs
+                // rescaling rarely; P stays <= 2^8.
+                bool resc = false;
+                float alpha = 1.f;
+                if (mx > m_run) {
+                    if (s == 0 || m_run == -INFINITY) {
+                        m_run = mx;
+                    } else if (mx > m_run + 8.f) {
+                        alpha = exp2f(m_run - mx);
+                        m_run = mx;
+                        resc = true;
+                    }
+                }
+                const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+                uint32_t pk[TB_N / 2];
+                float sum = 0.f;
+#pragma unroll
+                for (int j = 0; j < TB_N / 2; ++j) {
+                    const float p0 = exp2f(v[2 * j] - mu), p1 = exp2f(v[2 * j + 1] - mu);
+                    sum += p0 + p1;
+                    pk[j] = ptx::pack_bf16(p0, p1);
+                }
+                l = l * alpha + sum;
+                // the previous P has been consumed (and O is quiet) once the
+                // previous PV MMA has completed
+                if (!waitw(p_empty, (uint32_t)((pv & 1) ^ 1), 320u)) {
+                    stop = true;
+                    break;
+                }
+                if (__any_sync(0xffffffffu, resc)) {
+                    tb_fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        float o[32];
+                        tb_ld32(tmem + lane_base + 128 + c * 32, o);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) o[j] *= alpha;
+                        tb_st32(tmem + lane_base + 128 + c * 32, o);
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                ptx::fence_proxy_async();
+                tb_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(p_full);
+                ++pv;
+            }
+            if (stop) break;
+            // ---- the row's partial ----
+            if (!waitw(o_full, (uint32_t)(i & 1), 330u)) break;
+            tb_fence_after();
+            constexpr int PS = D + 4;
+            float* pp = a.P.part + (((size_t)(live ? T.slot[q] : 0) * a.Hq) + (size_t)T.h * a.hpg + hh) * PS;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                float o[32];
+                tb_ld32(tmem + lane_base + 128 + c * 32, o);
+                if (live) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        reinterpret_cast<float4*>(pp + c * 32)[j] =
+                            make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                }
+            }
+            if (live) *reinterpret_cast<float2*>(pp + D) = make_float2(m_run, l);
+            tb_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(o_empty);
+                ptx::mbar_arrive(&info_empty[ib]);
+            }
+        }
+    }
+    tb_fence_before();
+    __syncthreads();
+    if (warp == 3) {
+        tb_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem)
+                     : "memory");
+    }
+}
+
+bool bucket_attn_tc_supported(int Hq, int Hkv, int d, int G)
+{
+    return (d == 64 || d == 128) && Hq % Hkv == 0 && Hq / Hkv <= 8 && G <= TB_OPEN_MAX;
+}
+
+template <int D>
+static cudaError_t launch_tc_t(const BaArgs& a, cudaStream_t st)
+{
+    using C = TbCfg<D>;
+    auto kern = bucket_attn_tc_kernel<D>;
+    cudaError_t e = ensure_smem_attr((const void*)kern, C::BYTES);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, TB_THREADS, C::BYTES);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    kern<<<(unsigned)(sm_count() * per_sm), TB_THREADS, C::BYTES, st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bucket_attn_tc(const BaArgs& a, int d, cudaStream_t st)
+{
+    return (d == 128) ? launch_tc_t<128>(a, st) : launch_tc_t<64>(a, st);
+}
+
+}  // namespace lsa

@@ -362,7 +362,11 @@ cudaError_t launch_open_assign(const IndexView& ix, int64_t n_blk, int64_t j_end
     int64_t n_done = j_end - jo;
     if (n_done < 0) n_done = 0;
     if (n_done > ix.G) n_done = ix.G;
-    if (n_blk == 0 || n_blk >= ix.nblk_max) n_done = 0;  // nothing to assign / no open block
+    // the open block holds the pooled groups after the closed blocks, as far
+    // as the index's capacity reaches (a partial block when T_cap is not a
+    // whole number of blocks)
+    if (n_done > ix.NP - jo) n_done = ix.NP - jo;
+    if (n_blk == 0 || n_done < 0) n_done = 0;
     open_assign_kernel<<<dim3((unsigned)ix.G, (unsigned)ix.B), 256, 0, st>>>(ix, n_blk, n_done);
     note_launch();
     return cudaGetLastError();

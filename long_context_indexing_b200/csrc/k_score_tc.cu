@@ -145,6 +145,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
     const int64_t b = blockIdx.y;
     const int64_t q0 = (int64_t)blockIdx.x * TC_M;
     if (blockIdx.x == 0 && b == 0 && threadIdx.x == 0) *ws.fb_count = 0;
+    {
+        const int64_t cta = b * gridDim.x + blockIdx.x;
+        for (int64_t x = cta * blockDim.x + threadIdx.x; x < ws.plan.n_zero;
+             x += (int64_t)gridDim.x * gridDim.y * blockDim.x)
+            ws.plan.zero[x] = 0;
+    }
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(q_full, 1);

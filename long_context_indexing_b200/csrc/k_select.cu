@@ -304,6 +304,9 @@ __global__ void __launch_bounds__(SIMT_THREADS) score_topk_simt_kernel(IndexView
     const int64_t b = blockIdx.y, i = blockIdx.x;
     const int64_t row = b * Nq + i;
     if (row == 0 && threadIdx.x == 0) *ws.fb_count = 0;
+    for (int64_t x = row * blockDim.x + threadIdx.x; x < ws.plan.n_zero;
+         x += (int64_t)Nq * gridDim.y * blockDim.x)
+        ws.plan.zero[x] = 0;
     load_query(q_s, lq, row);
     __syncthreads();
     simt_nominate(ix, n_blk, q_s, b, row, pos.at(b, Nq, i), W, ws, sc);
@@ -322,8 +325,9 @@ struct FillCtx {
     bool open_live; // the open block has keys at or below hi
 };
 
-// Warp-cooperative count of available keys of bucket g.
-__device__ int64_t warp_avail(const FillCtx& f, int64_t g)
+// Warp-cooperative count of available keys of bucket g (closed members plus
+// open-block members); *closed_out, when given, receives the closed part.
+__device__ int64_t warp_avail(const FillCtx& f, int64_t g, int64_t* closed_out = nullptr)
 {
     const int lane = threadIdx.x & 31;
     const IndexView& ix = f.ix;
@@ -343,6 +347,7 @@ __device__ int64_t warp_avail(const FillCtx& f, int64_t g)
         for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
         a = c;
     }
+    if (closed_out) *closed_out = a;
     if (f.open_live) {
         const int32_t* open = ix.open_bucket + f.bseq * ix.G;
         const int64_t j0 = f.n_blk * ix.G;
@@ -353,6 +358,58 @@ __device__ int64_t warp_avail(const FillCtx& f, int64_t g)
         a += c;
     }
     return a;
+}
+
+// Closed keys of bucket g below the first sink-free position S: they open the
+// bucket's ascending key list (only block 0 can hold any).
+__device__ int64_t keys_below_sinks(const FillCtx& f, int64_t g)
+{
+    const IndexView& ix = f.ix;
+    const int p = ix.p;
+    const int64_t span = (int64_t)p * ix.G;
+    if ((g / ix.k) * span >= f.S) return 0;
+    const int32_t* off = ix.offsets + f.bseq * (ix.NBK + 1);
+    const int32_t* mem = ix.members + f.bseq * ix.NP;
+    int64_t n = 0;
+    for (int32_t x = off[g]; x < off[g + 1]; ++x) {
+        const int64_t lo = (int64_t)mem[x] * p;
+        if (lo >= f.S) break;
+        n += (f.S - lo < p) ? f.S - lo : p;
+    }
+    return n;
+}
+
+// Lists a row for bucket-major attention: reserves nt + 1 partial slots and
+// records every taken bucket as the range [lo, hi) of its closed key list
+// plus the count of open-block keys taken after it.  Rows that find no room
+// become gather rows.  Called by every thread of the fill CTA.
+__device__ void plan_list_row(const BucketPlan& P, int64_t row, int64_t bseq, int64_t NBK, int nt,
+                              const int* take_g, const int64_t* take_n, const int64_t* take_lo,
+                              const int64_t* take_closed, int* sh_base)
+{
+    if (threadIdx.x == 0) {
+        int base = atomicAdd(P.ctr + CTR_RESERVED, nt + 1);
+        if ((int64_t)base + nt + 1 > P.ent_cap) {
+            base = -1;
+            P.gather_rows[atomicAdd(P.ctr + CTR_GATHER, 1)] = (int32_t)row;
+        } else {
+            atomicMax(P.ctr + CTR_VALID_END, base + nt + 1);
+            P.ent[base + nt] = make_int4((int)row, -1, 0, 0);   // sinks + window slot
+        }
+        P.row_n[row] = (base < 0) ? -1 : nt;
+        P.row_base[row] = base;
+        *sh_base = base;
+    }
+    __syncthreads();
+    const int base = *sh_base;
+    if (base < 0) return;
+    for (int t = threadIdx.x; t < nt; t += blockDim.x) {
+        const int64_t gg = bseq * NBK + take_g[t];
+        const int64_t closed = (take_n[t] < take_closed[t]) ? take_n[t] : take_closed[t];
+        const int rank = atomicAdd(P.bucket_cnt + gg, 1);
+        P.ent[base + t] = make_int4((int)row, (int)gg, (int)take_lo[t], (int)(take_lo[t] + closed));
+        P.ent2[base + t] = make_int2(rank, (int)(take_n[t] - closed));
+    }
 }
 
 __device__ void warp_emit_partial(const FillCtx& f, int64_t g, int64_t take, int32_t* out);
@@ -377,7 +434,7 @@ __device__ void cta_emit(const FillCtx& f, int64_t g, int64_t take, int32_t* out
     const int64_t span = (int64_t)p * ix.G;
     const int64_t blk = g / ix.k;
     const int64_t bstart = blk * span, bend = bstart + span;
-    const int32_t o0 = off[g], o1 = off[g + 1];
+    const int32_t o0 = off[g];
     const bool full = (bstart >= f.S && bend - 1 <= f.hi) && !f.open_live;
     if (full) {
         for (int64_t x = threadIdx.x; x < take; x += blockDim.x)
@@ -638,8 +695,11 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     __shared__ double es[KC];
     __shared__ int order[KC];
     __shared__ int64_t av[KC];
+    __shared__ int64_t avc[KC];          // closed part of av
     __shared__ int take_g[KC];
     __shared__ int64_t take_n[KC];
+    __shared__ int64_t take_closed[KC];  // its available closed keys
+    __shared__ int64_t take_lo[KC];      // its closed keys below the sinks bound
     __shared__ int64_t take_off[KC];     // output offset of each taken bucket
     __shared__ int32_t take_o0[KC];      // its first CSR position
     __shared__ int take_full[KC];
@@ -688,7 +748,7 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     f.pos = pq;
     f.hi = pq - W;
     f.S = S;
-    f.open_live = (n_blk < ix.nblk_max) && (n_blk > 0) && (n_blk * (int64_t)ix.p * ix.G <= f.hi);
+    f.open_live = (n_blk * ix.G < ix.NP) && (n_blk > 0) && (n_blk * (int64_t)ix.p * ix.G <= f.hi);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     __shared__ int slow[KC];
     __shared__ int n_slow;
@@ -702,6 +762,7 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
         if (bucket_full(f, g)) {
             const int32_t* off = ix.offsets + b * (ix.NBK + 1);
             av[c] = (int64_t)(off[g + 1] - off[g]) * ix.p;
+            avc[c] = av[c];
         } else {
             slow[atomicAdd(&n_slow, 1)] = c;
         }
@@ -709,8 +770,12 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     __syncthreads();
     for (int e = warp; e < n_slow; e += FILL_THREADS / 32) {
         const int c = slow[e];
-        const int64_t a = warp_avail(f, cg[c]);
-        if (lane == 0) av[c] = a;
+        int64_t closed;
+        const int64_t a = warp_avail(f, cg[c], &closed);
+        if (lane == 0) {
+            av[c] = a;
+            avc[c] = closed;
+        }
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -723,6 +788,7 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
             const int64_t t = (a <= rem) ? a : rem;
             take_g[nt] = cg[c];
             take_n[nt] = t;
+            take_closed[nt] = avc[c];
             take_off[nt] = (int64_t)R - rem;
             ++nt;
             rem -= t;
@@ -748,6 +814,11 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
             const int slot = atomicAdd(ws.fb_count, 1);
             ws.fb_list[slot] = (int32_t)row;
             atomicAdd(ix.status + 1, 1u);
+            if (ws.plan.row_n) {   // the fallback's selection is attended key by key
+                ws.plan.row_n[row] = -1;
+                ws.plan.row_base[row] = -1;
+                ws.plan.gather_rows[atomicAdd(ws.plan.ctr + CTR_GATHER, 1)] = (int32_t)row;
+            }
         }
         return;
     }
@@ -760,8 +831,13 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     for (int t = threadIdx.x; t < nt; t += FILL_THREADS) {
         take_full[t] = bucket_full(f, take_g[t]) ? 1 : 0;
         take_o0[t] = offs[take_g[t]];
+        take_lo[t] = take_full[t] ? 0 : keys_below_sinks(f, take_g[t]);
     }
     __syncthreads();
+    if (ws.plan.row_n) {
+        __shared__ int sh_base;
+        plan_list_row(ws.plan, row, b, ix.NBK, nt, take_g, take_n, take_lo, take_closed, &sh_base);
+    }
     const int64_t n_lr = nt ? take_off[nt - 1] + take_n[nt - 1] : 0;
     // Whole-member buckets: every long-range slot independently (a binary
     // search finds its bucket), so all member reads are in flight at once.
@@ -842,7 +918,7 @@ __global__ void __launch_bounds__(FB_THREADS) select_fallback_kernel(IndexView i
         f.pos = pq;
         f.hi = pq - W;
         f.S = S;
-        f.open_live = (n_blk < ix.nblk_max) && (n_blk > 0) && (n_blk * (int64_t)ix.p * ix.G <= f.hi);
+        f.open_live = (n_blk * ix.G < ix.NP) && (n_blk > 0) && (n_blk * (int64_t)ix.p * ix.G <= f.hi);
         int32_t* out = indices + row * (int64_t)s_max;
         const int64_t n_s = (S < pq + 1) ? S : pq + 1;
         for (int64_t x = threadIdx.x; x < n_s; x += FB_THREADS) out[x] = (int32_t)x;
@@ -953,7 +1029,7 @@ __global__ void __launch_bounds__(SIMT_THREADS) decode_prep_kernel(
     if ((pq + 1) % p != 0) return;
     const int64_t j = (pq + 1) / p - 1;
     const int64_t o = j - n_blk * ix.G;
-    if (n_blk < 1 || o < 0 || o >= ix.G || n_blk >= ix.nblk_max) {
+    if (n_blk < 1 || o < 0 || o >= ix.G || j >= ix.NP) {
         if (threadIdx.x == 0) dev_error(ix.status, DEV_OPEN_FULL, (uint32_t)b);
         return;
     }
@@ -1113,6 +1189,7 @@ SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
     w.fb_scores = (double*)p;
     p += al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
     w.score_ld = score_ld_of(ix);
+    w.plan = BucketPlan{};
     w.scores = nullptr;
     w.cmax = nullptr;
     if (select_uses_tc(ix, Nq)) {

@@ -103,17 +103,93 @@ bool use_tc_path(const lsa_index* idx, int64_t Nq) { return select_uses_tc(idx->
 
 lsa_status run_select(const lsa_index* idx, const void* lq, PosSrc pos, int64_t Nq,
                       lsa_select_params sp, int32_t* indices, int32_t* counts, int s_max, void* ws,
-                      cudaStream_t st)
+                      cudaStream_t st, const BucketPlan* plan = nullptr)
 {
     const bool tc = use_tc_path(idx, Nq);
     if (!tc && idx->n_blk * idx->v.k > SIMT_MAX_BUCKETS)
         return fail(LSA_ERR_UNSUPPORTED, "%lld buckets exceed the SIMT scorer's %lld",
                     (long long)(idx->n_blk * idx->v.k), (long long)SIMT_MAX_BUCKETS);
     SelectWs w = select_ws_carve(ws, idx->v, Nq);
+    if (plan) w.plan = *plan;
     cudaError_t e = launch_select(idx->v, idx->n_blk, lq, pos, Nq, sp, indices, counts, s_max, w,
                                   tc, st);
     if (e != cudaSuccess) return cuda_fail(e, "select");
     return LSA_OK;
+}
+
+// Prefill workspace: selection output and scratch, then (bf16 with a
+// supported head shape) the bucket-major attention lists with ent_cap
+// partial slots of Hq * (d + 4) floats each.
+struct PrefillLayout {
+    size_t indices, counts, sel, zero, row_n, row_base, gather, ent, ent2, bucket_off, tiles,
+        sorted, part, recs, total;
+    int64_t ent_cap, tile_cap, n_zero;
+    bool bucket;
+};
+
+PrefillLayout prefill_layout(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d,
+                             lsa_select_params sp, int64_t ent_cap)
+{
+    const IndexView& v = idx->v;
+    const int64_t s_max = (int64_t)sp.budget + sp.window + sp.sinks;
+    const size_t rows = (size_t)v.B * (size_t)Nq;
+    PrefillLayout L{};
+    size_t o = 0;
+    L.indices = o; o += al256(rows * (size_t)s_max * 4);
+    L.counts = o;  o += al256(rows * 4);
+    L.sel = o;     o += select_ws_bytes(v, Nq);
+    // (sinks within the first block: no open-block key is ever below the sinks bound)
+    L.bucket = v.dtype == LSA_BF16 && bucket_attn_supported(Hq, Hkv, d) &&
+               (int64_t)sp.sinks <= (int64_t)v.p * v.G;
+    if (L.bucket) {
+        const int64_t nbt = v.B * v.NBK;
+        L.ent_cap = ent_cap;
+        L.tile_cap = ent_cap / BA_Q + (nbt < ent_cap ? nbt : ent_cap) + 1;
+        L.n_zero = nbt + CTR_N;
+        L.zero = o;       o += al256((size_t)L.n_zero * 4);
+        L.row_n = o;      o += al256(rows * 4);
+        L.row_base = o;   o += al256(rows * 4);
+        L.gather = o;     o += al256(rows * 4);
+        L.ent = o;        o += al256((size_t)ent_cap * 16);
+        L.ent2 = o;       o += al256((size_t)ent_cap * 8);
+        L.bucket_off = o; o += al256((size_t)nbt * 4);
+        L.tiles = o;      o += al256((size_t)L.tile_cap * 8);
+        L.sorted = o;     o += al256((size_t)ent_cap * 4);
+        L.part = o;       o += al256((size_t)ent_cap * Hq * (d + 4) * 4);
+        const int64_t n_wt = v.B * ((Nq + BA_Q - 1) / BA_Q);
+        L.recs = o;       o += al256((size_t)(n_wt + L.tile_cap) * TILE_REC_BYTES);
+    }
+    L.total = o;
+    return L;
+}
+
+// Partial slots per query row that the recommended workspace provides: one
+// per expected bucket (budget / mean bucket size) with half again as much
+// room, plus the sinks-and-window slot and one spare.  The slots are shared
+// by the whole chunk, so only the chunk's mean matters.
+int64_t default_ent_cap(const lsa_index* idx, int64_t Nq, lsa_select_params sp)
+{
+    const IndexView& v = idx->v;
+    int64_t bk = (int64_t)v.p * v.G / v.k;
+    if (bk < 1) bk = 1;
+    int64_t e = (3 * (int64_t)sp.budget + 2 * bk - 1) / (2 * bk) + 2;
+    if (e > KC + 1) e = KC + 1;
+    return v.B * Nq * e;
+}
+
+// Largest slot count whose layout fits in ws_bytes (-1: not even zero slots).
+int64_t ent_cap_for(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d, lsa_select_params sp,
+                    size_t ws_bytes)
+{
+    const PrefillLayout L0 = prefill_layout(idx, Nq, Hq, Hkv, d, sp, 0);
+    if (ws_bytes < L0.total) return -1;
+    if (!L0.bucket) return 0;
+    const size_t per = (size_t)Hq * (d + 4) * 4 + 16 + 8 + 4 + 8 + 8 + 2 * TILE_REC_BYTES;
+    int64_t e = (int64_t)((ws_bytes - L0.total) / per);
+    const int64_t cap = idx->v.B * Nq * (KC + 1);
+    if (e > cap) e = cap;
+    while (e > 0 && prefill_layout(idx, Nq, Hq, Hkv, d, sp, e).total > ws_bytes) --e;
+    return e;
 }
 
 struct DecodeLayout {
@@ -121,15 +197,6 @@ struct DecodeLayout {
     int ns, kps, n_hg;
 };
 
-int sm_count()
-{
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
-        return n;
-    cudaGetLastError();  // clear the error of a host without a device
-    return 148;
-}
 
 DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_select_params sp)
 {
@@ -176,6 +243,16 @@ lsa_status check_attn_shape(int Hq, int Hkv, int d, lsa_dtype dt)
 }
 
 }  // namespace
+
+int lsa::sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+        return n;
+    cudaGetLastError();  // clear the error of a host without a device
+    return 148;
+}
 
 void lsa::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
@@ -388,12 +465,122 @@ lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtyp
     return LSA_OK;
 }
 
-size_t lsa_prefill_workspace_bytes(const lsa_index* idx, int64_t Nq, lsa_select_params sp)
+size_t lsa_prefill_workspace_bytes(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d,
+                                   lsa_select_params sp)
 {
     if (!idx || Nq < 0 || sp.budget < 0 || sp.window < 0 || sp.sinks < 0) return 0;
-    const int64_t s_max = (int64_t)sp.budget + sp.window + sp.sinks;
-    const size_t rows = (size_t)idx->v.B * (size_t)Nq;
-    return al256(rows * (size_t)s_max * 4) + al256(rows * 4) + select_ws_bytes(idx->v, Nq);
+    if (Hq < 1 || Hkv < 1 || d < 1) return 0;
+    return prefill_layout(idx, Nq, Hq, Hkv, d, sp, default_ent_cap(idx, Nq, sp)).total;
+}
+
+int64_t lsa_prefill_partial_slots(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d,
+                                  lsa_select_params sp, size_t ws_bytes)
+{
+    if (!idx || Nq < 0 || sp.budget < 0 || sp.window < 0 || sp.sinks < 0) return -1;
+    if (Hq < 1 || Hkv < 1 || d < 1) return -1;
+    return ent_cap_for(idx, Nq, Hq, Hkv, d, sp, ws_bytes);
+}
+
+namespace {
+
+// Checks shared by the prefill entries; fills the layout and the plan view.
+lsa_status prefill_prepare(const lsa_index* idx, int64_t T_old, int64_t T_new, int Hq, int Hkv,
+                           int d, lsa_select_params sp, void* workspace, size_t ws_bytes,
+                           PrefillLayout* L, BucketPlan* P)
+{
+    const int64_t Nq = T_new - T_old;
+    if (Nq < 1) return fail(LSA_ERR_INVALID_ARG, "empty chunk");
+    const int s_max = sp.budget + sp.window + sp.sinks;
+    lsa_status s = check_select(idx, sp, s_max);
+    if (s != LSA_OK) return s;
+    // attention shape checks up front so that nothing launches on bad input
+    s = check_attn_shape(Hq, Hkv, d, idx->v.dtype);
+    if (s != LSA_OK) return s;
+    const int64_t ent_cap = ent_cap_for(idx, Nq, Hq, Hkv, d, sp, ws_bytes);
+    if (ent_cap < 0)
+        return fail(LSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes,
+                    prefill_layout(idx, Nq, Hq, Hkv, d, sp, 0).total);
+    if (!aligned16(workspace)) return fail(LSA_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+    *L = prefill_layout(idx, Nq, Hq, Hkv, d, sp, ent_cap);
+    if (L->bucket && (idx->v.B * Nq * (int64_t)(KC + 1) > 2147483647LL ||
+                      idx->v.B * idx->v.NBK > 2147483647LL))
+        return fail(LSA_ERR_UNSUPPORTED, "chunk too large for the bucket lists");
+    char* base = (char*)workspace;
+    *P = BucketPlan{};
+    if (L->bucket) {
+        P->zero = (int32_t*)(base + L->zero);
+        P->n_zero = L->n_zero;
+        P->bucket_cnt = P->zero;
+        P->ctr = P->zero + idx->v.B * idx->v.NBK;
+        P->row_n = (int32_t*)(base + L->row_n);
+        P->row_base = (int32_t*)(base + L->row_base);
+        P->gather_rows = (int32_t*)(base + L->gather);
+        P->ent = (int4*)(base + L->ent);
+        P->ent2 = (int2*)(base + L->ent2);
+        P->ent_cap = L->ent_cap;
+        P->bucket_off = (int32_t*)(base + L->bucket_off);
+        P->tiles = (int2*)(base + L->tiles);
+        P->tile_cap = L->tile_cap;
+        P->sorted = (int32_t*)(base + L->sorted);
+        P->part = (float*)(base + L->part);
+        P->recs = (unsigned char*)(base + L->recs);
+    }
+    return LSA_OK;
+}
+
+}  // namespace
+
+lsa_status lsa_prefill_select(lsa_index* idx, const void* latent_K, const void* latent_Q,
+                              int64_t T_old, int64_t T_new, int Hq, int Hkv, int d,
+                              lsa_select_params sp, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!idx || !latent_K || !latent_Q || !workspace)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    PrefillLayout L;
+    BucketPlan P;
+    lsa_status s = prefill_prepare(idx, T_old, T_new, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
+    if (s != LSA_OK) return s;
+    if (!aligned16(latent_Q)) return fail(LSA_ERR_ALIGNMENT, "latent_Q not 16-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    s = lsa_index_extend(idx, latent_K, T_old, T_new, stream);
+    if (s != LSA_OK) return s;
+    char* base = (char*)workspace;
+    const int s_max = sp.budget + sp.window + sp.sinks;
+    return run_select(idx, latent_Q, PosSrc{nullptr, T_old}, T_new - T_old, sp,
+                      (int32_t*)(base + L.indices), (int32_t*)(base + L.counts), s_max,
+                      base + L.sel, st, L.bucket ? &P : nullptr);
+}
+
+lsa_status lsa_prefill_attend(const lsa_index* idx, const void* Q, const void* K, const void* V,
+                              int64_t T_old, int64_t T_new, int Hq, int Hkv, int d,
+                              lsa_select_params sp, void* workspace, size_t ws_bytes, void* O,
+                              void* stream)
+{
+    if (!idx || !Q || !K || !V || !workspace || !O)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    PrefillLayout L;
+    BucketPlan P;
+    lsa_status s = prefill_prepare(idx, T_old, T_new, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
+    if (s != LSA_OK) return s;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+        return fail(LSA_ERR_ALIGNMENT, "Q, K, V and O must be 16-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t Nq = T_new - T_old;
+    const int s_max = sp.budget + sp.window + sp.sinks;
+    char* base = (char*)workspace;
+    const int32_t* indices = (const int32_t*)(base + L.indices);
+    const int32_t* counts = (const int32_t*)(base + L.counts);
+    const float scale = (float)(1.0 / sqrt((double)d));
+    cudaError_t e;
+    if (L.bucket)
+        e = launch_bucket_attn(idx->v, idx->n_blk, P, Q, K, V, Nq, Hq, Hkv, d,
+                               PosSrc{nullptr, T_old}, sp.window, sp.sinks, indices, counts,
+                               s_max, scale, O, st);
+    else
+        e = launch_attn_status(Q, K, V, idx->v.dtype, idx->v.B, Nq, idx->v.T_cap, Hq, Hkv, d,
+                               indices, counts, s_max, scale, O, nullptr, idx->v.status, st);
+    if (e != cudaSuccess) return cuda_fail(e, "sparse attention");
+    return LSA_OK;
 }
 
 lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* latent_Q,
@@ -403,37 +590,18 @@ lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* l
 {
     if (!idx || !latent_K || !latent_Q || !Q || !K || !V || !workspace || !O)
         return fail(LSA_ERR_INVALID_ARG, "NULL argument");
-    const int64_t Nq = T_new - T_old;
-    if (Nq < 1) return fail(LSA_ERR_INVALID_ARG, "empty chunk");
-    const int s_max = sp.budget + sp.window + sp.sinks;
-    lsa_status s = check_select(idx, sp, s_max);
+    PrefillLayout L;
+    BucketPlan P;
+    // every argument check of both halves before the first launch
+    lsa_status s = prefill_prepare(idx, T_old, T_new, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
     if (s != LSA_OK) return s;
-    if (ws_bytes < lsa_prefill_workspace_bytes(idx, Nq, sp))
-        return fail(LSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes,
-                    lsa_prefill_workspace_bytes(idx, Nq, sp));
-    if (!aligned16(workspace) || !aligned16(latent_Q) || !aligned16(Q) || !aligned16(O))
+    if (!aligned16(latent_Q) || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
         return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
-    // attention shape checks up front so that nothing launches on bad input
-    s = check_attn_shape(Hq, Hkv, d, idx->v.dtype);
+    s = lsa_prefill_select(idx, latent_K, latent_Q, T_old, T_new, Hq, Hkv, d, sp, workspace,
+                           ws_bytes, stream);
     if (s != LSA_OK) return s;
-    cudaStream_t st = (cudaStream_t)stream;
-    s = lsa_index_extend(idx, latent_K, T_old, T_new, stream);
-    if (s != LSA_OK) return s;
-    const size_t rows = (size_t)idx->v.B * (size_t)Nq;
-    char* p = (char*)workspace;
-    int32_t* indices = (int32_t*)p;
-    p += al256(rows * (size_t)s_max * 4);
-    int32_t* counts = (int32_t*)p;
-    p += al256(rows * 4);
-    PosSrc pos{nullptr, T_old};
-    s = run_select(idx, latent_Q, pos, Nq, sp, indices, counts, s_max, p, st);
-    if (s != LSA_OK) return s;
-    const float scale = (float)(1.0 / sqrt((double)d));
-    cudaError_t e = launch_attn_status(Q, K, V, idx->v.dtype, idx->v.B, Nq, idx->v.T_cap, Hq, Hkv,
-                                       d, indices, counts, s_max, scale, O, nullptr,
-                                       idx->v.status, st);
-    if (e != cudaSuccess) return cuda_fail(e, "sparse attention");
-    return LSA_OK;
+    return lsa_prefill_attend(idx, Q, K, V, T_old, T_new, Hq, Hkv, d, sp, workspace, ws_bytes, O,
+                              stream);
 }
 
 size_t lsa_decode_workspace_bytes(const lsa_index* idx, int Hq, int Hkv, int d,
@@ -459,7 +627,7 @@ lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
     if (s != LSA_OK) return s;
     s = check_attn_shape(Hq, Hkv, d, v.dtype);
     if (s != LSA_OK) return s;
-    if (idx->n_blk < 1 || idx->n_blk >= v.nblk_max)
+    if (idx->n_blk < 1 || idx->n_blk * v.G >= v.NP)
         return fail(LSA_ERR_INVALID_ARG,
                     "decode needs at least one closed block and room for an open block");
     const void* ptrs[] = {latent_K, K, V, new_latent_k, new_k, new_v, latent_q, q, pos, workspace, O};

@@ -75,6 +75,9 @@ __device__ __forceinline__ void dev_error(uint32_t* status, uint32_t code, uint3
 // Host-side count of kernel launches enqueued by the library (all threads).
 void note_launch();
 
+// Streaming multiprocessors of the current device (148 when it cannot be read).
+int sm_count();
+
 __device__ __forceinline__ float load_elt(const float* p) { return *p; }
 __device__ __forceinline__ float load_elt(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
@@ -95,6 +98,40 @@ cudaError_t launch_kmeans(const IndexView& ix, int64_t b0, int64_t b1, cudaStrea
 cudaError_t launch_open_assign(const IndexView& ix, int64_t n_blk, int64_t j_end,
                                cudaStream_t st);
 
+// Lists for bucket-major attention, written by the selection fill (bf16
+// prefill only; row_n == nullptr turns them off).  Every query row that the
+// fill ranks exactly and that finds room gets nt + 1 consecutive partial
+// slots: slot base + t for its t-th taken bucket, base + nt for its sinks and
+// recent window.  Other rows (exact fallback, no room) are listed in
+// gather_rows and attended key by key.
+enum PlanCtr : int {
+    CTR_RESERVED = 0,   // partial slots handed out (may pass ent_cap)
+    CTR_VALID_END = 1,  // end of the slots actually granted
+    CTR_GATHER = 2,     // rows in gather_rows
+    CTR_WORK = 3,       // work counter of the persistent attention kernel
+    CTR_TILES = 4,      // bucket tiles built by the plan kernel
+    CTR_N = 8
+};
+struct BucketPlan {
+    int32_t* zero;        // [n_zero] cleared by the scorer: bucket_cnt then ctr
+    int64_t n_zero;
+    int32_t* bucket_cnt;  // [B*NBK] taken entries per bucket
+    int32_t* ctr;         // [CTR_N]
+    int32_t* row_n;       // [rows] buckets taken by a listed row, -1 = gather row
+    int32_t* row_base;    // [rows] first partial slot of the row
+    int32_t* gather_rows; // [rows]
+    int4* ent;            // [ent_cap] (row, sequence-level bucket b*NBK+g or -1, lo, hi)
+    int2* ent2;           // [ent_cap] (rank of the entry inside its bucket, open keys taken)
+    int64_t ent_cap;
+    int32_t* bucket_off;  // [B*NBK] first sorted position of each bucket
+    int2* tiles;          // [tile_cap] (bucket, tile number inside the bucket)
+    int64_t tile_cap;
+    int32_t* sorted;      // [ent_cap] partial slots grouped by bucket
+    float* part;          // [ent_cap][Hq][d+4] softmax partials
+    unsigned char* recs;  // [window tiles + tile_cap] tile descriptions (TILE_REC_BYTES each)
+};
+constexpr int TILE_REC_BYTES = 448;
+
 // Selection workspace carve-up.
 struct SelectWs {
     int32_t* cand;       // [B][Nq][KC] candidate bucket ids (-1 padded)
@@ -106,6 +143,7 @@ struct SelectWs {
     __half* scores;      // [B*Nq][score_ld] tensor-core scores (tensor-core path only)
     __half* cmax;        // [B*Nq][score_ld/32] maximum of every 32-score chunk
     int64_t score_ld;
+    BucketPlan plan;     // bucket-major attention lists (all null when unused)
 };
 constexpr int FB_CTAS = 148;
 // The tensor-core scorer serves bf16 indices and at least one 128-query tile.
@@ -142,6 +180,13 @@ cudaError_t launch_attn_split(const void* Q, const void* K, const void* V, int64
                               uint32_t* status, int ns, int keys_per_split, float* part,
                               uint32_t* counter, int hg, cudaStream_t st);
 int attn_stage_keys(int Hkv);
+// bf16 attention of the rows row_list[0 .. *row_count) only (grid sized for
+// all B * Nq rows; CTAs past the count exit at once).
+cudaError_t launch_attn_rows(const void* Q, const void* K, const void* V, int64_t B, int64_t Nq,
+                             int64_t T_cap, int Hq, int Hkv, int d, const int32_t* indices,
+                             const int32_t* counts, int s_max, float scale, void* O,
+                             uint32_t* status, const int32_t* row_list, const int32_t* row_count,
+                             cudaStream_t st);
 // Merges the ns split partials of every (row, query head) into O (bf16) and lse.
 cudaError_t launch_attn_combine(const float* part, int ns, int64_t rows, int Hq, int d, void* O,
                                 float* lse, cudaStream_t st);
@@ -161,6 +206,17 @@ cudaError_t noalloc_select(const IndexView& ix, int64_t n_blk, const void* laten
                            const int32_t* positions, int64_t Nq, lsa_select_params sp,
                            int32_t* indices, int32_t* counts, int s_max, bool use_tc,
                            cudaStream_t st);
+
+// Bucket-major attention of a bf16 prefill chunk (k_attn_bucket.cu): plan,
+// scatter, the persistent tile kernel, the per-query kernel for gather rows
+// and the merge of every listed row's partials into O.
+constexpr int BA_Q = 16;   // queries per bucket or window tile
+bool bucket_attn_supported(int Hq, int Hkv, int d);
+cudaError_t launch_bucket_attn(const IndexView& ix, int64_t n_blk, const BucketPlan& P,
+                               const void* Q, const void* K, const void* V, int64_t Nq, int Hq,
+                               int Hkv, int d, PosSrc pos, int W, int S, const int32_t* indices,
+                               const int32_t* counts, int s_max, float scale, void* O,
+                               cudaStream_t st);
 
 // True when the tensor-core candidate scorer is compiled in.
 bool tc_scoring_available();

@@ -67,6 +67,51 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
         : "memory");
 }
 
+// ---- per-thread async copy (16 bytes, L2 only), global -> shared -----------
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src_gmem)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst_smem)),
+                 "l"(src_gmem)
+                 : "memory");
+}
+
+// Copies src_bytes (0 or 16) and zero-fills the rest of the 16 bytes.
+__device__ __forceinline__ void cp_async16_zfill(void* dst_smem, const void* src_gmem,
+                                                 uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst_smem)),
+                 "l"(src_gmem), "r"(src_bytes)
+                 : "memory");
+}
+
+// The mbarrier receives one arrival when every cp.async this thread issued
+// so far has completed (the arrival is not pre-counted: the barrier's
+// expected count must include it).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory accesses with later
+// async-proxy ones (tensor-core operand reads).
+__device__ __forceinline__ void fence_proxy_async()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Waits until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ---- warp-level MMA (bf16 in, fp32 accumulate) ----------------------------
 __device__ __forceinline__ void ldsm_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
                                         const void* p)

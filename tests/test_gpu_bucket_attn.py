@@ -1,0 +1,152 @@
+"""bf16 prefill chunks (bucket-major attention) against the oracle, whole chunk.
+
+Each case runs lsa_prefill_chunk on a small bf16 workload and checks, for every
+query of the chunk, the selection (row for row) and the output against
+oracle.attend on the oracle's selection (bf16 bars: 2e-2 max-abs, 2e-3
+mean-abs).  Cases: a chunk that ends inside a block (open-block members are
+taken), a chunk that starts at position 0 (sinks and window overlap, block-0
+buckets cut by the sinks bound), several sequences, every supported head
+shape, workspaces with too few partial slots (some or all rows then go
+through the per-query kernel), and exact-fallback rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+lsa = pytest.importorskip("long_context_indexing_b200")
+
+BF16_MAX, BF16_MEAN = 2e-2, 2e-3
+
+
+def _base(**kw):
+    # 256-token blocks of 4 buckets (64 keys each); a budget of ~6 buckets
+    args = dict(T=2760, nq=700, B=1, Hq=8, Hkv=2, d=64, M=48, p=4, G=64, k=4, L=3, R=384, W=48,
+                S=4, dtype="bf16")
+    args.update(kw)
+    return synth.workload("tiny", **args)
+
+
+def _run(w, seed=0, ws_bytes=None, same_latent=False, check_repeat=False):
+    T_old = w.T - w.nq
+    inp = synth.prefill_inputs(w, seed, "cpu")
+    if same_latent:   # every approximate score ties: rows go to the exact fallback
+        inp["latent_K"][:] = inp["latent_K"][:, :1]
+    dev = {k: v.cuda() for k, v in inp.items()}
+    gpu = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16)
+    gpu.build(dev["latent_K"], T_old)
+    if ws_bytes is None:
+        ws_bytes = lsa.lsa_prefill_workspace_bytes(gpu, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    O = lsa.lsa_prefill_chunk(gpu, dev["latent_K"], dev["latent_Q"], dev["Q"], dev["K"], dev["V"],
+                              T_old, w.T, w.R, w.W, w.S, workspace=ws)
+    torch.cuda.synchronize()
+    fallbacks = gpu.check()
+    g_idx, g_cnt = lsa.prefill_selection_views(ws, w.B, w.nq, w.s_max)
+    g_idx, g_cnt = g_idx.cpu().numpy(), g_cnt.cpu().numpy()
+    g_open = gpu.export()["open_bucket"].cpu().numpy()
+    errs = []
+    for b in range(w.B):
+        lat = inp["latent_K"][b].float().numpy()
+        orc = oracle.Index(w.T, w.p, w.G, w.k, w.L, rt_bf16=True)
+        orc.extend(lat, 0, T_old)
+        orc.extend(lat, T_old, w.T)
+        assert np.array_equal(g_open[b], orc.open_bucket)
+        pos = inp["positions"][b].numpy()
+        o_idx, o_cnt, _, _ = oracle.select(orc, inp["latent_Q"][b].float().numpy(), pos, w.R, w.W,
+                                           w.S)
+        assert np.array_equal(g_cnt[b], o_cnt)
+        assert np.array_equal(g_idx[b], o_idx)
+        O_ref, _ = oracle.attend(inp["Q"][b].float().numpy(), inp["K"][b].float().numpy(),
+                                 inp["V"][b].float().numpy(), o_idx, o_cnt,
+                                 oracle.default_scale(w.d))
+        err = np.abs(O[b].float().cpu().numpy().astype(np.float64) - O_ref)
+        assert err.max() <= BF16_MAX, (b, err.max())
+        assert err.mean() <= BF16_MEAN, (b, err.mean())
+        errs.append(err.max())
+    if check_repeat:
+        O2 = lsa.lsa_prefill_chunk(gpu, dev["latent_K"], dev["latent_Q"], dev["Q"], dev["K"],
+                                   dev["V"], T_old, w.T, w.R, w.W, w.S, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(O, O2)
+    return fallbacks, max(errs)
+
+
+def _ws_for_slots(w, want):
+    """Smallest workspace giving at least `want` partial slots (binary search)."""
+    gpu = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16)
+    hi = lsa.lsa_prefill_workspace_bytes(gpu, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S)
+    slots = lambda n: lsa.lsa_prefill_partial_slots(gpu, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S, n)
+    assert slots(hi) >= want
+    lo = 0
+    while lo < hi:
+        mid = (lo + hi) // 2
+        if slots(mid) >= want:
+            hi = mid
+        else:
+            lo = mid + 1
+    return hi
+
+
+def test_chunk_ending_inside_a_block():
+    w = _base()
+    span = w.p * w.G
+    # the last queries' long-range keys reach into the open block
+    assert w.T - 1 - w.W >= (w.T // span) * span + 64
+    fb, _ = _run(w, seed=11, check_repeat=True)
+    assert fb == 0
+
+
+def test_chunk_from_position_zero():
+    w = _base(T=2048, nq=2048, R=200, W=24, S=6)
+    _run(w, seed=12)
+
+
+def test_several_sequences():
+    w = _base(T=4096, nq=512, B=3, R=512)
+    _run(w, seed=13)
+
+
+@pytest.mark.parametrize("Hq,Hkv,d", [(8, 8, 64), (8, 4, 128), (16, 4, 64), (32, 4, 128),
+                                      (8, 1, 128), (4, 2, 64)])
+def test_head_shapes(Hq, Hkv, d):
+    w = _base(T=3000, nq=400, Hq=Hq, Hkv=Hkv, d=d)
+    _run(w, seed=14)
+
+
+def test_large_buckets_span_several_stages():
+    # 2 buckets of 1024-token blocks: ~512 keys per bucket, 8 pipeline stages
+    w = _base(T=6000, nq=600, G=256, k=2, R=1500, W=100)
+    _run(w, seed=15)
+
+
+def test_few_partial_slots():
+    w = _base()
+    ws = _ws_for_slots(w, w.nq * 2)     # room for a fraction of the rows
+    _run(w, seed=16, ws_bytes=ws)
+
+
+def test_no_partial_slots():
+    w = _base()
+    ws = _ws_for_slots(w, 0)            # minimum workspace: every row key by key
+    gpu = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16)
+    assert lsa.lsa_prefill_partial_slots(gpu, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S, ws) == 0
+    assert lsa.lsa_prefill_partial_slots(gpu, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S, ws - 1) == -1
+    _run(w, seed=17, ws_bytes=ws)
+
+
+def test_workspace_below_minimum_is_refused():
+    w = _base()
+    ws = _ws_for_slots(w, 0) - 256
+    with pytest.raises(lsa.LsaError):
+        _run(w, seed=17, ws_bytes=ws)
+
+
+def test_fallback_rows():
+    w = _base(T=2048, nq=512, G=16, R=300)      # 128 buckets: more than one candidate set
+    fb, _ = _run(w, seed=18, same_latent=True)
+    assert fb > 0

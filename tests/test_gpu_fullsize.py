@@ -40,8 +40,8 @@ def test_full_size_prefill_chunk_sampled(name):
     T_old = w.T - w.nq
     idx = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16)
     idx.build(inp["latent_K"], (T_old // span) * span)
-    ws = torch.empty(lsa.lsa_prefill_workspace_bytes(idx, w.nq, w.R, w.W, w.S), dtype=torch.uint8,
-                     device="cuda")
+    ws = torch.empty(lsa.lsa_prefill_workspace_bytes(idx, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S),
+                     dtype=torch.uint8, device="cuda")
     O = lsa.lsa_prefill_chunk(idx, inp["latent_K"], inp["latent_Q"], inp["Q"], inp["K"],
                               inp["V"], T_old, w.T, w.R, w.W, w.S, workspace=ws)
     torch.cuda.synchronize()

@@ -137,8 +137,8 @@ def test_prefill_chunk_matches_oracle(name):
     pos = inp["positions"][0].numpy()
     o_idx, o_cnt, o_mg, _ = oracle.select(orc, inp["latent_Q"][0].float().numpy(), pos, w.R, w.W,
                                           w.S)
-    ws = torch.empty(lsa.lsa_prefill_workspace_bytes(gpu, w.nq, w.R, w.W, w.S), dtype=torch.uint8,
-                     device="cuda")
+    ws = torch.empty(lsa.lsa_prefill_workspace_bytes(gpu, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S),
+                     dtype=torch.uint8, device="cuda")
     O = lsa.lsa_prefill_chunk(gpu, dev["latent_K"], dev["latent_Q"], dev["Q"], dev["K"], dev["V"],
                               T_old, w.T, w.R, w.W, w.S, workspace=ws)
     torch.cuda.synchronize()
