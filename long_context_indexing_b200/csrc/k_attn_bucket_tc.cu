@@ -116,6 +116,38 @@ __device__ __forceinline__ void tb_ld32(uint32_t taddr, float* v)
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+// Two 32-column TMEM loads in flight, one wait.
+__device__ __forceinline__ void tb_ld64(uint32_t taddr, float* v)
+{
+    uint32_t r[64];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+            "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+            "%28, %29, %30, %31}, [%32];"
+            : "=r"(r[32 * h + 0]), "=r"(r[32 * h + 1]), "=r"(r[32 * h + 2]), "=r"(r[32 * h + 3]),
+              "=r"(r[32 * h + 4]), "=r"(r[32 * h + 5]), "=r"(r[32 * h + 6]), "=r"(r[32 * h + 7]),
+              "=r"(r[32 * h + 8]), "=r"(r[32 * h + 9]), "=r"(r[32 * h + 10]), "=r"(r[32 * h + 11]),
+              "=r"(r[32 * h + 12]), "=r"(r[32 * h + 13]), "=r"(r[32 * h + 14]), "=r"(r[32 * h + 15]),
+              "=r"(r[32 * h + 16]), "=r"(r[32 * h + 17]), "=r"(r[32 * h + 18]), "=r"(r[32 * h + 19]),
+              "=r"(r[32 * h + 20]), "=r"(r[32 * h + 21]), "=r"(r[32 * h + 22]), "=r"(r[32 * h + 23]),
+              "=r"(r[32 * h + 24]), "=r"(r[32 * h + 25]), "=r"(r[32 * h + 26]), "=r"(r[32 * h + 27]),
+              "=r"(r[32 * h + 28]), "=r"(r[32 * h + 29]), "=r"(r[32 * h + 30]), "=r"(r[32 * h + 31])
+            : "r"(taddr + 32u * h));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 64; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// 2^x by the hardware approximation (flush-to-zero; 2^-inf = +0).
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void tb_st32(uint32_t taddr, const float* v)
 {
     asm volatile(
@@ -432,21 +464,42 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 }
                 tb_fence_after();
                 float v[TB_N];
-                tb_ld32(tmem + lane_base + sb * TB_N, v);
-                tb_ld32(tmem + lane_base + sb * TB_N + 32, v + 32);
+                tb_ld64(tmem + lane_base + sb * TB_N, v);
                 tb_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&s_empty[sb]);
 
                 const int kb = kbeg + s * TB_N;
-                const bool all_in = live && rg.covers(kb, kb + TB_N);
-                float mx = -INFINITY;
-#pragma unroll
-                for (int j = 0; j < TB_N; ++j) {
-                    const bool ok = all_in || (live && rg.has(kb + j));
-                    v[j] = ok ? v[j] * a.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, v[j]);
+                // keys of this stage the row's query reads, as a 64-bit mask
+                uint64_t keep = 0;
+                if (live) {
+                    auto bits = [&](int lo, int hi) -> uint64_t {
+                        int x = lo - kb, y = hi - kb;
+                        x = x < 0 ? 0 : (x > TB_N ? TB_N : x);
+                        y = y < 0 ? 0 : (y > TB_N ? TB_N : y);
+                        if (y <= x) return 0ull;
+                        const uint64_t up = (y == TB_N) ? ~0ull : ((1ull << y) - 1ull);
+                        return up & ~((1ull << x) - 1ull);
+                    };
+                    keep = bits(rg.lo0, rg.hi0) | bits(rg.lo1, rg.hi1);
                 }
+                if (keep != ~0ull) {
+#pragma unroll
+                    for (int j = 0; j < TB_N; ++j)
+                        if (!((keep >> j) & 1ull)) v[j] = -INFINITY;
+                }
+                // row maximum of the raw scores (scale > 0), as a tree
+                float t8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    float m = v[u];
+#pragma unroll
+                    for (int j = u + 8; j < TB_N; j += 8) m = fmaxf(m, v[j]);
+                    t8[u] = m;
+                }
+                const float mraw = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
+                                         fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+                const float mx = mraw * a.scale_log2;   // -inf stays -inf
                 // Lazy running max: raised only on the item's first stage, from
                 // nothing, or by more than 8 (a factor 2^8), so that O needs
                 // rescaling rarely; P stays <= 2^8.
@@ -456,20 +509,23 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                     if (s == 0 || m_run == -INFINITY) {
                         m_run = mx;
                     } else if (mx > m_run + 8.f) {
-                        alpha = exp2f(m_run - mx);
+                        alpha = ex2_approx(m_run - mx);
                         m_run = mx;
                         resc = true;
                     }
                 }
                 const float mu = (m_run == -INFINITY) ? 0.f : m_run;
                 uint32_t pk[TB_N / 2];
-                float sum = 0.f;
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int j = 0; j < TB_N / 2; ++j) {
-                    const float p0 = exp2f(v[2 * j] - mu), p1 = exp2f(v[2 * j + 1] - mu);
-                    sum += p0 + p1;
+                    // p = 2^(s * scale * log2(e) - m); a masked key gives 2^-inf = 0
+                    const float p0 = ex2_approx(fmaf(v[2 * j], a.scale_log2, -mu));
+                    const float p1 = ex2_approx(fmaf(v[2 * j + 1], a.scale_log2, -mu));
+                    s4[j & 3] += p0 + p1;
                     pk[j] = ptx::pack_bf16(p0, p1);
                 }
+                const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
                 l = l * alpha + sum;
                 // the previous P has been consumed (and O is quiet) once the
                 // previous PV MMA has completed
