@@ -210,34 +210,37 @@ __device__ __forceinline__ void ba_softmax(const float (&s)[4], int key_lo, cons
     pb1 = ptx::movmatrix_t(ptx::pack_bf16(p2, p3));
 }
 
-// Writes one query's partial for the query heads of KV head h:
-// [acc[0..D) | max (log2 units) | sum | 2 pad] per head, stride D + 4 floats.
+// Writes one query's partial for the query heads of KV head h: per head the
+// accumulator normalised by its own sum, as bf16 (po [hpg][D]), and the
+// (max in log2 units, sum) pair (pml [hpg]).
 template <int KSTEPS>
-__device__ __forceinline__ void ba_write_partial(float* pp, int hpg, float m0, float m1, float l0,
-                                                 float l1, const float (&o)[KSTEPS][4])
+__device__ __forceinline__ void ba_write_partial(__nv_bfloat16* po, float2* pml, int hpg, float m0,
+                                                 float m1, float l0, float l1,
+                                                 const float (&o)[KSTEPS][4])
 {
-    constexpr int D = KSTEPS * 16, PS = D + 4;
+    constexpr int D = KSTEPS * 16;
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int o_ = 4; o_ < 32; o_ <<= 1) {
         l0 += __shfl_xor_sync(0xffffffffu, l0, o_);
         l1 += __shfl_xor_sync(0xffffffffu, l1, o_);
     }
+    const float i0 = (l0 > 0.f) ? 1.f / l0 : 0.f, i1 = (l1 > 0.f) ? 1.f / l1 : 0.f;
     const int h0 = 2 * (lane & 3), dr = lane >> 2;
 #pragma unroll
     for (int mt = 0; mt < KSTEPS; ++mt) {
         if (h0 < hpg) {
-            pp[h0 * PS + mt * 16 + dr] = o[mt][0];
-            pp[h0 * PS + mt * 16 + dr + 8] = o[mt][2];
+            po[h0 * D + mt * 16 + dr] = __float2bfloat16_rn(o[mt][0] * i0);
+            po[h0 * D + mt * 16 + dr + 8] = __float2bfloat16_rn(o[mt][2] * i0);
         }
         if (h0 + 1 < hpg) {
-            pp[(h0 + 1) * PS + mt * 16 + dr] = o[mt][1];
-            pp[(h0 + 1) * PS + mt * 16 + dr + 8] = o[mt][3];
+            po[(h0 + 1) * D + mt * 16 + dr] = __float2bfloat16_rn(o[mt][1] * i1);
+            po[(h0 + 1) * D + mt * 16 + dr + 8] = __float2bfloat16_rn(o[mt][3] * i1);
         }
     }
     if (dr == 0) {
-        if (h0 < hpg) *reinterpret_cast<float2*>(pp + h0 * PS + D) = make_float2(m0, l0);
-        if (h0 + 1 < hpg) *reinterpret_cast<float2*>(pp + (h0 + 1) * PS + D) = make_float2(m1, l1);
+        if (h0 < hpg) pml[h0] = make_float2(m0, l0);
+        if (h0 + 1 < hpg) pml[h0 + 1] = make_float2(m1, l1);
     }
 }
 
@@ -414,26 +417,31 @@ __global__ void __launch_bounds__(BA_THREADS, LSA_BA_MIN_BLOCKS) bucket_attn_ker
         }
         ptx::cp_async_wait<0>();
 
-        if (liveA)
-            ba_write_partial<KSTEPS>(a.P.part + ((size_t)ti.slot[qa] * a.Hq + (size_t)h * a.hpg) * PS,
-                                     a.hpg, ma0, ma1, la0, la1, oa);
-        if (liveB)
-            ba_write_partial<KSTEPS>(a.P.part + ((size_t)ti.slot[qb] * a.Hq + (size_t)h * a.hpg) * PS,
-                                     a.hpg, mb0, mb1, lb0, lb1, ob);
+        if (liveA) {
+            const size_t ph = (size_t)ti.slot[qa] * a.Hq + (size_t)h * a.hpg;
+            ba_write_partial<KSTEPS>(a.P.part_o + ph * D, a.P.part_ml + ph, a.hpg, ma0, ma1, la0,
+                                     la1, oa);
+        }
+        if (liveB) {
+            const size_t ph = (size_t)ti.slot[qb] * a.Hq + (size_t)h * a.hpg;
+            ba_write_partial<KSTEPS>(a.P.part_o + ph * D, a.P.part_ml + ph, a.hpg, mb0, mb1, lb0,
+                                     lb1, ob);
+        }
         __syncthreads();   // the next tile rewrites the ring and the tile's shared state
     }
 }
 
 // ---------------------------------------------------------------------------
 // Merge: one warp per (listed row, query head) combines the row's nt + 1
-// partials: weights exp2(m_s - M) over the global max M, output
-// sum_s w_s acc_s / sum_s w_s l_s.
+// partials.  Partial s holds O_s / l_s (bf16) with its max m_s and sum l_s:
+// with M the largest max and w_s = l_s exp2(m_s - M), the output is
+// sum_s w_s (O_s / l_s) / sum_s w_s.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(128) bucket_merge_kernel(BucketPlan P, int64_t n_heads_total,
                                                            int Hq, __nv_bfloat16* O)
 {
-    constexpr int PS = D + 4;
+    constexpr int PER = D / 32;                  // output elements per lane
     const int lane = threadIdx.x & 31;
     const int64_t wid = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
     if (wid >= n_heads_total) return;
@@ -441,43 +449,48 @@ __global__ void __launch_bounds__(128) bucket_merge_kernel(BucketPlan P, int64_t
     const int nt = P.row_n[row];
     if (nt < 0) return;                       // gather row: written by the per-query kernel
     const int ns = nt + 1;
-    const float* base = P.part + ((int64_t)P.row_base[row] * Hq + hd) * PS;
-    const int64_t sstride = (int64_t)Hq * PS;
+    const int64_t p0 = (int64_t)P.row_base[row] * Hq + hd;   // partial (slot base, head)
     float M = -INFINITY;
     for (int s0 = 0; s0 < ns; s0 += 32)
-        if (s0 + lane < ns) M = fmaxf(M, __ldcg(base + (s0 + lane) * sstride + D));
+        if (s0 + lane < ns) M = fmaxf(M, __ldcg(&P.part_ml[p0 + (int64_t)(s0 + lane) * Hq]).x);
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const bool live = lane < D / 4;
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
     for (int s0 = 0; s0 < ns; s0 += 32) {
         float wgt = 0.f;
         if (s0 + lane < ns) {
-            const float2 ml =
-                __ldcg(reinterpret_cast<const float2*>(base + (s0 + lane) * sstride + D));
-            wgt = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-            L += ml.y * wgt;
+            const float2 mlv = __ldcg(&P.part_ml[p0 + (int64_t)(s0 + lane) * Hq]);
+            wgt = (mlv.x == -INFINITY) ? 0.f : mlv.y * exp2f(mlv.x - M);
+            L += wgt;
         }
         const int n = min(32, ns - s0);
         for (int j = 0; j < n; ++j) {
             const float wj = __shfl_sync(0xffffffffu, wgt, j);
-            if (live) {
-                const float4 v =
-                    __ldcg(reinterpret_cast<const float4*>(base + (s0 + j) * sstride) + lane);
-                acc.x += v.x * wj;
-                acc.y += v.y * wj;
-                acc.z += v.z * wj;
-                acc.w += v.w * wj;
+            const __nv_bfloat16* src = P.part_o + (p0 + (int64_t)(s0 + j) * Hq) * D + PER * lane;
+            if (PER == 4) {
+                const uint2 u = __ldcg(reinterpret_cast<const uint2*>(src));
+                const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+                const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+                acc[0] += a0.x * wj;
+                acc[1] += a0.y * wj;
+                acc[2] += a1.x * wj;
+                acc[3] += a1.y * wj;
+            } else {
+                const unsigned u = __ldcg(reinterpret_cast<const unsigned*>(src));
+                const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+                acc[0] += a0.x * wj;
+                acc[1] += a0.y * wj;
             }
         }
     }
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (live) {
-        const float inv = 1.f / L;
-        __nv_bfloat16* op = O + wid * D + 4 * lane;
-        *reinterpret_cast<__nv_bfloat162*>(op) = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-        *reinterpret_cast<__nv_bfloat162*>(op + 2) = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    }
+    const float inv = 1.f / L;
+    __nv_bfloat16* op = O + wid * D + PER * lane;
+#pragma unroll
+    for (int e = 0; e < PER; e += 2)
+        *reinterpret_cast<__nv_bfloat162*>(op + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
 }
 
 bool bucket_attn_supported(int Hq, int Hkv, int d)

@@ -9,9 +9,9 @@
 //
 //   S  = Q K^T   M = 128, N = 64 keys, K = d      (TMEM, double-buffered)
 //   P  = exp2(S * scale * log2 e - m)            (softmax warps, bf16 to smem)
-//   O += P V     M = 128, N = d, K = 64 keys      (TMEM, one accumulator)
+//   O += P V     M = 128, N = d, K = 64 keys      (TMEM, two accumulators)
 //
-// Warp roles (8 warps):
+// Warp roles (13 warps):
 //   warp 0     planner: claims work items and copies each tile's description
 //              (written by bucket_tile_records_kernel) and the bucket's member
 //              lists into shared memory, one item ahead;
@@ -20,11 +20,16 @@
 //              planes (the layout the MMA descriptors name); completion lands
 //              on mbarriers;
 //   warp 3     allocates TMEM; lane 0 issues all MMAs and commits;
+//   warp 12    Q loader: the tile's Q rows, as soon as its Q buffer is free;
 //   warps 4-7  softmax: thread = row = TMEM lane; reads its 64 scores of a
 //              stage, masks keys outside its query's ranges, keeps the
 //              running max (raised lazily: O and the sum are rescaled only
 //              when the max grows by more than 2^8), writes its P row, and at
-//              the end of the tile writes the row's partial (acc, max, sum).
+//              the end of the tile hands the row's (max, sum) on;
+//   warps 8-11 epilogue: write each row's partial (O row / sum as bf16, and
+//              the fp32 max and sum) from one
+//              of two TMEM accumulators (tiles alternate), overlapping the
+//              next tile's softmax.
 // Q and tile descriptions are double-buffered across work items and the K/V
 // ring continues across them, so loads of the next tile overlap this one.
 // Every wait is bounded; on a timeout the CTA records DEV_TIMEOUT, all roles
@@ -40,12 +45,11 @@ namespace lsa {
 
 constexpr int TB_M = 128;            // MMA rows: BA_Q queries x 8 query heads
 constexpr int TB_N = 64;             // keys per stage
-constexpr int TB_NS = 3;             // K/V stages in the ring
-constexpr int TB_OPEN_MAX = 2048;    // open-block members one tile can hold
-constexpr int TB_THREADS = 256;      // 8 warps
+constexpr int TB_OPEN_MAX = 2048;    // members of one bucket a tile can hold (block size bound)
+constexpr int TB_THREADS = 416;      // 13 warps
 constexpr uint32_t TB_WAIT = 1u << 22;
 
-template <int D>
+template <int D, int NS>
 struct TbCfg {
     static constexpr int CH = D / 8;                    // 16-byte chunks per row
     static constexpr int Q_PLANE = TB_M * 128;          // 64 dims of 128 rows
@@ -55,13 +59,14 @@ struct TbCfg {
     static constexpr int STAGE = 2 * K_BYTES;           // K then V
     static constexpr int P_BYTES = TB_M * TB_N * 2;
     static constexpr int OFF_Q = 0;                     // two buffers
-    static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
-    static constexpr int OFF_P = OFF_KV + TB_NS * STAGE;
-    static constexpr int OFF_OPEN = OFF_P + P_BYTES;    // two open-member lists
-    static constexpr int OFF_MEM = OFF_OPEN + 2 * TB_OPEN_MAX * 4;   // two closed-member lists
-    static constexpr int OFF_BAR = OFF_MEM + 2 * TB_OPEN_MAX * 4;
-    static constexpr int NBAR = 16 + 2 * TB_NS;
-    static constexpr int BYTES = OFF_BAR + NBAR * 8 + 1024;   // + alignment slack
+    static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;  // NS stages
+    static constexpr int OFF_P = OFF_KV + NS * STAGE;
+    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    static constexpr int NBAR = 20 + 2 * NS;
+    static constexpr int OFF_ML = OFF_BAR + NBAR * 8;      // [2][128] (max, sum) per row
+    static constexpr int OFF_LISTS = OFF_ML + 2 * TB_M * 8;   // then 4 member lists of G ints
+    // dynamic shared memory for a block of G pooled groups (+ alignment slack)
+    static constexpr int bytes(int G) { return OFF_LISTS + 4 * ((G + 3) & ~3) * 4 + 1024; }
     static constexpr uint32_t KSTEPS = D / 16;
     // kind::f16, fp32 accumulate, bf16 A and B, M = 128
     static constexpr uint32_t IDESC_S =
@@ -169,10 +174,10 @@ __device__ __forceinline__ void tb_st32(uint32_t taddr, const float* v)
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-template <int D>
+template <int D, int NS>
 __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
 {
-    using C = TbCfg<D>;
+    using C = TbCfg<D, NS>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -184,10 +189,17 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     uint64_t* s_empty = bars + 10;       // [2]
     uint64_t* p_full = bars + 12;
     uint64_t* p_empty = bars + 13;
-    uint64_t* o_full = bars + 14;
-    uint64_t* o_empty = bars + 15;
-    uint64_t* kv_full = bars + 16;       // [TB_NS]
-    uint64_t* kv_empty = kv_full + TB_NS;
+    uint64_t* o_full = bars + 14;        // [2] (two O accumulators, by item parity)
+    uint64_t* o_empty = bars + 16;       // [2]
+    uint64_t* ml_full = bars + 18;       // [2]
+    uint64_t* kv_full = bars + 20;       // [NS]
+    float2* ml = reinterpret_cast<float2*>(smem + C::OFF_ML);   // [2][TB_M]
+    uint64_t* kv_empty = kv_full + NS;
+    const int lcap = (a.ix.G + 3) & ~3;  // ints per member list
+    int32_t* lists = reinterpret_cast<int32_t*>(smem + C::OFF_LISTS);
+    // [0, 2): open-member lists of the two item buffers; [2, 4): closed-member lists
+    auto open_list = [&](int ib) { return lists + ib * lcap; };
+    auto mem_list = [&](int ib) { return lists + (2 + ib) * lcap; };
     __shared__ TileInfo ti[2];
     __shared__ uint32_t tmem_slot;
     __shared__ volatile int abort_flag;
@@ -203,17 +215,18 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&info_full[i], 1);
-            ptx::mbar_init(&info_empty[i], 7);     // 4 softmax warps, the MMA thread, 2 loader warps
-            ptx::mbar_init(&q_full[i], 64);        // every producer thread's cp.async arrival
+            ptx::mbar_init(&info_empty[i], 12);    // 4 softmax, 4 epilogue, MMA, 2 K/V loaders, Q loader
+            ptx::mbar_init(&o_full[i], 1);
+            ptx::mbar_init(&o_empty[i], 4);
+            ptx::mbar_init(&ml_full[i], 4);
+            ptx::mbar_init(&q_full[i], 32);        // every Q-loader lane's cp.async arrival
             ptx::mbar_init(&q_empty[i], 1);
             ptx::mbar_init(&s_full[i], 1);
             ptx::mbar_init(&s_empty[i], 4);
         }
         ptx::mbar_init(p_full, 4);
         ptx::mbar_init(p_empty, 1);
-        ptx::mbar_init(o_full, 1);
-        ptx::mbar_init(o_empty, 4);
-        for (int s = 0; s < TB_NS; ++s) {
+        for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(&kv_full[s], 64);
             ptx::mbar_init(&kv_empty[s], 1);
         }
@@ -222,7 +235,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
         ptx::fence_mbar_init();
     }
     if (warp == 3) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
                          ptx::smem_addr(&tmem_slot))
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -282,22 +295,54 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             __syncwarp();
             if (lane == 0) T.h = (int)(w % a.Hkv);
             if (T.kind == 1) {
-                int32_t* mem_l = reinterpret_cast<int32_t*>(smem + C::OFF_MEM) + ib * TB_OPEN_MAX;
+                int32_t* mem_l = mem_list(ib);
                 const int32_t* mem_g = ix.members + T.b * ix.NP + T.o0;
                 for (int x = lane; x < T.nclosed / p; x += 32) mem_l[x] = mem_g[x];
                 if (T.any_open) {
-                    int32_t* open_l = reinterpret_cast<int32_t*>(smem + C::OFF_OPEN) + ib * TB_OPEN_MAX;
+                    int32_t* open_l = open_list(ib);
                     ba_open_list(ix, a.n_blk, T.b, T.g, lane, 32, cnt_s, open_l, [] { __syncwarp(); });
                 }
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&info_full[ib]);
         }
+    } else if (warp == 12) {
+        // ============================ Q loader ============================
+        // The tile's Q rows (row r = query r / hpg, head r % hpg; rows of empty
+        // query positions are zero), as soon as the tile is described and its
+        // Q buffer is free.
+        for (int i = 0;; ++i) {
+            const int ib = i & 1;
+            const uint32_t iph = (uint32_t)((i >> 1) & 1);
+            const TileInfo& T = ti[ib];
+            if (!waitw(&info_full[ib], iph, 130u)) break;
+            if (T.n_st < 0) break;
+            if (!waitw(&q_empty[ib], iph ^ 1u, 140u)) break;
+            unsigned char* qs = smem + C::OFF_Q + ib * C::Q_BYTES;
+            // Query q's hpg head rows are contiguous (hpg * D bf16) and fill MMA
+            // rows q*hpg .. q*hpg+hpg-1.  Rows of empty query positions are
+            // not loaded: every key of such a row is masked, so whatever the
+            // buffer holds there never reaches a partial.
+            const int per_q = a.hpg * C::CH;               // 16-byte chunks per query
+            for (int q = 0; q < BA_Q; ++q) {
+                if (T.slot[q] < 0) continue;
+                const __nv_bfloat16* src_q = a.Q + ((size_t)T.row[q] * a.Hq + (size_t)T.h * a.hpg) * D;
+                for (int x = lane; x < per_q; x += 32) {
+                    const int hh = x / C::CH, c = x % C::CH;   // C::CH is a power of two
+                    const int r = q * a.hpg + hh;
+                    ptx::cp_async16(qs + (c >> 3) * C::Q_PLANE + r * 128 + (((c & 7) ^ (r & 7)) << 4),
+                                    src_q + (size_t)hh * D + c * 8);
+                }
+            }
+            ptx::cp_async_mbar_arrive(&q_full[ib]);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&info_empty[ib]);   // done with ti[ib]
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < 3) {
         // ============================ loaders ============================
-        // Gather the tile's Q rows and every stage's K and V rows of the KV
-        // head (tokens from the shared-memory member lists).
-        const int ltid = tid - 32;   // 0 .. 63
+        // Gather every stage's K and V rows of the KV head (tokens from the
+        // shared-memory member lists).
         const int lw = warp - 1;
         int64_t gs = 0;
         for (int i = 0;; ++i) {
@@ -307,22 +352,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             if (!waitw(&info_full[ib], iph, 105u)) break;
             const int n_st = T.n_st;
             if (n_st < 0) break;
-            const int32_t* mem_l = reinterpret_cast<const int32_t*>(smem + C::OFF_MEM) + ib * TB_OPEN_MAX;
-            const int32_t* open_l = reinterpret_cast<const int32_t*>(smem + C::OFF_OPEN) + ib * TB_OPEN_MAX;
-
-            // ---- the tile's Q rows: row r = query r / hpg, head r % hpg ----
-            if (!waitw(&q_empty[ib], iph ^ 1u, 110u)) break;
-            unsigned char* qs = smem + C::OFF_Q + ib * C::Q_BYTES;
-            for (int x = ltid; x < TB_M * C::CH; x += 64) {
-                const int r = x / C::CH, c = x % C::CH;
-                const int q = r / a.hpg, hh = r % a.hpg;
-                const bool live = q < BA_Q && T.slot[q] >= 0;
-                const __nv_bfloat16* src =
-                    a.Q + ((size_t)(live ? T.row[q] : 0) * a.Hq + (size_t)T.h * a.hpg + hh) * D + c * 8;
-                unsigned char* dst = qs + (c >> 3) * C::Q_PLANE + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-                ptx::cp_async16_zfill(dst, live ? (const void*)src : (const void*)a.Q, live ? 16u : 0u);
-            }
-            ptx::cp_async_mbar_arrive(&q_full[ib]);
+            const int32_t* mem_l = mem_list(ib);
+            const int32_t* open_l = open_list(ib);
 
             // ---- K / V stages ----
             const size_t tstride = (size_t)a.Hkv * D;
@@ -330,8 +361,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             const __nv_bfloat16* Vb = a.V + ((size_t)T.b * ix.T_cap * a.Hkv + T.h) * D;
             bool stop = false;
             for (int s = 0; s < n_st; ++s, ++gs) {
-                const int slot = (int)(gs % TB_NS);
-                if (!waitw(&kv_empty[slot], (uint32_t)(((gs / TB_NS) & 1) ^ 1), 120u)) {
+                const int slot = (int)(gs % NS);
+                if (!waitw(&kv_empty[slot], (uint32_t)(((gs / NS) & 1) ^ 1), 120u)) {
                     stop = true;
                     break;
                 }
@@ -372,7 +403,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             const uint32_t q_base = ptx::smem_addr(smem + C::OFF_Q);
             const uint32_t kv_base = ptx::smem_addr(smem + C::OFF_KV);
             const uint32_t p_base = ptx::smem_addr(smem + C::OFF_P);
-            const uint32_t t_o = tmem + 128;
             for (int i = 0; !stop; ++i) {
                 const int ib = i & 1;
                 const uint32_t iph = (uint32_t)((i >> 1) & 1);
@@ -385,7 +415,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 int prev_slot = 0;
                 auto do_pv = [&](int s, int slot) -> bool {
                     if (!wait1(p_full, (uint32_t)(pv & 1), 220u)) return false;
-                    if (s == 0 && !wait1(o_empty, (uint32_t)((i & 1) ^ 1), 230u)) return false;
+                    if (s == 0 && !wait1(&o_empty[ib], iph ^ 1u, 230u)) return false;
+                    const uint32_t t_o = tmem + 128 + 128 * ib;
                     tb_fence_after();
                     ptx::fence_proxy_async();
                     const uint32_t va = kv_base + slot * C::STAGE + C::K_BYTES;
@@ -400,9 +431,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                     return true;
                 };
                 for (int s = 0; s < n_st; ++s, ++gs) {
-                    const int slot = (int)(gs % TB_NS);
+                    const int slot = (int)(gs % NS);
                     const int sb = (int)(gs & 1);
-                    if (!wait1(&kv_full[slot], (uint32_t)((gs / TB_NS) & 1), 240u) ||
+                    if (!wait1(&kv_full[slot], (uint32_t)((gs / NS) & 1), 240u) ||
                         !wait1(&s_empty[sb], (uint32_t)(((gs >> 1) & 1) ^ 1), 250u)) {
                         stop = true;
                         break;
@@ -427,13 +458,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                     prev_slot = slot;
                 }
                 if (stop || !do_pv(n_st - 1, prev_slot)) break;
-                tb_commit(o_full);
+                tb_commit(&o_full[ib]);
             }
             // nothing of this CTA may still run on the tensor cores at exit
             tb_commit(&fin_bar);
             ptx::mbar_wait_bounded(&fin_bar, 0, TB_WAIT);
         }
-    } else {
+    } else if (warp < 8) {
         // ============================ softmax ============================
         const int r = 32 * (warp & 3) + lane;               // row = TMEM lane
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
@@ -450,7 +481,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 if (lane == 0) ptx::mbar_arrive(&info_empty[ib]);
                 break;
             }
-            const int q = r / a.hpg, hh = r % a.hpg;
+            const int q = r / a.hpg;
             const bool live = q < BA_Q && T.slot[q] >= 0;
             const QRange rg = live ? T.rng[q] : QRange{0, 0, 0, 0};
             const int kbeg = T.kbeg;
@@ -538,10 +569,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         float o[32];
-                        tb_ld32(tmem + lane_base + 128 + c * 32, o);
+                        tb_ld32(tmem + lane_base + 128 + 128 * ib + c * 32, o);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) o[j] *= alpha;
-                        tb_st32(tmem + lane_base + 128 + c * 32, o);
+                        tb_st32(tmem + lane_base + 128 + 128 * ib + c * 32, o);
                     }
                 }
 #pragma unroll
@@ -555,27 +586,55 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 ++pv;
             }
             if (stop) break;
-            // ---- the row's partial ----
-            if (!waitw(o_full, (uint32_t)(i & 1), 330u)) break;
+            // the row's (max, sum) for the epilogue warps
+            ml[ib * TB_M + r] = make_float2(m_run, l);
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(&ml_full[ib]);
+                ptx::mbar_arrive(&info_empty[ib]);
+            }
+        }
+    } else {
+        // ============================ epilogue ============================
+        // Warps 8-11 (TMEM lanes by warp % 4): each row's partial -- the
+        // unnormalised O row, max and sum -- once the tile's last P V MMA is
+        // done, while the softmax warps already work on the next tile.
+        const int r = 32 * (warp & 3) + lane;
+        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        for (int i = 0;; ++i) {
+            const int ib = i & 1;
+            const uint32_t iph = (uint32_t)((i >> 1) & 1);
+            if (!waitw(&info_full[ib], iph, 400u)) break;
+            const TileInfo& T = ti[ib];
+            if (T.n_st < 0) break;
+            const int q = r / a.hpg, hh = r % a.hpg;
+            const bool live = q < BA_Q && T.slot[q] >= 0;
+            if (!waitw(&ml_full[ib], iph, 410u) || !waitw(&o_full[ib], iph, 420u)) break;
             tb_fence_after();
-            constexpr int PS = D + 4;
-            float* pp = a.P.part + (((size_t)(live ? T.slot[q] : 0) * a.Hq) + (size_t)T.h * a.hpg + hh) * PS;
+            const float2 mlr = ml[ib * TB_M + r];
+            const size_t ph = ((size_t)(live ? T.slot[q] : 0) * a.Hq) + (size_t)T.h * a.hpg + hh;
+            __nv_bfloat16* po = a.P.part_o + ph * D;
+            // the row normalised by its own sum (a convex combination of V rows)
+            const float inv = (mlr.y > 0.f) ? 1.f / mlr.y : 0.f;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 float o[32];
-                tb_ld32(tmem + lane_base + 128 + c * 32, o);
+                tb_ld32(tmem + lane_base + 128 + 128 * ib + c * 32, o);
                 if (live) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        reinterpret_cast<float4*>(pp + c * 32)[j] =
-                            make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                    for (int j = 0; j < 4; ++j)
+                        reinterpret_cast<uint4*>(po + c * 32)[j] = make_uint4(
+                            ptx::pack_bf16(o[8 * j] * inv, o[8 * j + 1] * inv),
+                            ptx::pack_bf16(o[8 * j + 2] * inv, o[8 * j + 3] * inv),
+                            ptx::pack_bf16(o[8 * j + 4] * inv, o[8 * j + 5] * inv),
+                            ptx::pack_bf16(o[8 * j + 6] * inv, o[8 * j + 7] * inv));
                 }
             }
-            if (live) *reinterpret_cast<float2*>(pp + D) = make_float2(m_run, l);
+            if (live) a.P.part_ml[ph] = mlr;
             tb_fence_before();
             __syncwarp();
             if (lane == 0) {
-                ptx::mbar_arrive(o_empty);
+                ptx::mbar_arrive(&o_empty[ib]);
                 ptx::mbar_arrive(&info_empty[ib]);
             }
         }
@@ -584,7 +643,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     __syncthreads();
     if (warp == 3) {
         tb_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem)
                      : "memory");
     }
 }
@@ -594,25 +653,46 @@ bool bucket_attn_tc_supported(int Hq, int Hkv, int d, int G)
     return (d == 64 || d == 128) && Hq % Hkv == 0 && Hq / Hkv <= 8 && G <= TB_OPEN_MAX;
 }
 
-template <int D>
-static cudaError_t launch_tc_t(const BaArgs& a, cudaStream_t st)
+// Shared memory the device grants one block (opt-in maximum).
+static int smem_optin()
 {
-    using C = TbCfg<D>;
-    auto kern = bucket_attn_tc_kernel<D>;
-    cudaError_t e = ensure_smem_attr((const void*)kern, C::BYTES);
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return 0;
+    return v;
+}
+
+template <int D, int NS>
+static cudaError_t launch_tc_t(const BaArgs& a, int cap, cudaStream_t st)
+{
+    using C = TbCfg<D, NS>;
+    auto kern = bucket_attn_tc_kernel<D, NS>;
+    const int bytes = C::bytes(a.ix.G);
+    // the limit is raised once per device, for the largest block served
+    const int lim = C::bytes(TB_OPEN_MAX) < cap ? C::bytes(TB_OPEN_MAX) : cap;
+    if (bytes > lim) return cudaErrorInvalidConfiguration;
+    cudaError_t e = ensure_smem_attr((const void*)kern, lim);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, TB_THREADS, C::BYTES);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, TB_THREADS, bytes);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    kern<<<(unsigned)(sm_count() * per_sm), TB_THREADS, C::BYTES, st>>>(a);
+    kern<<<(unsigned)(sm_count() * per_sm), TB_THREADS, bytes, st>>>(a);
     note_launch();
     return cudaGetLastError();
 }
 
 cudaError_t launch_bucket_attn_tc(const BaArgs& a, int d, cudaStream_t st)
 {
-    return (d == 128) ? launch_tc_t<128>(a, st) : launch_tc_t<64>(a, st);
+    // a fourth K/V stage where the block's member lists leave room for it
+    constexpr int STATIC_SMEM = 1024;   // tile descriptions, flags (928 bytes; upper bound)
+    const int cap = smem_optin() - STATIC_SMEM;
+    if (d == 128)
+        return (TbCfg<128, 4>::bytes(a.ix.G) <= cap) ? launch_tc_t<128, 4>(a, cap, st)
+                                                       : launch_tc_t<128, 3>(a, cap, st);
+    return (TbCfg<64, 4>::bytes(a.ix.G) <= cap) ? launch_tc_t<64, 4>(a, cap, st)
+                                                  : launch_tc_t<64, 3>(a, cap, st);
 }
 
 }  // namespace lsa

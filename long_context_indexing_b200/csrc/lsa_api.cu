@@ -122,7 +122,7 @@ lsa_status run_select(const lsa_index* idx, const void* lq, PosSrc pos, int64_t 
 // partial slots of Hq * (d + 4) floats each.
 struct PrefillLayout {
     size_t indices, counts, sel, zero, row_n, row_base, gather, ent, ent2, bucket_off, tiles,
-        sorted, part, recs, total;
+        sorted, part, part_ml, recs, total;
     int64_t ent_cap, tile_cap, n_zero;
     bool bucket;
 };
@@ -155,7 +155,8 @@ PrefillLayout prefill_layout(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, 
         L.bucket_off = o; o += al256((size_t)nbt * 4);
         L.tiles = o;      o += al256((size_t)L.tile_cap * 8);
         L.sorted = o;     o += al256((size_t)ent_cap * 4);
-        L.part = o;       o += al256((size_t)ent_cap * Hq * (d + 4) * 4);
+        L.part = o;       o += al256((size_t)ent_cap * Hq * d * 2);
+        L.part_ml = o;    o += al256((size_t)ent_cap * Hq * 8);
         const int64_t n_wt = v.B * ((Nq + BA_Q - 1) / BA_Q);
         L.recs = o;       o += al256((size_t)(n_wt + L.tile_cap) * TILE_REC_BYTES);
     }
@@ -178,18 +179,23 @@ int64_t default_ent_cap(const lsa_index* idx, int64_t Nq, lsa_select_params sp)
 }
 
 // Largest slot count whose layout fits in ws_bytes (-1: not even zero slots).
+// The layout grows monotonically with the slot count, so a binary search over
+// the exact layout finds it (the recommended workspace gives exactly the
+// recommended slots).
 int64_t ent_cap_for(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d, lsa_select_params sp,
                     size_t ws_bytes)
 {
     const PrefillLayout L0 = prefill_layout(idx, Nq, Hq, Hkv, d, sp, 0);
     if (ws_bytes < L0.total) return -1;
     if (!L0.bucket) return 0;
-    const size_t per = (size_t)Hq * (d + 4) * 4 + 16 + 8 + 4 + 8 + 8 + 2 * TILE_REC_BYTES;
-    int64_t e = (int64_t)((ws_bytes - L0.total) / per);
-    const int64_t cap = idx->v.B * Nq * (KC + 1);
-    if (e > cap) e = cap;
-    while (e > 0 && prefill_layout(idx, Nq, Hq, Hkv, d, sp, e).total > ws_bytes) --e;
-    return e;
+    int64_t lo = 0, hi = idx->v.B * Nq * (KC + 1);
+    if (prefill_layout(idx, Nq, Hq, Hkv, d, sp, hi).total <= ws_bytes) return hi;
+    while (hi - lo > 1) {   // invariant: lo fits, hi does not
+        const int64_t mid = lo + (hi - lo) / 2;
+        if (prefill_layout(idx, Nq, Hq, Hkv, d, sp, mid).total <= ws_bytes) lo = mid;
+        else hi = mid;
+    }
+    return lo;
 }
 
 struct DecodeLayout {
@@ -522,7 +528,8 @@ lsa_status prefill_prepare(const lsa_index* idx, int64_t T_old, int64_t T_new, i
         P->tiles = (int2*)(base + L->tiles);
         P->tile_cap = L->tile_cap;
         P->sorted = (int32_t*)(base + L->sorted);
-        P->part = (float*)(base + L->part);
+        P->part_o = (__nv_bfloat16*)(base + L->part);
+        P->part_ml = (float2*)(base + L->part_ml);
         P->recs = (unsigned char*)(base + L->recs);
     }
     return LSA_OK;

@@ -127,7 +127,8 @@ struct BucketPlan {
     int2* tiles;          // [tile_cap] (bucket, tile number inside the bucket)
     int64_t tile_cap;
     int32_t* sorted;      // [ent_cap] partial slots grouped by bucket
-    float* part;          // [ent_cap][Hq][d+4] softmax partials
+    __nv_bfloat16* part_o; // [ent_cap][Hq][d] softmax partials, normalised by their own sum
+    float2* part_ml;       // [ent_cap][Hq] (max in log2 units, sum) of each partial
     unsigned char* recs;  // [window tiles + tile_cap] tile descriptions (TILE_REC_BYTES each)
 };
 constexpr int TILE_REC_BYTES = 448;

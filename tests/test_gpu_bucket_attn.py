@@ -150,3 +150,21 @@ def test_fallback_rows():
     w = _base(T=2048, nq=512, G=16, R=300)      # 128 buckets: more than one candidate set
     fb, _ = _run(w, seed=18, same_latent=True)
     assert fb > 0
+
+
+def test_blocks_too_large_for_the_tensor_core_tiles():
+    # 2560 pooled groups per block: the member lists do not fit the
+    # tensor-core kernel's shared memory, so the warp-MMA tile kernel runs
+    w = _base(T=23000, nq=600, p=1, G=2560, k=8, R=1200, W=40)
+    _run(w, seed=19)
+
+
+def test_recommended_workspace_gives_the_recommended_slots():
+    # 1.5 x (budget / mean bucket keys) + 2 slots per query row, capped at 65
+    w = _base()
+    gpu = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16)
+    nbytes = lsa.lsa_prefill_workspace_bytes(gpu, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S)
+    bk = w.p * w.G // w.k
+    per_row = min(65, (3 * w.R + 2 * bk - 1) // (2 * bk) + 2)
+    assert lsa.lsa_prefill_partial_slots(gpu, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S,
+                                         nbytes) == w.B * w.nq * per_row
