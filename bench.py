@@ -335,8 +335,9 @@ def run_lsa(args, rank, ws):
     achieved = floor / (attn_ms * 1e-3) / 1e9
     bucket = w.dtype == "bf16"
     traffic = _traffic_record("prefill_attend_" + args.workload)
-    roofline = {"kernel": ("lsa_prefill_attend: bucket_attn_kernel + plan, scatter, merge"
-                           if bucket else "lsa_prefill_attend: attn_f32_kernel"),
+    roofline = {"kernel": ("lsa_prefill_attend: bucket tiles (plan, scatter, tile records, "
+                           "bucket_attn_tc_kernel, merge)" if bucket
+                           else "lsa_prefill_attend: attn_f32_kernel"),
                 "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
