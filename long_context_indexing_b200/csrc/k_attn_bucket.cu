@@ -249,7 +249,6 @@ __global__ void __launch_bounds__(BA_THREADS, LSA_BA_MIN_BLOCKS) bucket_attn_ker
 {
     using C = BaCfg<D>;
     constexpr int KSTEPS = D / 16;
-    constexpr int PS = D + 4;
     extern __shared__ __align__(128) unsigned char smem[];
     int32_t* mem_list = reinterpret_cast<int32_t*>(smem + C::RING);    // [G] closed members
     int32_t* open_list = mem_list + a.ix.G;                             // [G] open members

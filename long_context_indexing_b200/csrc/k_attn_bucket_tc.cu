@@ -46,10 +46,19 @@ namespace lsa {
 constexpr int TB_M = 128;            // MMA rows: BA_Q queries x 8 query heads
 constexpr int TB_N = 64;             // keys per stage
 constexpr int TB_OPEN_MAX = 2048;    // members of one bucket a tile can hold (block size bound)
+constexpr int TB_SB = 3;             // S buffers in TMEM: S runs up to two stages ahead of P V
+constexpr uint32_t TB_COL_O = TB_SB * 64;   // first TMEM column of the two O accumulators
 constexpr int TB_THREADS = 416;      // 13 warps
 constexpr uint32_t TB_WAIT = 1u << 22;
 
-template <int D, int NS>
+#ifndef LSA_TB_QB
+#define LSA_TB_QB 2          // Q buffers (2: the next tile's Q loads during this tile)
+#endif
+#ifndef LSA_TB_NS_MAX
+#define LSA_TB_NS_MAX 4      // K/V stages when shared memory allows (else 3)
+#endif
+
+template <int D, int NS, int QB>
 struct TbCfg {
     static constexpr int CH = D / 8;                    // 16-byte chunks per row
     static constexpr int Q_PLANE = TB_M * 128;          // 64 dims of 128 rows
@@ -58,11 +67,11 @@ struct TbCfg {
     static constexpr int K_BYTES = (D / 64) * KV_PLANE;
     static constexpr int STAGE = 2 * K_BYTES;           // K then V
     static constexpr int P_BYTES = TB_M * TB_N * 2;
-    static constexpr int OFF_Q = 0;                     // two buffers
-    static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;  // NS stages
+    static constexpr int OFF_Q = 0;                     // QB buffers
+    static constexpr int OFF_KV = OFF_Q + QB * Q_BYTES; // NS stages
     static constexpr int OFF_P = OFF_KV + NS * STAGE;
     static constexpr int OFF_BAR = OFF_P + P_BYTES;
-    static constexpr int NBAR = 20 + 2 * NS;
+    static constexpr int NBAR = 22 + 2 * NS;
     static constexpr int OFF_ML = OFF_BAR + NBAR * 8;      // [2][128] (max, sum) per row
     static constexpr int OFF_LISTS = OFF_ML + 2 * TB_M * 8;   // then 4 member lists of G ints
     // dynamic shared memory for a block of G pooled groups (+ alignment slack)
@@ -174,10 +183,10 @@ __device__ __forceinline__ void tb_st32(uint32_t taddr, const float* v)
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-template <int D, int NS>
+template <int D, int NS, int QB>
 __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
 {
-    using C = TbCfg<D, NS>;
+    using C = TbCfg<D, NS, QB>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -185,14 +194,14 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     uint64_t* info_empty = bars + 2;     // [2]
     uint64_t* q_full = bars + 4;         // [2]
     uint64_t* q_empty = bars + 6;        // [2]
-    uint64_t* s_full = bars + 8;         // [2]
-    uint64_t* s_empty = bars + 10;       // [2]
-    uint64_t* p_full = bars + 12;
-    uint64_t* p_empty = bars + 13;
-    uint64_t* o_full = bars + 14;        // [2] (two O accumulators, by item parity)
-    uint64_t* o_empty = bars + 16;       // [2]
-    uint64_t* ml_full = bars + 18;       // [2]
-    uint64_t* kv_full = bars + 20;       // [NS]
+    uint64_t* s_full = bars + 8;         // [TB_SB]
+    uint64_t* s_empty = bars + 11;       // [TB_SB]
+    uint64_t* p_full = bars + 14;
+    uint64_t* p_empty = bars + 15;
+    uint64_t* o_full = bars + 16;        // [2] (two O accumulators, by item parity)
+    uint64_t* o_empty = bars + 18;       // [2]
+    uint64_t* ml_full = bars + 20;       // [2]
+    uint64_t* kv_full = bars + 22;       // [NS]
     float2* ml = reinterpret_cast<float2*>(smem + C::OFF_ML);   // [2][TB_M]
     uint64_t* kv_empty = kv_full + NS;
     const int lcap = (a.ix.G + 3) & ~3;  // ints per member list
@@ -221,6 +230,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             ptx::mbar_init(&ml_full[i], 4);
             ptx::mbar_init(&q_full[i], 32);        // every Q-loader lane's cp.async arrival
             ptx::mbar_init(&q_empty[i], 1);
+        }
+        for (int i = 0; i < TB_SB; ++i) {
             ptx::mbar_init(&s_full[i], 1);
             ptx::mbar_init(&s_empty[i], 4);
         }
@@ -317,8 +328,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             const TileInfo& T = ti[ib];
             if (!waitw(&info_full[ib], iph, 130u)) break;
             if (T.n_st < 0) break;
-            if (!waitw(&q_empty[ib], iph ^ 1u, 140u)) break;
-            unsigned char* qs = smem + C::OFF_Q + ib * C::Q_BYTES;
+            const int qb = i % QB;
+            if (!waitw(&q_empty[qb], (uint32_t)(((i / QB) & 1) ^ 1), 140u)) break;
+            unsigned char* qs = smem + C::OFF_Q + qb * C::Q_BYTES;
             // Query q's hpg head rows are contiguous (hpg * D bf16) and fill MMA
             // rows q*hpg .. q*hpg+hpg-1.  Rows of empty query positions are
             // not loaded: every key of such a row is masked, so whatever the
@@ -334,7 +346,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                                     src_q + (size_t)hh * D + c * 8);
                 }
             }
-            ptx::cp_async_mbar_arrive(&q_full[ib]);
+            ptx::cp_async_mbar_arrive(&q_full[qb]);
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&info_empty[ib]);   // done with ti[ib]
         }
@@ -403,62 +415,99 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             const uint32_t q_base = ptx::smem_addr(smem + C::OFF_Q);
             const uint32_t kv_base = ptx::smem_addr(smem + C::OFF_KV);
             const uint32_t p_base = ptx::smem_addr(smem + C::OFF_P);
-            for (int i = 0; !stop; ++i) {
-                const int ib = i & 1;
-                const uint32_t iph = (uint32_t)((i >> 1) & 1);
-                if (!wait1(&info_full[ib], iph, 200u)) break;
-                const int n_st = ti[ib].n_st;
-                ptx::mbar_arrive(&info_empty[ib]);
-                if (n_st < 0) break;
-                if (!wait1(&q_full[ib], iph, 210u)) break;
-                const uint32_t qa = q_base + ib * C::Q_BYTES;
-                int prev_slot = 0;
-                auto do_pv = [&](int s, int slot) -> bool {
-                    if (!wait1(p_full, (uint32_t)(pv & 1), 220u)) return false;
-                    if (s == 0 && !wait1(&o_empty[ib], iph ^ 1u, 230u)) return false;
-                    const uint32_t t_o = tmem + 128 + 128 * ib;
+            // Two cursors over one stream of stages (all items in order). The
+            // issuer polls: a P V MMA goes out as soon as its P is ready; an S
+            // MMA goes out, up to TB_SB - 1 stages ahead of the P V cursor and
+            // across item boundaries, as soon as its inputs have landed.  The S
+            // cursor starts a new item only while it is at most one item ahead
+            // of the P V cursor (item i + 2's description is written only after
+            // item i's epilogue, which needs item i's last P V).
+            int iS = 0, sS = 0, nS = 0;         // S cursor: item, stage, the item's stages
+            int iP = 0, sP = 0;                 // P V cursor
+            int64_t gP = 0;                     // global stage of the P V cursor (gs: S cursor)
+            int nst[2] = {0, 0};                // stages of the (at most two) open items
+            bool s_done = false, item_open = false;
+            uint32_t idle = 0;
+            while (!stop) {
+                if (abort_flag) break;
+                bool progress = false;
+                // ---- P V for the oldest stage whose P is ready ----
+                if (gP < gs && ptx::mbar_test(p_full, (uint32_t)(pv & 1)) &&
+                    (sP > 0 || ptx::mbar_test(&o_empty[iP & 1], (uint32_t)(((iP >> 1) & 1) ^ 1)))) {
+                    const int ib = iP & 1;
+                    const int slot = (int)(gP % NS);
+                    // P was fenced to the async proxy by the softmax threads before
+                    // they arrived on p_full
                     tb_fence_after();
-                    ptx::fence_proxy_async();
-                    const uint32_t va = kv_base + slot * C::STAGE + C::K_BYTES;
+                    const uint32_t t_o = tmem + TB_COL_O + 128 * ib;
+                    const uint64_t pd = tb_desc(p_base, 16, 1024);
+                    const uint64_t vd =
+                        tb_desc(kv_base + slot * C::STAGE + C::K_BYTES, C::KV_PLANE, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < TB_N / 16; ++kk)
-                        tb_mma(t_o, tb_desc(p_base + kk * 32, 16, 1024),
-                               tb_desc(va + kk * 2048, C::KV_PLANE, 1024), C::IDESC_PV,
-                               (s > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < TB_N / 16; ++kk)   // start address in 16-byte units
+                        tb_mma(t_o, pd + (uint64_t)(kk * 2), vd + (uint64_t)(kk * 128), C::IDESC_PV,
+                               (sP > 0 || kk > 0) ? 1u : 0u);
                     tb_commit(&kv_empty[slot]);
                     tb_commit(p_empty);
                     ++pv;
-                    return true;
-                };
-                for (int s = 0; s < n_st; ++s, ++gs) {
-                    const int slot = (int)(gs % NS);
-                    const int sb = (int)(gs & 1);
-                    if (!wait1(&kv_full[slot], (uint32_t)((gs / NS) & 1), 240u) ||
-                        !wait1(&s_empty[sb], (uint32_t)(((gs >> 1) & 1) ^ 1), 250u)) {
-                        stop = true;
-                        break;
+                    if (sP == nst[ib] - 1) tb_commit(&o_full[ib]);
+                    ++gP;
+                    if (++sP == nst[ib]) {
+                        ++iP;
+                        sP = 0;
                     }
-                    tb_fence_after();
-                    ptx::fence_proxy_async();
-                    const uint32_t ka = kv_base + slot * C::STAGE;
-#pragma unroll
-                    for (int kk = 0; kk < (int)C::KSTEPS; ++kk) {
-                        const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
-                        tb_mma(tmem + sb * TB_N,
-                               tb_desc(qa + (kk >> 2) * C::Q_PLANE + off, 16, 1024),
-                               tb_desc(ka + (kk >> 2) * C::KV_PLANE + off, 16, 1024), C::IDESC_S,
-                               kk > 0 ? 1u : 0u);
-                    }
-                    tb_commit(&s_full[sb]);
-                    if (s == n_st - 1) tb_commit(&q_empty[ib]);
-                    if (s > 0 && !do_pv(s - 1, prev_slot)) {
-                        stop = true;
-                        break;
-                    }
-                    prev_slot = slot;
+                    progress = true;
                 }
-                if (stop || !do_pv(n_st - 1, prev_slot)) break;
-                tb_commit(&o_full[ib]);
+                // ---- the next S, if its inputs are ready ----
+                if (!s_done && gs - gP < TB_SB && (sS > 0 || iS <= iP + 1)) {
+                    const int ib = iS & 1;
+                    const uint32_t iph = (uint32_t)((iS >> 1) & 1);
+                    if (sS == 0 && !item_open && ptx::mbar_test(&info_full[ib], iph)) {
+                        nS = ti[ib].n_st;
+                        ptx::mbar_arrive(&info_empty[ib]);
+                        if (nS < 0) {
+                            s_done = true;
+                        } else {
+                            nst[ib] = nS;
+                            item_open = true;
+                        }
+                        progress = true;
+                    }
+                    const int slot = (int)(gs % NS);
+                    const int sb = (int)(gs % TB_SB);
+                    const int qb = iS % QB;
+                    if (item_open && (sS > 0 || ptx::mbar_test(&q_full[qb], (uint32_t)((iS / QB) & 1))) &&
+                        ptx::mbar_test(&kv_full[slot], (uint32_t)((gs / NS) & 1)) &&
+                        ptx::mbar_test(&s_empty[sb], (uint32_t)(((gs / TB_SB) & 1) ^ 1))) {
+                        tb_fence_after();
+                        ptx::fence_proxy_async();   // the loaders' cp.async rows, to the async proxy
+                        const uint64_t qd = tb_desc(q_base + qb * C::Q_BYTES, 16, 1024);
+                        const uint64_t kd = tb_desc(kv_base + slot * C::STAGE, 16, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < (int)C::KSTEPS; ++kk) {
+                            // k-step kk: plane kk / 4, +32 bytes per step inside the row
+                            const uint64_t qo = (uint64_t)(((kk >> 2) * C::Q_PLANE + (kk & 3) * 32) >> 4);
+                            const uint64_t ko = (uint64_t)(((kk >> 2) * C::KV_PLANE + (kk & 3) * 32) >> 4);
+                            tb_mma(tmem + sb * TB_N, qd + qo, kd + ko, C::IDESC_S, kk > 0 ? 1u : 0u);
+                        }
+                        tb_commit(&s_full[sb]);
+                        if (sS == nS - 1) tb_commit(&q_empty[qb]);
+                        ++gs;
+                        if (++sS == nS) {
+                            ++iS;
+                            sS = 0;
+                            item_open = false;
+                        }
+                        progress = true;
+                    }
+                }
+                if (s_done && gP == gs) break;      // every item's P V is out
+                if (progress) {
+                    idle = 0;
+                } else if (++idle > (TB_WAIT << 3)) {   // nothing moved for a long time
+                    fail(260u);
+                    break;
+                }
             }
             // nothing of this CTA may still run on the tensor cores at exit
             tb_commit(&fin_bar);
@@ -488,8 +537,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             float m_run = -INFINITY, l = 0.f;
             bool stop = false;
             for (int s = 0; s < n_st; ++s, ++gs) {
-                const int sb = (int)(gs & 1);
-                if (!waitw(&s_full[sb], (uint32_t)((gs >> 1) & 1), 310u)) {
+                const int sb = (int)(gs % TB_SB);
+                if (!waitw(&s_full[sb], (uint32_t)((gs / TB_SB) & 1), 310u)) {
                     stop = true;
                     break;
                 }
@@ -569,10 +618,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         float o[32];
-                        tb_ld32(tmem + lane_base + 128 + 128 * ib + c * 32, o);
+                        tb_ld32(tmem + lane_base + TB_COL_O + 128 * ib + c * 32, o);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) o[j] *= alpha;
-                        tb_st32(tmem + lane_base + 128 + 128 * ib + c * 32, o);
+                        tb_st32(tmem + lane_base + TB_COL_O + 128 * ib + c * 32, o);
                     }
                 }
 #pragma unroll
@@ -619,7 +668,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 float o[32];
-                tb_ld32(tmem + lane_base + 128 + 128 * ib + c * 32, o);
+                tb_ld32(tmem + lane_base + TB_COL_O + 128 * ib + c * 32, o);
                 if (live) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
@@ -663,11 +712,11 @@ static int smem_optin()
     return v;
 }
 
-template <int D, int NS>
+template <int D, int NS, int QB>
 static cudaError_t launch_tc_t(const BaArgs& a, int cap, cudaStream_t st)
 {
-    using C = TbCfg<D, NS>;
-    auto kern = bucket_attn_tc_kernel<D, NS>;
+    using C = TbCfg<D, NS, QB>;
+    auto kern = bucket_attn_tc_kernel<D, NS, QB>;
     const int bytes = C::bytes(a.ix.G);
     // the limit is raised once per device, for the largest block served
     const int lim = C::bytes(TB_OPEN_MAX) < cap ? C::bytes(TB_OPEN_MAX) : cap;
@@ -685,14 +734,15 @@ static cudaError_t launch_tc_t(const BaArgs& a, int cap, cudaStream_t st)
 
 cudaError_t launch_bucket_attn_tc(const BaArgs& a, int d, cudaStream_t st)
 {
-    // a fourth K/V stage where the block's member lists leave room for it
+    // the deeper K/V ring where the block's member lists leave room for it
     constexpr int STATIC_SMEM = 1024;   // tile descriptions, flags (928 bytes; upper bound)
+    constexpr int NSX = LSA_TB_NS_MAX, QB = LSA_TB_QB;
     const int cap = smem_optin() - STATIC_SMEM;
     if (d == 128)
-        return (TbCfg<128, 4>::bytes(a.ix.G) <= cap) ? launch_tc_t<128, 4>(a, cap, st)
-                                                       : launch_tc_t<128, 3>(a, cap, st);
-    return (TbCfg<64, 4>::bytes(a.ix.G) <= cap) ? launch_tc_t<64, 4>(a, cap, st)
-                                                  : launch_tc_t<64, 3>(a, cap, st);
+        return (TbCfg<128, NSX, QB>::bytes(a.ix.G) <= cap) ? launch_tc_t<128, NSX, QB>(a, cap, st)
+                                                            : launch_tc_t<128, 3, QB>(a, cap, st);
+    return (TbCfg<64, NSX, QB>::bytes(a.ix.G) <= cap) ? launch_tc_t<64, NSX, QB>(a, cap, st)
+                                                       : launch_tc_t<64, 3, QB>(a, cap, st);
 }
 
 }  // namespace lsa
