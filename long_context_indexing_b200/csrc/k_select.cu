@@ -708,6 +708,26 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     const int64_t b = blockIdx.y, i = blockIdx.x;
     const int64_t row = b * Nq + i;
     const int64_t pq = pos.at(b, Nq, i);
+    if (ws.app_n > 0 && i == 0 && threadIdx.x == 0) {
+        // decode: the best of the sliced nearest-centroid searches (highest
+        // exact score, lowest bucket on ties) joins the open block.  The group
+        // lies inside this query's window, so the selection below never reads
+        // it; the barriers before any open-list read order it anyway.
+        const int o = ws.app_slot[b];
+        if (o >= 0) {
+            double bs = -INFINITY;
+            int bg = 0x7fffffff;
+            for (int x = 0; x < ws.app_n; ++x) {
+                const double sx = ws.app_score[b * ws.app_n + x];
+                const int gx = ws.app_g[b * ws.app_n + x];
+                if (sx > bs || (sx == bs && gx < bg)) {
+                    bs = sx;
+                    bg = gx;
+                }
+            }
+            if (bg != 0x7fffffff) ix.open_bucket[b * ix.G + o] = bg;
+        }
+    }
     load_query(q_s, lq, row);
     int nc;
     float tau;
@@ -978,70 +998,158 @@ __global__ void __launch_bounds__(FB_THREADS) select_fallback_kernel(IndexView i
 }
 
 // ---------------------------------------------------------------------------
-// Decode step, part 1.  grid (B, 2): role 0 appends sequence b's new token,
-// role 1 nominates candidates for its query.  The two are independent: a
-// pooled group that completes at position pos holds keys >= pos - p + 1,
-// which lie inside the recent window (W >= p - 1), so no selection made at
-// pos can read them.
-// Append: the new latent/key/value rows go to position pos of the caches; if
-// (pos + 1) % p == 0 the group j = (pos + 1)/p - 1 is pooled (binary32, left
-// to right), normalised (binary64 norm) and assigned to the closed bucket of
-// largest exact <u, c_g> (fp32 centroids, lowest g on ties).  A group beyond
-// the open block records DEV_OPEN_FULL and is not appended.
+// Decode step, part 1.  grid (B, n_slice): CTA (b, s) scores slice s of
+// sequence b's eligible buckets and, when b's new token completes a pooled
+// group, searches slice s of the closed buckets for the group's nearest
+// centroid.  The two are independent: a pooled group that completes at
+// position pos holds keys >= pos - p + 1, which lie inside the recent window
+// (W >= p - 1), so no selection made at pos can read them.
+// Scores: binary32 FMA over the retrieval copy (16-byte loads, 8 lanes per
+// row), written as fp16 with the fp16 maximum of every 32-score chunk -- the
+// same row the tensor-core scorer writes, which the fill nominates from.
+// Append: slice 0 writes the new latent/key/value rows at pos; every slice
+// pools the completed group j = (pos+1)/p - 1 (binary32, left to right; the
+// group's last row comes from the new latent row itself), normalises it
+// (binary64 norm) and takes the closed bucket of largest exact <u, c_g> in its
+// range (fp32 centroids, lowest g on ties); the fill takes the best of the
+// slices.  A group beyond the open block records DEV_OPEN_FULL.
 // ---------------------------------------------------------------------------
+constexpr int DEC_THREADS = 256;
+
 template <typename T>
-__global__ void __launch_bounds__(SIMT_THREADS) decode_prep_kernel(
+__global__ void __launch_bounds__(DEC_THREADS) decode_prep_kernel(
     IndexView ix, int64_t n_blk, T* latK, T* Kc, T* Vc, const T* nlk, const T* nk, const T* nv,
-    const T* lq, const int32_t* pos, int Hkv, int d, int W, SelectWs ws, uint32_t* attn_counter,
-    int counters_per_seq)
+    const T* lq, const int32_t* pos, int Hkv, int d, int W, SelectWs ws, double* app_score,
+    int32_t* app_g, int32_t* app_slot, int n_slice, uint32_t* attn_counter, int counters_per_seq)
 {
-    extern __shared__ float sc[];
     __shared__ float q_s[DL];
     __shared__ float x_s[DL];
+    __shared__ float sc[DEC_THREADS * 4];          // this slice's fp32 scores (<= 1024)
+    __shared__ float tile[64 * (DL + 1)];          // exact search: 64 centroid rows
     __shared__ double nrm_s;
-    __shared__ double rs[SIMT_THREADS / 32];
-    __shared__ int rg[SIMT_THREADS / 32];
+    __shared__ double rs[DEC_THREADS / 32];
+    __shared__ int rg[DEC_THREADS / 32];
     const int64_t b = blockIdx.x;
+    const int sl = blockIdx.y;
     const int64_t pq = pos[b];
-    if (blockIdx.y == 1) {
-        if (b == 0 && threadIdx.x == 0) *ws.fb_count = 0;
-        load_query(q_s, lq, b);
-        __syncthreads();
-        simt_nominate(ix, n_blk, q_s, b, b, pq, W, ws, sc);
-        return;
-    }
-    for (int x = threadIdx.x; x < counters_per_seq; x += blockDim.x)
-        attn_counter[b * counters_per_seq + x] = 0u;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (b == 0 && sl == 0 && threadIdx.x == 0) *ws.fb_count = 0;
     if (pq < 0 || pq >= ix.T_cap) {
-        if (threadIdx.x == 0) dev_error(ix.status, DEV_BAD_INDEX, (uint32_t)b);
+        if (sl == 0 && threadIdx.x == 0) {
+            dev_error(ix.status, DEV_BAD_INDEX, (uint32_t)b);
+            app_slot[b] = -1;
+        }
         return;
     }
-    T* lrow = latK + (b * ix.T_cap + pq) * DL;
-    for (int x = threadIdx.x; x < DL; x += blockDim.x) lrow[x] = nlk[b * DL + x];
-    const int64_t kvn = (int64_t)Hkv * d;
-    T* krow = Kc + (b * ix.T_cap + pq) * kvn;
-    T* vrow = Vc + (b * ix.T_cap + pq) * kvn;
-    for (int64_t x = threadIdx.x; x < kvn; x += blockDim.x) {
-        krow[x] = nk[b * kvn + x];
-        vrow[x] = nv[b * kvn + x];
+
+    // ---------------- scores of this slice ----------------
+    {
+        const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
+        const int64_t per = (((ix.NBK + n_slice - 1) / n_slice) + 31) / 32 * 32;
+        const int64_t g0 = sl * per;
+        const int64_t g1 = (g0 + per < nb) ? g0 + per : nb;
+        if (g0 < g1) {
+            load_query(q_s, lq, b);
+            __syncthreads();
+            // 8 lanes per 128-byte bf16 row (16 lanes per fp32 row), rows of the
+            // slice spread over the warps
+            const int n = (int)(g1 - g0);
+            if (ix.dtype == LSA_BF16) {
+                constexpr int LPR = 8, RPI = 32 / LPR;
+                const int sub = lane % LPR, rsel = lane / LPR;
+                float q[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) q[e] = q_s[sub * 8 + e];
+                const uint4* base = reinterpret_cast<const uint4*>(
+                    (const __nv_bfloat16*)ix.cent_rt + (b * ix.NBK + g0) * DL);
+                for (int r0 = warp * RPI; r0 < n; r0 += (DEC_THREADS / 32) * RPI) {
+                    const int r = r0 + rsel;
+                    const uint4 raw = (r < n) ? __ldg(base + (int64_t)r * (DL / 8) + sub) : make_uint4(0, 0, 0, 0);
+                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+                    float acc = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h[e]);
+                        acc = fmaf(q[2 * e], f.x, acc);
+                        acc = fmaf(q[2 * e + 1], f.y, acc);
+                    }
+#pragma unroll
+                    for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                    if (sub == 0 && r < n) sc[r] = acc;
+                }
+            } else {
+                constexpr int LPR = 16, RPI = 32 / LPR;
+                const int sub = lane % LPR, rsel = lane / LPR;
+                float q[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) q[e] = q_s[sub * 4 + e];
+                const float4* base = reinterpret_cast<const float4*>(
+                    (const float*)ix.cent_rt + (b * ix.NBK + g0) * DL);
+                for (int r0 = warp * RPI; r0 < n; r0 += (DEC_THREADS / 32) * RPI) {
+                    const int r = r0 + rsel;
+                    const float4 f = (r < n) ? __ldg(base + (int64_t)r * (DL / 4) + sub) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    float acc = fmaf(q[0], f.x, 0.f);
+                    acc = fmaf(q[1], f.y, acc);
+                    acc = fmaf(q[2], f.z, acc);
+                    acc = fmaf(q[3], f.w, acc);
+#pragma unroll
+                    for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                    if (sub == 0 && r < n) sc[r] = acc;
+                }
+            }
+            __syncthreads();
+            __half* srow = ws.scores + b * ws.score_ld + g0;
+            __half* crow = ws.cmax + b * (ws.score_ld / 32) + g0 / 32;
+            for (int r = threadIdx.x; r < n; r += DEC_THREADS) srow[r] = __float2half_rn(sc[r]);
+            // chunk maxima (fp16 rounding is monotone: the rounded maximum is
+            // the maximum of the rounded scores)
+            for (int c = warp; c * 32 < n; c += DEC_THREADS / 32) {
+                const int r = c * 32 + lane;
+                float m = (r < n) ? sc[r] : -INFINITY;
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (lane == 0) crow[c] = __float2half_rn(m);
+            }
+        }
+    }
+
+    // ---------------- append ----------------
+    if (sl == 0) {
+        for (int x = threadIdx.x; x < counters_per_seq; x += blockDim.x)
+            attn_counter[b * counters_per_seq + x] = 0u;
+        T* lrow = latK + (b * ix.T_cap + pq) * DL;
+        for (int x = threadIdx.x; x < DL; x += blockDim.x) lrow[x] = nlk[b * DL + x];
+        const int64_t kvn = (int64_t)Hkv * d;
+        T* krow = Kc + (b * ix.T_cap + pq) * kvn;
+        T* vrow = Vc + (b * ix.T_cap + pq) * kvn;
+        for (int64_t x = threadIdx.x; x < kvn; x += blockDim.x) {
+            krow[x] = nk[b * kvn + x];
+            vrow[x] = nv[b * kvn + x];
+        }
     }
     const int p = ix.p;
-    if ((pq + 1) % p != 0) return;
     const int64_t j = (pq + 1) / p - 1;
     const int64_t o = j - n_blk * ix.G;
-    if (n_blk < 1 || o < 0 || o >= ix.G || j >= ix.NP) {
-        if (threadIdx.x == 0) dev_error(ix.status, DEV_OPEN_FULL, (uint32_t)b);
+    if ((pq + 1) % p != 0) {
+        if (sl == 0 && threadIdx.x == 0) app_slot[b] = -1;
         return;
     }
-    __syncthreads();   // the new latent row is visible to the whole CTA
+    if (n_blk < 1 || o < 0 || o >= ix.G || j >= ix.NP) {
+        if (sl == 0 && threadIdx.x == 0) {
+            dev_error(ix.status, DEV_OPEN_FULL, (uint32_t)b);
+            app_slot[b] = -1;
+        }
+        return;
+    }
     if (threadIdx.x < DL) {
+        // rows j*p .. pos-1 from the cache, row pos from the new latent row
         const int i = threadIdx.x;
         const T* rows = latK + (b * ix.T_cap + j * p) * DL;
-        float s = load_elt(rows + i);
-        for (int r = 1; r < p; ++r) s = __fadd_rn(s, load_elt(rows + (int64_t)r * DL + i));
+        float s = (p == 1) ? load_elt(nlk + b * DL + i) : load_elt(rows + i);
+        for (int r = 1; r < p; ++r)
+            s = __fadd_rn(s, load_elt((r == p - 1) ? nlk + b * DL + i : rows + (int64_t)r * DL + i));
         const float xv = __fdiv_rn(s, (float)p);
         x_s[i] = xv;
-        ix.pooled[(b * ix.NP + j) * DL + i] = xv;
+        if (sl == 0) ix.pooled[(b * ix.NP + j) * DL + i] = xv;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -1053,23 +1161,24 @@ __global__ void __launch_bounds__(SIMT_THREADS) decode_prep_kernel(
     if (threadIdx.x < DL) {
         const int i = threadIdx.x;
         const float u = (nrm_s != 0.0) ? __double2float_rn(__ddiv_rn((double)x_s[i], nrm_s)) : 0.f;
-        ix.unit[(b * ix.NP + j) * DL + i] = u;
+        if (sl == 0) ix.unit[(b * ix.NP + j) * DL + i] = u;
         q_s[i] = u;   // reuse as the unit vector
     }
     __syncthreads();
-    // Exact scores against every closed centroid.  Tiles of SIMT_THREADS
-    // centroid rows are staged into shared memory with coalesced 16-byte loads
-    // (row pitch DL + 1 floats, so that thread t reading row t hits its own
-    // bank); each thread then sums its row in ascending dimension.
+    // Exact scores against this slice of the closed centroids: tiles of 64
+    // rows staged with coalesced 16-byte loads (row pitch DL + 1 floats, so
+    // that thread t reading row t hits its own bank); one thread per row sums
+    // it in ascending dimension.
     const float* cent = ix.cent + b * ix.NBK * DL;
     const int64_t nbk = n_blk * ix.k;
-    float* tile = sc;                                   // [SIMT_THREADS][DL + 1]
+    const int64_t per2 = (nbk + n_slice - 1) / n_slice;
+    const int64_t c0 = sl * per2, c1 = (c0 + per2 < nbk) ? c0 + per2 : nbk;
     double bs = -INFINITY;
     int bg = 0x7fffffff;
-    for (int64_t g0 = 0; g0 < nbk; g0 += SIMT_THREADS) {
-        const int rows = (int)((nbk - g0) < SIMT_THREADS ? (nbk - g0) : SIMT_THREADS);
+    for (int64_t t0 = c0; t0 < c1; t0 += 64) {
+        const int rows = (int)((c1 - t0) < 64 ? (c1 - t0) : 64);
         __syncthreads();
-        const float4* src = reinterpret_cast<const float4*>(cent + g0 * DL);
+        const float4* src = reinterpret_cast<const float4*>(cent + t0 * DL);
         for (int x = threadIdx.x; x < rows * (DL / 4); x += blockDim.x) {
             const float4 f = src[x];
             const int r = x / (DL / 4), c = (x % (DL / 4)) * 4;
@@ -1085,7 +1194,7 @@ __global__ void __launch_bounds__(SIMT_THREADS) decode_prep_kernel(
             double s = 0.0;
 #pragma unroll 16
             for (int i = 0; i < DL; ++i) s = __fma_rn((double)q_s[i], (double)c[i], s);
-            const int g = (int)(g0 + threadIdx.x);
+            const int g = (int)(t0 + threadIdx.x);
             if (s > bs || (s == bs && g < bg)) {
                 bs = s;
                 bg = g;
@@ -1100,49 +1209,45 @@ __global__ void __launch_bounds__(SIMT_THREADS) decode_prep_kernel(
             bg = og;
         }
     }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (lane == 0) {
         rs[warp] = bs;
         rg[warp] = bg;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        for (int w = 1; w < SIMT_THREADS / 32; ++w)
+        for (int w = 1; w < DEC_THREADS / 32; ++w)
             if (rs[w] > bs || (rs[w] == bs && rg[w] < bg)) {
                 bs = rs[w];
                 bg = rg[w];
             }
-        ix.open_bucket[b * ix.G + o] = bg;
+        app_score[b * n_slice + sl] = bs;
+        app_g[b * n_slice + sl] = bg;
+        if (sl == 0) app_slot[b] = (int32_t)o;
     }
 }
 
 cudaError_t launch_decode_prep(const IndexView& ix, int64_t n_blk, void* latent_K, void* K,
                                void* V, const void* new_latent_k, const void* new_k,
                                const void* new_v, const void* latent_q, const int32_t* pos,
-                               int Hkv, int d, int W, const SelectWs& ws, uint32_t* attn_counter,
-                               int counters_per_seq, cudaStream_t st)
+                               int Hkv, int d, int W, const SelectWs& ws, double* app_score,
+                               int32_t* app_g, int32_t* app_slot, int n_slice,
+                               uint32_t* attn_counter, int counters_per_seq, cudaStream_t st)
 {
-    size_t smem = (size_t)n_blk * ix.k * sizeof(float);          // nominator scores
-    const size_t tile = (size_t)SIMT_THREADS * (DL + 1) * sizeof(float);  // exact-search tile
-    if (smem < tile) smem = tile;
-    dim3 grid((unsigned)ix.B, 2);
-    cudaError_t e;
+    if (n_slice < 1 || (ix.NBK + n_slice - 1) / n_slice > DEC_THREADS * 4 - 31)
+        return cudaErrorInvalidValue;   // a slice's scores must fit the shared buffer
+    dim3 grid((unsigned)ix.B, (unsigned)n_slice);
     if (ix.dtype == LSA_BF16) {
         typedef __nv_bfloat16 T;
-        e = ensure_smem_attr((const void*)decode_prep_kernel<T>, (int)SIMT_SMEM_MAX);
-        if (e != cudaSuccess) return e;
-        decode_prep_kernel<T><<<grid, SIMT_THREADS, smem, st>>>(
+        decode_prep_kernel<T><<<grid, DEC_THREADS, 0, st>>>(
             ix, n_blk, (T*)latent_K, (T*)K, (T*)V, (const T*)new_latent_k, (const T*)new_k,
-            (const T*)new_v, (const T*)latent_q, pos, Hkv, d, W, ws, attn_counter,
-            counters_per_seq);
+            (const T*)new_v, (const T*)latent_q, pos, Hkv, d, W, ws, app_score, app_g, app_slot,
+            n_slice, attn_counter, counters_per_seq);
     } else {
         typedef float T;
-        e = ensure_smem_attr((const void*)decode_prep_kernel<T>, (int)SIMT_SMEM_MAX);
-        if (e != cudaSuccess) return e;
-        decode_prep_kernel<T><<<grid, SIMT_THREADS, smem, st>>>(
+        decode_prep_kernel<T><<<grid, DEC_THREADS, 0, st>>>(
             ix, n_blk, (T*)latent_K, (T*)K, (T*)V, (const T*)new_latent_k, (const T*)new_k,
-            (const T*)new_v, (const T*)latent_q, pos, Hkv, d, W, ws, attn_counter,
-            counters_per_seq);
+            (const T*)new_v, (const T*)latent_q, pos, Hkv, d, W, ws, app_score, app_g, app_slot,
+            n_slice, attn_counter, counters_per_seq);
     }
     note_launch();
     return cudaGetLastError();
@@ -1190,6 +1295,10 @@ SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
     p += al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
     w.score_ld = score_ld_of(ix);
     w.plan = BucketPlan{};
+    w.app_score = nullptr;
+    w.app_g = nullptr;
+    w.app_slot = nullptr;
+    w.app_n = 0;
     w.scores = nullptr;
     w.cmax = nullptr;
     if (select_uses_tc(ix, Nq)) {

@@ -199,8 +199,9 @@ int64_t ent_cap_for(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d, ls
 }
 
 struct DecodeLayout {
-    size_t indices, counts, sel, part, counter, total;
-    int ns, kps, n_hg;
+    size_t indices, counts, sel, part, counter, scores, cmax, app_score, app_g, app_slot, total;
+    int ns, kps, n_hg, n_slice;
+    int64_t score_ld;
 };
 
 
@@ -231,6 +232,19 @@ DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_sel
     L.sel = o;     o += select_ws_bytes(v, 1);
     L.part = o;    o += al256((size_t)v.B * ns * Hq * (d + 4) * 4);
     L.counter = o; o += al256((size_t)v.B * L.n_hg * 4);
+    // the append and scoring pass: about one CTA per SM over all sequences,
+    // with at most 992 buckets per slice
+    int64_t nsl = ((int64_t)sm_count() + v.B - 1) / v.B;
+    const int64_t min_sl = (v.NBK + 991) / 992;
+    if (nsl < min_sl) nsl = min_sl;
+    if (nsl > 65535) nsl = 65535;
+    L.n_slice = (int)nsl;
+    L.score_ld = ((v.NBK + 255) / 256) * 256;
+    L.scores = o;    o += al256((size_t)v.B * L.score_ld * 2);
+    L.cmax = o;      o += al256((size_t)v.B * (L.score_ld / 32) * 2);
+    L.app_score = o; o += al256((size_t)v.B * nsl * 8);
+    L.app_g = o;     o += al256((size_t)v.B * nsl * 4);
+    L.app_slot = o;  o += al256((size_t)v.B * 4);
     L.total = o;
     return L;
 }
@@ -648,6 +662,18 @@ lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
     int32_t* indices = (int32_t*)(base + L.indices);
     int32_t* counts = (int32_t*)(base + L.counts);
     SelectWs w = select_ws_carve(base + L.sel, v, 1);
+    // the fill nominates from the score row the prep pass writes, and finishes
+    // the prep pass's append
+    w.scores = (__half*)(base + L.scores);
+    w.cmax = (__half*)(base + L.cmax);
+    w.score_ld = L.score_ld;
+    double* app_score = (double*)(base + L.app_score);
+    int32_t* app_g = (int32_t*)(base + L.app_g);
+    int32_t* app_slot = (int32_t*)(base + L.app_slot);
+    w.app_score = app_score;
+    w.app_g = app_g;
+    w.app_slot = app_slot;
+    w.app_n = L.n_slice;
     float* part = (float*)(base + L.part);
     uint32_t* counter = (uint32_t*)(base + L.counter);
     if (!idx->status_clean) {
@@ -656,7 +682,8 @@ lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
         idx->status_clean = true;
     }
     cudaError_t e = launch_decode_prep(v, idx->n_blk, latent_K, K, V, new_latent_k, new_k, new_v,
-                                       latent_q, pos, Hkv, d, sp.window, w, counter, L.n_hg, st);
+                                       latent_q, pos, Hkv, d, sp.window, w, app_score, app_g,
+                                       app_slot, L.n_slice, counter, L.n_hg, st);
     if (e != cudaSuccess) return cuda_fail(e, "decode append/nominate");
     PosSrc ps{pos, 0};
     e = launch_select_finish(v, idx->n_blk, latent_q, ps, 1, sp, indices, counts, s_max, w, st);

@@ -145,6 +145,14 @@ struct SelectWs {
     __half* cmax;        // [B*Nq][score_ld/32] maximum of every 32-score chunk
     int64_t score_ld;
     BucketPlan plan;     // bucket-major attention lists (all null when unused)
+    // Decode append finished by the fill (app_n = 0 when unused): the exact
+    // nearest-centroid search of sequence b's completed group ran in app_n
+    // slices, each leaving its best (score, bucket); open slot app_slot[b]
+    // (-1: no group completed) receives the best of them.
+    const double* app_score;   // [B][app_n]
+    const int32_t* app_g;      // [B][app_n]
+    const int32_t* app_slot;   // [B]
+    int app_n;
 };
 constexpr int FB_CTAS = 148;
 // The tensor-core scorer serves bf16 indices and at least one 128-query tile.
@@ -193,12 +201,16 @@ cudaError_t launch_attn_combine(const float* part, int ns, int64_t rows, int Hq,
                                 float* lse, cudaStream_t st);
 int attn_head_group(int Hkv);
 
-// Decode: append + candidate nomination for one query per sequence.
+// Decode: append + approximate scores for one query per sequence, over
+// n_slice CTAs per sequence.  ws.scores / ws.cmax receive the fp16 score row
+// and its 32-score chunk maxima (as the tensor-core scorer writes them);
+// app_score / app_g / app_slot (in ws) the sliced nearest-centroid search.
 cudaError_t launch_decode_prep(const IndexView& ix, int64_t n_blk, void* latent_K, void* K,
                                void* V, const void* new_latent_k, const void* new_k,
                                const void* new_v, const void* latent_q, const int32_t* pos,
-                               int Hkv, int d, int W, const SelectWs& ws, uint32_t* attn_counter,
-                               int n_counter, cudaStream_t st);
+                               int Hkv, int d, int W, const SelectWs& ws, double* app_score,
+                               int32_t* app_g, int32_t* app_slot, int n_slice,
+                               uint32_t* attn_counter, int n_counter, cudaStream_t st);
 
 // Selection with scratch in a built-in device array (no caller workspace);
 // see k_select_noalloc.cu.
