@@ -378,14 +378,18 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                     stop = true;
                     break;
                 }
-                // this lane's key of the stage: one token per lane, shared by shuffles
-                int k = T.kbeg + s * TB_N + 32 * lw + lane;
-                if (k >= T.kend) k = T.kend - 1;   // padding rows repeat a real key (masked)
-                const int64_t t64 = ba_token(T, k, p, lp, mem_l, open_l);
-                int32_t tok = (int32_t)t64;
-                if (t64 < 0 || t64 >= ix.T_cap) {
-                    dev_error(ix.status, DEV_BAD_INDEX, (uint32_t)t64);
-                    tok = 0;
+                // this lane's key of the stage: one token per lane, shared by
+                // shuffles; rows past the tile's last key are zero-filled without
+                // a read (every query masks them, and 0 x 0 adds nothing to O)
+                const int k = T.kbeg + s * TB_N + 32 * lw + lane;
+                int32_t tok = -1;
+                if (k < T.kend) {
+                    const int64_t t64 = ba_token(T, k, p, lp, mem_l, open_l);
+                    tok = (int32_t)t64;
+                    if (t64 < 0 || t64 >= ix.T_cap) {
+                        dev_error(ix.status, DEV_BAD_INDEX, (uint32_t)t64);
+                        tok = 0;
+                    }
                 }
                 unsigned char* ks = smem + C::OFF_KV + slot * C::STAGE;
                 constexpr int KPI = 32 / C::CH;       // keys per warp instruction
@@ -396,9 +400,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                     const int32_t tk = __shfl_sync(0xffffffffu, tok, kl);
                     const int kr = 32 * lw + kl;                  // row inside the stage
                     const int soff = (c >> 3) * C::KV_PLANE + kr * 128 + (((c & 7) ^ (kr & 7)) << 4);
-                    const size_t goff = (size_t)tk * tstride + c * 8;
-                    ptx::cp_async16(ks + soff, Kb + goff);
-                    ptx::cp_async16(ks + C::K_BYTES + soff, Vb + goff);
+                    const bool real = tk >= 0;
+                    const size_t goff = real ? (size_t)tk * tstride + c * 8 : 0;
+                    ptx::cp_async16_zfill(ks + soff, Kb + goff, real ? 16u : 0u);
+                    ptx::cp_async16_zfill(ks + C::K_BYTES + soff, Vb + goff, real ? 16u : 0u);
                 }
                 ptx::cp_async_mbar_arrive(&kv_full[slot]);
             }

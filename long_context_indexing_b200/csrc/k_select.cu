@@ -323,7 +323,48 @@ struct FillCtx {
     int64_t hi;     // pos - W
     int64_t S;
     bool open_live; // the open block has keys at or below hi
+    // the open block's assigned groups in ascending order (shared memory):
+    // slot ol_o[x] of the open block belongs to bucket ol_g[x]
+    const int32_t* ol_o;
+    const int32_t* ol_g;
+    int ol_n;
 };
+
+// Compacts sequence bseq's open list into (slot, bucket) pairs in ascending
+// slot order; returns the count.  Called by every thread of the CTA (blockDim
+// a multiple of 32, at most 1024); cnt_s holds one int per warp.
+__device__ int build_open_list(const IndexView& ix, int64_t bseq, int32_t* ol_o, int32_t* ol_g,
+                               int* cnt_s)
+{
+    const int32_t* open = ix.open_bucket + bseq * ix.G;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int base = 0;
+    for (int x0 = 0; x0 < ix.G; x0 += blockDim.x) {
+        const int x = x0 + threadIdx.x;
+        const int32_t g = (x < ix.G) ? open[x] : -1;
+        const unsigned bal = __ballot_sync(0xffffffffu, g >= 0);
+        if (lane == 0) cnt_s[warp] = __popc(bal);
+        __syncthreads();
+        int before = base;
+        for (int w = 0; w < warp; ++w) before += cnt_s[w];
+        if (g >= 0) {
+            const int at = before + __popc(bal & ((1u << lane) - 1u));
+            ol_o[at] = x;
+            ol_g[at] = g;
+        }
+        for (int w = 0; w < nw; ++w) base += cnt_s[w];
+        __syncthreads();
+    }
+    return base;
+}
+
+// True when bucket g has a member in the open block.
+__device__ __forceinline__ bool has_open(const FillCtx& f, int64_t g)
+{
+    for (int x = 0; x < f.ol_n; ++x)
+        if (f.ol_g[x] == g) return true;
+    return false;
+}
 
 // Warp-cooperative count of available keys of bucket g (closed members plus
 // open-block members); *closed_out, when given, receives the closed part.
@@ -349,11 +390,10 @@ __device__ int64_t warp_avail(const FillCtx& f, int64_t g, int64_t* closed_out =
     }
     if (closed_out) *closed_out = a;
     if (f.open_live) {
-        const int32_t* open = ix.open_bucket + f.bseq * ix.G;
         const int64_t j0 = f.n_blk * ix.G;
         int64_t c = 0;
-        for (int o = lane; o < ix.G; o += 32)
-            if (open[o] == g) c += group_avail(j0 + o, p, f.S, f.hi);
+        for (int x = lane; x < f.ol_n; x += 32)
+            if (f.ol_g[x] == g) c += group_avail(j0 + f.ol_o[x], p, f.S, f.hi);
         for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
         a += c;
     }
@@ -414,13 +454,14 @@ __device__ void plan_list_row(const BucketPlan& P, int64_t row, int64_t bseq, in
 
 __device__ void warp_emit_partial(const FillCtx& f, int64_t g, int64_t take, int32_t* out);
 
-// True when every key of bucket g's closed members is available and no open
-// member can be: the bucket's available keys are then its members expanded.
+// True when every key of bucket g's closed members is available and it has no
+// available open member: the bucket's available keys are then its closed
+// members expanded.
 __device__ __forceinline__ bool bucket_full(const FillCtx& f, int64_t g)
 {
     const int64_t span = (int64_t)f.ix.p * f.ix.G;
     const int64_t bstart = (g / f.ix.k) * span;
-    return bstart >= f.S && bstart + span - 1 <= f.hi && !f.open_live;
+    return bstart >= f.S && bstart + span - 1 <= f.hi && !(f.open_live && has_open(f, g));
 }
 
 // Writes the first `take` available keys of bucket g (ascending) to out.
@@ -435,7 +476,7 @@ __device__ void cta_emit(const FillCtx& f, int64_t g, int64_t take, int32_t* out
     const int64_t blk = g / ix.k;
     const int64_t bstart = blk * span, bend = bstart + span;
     const int32_t o0 = off[g];
-    const bool full = (bstart >= f.S && bend - 1 <= f.hi) && !f.open_live;
+    const bool full = (bstart >= f.S && bend - 1 <= f.hi) && !(f.open_live && has_open(f, g));
     if (full) {
         for (int64_t x = threadIdx.x; x < take; x += blockDim.x)
             out[x] = mem[o0 + x / p] * p + (int32_t)(x % p);
@@ -468,18 +509,27 @@ __device__ void warp_emit_partial(const FillCtx& f, int64_t g, int64_t take, int
         cur += __popc(bal);
     }
     if (f.open_live) {
-        const int32_t* open = ix.open_bucket + f.bseq * ix.G;
+        // the bucket's open groups in ascending order; each contributes the
+        // contiguous run of its keys inside [S, hi]
         const int64_t j0 = f.n_blk * ix.G;
-        const int64_t nk = (int64_t)ix.G * p;
-        for (int64_t x0 = 0; x0 < nk && cur < take; x0 += 32) {
-            const int64_t x = x0 + lane;
-            int64_t t = -1;
-            if (x < nk && open[x / p] == g) t = (j0 + x / p) * p + x % p;
-            const bool ok = (t >= f.S) && (t <= f.hi);
-            const unsigned bal = __ballot_sync(0xffffffffu, ok);
-            const int64_t at = cur + __popc(bal & ((1u << lane) - 1u));
-            if (ok && at < take) out[at] = (int32_t)t;
-            cur += __popc(bal);
+        for (int x0 = 0; x0 < f.ol_n && cur < take; x0 += 32) {
+            const int x = x0 + lane;
+            int na = 0;
+            int64_t lo = 0;
+            if (x < f.ol_n && f.ol_g[x] == g) {
+                const int64_t jj = j0 + f.ol_o[x];
+                na = group_avail(jj, p, f.S, f.hi);
+                lo = (jj * p > f.S) ? jj * p : f.S;
+            }
+            int incl = na;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int64_t at0 = cur + incl - na;
+            for (int r = 0; r < na; ++r)
+                if (at0 + r < take) out[at0 + r] = (int32_t)(lo + r);
+            cur += __shfl_sync(0xffffffffu, incl, 31);
         }
     }
 }
@@ -690,6 +740,7 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
                                                                    int s_max, int32_t* indices,
                                                                    int32_t* counts, SelectWs ws)
 {
+    extern __shared__ int32_t open_sm[];   // [2][G] when the open block exists
     __shared__ float q_s[DL];
     __shared__ int cg[KC];
     __shared__ double es[KC];
@@ -769,6 +820,13 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     f.hi = pq - W;
     f.S = S;
     f.open_live = (n_blk * ix.G < ix.NP) && (n_blk > 0) && (n_blk * (int64_t)ix.p * ix.G <= f.hi);
+    f.ol_n = 0;
+    f.ol_o = open_sm;
+    f.ol_g = open_sm + ix.G;
+    if (f.open_live) {
+        __shared__ int cnt_w[FILL_THREADS / 32];
+        f.ol_n = build_open_list(ix, b, open_sm, open_sm + ix.G, cnt_w);
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     __shared__ int slow[KC];
     __shared__ int n_slow;
@@ -914,6 +972,8 @@ __global__ void __launch_bounds__(FB_THREADS) select_fallback_kernel(IndexView i
                                                                      int32_t* indices,
                                                                      int32_t* counts, SelectWs ws)
 {
+    extern __shared__ int32_t open_sm[];   // [2][G] when the open block exists
+    __shared__ int cnt_w[FB_THREADS / 32];
     __shared__ float q_s[DL];
     __shared__ double rs[FB_THREADS / 32];
     __shared__ int64_t rg[FB_THREADS / 32];
@@ -939,6 +999,10 @@ __global__ void __launch_bounds__(FB_THREADS) select_fallback_kernel(IndexView i
         f.hi = pq - W;
         f.S = S;
         f.open_live = (n_blk * ix.G < ix.NP) && (n_blk > 0) && (n_blk * (int64_t)ix.p * ix.G <= f.hi);
+        f.ol_n = 0;
+        f.ol_o = open_sm;
+        f.ol_g = open_sm + ix.G;
+        if (f.open_live) f.ol_n = build_open_list(ix, b, open_sm, open_sm + ix.G, cnt_w);
         int32_t* out = indices + row * (int64_t)s_max;
         const int64_t n_s = (S < pq + 1) ? S : pq + 1;
         for (int64_t x = threadIdx.x; x < n_s; x += FB_THREADS) out[x] = (int32_t)x;
@@ -1319,18 +1383,20 @@ static cudaError_t launch_finish_t(const IndexView& ix, int64_t n_blk, const T* 
                                    int32_t* counts, int s_max, const SelectWs& ws, cudaStream_t st)
 {
     dim3 grid((unsigned)Nq, (unsigned)ix.B);
+    // the compacted open list, when the index has an open block
+    const size_t osm = (n_blk > 0 && n_blk * ix.G < ix.NP) ? (size_t)ix.G * 2 * sizeof(int32_t) : 0;
     if (ws.scores)
-        select_fill_kernel<T, true><<<grid, FILL_THREADS, 0, st>>>(
+        select_fill_kernel<T, true><<<grid, FILL_THREADS, osm, st>>>(
             ix, n_blk, lq, pos, Nq, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
     else
-        select_fill_kernel<T, false><<<grid, FILL_THREADS, 0, st>>>(
+        select_fill_kernel<T, false><<<grid, FILL_THREADS, osm, st>>>(
             ix, n_blk, lq, pos, Nq, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
     note_launch();
     const int64_t rows = ix.B * Nq;
     const unsigned fb_grid = (unsigned)(rows < FB_CTAS ? rows : FB_CTAS);
-    select_fallback_kernel<T><<<fb_grid, FB_THREADS, 0, st>>>(ix, n_blk, lq, pos, Nq, sp.budget,
-                                                              sp.window, sp.sinks, s_max,
-                                                              indices, counts, ws);
+    select_fallback_kernel<T><<<fb_grid, FB_THREADS, osm, st>>>(ix, n_blk, lq, pos, Nq, sp.budget,
+                                                                sp.window, sp.sinks, s_max,
+                                                                indices, counts, ws);
     note_launch();
     return cudaGetLastError();
 }

@@ -205,6 +205,10 @@ struct DecodeLayout {
 };
 
 
+#ifndef LSA_DEC_SPLIT_MULT
+#define LSA_DEC_SPLIT_MULT 2
+#endif
+
 DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_select_params sp)
 {
     const IndexView& v = idx->v;
@@ -217,8 +221,9 @@ DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_sel
     L.n_hg = Hkv / hg;
     const int kt = attn_stage_keys(Hkv);
     const int64_t units = v.B * L.n_hg;
-    // about one CTA per SM over all (sequence, head group, split) triples
-    int64_t ns = ((int64_t)sm_count() + units - 1) / units;
+    // about LSA_DEC_SPLIT_MULT CTAs per SM over all (sequence, head group, split)
+    // triples
+    int64_t ns = ((int64_t)sm_count() * LSA_DEC_SPLIT_MULT + units - 1) / units;
     if (ns < 1) ns = 1;
     if (ns > 128) ns = 128;   // the combine keeps 2 * heads * ns floats in shared memory
     int64_t kps = (s_max + ns - 1) / ns;
