@@ -431,70 +431,75 @@ __global__ void __launch_bounds__(BA_THREADS, LSA_BA_MIN_BLOCKS) bucket_attn_ker
 }
 
 // ---------------------------------------------------------------------------
-// Merge: one warp per (listed row, query head) combines the row's nt + 1
-// partials.  Partial s holds O_s / l_s (bf16) with its max m_s and sum l_s:
-// with M the largest max and w_s = l_s exp2(m_s - M), the output is
-// sum_s w_s (O_s / l_s) / sum_s w_s.
+// Merge: one CTA per listed query row combines the row's nt + 1 partials.
+// Partial s holds O_s / l_s (bf16) with its max m_s and sum l_s per query
+// head: with M the head's largest max and w_s = l_s exp2(m_s - M), the output
+// is sum_s w_s (O_s / l_s) / sum_s w_s.  A row's partial slots are
+// consecutive, so the (max, sum) pairs of all its slots and heads are one
+// contiguous block, and each slot's outputs for all heads are another
+// (Hq * d bf16, 8 KB at 32 x 128): every load is coalesced.
 // ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(128) bucket_merge_kernel(BucketPlan P, int64_t n_heads_total,
-                                                           int Hq, __nv_bfloat16* O)
+constexpr int MERGE_THREADS = 256;
+constexpr int MERGE_MAX_SLOTS = KC + 1;
+constexpr int MERGE_MAX_HEADS = 64;
+
+__global__ void __launch_bounds__(MERGE_THREADS) bucket_merge_kernel(BucketPlan P, int Hq, int D,
+                                                                     __nv_bfloat16* O)
 {
-    constexpr int PER = D / 32;                  // output elements per lane
-    const int lane = threadIdx.x & 31;
-    const int64_t wid = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
-    if (wid >= n_heads_total) return;
-    const int64_t row = wid / Hq, hd = wid % Hq;
+    __shared__ float w_s[MERGE_MAX_SLOTS * MERGE_MAX_HEADS];   // weights [slot][head], normalised
+    const int64_t row = blockIdx.x;
     const int nt = P.row_n[row];
-    if (nt < 0) return;                       // gather row: written by the per-query kernel
+    if (nt < 0) return;                        // gather row: written by the per-query kernel
     const int ns = nt + 1;
-    const int64_t p0 = (int64_t)P.row_base[row] * Hq + hd;   // partial (slot base, head)
-    float M = -INFINITY;
-    for (int s0 = 0; s0 < ns; s0 += 32)
-        if (s0 + lane < ns) M = fmaxf(M, __ldcg(&P.part_ml[p0 + (int64_t)(s0 + lane) * Hq]).x);
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    float acc[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-    for (int s0 = 0; s0 < ns; s0 += 32) {
-        float wgt = 0.f;
-        if (s0 + lane < ns) {
-            const float2 mlv = __ldcg(&P.part_ml[p0 + (int64_t)(s0 + lane) * Hq]);
-            wgt = (mlv.x == -INFINITY) ? 0.f : mlv.y * exp2f(mlv.x - M);
-            L += wgt;
+    const int64_t base = (int64_t)P.row_base[row] * Hq;   // first (slot, head)
+    const float2* ml = P.part_ml + base;
+    // raw weights exp2(m) as pairs first: one pass per head over its slots
+    for (int h = threadIdx.x; h < Hq; h += MERGE_THREADS) {
+        float M = -INFINITY;
+        for (int sl = 0; sl < ns; ++sl) M = fmaxf(M, __ldcg(&ml[(int64_t)sl * Hq + h]).x);
+        float L = 0.f;
+        for (int sl = 0; sl < ns; ++sl) {
+            const float2 v = __ldcg(&ml[(int64_t)sl * Hq + h]);
+            const float wv = (v.x == -INFINITY) ? 0.f : v.y * exp2f(v.x - M);
+            w_s[sl * Hq + h] = wv;
+            L += wv;
         }
-        const int n = min(32, ns - s0);
-        for (int j = 0; j < n; ++j) {
-            const float wj = __shfl_sync(0xffffffffu, wgt, j);
-            const __nv_bfloat16* src = P.part_o + (p0 + (int64_t)(s0 + j) * Hq) * D + PER * lane;
-            if (PER == 4) {
-                const uint2 u = __ldcg(reinterpret_cast<const uint2*>(src));
-                const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-                const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-                acc[0] += a0.x * wj;
-                acc[1] += a0.y * wj;
-                acc[2] += a1.x * wj;
-                acc[3] += a1.y * wj;
-            } else {
-                const unsigned u = __ldcg(reinterpret_cast<const unsigned*>(src));
-                const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
-                acc[0] += a0.x * wj;
-                acc[1] += a0.y * wj;
+        const float inv = 1.f / L;
+        for (int sl = 0; sl < ns; ++sl) w_s[sl * Hq + h] *= inv;
+    }
+    __syncthreads();
+    const int n8 = Hq * D / 8;                 // 16-byte groups of the row's output
+    const __nv_bfloat16* src = P.part_o + base * D;
+    __nv_bfloat16* dst = O + row * (int64_t)Hq * D;
+    for (int c = threadIdx.x; c < n8; c += MERGE_THREADS) {
+        const int h = (c * 8) / D;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 4
+        for (int sl = 0; sl < ns; ++sl) {
+            const uint4 u = __ldcg(reinterpret_cast<const uint4*>(src + (int64_t)sl * Hq * D) + c);
+            const float wv = w_s[sl * Hq + h];
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(b2[e]);
+                acc[2 * e] = fmaf(f.x, wv, acc[2 * e]);
+                acc[2 * e + 1] = fmaf(f.y, wv, acc[2 * e + 1]);
             }
         }
-    }
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    const float inv = 1.f / L;
-    __nv_bfloat16* op = O + wid * D + PER * lane;
+        uint4 out;
+        uint32_t* o32 = reinterpret_cast<uint32_t*>(&out);
 #pragma unroll
-    for (int e = 0; e < PER; e += 2)
-        *reinterpret_cast<__nv_bfloat162*>(op + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+        for (int e = 0; e < 4; ++e) o32[e] = ptx::pack_bf16(acc[2 * e], acc[2 * e + 1]);
+        reinterpret_cast<uint4*>(dst)[c] = out;
+    }
 }
 
 bool bucket_attn_supported(int Hq, int Hkv, int d)
 {
-    return (d == 64 || d == 128) && Hkv >= 1 && Hq % Hkv == 0 && Hq / Hkv <= 8;
+    return (d == 64 || d == 128) && Hkv >= 1 && Hq % Hkv == 0 && Hq / Hkv <= 8 &&
+           Hq <= MERGE_MAX_HEADS;
 }
 
 template <int D>
@@ -555,12 +560,8 @@ cudaError_t launch_bucket_attn(const IndexView& ix, int64_t n_blk, const BucketP
     e = launch_attn_rows(Q, K, V, ix.B, Nq, ix.T_cap, Hq, Hkv, d, indices, counts, s_max, scale, O,
                          ix.status, P.gather_rows, P.ctr + CTR_GATHER, st);
     if (e != cudaSuccess) return e;
-    const int64_t n = ix.B * Nq * Hq;
-    const unsigned grid = (unsigned)((n + 3) / 4);
-    if (d == 128)
-        bucket_merge_kernel<128><<<grid, 128, 0, st>>>(P, n, Hq, (__nv_bfloat16*)O);
-    else
-        bucket_merge_kernel<64><<<grid, 128, 0, st>>>(P, n, Hq, (__nv_bfloat16*)O);
+    bucket_merge_kernel<<<(unsigned)(ix.B * Nq), MERGE_THREADS, 0, st>>>(P, Hq, d,
+                                                                        (__nv_bfloat16*)O);
     note_launch();
     return cudaGetLastError();
 }

@@ -14,10 +14,10 @@
 // once and read once.
 //
 // CTA = 128 queries of one sequence (one TMEM lane each), 6 warps:
-//   warp 0     TMA producer: the query tile once, then 256-centroid tiles into
+//   warp 0     TMA producer: the query tile once, then TC_N-centroid tiles into
 //              a TC_STAGES-deep shared-memory ring (128-byte swizzle);
-//   warp 1     owns 512 TMEM columns (two 256-column fp32 accumulators) and
-//              issues tcgen05.mma (M=128, N=256, K=16, four per tile);
+//   warp 1     owns 2 x TC_N TMEM columns (two fp32 accumulators) and
+//              issues tcgen05.mma (M=128, N=TC_N, K=16, four per tile);
 //   warps 2-5  epilogue: tcgen05.ld 32 columns at a time, fp32 -> fp16, and
 //              64-byte row segments straight to the score matrix.
 // Every mbarrier wait is bounded; on a timeout the CTA records DEV_TIMEOUT in
@@ -32,13 +32,18 @@
 namespace lsa {
 
 constexpr int TC_M = 128;
-constexpr int TC_N = 256;
+#ifndef LSA_TC_N
+#define LSA_TC_N 256         // centroids per tile (128 gives two CTAs per SM; measured slower)
+#endif
+constexpr int TC_N = LSA_TC_N;
+constexpr int TC_TMEM_COLS = 2 * TC_N;                    // two fp32 accumulators
+constexpr int TC_MIN_BLOCKS = (TC_N <= 128) ? 2 : 1;
 constexpr int TC_STAGES = 4;
 constexpr int TC_THREADS = 192;
 constexpr uint32_t TC_WAIT = 1u << 22;
 
 constexpr int TC_Q_BYTES = TC_M * DL * 2;                 // 16 KB
-constexpr int TC_C_BYTES = TC_N * DL * 2;                 // 32 KB per stage
+constexpr int TC_C_BYTES = TC_N * DL * 2;                 // 32 KB per stage at N = 256
 constexpr int TC_OFF_C = TC_Q_BYTES;
 constexpr int TC_OFF_BAR = TC_OFF_C + TC_STAGES * TC_C_BYTES;
 constexpr int TC_NBAR = 1 + 2 * TC_STAGES + 4;
@@ -68,7 +73,7 @@ __device__ __forceinline__ uint64_t sw128_desc(const void* smem_tile)
 }
 
 // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both
-// K-major, N = 256, M = 128.
+// K-major, N = TC_N, M = 128.
 constexpr uint32_t TC_IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_N >> 3) << 17) |
                               ((uint32_t)(TC_M >> 4) << 24);
 
@@ -121,7 +126,7 @@ __device__ __forceinline__ int64_t tc_eligible(const IndexView& ix, int64_t n_bl
     return nb * ix.k;
 }
 
-__global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
+__global__ void __launch_bounds__(TC_THREADS, TC_MIN_BLOCKS) score_topk_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC, IndexView ix,
     int64_t n_blk, PosSrc pos, int64_t Nq, int W, SelectWs ws)
 {
@@ -167,8 +172,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
-                         ptx::smem_addr((const void*)tmem_slot))
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         ptx::smem_addr((const void*)tmem_slot)), "n"(TC_TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -281,7 +286,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_topk_tc_kernel(
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(TC_TMEM_COLS)
                      : "memory");
     }
 }
