@@ -7,9 +7,11 @@
 // 16 queries x 8 query heads are the 128 rows of one MMA (a row per TMEM
 // lane), and the tile's keys stream through in 64-key stages:
 //
-//   S  = Q K^T   M = 128, N = 64 keys, K = d      (TMEM, double-buffered)
-//   P  = exp2(S * scale * log2 e - m)            (softmax warps, bf16 to smem)
-//   O += P V     M = 128, N = d, K = 64 keys      (TMEM, two accumulators)
+//   S  = Q K^T   M = 128, N = 64 keys, K = d      (TMEM, three buffers)
+//   P  = exp2(S * scale * log2 e - m)            (softmax warps, bf16 into the
+//                                                 first 32 columns of S's buffer)
+//   O += P V     M = 128, N = d, K = 64 keys      (A = P read from TMEM; TMEM,
+//                                                 two accumulators)
 //
 // Warp roles (13 warps):
 //   warp 0     planner: claims work items and copies each tile's description
@@ -24,14 +26,17 @@
 //   warps 4-7  softmax: thread = row = TMEM lane; reads its 64 scores of a
 //              stage, masks keys outside its query's ranges, keeps the
 //              running max (raised lazily: O and the sum are rescaled only
-//              when the max grows by more than 2^8), writes its P row, and at
-//              the end of the tile hands the row's (max, sum) on;
+//              when the max grows by more than 2^8), writes its P row back to
+//              TMEM over the scores, and at the end of the tile hands the
+//              row's (max, sum) on;
 //   warps 8-11 epilogue: write each row's partial (O row / sum as bf16, and
 //              the fp32 max and sum) from one
 //              of two TMEM accumulators (tiles alternate), overlapping the
 //              next tile's softmax.
 // Q and tile descriptions are double-buffered across work items and the K/V
-// ring continues across them, so loads of the next tile overlap this one.
+// ring continues across them, so loads of the next tile overlap this one.  An
+// S buffer (and the P in it) is released by the commit of its P V MMA, so the
+// softmax never waits for the tensor cores except to rescale O.
 // Every wait is bounded; on a timeout the CTA records DEV_TIMEOUT, all roles
 // leave, outstanding copies and MMAs are waited for, and TMEM is freed.
 #include <limits.h>
@@ -66,12 +71,10 @@ struct TbCfg {
     static constexpr int KV_PLANE = TB_N * 128;         // 64 dims of 64 keys
     static constexpr int K_BYTES = (D / 64) * KV_PLANE;
     static constexpr int STAGE = 2 * K_BYTES;           // K then V
-    static constexpr int P_BYTES = TB_M * TB_N * 2;
     static constexpr int OFF_Q = 0;                     // QB buffers
     static constexpr int OFF_KV = OFF_Q + QB * Q_BYTES; // NS stages
-    static constexpr int OFF_P = OFF_KV + NS * STAGE;
-    static constexpr int OFF_BAR = OFF_P + P_BYTES;
-    static constexpr int NBAR = 22 + 2 * NS;
+    static constexpr int OFF_BAR = OFF_KV + NS * STAGE;
+    static constexpr int NBAR = 23 + 2 * NS;
     static constexpr int OFF_ML = OFF_BAR + NBAR * 8;      // [2][128] (max, sum) per row
     static constexpr int OFF_LISTS = OFF_ML + 2 * TB_M * 8;   // then 4 member lists of G ints
     // dynamic shared memory for a block of G pooled groups (+ alignment slack)
@@ -100,6 +103,18 @@ __device__ __forceinline__ void tb_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// D (+)= A B with A (M x 16, bf16 pairs per 32-bit column, row m in lane m)
+// read from TMEM at column a_tmem.
+__device__ __forceinline__ void tb_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void tb_commit(uint64_t* bar)
@@ -183,6 +198,21 @@ __device__ __forceinline__ void tb_st32(uint32_t taddr, const float* v)
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tb_st32u(uint32_t taddr, const uint32_t* v)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+        "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 template <int D, int NS, int QB>
 __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
 {
@@ -195,13 +225,12 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     uint64_t* q_full = bars + 4;         // [2]
     uint64_t* q_empty = bars + 6;        // [2]
     uint64_t* s_full = bars + 8;         // [TB_SB]
-    uint64_t* s_empty = bars + 11;       // [TB_SB]
-    uint64_t* p_full = bars + 14;
-    uint64_t* p_empty = bars + 15;
-    uint64_t* o_full = bars + 16;        // [2] (two O accumulators, by item parity)
-    uint64_t* o_empty = bars + 18;       // [2]
-    uint64_t* ml_full = bars + 20;       // [2]
-    uint64_t* kv_full = bars + 22;       // [NS]
+    uint64_t* s_empty = bars + 11;       // [TB_SB] (committed after the buffer's P V)
+    uint64_t* p_full = bars + 14;        // [TB_SB]
+    uint64_t* o_full = bars + 17;        // [2] (two O accumulators, by item parity)
+    uint64_t* o_empty = bars + 19;       // [2]
+    uint64_t* ml_full = bars + 21;       // [2]
+    uint64_t* kv_full = bars + 23;       // [NS]
     float2* ml = reinterpret_cast<float2*>(smem + C::OFF_ML);   // [2][TB_M]
     uint64_t* kv_empty = kv_full + NS;
     const int lcap = (a.ix.G + 3) & ~3;  // ints per member list
@@ -233,10 +262,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
         }
         for (int i = 0; i < TB_SB; ++i) {
             ptx::mbar_init(&s_full[i], 1);
-            ptx::mbar_init(&s_empty[i], 4);
+            ptx::mbar_init(&s_empty[i], 1);
+            ptx::mbar_init(&p_full[i], 4);
         }
-        ptx::mbar_init(p_full, 4);
-        ptx::mbar_init(p_empty, 1);
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(&kv_full[s], 64);
             ptx::mbar_init(&kv_empty[s], 1);
@@ -415,11 +443,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     } else if (warp == 3) {
         // =========================== MMA issuer ===========================
         if (lane == 0) {
-            int64_t gs = 0, pv = 0;
+            int64_t gs = 0;
             bool stop = false;
             const uint32_t q_base = ptx::smem_addr(smem + C::OFF_Q);
             const uint32_t kv_base = ptx::smem_addr(smem + C::OFF_KV);
-            const uint32_t p_base = ptx::smem_addr(smem + C::OFF_P);
             // Two cursors over one stream of stages (all items in order). The
             // issuer polls: a P V MMA goes out as soon as its P is ready; an S
             // MMA goes out, up to TB_SB - 1 stages ahead of the P V cursor and
@@ -437,24 +464,23 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 if (abort_flag) break;
                 bool progress = false;
                 // ---- P V for the oldest stage whose P is ready ----
-                if (gP < gs && ptx::mbar_test(p_full, (uint32_t)(pv & 1)) &&
+                const int sbP = (int)(gP % TB_SB);
+                if (gP < gs && ptx::mbar_test(&p_full[sbP], (uint32_t)((gP / TB_SB) & 1)) &&
                     (sP > 0 || ptx::mbar_test(&o_empty[iP & 1], (uint32_t)(((iP >> 1) & 1) ^ 1)))) {
                     const int ib = iP & 1;
                     const int slot = (int)(gP % NS);
-                    // P was fenced to the async proxy by the softmax threads before
-                    // they arrived on p_full
+                    // the softmax threads' TMEM stores of P are ordered before
+                    // their arrivals on p_full
                     tb_fence_after();
                     const uint32_t t_o = tmem + TB_COL_O + 128 * ib;
-                    const uint64_t pd = tb_desc(p_base, 16, 1024);
                     const uint64_t vd =
                         tb_desc(kv_base + slot * C::STAGE + C::K_BYTES, C::KV_PLANE, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < TB_N / 16; ++kk)   // start address in 16-byte units
-                        tb_mma(t_o, pd + (uint64_t)(kk * 2), vd + (uint64_t)(kk * 128), C::IDESC_PV,
-                               (sP > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < TB_N / 16; ++kk)   // 16 keys = 8 TMEM columns of P
+                        tb_mma_ts(t_o, tmem + sbP * TB_N + kk * 8, vd + (uint64_t)(kk * 128),
+                                  C::IDESC_PV, (sP > 0 || kk > 0) ? 1u : 0u);
                     tb_commit(&kv_empty[slot]);
-                    tb_commit(p_empty);
-                    ++pv;
+                    tb_commit(&s_empty[sbP]);
                     if (sP == nst[ib] - 1) tb_commit(&o_full[ib]);
                     ++gP;
                     if (++sP == nst[ib]) {
@@ -522,8 +548,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
         // ============================ softmax ============================
         const int r = 32 * (warp & 3) + lane;               // row = TMEM lane
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-        int64_t gs = 0, pv = 0;
-        unsigned char* prow = smem + C::OFF_P + r * 128;
+        int64_t gs = 0;
         for (int i = 0;; ++i) {
             const int ib = i & 1;
             const uint32_t iph = (uint32_t)((i >> 1) & 1);
@@ -550,9 +575,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 tb_fence_after();
                 float v[TB_N];
                 tb_ld64(tmem + lane_base + sb * TB_N, v);
-                tb_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&s_empty[sb]);
 
                 const int kb = kbeg + s * TB_N;
                 // keys of this stage the row's query reads, as a 64-bit mask
@@ -612,13 +634,14 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 }
                 const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
                 l = l * alpha + sum;
-                // the previous P has been consumed (and O is quiet) once the
-                // previous PV MMA has completed
-                if (!waitw(p_empty, (uint32_t)((pv & 1) ^ 1), 320u)) {
-                    stop = true;
-                    break;
-                }
                 if (__any_sync(0xffffffffu, resc)) {
+                    // O is quiet once the previous stage's P V MMA (the commit
+                    // that released its S buffer) has completed
+                    const int64_t gq = gs - 1;
+                    if (!waitw(&s_empty[gq % TB_SB], (uint32_t)((gq / TB_SB) & 1), 320u)) {
+                        stop = true;
+                        break;
+                    }
                     tb_fence_after();
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
@@ -629,15 +652,11 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                         tb_st32(tmem + lane_base + TB_COL_O + 128 * ib + c * 32, o);
                     }
                 }
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
-                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                ptx::fence_proxy_async();
+                // P over the first 32 columns of the scores' buffer
+                tb_st32u(tmem + lane_base + sb * TB_N, pk);
                 tb_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(p_full);
-                ++pv;
+                if (lane == 0) ptx::mbar_arrive(&p_full[sb]);
             }
             if (stop) break;
             // the row's (max, sum) for the epilogue warps
