@@ -193,18 +193,29 @@ __device__ __forceinline__ void ba_open_list(const IndexView& ix, int64_t n_blk,
 {
     const int32_t* open = ix.open_bucket + b * ix.G;
     const int lane = tid & 31, warp = tid >> 5, nw = nthreads >> 5;
+    constexpr int U = 8;   // loads in flight per thread
     int base = 0;
-    for (int x0 = 0; x0 < ix.G; x0 += nthreads) {
-        const int x = x0 + tid;
-        const bool hit = x < ix.G && open[x] == g;
-        const unsigned bal = __ballot_sync(0xffffffffu, hit);
-        if (lane == 0) cnt_s[warp] = __popc(bal);
-        bar();
-        int before = base;
-        for (int w2 = 0; w2 < warp; ++w2) before += cnt_s[w2];
-        if (hit) open_list[before + __popc(bal & ((1u << lane) - 1u))] = (int32_t)(n_blk * ix.G + x);
-        for (int w2 = 0; w2 < nw; ++w2) base += cnt_s[w2];
-        bar();
+    for (int x00 = 0; x00 < ix.G; x00 += U * nthreads) {
+        int32_t bk[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int x = x00 + u * nthreads + tid;
+            bk[u] = (x < ix.G) ? open[x] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (x00 + u * nthreads >= ix.G) break;   // uniform over the threads
+            const int x = x00 + u * nthreads + tid;
+            const bool hit = x < ix.G && bk[u] == g;
+            const unsigned bal = __ballot_sync(0xffffffffu, hit);
+            if (lane == 0) cnt_s[warp] = __popc(bal);
+            bar();
+            int before = base;
+            for (int w2 = 0; w2 < warp; ++w2) before += cnt_s[w2];
+            if (hit) open_list[before + __popc(bal & ((1u << lane) - 1u))] = (int32_t)(n_blk * ix.G + x);
+            for (int w2 = 0; w2 < nw; ++w2) base += cnt_s[w2];
+            bar();
+        }
     }
 }
 

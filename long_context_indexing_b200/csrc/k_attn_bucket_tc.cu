@@ -13,14 +13,14 @@
 //   O += P V     M = 128, N = d, K = 64 keys      (A = P read from TMEM; TMEM,
 //                                                 two accumulators)
 //
-// Warp roles (13 warps):
+// Warp roles (15 warps):
 //   warp 0     planner: claims work items and copies each tile's description
 //              (written by bucket_tile_records_kernel) and the bucket's member
 //              lists into shared memory, one item ahead;
-//   warps 1-2  loaders: gather the tile's Q rows and every stage's K and V rows
-//              of the KV head with 16-byte cp.async into 128-byte-swizzled
-//              planes (the layout the MMA descriptors name); completion lands
-//              on mbarriers;
+//   warps 1-2, 13-14  loaders: gather every stage's K and V rows of the KV
+//              head (16 keys per warp) with 16-byte cp.async into
+//              128-byte-swizzled planes (the layout the MMA descriptors name);
+//              completion lands on mbarriers;
 //   warp 3     allocates TMEM; lane 0 issues all MMAs and commits;
 //   warp 12    Q loader: the tile's Q rows, as soon as its Q buffer is free;
 //   warps 4-7  softmax: thread = row = TMEM lane; reads its 64 scores of a
@@ -53,7 +53,13 @@ constexpr int TB_N = 64;             // keys per stage
 constexpr int TB_OPEN_MAX = 2048;    // members of one bucket a tile can hold (block size bound)
 constexpr int TB_SB = 3;             // S buffers in TMEM: S runs up to two stages ahead of P V
 constexpr uint32_t TB_COL_O = TB_SB * 64;   // first TMEM column of the two O accumulators
-constexpr int TB_THREADS = 416;      // 13 warps
+#ifndef LSA_TB_LOADERS
+#define LSA_TB_LOADERS 4     // K/V loader warps (2 or 4)
+#endif
+constexpr int TB_NL = LSA_TB_LOADERS;
+static_assert(TB_NL == 2 || TB_NL == 4, "K/V loader warps");
+constexpr int TB_KPW = 64 / TB_NL;                // keys of a stage per loader warp
+constexpr int TB_THREADS = 32 * (11 + TB_NL);     // 15 warps with four loaders
 constexpr uint32_t TB_WAIT = 1u << 22;
 
 #ifndef LSA_TB_QB
@@ -74,7 +80,7 @@ struct TbCfg {
     static constexpr int OFF_Q = 0;                     // QB buffers
     static constexpr int OFF_KV = OFF_Q + QB * Q_BYTES; // NS stages
     static constexpr int OFF_BAR = OFF_KV + NS * STAGE;
-    static constexpr int NBAR = 23 + 2 * NS;
+    static constexpr int NBAR = 25 + 2 * NS;
     static constexpr int OFF_ML = OFF_BAR + NBAR * 8;      // [2][128] (max, sum) per row
     static constexpr int OFF_LISTS = OFF_ML + 2 * TB_M * 8;   // then 4 member lists of G ints
     // dynamic shared memory for a block of G pooled groups (+ alignment slack)
@@ -230,7 +236,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     uint64_t* o_full = bars + 17;        // [2] (two O accumulators, by item parity)
     uint64_t* o_empty = bars + 19;       // [2]
     uint64_t* ml_full = bars + 21;       // [2]
-    uint64_t* kv_full = bars + 23;       // [NS]
+    uint64_t* ml_empty = bars + 23;      // [2]
+    uint64_t* kv_full = bars + 25;       // [NS]
     float2* ml = reinterpret_cast<float2*>(smem + C::OFF_ML);   // [2][TB_M]
     uint64_t* kv_empty = kv_full + NS;
     const int lcap = (a.ix.G + 3) & ~3;  // ints per member list
@@ -253,10 +260,11 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&info_full[i], 1);
-            ptx::mbar_init(&info_empty[i], 12);    // 4 softmax, 4 epilogue, MMA, 2 K/V loaders, Q loader
+            ptx::mbar_init(&info_empty[i], 10 + TB_NL);   // 4 softmax, 4 epilogue, MMA, K/V loaders, Q loader
             ptx::mbar_init(&o_full[i], 1);
             ptx::mbar_init(&o_empty[i], 4);
             ptx::mbar_init(&ml_full[i], 4);
+            ptx::mbar_init(&ml_empty[i], 4);
             ptx::mbar_init(&q_full[i], 32);        // every Q-loader lane's cp.async arrival
             ptx::mbar_init(&q_empty[i], 1);
         }
@@ -266,7 +274,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             ptx::mbar_init(&p_full[i], 4);
         }
         for (int s = 0; s < NS; ++s) {
-            ptx::mbar_init(&kv_full[s], 64);
+            ptx::mbar_init(&kv_full[s], 32 * TB_NL);
             ptx::mbar_init(&kv_empty[s], 1);
         }
         ptx::mbar_init(&fin_bar, 1);
@@ -307,36 +315,74 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     if (warp == 0) {
         // ============================ planner ============================
         // Claims work items and brings each tile's description and member
-        // lists into shared memory, one item ahead of the loaders.
-        int w_next = 0;
-        if (lane == 0) w_next = atomicAdd(a.P.ctr + CTR_WORK, 1);
-        const TileInfo* recs = reinterpret_cast<const TileInfo*>(a.P.recs);
+        // lists into shared memory.  Its global reads are software-pipelined
+        // so that the wait for a free description buffer hides them: the
+        // claim runs two items ahead; the description and the first
+        // 32 x PF_MEM member ids of the next item are in registers before the
+        // wait.
+        constexpr int REC_V = TILE_REC_BYTES / 16;     // a record is 28 x 16 bytes, a lane each
+        constexpr int PF_MEM = 4;
+        const uint4* recs = reinterpret_cast<const uint4*>(a.P.recs);
+        auto claim = [&]() -> int {
+            int wv = 0;
+            if (lane == 0) wv = atomicAdd(a.P.ctr + CTR_WORK, 1);
+            return wv;   // meaningful in lane 0
+        };
+        auto load_rec = [&](int64_t w) -> uint4 {
+            uint4 r = make_uint4(0u, 0u, 0u, 0u);
+            if (w < n_work && lane < REC_V) r = recs[(w / a.Hkv) * REC_V + lane];
+            return r;
+        };
+        // a 32-bit field of a record spread over the lanes (warp-uniform call)
+        auto rec_u32 = [&](const uint4& r, int off) -> uint32_t {
+            const int c = (off >> 2) & 3;
+            const uint32_t v = c == 0 ? r.x : c == 1 ? r.y : c == 2 ? r.z : r.w;
+            return __shfl_sync(0xffffffffu, v, off >> 4);
+        };
+        auto load_mem = [&](const uint4& r, int64_t w, int32_t* m) {
+#pragma unroll
+            for (int u = 0; u < PF_MEM; ++u) m[u] = 0;
+            if (w >= n_work || (int)rec_u32(r, (int)offsetof(TileInfo, kind)) != 1) return;
+            const int o0 = (int)rec_u32(r, (int)offsetof(TileInfo, o0));
+            const int ng = (int)rec_u32(r, (int)offsetof(TileInfo, nclosed)) / p;
+            const int64_t b = (int64_t)(((uint64_t)rec_u32(r, (int)offsetof(TileInfo, b) + 4) << 32) |
+                                        rec_u32(r, (int)offsetof(TileInfo, b)));
+            const int32_t* mem_g = ix.members + b * ix.NP + o0;
+#pragma unroll
+            for (int u = 0; u < PF_MEM; ++u)
+                if (lane + 32 * u < ng) m[u] = mem_g[lane + 32 * u];
+        };
+        int64_t w_cur = __shfl_sync(0xffffffffu, claim(), 0);
+        int c_next = claim();
+        uint4 rec_cur = load_rec(w_cur);
+        int32_t mem_cur[PF_MEM];
+        load_mem(rec_cur, w_cur, mem_cur);
         for (int i = 0;; ++i) {
             const int ib = i & 1;
             const uint32_t iph = (uint32_t)((i >> 1) & 1);
             TileInfo& T = ti[ib];
+            const int64_t w_nxt = __shfl_sync(0xffffffffu, c_next, 0);
+            if (w_cur < n_work) c_next = claim();
+            const uint4 rec_nxt = load_rec(w_nxt);
             if (!waitw(&info_empty[ib], iph ^ 1u, 100u)) break;
-            const int64_t w = __shfl_sync(0xffffffffu, w_next, 0);
-            if (lane == 0) w_next = atomicAdd(a.P.ctr + CTR_WORK, 1);
-            if (w >= n_work) {
+            if (w_cur >= n_work) {
                 if (lane == 0) {
                     T.n_st = -1;
                     ptx::mbar_arrive(&info_full[ib]);
                 }
                 break;
             }
-            const int64_t t = w / a.Hkv;
-            {
-                const uint4* src = reinterpret_cast<const uint4*>(recs + t);
-                uint4* dst = reinterpret_cast<uint4*>(&T);
-                for (int x = lane; x < TILE_REC_BYTES / 16; x += 32) dst[x] = src[x];
-            }
+            if (lane < REC_V) reinterpret_cast<uint4*>(&T)[lane] = rec_cur;
             __syncwarp();
-            if (lane == 0) T.h = (int)(w % a.Hkv);
+            if (lane == 0) T.h = (int)(w_cur % a.Hkv);
             if (T.kind == 1) {
                 int32_t* mem_l = mem_list(ib);
+                const int ng = T.nclosed / p;
+#pragma unroll
+                for (int u = 0; u < PF_MEM; ++u)
+                    if (lane + 32 * u < ng) mem_l[lane + 32 * u] = mem_cur[u];
                 const int32_t* mem_g = ix.members + T.b * ix.NP + T.o0;
-                for (int x = lane; x < T.nclosed / p; x += 32) mem_l[x] = mem_g[x];
+                for (int x = 32 * PF_MEM + lane; x < ng; x += 32) mem_l[x] = mem_g[x];
                 if (T.any_open) {
                     int32_t* open_l = open_list(ib);
                     ba_open_list(ix, a.n_blk, T.b, T.g, lane, 32, cnt_s, open_l, [] { __syncwarp(); });
@@ -344,6 +390,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&info_full[ib]);
+            w_cur = w_nxt;
+            rec_cur = rec_nxt;
+            load_mem(rec_cur, w_cur, mem_cur);
         }
     } else if (warp == 12) {
         // ============================ Q loader ============================
@@ -379,11 +428,11 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             if (lane == 0) ptx::mbar_arrive(&info_empty[ib]);   // done with ti[ib]
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
-    } else if (warp < 3) {
+    } else if (warp < 3 || warp >= 13) {
         // ============================ loaders ============================
         // Gather every stage's K and V rows of the KV head (tokens from the
         // shared-memory member lists).
-        const int lw = warp - 1;
+        const int lw = (warp < 3) ? warp - 1 : warp - 11;   // warps 1, 2, 13, 14
         int64_t gs = 0;
         for (int i = 0;; ++i) {
             const int ib = i & 1;
@@ -409,9 +458,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 // this lane's key of the stage: one token per lane, shared by
                 // shuffles; rows past the tile's last key are zero-filled without
                 // a read (every query masks them, and 0 x 0 adds nothing to O)
-                const int k = T.kbeg + s * TB_N + 32 * lw + lane;
+                const int k = T.kbeg + s * TB_N + TB_KPW * lw + lane;
                 int32_t tok = -1;
-                if (k < T.kend) {
+                if (lane < TB_KPW && k < T.kend) {
                     const int64_t t64 = ba_token(T, k, p, lp, mem_l, open_l);
                     tok = (int32_t)t64;
                     if (t64 < 0 || t64 >= ix.T_cap) {
@@ -422,11 +471,11 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 unsigned char* ks = smem + C::OFF_KV + slot * C::STAGE;
                 constexpr int KPI = 32 / C::CH;       // keys per warp instruction
 #pragma unroll 4
-                for (int j = 0; j < 32 / KPI; ++j) {
-                    const int kl = KPI * j + lane / C::CH;        // key inside this warp's 32
+                for (int j = 0; j < TB_KPW / KPI; ++j) {
+                    const int kl = KPI * j + lane / C::CH;        // key inside this warp's share
                     const int c = lane % C::CH;
                     const int32_t tk = __shfl_sync(0xffffffffu, tok, kl);
-                    const int kr = 32 * lw + kl;                  // row inside the stage
+                    const int kr = TB_KPW * lw + kl;              // row inside the stage
                     const int soff = (c >> 3) * C::KV_PLANE + kr * 128 + (((c & 7) ^ (kr & 7)) << 4);
                     const bool real = tk >= 0;
                     const size_t goff = real ? (size_t)tk * tstride + c * 8 : 0;
@@ -564,6 +613,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             const bool live = q < BA_Q && T.slot[q] >= 0;
             const QRange rg = live ? T.rng[q] : QRange{0, 0, 0, 0};
             const int kbeg = T.kbeg;
+            // what the row needs of the description is in registers: release it
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&info_empty[ib]);
             float m_run = -INFINITY, l = 0.f;
             bool stop = false;
             for (int s = 0; s < n_st; ++s, ++gs) {
@@ -659,13 +711,12 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 if (lane == 0) ptx::mbar_arrive(&p_full[sb]);
             }
             if (stop) break;
-            // the row's (max, sum) for the epilogue warps
+            // the row's (max, sum) for the epilogue warps, once they have read
+            // the pair of two items ago
+            if (!waitw(&ml_empty[ib], iph ^ 1u, 330u)) break;
             ml[ib * TB_M + r] = make_float2(m_run, l);
             __syncwarp();
-            if (lane == 0) {
-                ptx::mbar_arrive(&ml_full[ib]);
-                ptx::mbar_arrive(&info_empty[ib]);
-            }
+            if (lane == 0) ptx::mbar_arrive(&ml_full[ib]);
         }
     } else {
         // ============================ epilogue ============================
@@ -681,11 +732,16 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             const TileInfo& T = ti[ib];
             if (T.n_st < 0) break;
             const int q = r / a.hpg, hh = r % a.hpg;
-            const bool live = q < BA_Q && T.slot[q] >= 0;
+            const int slot = (q < BA_Q) ? T.slot[q] : -1;
+            const bool live = slot >= 0;
+            const size_t ph = ((size_t)(live ? slot : 0) * a.Hq) + (size_t)T.h * a.hpg + hh;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&info_empty[ib]);   // the rest is in registers
             if (!waitw(&ml_full[ib], iph, 410u) || !waitw(&o_full[ib], iph, 420u)) break;
             tb_fence_after();
             const float2 mlr = ml[ib * TB_M + r];
-            const size_t ph = ((size_t)(live ? T.slot[q] : 0) * a.Hq) + (size_t)T.h * a.hpg + hh;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&ml_empty[ib]);
             __nv_bfloat16* po = a.P.part_o + ph * D;
             // the row normalised by its own sum (a convex combination of V rows)
             const float inv = (mlr.y > 0.f) ? 1.f / mlr.y : 0.f;
@@ -706,10 +762,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             if (live) a.P.part_ml[ph] = mlr;
             tb_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                ptx::mbar_arrive(&o_empty[ib]);
-                ptx::mbar_arrive(&info_empty[ib]);
-            }
+            if (lane == 0) ptx::mbar_arrive(&o_empty[ib]);
         }
     }
     tb_fence_before();
