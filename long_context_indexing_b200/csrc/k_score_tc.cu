@@ -28,6 +28,7 @@
 
 #include "lsa_internal.cuh"
 #include "ptx.cuh"
+#include "tmap.cuh"
 
 namespace lsa {
 
@@ -292,30 +293,9 @@ __global__ void __launch_bounds__(TC_THREADS, TC_MIN_BLOCKS) score_topk_tc_kerne
 }
 
 // ---- host side ---------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = (EncodeTiledFn)p;
-    }
-    return fn;
-}
-
 static bool make_rows64_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows)
 {
-    EncodeTiledFn enc = encode_fn();
+    TmapEncodeFn enc = tmap_encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)DL, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)DL * 2};

@@ -6,8 +6,8 @@ oracle.attend on the oracle's selection (bf16 bars: 2e-2 max-abs, 2e-3
 mean-abs).  Cases: a chunk that ends inside a block (open-block members are
 taken), a chunk that starts at position 0 (sinks and window overlap, block-0
 buckets cut by the sinks bound), several sequences, every supported head
-shape, workspaces with too few partial slots (some or all rows then go
-through the per-query kernel), and exact-fallback rows.
+shape, pooling factors 2 and 8, workspaces with too few partial slots (some
+or all rows then go through the per-query kernel), and exact-fallback rows.
 """
 import numpy as np
 import pytest
@@ -116,6 +116,14 @@ def test_several_sequences():
 def test_head_shapes(Hq, Hkv, d):
     w = _base(T=3000, nq=400, Hq=Hq, Hkv=Hkv, d=d)
     _run(w, seed=14)
+
+
+@pytest.mark.parametrize("p,G", [(2, 128), (8, 32)])
+def test_pooling_factors(p, G):
+    # other group sizes: p-row K/V boxes, and window groups that straddle the
+    # sinks' end (S = 5 is no multiple of p)
+    w = _base(T=3000, nq=500, p=p, G=G, S=5)
+    _run(w, seed=20 + p)
 
 
 def test_large_buckets_span_several_stages():
