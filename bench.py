@@ -349,22 +349,19 @@ def run_lsa(args, rank, ws):
                 "traffic": traffic["dram_bytes_per_call"] if traffic else None,
                 "launch_ms": round(attn_ms, 4)}
 
-    # End to end through the C-ABI with host buffers: H2D of the step's inputs
-    # (the chunk's new latent/K/V rows, latent queries, queries), the fused
-    # call, D2H of the output.
-    h = {k: inp[k][:, T_old:w.T].cpu().pin_memory() for k in ("latent_K", "K", "V")}
+    # End to end through the C-ABI with host buffers (lsa_prefill_chunk_host):
+    # H2D of the step's inputs from page-locked memory (the chunk's new
+    # latent/K/V rows, latent queries, queries), the chunk, D2H of the output.
+    h = {k: inp[k][:, T_old:w.T].cpu().contiguous().pin_memory() for k in ("latent_K", "K", "V")}
     hq = {k: inp[k].cpu().pin_memory() for k in ("latent_Q", "Q")}
     hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in list(h.values()) + list(hq.values()))
     d2h = hO.numel() * hO.element_size()
 
     def e2e_step():
-        for k in ("latent_K", "K", "V"):
-            inp[k][:, T_old:w.T].copy_(h[k], non_blocking=True)
-        for k in ("latent_Q", "Q"):
-            inp[k].copy_(hq[k], non_blocking=True)
-        step()
-        hO.copy_(O, non_blocking=True)
+        lsa.lsa_prefill_chunk_host(idx, h["latent_K"], h["K"], h["V"], hq["latent_Q"], hq["Q"],
+                                   inp["latent_K"], inp["K"], inp["V"], inp["latent_Q"], inp["Q"],
+                                   T_old, w.T, w.R, w.W, w.S, work, O, hO)
 
     for _ in range(2):
         e2e_step()

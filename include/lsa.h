@@ -290,6 +290,27 @@ lsa_status lsa_prefill_attend(const lsa_index* idx, const void* Q, const void* K
                               lsa_select_params sp, void* workspace, size_t ws_bytes, void* O,
                               void* stream);
 
+/* lsa_prefill_chunk with the chunk's inputs and its output in host memory
+ * (this library's own entry; the pages serve from device caches).  The
+ * chunk's new rows h_latent_K [B][Nq][64] and h_K, h_V [B][Nq][Hkv][d] are
+ * copied into the device caches latent_K, K, V at rows [T_old, T_new) of every
+ * sequence, h_latent_Q [B][Nq][64] into latent_Q and h_Q [B][Nq][Hq][d] into Q
+ * (all in the index's dtype); after the chunk, O [B][Nq][Hq][d] is copied to
+ * h_O.  The latent rows travel first on `stream`; K, V and Q travel on
+ * `copy_stream` while the index extension and the selection run on `stream`,
+ * and the attention waits for them, so those copies overlap the selection.
+ * Host buffers should be page-locked (pageable memory works but does not
+ * overlap).  copy_stream must differ from stream; an event orders it after the
+ * work queued on stream before the call.  Every check of lsa_prefill_chunk is
+ * made before the first copy; a failure after that is LSA_ERR_CUDA.  On return
+ * the work is queued: h_O is valid once `stream` has synchronised. */
+lsa_status lsa_prefill_chunk_host(lsa_index* idx, const void* h_latent_K, const void* h_K,
+                                  const void* h_V, const void* h_latent_Q, const void* h_Q,
+                                  void* latent_K, void* K, void* V, void* latent_Q, void* Q,
+                                  int64_t T_old, int64_t T_new, int Hq, int Hkv, int d,
+                                  lsa_select_params sp, void* workspace, size_t ws_bytes,
+                                  void* O, void* h_O, void* stream, void* copy_stream);
+
 /* Workspace bytes for lsa_decode_step (depends on the device's SM count). */
 size_t lsa_decode_workspace_bytes(const lsa_index* idx, int Hq, int Hkv, int d,
                                   lsa_select_params sp);

@@ -20,6 +20,7 @@ __all__ = [
     "LsaError", "LsaIndex", "lsa_index_bytes", "lsa_build_index", "lsa_select",
     "lsa_sparse_attn", "lsa_prefill_chunk", "lsa_prefill_workspace_bytes",
     "lsa_prefill_partial_slots", "lsa_prefill_select", "lsa_prefill_attend",
+    "lsa_prefill_chunk_host",
     "lsa_decode_workspace_bytes", "lsa_decode_step", "lsa_select_noalloc", "library_path", "kernel_launches", "F32",
     "BF16",
 ]
@@ -72,6 +73,8 @@ def _declare(lib):
                               I),
         "lsa_prefill_select": ([P, P, P, I64, I64, I, I, I, SelectParams, P, SZ, P], I),
         "lsa_prefill_attend": ([P, P, P, P, I64, I64, I, I, I, SelectParams, P, SZ, P, P], I),
+        "lsa_prefill_chunk_host": ([P, P, P, P, P, P, P, P, P, P, P, I64, I64, I, I, I,
+                                    SelectParams, P, SZ, P, P, P, P], I),
         "lsa_decode_workspace_bytes": ([P, I, I, I, SelectParams], SZ),
         "lsa_select_noalloc": ([P, P, P, I64, SelectParams, P, P, I, P], I),
         "lsa_decode_step": ([P, P, P, P, P, P, P, P, P, P, I, I, I, SelectParams, P, SZ, P, P], I),
@@ -109,6 +112,10 @@ def _check(rc):
 
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _hptr(t):
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream=None):
@@ -309,6 +316,39 @@ def lsa_prefill_chunk(index, latent_K, latent_Q, Q, K, V, T_old, T_new, budget, 
                                   SelectParams(budget, window, sinks), _ptr(workspace),
                                   workspace.numel(), _ptr(O), _stream(stream)))
     return O
+
+
+_copy_streams = {}
+
+
+def lsa_prefill_chunk_host(index, h_latent_K, h_K, h_V, h_latent_Q, h_Q, latent_K, K, V,
+                           latent_Q, Q, T_old, T_new, budget, window, sinks, workspace, out,
+                           h_out, stream=None, copy_stream=None):
+    """A prefill chunk from host inputs to a host output (C: lsa_prefill_chunk_host).
+
+    h_latent_K [B][Nq][64], h_K and h_V [B][Nq][Hkv][d] are the chunk's new cache
+    rows, h_latent_Q and h_Q its queries (page-locked CPU tensors); they are
+    copied into the device tensors latent_K, K, V (at rows [T_old, T_new)),
+    latent_Q and Q, and O (`out`) is copied back to `h_out`.  K, V and Q
+    travel on `copy_stream` (one per device is kept when not given) under the
+    selection.  Returns h_out, valid once `stream` has synchronised."""
+    _cuda(latent_K, K, V, latent_Q, Q, workspace, out)
+    for t in (h_latent_K, h_K, h_V, h_latent_Q, h_Q, h_out):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host tensors must be contiguous CPU tensors")
+    B, Nq, Hq, d = Q.shape
+    Hkv = K.shape[2]
+    if copy_stream is None:
+        dev = Q.device.index
+        if dev not in _copy_streams:
+            _copy_streams[dev] = torch.cuda.Stream(device=Q.device)
+        copy_stream = _copy_streams[dev]
+    _check(_lib.lsa_prefill_chunk_host(
+        index.handle, _hptr(h_latent_K), _hptr(h_K), _hptr(h_V), _hptr(h_latent_Q), _hptr(h_Q),
+        _ptr(latent_K), _ptr(K), _ptr(V), _ptr(latent_Q), _ptr(Q), int(T_old), int(T_new), Hq,
+        Hkv, d, SelectParams(budget, window, sinks), _ptr(workspace), workspace.numel(),
+        _ptr(out), _hptr(h_out), _stream(stream), _stream(copy_stream)))
+    return h_out
 
 
 def lsa_prefill_select(index, latent_K, latent_Q, T_old, T_new, Hq, Hkv, d, budget, window,

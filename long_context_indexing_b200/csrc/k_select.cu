@@ -338,22 +338,33 @@ __device__ int build_open_list(const IndexView& ix, int64_t bseq, int32_t* ol_o,
 {
     const int32_t* open = ix.open_bucket + bseq * ix.G;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    constexpr int U = 8;   // loads in flight per thread
     int base = 0;
-    for (int x0 = 0; x0 < ix.G; x0 += blockDim.x) {
-        const int x = x0 + threadIdx.x;
-        const int32_t g = (x < ix.G) ? open[x] : -1;
-        const unsigned bal = __ballot_sync(0xffffffffu, g >= 0);
-        if (lane == 0) cnt_s[warp] = __popc(bal);
-        __syncthreads();
-        int before = base;
-        for (int w = 0; w < warp; ++w) before += cnt_s[w];
-        if (g >= 0) {
-            const int at = before + __popc(bal & ((1u << lane) - 1u));
-            ol_o[at] = x;
-            ol_g[at] = g;
+    for (int x00 = 0; x00 < ix.G; x00 += U * (int)blockDim.x) {
+        int32_t gv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int x = x00 + u * (int)blockDim.x + (int)threadIdx.x;
+            gv[u] = (x < ix.G) ? open[x] : -1;
         }
-        for (int w = 0; w < nw; ++w) base += cnt_s[w];
-        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (x00 + u * (int)blockDim.x >= ix.G) break;   // uniform over the CTA
+            const int x = x00 + u * (int)blockDim.x + (int)threadIdx.x;
+            const int32_t g = gv[u];
+            const unsigned bal = __ballot_sync(0xffffffffu, g >= 0);
+            if (lane == 0) cnt_s[warp] = __popc(bal);
+            __syncthreads();
+            int before = base;
+            for (int w = 0; w < warp; ++w) before += cnt_s[w];
+            if (g >= 0) {
+                const int at = before + __popc(bal & ((1u << lane) - 1u));
+                ol_o[at] = x;
+                ol_g[at] = g;
+            }
+            for (int w = 0; w < nw; ++w) base += cnt_s[w];
+            __syncthreads();
+        }
     }
     return base;
 }

@@ -630,6 +630,73 @@ lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* l
                               stream);
 }
 
+lsa_status lsa_prefill_chunk_host(lsa_index* idx, const void* h_latent_K, const void* h_K,
+                                  const void* h_V, const void* h_latent_Q, const void* h_Q,
+                                  void* latent_K, void* K, void* V, void* latent_Q, void* Q,
+                                  int64_t T_old, int64_t T_new, int Hq, int Hkv, int d,
+                                  lsa_select_params sp, void* workspace, size_t ws_bytes,
+                                  void* O, void* h_O, void* stream, void* copy_stream)
+{
+    if (!idx || !h_latent_K || !h_K || !h_V || !h_latent_Q || !h_Q || !latent_K || !K || !V ||
+        !latent_Q || !Q || !O || !h_O)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    if (stream == copy_stream) return fail(LSA_ERR_INVALID_ARG, "copy_stream must differ from stream");
+    PrefillLayout L;
+    BucketPlan P;
+    lsa_status s = prefill_prepare(idx, T_old, T_new, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
+    if (s != LSA_OK) return s;
+    if (!aligned16(latent_K) || !aligned16(latent_Q) || !aligned16(Q) || !aligned16(K) ||
+        !aligned16(V) || !aligned16(O))
+        return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    const IndexView& v = idx->v;
+    const size_t es = (v.dtype == LSA_BF16) ? 2 : 4;
+    const int64_t Nq = T_new - T_old, B = v.B;
+    const size_t lat_row = (size_t)DL * es, kv_row = (size_t)Hkv * d * es;
+    cudaStream_t st = (cudaStream_t)stream, cs = (cudaStream_t)copy_stream;
+    // one pair of events per host thread, reused call after call
+    static thread_local cudaEvent_t ev_in = nullptr, ev_kvq = nullptr;
+    cudaError_t e = cudaSuccess;
+    if (!ev_in) e = cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming);
+    if (e == cudaSuccess && !ev_kvq) e = cudaEventCreateWithFlags(&ev_kvq, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "event create");
+    // the copy stream starts after the work already queued on stream (which
+    // may still read the caches and Q)
+    e = cudaEventRecord(ev_in, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ev_in, 0);
+    // the latent rows first, on stream: the extension and the selection need them
+    for (int64_t b = 0; b < B && e == cudaSuccess; ++b)
+        e = cudaMemcpyAsync((char*)latent_K + ((size_t)b * v.T_cap + T_old) * lat_row,
+                            (const char*)h_latent_K + (size_t)b * Nq * lat_row, Nq * lat_row,
+                            cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(latent_Q, h_latent_Q, (size_t)B * Nq * lat_row, cudaMemcpyHostToDevice,
+                            st);
+    // K, V and Q on the copy stream, under the selection
+    for (int64_t b = 0; b < B && e == cudaSuccess; ++b) {
+        const size_t dst = ((size_t)b * v.T_cap + T_old) * kv_row, src = (size_t)b * Nq * kv_row;
+        e = cudaMemcpyAsync((char*)K + dst, (const char*)h_K + src, Nq * kv_row,
+                            cudaMemcpyHostToDevice, cs);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync((char*)V + dst, (const char*)h_V + src, Nq * kv_row,
+                                cudaMemcpyHostToDevice, cs);
+    }
+    const size_t q_bytes = (size_t)B * Nq * Hq * d * es;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(Q, h_Q, q_bytes, cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_kvq, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copies");
+    s = lsa_prefill_select(idx, latent_K, latent_Q, T_old, T_new, Hq, Hkv, d, sp, workspace,
+                           ws_bytes, stream);
+    if (s != LSA_OK) return s;
+    e = cudaStreamWaitEvent(st, ev_kvq, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "copy join");
+    s = lsa_prefill_attend(idx, Q, K, V, T_old, T_new, Hq, Hkv, d, sp, workspace, ws_bytes, O,
+                           stream);
+    if (s != LSA_OK) return s;
+    e = cudaMemcpyAsync(h_O, O, q_bytes, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+    return LSA_OK;
+}
+
 size_t lsa_decode_workspace_bytes(const lsa_index* idx, int Hq, int Hkv, int d,
                                   lsa_select_params sp)
 {

@@ -176,3 +176,66 @@ def test_recommended_workspace_gives_the_recommended_slots():
     per_row = min(65, (3 * w.R + 2 * bk - 1) // (2 * bk) + 2)
     assert lsa.lsa_prefill_partial_slots(gpu, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S,
                                          nbytes) == w.B * w.nq * per_row
+
+
+@pytest.mark.parametrize("dtype,B", [("bf16", 1), ("bf16", 2), ("f32", 2)])
+def test_host_entry_matches_device_entry(dtype, B):
+    # lsa_prefill_chunk_host copies the chunk's rows and queries in (K, V, Q on
+    # a second stream, under the selection), runs the chunk and copies O out:
+    # the same output as lsa_prefill_chunk on device inputs, bit for bit
+    w = _base(B=B, dtype=dtype)
+    T_old = w.T - w.nq
+    inp = synth.prefill_inputs(w, 22, "cpu")
+    lt = lsa.BF16 if dtype == "bf16" else lsa.F32
+
+    def fresh_index(latent_K):
+        idx = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lt)
+        idx.build(latent_K, T_old)
+        nb = lsa.lsa_prefill_workspace_bytes(idx, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S)
+        return idx, torch.empty(nb, dtype=torch.uint8, device="cuda")
+
+    dev = {k: v.cuda() for k, v in inp.items()}
+    idx, ws = fresh_index(dev["latent_K"])
+    O_dev = lsa.lsa_prefill_chunk(idx, dev["latent_K"], dev["latent_Q"], dev["Q"], dev["K"],
+                                  dev["V"], T_old, w.T, w.R, w.W, w.S, workspace=ws)
+    torch.cuda.synchronize()
+
+    # device caches hold only the prefix; the chunk's rows and queries come from host
+    dev2 = {k: v.cuda() for k, v in inp.items()}
+    for k in ("latent_K", "K", "V"):
+        dev2[k][:, T_old:w.T] = 0
+    dev2["latent_Q"].zero_()
+    dev2["Q"].zero_()
+    h = {k: inp[k][:, T_old:w.T].contiguous().pin_memory() for k in ("latent_K", "K", "V")}
+    hq = {k: inp[k].contiguous().pin_memory() for k in ("latent_Q", "Q")}
+    idx2, ws2 = fresh_index(dev2["latent_K"])
+    O2 = torch.empty_like(dev2["Q"])
+    hO = torch.empty(O2.shape, dtype=O2.dtype, pin_memory=True)
+    lsa.lsa_prefill_chunk_host(idx2, h["latent_K"], h["K"], h["V"], hq["latent_Q"], hq["Q"],
+                               dev2["latent_K"], dev2["K"], dev2["V"], dev2["latent_Q"], dev2["Q"],
+                               T_old, w.T, w.R, w.W, w.S, ws2, O2, hO)
+    torch.cuda.synchronize()
+    assert idx2.check() == idx.check()
+    assert torch.equal(hO, O_dev.cpu())
+    assert torch.equal(dev2["K"], dev["K"]) and torch.equal(dev2["V"], dev["V"])
+    assert torch.equal(dev2["latent_K"], dev["latent_K"])
+
+
+def test_host_entry_rejects_one_stream():
+    w = _base()
+    T_old = w.T - w.nq
+    inp = synth.prefill_inputs(w, 23, "cpu")
+    dev = {k: v.cuda() for k, v in inp.items()}
+    idx = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16)
+    idx.build(dev["latent_K"], T_old)
+    nb = lsa.lsa_prefill_workspace_bytes(idx, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    h = {k: inp[k][:, T_old:w.T].contiguous().pin_memory() for k in ("latent_K", "K", "V")}
+    hq = {k: inp[k].contiguous().pin_memory() for k in ("latent_Q", "Q")}
+    O = torch.empty_like(dev["Q"])
+    hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    s = torch.cuda.current_stream()
+    with pytest.raises(lsa.LsaError):
+        lsa.lsa_prefill_chunk_host(idx, h["latent_K"], h["K"], h["V"], hq["latent_Q"], hq["Q"],
+                                   dev["latent_K"], dev["K"], dev["V"], dev["latent_Q"], dev["Q"],
+                                   T_old, w.T, w.R, w.W, w.S, ws, O, hO, stream=s, copy_stream=s)
