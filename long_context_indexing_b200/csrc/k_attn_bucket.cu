@@ -443,32 +443,29 @@ constexpr int MERGE_THREADS = 256;
 constexpr int MERGE_MAX_SLOTS = KC + 1;
 constexpr int MERGE_MAX_HEADS = 64;
 
-__global__ void __launch_bounds__(MERGE_THREADS, 6) bucket_merge_kernel(BucketPlan P, int Hq, int D,
+__global__ void __launch_bounds__(MERGE_THREADS) bucket_merge_kernel(BucketPlan P, int Hq, int D,
                                                                      __nv_bfloat16* O)
 {
-    // [slot][head]: the partials' (max, sum), then (max, normalised weight)
-    extern __shared__ float2 mlw_s[];
+    __shared__ float w_s[MERGE_MAX_SLOTS * MERGE_MAX_HEADS];   // weights [slot][head], normalised
     const int64_t row = blockIdx.x;
     const int nt = P.row_n[row];
     if (nt < 0) return;                        // gather row: written by the per-query kernel
     const int ns = nt + 1;
     const int64_t base = (int64_t)P.row_base[row] * Hq;   // first (slot, head)
     const float2* ml = P.part_ml + base;
-    // every (slot, head) pair at once, then one pass per head in shared memory
-    for (int x = threadIdx.x; x < ns * Hq; x += MERGE_THREADS) mlw_s[x] = __ldcg(&ml[x]);
-    __syncthreads();
+    // raw weights exp2(m) as pairs first: one pass per head over its slots
     for (int h = threadIdx.x; h < Hq; h += MERGE_THREADS) {
         float M = -INFINITY;
-        for (int sl = 0; sl < ns; ++sl) M = fmaxf(M, mlw_s[sl * Hq + h].x);
+        for (int sl = 0; sl < ns; ++sl) M = fmaxf(M, __ldcg(&ml[(int64_t)sl * Hq + h]).x);
         float L = 0.f;
         for (int sl = 0; sl < ns; ++sl) {
-            const float2 v = mlw_s[sl * Hq + h];
+            const float2 v = __ldcg(&ml[(int64_t)sl * Hq + h]);
             const float wv = (v.x == -INFINITY) ? 0.f : v.y * exp2f(v.x - M);
-            mlw_s[sl * Hq + h].y = wv;
+            w_s[sl * Hq + h] = wv;
             L += wv;
         }
         const float inv = 1.f / L;
-        for (int sl = 0; sl < ns; ++sl) mlw_s[sl * Hq + h].y *= inv;
+        for (int sl = 0; sl < ns; ++sl) w_s[sl * Hq + h] *= inv;
     }
     __syncthreads();
     const int n8 = Hq * D / 8;                 // 16-byte groups of the row's output
@@ -482,7 +479,7 @@ __global__ void __launch_bounds__(MERGE_THREADS, 6) bucket_merge_kernel(BucketPl
 #pragma unroll 4
         for (int sl = 0; sl < ns; ++sl) {
             const uint4 u = __ldcg(reinterpret_cast<const uint4*>(src + (int64_t)sl * Hq * D) + c);
-            const float wv = mlw_s[sl * Hq + h].y;
+            const float wv = w_s[sl * Hq + h];
             const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -563,9 +560,8 @@ cudaError_t launch_bucket_attn(const IndexView& ix, int64_t n_blk, const BucketP
     e = launch_attn_rows(Q, K, V, ix.B, Nq, ix.T_cap, Hq, Hkv, d, indices, counts, s_max, scale, O,
                          ix.status, P.gather_rows, P.ctr + CTR_GATHER, st);
     if (e != cudaSuccess) return e;
-    bucket_merge_kernel<<<(unsigned)(ix.B * Nq), MERGE_THREADS,
-                          (size_t)MERGE_MAX_SLOTS * Hq * sizeof(float2), st>>>(P, Hq, d,
-                                                                              (__nv_bfloat16*)O);
+    bucket_merge_kernel<<<(unsigned)(ix.B * Nq), MERGE_THREADS, 0, st>>>(P, Hq, d,
+                                                                        (__nv_bfloat16*)O);
     note_launch();
     return cudaGetLastError();
 }
