@@ -333,7 +333,12 @@ size_t lsa_decode_workspace_bytes(const lsa_index* idx, int Hq, int Hkv, int d,
  *      (split over keys, partials combined in fp32), scale 1/sqrt(d).
  * The selection of step 3 never depends on the append of step 2 (a group
  * that completes at pos lies inside the recent window), so the two run
- * concurrently.  Graph-capturable: no synchronisation, no allocation. */
+ * concurrently.  Graph-capturable: no synchronisation, no allocation.
+ * When the sequences' open block is full (the step that wrote its last key,
+ * pos[b] + 1 a multiple of p * block for every b), the caller closes it with
+ * lsa_index_extend(idx, latent_K, pos + 1 - p * block, pos + 1): the block is
+ * clustered into buckets like any other and decoding continues into an empty
+ * open block after it. */
 lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
                            const void* new_latent_k, const void* new_k, const void* new_v,
                            const void* latent_q, const void* q, const int32_t* pos, int Hq,
