@@ -41,29 +41,51 @@ PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 # ------------------------------------------------------------------ helpers --
 
-def _dist():
+def _dist(timeout_s=300):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE / MASTER_*):
+    NCCL on GPUs; gloo where no GPU is visible (the host-side logic, on CPU)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws > 1 and not torch.distributed.is_initialized():
         import datetime
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        torch.distributed.init_process_group(backend,
+                                             timeout=datetime.timedelta(seconds=timeout_s))
     rank = torch.distributed.get_rank() if ws > 1 else 0
     return rank, ws
 
 
+def _coll_device():
+    return ("cuda" if torch.distributed.is_initialized()
+            and torch.distributed.get_backend() == "nccl" else "cpu")
+
+
 def _max_over_ranks(x, ws):
+    """The largest of every rank's x (every rank gets it)."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_coll_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
 
+def _sync():
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
 def _barrier(ws):
-    torch.cuda.synchronize()
+    _sync()
     if ws > 1:
         torch.distributed.barrier()
-        torch.cuda.synchronize()
+        _sync()
+
+
+def _job_rate(units_per_rank, ms_max, ws):
+    """Whole-job throughput: the units all ranks processed / the slowest
+    rank's time (weak scaling: every rank processes its own units)."""
+    return ws * units_per_rank / (ms_max * 1e-3)
 
 
 def _peaks():
@@ -388,13 +410,13 @@ def run_lsa(args, rank, ws):
         torch.cuda.empty_cache()
         decode = run_decode(args, peaks, peak_src, ws)
 
-    value = ws * w.nq / (ms * 1e-3)
+    value = _job_rate(w.nq, ms, ws)
     line = {"metric": METRIC, "value": round(value, 2), "unit": "queries/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic (seeded clustered mixture; no model weights or datasets)",
             "config": _config(w, ws), "roofline": roofline, "cpu_baseline": cpu,
-            "e2e": {"value": round(ws * w.nq / (e2e_ms * 1e-3), 2), "unit": "queries/s",
+            "e2e": {"value": round(_job_rate(w.nq, e2e_ms, ws), 2), "unit": "queries/s",
                     "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches, "clocks": clocks,

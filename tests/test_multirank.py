@@ -1,0 +1,76 @@
+"""The N > 1 path of bench.py on CPU: world size 2 over gloo.
+
+Under torchrun bench.py runs one process per GPU.  Every rank processes its
+own chunk (the path shards by independent problems: no collective on the data
+path), the step time is the max over ranks, the value is the units of all
+ranks over that time, and rank 0 alone prints the JSON line.  Here the ranks
+are CPU processes over gloo (bench picks gloo when no GPU is visible):
+- the rank helpers agree on every rank (barrier, max over ranks, job rate);
+- the reference arm under torchrun prints exactly one line, from rank 0,
+  with n_gpus = 2, and every rank exits 0.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_worker(rank, ws, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(ws), LOCAL_RANK=str(rank), CUDA_VISIBLE_DEVICES="")
+    sys.path.insert(0, ROOT)
+    import bench
+    r, w = bench._dist(timeout_s=60)
+    local_ms = 10.0 + 5.0 * r              # rank 1 is the slower one
+    bench._barrier(w)
+    mx = bench._max_over_ranks(local_ms, w)
+    rate = bench._job_rate(32768, mx, w)
+    backend = torch.distributed.get_backend()
+    torch.distributed.destroy_process_group()
+    q.put((r, w, mx, rate, backend))
+
+
+def test_rank_helpers_over_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r for r, *_ in res] == [0, 1]
+    for _, w, mx, rate, backend in res:
+        assert w == 2 and backend == "gloo"
+        assert mx == 15.0                                  # the slowest rank's time
+        assert rate == 2 * 32768 / 0.015                   # both ranks' queries / that time
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+           "--steps", "1", "--warmup", "3", "--ref-queries", "4", "--gpus", "2"]
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", OMP_NUM_THREADS="2")
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=600, env=env, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-3000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["n_gpus"] == 2 and j["scaling"] == "weak"
+    assert j["value"] > 0 and j["cpu_baseline"]["kind"] == "oracle"
