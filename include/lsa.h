@@ -311,6 +311,16 @@ lsa_status lsa_prefill_chunk_host(lsa_index* idx, const void* h_latent_K, const 
                                   lsa_select_params sp, void* workspace, size_t ws_bytes,
                                   void* O, void* h_O, void* stream, void* copy_stream);
 
+/* Test hook (this library's own; not part of the method): the number of
+ * polls each bounded wait of the tensor-core centroid scorer (bf16 selection
+ * with Nq >= 128) makes before it gives up.  A wait that gives up records
+ * LSA_ERR_TIMEOUT for lsa_index_check, and the kernel still leaves cleanly
+ * (its copies and MMAs in flight are waited for with the default limit), so
+ * the context stays usable.  polls < 0 restores the default (about 4
+ * million); 0 makes every such wait give up at once.  Synchronous; applies to
+ * later launches on the current device. */
+lsa_status lsa_set_wait_limit(int64_t polls);
+
 /* Workspace bytes for lsa_decode_step (depends on the device's SM count). */
 size_t lsa_decode_workspace_bytes(const lsa_index* idx, int Hq, int Hkv, int d,
                                   lsa_select_params sp);

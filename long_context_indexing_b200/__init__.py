@@ -20,7 +20,7 @@ __all__ = [
     "LsaError", "LsaIndex", "lsa_index_bytes", "lsa_build_index", "lsa_select",
     "lsa_sparse_attn", "lsa_prefill_chunk", "lsa_prefill_workspace_bytes",
     "lsa_prefill_partial_slots", "lsa_prefill_select", "lsa_prefill_attend",
-    "lsa_prefill_chunk_host",
+    "lsa_prefill_chunk_host", "set_wait_limit",
     "lsa_decode_workspace_bytes", "lsa_decode_step", "lsa_select_noalloc", "library_path", "kernel_launches", "F32",
     "BF16",
 ]
@@ -76,6 +76,7 @@ def _declare(lib):
         "lsa_prefill_chunk_host": ([P, P, P, P, P, P, P, P, P, P, P, I64, I64, I, I, I,
                                     SelectParams, P, SZ, P, P, P, P], I),
         "lsa_decode_workspace_bytes": ([P, I, I, I, SelectParams], SZ),
+        "lsa_set_wait_limit": ([I64], I),
         "lsa_select_noalloc": ([P, P, P, I64, SelectParams, P, P, I, P], I),
         "lsa_decode_step": ([P, P, P, P, P, P, P, P, P, P, I, I, I, SelectParams, P, SZ, P, P], I),
     }
@@ -316,6 +317,12 @@ def lsa_prefill_chunk(index, latent_K, latent_Q, Q, K, V, T_old, T_new, budget, 
                                   SelectParams(budget, window, sinks), _ptr(workspace),
                                   workspace.numel(), _ptr(O), _stream(stream)))
     return O
+
+
+def set_wait_limit(polls):
+    """Test hook (C: lsa_set_wait_limit): polls each bounded wait of the
+    tensor-core scorer makes before it gives up; polls < 0 restores the default."""
+    _check(_lib.lsa_set_wait_limit(int(polls)))
 
 
 _copy_streams = {}

@@ -28,6 +28,7 @@
 
 #include "lsa_internal.cuh"
 #include "ptx.cuh"
+#include "hooks.cuh"
 #include "tmap.cuh"
 
 namespace lsa {
@@ -43,11 +44,16 @@ constexpr int TC_STAGES = 4;
 constexpr int TC_THREADS = 192;
 constexpr uint32_t TC_WAIT = 1u << 22;
 
+// Polls each bounded wait of the scorer's roles makes before it gives up.  A
+// test hook (lsa_set_wait_limit) lowers it to make the waits run out; the
+// drains on the way out always allow TC_WAIT.
+__device__ uint32_t g_tc_wait = TC_WAIT;
+
 constexpr int TC_Q_BYTES = TC_M * DL * 2;                 // 16 KB
 constexpr int TC_C_BYTES = TC_N * DL * 2;                 // 32 KB per stage at N = 256
 constexpr int TC_OFF_C = TC_Q_BYTES;
 constexpr int TC_OFF_BAR = TC_OFF_C + TC_STAGES * TC_C_BYTES;
-constexpr int TC_NBAR = 1 + 2 * TC_STAGES + 4;
+constexpr int TC_NBAR = 1 + 2 * TC_STAGES + 4 + 1;
 constexpr int TC_OFF_MISC = TC_OFF_BAR + TC_NBAR * 8;
 constexpr int TC_SMEM = TC_OFF_MISC + 64 + 1024;          // + alignment slack
 
@@ -142,6 +148,7 @@ __global__ void __launch_bounds__(TC_THREADS, TC_MIN_BLOCKS) score_topk_tc_kerne
     uint64_t* empty = full + TC_STAGES;
     uint64_t* acc_full = empty + TC_STAGES;
     uint64_t* acc_empty = acc_full + 2;
+    uint64_t* fin = acc_empty + 2;        // the MMA thread's last MMAs are done
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + TC_OFF_MISC);
     volatile uint32_t* tmem_slot = misc;        // [0]
     volatile uint32_t* abort_flag = misc + 1;   // [1]
@@ -168,6 +175,7 @@ __global__ void __launch_bounds__(TC_THREADS, TC_MIN_BLOCKS) score_topk_tc_kerne
             ptx::mbar_init(&acc_full[a], 1);
             ptx::mbar_init(&acc_empty[a], 4);
         }
+        ptx::mbar_init(fin, 1);
         *abort_flag = 0;
         *nb_max = 0;
         ptx::fence_mbar_init();
@@ -194,16 +202,18 @@ __global__ void __launch_bounds__(TC_THREADS, TC_MIN_BLOCKS) score_topk_tc_kerne
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int n_tiles = (int)((*nb_max + TC_N - 1) / TC_N);
+    const uint32_t wl = g_tc_wait;
 
     if (warp == 0 && lane == 0 && n_tiles > 0) {
         // ---------------- TMA producer ----------------
         ptx::mbar_arrive_expect_tx(q_full, TC_Q_BYTES);
         tma_load_2d(q_s, &tmQ, 0, (int)(b * Nq + q0), q_full);
+        int issued = 0;
         for (int t = 0; t < n_tiles; ++t) {
             const int s = t % TC_STAGES;
             const uint32_t ph = (uint32_t)((t / TC_STAGES) & 1);
             if (*abort_flag) break;
-            if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1u, TC_WAIT)) {
+            if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1u, wl)) {
                 *abort_flag = 1;
                 dev_error(ix.status, DEV_TIMEOUT, 1000u + (uint32_t)t);
                 break;
@@ -211,10 +221,20 @@ __global__ void __launch_bounds__(TC_THREADS, TC_MIN_BLOCKS) score_topk_tc_kerne
             ptx::mbar_arrive_expect_tx(&full[s], TC_C_BYTES);
             tma_load_2d(c_s + s * TC_C_BYTES, &tmC, 0, (int)(b * ix.NBK + (int64_t)t * TC_N),
                         &full[s]);
+            issued = t + 1;
+        }
+        if (*abort_flag) {
+            // no copy may still be writing shared memory when the CTA exits:
+            // the latest load of every stage (and the query tile) has landed,
+            // or a bounded wait gives up on it
+            ptx::mbar_wait_bounded(q_full, 0, TC_WAIT);
+            for (int t = (issued > TC_STAGES ? issued - TC_STAGES : 0); t < issued; ++t)
+                ptx::mbar_wait_bounded(&full[t % TC_STAGES], (uint32_t)((t / TC_STAGES) & 1),
+                                       TC_WAIT);
         }
     } else if (warp == 1 && lane == 0 && n_tiles > 0) {
         // ---------------- MMA issuer ----------------
-        bool ok = ptx::mbar_wait_bounded(q_full, 0, TC_WAIT);
+        bool ok = ptx::mbar_wait_bounded(q_full, 0, wl);
         if (!ok) {
             *abort_flag = 1;
             dev_error(ix.status, DEV_TIMEOUT, 2000u);
@@ -226,8 +246,8 @@ __global__ void __launch_bounds__(TC_THREADS, TC_MIN_BLOCKS) score_topk_tc_kerne
             const int buf = t & 1;
             const uint32_t aph = (uint32_t)((t >> 1) & 1);
             if (*abort_flag) break;
-            if (!ptx::mbar_wait_bounded(&full[s], ph, TC_WAIT) ||
-                !ptx::mbar_wait_bounded(&acc_empty[buf], aph ^ 1u, TC_WAIT)) {
+            if (!ptx::mbar_wait_bounded(&full[s], ph, wl) ||
+                !ptx::mbar_wait_bounded(&acc_empty[buf], aph ^ 1u, wl)) {
                 *abort_flag = 1;
                 dev_error(ix.status, DEV_TIMEOUT, 3000u + (uint32_t)t);
                 break;
@@ -241,6 +261,9 @@ __global__ void __launch_bounds__(TC_THREADS, TC_MIN_BLOCKS) score_topk_tc_kerne
             mma_commit(&empty[s]);
             mma_commit(&acc_full[buf]);
         }
+        // nothing of this CTA may still run on the tensor cores when TMEM is freed
+        mma_commit(fin);
+        ptx::mbar_wait_bounded(fin, 0, TC_WAIT);
     } else if (warp >= 2) {
         // ---------------- epilogue ----------------
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
@@ -250,7 +273,7 @@ __global__ void __launch_bounds__(TC_THREADS, TC_MIN_BLOCKS) score_topk_tc_kerne
             const int buf = t & 1;
             const uint32_t ph = (uint32_t)((t >> 1) & 1);
             if (*abort_flag) break;
-            if (!ptx::mbar_wait_bounded(&acc_full[buf], ph, TC_WAIT)) {
+            if (!ptx::mbar_wait_bounded(&acc_full[buf], ph, wl)) {
                 *abort_flag = 1;
                 dev_error(ix.status, DEV_TIMEOUT, 4000u + (uint32_t)t);
                 break;
@@ -307,6 +330,12 @@ static bool make_rows64_bf16(CUtensorMap* m, const void* base, uint64_t rows, ui
 }
 
 bool tc_scoring_available() { return true; }
+
+cudaError_t set_score_wait_polls(int64_t polls)
+{
+    const uint32_t v = (polls < 0 || polls > (int64_t)TC_WAIT) ? TC_WAIT : (uint32_t)polls;
+    return cudaMemcpyToSymbol(g_tc_wait, &v, sizeof(v));
+}
 
 cudaError_t launch_score_topk_tc(const IndexView& ix, int64_t n_blk, const void* latent_Q,
                                  PosSrc pos, int64_t Nq, int W, const SelectWs& ws,

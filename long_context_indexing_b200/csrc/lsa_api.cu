@@ -11,6 +11,7 @@
 #include <atomic>
 #include <new>
 
+#include "hooks.cuh"
 #include "lsa_internal.cuh"
 
 using namespace lsa;
@@ -694,6 +695,13 @@ lsa_status lsa_prefill_chunk_host(lsa_index* idx, const void* h_latent_K, const 
     if (s != LSA_OK) return s;
     e = cudaMemcpyAsync(h_O, O, q_bytes, cudaMemcpyDeviceToHost, st);
     if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+    return LSA_OK;
+}
+
+lsa_status lsa_set_wait_limit(int64_t polls)
+{
+    cudaError_t e = set_score_wait_polls(polls);
+    if (e != cudaSuccess) return cuda_fail(e, "wait limit");
     return LSA_OK;
 }
 

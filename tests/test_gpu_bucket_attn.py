@@ -239,3 +239,30 @@ def test_host_entry_rejects_one_stream():
         lsa.lsa_prefill_chunk_host(idx, h["latent_K"], h["K"], h["V"], hq["latent_Q"], hq["Q"],
                                    dev["latent_K"], dev["K"], dev["V"], dev["latent_Q"], dev["Q"],
                                    T_old, w.T, w.R, w.W, w.S, ws, O, hO, stream=s, copy_stream=s)
+
+
+def test_scorer_wait_that_runs_out_reports_a_timeout():
+    # Failure detection without a fault: with the scorer's wait limit at 0
+    # polls every one of its waits gives up at once; the kernel records
+    # LSA_ERR_TIMEOUT, drains its copies and MMAs and leaves.  The context
+    # stays usable: with the default limit back, a chunk matches the oracle.
+    w = _base()
+    T_old = w.T - w.nq
+    inp = synth.prefill_inputs(w, 24, "cpu")
+    dev = {k: v.cuda() for k, v in inp.items()}
+    gpu = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16)
+    gpu.build(dev["latent_K"], T_old)
+    nb = lsa.lsa_prefill_workspace_bytes(gpu, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    lsa.set_wait_limit(0)
+    try:
+        lsa.lsa_prefill_select(gpu, dev["latent_K"], dev["latent_Q"], T_old, w.T, w.Hq, w.Hkv,
+                               w.d, w.R, w.W, w.S, ws)
+        torch.cuda.synchronize()
+        with pytest.raises(lsa.LsaError, match="TIMEOUT"):
+            gpu.check()
+    finally:
+        lsa.set_wait_limit(-1)
+    gpu.check()                          # the status word was cleared by the report
+    fb, _ = _run(w, seed=24)
+    assert fb == 0
