@@ -71,7 +71,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     return false;
 }
 
-// ---- bulk copy (non-tensor TMA), global -> shared, no multicast -----------
+// ---- bulk copy (non-tensor TMA), global -> shared, this CTA only ----------
 __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes,
                                          uint64_t* bar)
 {
