@@ -75,3 +75,37 @@ def test_open_assign_ties_go_to_lowest_bucket():
     idx.append(lat, w.T + w.steps)
     n_new = w.steps // w.p
     assert np.all(idx.open_bucket[:n_new] == 0)
+
+
+def test_closing_a_filled_open_block_equals_building_the_longer_prefix():
+    # The index past the open block: decode appends fill the open block, then
+    # extend over that block closes it.  The result is the index built over
+    # the longer prefix in one go (same pooled keys, centroids, CSR,
+    # assignments), with an empty open block.
+    w = synth.workload("decode", T=1024, B=1, M=16, G=16, k=4, R=200, W=8, S=4, steps=140,
+                       Hq=4, Hkv=1, d=64, dtype="f32")
+    inp = synth.decode_inputs(w, 5, "cpu")
+    lat = inp["latent_K"][0].numpy()
+    span = w.p * w.G
+    t_cap = w.T + w.steps + span
+    idx = oracle.Index(t_cap, w.p, w.G, w.k, w.L, rt_bf16=False)
+    idx.extend(lat, 0, w.T)
+    t_end = w.T
+    for pos in range(w.T, w.T + 2 * span):
+        idx.append(lat, pos + 1)
+        if (pos + 1) % span == 0:
+            assert np.all(idx.open_bucket >= 0)            # the block's G groups are all assigned
+            idx.extend(lat, pos + 1 - span, pos + 1)
+            t_end = pos + 1
+            assert np.all(idx.open_bucket == -1)
+    assert t_end == w.T + 2 * span and idx.n_blocks == t_end // span
+    ref = oracle.Index(t_cap, w.p, w.G, w.k, w.L, rt_bf16=False)
+    ref.extend(lat, 0, t_end)
+    nb, npool = ref.n_buckets, t_end // w.p
+    assert np.array_equal(idx.pooled[:npool], ref.pooled[:npool])
+    assert np.array_equal(idx.unit[:npool], ref.unit[:npool])
+    assert np.array_equal(idx.cent[:nb], ref.cent[:nb])
+    assert np.array_equal(idx.offsets[:nb + 1], ref.offsets[:nb + 1])
+    assert np.array_equal(idx.members[:npool], ref.members[:npool])
+    assert np.array_equal(idx.assign[:npool], ref.assign[:npool])
+    assert np.array_equal(idx.open_bucket, ref.open_bucket)
