@@ -14,9 +14,9 @@
 //                                                 two accumulators)
 //
 // Warp roles (15 warps):
-//   warp 0     planner: claims work items and copies each tile's description
-//              (written by bucket_tile_records_kernel) and the bucket's member
-//              lists into shared memory, one item ahead;
+//   warp 0     planner: claims work items (two ahead) and copies each tile's
+//              description (bucket_tile_records_kernel) and member lists into
+//              shared memory, prefetched to registers one item ahead;
 //   warps 1-2, 13-14  loaders: gather every stage's K and V rows of the KV
 //              head (16 keys per warp) with 16-byte cp.async into
 //              128-byte-swizzled planes (the layout the MMA descriptors name);
@@ -30,9 +30,9 @@
 //              TMEM over the scores, and at the end of the tile hands the
 //              row's (max, sum) on;
 //   warps 8-11 epilogue: write each row's partial (O row / sum as bf16, and
-//              the fp32 max and sum) from one
-//              of two TMEM accumulators (tiles alternate), overlapping the
-//              next tile's softmax.
+//              the fp32 max and sum) from one of two TMEM accumulators (tiles
+//              alternate), overlapping the next tile's softmax; softmax and
+//              epilogue keep what they need of a description in registers.
 // Q and tile descriptions are double-buffered across work items and the K/V
 // ring continues across them, so loads of the next tile overlap this one.  An
 // S buffer (and the P in it) is released by the commit of its P V MMA, so the
