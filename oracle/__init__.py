@@ -252,3 +252,68 @@ def attend(Q, K, V, idx, cnt, scale=None):
 def default_scale(d):
     """1/sqrt(d) rounded to binary32 (READING: the usual softmax scale)."""
     return float(np.float32(1.0 / math.sqrt(d)))
+
+
+# --------------------------------------------------------------------------
+# Per-key indexer: the comparison baseline LSA replaces [P4 "What it changes"]
+# --------------------------------------------------------------------------
+
+def per_key_scores(lat, q):
+    """<q, latent_k[t]> for every key row of lat [n][dl]: the exact products
+    summed in binary64 in ascending dimension (R10's rule, applied per key)."""
+    lat = np.asarray(lat, dtype=np.float64)
+    q = np.asarray(q, dtype=np.float64)
+    s = np.zeros(lat.shape[0], np.float64)
+    for d in range(lat.shape[1]):
+        s += lat[:, d] * q[d]
+    return s
+
+
+def select_per_key(lat, q, pos, R, W, S, s_max=None):
+    """Brute-force latent per-key indexer (READING of the indexer that LSA's
+    bucket retrieval replaces: every earlier key scored against the query, the
+    best ones read).  Per query at pos: every long-range-available key t
+    (S <= t <= pos - W, R11) is scored by per_key_scores; the R best keys are
+    taken (score descending, lowest position on ties).  Emitted: sinks, the
+    taken keys in ascending position, the recent window ascending (R13); -1
+    pads to s_max.
+
+    lat [>= max(pos)+1][dl] latent keys of the sequence, q [nq][dl], pos [nq].
+    Returns (indices [nq][s_max] int32, counts [nq] int32)."""
+    q = np.asarray(q)
+    pos = np.asarray(pos, dtype=np.int64)
+    nq = q.shape[0]
+    if s_max is None:
+        s_max = R + W + S
+    out = np.full((nq, s_max), -1, np.int32)
+    cnt = np.zeros(nq, np.int32)
+    for i in range(nq):
+        p = int(pos[i])
+        n_s = min(S, p + 1)
+        w0 = max(p - W + 1, n_s)
+        lo, hi = S, p - W                        # long-range keys [lo, hi]
+        taken = np.zeros(0, np.int64)
+        if hi >= lo and R > 0:
+            t = np.arange(lo, hi + 1, dtype=np.int64)
+            sc = per_key_scores(lat[lo:hi + 1], q[i])
+            order = np.lexsort((t, -sc))         # score desc, then position asc
+            taken = np.sort(t[order[:R]])
+        row = np.concatenate([np.arange(n_s, dtype=np.int64), taken,
+                              np.arange(w0, p + 1, dtype=np.int64)])
+        out[i, :row.size] = row
+        cnt[i] = row.size
+    return out, cnt
+
+
+def recall(sel_idx, sel_cnt, ref_idx, ref_cnt, pos, S, W):
+    """Per query at pos, the fraction of the reference's long-range keys
+    (S <= t <= pos - W) that the selection also reads; 1.0 where the reference
+    takes none."""
+    out = np.ones(len(sel_cnt), np.float64)
+    for i in range(len(sel_cnt)):
+        lo, hi = S, int(pos[i]) - W
+        ref = {int(x) for x in ref_idx[i, :ref_cnt[i]] if lo <= x <= hi}
+        if ref:
+            sel = {int(x) for x in sel_idx[i, :sel_cnt[i]]}
+            out[i] = len(ref & sel) / len(ref)
+    return out
