@@ -114,3 +114,35 @@ def test_calls_without_gpu_fail_cleanly():
     rc = lsa._lib.lsa_sparse_attn(fake, fake, fake, lsa.BF16, 1, 4, 100, 8, 1, 64, fake, fake, 8,
                                   0.125, fake, None, None)
     assert rc == 4
+
+
+def test_host_entry_and_wait_hook_argument_checks():
+    P = lsa.IndexParams(4, 256, 8, 3)
+    need = lsa._lib.lsa_index_bytes(1, 8192, P, lsa.BF16)
+    h = ctypes.c_void_p()
+    assert lsa._lib.lsa_index_init(ctypes.c_void_p(1 << 20), need, 1, 8192, P, lsa.BF16,
+                                   ctypes.byref(h)) == 0
+    fake = ctypes.c_void_p(1 << 22)
+    S = lsa.SelectParams(512, 64, 4)
+    f = lsa._lib.lsa_prefill_chunk_host
+    s1, s2 = ctypes.c_void_p(1 << 10), ctypes.c_void_p(1 << 11)
+    args = [fake] * 10                     # 5 host inputs, 5 device tensors
+    # NULL host input; one stream for both roles; the prefill checks (block-aligned T_old)
+    assert f(h, None, *args[1:], 4096, 4160, 8, 2, 64, S, fake, 1 << 30, fake, fake, s1, s2) == 1
+    assert f(h, *args, 4096, 4160, 8, 2, 64, S, fake, 1 << 30, fake, fake, s1, s1) == 1
+    assert b"copy_stream" in lsa._lib.lsa_last_error()
+    assert f(h, *args, 4000, 4160, 8, 2, 64, S, fake, 1 << 30, fake, fake, s1, s2) != 0
+    # a misaligned device buffer is refused before any copy
+    mis = ctypes.c_void_p((1 << 22) + 8)
+    bad = [fake] * 5 + [mis] + [fake] * 4
+    ws = lsa._lib.lsa_prefill_workspace_bytes(h, 64, 8, 2, 64, S)
+    rc = f(h, *bad, 4096, 4160, 8, 2, 64, S, fake, ws, fake, fake, s1, s2)
+    assert rc != 0
+    lsa._lib.lsa_index_release(h)
+
+
+def test_wait_hook_without_gpu_fails_cleanly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert lsa._lib.lsa_set_wait_limit(0) == 4                           # LSA_ERR_CUDA
