@@ -654,9 +654,15 @@ lsa_status lsa_prefill_chunk_host(lsa_index* idx, const void* h_latent_K, const 
     const int64_t Nq = T_new - T_old, B = v.B;
     const size_t lat_row = (size_t)DL * es, kv_row = (size_t)Hkv * d * es;
     cudaStream_t st = (cudaStream_t)stream, cs = (cudaStream_t)copy_stream;
-    // one pair of events per host thread, reused call after call
-    static thread_local cudaEvent_t ev_in = nullptr, ev_kvq = nullptr;
-    cudaError_t e = cudaSuccess;
+    // one pair of events per host thread and device, reused call after call
+    constexpr int MAX_DEV = 64;
+    static thread_local cudaEvent_t evs[MAX_DEV][2] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "current device");
+    if (dev < 0 || dev >= MAX_DEV) return fail(LSA_ERR_UNSUPPORTED, "device %d", dev);
+    cudaEvent_t& ev_in = evs[dev][0];
+    cudaEvent_t& ev_kvq = evs[dev][1];
     if (!ev_in) e = cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming);
     if (e == cudaSuccess && !ev_kvq) e = cudaEventCreateWithFlags(&ev_kvq, cudaEventDisableTiming);
     if (e != cudaSuccess) return cuda_fail(e, "event create");
