@@ -482,7 +482,12 @@ def run_decode(args, peaks, peak_src, ws=1):
     alg = kv + qo + cent + n_sel * 4
     achieved = alg / (us * 1e-6) / 1e9
     del graph
+    cpu = None
+    if not args.no_cpu_baseline and (not torch.distributed.is_initialized()
+                                     or torch.distributed.get_rank() == 0):
+        cpu = _decode_cpu_baseline(w, inp, t_cap, args.cpu_decode_steps)
     return {"value": round(us, 3), "unit": "µs/step", "higher_is_better": False,
+            "cpu_baseline": cpu,
             "workload": "D-LSA Flat decode: %d sequences x %d-token context, 1 query/sequence/step, "
                         "%d steps in one CUDA graph, replayed %d times" % (w.B, w.T, w.steps, reps),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
@@ -490,6 +495,44 @@ def run_decode(args, peaks, peak_src, ws=1):
                          "peak_source": "%s (copy bandwidth)" % peak_src,
                          "algorithmic_bytes_per_step": alg},
             "gpu_launches_per_step": launches_per_step}
+
+
+def _decode_cpu_baseline(w, inp, t_cap, steps):
+    """The oracle on the decode workload's first `steps` steps for all
+    sequences: per step and sequence, the append of the new key, the selection
+    and the attention (host gathers of the selected K/V rows untimed)."""
+    import oracle
+    orcs, lats = [], []
+    t = time.time()
+    for b in range(w.B):
+        lat = inp["latent_K"][b, :w.T + steps].float().cpu().numpy()
+        o = oracle.Index(t_cap, w.p, w.G, w.k, w.L, rt_bf16=True)
+        o.extend(lat, 0, w.T)
+        orcs.append(o)
+        lats.append(lat)
+    setup_s = time.time() - t
+    timed = 0.0
+    for s in range(steps):
+        for b in range(w.B):
+            t0 = time.time()
+            orcs[b].append(lats[b], w.T + s + 1)
+            sel, cnt, _, _ = oracle.select(orcs[b], inp["latent_q"][s][b:b + 1].float().cpu().numpy(),
+                                           np.array([w.T + s]), w.R, w.W, w.S)
+            t1 = time.time()
+            uniq, inv = np.unique(np.where(sel >= 0, sel, 0), return_inverse=True)
+            remap = np.where(sel >= 0, inv.reshape(sel.shape), -1).astype(np.int32)
+            ui = torch.from_numpy(uniq).to(inp["K"].device)
+            K = inp["K"][b].index_select(0, ui).float().cpu().numpy()
+            V = inp["V"][b].index_select(0, ui).float().cpu().numpy()
+            q = inp["q"][s][b:b + 1].float().cpu().numpy()
+            t2 = time.time()
+            oracle.attend(q, K, V, remap, cnt, oracle.default_scale(w.d))
+            timed += (t1 - t0) + (time.time() - t2)
+    return {"value": round(1e6 * timed / steps, 1), "unit": "µs/step",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "the first %d of the %d decode steps, all %d sequences (append, selection, "
+                      "attention); per-sequence prefix indices built untimed in %.1f s"
+                      % (steps, w.steps, w.B, setup_s)}
 
 
 # ---------------------------------------------------------------- reference --
@@ -533,7 +576,8 @@ def main():
     ap.add_argument("--T", type=int, default=None, help="override the context length")
     ap.add_argument("--nq", type=int, default=None, help="override the chunk query count")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--cpu-queries", type=int, default=128)
+    ap.add_argument("--cpu-queries", type=int, default=256)
+    ap.add_argument("--cpu-decode-steps", type=int, default=4)
     ap.add_argument("--ref-queries", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")

@@ -200,13 +200,17 @@ lsa_status lsa_select(const lsa_index* idx, const void* latent_Q, const int32_t*
  * allocator): no workspace argument and no allocation.  The pages describe no
  * such call; it exists for those callers.  Its scratch is one built-in 8 MiB
  * device array that every GPU loading the library keeps until the process
- * exits; a request needing more (lsa_select_workspace_bytes(idx, Nq) >
- * 8 MiB, roughly Nq * 272 B + 148 * buckets * 8 B) returns
- * LSA_ERR_WORKSPACE and launches nothing.  The first call on each device
- * looks up the array's device address (cudaGetSymbolAddress); make that first
- * call before any stream capture.  All calls share the array: calls that
- * overlap on the GPU (other streams, other threads) race and must be
- * serialised by the caller.  Results are identical to lsa_select's. */
+ * exits.  A call is refused (LSA_ERR_WORKSPACE, nothing launched) exactly
+ * when lsa_select_workspace_bytes(idx, Nq) exceeds 8 MiB; that size counts
+ * every query row of every sequence (B * Nq rows) and grows with the number
+ * of buckets per sequence, so ask lsa_select_workspace_bytes rather than
+ * estimate it.  The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress) and keeps it for the process; make that
+ * first call before any stream capture, and do not call this entry again on
+ * a device after cudaDeviceReset (the kept address would be stale).  All
+ * calls share the array: calls that overlap on the GPU (other streams, other
+ * threads) race and must be serialised by the caller.  Results are identical
+ * to lsa_select's. */
 lsa_status lsa_select_noalloc(const lsa_index* idx, const void* latent_Q,
                               const int32_t* positions, int64_t Nq, lsa_select_params sp,
                               int32_t* indices, int32_t* counts, int s_max, void* stream);
@@ -312,13 +316,18 @@ lsa_status lsa_prefill_chunk_host(lsa_index* idx, const void* h_latent_K, const 
                                   void* O, void* h_O, void* stream, void* copy_stream);
 
 /* Test hook (this library's own; not part of the method): the number of
- * polls each bounded wait of the tensor-core centroid scorer (bf16 selection
- * with Nq >= 128) makes before it gives up.  A wait that gives up records
- * LSA_ERR_TIMEOUT for lsa_index_check, and the kernel still leaves cleanly
- * (its copies and MMAs in flight are waited for with the default limit), so
- * the context stays usable.  polls < 0 restores the default (about 4
- * million); 0 makes every such wait give up at once.  Synchronous; applies to
- * later launches on the current device. */
+ * polls each bounded wait makes before it gives up, in every kernel that waits
+ * on a copy or on another warp: the tensor-core centroid scorer (bf16
+ * selection with Nq >= 128), the tensor-core attention tiles of bf16 prefill
+ * chunks, and the per-query bf16 attention kernel (decode steps, prefill rows
+ * attended key by key, lsa_sparse_attn).  A wait that gives up records
+ * LSA_ERR_TIMEOUT in the index status word for lsa_index_check (lsa_sparse_attn
+ * has no index and no status word), and the kernel still leaves cleanly: its
+ * copies and MMAs in flight are waited for with the default limit, so the
+ * context stays usable; the outputs of such a launch are undefined.  polls < 0
+ * restores the defaults (about 4 million polls for the tensor-core kernels, 16
+ * million for the per-query kernel); 0 makes every such wait give up at once.
+ * Synchronous; applies to later launches on the current device. */
 lsa_status lsa_set_wait_limit(int64_t polls);
 
 /* Workspace bytes for lsa_decode_step (depends on the device's SM count). */

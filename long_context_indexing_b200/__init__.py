@@ -321,7 +321,8 @@ def lsa_prefill_chunk(index, latent_K, latent_Q, Q, K, V, T_old, T_new, budget, 
 
 def set_wait_limit(polls):
     """Test hook (C: lsa_set_wait_limit): polls each bounded wait of the
-    tensor-core scorer makes before it gives up; polls < 0 restores the default."""
+    library's kernels (tensor-core scorer, attention tiles, per-query
+    attention) makes before it gives up; polls < 0 restores the defaults."""
     _check(_lib.lsa_set_wait_limit(int(polls)))
 
 

@@ -26,6 +26,11 @@ namespace lsa {
 
 constexpr uint32_t WAIT_LIMIT = 1u << 24;
 
+// Polls each bounded wait of the bf16 attention kernel makes before it gives
+// up.  A test hook (lsa_set_wait_limit) lowers it to make the waits run out;
+// the drain of copies in flight on the way out always allows WAIT_LIMIT.
+__device__ uint32_t g_attn_wait = WAIT_LIMIT;
+
 __device__ __forceinline__ int32_t checked_index(int32_t t, int64_t T_cap, uint32_t* status)
 {
     if (t < 0 || t >= T_cap) {
@@ -237,6 +242,8 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
     }
     __syncthreads();
 
+    const uint32_t wl = g_attn_wait;
+    int issued = 0;                      // stages the producer warp has issued
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float oacc[KSTEPS][4];
 #pragma unroll
@@ -250,10 +257,13 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
         for (int j = 0; j < n_st; ++j) {
             const int s = j % STAGES;
             const uint32_t ph = (uint32_t)((j / STAGES) & 1);
-            if (*abort_flag) break;
-            if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1u, WAIT_LIMIT)) {
-                *abort_flag = 1;
-                if (status) dev_error(status, DEV_TIMEOUT, (uint32_t)row);
+            // the warp agrees on every decision, so it never diverges here
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ph ^ 1u, wl))) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    if (status) dev_error(status, DEV_TIMEOUT, (uint32_t)row);
+                }
                 break;
             }
             if (lane == 0) ptx::mbar_arrive_expect_tx(&full[s], 2u * C::KT * C::RB);
@@ -269,6 +279,7 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
                 else
                     ptx::bulk_g2s(kt + C::TILE + r * C::PITCH, V + off, C::RB, &full[s]);
             }
+            issued = j + 1;
         }
     } else {
         // ---------------- consumers ----------------
@@ -291,10 +302,12 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
         for (int j = 0; j < n_st; ++j) {
             const int s = j % STAGES;
             const uint32_t ph = (uint32_t)((j / STAGES) & 1);
-            if (*abort_flag) break;
-            if (!ptx::mbar_wait_bounded(&full[s], ph, WAIT_LIMIT)) {
-                *abort_flag = 1;
-                if (status) dev_error(status, DEV_TIMEOUT, (uint32_t)row);
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&full[s], ph, wl))) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    if (status) dev_error(status, DEV_TIMEOUT, (uint32_t)row);
+                }
                 break;
             }
             const unsigned char* kt = smem + s * C::STAGE + sub * 16 * C::PITCH + hoff;
@@ -362,10 +375,11 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
             l1 += __shfl_xor_sync(0xffffffffu, l1, o);
         }
     }
-    // Copies of an aborted stage may still be in flight: give them a bounded
-    // chance to land before the ring is reused for the merge.
+    // Copies of an aborted stage may still be in flight: the latest issue of
+    // every ring slot gets a bounded chance to land before the ring is reused
+    // for the merge (slots never issued are not waited for).
     if (*abort_flag && warp == CONS_WARPS)
-        for (int j = 0; j < n_st && j < STAGES; ++j)
+        for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
             ptx::mbar_wait_bounded(&full[j % STAGES], (uint32_t)((j / STAGES) & 1), WAIT_LIMIT);
     __syncthreads();
 
@@ -719,6 +733,12 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, lsa_dtype d
 {
     return launch_attn_status(Q, K, V, dt, B, Nq, T_cap, Hq, Hkv, d, indices, counts, s_max, scale,
                               O, lse, nullptr, st);
+}
+
+cudaError_t set_attn_wait_polls(int64_t polls)
+{
+    const uint32_t v = (polls < 0 || polls > (int64_t)WAIT_LIMIT) ? WAIT_LIMIT : (uint32_t)polls;
+    return cudaMemcpyToSymbol(g_attn_wait, &v, sizeof(v));
 }
 
 }  // namespace lsa

@@ -62,6 +62,12 @@ constexpr int TB_KPW = 64 / TB_NL;                // keys of a stage per loader 
 constexpr int TB_THREADS = 32 * (11 + TB_NL);     // 15 warps with four loaders
 constexpr uint32_t TB_WAIT = 1u << 22;
 
+// Polls each bounded wait of the tile kernel's roles makes before it gives up
+// (and, times 8, the MMA issuer's polls without progress).  A test hook
+// (lsa_set_wait_limit) lowers it to make the waits run out; the drain of the
+// MMAs in flight on the way out always allows TB_WAIT.
+__device__ uint32_t g_tb_wait = TB_WAIT;
+
 #ifndef LSA_TB_QB
 #define LSA_TB_QB 2          // Q buffers (2: the next tile's Q loads during this tile)
 #endif
@@ -291,6 +297,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     __syncthreads();
     tb_fence_after();
     const uint32_t tmem = tmem_slot;
+    const uint32_t wl = g_tb_wait;
 
     // Bounded waits.  wait1: one thread.  waitw: every lane of a warp polls
     // (each gets the barrier's acquire) and the warp agrees on the outcome,
@@ -301,12 +308,12 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     };
     auto wait1 = [&](uint64_t* bar, uint32_t parity, uint32_t where) -> bool {
         if (abort_flag) return false;
-        if (ptx::mbar_wait_bounded(bar, parity, TB_WAIT)) return true;
+        if (ptx::mbar_wait_bounded(bar, parity, wl)) return true;
         fail(where);
         return false;
     };
     auto waitw = [&](uint64_t* bar, uint32_t parity, uint32_t where) -> bool {
-        bool ok = !abort_flag && ptx::mbar_wait_bounded(bar, parity, TB_WAIT);
+        bool ok = !abort_flag && ptx::mbar_wait_bounded(bar, parity, wl);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok && lane == 0) fail(where);
         return ok;
@@ -584,7 +591,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 if (s_done && gP == gs) break;      // every item's P V is out
                 if (progress) {
                     idle = 0;
-                } else if (++idle > (TB_WAIT << 3)) {   // nothing moved for a long time
+                } else if (++idle > (wl << 3)) {   // nothing moved for a long time
                     fail(260u);
                     break;
                 }
@@ -772,6 +779,12 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem)
                      : "memory");
     }
+}
+
+cudaError_t set_tile_wait_polls(int64_t polls)
+{
+    const uint32_t v = (polls < 0 || polls > (int64_t)TB_WAIT) ? TB_WAIT : (uint32_t)polls;
+    return cudaMemcpyToSymbol(g_tb_wait, &v, sizeof(v));
 }
 
 bool bucket_attn_tc_supported(int Hq, int Hkv, int d, int G)

@@ -707,6 +707,8 @@ lsa_status lsa_prefill_chunk_host(lsa_index* idx, const void* h_latent_K, const 
 lsa_status lsa_set_wait_limit(int64_t polls)
 {
     cudaError_t e = set_score_wait_polls(polls);
+    if (e == cudaSuccess) e = set_tile_wait_polls(polls);
+    if (e == cudaSuccess) e = set_attn_wait_polls(polls);
     if (e != cudaSuccess) return cuda_fail(e, "wait limit");
     return LSA_OK;
 }

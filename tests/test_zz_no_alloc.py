@@ -58,3 +58,38 @@ def test_noalloc_select_refuses_requests_beyond_its_array():
     assert e.value.code == 3 and "built-in array" in str(e.value)
     torch.cuda.synchronize()
     assert int(out_c.min()) == 5 and int(out_c.max()) == 5   # nothing was launched
+
+
+def test_noalloc_select_at_its_size_limit_with_two_sequences():
+    # Two sequences on the tensor-core path (bf16, Nq >= 128): the largest
+    # query count whose scratch fits the 8 MiB array gives lsa_select's
+    # selections; one query more is refused before any launch.
+    w, idx, lq, pos = _case("bf16", 4096, seed=23)
+    limit = 8 << 20
+    need = lambda n: int(lsa._lib.lsa_select_workspace_bytes(idx.handle, n))
+    lo, hi = 128, w.nq
+    assert need(lo) <= limit < need(hi)
+    while hi - lo > 1:                       # need(lo) <= limit < need(hi)
+        mid = (lo + hi) // 2
+        if need(mid) <= limit:
+            lo = mid
+        else:
+            hi = mid
+    n_fit = lo
+    lq_fit, pos_fit = lq[:, :n_fit].contiguous(), pos[:, :n_fit].contiguous()
+    ref_i, ref_c = lsa.lsa_select(idx, lq_fit, pos_fit, w.R, w.W, w.S)
+    out_i = torch.full_like(ref_i, 0x7f7f7f7f)
+    out_c = torch.full_like(ref_c, -7)
+    lsa.lsa_select_noalloc(idx, lq_fit, pos_fit, w.R, w.W, w.S, out_i, out_c)
+    torch.cuda.synchronize()
+    assert torch.equal(out_c, ref_c) and torch.equal(out_i, ref_i)
+    n_over = n_fit + 1
+    big_i = torch.full((w.B, n_over, w.s_max), 5, dtype=torch.int32, device="cuda")
+    big_c = torch.full((w.B, n_over), 5, dtype=torch.int32, device="cuda")
+    with pytest.raises(lsa.LsaError) as e:
+        lsa.lsa_select_noalloc(idx, lq[:, :n_over].contiguous(), pos[:, :n_over].contiguous(),
+                               w.R, w.W, w.S, big_i, big_c)
+    assert e.value.code == 3
+    torch.cuda.synchronize()
+    assert int(big_c.min()) == 5 and int(big_c.max()) == 5
+    assert idx.check() >= 0
