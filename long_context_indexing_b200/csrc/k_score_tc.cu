@@ -1,5 +1,5 @@
-// k_score_tc.cu -- tensor-core candidate nomination for bf16 indices
-// (tcgen05 MMA, TMEM accumulators, TMA tile loads; sm_100a).
+// k_score_tc.cu -- tensor-core candidate lists for bf16 indices (tcgen05 MMA,
+// TMEM accumulators, TMA tile loads; sm_100a).
 //
 // Method: "Latent Sparse Attention: un indice gerarchico per contesti
 // lunghi", paragraph on retrieval: each query is compared with the centroids
@@ -7,21 +7,39 @@
 // path: scores S = Q C^T with Q [queries][64] and C [buckets][64], both bf16,
 // accumulated in fp32.
 //
-// These approximate scores are written as fp16 to a [queries][buckets] matrix
-// in the selection workspace; select_fill_kernel (k_select.cu) nominates each
-// query's candidates from its row and then ranks them with exact binary64
-// scores.  At 10M context the matrix is 32768 x 40960 fp16 (2.7 GB), written
-// once and read once.
+// No score matrix is written.  A work item is (sequence, 128-query tile,
+// split), where a split is a contiguous range of centroid tiles; every item
+// computes its scores twice on the tensor cores:
+//   sweep 1  the epilogue keeps, per query row, the maximum of every group of
+//            gw consecutive eligible scores (rounded down to fp16) and then
+//            picks theta, the m-th largest group maximum: at least m scores of
+//            the split are >= theta (each of the m groups holds one);
+//   sweep 2  every eligible score >= theta is appended to the row's list for
+//            the split (bucket id), up to the list's capacity.
+// Every bucket of the split left out of the list scored below theta, or was
+// an appended score that found the list full (the largest of those is kept),
+// so tau = max(theta, largest lost score) bounds the approximate score of
+// every bucket of the split that is not in the list.  A row whose split holds
+// no more eligible buckets than the list capacity lists them all (theta =
+// -inf: the list is complete).  select_fill_kernel (k_select.cu) merges a
+// row's lists, ranks the candidates with exact binary64 scores and proves the
+// exact ranking against the largest tau, or sends the row to the exact
+// fallback.
 //
-// CTA = 128 queries of one sequence (one TMEM lane each), 6 warps:
-//   warp 0     TMA producer: the query tile once, then TC_N-centroid tiles into
-//              a TC_STAGES-deep shared-memory ring (128-byte swizzle);
-//   warp 1     owns 2 x TC_N TMEM columns (two fp32 accumulators) and
-//              issues tcgen05.mma (M=128, N=TC_N, K=16, four per tile);
-//   warps 2-5  epilogue: tcgen05.ld 32 columns at a time, fp32 -> fp16, and
-//              64-byte row segments straight to the score matrix.
-// Every mbarrier wait is bounded; on a timeout the CTA records DEV_TIMEOUT in
-// the index status word, stops waiting, and still frees its TMEM.
+// Persistent CTAs (one per SM) take the items in a fixed round-robin order.
+// CTA = 10 warps:
+//   warp 0     TMA producer: each item's query tile (two buffers), then its
+//              centroid tiles, twice, into a TC_STAGES-deep ring (128-byte
+//              swizzle);
+//   warp 1     owns 2 x TC_N TMEM columns (two fp32 accumulators) and issues
+//              tcgen05.mma (M = 128, N = TC_N, K = 16, four per tile);
+//   warps 2-9  epilogue: thread = (query row, half of every tile's columns);
+//              tcgen05.ld 32 columns at a time.
+// Every mbarrier wait is bounded; after a timeout the CTA records DEV_TIMEOUT
+// in the index status word, the producer and the MMA thread stop, the
+// epilogue runs through its remaining items without waiting (so its named
+// barriers stay matched), copies and MMAs in flight are waited for, and TMEM
+// is freed.
 #include <cuda.h>
 
 #include <cuda_fp16.h>
@@ -34,14 +52,13 @@
 namespace lsa {
 
 constexpr int TC_M = 128;
-#ifndef LSA_TC_N
-#define LSA_TC_N 256         // centroids per tile (128 gives two CTAs per SM; measured slower)
-#endif
-constexpr int TC_N = LSA_TC_N;
+constexpr int TC_N = 256;                                 // centroids per tile
 constexpr int TC_TMEM_COLS = 2 * TC_N;                    // two fp32 accumulators
-constexpr int TC_MIN_BLOCKS = (TC_N <= 128) ? 2 : 1;
 constexpr int TC_STAGES = 4;
-constexpr int TC_THREADS = 192;
+constexpr int TC_EPI_WARPS = 8;
+constexpr int TC_EPI_THREADS = 32 * TC_EPI_WARPS;
+constexpr int TC_THREADS = 64 + TC_EPI_THREADS;           // producer, MMA, epilogue
+constexpr int TC_NG = 64;                                 // group maxima per row and split
 constexpr uint32_t TC_WAIT = 1u << 22;
 
 // Polls each bounded wait of the scorer's roles makes before it gives up.  A
@@ -49,14 +66,17 @@ constexpr uint32_t TC_WAIT = 1u << 22;
 // drains on the way out always allow TC_WAIT.
 __device__ uint32_t g_tc_wait = TC_WAIT;
 
-constexpr int TC_Q_BYTES = TC_M * DL * 2;                 // 16 KB
-constexpr int TC_C_BYTES = TC_N * DL * 2;                 // 32 KB per stage at N = 256
-constexpr int TC_OFF_C = TC_Q_BYTES;
-constexpr int TC_OFF_BAR = TC_OFF_C + TC_STAGES * TC_C_BYTES;
-constexpr int TC_NBAR = 1 + 2 * TC_STAGES + 4 + 1;
+constexpr int TC_Q_BYTES = TC_M * DL * 2;                 // 16 KB per query buffer
+constexpr int TC_C_BYTES = TC_N * DL * 2;                 // 32 KB per ring stage
+constexpr int TC_OFF_C = 2 * TC_Q_BYTES;
+constexpr int TC_OFF_G = TC_OFF_C + TC_STAGES * TC_C_BYTES;
+constexpr int TC_G_BYTES = TC_M * TC_NG * 4;              // group maxima; sweep-2 staging
+static_assert(TC_G_BYTES == TC_EPI_THREADS * 32 * 4, "staging area = group-maximum area");
+constexpr int TC_OFF_BAR = TC_OFF_G + TC_G_BYTES;
+constexpr int TC_NBAR = 2 + 2 + 2 * TC_STAGES + 2 + 2 + 1;
 constexpr int TC_OFF_MISC = TC_OFF_BAR + TC_NBAR * 8;
-constexpr int TC_SMEM = TC_OFF_MISC + 64 + 1024;          // + alignment slack
-
+constexpr int TC_MISC_BYTES = TC_M * 4 + TC_EPI_THREADS * 4 + 64;
+constexpr int TC_SMEM = TC_OFF_MISC + TC_MISC_BYTES + 1024;   // + alignment slack
 
 // ---- tcgen05 / TMA wrappers -------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
@@ -122,6 +142,25 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v)
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+// Named barrier of the epilogue warps only.
+__device__ __forceinline__ void epi_sync()
+{
+    asm volatile("bar.sync 1, %0;" ::"n"(TC_EPI_THREADS) : "memory");
+}
+
+// Ordered 16-bit key of an fp16 value (larger value, larger key; never 0).
+__device__ __forceinline__ uint32_t tc_half_key(__half h)
+{
+    const uint32_t u = __half_as_ushort(h);
+    return (u & 0x8000u) ? (~u & 0xFFFFu) : (u | 0x8000u);
+}
+
+__device__ __forceinline__ float tc_key_value(uint32_t k)
+{
+    const uint16_t u = (k & 0x8000u) ? (uint16_t)(k & 0x7FFFu) : (uint16_t)(~k & 0xFFFFu);
+    return __half2float(__ushort_as_half(u));
+}
+
 __device__ __forceinline__ int64_t tc_eligible(const IndexView& ix, int64_t n_blk, int64_t pos,
                                                int W)
 {
@@ -133,177 +172,370 @@ __device__ __forceinline__ int64_t tc_eligible(const IndexView& ix, int64_t n_bl
     return nb * ix.k;
 }
 
-__global__ void __launch_bounds__(TC_THREADS, TC_MIN_BLOCKS) score_topk_tc_kernel(
+// Geometry of one work item, computed identically by every role.
+struct TcItem {
+    int64_t b, q0;      // sequence, first query of the tile
+    int s;              // split
+    int t0, t1;         // centroid tiles [t0, t1) of this item (t1 <= t0: nothing eligible)
+};
+
+// Every lane of the calling warp takes part (warp-collective).
+__device__ __forceinline__ TcItem tc_item(int64_t it, const IndexView& ix, int64_t n_blk,
+                                          const PosSrc& pos, int64_t Nq, int W, const TcSplit& sp)
+{
+    TcItem r;
+    r.s = (int)(it % sp.n_split);
+    const int64_t qt = it / sp.n_split;
+    r.b = qt / sp.n_qt;
+    r.q0 = (qt % sp.n_qt) * TC_M;
+    const int lane = threadIdx.x & 31;
+    unsigned nb = 0;
+#pragma unroll
+    for (int u = 0; u < TC_M / 32; ++u) {
+        const int64_t q = r.q0 + lane + 32 * u;
+        if (q < Nq) {
+            const int64_t e = tc_eligible(ix, n_blk, pos.at(r.b, Nq, q), W);
+            if ((unsigned)e > nb) nb = (unsigned)e;
+        }
+    }
+    nb = __reduce_max_sync(0xffffffffu, nb);
+    const int n_ct = (int)((nb + TC_N - 1) / TC_N);
+    r.t0 = r.s * sp.tps;
+    r.t1 = min(r.t0 + sp.tps, n_ct);
+    return r;
+}
+
+__global__ void __launch_bounds__(TC_THREADS, 1) score_lists_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC, IndexView ix,
-    int64_t n_blk, PosSrc pos, int64_t Nq, int W, SelectWs ws)
+    int64_t n_blk, PosSrc pos, int64_t Nq, int W, SelectWs ws, TcSplit sp)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem =
         (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);  // 1 KB aligned
-    unsigned char* q_s = smem;
-    unsigned char* c_s = smem + TC_OFF_C;
+    unsigned char* q_s = smem;                        // [2][TC_Q_BYTES]
+    unsigned char* c_s = smem + TC_OFF_C;             // [TC_STAGES][TC_C_BYTES]
+    uint32_t* gm = reinterpret_cast<uint32_t*>(smem + TC_OFF_G);   // [TC_M][TC_NG] two halves
+    float* stage = reinterpret_cast<float*>(smem + TC_OFF_G);      // [TC_EPI_THREADS][32]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TC_OFF_BAR);
-    uint64_t* q_full = bars;
-    uint64_t* full = bars + 1;
-    uint64_t* empty = full + TC_STAGES;
-    uint64_t* acc_full = empty + TC_STAGES;
-    uint64_t* acc_empty = acc_full + 2;
-    uint64_t* fin = acc_empty + 2;        // the MMA thread's last MMAs are done
-    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + TC_OFF_MISC);
+    uint64_t* q_full = bars;                  // [2]
+    uint64_t* q_empty = bars + 2;             // [2]
+    uint64_t* full = bars + 4;                // [TC_STAGES]
+    uint64_t* empty = full + TC_STAGES;       // [TC_STAGES]
+    uint64_t* acc_full = empty + TC_STAGES;   // [2]
+    uint64_t* acc_empty = acc_full + 2;       // [2]
+    uint64_t* fin = acc_empty + 2;            // the MMA thread's last MMAs are done
+    int* rcnt = reinterpret_cast<int*>(smem + TC_OFF_MISC);                 // [TC_M]
+    float* lostv = reinterpret_cast<float*>(smem + TC_OFF_MISC + TC_M * 4); // [TC_EPI_THREADS]
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + TC_OFF_MISC + TC_M * 4 + TC_EPI_THREADS * 4);
     volatile uint32_t* tmem_slot = misc;        // [0]
     volatile uint32_t* abort_flag = misc + 1;   // [1]
-    uint32_t* nb_max = misc + 2;                // [2]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t b = blockIdx.y;
-    const int64_t q0 = (int64_t)blockIdx.x * TC_M;
-    if (blockIdx.x == 0 && b == 0 && threadIdx.x == 0) *ws.fb_count = 0;
-    {
-        const int64_t cta = b * gridDim.x + blockIdx.x;
-        for (int64_t x = cta * blockDim.x + threadIdx.x; x < ws.plan.n_zero;
-             x += (int64_t)gridDim.x * gridDim.y * blockDim.x)
-            ws.plan.zero[x] = 0;
-    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) *ws.fb_count = 0;
+    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < ws.plan.n_zero;
+         x += (int64_t)gridDim.x * blockDim.x)
+        ws.plan.zero[x] = 0;
 
     if (threadIdx.x == 0) {
-        ptx::mbar_init(q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&q_full[i], 1);
+            ptx::mbar_init(&q_empty[i], 1);
+            ptx::mbar_init(&acc_full[i], 1);
+            ptx::mbar_init(&acc_empty[i], TC_EPI_WARPS);
+        }
         for (int s = 0; s < TC_STAGES; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
-            ptx::mbar_init(&acc_full[a], 1);
-            ptx::mbar_init(&acc_empty[a], 4);
-        }
         ptx::mbar_init(fin, 1);
         *abort_flag = 0;
-        *nb_max = 0;
         ptx::fence_mbar_init();
     }
+    if (threadIdx.x < TC_M) rcnt[threadIdx.x] = 0;
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          ptx::smem_addr((const void*)tmem_slot)), "n"(TC_TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // per-row eligibility (epilogue threads own rows)
-    int64_t nb_row = 0;
-    int r = 0;
-    bool row_valid = false;
-    if (warp >= 2) {
-        r = 32 * (warp & 3) + lane;
-        row_valid = (q0 + r) < Nq;
-        if (row_valid) nb_row = tc_eligible(ix, n_blk, pos.at(b, Nq, q0 + r), W);
-    }
-    __syncthreads();
-    if (warp >= 2) atomicMax(nb_max, (uint32_t)nb_row);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_tiles = (int)((*nb_max + TC_N - 1) / TC_N);
     const uint32_t wl = g_tc_wait;
 
-    if (warp == 0 && lane == 0 && n_tiles > 0) {
-        // ---------------- TMA producer ----------------
-        ptx::mbar_arrive_expect_tx(q_full, TC_Q_BYTES);
-        tma_load_2d(q_s, &tmQ, 0, (int)(b * Nq + q0), q_full);
-        int issued = 0;
-        for (int t = 0; t < n_tiles; ++t) {
-            const int s = t % TC_STAGES;
-            const uint32_t ph = (uint32_t)((t / TC_STAGES) & 1);
-            if (*abort_flag) break;
-            if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1u, wl)) {
-                *abort_flag = 1;
-                dev_error(ix.status, DEV_TIMEOUT, 1000u + (uint32_t)t);
-                break;
-            }
-            ptx::mbar_arrive_expect_tx(&full[s], TC_C_BYTES);
-            tma_load_2d(c_s + s * TC_C_BYTES, &tmC, 0, (int)(b * ix.NBK + (int64_t)t * TC_N),
-                        &full[s]);
-            issued = t + 1;
-        }
-        if (*abort_flag) {
-            // no copy may still be writing shared memory when the CTA exits:
-            // the latest load of every stage (and the query tile) has landed,
-            // or a bounded wait gives up on it
-            ptx::mbar_wait_bounded(q_full, 0, TC_WAIT);
-            for (int t = (issued > TC_STAGES ? issued - TC_STAGES : 0); t < issued; ++t)
-                ptx::mbar_wait_bounded(&full[t % TC_STAGES], (uint32_t)((t / TC_STAGES) & 1),
-                                       TC_WAIT);
-        }
-    } else if (warp == 1 && lane == 0 && n_tiles > 0) {
-        // ---------------- MMA issuer ----------------
-        bool ok = ptx::mbar_wait_bounded(q_full, 0, wl);
-        if (!ok) {
+    // warp-uniform bounded wait: every lane polls, the warp agrees
+    auto waitw = [&](uint64_t* bar, uint32_t parity, uint32_t where) -> bool {
+        bool ok = (*abort_flag == 0) && ptx::mbar_wait_bounded(bar, parity, wl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok && lane == 0 && *abort_flag == 0) {
             *abort_flag = 1;
-            dev_error(ix.status, DEV_TIMEOUT, 2000u);
+            dev_error(ix.status, DEV_TIMEOUT, where);
         }
-        const uint64_t adesc = sw128_desc(q_s);
-        for (int t = 0; ok && t < n_tiles; ++t) {
-            const int s = t % TC_STAGES;
-            const uint32_t ph = (uint32_t)((t / TC_STAGES) & 1);
-            const int buf = t & 1;
-            const uint32_t aph = (uint32_t)((t >> 1) & 1);
-            if (*abort_flag) break;
-            if (!ptx::mbar_wait_bounded(&full[s], ph, wl) ||
-                !ptx::mbar_wait_bounded(&acc_empty[buf], aph ^ 1u, wl)) {
-                *abort_flag = 1;
-                dev_error(ix.status, DEV_TIMEOUT, 3000u + (uint32_t)t);
-                break;
+        return ok;
+    };
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        int64_t gt = 0, qi = 0;
+        bool stop = false;
+        for (int64_t it = blockIdx.x; it < sp.n_items && !stop; it += gridDim.x) {
+            const TcItem I = tc_item(it, ix, n_blk, pos, Nq, W, sp);
+            if (I.t1 <= I.t0) continue;
+            const int qb = (int)(qi & 1);
+            if (!waitw(&q_empty[qb], (uint32_t)(((qi >> 1) & 1) ^ 1), 1000u)) break;
+            if (lane == 0) {
+                ptx::mbar_arrive_expect_tx(&q_full[qb], TC_Q_BYTES);
+                tma_load_2d(q_s + qb * TC_Q_BYTES, &tmQ, 0, (int)(I.b * Nq + I.q0), &q_full[qb]);
             }
-            tc_fence_after();
-            const uint64_t bdesc = sw128_desc(c_s + s * TC_C_BYTES);
-            const uint32_t d = tmem + (uint32_t)(buf * TC_N);
+            ++qi;
+            for (int sw = 0; sw < 2 && !stop; ++sw)
+                for (int t = I.t0; t < I.t1; ++t, ++gt) {
+                    const int s = (int)(gt % TC_STAGES);
+                    if (!waitw(&empty[s], (uint32_t)(((gt / TC_STAGES) & 1) ^ 1), 1100u)) {
+                        stop = true;
+                        break;
+                    }
+                    if (lane == 0) {
+                        ptx::mbar_arrive_expect_tx(&full[s], TC_C_BYTES);
+                        tma_load_2d(c_s + s * TC_C_BYTES, &tmC, 0,
+                                    (int)(I.b * ix.NBK + (int64_t)t * TC_N), &full[s]);
+                    }
+                }
+        }
+        if (*abort_flag && lane == 0) {
+            // no copy may still be writing shared memory when the CTA exits:
+            // the latest load of every stage and query buffer has landed, or a
+            // bounded wait gives up on it
+            for (int64_t g = (gt > TC_STAGES ? gt - TC_STAGES : 0); g < gt; ++g)
+                ptx::mbar_wait_bounded(&full[g % TC_STAGES], (uint32_t)((g / TC_STAGES) & 1),
+                                       TC_WAIT);
+            for (int64_t q = (qi > 2 ? qi - 2 : 0); q < qi; ++q)
+                ptx::mbar_wait_bounded(&q_full[q & 1], (uint32_t)((q >> 1) & 1), TC_WAIT);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        int64_t gt = 0, qi = 0;
+        bool stop = false;
+        for (int64_t it = blockIdx.x; it < sp.n_items && !stop; it += gridDim.x) {
+            const TcItem I = tc_item(it, ix, n_blk, pos, Nq, W, sp);
+            if (I.t1 <= I.t0) continue;
+            const int qb = (int)(qi & 1);
+            if (!waitw(&q_full[qb], (uint32_t)((qi >> 1) & 1), 2000u)) break;
+            const uint64_t adesc = sw128_desc(q_s + qb * TC_Q_BYTES);
+            ++qi;
+            for (int sw = 0; sw < 2 && !stop; ++sw)
+                for (int t = I.t0; t < I.t1; ++t, ++gt) {
+                    const int s = (int)(gt % TC_STAGES);
+                    const int buf = (int)(gt & 1);
+                    if (!waitw(&full[s], (uint32_t)((gt / TC_STAGES) & 1), 2100u) ||
+                        !waitw(&acc_empty[buf], (uint32_t)(((gt >> 1) & 1) ^ 1), 2200u)) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint64_t bdesc = sw128_desc(c_s + s * TC_C_BYTES);
+                        const uint32_t d = tmem + (uint32_t)(buf * TC_N);
 #pragma unroll
-            for (int kk = 0; kk < DL / 16; ++kk)
-                mma_bf16(d, adesc + 2ull * kk, bdesc + 2ull * kk, kk > 0 ? 1u : 0u);
-            mma_commit(&empty[s]);
-            mma_commit(&acc_full[buf]);
+                        for (int kk = 0; kk < DL / 16; ++kk)
+                            mma_bf16(d, adesc + 2ull * kk, bdesc + 2ull * kk, kk > 0 ? 1u : 0u);
+                        mma_commit(&empty[s]);
+                        mma_commit(&acc_full[buf]);
+                    }
+                    __syncwarp();
+                }
+            if (!stop && lane == 0) mma_commit(&q_empty[qb]);
+            __syncwarp();
         }
         // nothing of this CTA may still run on the tensor cores when TMEM is freed
-        mma_commit(fin);
-        ptx::mbar_wait_bounded(fin, 0, TC_WAIT);
-    } else if (warp >= 2) {
+        if (lane == 0) {
+            mma_commit(fin);
+            ptx::mbar_wait_bounded(fin, 0, TC_WAIT);
+        }
+        __syncwarp();
+    } else {
         // ---------------- epilogue ----------------
+        const int et = threadIdx.x - 64;                  // 0 .. 255
+        const int h = (warp - 2) >> 2;                    // half of every tile's columns
+        const int r = 32 * (warp & 3) + lane;             // query row = TMEM lane
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-        __half* srow = ws.scores + (b * Nq + q0 + r) * ws.score_ld;
-        __half* crow = ws.cmax + (b * Nq + q0 + r) * (ws.score_ld / 32);
-        for (int t = 0; t < n_tiles; ++t) {
-            const int buf = t & 1;
-            const uint32_t ph = (uint32_t)((t >> 1) & 1);
-            if (*abort_flag) break;
-            if (!ptx::mbar_wait_bounded(&acc_full[buf], ph, wl)) {
-                *abort_flag = 1;
-                dev_error(ix.status, DEV_TIMEOUT, 4000u + (uint32_t)t);
-                break;
+        uint16_t* gm16 = reinterpret_cast<uint16_t*>(gm);
+        float* my_stage = stage + et * 32;
+        int64_t gt = 0;
+        for (int64_t it = blockIdx.x; it < sp.n_items; it += gridDim.x) {
+            const TcItem I = tc_item(it, ix, n_blk, pos, Nq, W, sp);
+            const bool row_valid = I.q0 + r < Nq;
+            const int64_t row = I.b * Nq + I.q0 + r;
+            const int64_t nb_row =
+                row_valid ? tc_eligible(ix, n_blk, pos.at(I.b, Nq, I.q0 + r), W) : 0;
+            const int64_t cs0 = (int64_t)I.s * sp.tps * TC_N;     // first column of the split
+            const int64_t cs1 = cs0 + (int64_t)sp.tps * TC_N;
+            const int64_t n_el = max((int64_t)0, min(nb_row, cs1) - cs0);   // eligible here
+            const int64_t lslot = row * sp.n_split + I.s;
+            if (I.t1 <= I.t0) {
+                if (h == 0 && row_valid) {
+                    ws.lst_n[lslot] = 0;
+                    ws.lst_tau[lslot] = -INFINITY;
+                }
+                continue;
             }
-            tc_fence_after();
-            for (int c = 0; c < TC_N / 32; ++c) {
-                float v[32];
+            const bool take_all = n_el <= ws.lst_cap;
+            const bool go = __all_sync(0xffffffffu, *abort_flag == 0);   // warp-uniform
+            // ---- sweep 1: group maxima (fp16, rounded down) ----
+            for (int g = 0; g < TC_NG; ++g) gm16[(r * TC_NG + g) * 2 + h] = 0;
+            float gacc = -INFINITY;
+            int gcur = -1;
+            auto flush = [&]() {
+                if (gcur >= 0 && gacc > -INFINITY)
+                    gm16[(r * TC_NG + gcur) * 2 + h] = (uint16_t)tc_half_key(__float2half_rd(gacc));
+            };
+            for (int t = I.t0; t < I.t1; ++t, ++gt) {
+                const int buf = (int)(gt & 1);
+                const bool ok = go && waitw(&acc_full[buf], (uint32_t)((gt >> 1) & 1), 4000u);
+                if (ok) {
+                    tc_fence_after();
+                    for (int c = 0; c < 4; ++c) {
+                        float v[32];
+                        __syncwarp();
+                        tmem_ld32(tmem + lane_base + (uint32_t)(buf * TC_N + h * 128 + c * 32), v);
+                        const int64_t g0 = (int64_t)t * TC_N + h * 128 + c * 32;
+                        if (take_all || g0 >= nb_row) continue;
+                        if (g0 + 32 > nb_row) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (g0 + j >= nb_row) v[j] = -INFINITY;
+                        }
+                        // maxima of 1 .. 32 consecutive scores as a tree
+                        float m16[16], m8[8], m4[4], m2[2];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) m16[j] = fmaxf(v[2 * j], v[2 * j + 1]);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) m8[j] = fmaxf(m16[2 * j], m16[2 * j + 1]);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) m4[j] = fmaxf(m8[2 * j], m8[2 * j + 1]);
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) m2[j] = fmaxf(m4[2 * j], m4[2 * j + 1]);
+                        const float m1 = fmaxf(m2[0], m2[1]);
+                        const int rel = (int)(g0 - cs0);
+                        if (sp.gw_log2 >= 5) {
+                            const int grp = rel >> sp.gw_log2;
+                            if (grp != gcur) {
+                                flush();
+                                gcur = grp;
+                                gacc = -INFINITY;
+                            }
+                            gacc = fmaxf(gacc, m1);
+                        } else {
+                            // groups narrower than a load: write each directly
+                            const int gb = rel >> sp.gw_log2;
+                            auto put = [&](int u, float x) {
+                                if (x > -INFINITY)
+                                    gm16[(r * TC_NG + gb + u) * 2 + h] =
+                                        (uint16_t)tc_half_key(__float2half_rd(x));
+                            };
+                            if (sp.gw_log2 == 4) {
+#pragma unroll
+                                for (int u = 0; u < 2; ++u) put(u, m2[u]);
+                            } else if (sp.gw_log2 == 3) {
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) put(u, m4[u]);
+                            } else if (sp.gw_log2 == 2) {
+#pragma unroll
+                                for (int u = 0; u < 8; ++u) put(u, m8[u]);
+                            } else {
+#pragma unroll
+                                for (int u = 0; u < 16; ++u) put(u, m16[u]);
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                }
                 __syncwarp();
-                tmem_ld32(tmem + lane_base + (uint32_t)(buf * TC_N + c * 32), v);
-                const int64_t g0 = (int64_t)t * TC_N + c * 32;
-                if (row_valid && g0 < nb_row) {
-                    uint4 pk[4];
-                    __half2* h = reinterpret_cast<__half2*>(pk);
-                    float mx = -INFINITY;
+                if (ok && lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
+            }
+            flush();
+            epi_sync();
+            // ---- theta: the m-th largest group maximum of the row ----
+            float theta = -INFINITY;
+            if (!take_all) {
+                uint32_t key[TC_NG];
+                int nz = 0;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (g0 + j < nb_row) mx = fmaxf(mx, v[j]);
+                for (int g = 0; g < TC_NG; ++g) {
+                    const uint32_t w = gm[r * TC_NG + g];
+                    key[g] = max(w & 0xFFFFu, w >> 16);
+                    nz += key[g] != 0u;
+                }
+                if (nz >= sp.m) {
+                    uint32_t lo = 1u, hi = 0xFFFFu;       // count(key >= lo) >= m
+                    while (lo < hi) {
+                        const uint32_t mid = (lo + hi + 1u) >> 1;
+                        int cnt = 0;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) h[j] = __floats2half2_rn(v[2 * j], v[2 * j + 1]);
-                    uint4* dst = reinterpret_cast<uint4*>(srow + g0);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) dst[j] = pk[j];
-                    // fp16 rounding is monotone: the rounded maximum is the
-                    // maximum of the rounded scores of the chunk
-                    crow[g0 / 32] = __float2half_rn(mx);
+                        for (int g = 0; g < TC_NG; ++g) cnt += key[g] >= mid;
+                        if (cnt >= sp.m) lo = mid;
+                        else hi = mid - 1u;
+                    }
+                    theta = tc_key_value(lo);
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
+            epi_sync();          // the group maxima become the staging area
+            // ---- sweep 2: append every eligible score >= theta ----
+            float lost = -INFINITY;
+            const bool go2 = __all_sync(0xffffffffu, *abort_flag == 0);
+            for (int t = I.t0; t < I.t1; ++t, ++gt) {
+                const int buf = (int)(gt & 1);
+                const bool ok = go2 && waitw(&acc_full[buf], (uint32_t)((gt >> 1) & 1), 4100u);
+                if (ok) {
+                    tc_fence_after();
+                    for (int c = 0; c < 4; ++c) {
+                        float v[32];
+                        __syncwarp();
+                        tmem_ld32(tmem + lane_base + (uint32_t)(buf * TC_N + h * 128 + c * 32), v);
+                        const int64_t g0 = (int64_t)t * TC_N + h * 128 + c * 32;
+                        uint32_t vm = 0u;
+                        if (g0 + 32 <= nb_row) vm = 0xFFFFFFFFu;
+                        else if (g0 < nb_row) vm = (1u << (uint32_t)(nb_row - g0)) - 1u;
+                        uint32_t msk = 0u;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) msk |= (v[j] >= theta) ? (1u << j) : 0u;
+                        msk &= vm;
+                        if (__any_sync(0xffffffffu, msk != 0u)) {
+                            if (msk) {
+                                float4* st4 = reinterpret_cast<float4*>(my_stage);
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+                                    st4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2],
+                                                         v[4 * j + 3]);
+                            }
+                            while (msk) {
+                                const int j = __ffs(msk) - 1;
+                                msk &= msk - 1u;
+                                const int slot = atomicAdd(&rcnt[r], 1);
+                                if (slot < ws.lst_cap)
+                                    ws.lst_g[lslot * ws.lst_cap + slot] = (int32_t)(g0 + j);
+                                else
+                                    lost = fmaxf(lost, my_stage[j]);
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                }
+                __syncwarp();
+                if (ok && lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
+            }
+            lostv[et] = lost;
+            epi_sync();
+            if (h == 0) {
+                if (row_valid) {
+                    const int n = rcnt[r];
+                    const float l2 = fmaxf(lost, lostv[et + 128]);   // the other half's thread
+                    ws.lst_n[lslot] = min(n, ws.lst_cap);
+                    ws.lst_tau[lslot] = take_all ? l2 : fmaxf(theta, l2);
+                }
+                rcnt[r] = 0;
+            }
         }
     }
     tc_fence_before();
@@ -331,25 +563,54 @@ static bool make_rows64_bf16(CUtensorMap* m, const void* base, uint64_t rows, ui
 
 bool tc_scoring_available() { return true; }
 
+TcSplit tc_split_plan(const IndexView& ix, int64_t Nq)
+{
+    TcSplit sp;
+    sp.n_qt = (Nq + TC_M - 1) / TC_M;
+    const int64_t n_ct = (ix.NBK + TC_N - 1) / TC_N;       // centroid tiles of a sequence
+    const int64_t tiles = ix.B * sp.n_qt;
+    // enough items for the persistent CTAs to end within one item of each other
+    int ns = 1;
+    while (ns < TC_MAX_SPLITS && tiles * ns < 4LL * sm_count() && ns < n_ct) ns *= 2;
+    sp.tps = (int)((n_ct + ns - 1) / ns);
+    sp.n_split = (int)((n_ct + sp.tps - 1) / sp.tps);
+    if (sp.n_split < 1) sp.n_split = 1;
+    sp.n_items = tiles * sp.n_split;
+    // m-th largest of the group maxima: the m groups (of gw scores) hold at
+    // least m candidates; with at least 2m groups per split the list holds
+    // about 1.4 m on scores without structure
+    sp.m = (TC_TARGET + sp.n_split - 1) / sp.n_split;
+    const int64_t split_w = (int64_t)sp.tps * TC_N;
+    int gl = 5;
+    while (gl > 0 && (split_w >> gl) < 2LL * sp.m) --gl;   // at least 2m groups
+    while ((split_w >> gl) > TC_NG) ++gl;                 // at most TC_NG groups
+    sp.gw_log2 = gl;
+    if ((split_w >> gl) < 2LL * sp.m) sp.m = (int)max((int64_t)1, (split_w >> gl) / 2);
+    return sp;
+}
+
 cudaError_t set_score_wait_polls(int64_t polls)
 {
     const uint32_t v = (polls < 0 || polls > (int64_t)TC_WAIT) ? TC_WAIT : (uint32_t)polls;
     return cudaMemcpyToSymbol(g_tc_wait, &v, sizeof(v));
 }
 
-cudaError_t launch_score_topk_tc(const IndexView& ix, int64_t n_blk, const void* latent_Q,
-                                 PosSrc pos, int64_t Nq, int W, const SelectWs& ws,
-                                 cudaStream_t st)
+cudaError_t launch_score_lists_tc(const IndexView& ix, int64_t n_blk, const void* latent_Q,
+                                  PosSrc pos, int64_t Nq, int W, const SelectWs& ws,
+                                  cudaStream_t st)
 {
     if (ix.dtype != LSA_BF16) return cudaErrorInvalidValue;
+    const TcSplit sp = tc_split_plan(ix, Nq);
+    if (ws.n_lst != sp.n_split || ws.lst_cap != TC_LIST_CAP) return cudaErrorInvalidValue;
     CUtensorMap tmQ, tmC;
     if (!make_rows64_bf16(&tmQ, latent_Q, (uint64_t)ix.B * Nq, TC_M) ||
         !make_rows64_bf16(&tmC, ix.cent_rt, (uint64_t)ix.B * ix.NBK, TC_N))
         return cudaErrorInvalidValue;
-    cudaError_t e = ensure_smem_attr((const void*)score_topk_tc_kernel, TC_SMEM);
+    cudaError_t e = ensure_smem_attr((const void*)score_lists_tc_kernel, TC_SMEM);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((Nq + TC_M - 1) / TC_M), (unsigned)ix.B);
-    score_topk_tc_kernel<<<grid, TC_THREADS, TC_SMEM, st>>>(tmQ, tmC, ix, n_blk, pos, Nq, W, ws);
+    const int64_t n_cta = sp.n_items < sm_count() ? sp.n_items : sm_count();
+    score_lists_tc_kernel<<<(unsigned)n_cta, TC_THREADS, TC_SMEM, st>>>(tmQ, tmC, ix, n_blk, pos,
+                                                                        Nq, W, ws, sp);
     note_launch();
     return cudaGetLastError();
 }

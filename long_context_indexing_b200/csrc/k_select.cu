@@ -206,12 +206,12 @@ __device__ void simt_nominate(const IndexView& ix, int64_t n_blk, const float* q
     __shared__ uint32_t sh_prefix, sh_want;
     __shared__ int sh_gt, sh_eq;
     const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
-    int32_t* cand = ws.cand + row * KC;
+    int32_t* cand = ws.lst_g + row * KC;      // one list of KC per row
     if (nb <= KC) {
         for (int x = threadIdx.x; x < KC; x += blockDim.x) cand[x] = (x < nb) ? x : -1;
         if (threadIdx.x == 0) {
-            ws.ncand[row] = (int32_t)nb;
-            ws.tau[row] = -INFINITY;
+            ws.lst_n[row] = (int32_t)nb;
+            ws.lst_tau[row] = -INFINITY;
         }
         return;
     }
@@ -282,8 +282,8 @@ __device__ void simt_nominate(const IndexView& ix, int64_t n_blk, const float* q
         }
     }
     if (threadIdx.x == 0) {
-        ws.ncand[row] = KC;
-        ws.tau[row] = key_to_float(thr);
+        ws.lst_n[row] = KC;
+        ws.lst_tau[row] = key_to_float(thr);
     }
 }
 
@@ -556,195 +556,13 @@ __device__ void cta_emit_tail(int64_t pq, int W, int64_t n_s, int64_t off, int s
     if (threadIdx.x == 0) *count = (int32_t)(off + n_w);
 }
 
-// ---------------------------------------------------------------------------
-// Candidate nomination from a query's fp16 tensor-core scores.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t half_key(uint32_t u)
-{
-    u &= 0xFFFFu;
-    return (u & 0x8000u) ? (~u & 0xFFFFu) : (u | 0x8000u);
-}
-
-__device__ __forceinline__ float key_half_value(uint32_t k)
-{
-    const uint16_t u = (k & 0x8000u) ? (uint16_t)(k & 0x7FFFu) : (uint16_t)(~k & 0xFFFFu);
-    return __half2float(__ushort_as_half(u));
-}
-
 constexpr int FILL_THREADS = 128;
-// Radix select (two 8-bit passes over 16-bit keys) shared by the nominator:
-// every thread offers up to NK keys (0 = none); returns the key of the
-// want-th largest and, in *need_eq, how many keys equal to it are needed to
-// make up `want`.
-template <int NK>
-__device__ uint32_t radix16_kth(const uint32_t (&key)[NK], uint32_t want, int* need_eq)
-{
-    __shared__ unsigned hist[256];
-    __shared__ uint32_t sh_prefix, sh_want;
-    if (threadIdx.x == 0) {
-        sh_prefix = 0;
-        sh_want = want;
-    }
-    uint32_t mask = 0;
-    for (int pass = 1; pass >= 0; --pass) {
-        const int sh = 8 * pass;
-        for (int x = threadIdx.x; x < 256; x += blockDim.x) hist[x] = 0;
-        __syncthreads();
-        const uint32_t prefix = sh_prefix;
-#pragma unroll
-        for (int i = 0; i < NK; ++i)
-            if (key[i] != 0u && (key[i] & mask) == prefix) atomicAdd(&hist[(key[i] >> sh) & 255u], 1u);
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            const int l = threadIdx.x;
-            uint32_t hb[8], tot = 0;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                hb[e] = hist[255 - 8 * l - e];
-                tot += hb[e];
-            }
-            uint32_t incl = tot;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (l >= o) incl += y;
-            }
-            const uint32_t w = sh_want;
-            uint32_t cum = incl - tot;
-            if (cum < w && incl >= w) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    if (cum + hb[e] >= w) {
-                        sh_prefix = prefix | ((uint32_t)(255 - 8 * l - e) << sh);
-                        sh_want = w - cum;
-                        break;
-                    }
-                    cum += hb[e];
-                }
-            }
-        }
-        mask |= 255u << sh;
-        __syncthreads();
-    }
-    *need_eq = (int)sh_want;
-    const uint32_t T = sh_prefix;
-    __syncthreads();
-    return T;
-}
-
-constexpr int NOM_CHUNK_MAX = 2048;   // chunk maxima held in registers: up to 65536 buckets
-
-// Candidate nomination from a query's fp16 tensor-core scores (CTA of
-// FILL_THREADS threads, nb > KC eligible buckets).  The scores come in chunks
-// of 32 with each chunk's maximum stored beside them.  The KC chunks with the
-// largest maxima hold the KC largest scores (each of those scores is at least
-// the KC-th largest chunk maximum, so it lies in a chunk whose maximum is at
-// least that), so only those chunks are read: the KC largest of their scores
-// are the candidates.  Every bucket left out scored at most
-// tau16 = max(the KC-th largest key among the read scores, the largest
-// maximum of a chunk that was not read).  Returns the fp32 upper bound of the
-// approximate binary32 score of every bucket left out: the midpoint between
-// tau16 and the next fp16 value above it (round to nearest put every such
-// score at or below it).
-__device__ float nominate_from_scores(const __half* srow, const __half* crow, int64_t nb,
-                                      int* cg)
-{
-    __shared__ int chunk_sel[KC];
-    __shared__ uint8_t in_sel[NOM_CHUNK_MAX];
-    __shared__ uint32_t sh_rest;
-    __shared__ int sh_gt, sh_eq;
-    const int nch = (int)((nb + 31) / 32);
-    constexpr int CPT = NOM_CHUNK_MAX / FILL_THREADS;       // chunk keys per thread
-    if (threadIdx.x == 0) {
-        sh_rest = 0;
-        sh_gt = 0;
-        sh_eq = 0;
-    }
-    for (int c = threadIdx.x; c < nch; c += FILL_THREADS) in_sel[c] = 0;
-    // 1. the KC chunks with the largest maxima (all of them when nch <= KC)
-    uint32_t ck[CPT];
-#pragma unroll
-    for (int i = 0; i < CPT; ++i) {
-        const int c = threadIdx.x + i * FILL_THREADS;
-        ck[i] = (c < nch) ? half_key(__half_as_ushort(crow[c])) : 0u;
-    }
-    int n_read;
-    if (nch <= KC) {
-        for (int c = threadIdx.x; c < nch; c += FILL_THREADS) chunk_sel[c] = c;
-        n_read = nch;
-        __syncthreads();
-    } else {
-        int need;
-        const uint32_t Tc = radix16_kth<CPT>(ck, KC, &need);
-#pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-            const int c = threadIdx.x + i * FILL_THREADS;
-            if (ck[i] > Tc) {
-                const int q = atomicAdd(&sh_gt, 1);
-                chunk_sel[q] = c;
-                in_sel[c] = 1;
-            } else if (ck[i] == Tc && ck[i] != 0u) {
-                const int q = atomicAdd(&sh_eq, 1);
-                if (q < need) {
-                    chunk_sel[KC - need + q] = c;
-                    in_sel[c] = 1;
-                }
-            }
-        }
-        __syncthreads();
-        // the largest maximum among chunks not read bounds every score in them
-#pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-            const int c = threadIdx.x + i * FILL_THREADS;
-            if (c < nch && !in_sel[c]) atomicMax(&sh_rest, ck[i]);
-        }
-        n_read = KC;
-    }
-    // 2. the read chunks' scores: KC chunks x 32 = 2048 keys, 16 per thread
-    constexpr int EPT = KC * 32 / FILL_THREADS;
-    uint32_t ek[EPT];
-    int eg[EPT];
-#pragma unroll
-    for (int i = 0; i < EPT; ++i) {
-        const int slot = threadIdx.x + i * FILL_THREADS;      // slot = chunk rank * 32 + lane
-        const int ci = slot >> 5, j = slot & 31;
-        ek[i] = 0u;
-        eg[i] = -1;
-        if (ci < n_read) {
-            const int64_t g = (int64_t)chunk_sel[ci] * 32 + j;
-            if (g < nb) {
-                ek[i] = half_key(__half_as_ushort(srow[g]));
-                eg[i] = (int)g;
-            }
-        }
-    }
-    if (threadIdx.x == 0) {
-        sh_gt = 0;
-        sh_eq = 0;
-    }
-    int need;
-    const uint32_t T = radix16_kth<EPT>(ek, KC, &need);
-#pragma unroll
-    for (int i = 0; i < EPT; ++i) {
-        if (ek[i] == 0u) continue;
-        if (ek[i] > T) {
-            cg[atomicAdd(&sh_gt, 1)] = eg[i];
-        } else if (ek[i] == T) {
-            const int q = atomicAdd(&sh_eq, 1);
-            if (q < need) cg[KC - need + q] = eg[i];
-        }
-    }
-    __syncthreads();
-    const uint32_t k = T > sh_rest ? T : sh_rest;
-    const float tv = key_half_value(k);
-    const float above = (k >= 0xFFFFu) ? INFINITY : key_half_value(k + 1);
-    return tv + 0.5f * (above - tv);
-}
+static_assert(FILL_THREADS == KCF, "one candidate per fill thread");
 
 // ---------------------------------------------------------------------------
 // Exact ranking + greedy fill + emission.  One CTA (128 threads) per query.
 // ---------------------------------------------------------------------------
-template <typename T, bool FROM_SCORES>
+template <typename T>
 __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix, int64_t n_blk,
                                                                    const T* lq, PosSrc pos,
                                                                    int64_t Nq, int R, int W, int S,
@@ -753,20 +571,22 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
 {
     extern __shared__ int32_t open_sm[];   // [2][G] when the open block exists
     __shared__ float q_s[DL];
-    __shared__ int cg[KC];
-    __shared__ double es[KC];
-    __shared__ int order[KC];
-    __shared__ int64_t av[KC];
-    __shared__ int64_t avc[KC];          // closed part of av
-    __shared__ int take_g[KC];
-    __shared__ int64_t take_n[KC];
-    __shared__ int64_t take_closed[KC];  // its available closed keys
-    __shared__ int64_t take_lo[KC];      // its closed keys below the sinks bound
-    __shared__ int64_t take_off[KC];     // output offset of each taken bucket
-    __shared__ int32_t take_o0[KC];      // its first CSR position
-    __shared__ int take_full[KC];
-    __shared__ int sh_ntake, sh_exact;
-    __shared__ float sh_l1;
+    __shared__ int cg[KCF];
+    __shared__ double es[KCF];
+    __shared__ int order[KCF];
+    __shared__ int64_t av[KCF];
+    __shared__ int64_t avc[KCF];          // closed part of av
+    __shared__ int take_g[KCF];
+    __shared__ int64_t take_n[KCF];
+    __shared__ int64_t take_closed[KCF];  // its available closed keys
+    __shared__ int64_t take_lo[KCF];      // its closed keys below the sinks bound
+    __shared__ int64_t take_off[KCF];     // output offset of each taken bucket
+    __shared__ int32_t take_o0[KCF];      // its first CSR position
+    __shared__ int take_full[KCF];
+    __shared__ int sh_ntake, sh_exact, sh_nc, sh_complete;
+    __shared__ float sh_l1, sh_tau;
+    __shared__ int lst_off[FILL_THREADS + 1];
+    __shared__ float lst_tau_s[FILL_THREADS];
     const int64_t b = blockIdx.y, i = blockIdx.x;
     const int64_t row = b * Nq + i;
     const int64_t pq = pos.at(b, Nq, i);
@@ -791,24 +611,57 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
         }
     }
     load_query(q_s, lq, row);
-    int nc;
-    float tau;
-    if (FROM_SCORES) {
-        const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
-        if (nb <= KC) {
-            if (threadIdx.x < KC) cg[threadIdx.x] = (threadIdx.x < nb) ? (int)threadIdx.x : -1;
-            nc = (int)nb;
-            tau = -INFINITY;
-        } else {
-            tau = nominate_from_scores(ws.scores + row * ws.score_ld,
-                                       ws.cmax + row * (ws.score_ld / 32), nb, cg);
-            nc = KC;
+    // The row's candidate lists (n_lst <= FILL_THREADS): counts and bounds in
+    // parallel, their offsets by one thread, then the bucket ids.  tau bounds
+    // every eligible bucket left out of the lists; with every list complete
+    // there is none.
+    {
+        const int nl = ws.n_lst;
+        if ((int)threadIdx.x < nl) {
+            lst_off[threadIdx.x + 1] = ws.lst_n[row * nl + threadIdx.x];
+            lst_tau_s[threadIdx.x] = ws.lst_tau[row * nl + threadIdx.x];
         }
-    } else {
-        nc = ws.ncand[row];
-        tau = ws.tau[row];
-        if (threadIdx.x < KC) cg[threadIdx.x] = ws.cand[row * KC + threadIdx.x];
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int tot = 0, comp = 1;
+            float tmax = -INFINITY;
+            lst_off[0] = 0;
+            for (int l = 0; l < nl; ++l) {
+                tot += lst_off[l + 1];
+                lst_off[l + 1] = tot;
+                const float t = lst_tau_s[l];
+                if (t > -INFINITY) comp = 0;
+                tmax = fmaxf(tmax, t);
+            }
+            sh_nc = tot;
+            sh_tau = tmax;
+            sh_complete = comp;
+        }
+        __syncthreads();
+        const int tot = sh_nc;
+        if (tot > KCF) {
+            // more candidates than the fill ranks: the exact fallback takes the row
+            if (threadIdx.x == 0) {
+                const int slot = atomicAdd(ws.fb_count, 1);
+                ws.fb_list[slot] = (int32_t)row;
+                atomicAdd(ix.status + 1, 1u);
+                if (ws.plan.row_n) {
+                    ws.plan.row_n[row] = -1;
+                    ws.plan.row_base[row] = -1;
+                    ws.plan.gather_rows[atomicAdd(ws.plan.ctr + CTR_GATHER, 1)] = (int32_t)row;
+                }
+            }
+            return;
+        }
+        if ((int)threadIdx.x < tot) {
+            int l = 0;
+            while (lst_off[l + 1] <= (int)threadIdx.x) ++l;
+            cg[threadIdx.x] =
+                ws.lst_g[(row * nl + l) * ws.lst_cap + ((int)threadIdx.x - lst_off[l])];
+        }
     }
+    const int nc = sh_nc;
+    const float tau = sh_tau;
     __syncthreads();
     if (threadIdx.x == 0) {
         float l1 = 0.f;
@@ -839,7 +692,7 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
         f.ol_n = build_open_list(ix, b, open_sm, open_sm + ix.G, cnt_w);
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __shared__ int slow[KC];
+    __shared__ int slow[KCF];
     __shared__ int n_slow;
     if (threadIdx.x == 0) n_slow = 0;
     __syncthreads();
@@ -884,7 +737,7 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
             if (rem == 0) cut = c;
         }
         int exact = 1;
-        if (nc == KC) {
+        if (!sh_complete) {
             const double eps = ldexp((double)sh_l1, -12);
             if (rem > 0) {
                 int64_t total = f.hi - S + 1;  // keys in [S, pos - W]
@@ -1173,17 +1026,27 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_prep_kernel(
                 }
             }
             __syncthreads();
-            __half* srow = ws.scores + b * ws.score_ld + g0;
-            __half* crow = ws.cmax + b * (ws.score_ld / 32) + g0 / 32;
-            for (int r = threadIdx.x; r < n; r += DEC_THREADS) srow[r] = __float2half_rn(sc[r]);
-            // chunk maxima (fp16 rounding is monotone: the rounded maximum is
-            // the maximum of the rounded scores)
-            for (int c = warp; c * 32 < n; c += DEC_THREADS / 32) {
-                const int r = c * 32 + lane;
-                float m = (r < n) ? sc[r] : -INFINITY;
-                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                if (lane == 0) crow[c] = __float2half_rn(m);
+            // this slice's candidate list: the m largest scores (ties to the
+            // lower bucket), each at its rank; tau = the next score
+            const int m = ws.lst_cap;
+            int32_t* lg = ws.lst_g + ((int64_t)b * ws.n_lst + sl) * m;
+            for (int t = threadIdx.x; t < n; t += DEC_THREADS) {
+                const float x = sc[t];
+                int rank = 0;
+                for (int u = 0; u < n; ++u) {
+                    const float y = sc[u];
+                    rank += (y > x) || (y == x && u < t);
+                }
+                if (rank < m) lg[rank] = (int32_t)(g0 + t);
+                else if (rank == m) ws.lst_tau[b * ws.n_lst + sl] = x;
             }
+            if (threadIdx.x == 0) {
+                ws.lst_n[b * ws.n_lst + sl] = min(n, m);
+                if (n <= m) ws.lst_tau[b * ws.n_lst + sl] = -INFINITY;
+            }
+        } else if (threadIdx.x == 0) {
+            ws.lst_n[b * ws.n_lst + sl] = 0;
+            ws.lst_tau[b * ws.n_lst + sl] = -INFINITY;
         }
     }
 
@@ -1335,58 +1198,63 @@ static inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 bool select_uses_tc(const IndexView& ix, int64_t Nq)
 {
-    return ix.dtype == LSA_BF16 && Nq >= 128 && ix.NBK <= (int64_t)NOM_CHUNK_MAX * 32 &&
-           tc_scoring_available();
+    return ix.dtype == LSA_BF16 && Nq >= 128 && tc_scoring_available();
 }
 
-static int64_t score_ld_of(const IndexView& ix) { return ((ix.NBK + 255) / 256) * 256; }
+// Candidate lists per row: one per tensor-core split, or one of KC from the
+// SIMT nominator.
+static void list_shape(const IndexView& ix, int64_t Nq, int* n_lst, int* cap)
+{
+    if (select_uses_tc(ix, Nq)) {
+        *n_lst = tc_split_plan(ix, Nq).n_split;
+        *cap = TC_LIST_CAP;
+    } else {
+        *n_lst = 1;
+        *cap = KC;
+    }
+}
 
 size_t select_ws_bytes(const IndexView& ix, int64_t Nq)
 {
     const size_t rows = (size_t)ix.B * (size_t)Nq;
-    size_t n = al256(rows * KC * 4) + al256(rows * 4) + al256(rows * 4) + al256(rows * 4) + al256(4) +
-               al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
-    if (select_uses_tc(ix, Nq))
-        n += al256(rows * (size_t)score_ld_of(ix) * 2) + al256(rows * (size_t)score_ld_of(ix) / 16);
-    return n;
+    int nl, cap;
+    list_shape(ix, Nq, &nl, &cap);
+    return al256(rows * nl * cap * 4) + al256(rows * nl * 4) + al256(rows * nl * 4) +
+           al256(rows * 4) + al256(4) + al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
 }
 
 SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
 {
     const size_t rows = (size_t)ix.B * (size_t)Nq;
+    int nl, cap;
+    list_shape(ix, Nq, &nl, &cap);
     char* p = (char*)ws;
     SelectWs w;
-    w.cand = (int32_t*)p;
-    p += al256(rows * KC * 4);
-    w.tau = (float*)p;
-    p += al256(rows * 4);
-    w.ncand = (int32_t*)p;
-    p += al256(rows * 4);
+    w.n_lst = nl;
+    w.lst_cap = cap;
+    w.lst_g = (int32_t*)p;
+    p += al256(rows * nl * cap * 4);
+    w.lst_n = (int32_t*)p;
+    p += al256(rows * nl * 4);
+    w.lst_tau = (float*)p;
+    p += al256(rows * nl * 4);
     w.fb_list = (int32_t*)p;
     p += al256(rows * 4);
     w.fb_count = (int32_t*)p;
     p += al256(4);
     w.fb_scores = (double*)p;
     p += al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
-    w.score_ld = score_ld_of(ix);
     w.plan = BucketPlan{};
     w.app_score = nullptr;
     w.app_g = nullptr;
     w.app_slot = nullptr;
     w.app_n = 0;
-    w.scores = nullptr;
-    w.cmax = nullptr;
-    if (select_uses_tc(ix, Nq)) {
-        w.scores = (__half*)p;
-        p += al256(rows * (size_t)w.score_ld * 2);
-        w.cmax = (__half*)p;
-    }
     return w;
 }
 
-cudaError_t launch_score_topk_tc(const IndexView& ix, int64_t n_blk, const void* latent_Q,
-                                 PosSrc pos, int64_t Nq, int W, const SelectWs& ws,
-                                 cudaStream_t st);
+cudaError_t launch_score_lists_tc(const IndexView& ix, int64_t n_blk, const void* latent_Q,
+                                  PosSrc pos, int64_t Nq, int W, const SelectWs& ws,
+                                  cudaStream_t st);
 
 template <typename T>
 static cudaError_t launch_finish_t(const IndexView& ix, int64_t n_blk, const T* lq, PosSrc pos,
@@ -1396,12 +1264,9 @@ static cudaError_t launch_finish_t(const IndexView& ix, int64_t n_blk, const T* 
     dim3 grid((unsigned)Nq, (unsigned)ix.B);
     // the compacted open list, when the index has an open block
     const size_t osm = (n_blk > 0 && n_blk * ix.G < ix.NP) ? (size_t)ix.G * 2 * sizeof(int32_t) : 0;
-    if (ws.scores)
-        select_fill_kernel<T, true><<<grid, FILL_THREADS, osm, st>>>(
-            ix, n_blk, lq, pos, Nq, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
-    else
-        select_fill_kernel<T, false><<<grid, FILL_THREADS, osm, st>>>(
-            ix, n_blk, lq, pos, Nq, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
+    if (ws.n_lst < 1 || ws.n_lst > FILL_THREADS || ws.lst_cap < 1) return cudaErrorInvalidValue;
+    select_fill_kernel<T><<<grid, FILL_THREADS, osm, st>>>(
+        ix, n_blk, lq, pos, Nq, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
     note_launch();
     const int64_t rows = ix.B * Nq;
     const unsigned fb_grid = (unsigned)(rows < FB_CTAS ? rows : FB_CTAS);
@@ -1421,7 +1286,7 @@ static cudaError_t launch_select_t(const IndexView& ix, int64_t n_blk, const T* 
     dim3 grid((unsigned)Nq, (unsigned)ix.B);
     cudaError_t e;
     if (use_tc) {
-        e = launch_score_topk_tc(ix, n_blk, lq, pos, Nq, sp.window, ws, st);
+        e = launch_score_lists_tc(ix, n_blk, lq, pos, Nq, sp.window, ws, st);
         if (e != cudaSuccess) return e;
     } else {
         const size_t smem = (size_t)n_blk * ix.k * sizeof(float);

@@ -200,9 +200,9 @@ int64_t ent_cap_for(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d, ls
 }
 
 struct DecodeLayout {
-    size_t indices, counts, sel, part, counter, scores, cmax, app_score, app_g, app_slot, total;
-    int ns, kps, n_hg, n_slice;
-    int64_t score_ld;
+    size_t indices, counts, sel, part, counter, lst_g, lst_n, lst_tau, app_score, app_g, app_slot,
+        total;
+    int ns, kps, n_hg, n_slice, lst_cap;
 };
 
 
@@ -239,15 +239,17 @@ DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_sel
     L.part = o;    o += al256((size_t)v.B * ns * Hq * (d + 4) * 4);
     L.counter = o; o += al256((size_t)v.B * L.n_hg * 4);
     // the append and scoring pass: about one CTA per SM over all sequences,
-    // with at most 992 buckets per slice
+    // with at most 992 buckets per slice and at most 128 slices (the fill
+    // merges one candidate list per slice); each slice nominates its m best
     int64_t nsl = ((int64_t)sm_count() + v.B - 1) / v.B;
     const int64_t min_sl = (v.NBK + 991) / 992;
     if (nsl < min_sl) nsl = min_sl;
-    if (nsl > 65535) nsl = 65535;
+    if (nsl > 128) nsl = 128;
     L.n_slice = (int)nsl;
-    L.score_ld = ((v.NBK + 255) / 256) * 256;
-    L.scores = o;    o += al256((size_t)v.B * L.score_ld * 2);
-    L.cmax = o;      o += al256((size_t)v.B * (L.score_ld / 32) * 2);
+    L.lst_cap = (int)((DEC_TARGET + nsl - 1) / nsl);
+    L.lst_g = o;     o += al256((size_t)v.B * nsl * L.lst_cap * 4);
+    L.lst_n = o;     o += al256((size_t)v.B * nsl * 4);
+    L.lst_tau = o;   o += al256((size_t)v.B * nsl * 4);
     L.app_score = o; o += al256((size_t)v.B * nsl * 8);
     L.app_g = o;     o += al256((size_t)v.B * nsl * 4);
     L.app_slot = o;  o += al256((size_t)v.B * 4);
@@ -750,11 +752,13 @@ lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
     int32_t* indices = (int32_t*)(base + L.indices);
     int32_t* counts = (int32_t*)(base + L.counts);
     SelectWs w = select_ws_carve(base + L.sel, v, 1);
-    // the fill nominates from the score row the prep pass writes, and finishes
-    // the prep pass's append
-    w.scores = (__half*)(base + L.scores);
-    w.cmax = (__half*)(base + L.cmax);
-    w.score_ld = L.score_ld;
+    // the fill ranks the candidate lists the prep pass writes (one per
+    // slice), and finishes the prep pass's append
+    w.lst_g = (int32_t*)(base + L.lst_g);
+    w.lst_n = (int32_t*)(base + L.lst_n);
+    w.lst_tau = (float*)(base + L.lst_tau);
+    w.n_lst = L.n_slice;
+    w.lst_cap = L.lst_cap;
     double* app_score = (double*)(base + L.app_score);
     int32_t* app_g = (int32_t*)(base + L.app_g);
     int32_t* app_slot = (int32_t*)(base + L.app_slot);

@@ -133,17 +133,19 @@ struct BucketPlan {
 };
 constexpr int TILE_REC_BYTES = 448;
 
-// Selection workspace carve-up.
+// Selection workspace carve-up.  Candidates reach the fill as n_lst lists
+// per query row (one per tensor-core split, per decode slice, or one from the
+// SIMT nominator): list l of row r holds lst_n[r*n_lst+l] <= lst_cap bucket
+// ids, and lst_tau[r*n_lst+l] bounds the approximate score of every eligible
+// bucket of the list's range that it does not hold (-inf: it holds them all).
 struct SelectWs {
-    int32_t* cand;       // [B][Nq][KC] candidate bucket ids (-1 padded)
-    float* tau;          // [B][Nq]     approximate score bound of non-candidates
-    int32_t* ncand;      // [B][Nq]
+    int32_t* lst_g;      // [B*Nq][n_lst][lst_cap] candidate bucket ids
+    int32_t* lst_n;      // [B*Nq][n_lst]
+    float* lst_tau;      // [B*Nq][n_lst]
+    int n_lst, lst_cap;
     int32_t* fb_list;    // [B*Nq]      queries that need the exact fallback
     int32_t* fb_count;   // [1]
     double* fb_scores;   // [FB_CTAS][NBK] scratch of the fallback
-    __half* scores;      // [B*Nq][score_ld] tensor-core scores (tensor-core path only)
-    __half* cmax;        // [B*Nq][score_ld/32] maximum of every 32-score chunk
-    int64_t score_ld;
     BucketPlan plan;     // bucket-major attention lists (all null when unused)
     // Decode append finished by the fill (app_n = 0 when unused): the exact
     // nearest-centroid search of sequence b's completed group ran in app_n
@@ -155,6 +157,22 @@ struct SelectWs {
     int app_n;
 };
 constexpr int FB_CTAS = 148;
+constexpr int KCF = 128;          // candidates the fill ranks at most (one per thread)
+constexpr int TC_LIST_CAP = 64;   // candidates per (row, tensor-core split)
+constexpr int TC_MAX_SPLITS = 8;
+constexpr int TC_TARGET = 48;     // threshold ranks summed over a row's splits
+constexpr int DEC_TARGET = 64;    // candidates summed over a decode query's slices
+
+// Work split of the tensor-core scorer (k_score_tc.cu).
+struct TcSplit {
+    int n_split;      // centroid ranges (lists per row)
+    int tps;          // centroid tiles of 256 per range
+    int gw_log2;      // group width (columns) of the threshold's group maxima
+    int m;            // threshold rank per range
+    int64_t n_qt;     // 128-query tiles per sequence
+    int64_t n_items;  // B * n_qt * n_split
+};
+TcSplit tc_split_plan(const IndexView& ix, int64_t Nq);
 // The tensor-core scorer serves bf16 indices and at least one 128-query tile.
 bool select_uses_tc(const IndexView& ix, int64_t Nq);
 size_t select_ws_bytes(const IndexView& ix, int64_t Nq);

@@ -64,7 +64,7 @@ def test_noalloc_select_at_its_size_limit_with_two_sequences():
     # Two sequences on the tensor-core path (bf16, Nq >= 128): the largest
     # query count whose scratch fits the 8 MiB array gives lsa_select's
     # selections; one query more is refused before any launch.
-    w, idx, lq, pos = _case("bf16", 4096, seed=23)
+    w, idx, lq, pos = _case("bf16", 12000, seed=23)
     limit = 8 << 20
     need = lambda n: int(lsa._lib.lsa_select_workspace_bytes(idx.handle, n))
     lo, hi = 128, w.nq
