@@ -8,29 +8,30 @@
 // accumulated in fp32.
 //
 // No score matrix is written.  A work item is (sequence, 128-query tile,
-// split), where a split is a contiguous range of centroid tiles; every item
-// computes its scores twice on the tensor cores:
-//   sweep 1  the epilogue keeps, per query row, the maximum of every group of
-//            gw consecutive eligible scores (rounded down to fp16) and then
-//            picks theta, the m-th largest group maximum: at least m scores of
-//            the split are >= theta (each of the m groups holds one);
-//   sweep 2  every eligible score >= theta is appended to the row's list for
-//            the split (bucket id), up to the list's capacity.
-// Every bucket of the split left out of the list scored below theta, or was
-// an appended score that found the list full (the largest of those is kept),
-// so tau = max(theta, largest lost score) bounds the approximate score of
-// every bucket of the split that is not in the list.  A row whose split holds
-// no more eligible buckets than the list capacity lists them all (theta =
-// -inf: the list is complete).  select_fill_kernel (k_select.cu) merges a
-// row's lists, ranks the candidates with exact binary64 scores and proves the
-// exact ranking against the largest tau, or sends the row to the exact
-// fallback.
+// split), where a split is a contiguous range of centroid tiles; persistent
+// CTAs (one per SM) take the items in a fixed round-robin order.  Three
+// launches:
+//   pass 1   (score_tc_kernel<1>) the epilogue writes, per query row, the
+//            maximum of every group of gw consecutive eligible scores, rounded
+//            down to fp16, as ordered 16-bit keys;
+//   theta    (score_theta_kernel, a warp per row) picks theta, the m-th largest
+//            of the row's group maxima over all splits: at least m scores of
+//            the row are >= theta (each of the m groups holds one);
+//   pass 2   (score_tc_kernel<2>) recomputes the scores and appends every
+//            eligible score >= theta to the row's list for the split (bucket
+//            id), up to the list's capacity.
+// Every eligible bucket left out of a list scored below theta, or was an
+// appended score that found the list full (the largest of those is kept), so
+// tau = max(theta, largest lost score) bounds the approximate score of every
+// bucket of the split that is not in the list.  A row with at most KCF
+// eligible buckets lists them all (theta = -inf: the lists are complete).
+// select_fill_kernel (k_select.cu) merges a row's lists, ranks the candidates
+// with exact binary64 scores and proves the exact ranking against the largest
+// tau, or sends the row to the exact fallback.
 //
-// Persistent CTAs (one per SM) take the items in a fixed round-robin order.
 // CTA = 10 warps:
 //   warp 0     TMA producer: each item's query tile (two buffers), then its
-//              centroid tiles, twice, into a TC_STAGES-deep ring (128-byte
-//              swizzle);
+//              centroid tiles into a TC_STAGES-deep ring (128-byte swizzle);
 //   warp 1     owns 2 x TC_N TMEM columns (two fp32 accumulators) and issues
 //              tcgen05.mma (M = 128, N = TC_N, K = 16, four per tile);
 //   warps 2-9  epilogue: thread = (query row, half of every tile's columns);
@@ -58,7 +59,6 @@ constexpr int TC_STAGES = 4;
 constexpr int TC_EPI_WARPS = 8;
 constexpr int TC_EPI_THREADS = 32 * TC_EPI_WARPS;
 constexpr int TC_THREADS = 64 + TC_EPI_THREADS;           // producer, MMA, epilogue
-constexpr int TC_NG = 64;                                 // group maxima per row and split
 constexpr uint32_t TC_WAIT = 1u << 22;
 
 // Polls each bounded wait of the scorer's roles makes before it gives up.  A
@@ -70,8 +70,7 @@ constexpr int TC_Q_BYTES = TC_M * DL * 2;                 // 16 KB per query buf
 constexpr int TC_C_BYTES = TC_N * DL * 2;                 // 32 KB per ring stage
 constexpr int TC_OFF_C = 2 * TC_Q_BYTES;
 constexpr int TC_OFF_G = TC_OFF_C + TC_STAGES * TC_C_BYTES;
-constexpr int TC_G_BYTES = TC_M * TC_NG * 4;              // group maxima; sweep-2 staging
-static_assert(TC_G_BYTES == TC_EPI_THREADS * 32 * 4, "staging area = group-maximum area");
+constexpr int TC_G_BYTES = TC_EPI_THREADS * 32 * 4;      // pass-2 staging of 32 scores
 constexpr int TC_OFF_BAR = TC_OFF_G + TC_G_BYTES;
 constexpr int TC_NBAR = 2 + 2 + 2 * TC_STAGES + 2 + 2 + 1;
 constexpr int TC_OFF_MISC = TC_OFF_BAR + TC_NBAR * 8;
@@ -205,7 +204,8 @@ __device__ __forceinline__ TcItem tc_item(int64_t it, const IndexView& ix, int64
     return r;
 }
 
-__global__ void __launch_bounds__(TC_THREADS, 1) score_lists_tc_kernel(
+template <int PASS>
+__global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC, IndexView ix,
     int64_t n_blk, PosSrc pos, int64_t Nq, int W, SelectWs ws, TcSplit sp)
 {
@@ -214,7 +214,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_lists_tc_kernel(
         (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);  // 1 KB aligned
     unsigned char* q_s = smem;                        // [2][TC_Q_BYTES]
     unsigned char* c_s = smem + TC_OFF_C;             // [TC_STAGES][TC_C_BYTES]
-    uint32_t* gm = reinterpret_cast<uint32_t*>(smem + TC_OFF_G);   // [TC_M][TC_NG] two halves
     float* stage = reinterpret_cast<float*>(smem + TC_OFF_G);      // [TC_EPI_THREADS][32]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TC_OFF_BAR);
     uint64_t* q_full = bars;                  // [2]
@@ -231,10 +230,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_lists_tc_kernel(
     volatile uint32_t* abort_flag = misc + 1;   // [1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (blockIdx.x == 0 && threadIdx.x == 0) *ws.fb_count = 0;
-    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < ws.plan.n_zero;
-         x += (int64_t)gridDim.x * blockDim.x)
-        ws.plan.zero[x] = 0;
+    if (PASS == 1) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) *ws.fb_count = 0;
+        for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < ws.plan.n_zero;
+             x += (int64_t)gridDim.x * blockDim.x)
+            ws.plan.zero[x] = 0;
+    }
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -289,19 +290,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_lists_tc_kernel(
                 tma_load_2d(q_s + qb * TC_Q_BYTES, &tmQ, 0, (int)(I.b * Nq + I.q0), &q_full[qb]);
             }
             ++qi;
-            for (int sw = 0; sw < 2 && !stop; ++sw)
-                for (int t = I.t0; t < I.t1; ++t, ++gt) {
-                    const int s = (int)(gt % TC_STAGES);
-                    if (!waitw(&empty[s], (uint32_t)(((gt / TC_STAGES) & 1) ^ 1), 1100u)) {
-                        stop = true;
-                        break;
-                    }
-                    if (lane == 0) {
-                        ptx::mbar_arrive_expect_tx(&full[s], TC_C_BYTES);
-                        tma_load_2d(c_s + s * TC_C_BYTES, &tmC, 0,
-                                    (int)(I.b * ix.NBK + (int64_t)t * TC_N), &full[s]);
-                    }
+            for (int t = I.t0; t < I.t1; ++t, ++gt) {
+                const int s = (int)(gt % TC_STAGES);
+                if (!waitw(&empty[s], (uint32_t)(((gt / TC_STAGES) & 1) ^ 1), 1100u)) {
+                    stop = true;
+                    break;
                 }
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(&full[s], TC_C_BYTES);
+                    tma_load_2d(c_s + s * TC_C_BYTES, &tmC, 0,
+                                (int)(I.b * ix.NBK + (int64_t)t * TC_N), &full[s]);
+                }
+            }
         }
         if (*abort_flag && lane == 0) {
             // no copy may still be writing shared memory when the CTA exits:
@@ -324,27 +324,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_lists_tc_kernel(
             if (!waitw(&q_full[qb], (uint32_t)((qi >> 1) & 1), 2000u)) break;
             const uint64_t adesc = sw128_desc(q_s + qb * TC_Q_BYTES);
             ++qi;
-            for (int sw = 0; sw < 2 && !stop; ++sw)
-                for (int t = I.t0; t < I.t1; ++t, ++gt) {
-                    const int s = (int)(gt % TC_STAGES);
-                    const int buf = (int)(gt & 1);
-                    if (!waitw(&full[s], (uint32_t)((gt / TC_STAGES) & 1), 2100u) ||
-                        !waitw(&acc_empty[buf], (uint32_t)(((gt >> 1) & 1) ^ 1), 2200u)) {
-                        stop = true;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (lane == 0) {
-                        const uint64_t bdesc = sw128_desc(c_s + s * TC_C_BYTES);
-                        const uint32_t d = tmem + (uint32_t)(buf * TC_N);
-#pragma unroll
-                        for (int kk = 0; kk < DL / 16; ++kk)
-                            mma_bf16(d, adesc + 2ull * kk, bdesc + 2ull * kk, kk > 0 ? 1u : 0u);
-                        mma_commit(&empty[s]);
-                        mma_commit(&acc_full[buf]);
-                    }
-                    __syncwarp();
+            for (int t = I.t0; t < I.t1; ++t, ++gt) {
+                const int s = (int)(gt % TC_STAGES);
+                const int buf = (int)(gt & 1);
+                if (!waitw(&full[s], (uint32_t)((gt / TC_STAGES) & 1), 2100u) ||
+                    !waitw(&acc_empty[buf], (uint32_t)(((gt >> 1) & 1) ^ 1), 2200u)) {
+                    stop = true;
+                    break;
                 }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint64_t bdesc = sw128_desc(c_s + s * TC_C_BYTES);
+                    const uint32_t d = tmem + (uint32_t)(buf * TC_N);
+#pragma unroll
+                    for (int kk = 0; kk < DL / 16; ++kk)
+                        mma_bf16(d, adesc + 2ull * kk, bdesc + 2ull * kk, kk > 0 ? 1u : 0u);
+                    mma_commit(&empty[s]);
+                    mma_commit(&acc_full[buf]);
+                }
+                __syncwarp();
+            }
             if (!stop && lane == 0) mma_commit(&q_empty[qb]);
             __syncwarp();
         }
@@ -360,8 +359,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_lists_tc_kernel(
         const int h = (warp - 2) >> 2;                    // half of every tile's columns
         const int r = 32 * (warp & 3) + lane;             // query row = TMEM lane
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-        uint16_t* gm16 = reinterpret_cast<uint16_t*>(gm);
         float* my_stage = stage + et * 32;
+        const int gl = sp.gw_log2;                        // 2 .. 5
         int64_t gt = 0;
         for (int64_t it = blockIdx.x; it < sp.n_items; it += gridDim.x) {
             const TcItem I = tc_item(it, ix, n_blk, pos, Nq, W, sp);
@@ -369,27 +368,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_lists_tc_kernel(
             const int64_t row = I.b * Nq + I.q0 + r;
             const int64_t nb_row =
                 row_valid ? tc_eligible(ix, n_blk, pos.at(I.b, Nq, I.q0 + r), W) : 0;
-            const int64_t cs0 = (int64_t)I.s * sp.tps * TC_N;     // first column of the split
-            const int64_t cs1 = cs0 + (int64_t)sp.tps * TC_N;
-            const int64_t n_el = max((int64_t)0, min(nb_row, cs1) - cs0);   // eligible here
             const int64_t lslot = row * sp.n_split + I.s;
             if (I.t1 <= I.t0) {
-                if (h == 0 && row_valid) {
+                if (PASS == 2 && h == 0 && row_valid) {
                     ws.lst_n[lslot] = 0;
                     ws.lst_tau[lslot] = -INFINITY;
                 }
                 continue;
             }
-            const bool take_all = n_el <= ws.lst_cap;
+            const float theta = (PASS == 2 && row_valid) ? ws.theta[row] : -INFINITY;
+            uint16_t* grow = ws.gmax + row * ws.n_grp;
+            float lost = -INFINITY;
             const bool go = __all_sync(0xffffffffu, *abort_flag == 0);   // warp-uniform
-            // ---- sweep 1: group maxima (fp16, rounded down) ----
-            for (int g = 0; g < TC_NG; ++g) gm16[(r * TC_NG + g) * 2 + h] = 0;
-            float gacc = -INFINITY;
-            int gcur = -1;
-            auto flush = [&]() {
-                if (gcur >= 0 && gacc > -INFINITY)
-                    gm16[(r * TC_NG + gcur) * 2 + h] = (uint16_t)tc_half_key(__float2half_rd(gacc));
-            };
             for (int t = I.t0; t < I.t1; ++t, ++gt) {
                 const int buf = (int)(gt & 1);
                 const bool ok = go && waitw(&acc_full[buf], (uint32_t)((gt >> 1) & 1), 4000u);
@@ -400,52 +390,69 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_lists_tc_kernel(
                         __syncwarp();
                         tmem_ld32(tmem + lane_base + (uint32_t)(buf * TC_N + h * 128 + c * 32), v);
                         const int64_t g0 = (int64_t)t * TC_N + h * 128 + c * 32;
-                        if (take_all || g0 >= nb_row) continue;
-                        if (g0 + 32 > nb_row) {
+                        if (PASS == 1) {
+                            // group maxima of the eligible scores, as fp16 keys
+                            // rounded down (0 = no eligible score in the group)
+                            if (!row_valid || g0 >= nb_row) continue;
+                            if (g0 + 32 > nb_row) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (g0 + j >= nb_row) v[j] = -INFINITY;
-                        }
-                        // maxima of 1 .. 32 consecutive scores as a tree
-                        float m16[16], m8[8], m4[4], m2[2];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) m16[j] = fmaxf(v[2 * j], v[2 * j + 1]);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) m8[j] = fmaxf(m16[2 * j], m16[2 * j + 1]);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) m4[j] = fmaxf(m8[2 * j], m8[2 * j + 1]);
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) m2[j] = fmaxf(m4[2 * j], m4[2 * j + 1]);
-                        const float m1 = fmaxf(m2[0], m2[1]);
-                        const int rel = (int)(g0 - cs0);
-                        if (sp.gw_log2 >= 5) {
-                            const int grp = rel >> sp.gw_log2;
-                            if (grp != gcur) {
-                                flush();
-                                gcur = grp;
-                                gacc = -INFINITY;
+                                for (int j = 0; j < 32; ++j)
+                                    if (g0 + j >= nb_row) v[j] = -INFINITY;
                             }
-                            gacc = fmaxf(gacc, m1);
-                        } else {
-                            // groups narrower than a load: write each directly
-                            const int gb = rel >> sp.gw_log2;
-                            auto put = [&](int u, float x) {
-                                if (x > -INFINITY)
-                                    gm16[(r * TC_NG + gb + u) * 2 + h] =
-                                        (uint16_t)tc_half_key(__float2half_rd(x));
+                            float m16[16], m8[8], m4[4], m2[2];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) m16[j] = fmaxf(v[2 * j], v[2 * j + 1]);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) m8[j] = fmaxf(m16[2 * j], m16[2 * j + 1]);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) m4[j] = fmaxf(m8[2 * j], m8[2 * j + 1]);
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) m2[j] = fmaxf(m4[2 * j], m4[2 * j + 1]);
+                            auto key = [](float x) -> uint32_t {
+                                return x > -INFINITY ? tc_half_key(__float2half_rd(x)) : 0u;
                             };
-                            if (sp.gw_log2 == 4) {
-#pragma unroll
-                                for (int u = 0; u < 2; ++u) put(u, m2[u]);
-                            } else if (sp.gw_log2 == 3) {
-#pragma unroll
-                                for (int u = 0; u < 4; ++u) put(u, m4[u]);
-                            } else if (sp.gw_log2 == 2) {
-#pragma unroll
-                                for (int u = 0; u < 8; ++u) put(u, m8[u]);
+                            if (gl == 5) {
+                                grow[g0 >> 5] = (uint16_t)key(fmaxf(m2[0], m2[1]));
+                            } else if (gl == 4) {
+                                *reinterpret_cast<uint32_t*>(grow + (g0 >> 4)) =
+                                    key(m2[0]) | (key(m2[1]) << 16);
+                            } else if (gl == 3) {
+                                *reinterpret_cast<uint2*>(grow + (g0 >> 3)) =
+                                    make_uint2(key(m4[0]) | (key(m4[1]) << 16),
+                                               key(m4[2]) | (key(m4[3]) << 16));
                             } else {
+                                uint4* dst = reinterpret_cast<uint4*>(grow + (g0 >> 2));
+                                dst[0] = make_uint4(key(m8[0]) | (key(m8[1]) << 16),
+                                                    key(m8[2]) | (key(m8[3]) << 16),
+                                                    key(m8[4]) | (key(m8[5]) << 16),
+                                                    key(m8[6]) | (key(m8[7]) << 16));
+                            }
+                        } else {
+                            // append every eligible score >= theta
+                            uint32_t vm = 0u;
+                            if (g0 + 32 <= nb_row) vm = 0xFFFFFFFFu;
+                            else if (g0 < nb_row) vm = (1u << (uint32_t)(nb_row - g0)) - 1u;
+                            uint32_t msk = 0u;
 #pragma unroll
-                                for (int u = 0; u < 16; ++u) put(u, m16[u]);
+                            for (int j = 0; j < 32; ++j) msk |= (v[j] >= theta) ? (1u << j) : 0u;
+                            msk &= vm;
+                            if (__any_sync(0xffffffffu, msk != 0u)) {
+                                if (msk) {
+                                    float4* st4 = reinterpret_cast<float4*>(my_stage);
+#pragma unroll
+                                    for (int j = 0; j < 8; ++j)
+                                        st4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2],
+                                                             v[4 * j + 3]);
+                                }
+                                while (msk) {
+                                    const int j = __ffs(msk) - 1;
+                                    msk &= msk - 1u;
+                                    const int slot = atomicAdd(&rcnt[r], 1);
+                                    if (slot < ws.lst_cap)
+                                        ws.lst_g[lslot * ws.lst_cap + slot] = (int32_t)(g0 + j);
+                                    else
+                                        lost = fmaxf(lost, my_stage[j]);
+                                }
                             }
                         }
                     }
@@ -454,87 +461,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_lists_tc_kernel(
                 __syncwarp();
                 if (ok && lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
             }
-            flush();
-            epi_sync();
-            // ---- theta: the m-th largest group maximum of the row ----
-            float theta = -INFINITY;
-            if (!take_all) {
-                uint32_t key[TC_NG];
-                int nz = 0;
-#pragma unroll
-                for (int g = 0; g < TC_NG; ++g) {
-                    const uint32_t w = gm[r * TC_NG + g];
-                    key[g] = max(w & 0xFFFFu, w >> 16);
-                    nz += key[g] != 0u;
-                }
-                if (nz >= sp.m) {
-                    uint32_t lo = 1u, hi = 0xFFFFu;       // count(key >= lo) >= m
-                    while (lo < hi) {
-                        const uint32_t mid = (lo + hi + 1u) >> 1;
-                        int cnt = 0;
-#pragma unroll
-                        for (int g = 0; g < TC_NG; ++g) cnt += key[g] >= mid;
-                        if (cnt >= sp.m) lo = mid;
-                        else hi = mid - 1u;
+            if (PASS == 2) {
+                lostv[et] = lost;
+                epi_sync();
+                if (h == 0) {
+                    if (row_valid) {
+                        const float l2 = fmaxf(lost, lostv[et + 128]);   // the other half's thread
+                        ws.lst_n[lslot] = min(rcnt[r], ws.lst_cap);
+                        ws.lst_tau[lslot] = (theta > -INFINITY) ? fmaxf(theta, l2) : l2;
                     }
-                    theta = tc_key_value(lo);
+                    rcnt[r] = 0;
                 }
-            }
-            epi_sync();          // the group maxima become the staging area
-            // ---- sweep 2: append every eligible score >= theta ----
-            float lost = -INFINITY;
-            const bool go2 = __all_sync(0xffffffffu, *abort_flag == 0);
-            for (int t = I.t0; t < I.t1; ++t, ++gt) {
-                const int buf = (int)(gt & 1);
-                const bool ok = go2 && waitw(&acc_full[buf], (uint32_t)((gt >> 1) & 1), 4100u);
-                if (ok) {
-                    tc_fence_after();
-                    for (int c = 0; c < 4; ++c) {
-                        float v[32];
-                        __syncwarp();
-                        tmem_ld32(tmem + lane_base + (uint32_t)(buf * TC_N + h * 128 + c * 32), v);
-                        const int64_t g0 = (int64_t)t * TC_N + h * 128 + c * 32;
-                        uint32_t vm = 0u;
-                        if (g0 + 32 <= nb_row) vm = 0xFFFFFFFFu;
-                        else if (g0 < nb_row) vm = (1u << (uint32_t)(nb_row - g0)) - 1u;
-                        uint32_t msk = 0u;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) msk |= (v[j] >= theta) ? (1u << j) : 0u;
-                        msk &= vm;
-                        if (__any_sync(0xffffffffu, msk != 0u)) {
-                            if (msk) {
-                                float4* st4 = reinterpret_cast<float4*>(my_stage);
-#pragma unroll
-                                for (int j = 0; j < 8; ++j)
-                                    st4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2],
-                                                         v[4 * j + 3]);
-                            }
-                            while (msk) {
-                                const int j = __ffs(msk) - 1;
-                                msk &= msk - 1u;
-                                const int slot = atomicAdd(&rcnt[r], 1);
-                                if (slot < ws.lst_cap)
-                                    ws.lst_g[lslot * ws.lst_cap + slot] = (int32_t)(g0 + j);
-                                else
-                                    lost = fmaxf(lost, my_stage[j]);
-                            }
-                        }
-                    }
-                    tc_fence_before();
-                }
-                __syncwarp();
-                if (ok && lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
-            }
-            lostv[et] = lost;
-            epi_sync();
-            if (h == 0) {
-                if (row_valid) {
-                    const int n = rcnt[r];
-                    const float l2 = fmaxf(lost, lostv[et + 128]);   // the other half's thread
-                    ws.lst_n[lslot] = min(n, ws.lst_cap);
-                    ws.lst_tau[lslot] = take_all ? l2 : fmaxf(theta, l2);
-                }
-                rcnt[r] = 0;
+                epi_sync();      // the counters are clear before the next item appends
             }
         }
     }
@@ -545,6 +483,38 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_lists_tc_kernel(
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(TC_TMEM_COLS)
                      : "memory");
     }
+}
+
+// theta of every query row: a warp per row finds the m-th largest of the
+// row's group maxima by bisection over the 16-bit keys.  A row with at most
+// KCF eligible buckets gets -inf (its lists take every eligible bucket); a row
+// with fewer than 2m groups uses half of them.
+__global__ void __launch_bounds__(256) score_theta_kernel(IndexView ix, int64_t n_blk, PosSrc pos,
+                                                          int64_t Nq, int W, SelectWs ws,
+                                                          TcSplit sp)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (row >= ix.B * Nq) return;                 // warp-uniform
+    const int64_t b = row / Nq, i = row % Nq;
+    const int64_t nb = tc_eligible(ix, n_blk, pos.at(b, Nq, i), W);
+    if (nb <= KCF) {
+        if (lane == 0) ws.theta[row] = -INFINITY;
+        return;
+    }
+    const int64_t ng = (nb + (1 << sp.gw_log2) - 1) >> sp.gw_log2;
+    const int m = (int)min((int64_t)sp.m, max((int64_t)1, ng / 2));
+    const uint16_t* keys = ws.gmax + row * ws.n_grp;
+    uint32_t lo = 1u, hi = 0xFFFFu;               // count(key >= lo) >= m
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi + 1u) >> 1;
+        int cnt = 0;
+        for (int64_t x = lane; x < ng; x += 32) cnt += keys[x] >= mid;
+        cnt = __reduce_add_sync(0xffffffffu, cnt);
+        if (cnt >= m) lo = mid;
+        else hi = mid - 1u;
+    }
+    if (lane == 0) ws.theta[row] = tc_key_value(lo);
 }
 
 // ---- host side ---------------------------------------------------------------
@@ -576,16 +546,14 @@ TcSplit tc_split_plan(const IndexView& ix, int64_t Nq)
     sp.n_split = (int)((n_ct + sp.tps - 1) / sp.tps);
     if (sp.n_split < 1) sp.n_split = 1;
     sp.n_items = tiles * sp.n_split;
-    // m-th largest of the group maxima: the m groups (of gw scores) hold at
-    // least m candidates; with at least 2m groups per split the list holds
-    // about 1.4 m on scores without structure
-    sp.m = (TC_TARGET + sp.n_split - 1) / sp.n_split;
-    const int64_t split_w = (int64_t)sp.tps * TC_N;
+    // groups of 32 scores, narrower (down to 4) while a sequence has fewer than
+    // 4m groups: with g groups and the m-th largest maximum as the threshold,
+    // scores without structure put about -g ln(1 - m/g) of them above it
+    sp.m = TC_TARGET;
     int gl = 5;
-    while (gl > 0 && (split_w >> gl) < 2LL * sp.m) --gl;   // at least 2m groups
-    while ((split_w >> gl) > TC_NG) ++gl;                 // at most TC_NG groups
+    while (gl > 2 && (ix.NBK >> gl) < 4LL * sp.m) --gl;
     sp.gw_log2 = gl;
-    if ((split_w >> gl) < 2LL * sp.m) sp.m = (int)max((int64_t)1, (split_w >> gl) / 2);
+    sp.n_grp = (n_ct * TC_N) >> gl;
     return sp;
 }
 
@@ -601,16 +569,23 @@ cudaError_t launch_score_lists_tc(const IndexView& ix, int64_t n_blk, const void
 {
     if (ix.dtype != LSA_BF16) return cudaErrorInvalidValue;
     const TcSplit sp = tc_split_plan(ix, Nq);
-    if (ws.n_lst != sp.n_split || ws.lst_cap != TC_LIST_CAP) return cudaErrorInvalidValue;
+    if (ws.n_lst != sp.n_split || ws.lst_cap != TC_LIST_CAP || !ws.gmax || !ws.theta ||
+        ws.n_grp != sp.n_grp)
+        return cudaErrorInvalidValue;
     CUtensorMap tmQ, tmC;
     if (!make_rows64_bf16(&tmQ, latent_Q, (uint64_t)ix.B * Nq, TC_M) ||
         !make_rows64_bf16(&tmC, ix.cent_rt, (uint64_t)ix.B * ix.NBK, TC_N))
         return cudaErrorInvalidValue;
-    cudaError_t e = ensure_smem_attr((const void*)score_lists_tc_kernel, TC_SMEM);
+    cudaError_t e = ensure_smem_attr((const void*)score_tc_kernel<1>, TC_SMEM);
+    if (e == cudaSuccess) e = ensure_smem_attr((const void*)score_tc_kernel<2>, TC_SMEM);
     if (e != cudaSuccess) return e;
-    const int64_t n_cta = sp.n_items < sm_count() ? sp.n_items : sm_count();
-    score_lists_tc_kernel<<<(unsigned)n_cta, TC_THREADS, TC_SMEM, st>>>(tmQ, tmC, ix, n_blk, pos,
-                                                                        Nq, W, ws, sp);
+    const unsigned n_cta = (unsigned)(sp.n_items < sm_count() ? sp.n_items : sm_count());
+    score_tc_kernel<1><<<n_cta, TC_THREADS, TC_SMEM, st>>>(tmQ, tmC, ix, n_blk, pos, Nq, W, ws, sp);
+    note_launch();
+    const int64_t rows = ix.B * Nq;
+    score_theta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(ix, n_blk, pos, Nq, W, ws, sp);
+    note_launch();
+    score_tc_kernel<2><<<n_cta, TC_THREADS, TC_SMEM, st>>>(tmQ, tmC, ix, n_blk, pos, Nq, W, ws, sp);
     note_launch();
     return cudaGetLastError();
 }

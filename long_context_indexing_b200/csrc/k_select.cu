@@ -1214,13 +1214,22 @@ static void list_shape(const IndexView& ix, int64_t Nq, int* n_lst, int* cap)
     }
 }
 
+// Group maxima per row of the tensor-core path (0 otherwise).
+static int64_t n_grp_of(const IndexView& ix, int64_t Nq)
+{
+    return select_uses_tc(ix, Nq) ? tc_split_plan(ix, Nq).n_grp : 0;
+}
+
 size_t select_ws_bytes(const IndexView& ix, int64_t Nq)
 {
     const size_t rows = (size_t)ix.B * (size_t)Nq;
     int nl, cap;
     list_shape(ix, Nq, &nl, &cap);
-    return al256(rows * nl * cap * 4) + al256(rows * nl * 4) + al256(rows * nl * 4) +
-           al256(rows * 4) + al256(4) + al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
+    const size_t ng = (size_t)n_grp_of(ix, Nq);
+    size_t n = al256(rows * nl * cap * 4) + al256(rows * nl * 4) + al256(rows * nl * 4) +
+               al256(rows * 4) + al256(4) + al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
+    if (ng) n += al256(rows * ng * 2) + al256(rows * 4);
+    return n;
 }
 
 SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
@@ -1244,6 +1253,15 @@ SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
     p += al256(4);
     w.fb_scores = (double*)p;
     p += al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
+    w.n_grp = n_grp_of(ix, Nq);
+    w.gmax = nullptr;
+    w.theta = nullptr;
+    if (w.n_grp) {
+        w.gmax = (uint16_t*)p;
+        p += al256(rows * (size_t)w.n_grp * 2);
+        w.theta = (float*)p;
+        p += al256(rows * 4);
+    }
     w.plan = BucketPlan{};
     w.app_score = nullptr;
     w.app_g = nullptr;

@@ -246,7 +246,10 @@ DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_sel
     if (nsl < min_sl) nsl = min_sl;
     if (nsl > 128) nsl = 128;
     L.n_slice = (int)nsl;
-    L.lst_cap = (int)((DEC_TARGET + nsl - 1) / nsl);
+    // slices of `per` buckets (a multiple of 32); only the first ones hold any
+    const int64_t per = (((v.NBK + nsl - 1) / nsl) + 31) / 32 * 32;
+    const int64_t used = (v.NBK + per - 1) / per;
+    L.lst_cap = (int)((DEC_TARGET + used - 1) / used);
     L.lst_g = o;     o += al256((size_t)v.B * nsl * L.lst_cap * 4);
     L.lst_n = o;     o += al256((size_t)v.B * nsl * 4);
     L.lst_tau = o;   o += al256((size_t)v.B * nsl * 4);

@@ -143,6 +143,9 @@ struct SelectWs {
     int32_t* lst_n;      // [B*Nq][n_lst]
     float* lst_tau;      // [B*Nq][n_lst]
     int n_lst, lst_cap;
+    uint16_t* gmax;      // [B*Nq][n_grp] tensor-core path: group maxima (fp16 keys)
+    float* theta;        // [B*Nq] tensor-core path: each row's list threshold
+    int64_t n_grp;
     int32_t* fb_list;    // [B*Nq]      queries that need the exact fallback
     int32_t* fb_count;   // [1]
     double* fb_scores;   // [FB_CTAS][NBK] scratch of the fallback
@@ -158,17 +161,18 @@ struct SelectWs {
 };
 constexpr int FB_CTAS = 148;
 constexpr int KCF = 128;          // candidates the fill ranks at most (one per thread)
-constexpr int TC_LIST_CAP = 64;   // candidates per (row, tensor-core split)
+constexpr int TC_LIST_CAP = KCF;  // candidates per (row, tensor-core split)
 constexpr int TC_MAX_SPLITS = 8;
-constexpr int TC_TARGET = 48;     // threshold ranks summed over a row's splits
+constexpr int TC_TARGET = 48;     // rank of a row's threshold among its group maxima
 constexpr int DEC_TARGET = 64;    // candidates summed over a decode query's slices
 
 // Work split of the tensor-core scorer (k_score_tc.cu).
 struct TcSplit {
     int n_split;      // centroid ranges (lists per row)
     int tps;          // centroid tiles of 256 per range
-    int gw_log2;      // group width (columns) of the threshold's group maxima
-    int m;            // threshold rank per range
+    int gw_log2;      // group width (columns) of the group maxima, 2 .. 5
+    int m;            // threshold rank among a row's group maxima
+    int64_t n_grp;    // group maxima per row (all ranges)
     int64_t n_qt;     // 128-query tiles per sequence
     int64_t n_items;  // B * n_qt * n_split
 };
