@@ -141,6 +141,31 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v)
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+// Four 32-column loads in flight, one wait: 128 consecutive columns of this
+// thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v)
+{
+    uint32_t r[128];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+            "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+            "%28, %29, %30, %31}, [%32];"
+            : "=r"(r[32 * q + 0]), "=r"(r[32 * q + 1]), "=r"(r[32 * q + 2]), "=r"(r[32 * q + 3]),
+              "=r"(r[32 * q + 4]), "=r"(r[32 * q + 5]), "=r"(r[32 * q + 6]), "=r"(r[32 * q + 7]),
+              "=r"(r[32 * q + 8]), "=r"(r[32 * q + 9]), "=r"(r[32 * q + 10]), "=r"(r[32 * q + 11]),
+              "=r"(r[32 * q + 12]), "=r"(r[32 * q + 13]), "=r"(r[32 * q + 14]), "=r"(r[32 * q + 15]),
+              "=r"(r[32 * q + 16]), "=r"(r[32 * q + 17]), "=r"(r[32 * q + 18]), "=r"(r[32 * q + 19]),
+              "=r"(r[32 * q + 20]), "=r"(r[32 * q + 21]), "=r"(r[32 * q + 22]), "=r"(r[32 * q + 23]),
+              "=r"(r[32 * q + 24]), "=r"(r[32 * q + 25]), "=r"(r[32 * q + 26]), "=r"(r[32 * q + 27]),
+              "=r"(r[32 * q + 28]), "=r"(r[32 * q + 29]), "=r"(r[32 * q + 30]), "=r"(r[32 * q + 31])
+            : "r"(taddr + 32u * q));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 128; ++j) v[j] = __uint_as_float(r[j]);
+}
+
 // Named barrier of the epilogue warps only.
 __device__ __forceinline__ void epi_sync()
 {
@@ -385,10 +410,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
                 const bool ok = go && waitw(&acc_full[buf], (uint32_t)((gt >> 1) & 1), 4000u);
                 if (ok) {
                     tc_fence_after();
+                    float va[128];
+                    __syncwarp();
+                    tmem_ld128(tmem + lane_base + (uint32_t)(buf * TC_N + h * 128), va);
+                    // the accumulator is in registers: hand it back before the work
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
+#pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        float v[32];
-                        __syncwarp();
-                        tmem_ld32(tmem + lane_base + (uint32_t)(buf * TC_N + h * 128 + c * 32), v);
+                        float* v = va + 32 * c;
                         const int64_t g0 = (int64_t)t * TC_N + h * 128 + c * 32;
                         if (PASS == 1) {
                             // group maxima of the eligible scores, as fp16 keys
@@ -456,10 +487,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
                             }
                         }
                     }
-                    tc_fence_before();
                 }
                 __syncwarp();
-                if (ok && lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
             }
             if (PASS == 2) {
                 lostv[et] = lost;
@@ -485,6 +514,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
     }
 }
 
+constexpr int TH_REG = 64;   // group-maximum keys per lane held in registers (2048 per row)
+
 // theta of every query row: a warp per row finds the m-th largest of the
 // row's group maxima by bisection over the 16-bit keys.  A row with at most
 // KCF eligible buckets gets -inf (its lists take every eligible bucket); a row
@@ -506,13 +537,45 @@ __global__ void __launch_bounds__(256) score_theta_kernel(IndexView ix, int64_t 
     const int m = (int)min((int64_t)sp.m, max((int64_t)1, ng / 2));
     const uint16_t* keys = ws.gmax + row * ws.n_grp;
     uint32_t lo = 1u, hi = 0xFFFFu;               // count(key >= lo) >= m
-    while (lo < hi) {
-        const uint32_t mid = (lo + hi + 1u) >> 1;
-        int cnt = 0;
-        for (int64_t x = lane; x < ng; x += 32) cnt += keys[x] >= mid;
-        cnt = __reduce_add_sync(0xffffffffu, cnt);
-        if (cnt >= m) lo = mid;
-        else hi = mid - 1u;
+    if (ng <= 32 * TH_REG) {
+        // the row's keys in registers, 8 per 16-byte load (n_grp is a multiple
+        // of 8; keys past ng count as 0)
+        uint32_t kw[TH_REG / 2];
+        const uint4* k4 = reinterpret_cast<const uint4*>(keys);
+#pragma unroll
+        for (int u = 0; u < TH_REG / 8; ++u) {
+            const int64_t c = (int64_t)u * 32 + lane;        // 16-byte chunk
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            if (c * 8 < ng) w = k4[c];
+            const uint32_t e[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t x = e[q];
+                const int64_t k0 = c * 8 + 2 * q;
+                if (k0 >= ng) x = 0u;
+                else if (k0 + 1 >= ng) x &= 0xFFFFu;
+                kw[u * 4 + q] = x;
+            }
+        }
+        while (lo < hi) {
+            const uint32_t mid = (lo + hi + 1u) >> 1;
+            int cnt = 0;
+#pragma unroll
+            for (int u = 0; u < TH_REG / 2; ++u)
+                cnt += (int)((kw[u] & 0xFFFFu) >= mid) + (int)((kw[u] >> 16) >= mid);
+            cnt = __reduce_add_sync(0xffffffffu, cnt);
+            if (cnt >= m) lo = mid;
+            else hi = mid - 1u;
+        }
+    } else {
+        while (lo < hi) {
+            const uint32_t mid = (lo + hi + 1u) >> 1;
+            int cnt = 0;
+            for (int64_t x = lane; x < ng; x += 32) cnt += keys[x] >= mid;
+            cnt = __reduce_add_sync(0xffffffffu, cnt);
+            if (cnt >= m) lo = mid;
+            else hi = mid - 1u;
+        }
     }
     if (lane == 0) ws.theta[row] = tc_key_value(lo);
 }

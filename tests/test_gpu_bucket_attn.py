@@ -155,7 +155,7 @@ def test_workspace_below_minimum_is_refused():
 
 
 def test_fallback_rows():
-    w = _base(T=2048, nq=512, G=16, R=300)      # 128 buckets: more than one candidate set
+    w = _base(T=2048, nq=512, G=8, R=300)       # 256 buckets, all tied: more than the fill ranks
     fb, _ = _run(w, seed=18, same_latent=True)
     assert fb > 0
 
