@@ -822,6 +822,356 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
 }
 
 // ---------------------------------------------------------------------------
+// Exact ranking + greedy fill + emission, one warp per query row: the same
+// steps and results as select_fill_kernel, for launches with many rows (a
+// prefill chunk).  Each warp works alone -- no barrier spans the CTA -- so an
+// SM keeps several times more rows in flight, and every serial step of the
+// CTA kernel becomes a warp-wide scan: the greedy fill is a prefix sum of the
+// ranked candidates' available keys, and whole buckets are emitted member by
+// member (p keys per member load).
+// ---------------------------------------------------------------------------
+constexpr int FW_WARPS = 4;            // query rows per CTA
+constexpr int64_t FW_MIN_ROWS = 64;    // fewer rows: a CTA per row (shorter latency per row)
+constexpr int FW_DSMEM_MAX = 192 * 1024;   // dynamic shared memory (open lists) it may use
+constexpr int FW_LISTS = 32;           // candidate lists per row this kernel takes
+constexpr int FW_PL = KCF / 32;        // candidates per lane
+
+struct FwRow {
+    float q[DL];
+    double es[KCF];
+    int cg[KCF];
+    int av[KCF];          // available keys of candidate c
+    int avc[KCF];         // its closed part
+    int order[KCF];       // candidate at rank r
+    int t_g[KCF];         // taken bucket t: id
+    int t_n[KCF];         //   keys taken
+    int t_off[KCF];       //   first long-range slot
+    int t_o0[KCF];        //   first CSR position
+    int t_closed[KCF];    //   available closed keys
+    int t_lo[KCF];        //   closed keys below the sinks bound
+    int t_full[KCF];      //   every closed key available, no open member
+    int t_mc[KCF + 1];    //   members of the whole buckets before it (prefix)
+    int lst_off[FW_LISTS];
+};
+
+template <typename T>
+__global__ void __launch_bounds__(32 * FW_WARPS) select_fill_warp_kernel(
+    IndexView ix, int64_t n_blk, const T* lq, PosSrc pos, int64_t Nq, int R, int W, int S,
+    int s_max, int32_t* indices, int32_t* counts, SelectWs ws)
+{
+    extern __shared__ int32_t fw_open[];   // [FW_WARPS][2][G] when the open block may hold keys
+    __shared__ FwRow fw[FW_WARPS];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * FW_WARPS + warp;
+    if (row >= ix.B * Nq) return;          // warp-uniform; no barrier spans the CTA
+    const unsigned FULL = 0xffffffffu;
+    FwRow& F = fw[warp];
+    const int64_t b = row / Nq, i = row % Nq;
+    const int64_t pq = pos.at(b, Nq, i);
+    F.q[lane] = load_elt(lq + row * DL + lane);
+    F.q[lane + 32] = load_elt(lq + row * DL + lane + 32);
+
+    // ---- the row's candidate lists ----
+    const int nl = ws.n_lst;               // <= FW_LISTS (checked at launch)
+    int ln = 0;
+    float lt = -INFINITY;
+    if (lane < nl) {
+        ln = ws.lst_n[row * nl + lane];
+        lt = ws.lst_tau[row * nl + lane];
+    }
+    int incl = ln;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const int tot = __shfl_sync(FULL, incl, 31);
+    if (lane < nl) F.lst_off[lane] = incl - ln;
+    float tau = lt;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tau = fmaxf(tau, __shfl_xor_sync(FULL, tau, o));
+    const bool complete = !(tau > -INFINITY);   // every list holds all of its range
+    auto to_fallback = [&]() {
+        if (lane == 0) {
+            const int slot = atomicAdd(ws.fb_count, 1);
+            ws.fb_list[slot] = (int32_t)row;
+            atomicAdd(ix.status + 1, 1u);
+            if (ws.plan.row_n) {   // the fallback's selection is attended key by key
+                ws.plan.row_n[row] = -1;
+                ws.plan.row_base[row] = -1;
+                ws.plan.gather_rows[atomicAdd(ws.plan.ctr + CTR_GATHER, 1)] = (int32_t)row;
+            }
+        }
+    };
+    if (tot > KCF) {                       // more candidates than the fill ranks
+        to_fallback();
+        return;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < FW_PL; ++u) {
+        const int c = lane + 32 * u;
+        if (c < tot) {
+            int l = 0;
+            while (l + 1 < nl && F.lst_off[l + 1] <= c) ++l;
+            F.cg[c] = ws.lst_g[(row * nl + l) * ws.lst_cap + (c - F.lst_off[l])];
+        }
+    }
+    __syncwarp();
+
+    // ---- exact scores and ranking ----
+    float l1 = fabsf(F.q[lane]) + fabsf(F.q[lane + 32]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l1 += __shfl_xor_sync(FULL, l1, o);
+#pragma unroll
+    for (int u = 0; u < FW_PL; ++u) {
+        const int c = lane + 32 * u;
+        if (c < tot) F.es[c] = exact_score(ix, b, F.cg[c], F.q);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < FW_PL; ++u) {
+        const int c = lane + 32 * u;
+        if (c < tot) {
+            const double e = F.es[c];
+            const int g = F.cg[c];
+            int r = 0;
+            for (int c2 = 0; c2 < tot; ++c2) r += rank_before(F.es[c2], F.cg[c2], e, g);
+            F.order[r] = c;
+        }
+    }
+
+    // ---- availability of every candidate ----
+    FillCtx f;
+    f.ix = ix;
+    f.bseq = b;
+    f.n_blk = n_blk;
+    f.pos = pq;
+    f.hi = pq - W;
+    f.S = S;
+    f.open_live = (n_blk * ix.G < ix.NP) && (n_blk > 0) && (n_blk * (int64_t)ix.p * ix.G <= f.hi);
+    f.ol_n = 0;
+    int32_t* ol_o = fw_open + (size_t)warp * 2 * ix.G;
+    int32_t* ol_g = ol_o + ix.G;
+    f.ol_o = ol_o;
+    f.ol_g = ol_g;
+    if (f.open_live) {
+        // the open block's assigned groups in ascending slot order
+        const int32_t* open = ix.open_bucket + b * ix.G;
+        int n = 0;
+        for (int x0 = 0; x0 < ix.G; x0 += 32) {
+            const int x = x0 + lane;
+            const int32_t g = (x < ix.G) ? open[x] : -1;
+            const unsigned bal = __ballot_sync(FULL, g >= 0);
+            if (g >= 0) {
+                const int at = n + __popc(bal & ((1u << lane) - 1u));
+                ol_o[at] = x;
+                ol_g[at] = g;
+            }
+            n += __popc(bal);
+        }
+        f.ol_n = n;
+    }
+    __syncwarp();
+    const int32_t* offs = ix.offsets + b * (ix.NBK + 1);
+    const int32_t* mem = ix.members + b * ix.NP;
+    const int p = ix.p;
+    unsigned slow_u = 0;                   // bit u: candidate lane + 32u needs a member scan
+#pragma unroll
+    for (int u = 0; u < FW_PL; ++u) {
+        const int c = lane + 32 * u;
+        if (c < tot) {
+            const int g = F.cg[c];
+            if (bucket_full(f, g)) {
+                F.av[c] = (offs[g + 1] - offs[g]) * p;
+                F.avc[c] = F.av[c];
+            } else {
+                slow_u |= 1u << u;
+            }
+        }
+    }
+    for (int u = 0; u < FW_PL; ++u) {
+        unsigned bal = __ballot_sync(FULL, (slow_u >> u) & 1u);
+        while (bal) {
+            const int src = __ffs(bal) - 1;
+            bal &= bal - 1u;
+            const int c = src + 32 * u;
+            int64_t closed;
+            const int64_t a = warp_avail(f, F.cg[c], &closed);
+            if (lane == 0) {
+                F.av[c] = (int)a;
+                F.avc[c] = (int)closed;
+            }
+        }
+    }
+    __syncwarp();
+
+    // ---- greedy fill: a prefix sum over the ranked candidates ----
+    // lane holds ranks FW_PL*lane .. FW_PL*lane + FW_PL - 1
+    int rc[FW_PL], ra[FW_PL], pre[FW_PL];
+    int lsum = 0;
+#pragma unroll
+    for (int u = 0; u < FW_PL; ++u) {
+        const int r = FW_PL * lane + u;
+        rc[u] = (r < tot) ? F.order[r] : -1;
+        ra[u] = (rc[u] >= 0) ? F.av[rc[u]] : 0;
+        pre[u] = lsum;
+        lsum += ra[u];
+    }
+    int sc = lsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL, sc, o);
+        if (lane >= o) sc += y;
+    }
+    const int total_av = __shfl_sync(FULL, sc, 31);
+    const int lbase = sc - lsum;           // keys available before this lane's ranks
+    // taken: available keys and fewer than R keys before it
+    int n_take = 0;
+    int cut_c = -1;
+#pragma unroll
+    for (int u = 0; u < FW_PL; ++u) {
+        const int A = lbase + pre[u];
+        if (ra[u] > 0 && A < R) {
+            ++n_take;
+            if (A + ra[u] >= R) cut_c = rc[u];
+        }
+    }
+    int tinc = n_take;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL, tinc, o);
+        if (lane >= o) tinc += y;
+    }
+    const int nt = __shfl_sync(FULL, tinc, 31);
+    int t = tinc - n_take;
+#pragma unroll
+    for (int u = 0; u < FW_PL; ++u) {
+        const int A = lbase + pre[u];
+        if (ra[u] > 0 && A < R) {
+            const int c = rc[u];
+            const int g = F.cg[c];
+            const int full = bucket_full(f, g) ? 1 : 0;
+            F.t_g[t] = g;
+            F.t_n[t] = min(ra[u], R - A);
+            F.t_off[t] = A;
+            F.t_o0[t] = offs[g];
+            F.t_closed[t] = F.avc[c];
+            F.t_full[t] = full;
+            F.t_lo[t] = full ? 0 : (int)keys_below_sinks(f, g);
+            ++t;
+        }
+    }
+    // the cut candidate (rank at which the budget is met), if any
+    const unsigned cb = __ballot_sync(FULL, cut_c >= 0);
+    cut_c = cb ? __shfl_sync(FULL, cut_c, __ffs(cb) - 1) : -1;
+    bool exact = true;
+    if (!complete) {
+        const double eps = ldexp((double)l1, -12);
+        if (total_av < R) {
+            int64_t total = f.hi - S + 1;      // keys in [S, pos - W]
+            if (total < 0) total = 0;
+            exact = (int64_t)total_av >= total;
+        } else if (cut_c >= 0) {
+            exact = F.es[cut_c] > (double)tau + eps;
+        }
+    }
+    if (!exact) {
+        to_fallback();
+        return;
+    }
+    __syncwarp();
+
+    int32_t* out = indices + row * (int64_t)s_max;
+    const int64_t n_s = (S < pq + 1) ? S : pq + 1;
+    for (int64_t x = lane; x < n_s; x += 32) out[x] = (int32_t)x;
+    // bucket-major attention lists of the row
+    if (ws.plan.row_n) {
+        const BucketPlan& P = ws.plan;
+        int base = 0;
+        if (lane == 0) {
+            base = atomicAdd(P.ctr + CTR_RESERVED, nt + 1);
+            if ((int64_t)base + nt + 1 > P.ent_cap) {
+                base = -1;
+                P.gather_rows[atomicAdd(P.ctr + CTR_GATHER, 1)] = (int32_t)row;
+            } else {
+                atomicMax(P.ctr + CTR_VALID_END, base + nt + 1);
+                P.ent[base + nt] = make_int4((int)row, -1, 0, 0);   // sinks + window slot
+            }
+            P.row_n[row] = (base < 0) ? -1 : nt;
+            P.row_base[row] = base;
+        }
+        base = __shfl_sync(FULL, base, 0);
+        if (base >= 0) {
+            for (int tt = lane; tt < nt; tt += 32) {
+                const int64_t gg = b * ix.NBK + F.t_g[tt];
+                const int closed = min(F.t_n[tt], F.t_closed[tt]);
+                const int rank = atomicAdd(P.bucket_cnt + gg, 1);
+                P.ent[base + tt] =
+                    make_int4((int)row, (int)gg, F.t_lo[tt], F.t_lo[tt] + closed);
+                P.ent2[base + tt] = make_int2(rank, F.t_n[tt] - closed);
+            }
+        }
+    }
+    // whole buckets, member by member: prefix of their member counts
+    if (lane == 0) {
+        int acc = 0;
+        for (int tt = 0; tt < nt; ++tt) {
+            F.t_mc[tt] = acc;
+            if (F.t_full[tt]) acc += (F.t_n[tt] + p - 1) / p;
+        }
+        F.t_mc[nt] = acc;
+    }
+    __syncwarp();
+    const int n_mem = F.t_mc[nt];
+    int32_t* lr = out + n_s;
+    constexpr int EU = 4;                  // member loads in flight per lane
+    for (int m0 = lane; m0 < n_mem; m0 += 32 * EU) {
+        int tk[EU], mi[EU];
+        int32_t mv[EU];
+#pragma unroll
+        for (int e = 0; e < EU; ++e) {
+            const int m = m0 + 32 * e;
+            tk[e] = -1;
+            if (m < n_mem) {
+                int lo = 0, hi = nt - 1;   // last bucket with t_mc <= m among whole ones
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (F.t_mc[mid] <= m) lo = mid;
+                    else hi = mid - 1;
+                }
+                while (lo + 1 < nt && (!F.t_full[lo] || F.t_mc[lo + 1] <= m)) ++lo;
+                tk[e] = lo;
+                mi[e] = m - F.t_mc[lo];
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < EU; ++e) mv[e] = (tk[e] >= 0) ? __ldg(mem + F.t_o0[tk[e]] + mi[e]) : 0;
+#pragma unroll
+        for (int e = 0; e < EU; ++e) {
+            if (tk[e] < 0) continue;
+            const int tt = tk[e];
+            const int k0 = mi[e] * p;
+            int32_t* dst = lr + F.t_off[tt];
+            const int nk = min(p, F.t_n[tt] - k0);
+            for (int q = 0; q < nk; ++q) dst[k0 + q] = mv[e] * p + q;
+        }
+    }
+    // buckets cut by the window or the sinks, or with open members
+    for (int tt = 0; tt < nt; ++tt)
+        if (!F.t_full[tt]) warp_emit_partial(f, F.t_g[tt], F.t_n[tt], lr + F.t_off[tt]);
+    // recent window, padding, count
+    const int64_t n_lr = nt ? (int64_t)F.t_off[nt - 1] + F.t_n[nt - 1] : 0;
+    const int64_t off = n_s + n_lr;
+    int64_t w0 = pq - W + 1;
+    if (w0 < n_s) w0 = n_s;
+    const int64_t n_w = pq + 1 - w0;
+    for (int64_t x = lane; x < n_w; x += 32) out[off + x] = (int32_t)(w0 + x);
+    for (int64_t x = off + n_w + lane; x < s_max; x += 32) out[x] = -1;
+    if (lane == 0) counts[row] = (int32_t)(off + n_w);
+}
+
+// ---------------------------------------------------------------------------
 // Exact fallback: persistent CTAs walk the list of flagged queries.  Every
 // eligible bucket gets its exact binary64 score; the fill repeatedly takes the
 // best remaining bucket (score desc, lowest id) until the budget is met.
@@ -1283,8 +1633,21 @@ static cudaError_t launch_finish_t(const IndexView& ix, int64_t n_blk, const T* 
     // the compacted open list, when the index has an open block
     const size_t osm = (n_blk > 0 && n_blk * ix.G < ix.NP) ? (size_t)ix.G * 2 * sizeof(int32_t) : 0;
     if (ws.n_lst < 1 || ws.n_lst > FILL_THREADS || ws.lst_cap < 1) return cudaErrorInvalidValue;
-    select_fill_kernel<T><<<grid, FILL_THREADS, osm, st>>>(
-        ix, n_blk, lq, pos, Nq, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
+    const int64_t rows_all = ix.B * Nq;
+    const size_t wsm = (size_t)FW_WARPS * osm;   // one open list per warp
+    if (rows_all >= FW_MIN_ROWS && ws.n_lst <= FW_LISTS && wsm <= FW_DSMEM_MAX) {
+        // many rows: a warp per row
+        const void* kern = (const void*)select_fill_warp_kernel<T>;
+        cudaError_t e = ensure_smem_attr(kern, FW_DSMEM_MAX);
+        if (e != cudaSuccess) return e;
+        select_fill_warp_kernel<T><<<(unsigned)((rows_all + FW_WARPS - 1) / FW_WARPS),
+                                     32 * FW_WARPS, wsm, st>>>(ix, n_blk, lq, pos, Nq, sp.budget,
+                                                               sp.window, sp.sinks, s_max,
+                                                               indices, counts, ws);
+    } else {
+        select_fill_kernel<T><<<grid, FILL_THREADS, osm, st>>>(
+            ix, n_blk, lq, pos, Nq, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
+    }
     note_launch();
     const int64_t rows = ix.B * Nq;
     const unsigned fb_grid = (unsigned)(rows < FB_CTAS ? rows : FB_CTAS);
