@@ -417,19 +417,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
+                    const int64_t gh = (int64_t)t * TC_N + h * 128;   // this thread's 128 columns
+                    if (PASS == 1 && row_valid && gh < nb_row) {
+                        // group maxima of the eligible scores, as fp16 keys
+                        // rounded down (0 = no eligible score in the group)
+                        if (gh + 128 > nb_row) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        float* v = va + 32 * c;
-                        const int64_t g0 = (int64_t)t * TC_N + h * 128 + c * 32;
-                        if (PASS == 1) {
-                            // group maxima of the eligible scores, as fp16 keys
-                            // rounded down (0 = no eligible score in the group)
-                            if (!row_valid || g0 >= nb_row) continue;
-                            if (g0 + 32 > nb_row) {
+                            for (int j = 0; j < 128; ++j)
+                                if (gh + j >= nb_row) va[j] = -INFINITY;
+                        }
+                        auto key = [](float x) -> uint32_t {
+                            return x > -INFINITY ? tc_half_key(__float2half_rd(x)) : 0u;
+                        };
+                        float m32[4];
 #pragma unroll
-                                for (int j = 0; j < 32; ++j)
-                                    if (g0 + j >= nb_row) v[j] = -INFINITY;
-                            }
+                        for (int c = 0; c < 4; ++c) {
+                            const float* v = va + 32 * c;
                             float m16[16], m8[8], m4[4], m2[2];
 #pragma unroll
                             for (int j = 0; j < 16; ++j) m16[j] = fmaxf(v[2 * j], v[2 * j + 1]);
@@ -439,26 +442,40 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
                             for (int j = 0; j < 4; ++j) m4[j] = fmaxf(m8[2 * j], m8[2 * j + 1]);
 #pragma unroll
                             for (int j = 0; j < 2; ++j) m2[j] = fmaxf(m4[2 * j], m4[2 * j + 1]);
-                            auto key = [](float x) -> uint32_t {
-                                return x > -INFINITY ? tc_half_key(__float2half_rd(x)) : 0u;
-                            };
-                            if (gl == 5) {
-                                grow[g0 >> 5] = (uint16_t)key(fmaxf(m2[0], m2[1]));
-                            } else if (gl == 4) {
+                            m32[c] = fmaxf(m2[0], m2[1]);
+                            const int64_t g0 = gh + 32 * c;
+                            if (gl == 4) {
                                 *reinterpret_cast<uint32_t*>(grow + (g0 >> 4)) =
                                     key(m2[0]) | (key(m2[1]) << 16);
                             } else if (gl == 3) {
                                 *reinterpret_cast<uint2*>(grow + (g0 >> 3)) =
                                     make_uint2(key(m4[0]) | (key(m4[1]) << 16),
                                                key(m4[2]) | (key(m4[3]) << 16));
-                            } else {
-                                uint4* dst = reinterpret_cast<uint4*>(grow + (g0 >> 2));
-                                dst[0] = make_uint4(key(m8[0]) | (key(m8[1]) << 16),
-                                                    key(m8[2]) | (key(m8[3]) << 16),
-                                                    key(m8[4]) | (key(m8[5]) << 16),
-                                                    key(m8[6]) | (key(m8[7]) << 16));
+                            } else if (gl == 2) {
+                                *reinterpret_cast<uint4*>(grow + (g0 >> 2)) =
+                                    make_uint4(key(m8[0]) | (key(m8[1]) << 16),
+                                               key(m8[2]) | (key(m8[3]) << 16),
+                                               key(m8[4]) | (key(m8[5]) << 16),
+                                               key(m8[6]) | (key(m8[7]) << 16));
                             }
-                        } else {
+                        }
+                        if (gl == 5) {
+                            *reinterpret_cast<uint2*>(grow + (gh >> 5)) =
+                                make_uint2(key(m32[0]) | (key(m32[1]) << 16),
+                                           key(m32[2]) | (key(m32[3]) << 16));
+                        } else if (gl == 6) {
+                            *reinterpret_cast<uint32_t*>(grow + (gh >> 6)) =
+                                key(fmaxf(m32[0], m32[1])) | (key(fmaxf(m32[2], m32[3])) << 16);
+                        } else if (gl == 7) {
+                            grow[gh >> 7] =
+                                (uint16_t)key(fmaxf(fmaxf(m32[0], m32[1]), fmaxf(m32[2], m32[3])));
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4 && PASS == 2; ++c) {
+                        float* v = va + 32 * c;
+                        const int64_t g0 = gh + c * 32;
+                        {
                             // append every eligible score >= theta
                             uint32_t vm = 0u;
                             if (g0 + 32 <= nb_row) vm = 0xFFFFFFFFu;
@@ -542,11 +559,12 @@ __global__ void __launch_bounds__(256) score_theta_kernel(IndexView ix, int64_t 
         // of 8; keys past ng count as 0)
         uint32_t kw[TH_REG / 2];
         const uint4* k4 = reinterpret_cast<const uint4*>(keys);
+        const int n_u = (int)((ng + 255) / 256);              // 16-byte chunks per lane in use
 #pragma unroll
         for (int u = 0; u < TH_REG / 8; ++u) {
             const int64_t c = (int64_t)u * 32 + lane;        // 16-byte chunk
             uint4 w = make_uint4(0u, 0u, 0u, 0u);
-            if (c * 8 < ng) w = k4[c];
+            if (u < n_u && c * 8 < ng) w = k4[c];
             const uint32_t e[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -561,8 +579,12 @@ __global__ void __launch_bounds__(256) score_theta_kernel(IndexView ix, int64_t 
             const uint32_t mid = (lo + hi + 1u) >> 1;
             int cnt = 0;
 #pragma unroll
-            for (int u = 0; u < TH_REG / 2; ++u)
-                cnt += (int)((kw[u] & 0xFFFFu) >= mid) + (int)((kw[u] >> 16) >= mid);
+            for (int u = 0; u < TH_REG / 8; ++u) {
+                if (u >= n_u) break;                          // warp-uniform
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    cnt += (int)((kw[4 * u + q] & 0xFFFFu) >= mid) + (int)((kw[4 * u + q] >> 16) >= mid);
+            }
             cnt = __reduce_add_sync(0xffffffffu, cnt);
             if (cnt >= m) lo = mid;
             else hi = mid - 1u;
@@ -609,14 +631,15 @@ TcSplit tc_split_plan(const IndexView& ix, int64_t Nq)
     sp.n_split = (int)((n_ct + sp.tps - 1) / sp.tps);
     if (sp.n_split < 1) sp.n_split = 1;
     sp.n_items = tiles * sp.n_split;
-    // groups of 32 scores, narrower (down to 4) while a sequence has fewer than
-    // 4m groups: with g groups and the m-th largest maximum as the threshold,
-    // scores without structure put about -g ln(1 - m/g) of them above it
+    // groups of 128 scores (one per epilogue thread and tile), narrower (down
+    // to 4) while a sequence has fewer than 4m groups: with g groups and the
+    // m-th largest maximum as the threshold, scores without structure put
+    // about -g ln(1 - m/g) ~ m (1 + m / 2g) of them above it
     sp.m = TC_TARGET;
-    int gl = 5;
+    int gl = 7;
     while (gl > 2 && (ix.NBK >> gl) < 4LL * sp.m) --gl;
     sp.gw_log2 = gl;
-    sp.n_grp = (n_ct * TC_N) >> gl;
+    sp.n_grp = (((n_ct * TC_N) >> gl) + 7) / 8 * 8;   // rows of keys start on 16 bytes
     return sp;
 }
 
