@@ -56,7 +56,8 @@ constexpr int TC_M = 128;
 constexpr int TC_N = 256;                                 // centroids per tile
 constexpr int TC_TMEM_COLS = 2 * TC_N;                    // two fp32 accumulators
 constexpr int TC_STAGES = 4;
-constexpr int TC_EPI_WARPS = 8;
+constexpr int TC_EPI_WARPS = 16;                          // 4 per TMEM lane quarter
+constexpr int TC_COLS = TC_N / 4;                         // columns of a tile per epilogue thread
 constexpr int TC_EPI_THREADS = 32 * TC_EPI_WARPS;
 constexpr int TC_THREADS = 64 + TC_EPI_THREADS;           // producer, MMA, epilogue
 constexpr uint32_t TC_WAIT = 1u << 22;
@@ -69,9 +70,7 @@ __device__ uint32_t g_tc_wait = TC_WAIT;
 constexpr int TC_Q_BYTES = TC_M * DL * 2;                 // 16 KB per query buffer
 constexpr int TC_C_BYTES = TC_N * DL * 2;                 // 32 KB per ring stage
 constexpr int TC_OFF_C = 2 * TC_Q_BYTES;
-constexpr int TC_OFF_G = TC_OFF_C + TC_STAGES * TC_C_BYTES;
-constexpr int TC_G_BYTES = TC_EPI_THREADS * 32 * 4;      // pass-2 staging of 32 scores
-constexpr int TC_OFF_BAR = TC_OFF_G + TC_G_BYTES;
+constexpr int TC_OFF_BAR = TC_OFF_C + TC_STAGES * TC_C_BYTES;
 constexpr int TC_NBAR = 2 + 2 + 2 * TC_STAGES + 2 + 2 + 1;
 constexpr int TC_OFF_MISC = TC_OFF_BAR + TC_NBAR * 8;
 constexpr int TC_MISC_BYTES = TC_M * 4 + TC_EPI_THREADS * 4 + 64;
@@ -166,6 +165,40 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v)
     for (int j = 0; j < 128; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+// Two 32-column loads in flight, one wait: 64 consecutive columns of this
+// thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v)
+{
+    uint32_t r[64];
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+            "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+            "%28, %29, %30, %31}, [%32];"
+            : "=r"(r[32 * q + 0]), "=r"(r[32 * q + 1]), "=r"(r[32 * q + 2]), "=r"(r[32 * q + 3]),
+              "=r"(r[32 * q + 4]), "=r"(r[32 * q + 5]), "=r"(r[32 * q + 6]), "=r"(r[32 * q + 7]),
+              "=r"(r[32 * q + 8]), "=r"(r[32 * q + 9]), "=r"(r[32 * q + 10]), "=r"(r[32 * q + 11]),
+              "=r"(r[32 * q + 12]), "=r"(r[32 * q + 13]), "=r"(r[32 * q + 14]), "=r"(r[32 * q + 15]),
+              "=r"(r[32 * q + 16]), "=r"(r[32 * q + 17]), "=r"(r[32 * q + 18]), "=r"(r[32 * q + 19]),
+              "=r"(r[32 * q + 20]), "=r"(r[32 * q + 21]), "=r"(r[32 * q + 22]), "=r"(r[32 * q + 23]),
+              "=r"(r[32 * q + 24]), "=r"(r[32 * q + 25]), "=r"(r[32 * q + 26]), "=r"(r[32 * q + 27]),
+              "=r"(r[32 * q + 28]), "=r"(r[32 * q + 29]), "=r"(r[32 * q + 30]), "=r"(r[32 * q + 31])
+            : "r"(taddr + 32u * q));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 64; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// One of 8 values by a 3-bit index (selects, no indexed registers).
+__device__ __forceinline__ float pick8(const float* v, int e)
+{
+    const float a = (e & 1) ? v[1] : v[0], b = (e & 1) ? v[3] : v[2];
+    const float c = (e & 1) ? v[5] : v[4], d = (e & 1) ? v[7] : v[6];
+    const float ab = (e & 2) ? b : a, cd = (e & 2) ? d : c;
+    return (e & 4) ? cd : ab;
+}
+
 // Named barrier of the epilogue warps only.
 __device__ __forceinline__ void epi_sync()
 {
@@ -239,7 +272,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
         (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);  // 1 KB aligned
     unsigned char* q_s = smem;                        // [2][TC_Q_BYTES]
     unsigned char* c_s = smem + TC_OFF_C;             // [TC_STAGES][TC_C_BYTES]
-    float* stage = reinterpret_cast<float*>(smem + TC_OFF_G);      // [TC_EPI_THREADS][32]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TC_OFF_BAR);
     uint64_t* q_full = bars;                  // [2]
     uint64_t* q_empty = bars + 2;             // [2]
@@ -380,12 +412,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
         __syncwarp();
     } else {
         // ---------------- epilogue ----------------
-        const int et = threadIdx.x - 64;                  // 0 .. 255
-        const int h = (warp - 2) >> 2;                    // half of every tile's columns
+        const int et = threadIdx.x - 64;                  // 0 .. TC_EPI_THREADS - 1
+        const int sl = (warp - 2) >> 2;                   // column slice of every tile
         const int r = 32 * (warp & 3) + lane;             // query row = TMEM lane
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-        float* my_stage = stage + et * 32;
-        const int gl = sp.gw_log2;                        // 2 .. 5
+        const int gl = sp.gw_log2;                        // 2 .. 6
+        const unsigned FULL = 0xffffffffu;
         int64_t gt = 0;
         for (int64_t it = blockIdx.x; it < sp.n_items; it += gridDim.x) {
             const TcItem I = tc_item(it, ix, n_blk, pos, Nq, W, sp);
@@ -395,7 +427,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
                 row_valid ? tc_eligible(ix, n_blk, pos.at(I.b, Nq, I.q0 + r), W) : 0;
             const int64_t lslot = row * sp.n_split + I.s;
             if (I.t1 <= I.t0) {
-                if (PASS == 2 && h == 0 && row_valid) {
+                if (PASS == 2 && sl == 0 && row_valid) {
                     ws.lst_n[lslot] = 0;
                     ws.lst_tau[lslot] = -INFINITY;
                 }
@@ -404,34 +436,34 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
             const float theta = (PASS == 2 && row_valid) ? ws.theta[row] : -INFINITY;
             uint16_t* grow = ws.gmax + row * ws.n_grp;
             float lost = -INFINITY;
-            const bool go = __all_sync(0xffffffffu, *abort_flag == 0);   // warp-uniform
+            const bool go = __all_sync(FULL, *abort_flag == 0);   // warp-uniform
             for (int t = I.t0; t < I.t1; ++t, ++gt) {
                 const int buf = (int)(gt & 1);
                 const bool ok = go && waitw(&acc_full[buf], (uint32_t)((gt >> 1) & 1), 4000u);
                 if (ok) {
                     tc_fence_after();
-                    float va[128];
+                    float va[TC_COLS];
                     __syncwarp();
-                    tmem_ld128(tmem + lane_base + (uint32_t)(buf * TC_N + h * 128), va);
+                    tmem_ld64(tmem + lane_base + (uint32_t)(buf * TC_N + sl * TC_COLS), va);
                     // the accumulator is in registers: hand it back before the work
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
-                    const int64_t gh = (int64_t)t * TC_N + h * 128;   // this thread's 128 columns
+                    const int64_t gh = (int64_t)t * TC_N + sl * TC_COLS;   // first column here
                     if (PASS == 1 && row_valid && gh < nb_row) {
                         // group maxima of the eligible scores, as fp16 keys
                         // rounded down (0 = no eligible score in the group)
-                        if (gh + 128 > nb_row) {
+                        if (gh + TC_COLS > nb_row) {
 #pragma unroll
-                            for (int j = 0; j < 128; ++j)
+                            for (int j = 0; j < TC_COLS; ++j)
                                 if (gh + j >= nb_row) va[j] = -INFINITY;
                         }
                         auto key = [](float x) -> uint32_t {
                             return x > -INFINITY ? tc_half_key(__float2half_rd(x)) : 0u;
                         };
-                        float m32[4];
+                        float m32[2];
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
+                        for (int c = 0; c < 2; ++c) {
                             const float* v = va + 32 * c;
                             float m16[16], m8[8], m4[4], m2[2];
 #pragma unroll
@@ -459,47 +491,44 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
                                                key(m8[6]) | (key(m8[7]) << 16));
                             }
                         }
-                        if (gl == 5) {
-                            *reinterpret_cast<uint2*>(grow + (gh >> 5)) =
-                                make_uint2(key(m32[0]) | (key(m32[1]) << 16),
-                                           key(m32[2]) | (key(m32[3]) << 16));
-                        } else if (gl == 6) {
-                            *reinterpret_cast<uint32_t*>(grow + (gh >> 6)) =
-                                key(fmaxf(m32[0], m32[1])) | (key(fmaxf(m32[2], m32[3])) << 16);
-                        } else if (gl == 7) {
-                            grow[gh >> 7] =
-                                (uint16_t)key(fmaxf(fmaxf(m32[0], m32[1]), fmaxf(m32[2], m32[3])));
-                        }
+                        if (gl == 5)
+                            *reinterpret_cast<uint32_t*>(grow + (gh >> 5)) =
+                                key(m32[0]) | (key(m32[1]) << 16);
+                        else if (gl == 6)
+                            grow[gh >> 6] = (uint16_t)key(fmaxf(m32[0], m32[1]));
                     }
+                    if (PASS == 2) {
+                        // append every eligible score >= theta: 8-score
+                        // sub-batches that no row of the warp can reach are
+                        // skipped after one warp vote
+                        uint64_t vm = 0ull;              // eligible columns of the 64
+                        if (gh + TC_COLS <= nb_row) vm = ~0ull;
+                        else if (gh < nb_row) vm = (1ull << (uint32_t)(nb_row - gh)) - 1ull;
+                        float m16[32], m8[16];
 #pragma unroll
-                    for (int c = 0; c < 4 && PASS == 2; ++c) {
-                        float* v = va + 32 * c;
-                        const int64_t g0 = gh + c * 32;
-                        {
-                            // append every eligible score >= theta
-                            uint32_t vm = 0u;
-                            if (g0 + 32 <= nb_row) vm = 0xFFFFFFFFu;
-                            else if (g0 < nb_row) vm = (1u << (uint32_t)(nb_row - g0)) - 1u;
-                            uint32_t msk = 0u;
+                        for (int j = 0; j < 32; ++j) m16[j] = fmaxf(va[2 * j], va[2 * j + 1]);
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) msk |= (v[j] >= theta) ? (1u << j) : 0u;
-                            msk &= vm;
-                            if (__any_sync(0xffffffffu, msk != 0u)) {
-                                if (msk) {
-                                    float4* st4 = reinterpret_cast<float4*>(my_stage);
+                        for (int j = 0; j < 16; ++j) m8[j] = fmaxf(m16[2 * j], m16[2 * j + 1]);
 #pragma unroll
-                                    for (int j = 0; j < 8; ++j)
-                                        st4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2],
-                                                             v[4 * j + 3]);
+                        for (int q = 0; q < 8; ++q) {
+                            const float* v = va + 8 * q;
+                            const uint32_t em = (uint32_t)(vm >> (8 * q)) & 0xFFu;
+                            const bool act = em != 0u && fmaxf(m8[2 * q], m8[2 * q + 1]) >= theta;
+                            if (__any_sync(FULL, act)) {
+                                uint32_t bits = 0u;
+                                if (act) {
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) bits |= (v[e] >= theta) ? (1u << e) : 0u;
+                                    bits &= em;
                                 }
-                                while (msk) {
-                                    const int j = __ffs(msk) - 1;
-                                    msk &= msk - 1u;
+                                while (bits) {
+                                    const int e = __ffs(bits) - 1;
+                                    bits &= bits - 1u;
                                     const int slot = atomicAdd(&rcnt[r], 1);
                                     if (slot < ws.lst_cap)
-                                        ws.lst_g[lslot * ws.lst_cap + slot] = (int32_t)(g0 + j);
+                                        ws.lst_g[lslot * ws.lst_cap + slot] = (int32_t)(gh + 8 * q + e);
                                     else
-                                        lost = fmaxf(lost, my_stage[j]);
+                                        lost = fmaxf(lost, pick8(v, e));
                                 }
                             }
                         }
@@ -510,9 +539,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
             if (PASS == 2) {
                 lostv[et] = lost;
                 epi_sync();
-                if (h == 0) {
+                if (sl == 0) {
                     if (row_valid) {
-                        const float l2 = fmaxf(lost, lostv[et + 128]);   // the other half's thread
+                        // the row's four threads (one per column slice)
+                        const float l2 = fmaxf(fmaxf(lost, lostv[et + 128]),
+                                               fmaxf(lostv[et + 256], lostv[et + 384]));
                         ws.lst_n[lslot] = min(rcnt[r], ws.lst_cap);
                         ws.lst_tau[lslot] = (theta > -INFINITY) ? fmaxf(theta, l2) : l2;
                     }
@@ -631,12 +662,12 @@ TcSplit tc_split_plan(const IndexView& ix, int64_t Nq)
     sp.n_split = (int)((n_ct + sp.tps - 1) / sp.tps);
     if (sp.n_split < 1) sp.n_split = 1;
     sp.n_items = tiles * sp.n_split;
-    // groups of 128 scores (one per epilogue thread and tile), narrower (down
+    // groups of 64 scores (one per epilogue thread and tile), narrower (down
     // to 4) while a sequence has fewer than 4m groups: with g groups and the
     // m-th largest maximum as the threshold, scores without structure put
     // about -g ln(1 - m/g) ~ m (1 + m / 2g) of them above it
     sp.m = TC_TARGET;
-    int gl = 7;
+    int gl = 6;
     while (gl > 2 && (ix.NBK >> gl) < 4LL * sp.m) --gl;
     sp.gw_log2 = gl;
     sp.n_grp = (((n_ct * TC_N) >> gl) + 7) / 8 * 8;   // rows of keys start on 16 bytes
