@@ -563,18 +563,63 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
 }
 
 constexpr int TH_REG = 64;   // group-maximum keys per lane held in registers (2048 per row)
+constexpr int TH_WARPS = 8;
 
-// theta of every query row: a warp per row finds the m-th largest of the
-// row's group maxima by bisection over the 16-bit keys.  A row with at most
-// KCF eligible buckets gets -inf (its lists take every eligible bucket); a row
-// with fewer than 2m groups uses half of them.
-__global__ void __launch_bounds__(256) score_theta_kernel(IndexView ix, int64_t n_blk, PosSrc pos,
-                                                          int64_t Nq, int W, SelectWs ws,
-                                                          TcSplit sp)
+// The bin (0 .. 255) holding the want-th largest count-weighted entry of a
+// warp's 256-bin histogram, bins counted from the top; *above receives the
+// entries in higher bins.  Lane l reads bins 255-8l .. 248-8l.
+__device__ __forceinline__ int th_bin(const unsigned* hist, int want, int* above)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (row >= ix.B * Nq) return;                 // warp-uniform
+    unsigned hb[8], tot = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        hb[e] = hist[255 - 8 * lane - e];
+        tot += hb[e];
+    }
+    unsigned incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const unsigned excl = incl - tot;
+    int bin = -1, abv = 0;
+    if (excl < (unsigned)want && incl >= (unsigned)want) {
+        unsigned cum = excl;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (bin < 0 && cum + hb[e] >= (unsigned)want) {
+                bin = 255 - 8 * lane - e;
+                abv = (int)cum;
+            }
+            cum += hb[e];
+        }
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, bin >= 0);
+    if (!who) {                 // fewer than want entries (not reached: callers check)
+        *above = 0;
+        return -1;
+    }
+    const int src = __ffs(who) - 1;
+    *above = __shfl_sync(0xffffffffu, abv, src);
+    return __shfl_sync(0xffffffffu, bin, src);
+}
+
+// theta of every query row: a warp per row finds the m-th largest of the
+// row's group maxima (16-bit keys) by a two-pass radix select, high byte then
+// low byte, over keys held in registers.  A row with at most KCF eligible
+// buckets gets -inf (its lists take every eligible bucket); a row with fewer
+// than 2m groups uses half of them.
+__global__ void __launch_bounds__(32 * TH_WARPS) score_theta_kernel(IndexView ix, int64_t n_blk,
+                                                                    PosSrc pos, int64_t Nq,
+                                                                    int W, SelectWs ws, TcSplit sp)
+{
+    __shared__ unsigned hist_s[TH_WARPS][256];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * TH_WARPS + warp;
+    if (row >= ix.B * Nq) return;                 // warp-uniform; no CTA barrier here
+    unsigned* hist = hist_s[warp];
     const int64_t b = row / Nq, i = row % Nq;
     const int64_t nb = tc_eligible(ix, n_blk, pos.at(b, Nq, i), W);
     if (nb <= KCF) {
@@ -584,10 +629,10 @@ __global__ void __launch_bounds__(256) score_theta_kernel(IndexView ix, int64_t 
     const int64_t ng = (nb + (1 << sp.gw_log2) - 1) >> sp.gw_log2;
     const int m = (int)min((int64_t)sp.m, max((int64_t)1, ng / 2));
     const uint16_t* keys = ws.gmax + row * ws.n_grp;
-    uint32_t lo = 1u, hi = 0xFFFFu;               // count(key >= lo) >= m
+    uint32_t th;
     if (ng <= 32 * TH_REG) {
-        // the row's keys in registers, 8 per 16-byte load (n_grp is a multiple
-        // of 8; keys past ng count as 0)
+        // keys in registers, 8 per 16-byte load (n_grp is a multiple of 8;
+        // keys past ng count as 0, which no bin below 1 holds)
         uint32_t kw[TH_REG / 2];
         const uint4* k4 = reinterpret_cast<const uint4*>(keys);
         const int n_u = (int)((ng + 255) / 256);              // 16-byte chunks per lane in use
@@ -606,21 +651,43 @@ __global__ void __launch_bounds__(256) score_theta_kernel(IndexView ix, int64_t 
                 kw[u * 4 + q] = x;
             }
         }
-        while (lo < hi) {
-            const uint32_t mid = (lo + hi + 1u) >> 1;
-            int cnt = 0;
+        // high byte
 #pragma unroll
-            for (int u = 0; u < TH_REG / 8; ++u) {
-                if (u >= n_u) break;                          // warp-uniform
+        for (int e = 0; e < 8; ++e) hist[8 * lane + e] = 0u;
+        __syncwarp();
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    cnt += (int)((kw[4 * u + q] & 0xFFFFu) >= mid) + (int)((kw[4 * u + q] >> 16) >= mid);
+        for (int u = 0; u < TH_REG / 8; ++u) {
+            if (u >= n_u) break;                              // warp-uniform
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t k = (q & 1) ? (kw[4 * u + q / 2] >> 16) : (kw[4 * u + q / 2] & 0xFFFFu);
+                if (k) atomicAdd(&hist[k >> 8], 1u);
             }
-            cnt = __reduce_add_sync(0xffffffffu, cnt);
-            if (cnt >= m) lo = mid;
-            else hi = mid - 1u;
         }
+        __syncwarp();
+        int above;
+        const int b1 = th_bin(hist, m, &above);
+        const int m2 = m - above;
+        // low byte among the keys of that high byte
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) hist[8 * lane + e] = 0u;
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < TH_REG / 8; ++u) {
+            if (u >= n_u) break;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t k = (q & 1) ? (kw[4 * u + q / 2] >> 16) : (kw[4 * u + q / 2] & 0xFFFFu);
+                if (k && (int)(k >> 8) == b1) atomicAdd(&hist[k & 255u], 1u);
+            }
+        }
+        __syncwarp();
+        int above2;
+        const int b2 = (b1 >= 0) ? th_bin(hist, m2, &above2) : -1;
+        th = (b1 >= 0 && b2 >= 0) ? (((uint32_t)b1 << 8) | (uint32_t)b2) : 0u;
     } else {
+        uint32_t lo = 1u, hi = 0xFFFFu;               // count(key >= lo) >= m
         while (lo < hi) {
             const uint32_t mid = (lo + hi + 1u) >> 1;
             int cnt = 0;
@@ -629,8 +696,10 @@ __global__ void __launch_bounds__(256) score_theta_kernel(IndexView ix, int64_t 
             if (cnt >= m) lo = mid;
             else hi = mid - 1u;
         }
+        th = lo;
     }
-    if (lane == 0) ws.theta[row] = tc_key_value(lo);
+    // key 0 marks no threshold found: every eligible bucket is listed
+    if (lane == 0) ws.theta[row] = th ? tc_key_value(th) : -INFINITY;
 }
 
 // ---- host side ---------------------------------------------------------------
@@ -700,7 +769,8 @@ cudaError_t launch_score_lists_tc(const IndexView& ix, int64_t n_blk, const void
     score_tc_kernel<1><<<n_cta, TC_THREADS, TC_SMEM, st>>>(tmQ, tmC, ix, n_blk, pos, Nq, W, ws, sp);
     note_launch();
     const int64_t rows = ix.B * Nq;
-    score_theta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(ix, n_blk, pos, Nq, W, ws, sp);
+    score_theta_kernel<<<(unsigned)((rows + TH_WARPS - 1) / TH_WARPS), 32 * TH_WARPS, 0, st>>>(
+        ix, n_blk, pos, Nq, W, ws, sp);
     note_launch();
     score_tc_kernel<2><<<n_cta, TC_THREADS, TC_SMEM, st>>>(tmQ, tmC, ix, n_blk, pos, Nq, W, ws, sp);
     note_launch();
