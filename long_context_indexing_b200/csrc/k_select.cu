@@ -839,7 +839,6 @@ constexpr int FW_PL = KCF / 32;        // candidates per lane
 struct FwRow {
     float q[DL];
     double es[KCF];
-    uint64_t ek[KCF];     // ordered key of es
     int cg[KCF];
     int av[KCF];          // available keys of candidate c
     int avc[KCF];         // its closed part
@@ -924,31 +923,20 @@ __global__ void __launch_bounds__(32 * FW_WARPS) select_fill_warp_kernel(
     float l1 = fabsf(F.q[lane]) + fabsf(F.q[lane + 32]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) l1 += __shfl_xor_sync(FULL, l1, o);
-    // rank keys: the exact score as an ordered 64-bit integer (+0 for both
-    // zeros, so that equal scores tie as in binary64), then the bucket id
 #pragma unroll
     for (int u = 0; u < FW_PL; ++u) {
         const int c = lane + 32 * u;
-        if (c < tot) {
-            double e = exact_score(ix, b, F.cg[c], F.q);
-            if (e == 0.0) e = 0.0;
-            F.es[c] = e;
-            const uint64_t x = (uint64_t)__double_as_longlong(e);
-            F.ek[c] = (x >> 63) ? ~x : (x | 0x8000000000000000ull);
-        }
+        if (c < tot) F.es[c] = exact_score(ix, b, F.cg[c], F.q);
     }
     __syncwarp();
 #pragma unroll
     for (int u = 0; u < FW_PL; ++u) {
         const int c = lane + 32 * u;
         if (c < tot) {
-            const uint64_t k = F.ek[c];
+            const double e = F.es[c];
             const int g = F.cg[c];
             int r = 0;
-            for (int c2 = 0; c2 < tot; ++c2) {
-                const uint64_t k2 = F.ek[c2];
-                r += (k2 > k) || (k2 == k && F.cg[c2] < g);
-            }
+            for (int c2 = 0; c2 < tot; ++c2) r += rank_before(F.es[c2], F.cg[c2], e, g);
             F.order[r] = c;
         }
     }
