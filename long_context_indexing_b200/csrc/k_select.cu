@@ -197,25 +197,17 @@ __device__ __forceinline__ double exact_score(const IndexView& ix, int64_t bseq,
     return s;
 }
 
-// Body of the SIMT nominator for query `row` at position pq; q_s holds the
-// latent query (every thread of the CTA calls it; sc holds n_blk*k floats).
-__device__ void simt_nominate(const IndexView& ix, int64_t n_blk, const float* q_s, int64_t bseq,
-                              int64_t row, int64_t pq, int W, const SelectWs& ws, float* sc)
+// The KC largest of the nb > KC approximate scores sc[0 .. nb) (shared
+// memory), by an MSB-first radix select of the KC-th largest (4 passes of 8
+// bits over ordered keys): every bucket above that score plus enough of those
+// equal to it, written to cand[0 .. KC) (any memory).  Returns tau = that
+// score, which bounds every bucket left out.  Called by every thread of the
+// CTA.
+__device__ float radix_top_kc(const float* sc, int64_t nb, int32_t* cand)
 {
     __shared__ unsigned hist[256];
     __shared__ uint32_t sh_prefix, sh_want;
     __shared__ int sh_gt, sh_eq;
-    const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
-    int32_t* cand = ws.lst_g + row * KC;      // one list of KC per row
-    if (nb <= KC) {
-        for (int x = threadIdx.x; x < KC; x += blockDim.x) cand[x] = (x < nb) ? x : -1;
-        if (threadIdx.x == 0) {
-            ws.lst_n[row] = (int32_t)nb;
-            ws.lst_tau[row] = -INFINITY;
-        }
-        return;
-    }
-    approx_scores(ix, q_s, bseq, nb, sc);
     if (threadIdx.x == 0) {
         sh_prefix = 0;
         sh_want = KC;
@@ -281,9 +273,31 @@ __device__ void simt_nominate(const IndexView& ix, int64_t n_blk, const float* q
             if (s < need_eq) cand[KC - need_eq + s] = (int32_t)g;
         }
     }
+    __syncthreads();
+    return key_to_float(thr);
+}
+
+// Body of the SIMT nominator for query `row` at position pq; q_s holds the
+// latent query (every thread of the CTA calls it; sc holds n_blk*k floats).
+__device__ void simt_nominate(const IndexView& ix, int64_t n_blk, const float* q_s, int64_t bseq,
+                              int64_t row, int64_t pq, int W, const SelectWs& ws, float* sc)
+{
+    const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
+    int32_t* cand = ws.lst_g + row * KC;      // one list of KC per row
+    if (nb <= KC) {
+        for (int x = threadIdx.x; x < KC; x += blockDim.x) cand[x] = (x < nb) ? x : -1;
+        if (threadIdx.x == 0) {
+            ws.lst_n[row] = (int32_t)nb;
+            ws.lst_tau[row] = -INFINITY;
+        }
+        return;
+    }
+    approx_scores(ix, q_s, bseq, nb, sc);
+    __syncthreads();
+    const float tau = radix_top_kc(sc, nb, cand);
     if (threadIdx.x == 0) {
         ws.lst_n[row] = KC;
-        ws.lst_tau[row] = key_to_float(thr);
+        ws.lst_tau[row] = tau;
     }
 }
 
@@ -558,6 +572,7 @@ __device__ void cta_emit_tail(int64_t pq, int W, int64_t n_s, int64_t off, int s
 
 constexpr int FILL_THREADS = 128;
 static_assert(FILL_THREADS == KCF, "one candidate per fill thread");
+constexpr int ROW_SC_SMEM = 160 * 1024;   // decode score rows up to 40960 buckets in shared memory
 
 // ---------------------------------------------------------------------------
 // Exact ranking + greedy fill + emission.  One CTA (128 threads) per query.
@@ -611,6 +626,35 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
         }
     }
     load_query(q_s, lq, row);
+    if (ws.row_sc) {
+        // decode: the row's scores of every eligible bucket; the KC largest
+        // (radix select, from shared memory when the row fits) are the candidates
+        const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
+        if (nb <= KC) {
+            if ((int)threadIdx.x < KCF) cg[threadIdx.x] = ((int64_t)threadIdx.x < nb) ? (int)threadIdx.x : -1;
+            if (threadIdx.x == 0) {
+                sh_nc = (int)nb;
+                sh_tau = -INFINITY;
+                sh_complete = 1;
+            }
+        } else {
+            const float* src = ws.row_sc + row * ws.row_ld;
+            const float* sc = src;
+            if (ws.row_ld * 4 <= ROW_SC_SMEM) {
+                float* sm = reinterpret_cast<float*>(open_sm + 2 * ix.G);
+                for (int64_t g = threadIdx.x; g < nb; g += blockDim.x) sm[g] = src[g];
+                __syncthreads();
+                sc = sm;
+            }
+            const float t = radix_top_kc(sc, nb, cg);
+            if (threadIdx.x == 0) {
+                sh_nc = KC;
+                sh_tau = t;
+                sh_complete = 0;
+            }
+        }
+        __syncthreads();
+    } else {
     // The row's candidate lists (n_lst <= FILL_THREADS): counts and bounds in
     // parallel, their offsets by one thread, then the bucket ids.  tau bounds
     // every eligible bucket left out of the lists; with every list complete
@@ -659,6 +703,7 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
             cg[threadIdx.x] =
                 ws.lst_g[(row * nl + l) * ws.lst_cap + ((int)threadIdx.x - lst_off[l])];
         }
+    }
     }
     const int nc = sh_nc;
     const float tau = sh_tau;
@@ -1376,27 +1421,9 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_prep_kernel(
                 }
             }
             __syncthreads();
-            // this slice's candidate list: the m largest scores (ties to the
-            // lower bucket), each at its rank; tau = the next score
-            const int m = ws.lst_cap;
-            int32_t* lg = ws.lst_g + ((int64_t)b * ws.n_lst + sl) * m;
-            for (int t = threadIdx.x; t < n; t += DEC_THREADS) {
-                const float x = sc[t];
-                int rank = 0;
-                for (int u = 0; u < n; ++u) {
-                    const float y = sc[u];
-                    rank += (y > x) || (y == x && u < t);
-                }
-                if (rank < m) lg[rank] = (int32_t)(g0 + t);
-                else if (rank == m) ws.lst_tau[b * ws.n_lst + sl] = x;
-            }
-            if (threadIdx.x == 0) {
-                ws.lst_n[b * ws.n_lst + sl] = min(n, m);
-                if (n <= m) ws.lst_tau[b * ws.n_lst + sl] = -INFINITY;
-            }
-        } else if (threadIdx.x == 0) {
-            ws.lst_n[b * ws.n_lst + sl] = 0;
-            ws.lst_tau[b * ws.n_lst + sl] = -INFINITY;
+            // this slice's scores join the sequence's score row
+            float* dst = const_cast<float*>(ws.row_sc) + b * ws.row_ld + g0;
+            for (int t = threadIdx.x; t < n; t += DEC_THREADS) dst[t] = sc[t];
         }
     }
 
@@ -1603,6 +1630,8 @@ SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
     p += al256(4);
     w.fb_scores = (double*)p;
     p += al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
+    w.row_sc = nullptr;
+    w.row_ld = 0;
     w.n_grp = n_grp_of(ix, Nq);
     w.gmax = nullptr;
     w.theta = nullptr;
@@ -1635,7 +1664,7 @@ static cudaError_t launch_finish_t(const IndexView& ix, int64_t n_blk, const T* 
     if (ws.n_lst < 1 || ws.n_lst > FILL_THREADS || ws.lst_cap < 1) return cudaErrorInvalidValue;
     const int64_t rows_all = ix.B * Nq;
     const size_t wsm = (size_t)FW_WARPS * osm;   // one open list per warp
-    if (rows_all >= FW_MIN_ROWS && ws.n_lst <= FW_LISTS && wsm <= FW_DSMEM_MAX) {
+    if (!ws.row_sc && rows_all >= FW_MIN_ROWS && ws.n_lst <= FW_LISTS && wsm <= FW_DSMEM_MAX) {
         // many rows: a warp per row
         const void* kern = (const void*)select_fill_warp_kernel<T>;
         cudaError_t e = ensure_smem_attr(kern, FW_DSMEM_MAX);
@@ -1645,7 +1674,17 @@ static cudaError_t launch_finish_t(const IndexView& ix, int64_t n_blk, const T* 
                                                                sp.window, sp.sinks, s_max,
                                                                indices, counts, ws);
     } else {
-        select_fill_kernel<T><<<grid, FILL_THREADS, osm, st>>>(
+        size_t csm = osm;
+        if (ws.row_sc) {
+            // open-list area, then the score row when it fits
+            csm = (size_t)ix.G * 2 * sizeof(int32_t);
+            if (ws.row_ld * 4 <= ROW_SC_SMEM) csm += (size_t)ws.row_ld * 4;
+            cudaError_t e = ensure_smem_attr((const void*)select_fill_kernel<T>,
+                                             ROW_SC_SMEM + 2 * 4096 * 4);
+            if (e != cudaSuccess) return e;
+            if (csm > (size_t)ROW_SC_SMEM + 2 * 4096 * 4) return cudaErrorInvalidValue;
+        }
+        select_fill_kernel<T><<<grid, FILL_THREADS, csm, st>>>(
             ix, n_blk, lq, pos, Nq, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
     }
     note_launch();

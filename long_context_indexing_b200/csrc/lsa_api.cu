@@ -200,9 +200,9 @@ int64_t ent_cap_for(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d, ls
 }
 
 struct DecodeLayout {
-    size_t indices, counts, sel, part, counter, lst_g, lst_n, lst_tau, app_score, app_g, app_slot,
-        total;
-    int ns, kps, n_hg, n_slice, lst_cap;
+    size_t indices, counts, sel, part, counter, row_sc, app_score, app_g, app_slot, total;
+    int ns, kps, n_hg, n_slice;
+    int64_t row_ld;
 };
 
 
@@ -246,13 +246,9 @@ DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_sel
     if (nsl < min_sl) nsl = min_sl;
     if (nsl > 128) nsl = 128;
     L.n_slice = (int)nsl;
-    // slices of `per` buckets (a multiple of 32); only the first ones hold any
-    const int64_t per = (((v.NBK + nsl - 1) / nsl) + 31) / 32 * 32;
-    const int64_t used = (v.NBK + per - 1) / per;
-    L.lst_cap = (int)((DEC_TARGET + used - 1) / used);
-    L.lst_g = o;     o += al256((size_t)v.B * nsl * L.lst_cap * 4);
-    L.lst_n = o;     o += al256((size_t)v.B * nsl * 4);
-    L.lst_tau = o;   o += al256((size_t)v.B * nsl * 4);
+    // each sequence's row of approximate scores (the fill nominates from it)
+    L.row_ld = ((v.NBK + 63) / 64) * 64;
+    L.row_sc = o;    o += al256((size_t)v.B * L.row_ld * 4);
     L.app_score = o; o += al256((size_t)v.B * nsl * 8);
     L.app_g = o;     o += al256((size_t)v.B * nsl * 4);
     L.app_slot = o;  o += al256((size_t)v.B * 4);
@@ -755,13 +751,10 @@ lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
     int32_t* indices = (int32_t*)(base + L.indices);
     int32_t* counts = (int32_t*)(base + L.counts);
     SelectWs w = select_ws_carve(base + L.sel, v, 1);
-    // the fill ranks the candidate lists the prep pass writes (one per
-    // slice), and finishes the prep pass's append
-    w.lst_g = (int32_t*)(base + L.lst_g);
-    w.lst_n = (int32_t*)(base + L.lst_n);
-    w.lst_tau = (float*)(base + L.lst_tau);
-    w.n_lst = L.n_slice;
-    w.lst_cap = L.lst_cap;
+    // the fill nominates from the score rows the prep pass writes, and
+    // finishes the prep pass's append
+    w.row_sc = (const float*)(base + L.row_sc);
+    w.row_ld = L.row_ld;
     double* app_score = (double*)(base + L.app_score);
     int32_t* app_g = (int32_t*)(base + L.app_g);
     int32_t* app_slot = (int32_t*)(base + L.app_slot);

@@ -146,6 +146,10 @@ struct SelectWs {
     uint16_t* gmax;      // [B*Nq][n_grp] tensor-core path: group maxima (fp16 keys)
     float* theta;        // [B*Nq] tensor-core path: each row's list threshold
     int64_t n_grp;
+    // Decode: every eligible bucket's approximate score of row r at
+    // row_sc[r * row_ld]; when set, the fill nominates from it instead of lists.
+    const float* row_sc;
+    int64_t row_ld;
     int32_t* fb_list;    // [B*Nq]      queries that need the exact fallback
     int32_t* fb_count;   // [1]
     double* fb_scores;   // [FB_CTAS][NBK] scratch of the fallback
@@ -164,7 +168,6 @@ constexpr int KCF = 128;          // candidates the fill ranks at most (one per 
 constexpr int TC_LIST_CAP = KCF;  // candidates per (row, tensor-core split)
 constexpr int TC_MAX_SPLITS = 8;
 constexpr int TC_TARGET = 48;     // rank of a row's threshold among its group maxima
-constexpr int DEC_TARGET = 64;    // candidates summed over a decode query's slices
 
 // Work split of the tensor-core scorer (k_score_tc.cu).
 struct TcSplit {
