@@ -473,7 +473,7 @@ def run_decode(args, peaks, peak_src, ws=1):
     reps = max(1, args.steps // 2)
     ms = _events_time(graph.replay, reps, stream)
     us = _max_over_ranks(1e3 * ms / w.steps, ws)
-    idx.check()
+    fallbacks = idx.check()
     _, counts = lsa.decode_selection_views(work, w.B, w.s_max)
     n_sel = int(counts.sum().item())
     kv = n_sel * w.Hkv * w.d * 2 * 2
@@ -494,7 +494,8 @@ def run_decode(args, peaks, peak_src, ws=1):
                          "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                          "peak_source": "%s (copy bandwidth)" % peak_src,
                          "algorithmic_bytes_per_step": alg},
-            "gpu_launches_per_step": launches_per_step}
+            "gpu_launches_per_step": launches_per_step,
+            "selection_fallbacks": fallbacks}
 
 
 def _decode_cpu_baseline(w, inp, t_cap, steps):

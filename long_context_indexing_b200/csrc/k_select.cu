@@ -221,9 +221,18 @@ __device__ float radix_top_kc(const float* sc, int64_t nb, int32_t* cand)
         for (int x = threadIdx.x; x < 256; x += blockDim.x) hist[x] = 0;
         __syncthreads();
         const uint32_t prefix = sh_prefix;
-        for (int64_t g = threadIdx.x; g < nb; g += blockDim.x) {
-            const uint32_t kk = ord_key(sc[g]);
-            if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> sh) & 255u], 1u);
+        // warp-aggregated counts: scores share their leading bytes, so one
+        // atomic per distinct bin of a warp instead of one per score
+        const int64_t nb_up = (nb + 31) & ~(int64_t)31;
+        for (int64_t g = threadIdx.x; g < nb_up; g += blockDim.x) {
+            uint32_t bin = 0xFFFFFFFFu;
+            if (g < nb) {
+                const uint32_t kk = ord_key(sc[g]);
+                if ((kk & mask) == prefix) bin = (kk >> sh) & 255u;
+            }
+            const unsigned same = __match_any_sync(0xffffffffu, bin);
+            if (bin != 0xFFFFFFFFu && (threadIdx.x & 31) == __ffs(same) - 1)
+                atomicAdd(&hist[bin], (unsigned)__popc(same));
         }
         __syncthreads();
         if (threadIdx.x < 32) {
@@ -605,7 +614,7 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
     const int64_t b = blockIdx.y, i = blockIdx.x;
     const int64_t row = b * Nq + i;
     const int64_t pq = pos.at(b, Nq, i);
-    if (ws.app_n > 0 && i == 0 && threadIdx.x == 0) {
+    if (ws.app_n > 0 && i == 0 && threadIdx.x < 32) {
         // decode: the best of the sliced nearest-centroid searches (highest
         // exact score, lowest bucket on ties) joins the open block.  The group
         // lies inside this query's window, so the selection below never reads
@@ -614,7 +623,7 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
         if (o >= 0) {
             double bs = -INFINITY;
             int bg = 0x7fffffff;
-            for (int x = 0; x < ws.app_n; ++x) {
+            for (int x = threadIdx.x; x < ws.app_n; x += 32) {
                 const double sx = ws.app_score[b * ws.app_n + x];
                 const int gx = ws.app_g[b * ws.app_n + x];
                 if (sx > bs || (sx == bs && gx < bg)) {
@@ -622,7 +631,15 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
                     bg = gx;
                 }
             }
-            if (bg != 0x7fffffff) ix.open_bucket[b * ix.G + o] = bg;
+            for (int off = 16; off > 0; off >>= 1) {
+                const double os = __shfl_xor_sync(0xffffffffu, bs, off);
+                const int og = __shfl_xor_sync(0xffffffffu, bg, off);
+                if (os > bs || (os == bs && og < bg)) {
+                    bs = os;
+                    bg = og;
+                }
+            }
+            if (threadIdx.x == 0 && bg != 0x7fffffff) ix.open_bucket[b * ix.G + o] = bg;
         }
     }
     load_query(q_s, lq, row);
