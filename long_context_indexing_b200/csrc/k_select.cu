@@ -658,10 +658,27 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
             const float* src = ws.row_sc + row * ws.row_ld;
             const float* sc = src;
             if (ws.row_ld * 4 <= ROW_SC_SMEM) {
-                float* sm = reinterpret_cast<float*>(open_sm + 2 * ix.G);
-                for (int64_t g = threadIdx.x; g < nb; g += blockDim.x) sm[g] = src[g];
+                // 16-byte loads, eight in flight per thread (the row is a
+                // multiple of 64 floats, 256-byte aligned)
+                float4* sm = reinterpret_cast<float4*>(open_sm + ((2 * ix.G + 3) & ~3));
+                const float4* s4 = reinterpret_cast<const float4*>(src);
+                const int64_t n4 = (nb + 3) / 4;
+                constexpr int U = 8;
+                for (int64_t x0 = threadIdx.x; x0 < n4; x0 += (int64_t)U * blockDim.x) {
+                    float4 v[U];
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int64_t x = x0 + (int64_t)u * blockDim.x;
+                        if (x < n4) v[u] = s4[x];
+                    }
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int64_t x = x0 + (int64_t)u * blockDim.x;
+                        if (x < n4) sm[x] = v[u];
+                    }
+                }
                 __syncthreads();
-                sc = sm;
+                sc = reinterpret_cast<const float*>(sm);
             }
             const float t = radix_top_kc(sc, nb, cg);
             if (threadIdx.x == 0) {
@@ -1694,7 +1711,7 @@ static cudaError_t launch_finish_t(const IndexView& ix, int64_t n_blk, const T* 
         size_t csm = osm;
         if (ws.row_sc) {
             // open-list area, then the score row when it fits
-            csm = (size_t)ix.G * 2 * sizeof(int32_t);
+            csm = (size_t)((2 * ix.G + 3) & ~3) * sizeof(int32_t);
             if (ws.row_ld * 4 <= ROW_SC_SMEM) csm += (size_t)ws.row_ld * 4;
             cudaError_t e = ensure_smem_attr((const void*)select_fill_kernel<T>,
                                              ROW_SC_SMEM + 2 * 4096 * 4);
