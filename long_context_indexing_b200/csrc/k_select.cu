@@ -581,7 +581,6 @@ __device__ void cta_emit_tail(int64_t pq, int W, int64_t n_s, int64_t off, int s
 
 constexpr int FILL_THREADS = 128;
 static_assert(FILL_THREADS == KCF, "one candidate per fill thread");
-constexpr int ROW_SC_SMEM = 160 * 1024;   // decode score rows up to 40960 buckets in shared memory
 
 // ---------------------------------------------------------------------------
 // Exact ranking + greedy fill + emission.  One CTA (128 threads) per query.
@@ -643,52 +642,6 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
         }
     }
     load_query(q_s, lq, row);
-    if (ws.row_sc) {
-        // decode: the row's scores of every eligible bucket; the KC largest
-        // (radix select, from shared memory when the row fits) are the candidates
-        const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
-        if (nb <= KC) {
-            if ((int)threadIdx.x < KCF) cg[threadIdx.x] = ((int64_t)threadIdx.x < nb) ? (int)threadIdx.x : -1;
-            if (threadIdx.x == 0) {
-                sh_nc = (int)nb;
-                sh_tau = -INFINITY;
-                sh_complete = 1;
-            }
-        } else {
-            const float* src = ws.row_sc + row * ws.row_ld;
-            const float* sc = src;
-            if (ws.row_ld * 4 <= ROW_SC_SMEM) {
-                // 16-byte loads, eight in flight per thread (the row is a
-                // multiple of 64 floats, 256-byte aligned)
-                float4* sm = reinterpret_cast<float4*>(open_sm + ((2 * ix.G + 3) & ~3));
-                const float4* s4 = reinterpret_cast<const float4*>(src);
-                const int64_t n4 = (nb + 3) / 4;
-                constexpr int U = 8;
-                for (int64_t x0 = threadIdx.x; x0 < n4; x0 += (int64_t)U * blockDim.x) {
-                    float4 v[U];
-#pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        const int64_t x = x0 + (int64_t)u * blockDim.x;
-                        if (x < n4) v[u] = s4[x];
-                    }
-#pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        const int64_t x = x0 + (int64_t)u * blockDim.x;
-                        if (x < n4) sm[x] = v[u];
-                    }
-                }
-                __syncthreads();
-                sc = reinterpret_cast<const float*>(sm);
-            }
-            const float t = radix_top_kc(sc, nb, cg);
-            if (threadIdx.x == 0) {
-                sh_nc = KC;
-                sh_tau = t;
-                sh_complete = 0;
-            }
-        }
-        __syncthreads();
-    } else {
     // The row's candidate lists (n_lst <= FILL_THREADS): counts and bounds in
     // parallel, their offsets by one thread, then the bucket ids.  tau bounds
     // every eligible bucket left out of the lists; with every list complete
@@ -737,7 +690,6 @@ __global__ void __launch_bounds__(FILL_THREADS) select_fill_kernel(IndexView ix,
             cg[threadIdx.x] =
                 ws.lst_g[(row * nl + l) * ws.lst_cap + ((int)threadIdx.x - lst_off[l])];
         }
-    }
     }
     const int nc = sh_nc;
     const float tau = sh_tau;
@@ -1251,6 +1203,290 @@ __global__ void __launch_bounds__(32 * FW_WARPS) select_fill_warp_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// Decode selection, one CTA of DF_THREADS per sequence (latency matters: a
+// decode step has one query per sequence).  Candidates: the KC best of the
+// union of the slices' sorted lists (rank by counting); tau = the larger of
+// the union's next score and every slice's next unlisted score, which bounds
+// every bucket left out.  Then the steps of select_fill_kernel: exact
+// binary64 rescoring, ranking, availability, a prefix-sum greedy fill (one
+// warp), emission of whole buckets member by member over the CTA, partial
+// buckets by warps, recent window.
+// ---------------------------------------------------------------------------
+constexpr int DF_THREADS = 512;
+constexpr int DF_UNION = DEC_MAX_SLICES * DEC_M;
+
+template <typename T>
+__global__ void __launch_bounds__(DF_THREADS) decode_fill_kernel(IndexView ix, int64_t n_blk,
+                                                                 const T* lq, const int32_t* pos,
+                                                                 int R, int W, int S, int s_max,
+                                                                 int32_t* indices,
+                                                                 int32_t* counts, SelectWs ws)
+{
+    extern __shared__ int32_t open_sm[];   // [2][G] when the open block exists
+    __shared__ float q_s[DL];
+    __shared__ float us[DF_UNION];
+    __shared__ int ug[DF_UNION];
+    __shared__ int cg[KC];
+    __shared__ double es[KC];
+    __shared__ int order[KC];
+    __shared__ int av[KC], avc[KC];
+    __shared__ int t_g[KC], t_n[KC], t_off[KC], t_o0[KC], t_full[KC], t_mc[KC + 1];
+    __shared__ int sh_nc, sh_nt, sh_exact, sh_cmpl, sh_tot;
+    __shared__ float sh_tau;
+    __shared__ unsigned sh_slow;
+    const unsigned FULL = 0xffffffffu;
+    const int64_t b = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t pq = pos[b];
+    if (pq < 0 || pq >= ix.T_cap) return;       // recorded by the prep pass
+    // the best of the sliced nearest-centroid searches joins the open block
+    if (ws.app_n > 0 && warp == 0) {
+        const int o = ws.app_slot[b];
+        if (o >= 0) {
+            double bs = -INFINITY;
+            int bg = 0x7fffffff;
+            for (int x = lane; x < ws.app_n; x += 32) {
+                const double sx = ws.app_score[b * ws.app_n + x];
+                const int gx = ws.app_g[b * ws.app_n + x];
+                if (sx > bs || (sx == bs && gx < bg)) {
+                    bs = sx;
+                    bg = gx;
+                }
+            }
+            for (int off = 16; off > 0; off >>= 1) {
+                const double os = __shfl_xor_sync(FULL, bs, off);
+                const int og = __shfl_xor_sync(FULL, bg, off);
+                if (os > bs || (os == bs && og < bg)) {
+                    bs = os;
+                    bg = og;
+                }
+            }
+            if (lane == 0 && bg != 0x7fffffff) ix.open_bucket[b * ix.G + o] = bg;
+        }
+    }
+    load_query(q_s, lq, b);
+    // ---- the union of the slices' lists ----
+    const int nsl = ws.n_slice;
+    const int nu = nsl * DEC_M;
+    for (int e = threadIdx.x; e < nu; e += DF_THREADS) {
+        const int sl = e / DEC_M, r = e % DEC_M;
+        const int64_t ls = b * nsl + sl;
+        const bool ok = r < ws.dl_n[ls];
+        us[e] = ok ? ws.dl_s[ls * DEC_M + r] : -INFINITY;
+        ug[e] = ok ? ws.dl_g[ls * DEC_M + r] : -1;
+    }
+    if (warp == 0) {
+        float tm = -INFINITY;
+        int tot = 0;
+        for (int sl = lane; sl < nsl; sl += 32) {
+            tm = fmaxf(tm, ws.dl_tau[b * nsl + sl]);
+            tot += ws.dl_n[b * nsl + sl];
+        }
+        for (int off = 16; off > 0; off >>= 1) {
+            tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, off));
+            tot += __shfl_xor_sync(FULL, tot, off);
+        }
+        if (lane == 0) {
+            sh_tau = tm;                 // every slice's next unlisted score
+            sh_tot = tot;
+            sh_nc = min(tot, KC);
+            sh_cmpl = (tm == -INFINITY) && tot <= KC;
+        }
+    }
+    __shared__ float sh_next;                 // the union's score after its KC best
+    if (threadIdx.x == 0) sh_next = -INFINITY;
+    __syncthreads();
+    for (int e = threadIdx.x; e < nu; e += DF_THREADS) {
+        const int g = ug[e];
+        if (g < 0) continue;
+        const float x = us[e];
+        int rank = 0;
+        for (int u = 0; u < nu; ++u) {
+            const int g2 = ug[u];
+            if (g2 < 0) continue;
+            const float y = us[u];
+            rank += (y > x) || (y == x && g2 < g);
+        }
+        if (rank < KC) cg[rank] = g;
+        else if (rank == KC) sh_next = x;       // ranks are distinct: one writer
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) sh_tau = fmaxf(sh_tau, sh_next);
+    __syncthreads();
+    const int nc = sh_nc;
+    const float tau = sh_tau;
+    const bool complete = sh_cmpl != 0;
+    float l1 = 0.f;
+    // ---- exact scores, ranking, availability ----
+    if ((int)threadIdx.x < nc) es[threadIdx.x] = exact_score(ix, b, cg[threadIdx.x], q_s);
+    if (warp == 1) {
+        float a = fabsf(q_s[lane]) + fabsf(q_s[lane + 32]);
+        for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(FULL, a, off);
+        if (lane == 0) sh_exact = __float_as_int(a);    // |q|_1, handed on below
+    }
+    __syncthreads();
+    l1 = __int_as_float(sh_exact);
+    if ((int)threadIdx.x < nc) {
+        const int c = threadIdx.x;
+        int r = 0;
+        for (int c2 = 0; c2 < nc; ++c2) r += rank_before(es[c2], cg[c2], es[c], cg[c]);
+        order[r] = c;
+    }
+    FillCtx f;
+    f.ix = ix;
+    f.bseq = b;
+    f.n_blk = n_blk;
+    f.pos = pq;
+    f.hi = pq - W;
+    f.S = S;
+    f.open_live = (n_blk * ix.G < ix.NP) && (n_blk > 0) && (n_blk * (int64_t)ix.p * ix.G <= f.hi);
+    f.ol_n = 0;
+    f.ol_o = open_sm;
+    f.ol_g = open_sm + ix.G;
+    if (f.open_live) {
+        __shared__ int cnt_w[DF_THREADS / 32];
+        f.ol_n = build_open_list(ix, b, open_sm, open_sm + ix.G, cnt_w);
+    }
+    if (threadIdx.x == 0) sh_slow = 0u;
+    __syncthreads();
+    const int32_t* offs = ix.offsets + b * (ix.NBK + 1);
+    const int32_t* mem = ix.members + b * ix.NP;
+    const int p = ix.p;
+    if ((int)threadIdx.x < nc) {
+        const int c = threadIdx.x;
+        const int g = cg[c];
+        if (bucket_full(f, g)) {
+            av[c] = (offs[g + 1] - offs[g]) * p;
+            avc[c] = av[c];
+        } else {
+            atomicOr(&sh_slow, 1u << (c & 31));     // marks a group of candidates
+            av[c] = -1;
+        }
+    }
+    __syncthreads();
+    if (sh_slow) {
+        // buckets cut by the window or the sinks, or with open members: a warp each
+        for (int c = warp; c < nc; c += DF_THREADS / 32) {
+            if (av[c] >= 0) continue;                 // uniform over the warp
+            int64_t closed;
+            const int64_t a = warp_avail(f, cg[c], &closed);
+            if (lane == 0) {
+                av[c] = (int)a;
+                avc[c] = (int)closed;
+            }
+        }
+        __syncthreads();
+    }
+    // ---- greedy fill: warp 0, a prefix sum over the ranked candidates ----
+    if (warp == 0) {
+        constexpr int PL = KC / 32;
+        int rc[PL], ra[PL], pre[PL];
+        int lsum = 0;
+#pragma unroll
+        for (int u = 0; u < PL; ++u) {
+            const int r = PL * lane + u;
+            rc[u] = (r < nc) ? order[r] : -1;
+            ra[u] = (rc[u] >= 0) ? av[rc[u]] : 0;
+            pre[u] = lsum;
+            lsum += ra[u];
+        }
+        int sc = lsum;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(FULL, sc, o);
+            if (lane >= o) sc += y;
+        }
+        const int total_av = __shfl_sync(FULL, sc, 31);
+        const int lbase = sc - lsum;
+        int n_take = 0, cut_c = -1;
+#pragma unroll
+        for (int u = 0; u < PL; ++u) {
+            const int A = lbase + pre[u];
+            if (ra[u] > 0 && A < R) {
+                ++n_take;
+                if (A + ra[u] >= R) cut_c = rc[u];
+            }
+        }
+        int tinc = n_take;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(FULL, tinc, o);
+            if (lane >= o) tinc += y;
+        }
+        const int nt = __shfl_sync(FULL, tinc, 31);
+        int t = tinc - n_take;
+#pragma unroll
+        for (int u = 0; u < PL; ++u) {
+            const int A = lbase + pre[u];
+            if (ra[u] > 0 && A < R) {
+                const int c = rc[u];
+                const int g = cg[c];
+                t_g[t] = g;
+                t_n[t] = min(ra[u], R - A);
+                t_off[t] = A;
+                t_o0[t] = offs[g];
+                t_full[t] = bucket_full(f, g) ? 1 : 0;
+                ++t;
+            }
+        }
+        const unsigned cb = __ballot_sync(FULL, cut_c >= 0);
+        cut_c = cb ? __shfl_sync(FULL, cut_c, __ffs(cb) - 1) : -1;
+        bool exact = true;
+        if (!complete) {
+            const double eps = ldexp((double)l1, -12);
+            if (total_av < R) {
+                int64_t total = f.hi - S + 1;      // keys in [S, pos - W]
+                if (total < 0) total = 0;
+                exact = (int64_t)total_av >= total;
+            } else if (cut_c >= 0) {
+                exact = es[cut_c] > (double)tau + eps;
+            }
+        }
+        __syncwarp();
+        if (lane == 0) {
+            sh_nt = nt;
+            sh_exact = exact ? 1 : 0;
+            int acc = 0;                               // members of whole buckets before t
+            for (int tt = 0; tt < nt; ++tt) {
+                t_mc[tt] = acc;
+                if (t_full[tt]) acc += (t_n[tt] + p - 1) / p;
+            }
+            t_mc[nt] = acc;
+            if (!exact) {
+                const int slot = atomicAdd(ws.fb_count, 1);
+                ws.fb_list[slot] = (int32_t)b;
+                atomicAdd(ix.status + 1, 1u);
+            }
+        }
+    }
+    __syncthreads();
+    if (!sh_exact) return;
+    // ---- emission ----
+    const int nt = sh_nt;
+    int32_t* out = indices + b * (int64_t)s_max;
+    const int64_t n_s = (S < pq + 1) ? S : pq + 1;
+    for (int64_t x = threadIdx.x; x < n_s; x += DF_THREADS) out[x] = (int32_t)x;
+    int32_t* lr = out + n_s;
+    const int n_mem = t_mc[nt];
+    for (int m = threadIdx.x; m < n_mem; m += DF_THREADS) {
+        int lo = 0, hi = nt - 1;                       // last bucket with t_mc <= m
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (t_mc[mid] <= m) lo = mid;
+            else hi = mid - 1;
+        }
+        while (lo + 1 < nt && (!t_full[lo] || t_mc[lo + 1] <= m)) ++lo;
+        const int mi = m - t_mc[lo];
+        const int32_t mv = __ldg(mem + t_o0[lo] + mi);
+        const int k0 = mi * p;
+        const int nk = min(p, t_n[lo] - k0);
+        for (int q = 0; q < nk; ++q) lr[t_off[lo] + k0 + q] = mv * p + q;
+    }
+    for (int tt = warp; tt < nt; tt += DF_THREADS / 32)
+        if (!t_full[tt]) warp_emit_partial(f, t_g[tt], t_n[tt], lr + t_off[tt]);
+    const int64_t n_lr = nt ? (int64_t)t_off[nt - 1] + t_n[nt - 1] : 0;
+    cta_emit_tail(pq, W, n_s, n_s + n_lr, s_max, out, counts + b);
+}
+
+// ---------------------------------------------------------------------------
 // Exact fallback: persistent CTAs walk the list of flagged queries.  Every
 // eligible bucket gets its exact binary64 score; the fill repeatedly takes the
 // best remaining bucket (score desc, lowest id) until the budget is met.
@@ -1455,9 +1691,30 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_prep_kernel(
                 }
             }
             __syncthreads();
-            // this slice's scores join the sequence's score row
-            float* dst = const_cast<float*>(ws.row_sc) + b * ws.row_ld + g0;
-            for (int t = threadIdx.x; t < n; t += DEC_THREADS) dst[t] = sc[t];
+            // this slice's DEC_M best scores, sorted (ties to the lower
+            // bucket), and the next one
+            const int64_t ls = b * n_slice + sl;
+            for (int t = threadIdx.x; t < n; t += DEC_THREADS) {
+                const float x = sc[t];
+                int rank = 0;
+                for (int u = 0; u < n; ++u) {
+                    const float y = sc[u];
+                    rank += (y > x) || (y == x && u < t);
+                }
+                if (rank < DEC_M) {
+                    ws.dl_s[ls * DEC_M + rank] = x;
+                    ws.dl_g[ls * DEC_M + rank] = (int32_t)(g0 + t);
+                } else if (rank == DEC_M) {
+                    ws.dl_tau[ls] = x;
+                }
+            }
+            if (threadIdx.x == 0) {
+                ws.dl_n[ls] = min(n, DEC_M);
+                if (n <= DEC_M) ws.dl_tau[ls] = -INFINITY;
+            }
+        } else if (threadIdx.x == 0) {
+            ws.dl_n[b * n_slice + sl] = 0;
+            ws.dl_tau[b * n_slice + sl] = -INFINITY;
         }
     }
 
@@ -1664,8 +1921,11 @@ SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
     p += al256(4);
     w.fb_scores = (double*)p;
     p += al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
-    w.row_sc = nullptr;
-    w.row_ld = 0;
+    w.dl_s = nullptr;
+    w.dl_g = nullptr;
+    w.dl_n = nullptr;
+    w.dl_tau = nullptr;
+    w.n_slice = 0;
     w.n_grp = n_grp_of(ix, Nq);
     w.gmax = nullptr;
     w.theta = nullptr;
@@ -1698,7 +1958,7 @@ static cudaError_t launch_finish_t(const IndexView& ix, int64_t n_blk, const T* 
     if (ws.n_lst < 1 || ws.n_lst > FILL_THREADS || ws.lst_cap < 1) return cudaErrorInvalidValue;
     const int64_t rows_all = ix.B * Nq;
     const size_t wsm = (size_t)FW_WARPS * osm;   // one open list per warp
-    if (!ws.row_sc && rows_all >= FW_MIN_ROWS && ws.n_lst <= FW_LISTS && wsm <= FW_DSMEM_MAX) {
+    if (rows_all >= FW_MIN_ROWS && ws.n_lst <= FW_LISTS && wsm <= FW_DSMEM_MAX) {
         // many rows: a warp per row
         const void* kern = (const void*)select_fill_warp_kernel<T>;
         cudaError_t e = ensure_smem_attr(kern, FW_DSMEM_MAX);
@@ -1708,17 +1968,7 @@ static cudaError_t launch_finish_t(const IndexView& ix, int64_t n_blk, const T* 
                                                                sp.window, sp.sinks, s_max,
                                                                indices, counts, ws);
     } else {
-        size_t csm = osm;
-        if (ws.row_sc) {
-            // open-list area, then the score row when it fits
-            csm = (size_t)((2 * ix.G + 3) & ~3) * sizeof(int32_t);
-            if (ws.row_ld * 4 <= ROW_SC_SMEM) csm += (size_t)ws.row_ld * 4;
-            cudaError_t e = ensure_smem_attr((const void*)select_fill_kernel<T>,
-                                             ROW_SC_SMEM + 2 * 4096 * 4);
-            if (e != cudaSuccess) return e;
-            if (csm > (size_t)ROW_SC_SMEM + 2 * 4096 * 4) return cudaErrorInvalidValue;
-        }
-        select_fill_kernel<T><<<grid, FILL_THREADS, csm, st>>>(
+        select_fill_kernel<T><<<grid, FILL_THREADS, osm, st>>>(
             ix, n_blk, lq, pos, Nq, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
     }
     note_launch();
@@ -1763,6 +2013,36 @@ cudaError_t launch_select(const IndexView& ix, int64_t n_blk, const void* latent
                                counts, s_max, ws, use_tc, st);
     return launch_select_t(ix, n_blk, (const float*)latent_Q, pos, Nq, sp, indices, counts, s_max,
                            ws, false, st);
+}
+
+template <typename T>
+static cudaError_t launch_decode_finish_t(const IndexView& ix, int64_t n_blk, const T* lq,
+                                          const int32_t* pos, lsa_select_params sp,
+                                          int32_t* indices, int32_t* counts, int s_max,
+                                          const SelectWs& ws, cudaStream_t st)
+{
+    if (ws.n_slice < 1 || ws.n_slice > DEC_MAX_SLICES || !ws.dl_s) return cudaErrorInvalidValue;
+    const size_t osm = (n_blk > 0 && n_blk * ix.G < ix.NP) ? (size_t)ix.G * 2 * sizeof(int32_t) : 0;
+    decode_fill_kernel<T><<<(unsigned)ix.B, DF_THREADS, osm, st>>>(
+        ix, n_blk, lq, pos, sp.budget, sp.window, sp.sinks, s_max, indices, counts, ws);
+    note_launch();
+    const unsigned fb_grid = (unsigned)(ix.B < FB_CTAS ? ix.B : FB_CTAS);
+    select_fallback_kernel<T><<<fb_grid, FB_THREADS, osm, st>>>(ix, n_blk, lq, PosSrc{pos, 0}, 1,
+                                                                sp.budget, sp.window, sp.sinks,
+                                                                s_max, indices, counts, ws);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_finish(const IndexView& ix, int64_t n_blk, const void* latent_q,
+                                 const int32_t* pos, lsa_select_params sp, int32_t* indices,
+                                 int32_t* counts, int s_max, const SelectWs& ws, cudaStream_t st)
+{
+    if (ix.dtype == LSA_BF16)
+        return launch_decode_finish_t(ix, n_blk, (const __nv_bfloat16*)latent_q, pos, sp, indices,
+                                      counts, s_max, ws, st);
+    return launch_decode_finish_t(ix, n_blk, (const float*)latent_q, pos, sp, indices, counts,
+                                  s_max, ws, st);
 }
 
 cudaError_t launch_select_finish(const IndexView& ix, int64_t n_blk, const void* latent_Q,

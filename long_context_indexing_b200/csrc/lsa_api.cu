@@ -200,9 +200,9 @@ int64_t ent_cap_for(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d, ls
 }
 
 struct DecodeLayout {
-    size_t indices, counts, sel, part, counter, row_sc, app_score, app_g, app_slot, total;
+    size_t indices, counts, sel, part, counter, dl_s, dl_g, dl_n, dl_tau, app_score, app_g,
+        app_slot, total;
     int ns, kps, n_hg, n_slice;
-    int64_t row_ld;
 };
 
 
@@ -244,11 +244,13 @@ DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_sel
     int64_t nsl = ((int64_t)sm_count() + v.B - 1) / v.B;
     const int64_t min_sl = (v.NBK + 991) / 992;
     if (nsl < min_sl) nsl = min_sl;
-    if (nsl > 128) nsl = 128;
+    if (nsl > DEC_MAX_SLICES) nsl = DEC_MAX_SLICES;
     L.n_slice = (int)nsl;
-    // each sequence's row of approximate scores (the fill nominates from it)
-    L.row_ld = ((v.NBK + 63) / 64) * 64;
-    L.row_sc = o;    o += al256((size_t)v.B * L.row_ld * 4);
+    // each slice's sorted list of its DEC_M best scores (the fill merges them)
+    L.dl_s = o;      o += al256((size_t)v.B * nsl * DEC_M * 4);
+    L.dl_g = o;      o += al256((size_t)v.B * nsl * DEC_M * 4);
+    L.dl_n = o;      o += al256((size_t)v.B * nsl * 4);
+    L.dl_tau = o;    o += al256((size_t)v.B * nsl * 4);
     L.app_score = o; o += al256((size_t)v.B * nsl * 8);
     L.app_g = o;     o += al256((size_t)v.B * nsl * 4);
     L.app_slot = o;  o += al256((size_t)v.B * 4);
@@ -751,10 +753,13 @@ lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
     int32_t* indices = (int32_t*)(base + L.indices);
     int32_t* counts = (int32_t*)(base + L.counts);
     SelectWs w = select_ws_carve(base + L.sel, v, 1);
-    // the fill nominates from the score rows the prep pass writes, and
-    // finishes the prep pass's append
-    w.row_sc = (const float*)(base + L.row_sc);
-    w.row_ld = L.row_ld;
+    // the fill merges the slices' lists the prep pass writes, and finishes
+    // the prep pass's append
+    w.dl_s = (float*)(base + L.dl_s);
+    w.dl_g = (int32_t*)(base + L.dl_g);
+    w.dl_n = (int32_t*)(base + L.dl_n);
+    w.dl_tau = (float*)(base + L.dl_tau);
+    w.n_slice = L.n_slice;
     double* app_score = (double*)(base + L.app_score);
     int32_t* app_g = (int32_t*)(base + L.app_g);
     int32_t* app_slot = (int32_t*)(base + L.app_slot);
@@ -773,8 +778,7 @@ lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
                                        latent_q, pos, Hkv, d, sp.window, w, app_score, app_g,
                                        app_slot, L.n_slice, counter, L.n_hg, st);
     if (e != cudaSuccess) return cuda_fail(e, "decode append/nominate");
-    PosSrc ps{pos, 0};
-    e = launch_select_finish(v, idx->n_blk, latent_q, ps, 1, sp, indices, counts, s_max, w, st);
+    e = launch_decode_finish(v, idx->n_blk, latent_q, pos, sp, indices, counts, s_max, w, st);
     if (e != cudaSuccess) return cuda_fail(e, "decode select");
     const float scale = (float)(1.0 / sqrt((double)d));
     if (v.dtype == LSA_BF16)

@@ -146,10 +146,14 @@ struct SelectWs {
     uint16_t* gmax;      // [B*Nq][n_grp] tensor-core path: group maxima (fp16 keys)
     float* theta;        // [B*Nq] tensor-core path: each row's list threshold
     int64_t n_grp;
-    // Decode: every eligible bucket's approximate score of row r at
-    // row_sc[r * row_ld]; when set, the fill nominates from it instead of lists.
-    const float* row_sc;
-    int64_t row_ld;
+    // Decode: slice s of sequence b lists its DEC_M best approximate scores,
+    // sorted (dl_s, dl_g at [(b * n_slice + s) * DEC_M]), their count dl_n and
+    // dl_tau, the slice's next score (-inf when it listed all of them).
+    float* dl_s;
+    int32_t* dl_g;
+    int32_t* dl_n;
+    float* dl_tau;
+    int n_slice;
     int32_t* fb_list;    // [B*Nq]      queries that need the exact fallback
     int32_t* fb_count;   // [1]
     double* fb_scores;   // [FB_CTAS][NBK] scratch of the fallback
@@ -168,6 +172,8 @@ constexpr int KCF = 128;          // candidates the fill ranks at most (one per 
 constexpr int TC_LIST_CAP = KCF;  // candidates per (row, tensor-core split)
 constexpr int TC_MAX_SPLITS = 8;
 constexpr int TC_TARGET = 48;     // rank of a row's threshold among its group maxima
+constexpr int DEC_M = 16;         // best scores a decode slice lists
+constexpr int DEC_MAX_SLICES = 128;
 
 // Work split of the tensor-core scorer (k_score_tc.cu).
 struct TcSplit {
@@ -188,6 +194,12 @@ SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq);
 cudaError_t launch_select(const IndexView& ix, int64_t n_blk, const void* latent_Q, PosSrc pos,
                           int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
                           int s_max, const SelectWs& ws, bool use_tc, cudaStream_t st);
+
+// Decode: exact fill + emission from the slices' sorted lists, then the
+// exact fallback (one query per sequence).
+cudaError_t launch_decode_finish(const IndexView& ix, int64_t n_blk, const void* latent_q,
+                                 const int32_t* pos, lsa_select_params sp, int32_t* indices,
+                                 int32_t* counts, int s_max, const SelectWs& ws, cudaStream_t st);
 
 // Exact fill + emission + fallback only (candidates already nominated).
 cudaError_t launch_select_finish(const IndexView& ix, int64_t n_blk, const void* latent_Q,
