@@ -254,9 +254,26 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
     if (warp == CONS_WARPS) {
         // ---------------- producer ----------------
         const int32_t last = (n_all > 0) ? idx[n_all - 1] : 0;
+        // this lane's key ids of the next stage are read before the wait for
+        // a free slot, so the index loads overlap the copies in flight
+        constexpr int XPL = (2 * C::KT + 31) / 32;   // copies per lane per stage
+        int32_t tn[XPL];
+        auto load_tok = [&](int j) {
+#pragma unroll
+            for (int u = 0; u < XPL; ++u) {
+                const int x = lane + 32 * u;
+                const int key = k_lo + j * C::KT + x % C::KT;
+                tn[u] = (x < 2 * C::KT && key < k_hi) ? idx[key] : last;
+            }
+        };
+        if (n_st > 0) load_tok(0);
         for (int j = 0; j < n_st; ++j) {
             const int s = j % STAGES;
             const uint32_t ph = (uint32_t)((j / STAGES) & 1);
+            int32_t tc[XPL];
+#pragma unroll
+            for (int u = 0; u < XPL; ++u) tc[u] = tn[u];
+            if (j + 1 < n_st) load_tok(j + 1);
             // the warp agrees on every decision, so it never diverges here
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
             if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ph ^ 1u, wl))) {
@@ -269,10 +286,12 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
             if (lane == 0) ptx::mbar_arrive_expect_tx(&full[s], 2u * C::KT * C::RB);
             __syncwarp();
             unsigned char* kt = smem + s * C::STAGE;
-            for (int x = lane; x < 2 * C::KT; x += 32) {
+#pragma unroll
+            for (int u = 0; u < XPL; ++u) {
+                const int x = lane + 32 * u;
+                if (x >= 2 * C::KT) break;
                 const int r = x % C::KT;
-                const int key = k_lo + j * C::KT + r;
-                const int32_t t = checked_index(key < k_hi ? idx[key] : last, T_cap, status);
+                const int32_t t = checked_index(tc[u], T_cap, status);
                 const int64_t off = ((b * T_cap + t) * Hkv + g0) * (int64_t)D;
                 if (x < C::KT)
                     ptx::bulk_g2s(kt + r * C::PITCH, K + off, C::RB, &full[s]);
@@ -547,15 +566,24 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restri
             L += ml.y * w;
         }
         const int n = min(32, ns - s0);
-        for (int j = 0; j < n; ++j) {
-            const float wj = __shfl_sync(0xffffffffu, w, j);
-            if (live) {
-                const float4 v =
-                    __ldcg(reinterpret_cast<const float4*>(base + (s0 + j) * sstride) + lane);
-                acc.x += v.x * wj;
-                acc.y += v.y * wj;
-                acc.z += v.z * wj;
-                acc.w += v.w * wj;
+        // eight splits' loads in flight at a time
+        for (int j0 = 0; j0 < n; j0 += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (live && j0 + u < n)
+                    v[u] = __ldcg(reinterpret_cast<const float4*>(base + (s0 + j0 + u) * sstride) + lane);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float wj = __shfl_sync(0xffffffffu, w, (j0 + u) & 31);
+                if (j0 + u < n) {
+                    acc.x += v[u].x * wj;
+                    acc.y += v[u].y * wj;
+                    acc.z += v[u].z * wj;
+                    acc.w += v[u].w * wj;
+                }
             }
         }
     }

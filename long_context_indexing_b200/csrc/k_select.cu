@@ -1231,6 +1231,7 @@ __global__ void __launch_bounds__(DF_THREADS) decode_fill_kernel(IndexView ix, i
     __shared__ int order[KC];
     __shared__ int av[KC], avc[KC];
     __shared__ int t_g[KC], t_n[KC], t_off[KC], t_o0[KC], t_full[KC], t_mc[KC + 1];
+    __shared__ int c_o0[KC], c_full[KC];    // per candidate: first CSR position, all keys available
     __shared__ int sh_nc, sh_nt, sh_exact, sh_cmpl, sh_tot;
     __shared__ float sh_tau;
     __shared__ unsigned sh_slow;
@@ -1300,12 +1301,23 @@ __global__ void __launch_bounds__(DF_THREADS) decode_fill_kernel(IndexView ix, i
         const int g = ug[e];
         if (g < 0) continue;
         const float x = us[e];
+        // every slice's list is sorted (score desc, bucket asc; unlisted
+        // entries at the end): the entries ranking before (x, g) are a prefix,
+        // found by binary search
         int rank = 0;
-        for (int u = 0; u < nu; ++u) {
-            const int g2 = ug[u];
-            if (g2 < 0) continue;
-            const float y = us[u];
-            rank += (y > x) || (y == x && g2 < g);
+        for (int sl = 0; sl < nsl; ++sl) {
+            const float* ys = us + sl * DEC_M;
+            const int* gs = ug + sl * DEC_M;
+            int lo = 0, hi = DEC_M;                 // first entry not before (x, g)
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                const int g2 = gs[mid];
+                const float y = ys[mid];
+                const bool before = g2 >= 0 && ((y > x) || (y == x && g2 < g));
+                if (before) lo = mid + 1;
+                else hi = mid;
+            }
+            rank += lo;
         }
         if (rank < KC) cg[rank] = g;
         else if (rank == KC) sh_next = x;       // ranks are distinct: one writer
@@ -1355,10 +1367,14 @@ __global__ void __launch_bounds__(DF_THREADS) decode_fill_kernel(IndexView ix, i
     if ((int)threadIdx.x < nc) {
         const int c = threadIdx.x;
         const int g = cg[c];
+        const int o0 = offs[g];
+        c_o0[c] = o0;
         if (bucket_full(f, g)) {
-            av[c] = (offs[g + 1] - offs[g]) * p;
+            c_full[c] = 1;
+            av[c] = (offs[g + 1] - o0) * p;
             avc[c] = av[c];
         } else {
+            c_full[c] = 0;
             atomicOr(&sh_slow, 1u << (c & 31));     // marks a group of candidates
             av[c] = -1;
         }
@@ -1422,8 +1438,8 @@ __global__ void __launch_bounds__(DF_THREADS) decode_fill_kernel(IndexView ix, i
                 t_g[t] = g;
                 t_n[t] = min(ra[u], R - A);
                 t_off[t] = A;
-                t_o0[t] = offs[g];
-                t_full[t] = bucket_full(f, g) ? 1 : 0;
+                t_o0[t] = c_o0[c];
+                t_full[t] = c_full[c];
                 ++t;
             }
         }
@@ -1655,20 +1671,31 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_prep_kernel(
                 for (int e = 0; e < 8; ++e) q[e] = q_s[sub * 8 + e];
                 const uint4* base = reinterpret_cast<const uint4*>(
                     (const __nv_bfloat16*)ix.cent_rt + (b * ix.NBK + g0) * DL);
-                for (int r0 = warp * RPI; r0 < n; r0 += (DEC_THREADS / 32) * RPI) {
-                    const int r = r0 + rsel;
-                    const uint4 raw = (r < n) ? __ldg(base + (int64_t)r * (DL / 8) + sub) : make_uint4(0, 0, 0, 0);
-                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-                    float acc = 0.f;
+                // eight rows' loads in flight per lane, then their dot products
+                constexpr int RU = 8;
+                constexpr int STEP = (DEC_THREADS / 32) * RPI;
+                for (int r00 = warp * RPI; r00 < n; r00 += RU * STEP) {
+                    uint4 raw[RU];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(h[e]);
-                        acc = fmaf(q[2 * e], f.x, acc);
-                        acc = fmaf(q[2 * e + 1], f.y, acc);
+                    for (int u = 0; u < RU; ++u) {
+                        const int r = r00 + u * STEP + rsel;
+                        raw[u] = (r < n) ? __ldg(base + (int64_t)r * (DL / 8) + sub) : make_uint4(0, 0, 0, 0);
                     }
 #pragma unroll
-                    for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-                    if (sub == 0 && r < n) sc[r] = acc;
+                    for (int u = 0; u < RU; ++u) {
+                        const int r = r00 + u * STEP + rsel;
+                        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+                        float acc = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(h[e]);
+                            acc = fmaf(q[2 * e], f.x, acc);
+                            acc = fmaf(q[2 * e + 1], f.y, acc);
+                        }
+#pragma unroll
+                        for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                        if (sub == 0 && r < n) sc[r] = acc;
+                    }
                 }
             } else {
                 constexpr int LPR = 16, RPI = 32 / LPR;
@@ -1785,14 +1812,27 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_prep_kernel(
         const int rows = (int)((c1 - t0) < 64 ? (c1 - t0) : 64);
         __syncthreads();
         const float4* src = reinterpret_cast<const float4*>(cent + t0 * DL);
-        for (int x = threadIdx.x; x < rows * (DL / 4); x += blockDim.x) {
-            const float4 f = src[x];
-            const int r = x / (DL / 4), c = (x % (DL / 4)) * 4;
-            float* dst = tile + r * (DL + 1) + c;
-            dst[0] = f.x;
-            dst[1] = f.y;
-            dst[2] = f.z;
-            dst[3] = f.w;
+        {
+            // all of the tile's loads in flight (64 rows x 16 float4 over the CTA)
+            constexpr int TU = (64 * (DL / 4) + DEC_THREADS - 1) / DEC_THREADS;
+            float4 fv[TU];
+#pragma unroll
+            for (int u = 0; u < TU; ++u) {
+                const int x = threadIdx.x + u * DEC_THREADS;
+                if (x < rows * (DL / 4)) fv[u] = src[x];
+            }
+#pragma unroll
+            for (int u = 0; u < TU; ++u) {
+                const int x = threadIdx.x + u * DEC_THREADS;
+                if (x < rows * (DL / 4)) {
+                    const int r = x / (DL / 4), c = (x % (DL / 4)) * 4;
+                    float* dst = tile + r * (DL + 1) + c;
+                    dst[0] = fv[u].x;
+                    dst[1] = fv[u].y;
+                    dst[2] = fv[u].z;
+                    dst[3] = fv[u].w;
+                }
+            }
         }
         __syncthreads();
         if ((int)threadIdx.x < rows) {
