@@ -23,15 +23,19 @@ namespace lsa {
 
 // ---------------------------------------------------------------------------
 // Pool + normalise.  One warp per 32 consecutive pooled groups.
-//   phase 1 (lanes = dimension pairs): x = (((r0 + r1) + r2) + ...) / p,
-//            coalesced reads of the p latent rows, writes pooled;
+//   phase 1 x = (((r0 + r1) + r2) + ...) / p, writes pooled: bf16 rows with
+//            p in {1, 2, 4, 8} are read as one contiguous run per group with
+//            16-byte lanes and summed after shuffles; otherwise lanes =
+//            dimension pairs;
 //   phase 2 (lane = group): ss = sum_i x_i^2 in ascending i (binary64),
 //            nrm = sqrt(ss);
 //   phase 3 (lanes = dimension pairs): u_i = x_i / nrm, writes unit.
 // ---------------------------------------------------------------------------
 constexpr int POOL_WARPS = 4;
 
-template <typename T>
+// P > 0: bf16 rows with P rows per group (vectorised path); P = 0: any dtype
+// and pool size.
+template <typename T, int P>
 __global__ void __launch_bounds__(POOL_WARPS * 32) pool_unit_kernel(IndexView ix,
                                                                     const T* __restrict__ lat,
                                                                     int64_t j0, int64_t j1)
@@ -48,19 +52,81 @@ __global__ void __launch_bounds__(POOL_WARPS * 32) pool_unit_kernel(IndexView ix
     float* pooled = ix.pooled + b * ix.NP * DL;
     float* unit = ix.unit + b * ix.NP * DL;
 
-    for (int g = 0; g < n; ++g) {
-        const int64_t j = jw + g;
-        const T* row = seq + (j * p) * DL;
-        float s0 = load_elt(row + 2 * lane), s1 = load_elt(row + 2 * lane + 1);
-        for (int r = 1; r < p; ++r) {
-            s0 = __fadd_rn(s0, load_elt(row + (int64_t)r * DL + 2 * lane));
-            s1 = __fadd_rn(s1, load_elt(row + (int64_t)r * DL + 2 * lane + 1));
+    if (P > 0) {
+        // bf16 rows, P rows per group: the group's P consecutive 128-byte rows
+        // are one contiguous run, read with 16-byte lanes (8 lanes per row),
+        // four groups' loads in flight; lane L < 8 then gathers dimensions
+        // 8L .. 8L+7 of rows 0 .. P-1 by shuffles and sums them in row order
+        constexpr int CH = P * 8;                   // 16-byte chunks per group
+        constexpr int NU = (CH + 31) / 32 > 0 ? (CH + 31) / 32 : 1;   // loads per lane per group
+        constexpr int GU = 4;                       // groups per batch
+        const int L = lane & 7;
+        for (int g0 = 0; g0 < n; g0 += GU) {
+            uint4 v[GU][NU];
+#pragma unroll
+            for (int gg = 0; gg < GU; ++gg) {
+                const uint4* src = reinterpret_cast<const uint4*>(seq + (jw + g0 + gg) * P * DL);
+#pragma unroll
+                for (int u = 0; u < NU; ++u) {
+                    const int c = lane + 32 * u;
+                    v[gg][u] = (g0 + gg < n && c < CH) ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+#pragma unroll
+            for (int gg = 0; gg < GU; ++gg) {
+                float sacc[8];
+#pragma unroll
+                for (int r = 0; r < P; ++r) {
+                    const uint4 w = v[gg][r / 4];
+                    const int srcl = (r % 4) * 8 + L;
+                    uint4 y;
+                    y.x = __shfl_sync(0xffffffffu, w.x, srcl);
+                    y.y = __shfl_sync(0xffffffffu, w.y, srcl);
+                    y.z = __shfl_sync(0xffffffffu, w.z, srcl);
+                    y.w = __shfl_sync(0xffffffffu, w.w, srcl);
+                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&y);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h[e]);
+                        if (r == 0) {
+                            sacc[2 * e] = f.x;
+                            sacc[2 * e + 1] = f.y;
+                        } else {
+                            sacc[2 * e] = __fadd_rn(sacc[2 * e], f.x);
+                            sacc[2 * e + 1] = __fadd_rn(sacc[2 * e + 1], f.y);
+                        }
+                    }
+                }
+                const int g = g0 + gg;
+                if (lane < 8 && g < n) {
+                    const float fp = (float)P;
+                    float xv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        xv[e] = __fdiv_rn(sacc[e], fp);
+                        xs[warp][g][8 * L + e] = xv[e];
+                    }
+                    float4* dst = reinterpret_cast<float4*>(pooled + (jw + g) * DL + 8 * L);
+                    dst[0] = make_float4(xv[0], xv[1], xv[2], xv[3]);
+                    dst[1] = make_float4(xv[4], xv[5], xv[6], xv[7]);
+                }
+            }
         }
-        const float fp = (float)p;
-        const float x0 = __fdiv_rn(s0, fp), x1 = __fdiv_rn(s1, fp);
-        *reinterpret_cast<float2*>(pooled + j * DL + 2 * lane) = make_float2(x0, x1);
-        xs[warp][g][2 * lane] = x0;
-        xs[warp][g][2 * lane + 1] = x1;
+    } else {
+        for (int g = 0; g < n; ++g) {
+            const int64_t j = jw + g;
+            const T* row = seq + (j * p) * DL;
+            float s0 = load_elt(row + 2 * lane), s1 = load_elt(row + 2 * lane + 1);
+            for (int r = 1; r < p; ++r) {
+                s0 = __fadd_rn(s0, load_elt(row + (int64_t)r * DL + 2 * lane));
+                s1 = __fadd_rn(s1, load_elt(row + (int64_t)r * DL + 2 * lane + 1));
+            }
+            const float fp = (float)p;
+            const float x0 = __fdiv_rn(s0, fp), x1 = __fdiv_rn(s1, fp);
+            *reinterpret_cast<float2*>(pooled + j * DL + 2 * lane) = make_float2(x0, x1);
+            xs[warp][g][2 * lane] = x0;
+            xs[warp][g][2 * lane + 1] = x1;
+        }
     }
     __syncwarp();
     if (lane < n) {
@@ -92,11 +158,19 @@ cudaError_t launch_pool_unit(const IndexView& ix, const void* latent_K, int64_t 
     const int64_t groups = j1 - j0;
     const int per_cta = POOL_WARPS * 32;
     dim3 grid((unsigned)((groups + per_cta - 1) / per_cta), (unsigned)ix.B);
-    if (ix.dtype == LSA_BF16)
-        pool_unit_kernel<__nv_bfloat16><<<grid, per_cta, 0, st>>>(
-            ix, (const __nv_bfloat16*)latent_K, j0, j1);
-    else
-        pool_unit_kernel<float><<<grid, per_cta, 0, st>>>(ix, (const float*)latent_K, j0, j1);
+    if (ix.dtype == LSA_BF16) {
+        typedef __nv_bfloat16 B;
+        const B* lk = (const B*)latent_K;
+        switch (ix.p) {
+        case 1: pool_unit_kernel<B, 1><<<grid, per_cta, 0, st>>>(ix, lk, j0, j1); break;
+        case 2: pool_unit_kernel<B, 2><<<grid, per_cta, 0, st>>>(ix, lk, j0, j1); break;
+        case 4: pool_unit_kernel<B, 4><<<grid, per_cta, 0, st>>>(ix, lk, j0, j1); break;
+        case 8: pool_unit_kernel<B, 8><<<grid, per_cta, 0, st>>>(ix, lk, j0, j1); break;
+        default: pool_unit_kernel<B, 0><<<grid, per_cta, 0, st>>>(ix, lk, j0, j1); break;
+        }
+    } else {
+        pool_unit_kernel<float, 0><<<grid, per_cta, 0, st>>>(ix, (const float*)latent_K, j0, j1);
+    }
     note_launch();
     return cudaGetLastError();
 }
