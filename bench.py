@@ -284,6 +284,82 @@ def _sample_rows(w, n, device):
     return torch.arange(0, n * stride, stride, device=device)[:n]
 
 
+# -------------------------------------------------------- split of one chunk --
+
+def _query_slice(nq, rank, ws):
+    """Contiguous rows [q0, q1) of an nq-query chunk for `rank` of `ws` (equal
+    shares; nq must be a multiple of ws)."""
+    if nq % ws:
+        raise ValueError("%d chunk queries do not split evenly over %d ranks" % (nq, ws))
+    n = nq // ws
+    return rank * n, (rank + 1) * n
+
+
+def _gather_rows(part, ws):
+    """All ranks' row blocks [n][...] concatenated in rank order ([ws * n][...]),
+    on every rank."""
+    if ws == 1:
+        return part
+    part = part.contiguous()
+    if torch.distributed.get_backend() == "nccl":
+        out = torch.empty((ws * part.shape[0],) + tuple(part.shape[1:]), dtype=part.dtype,
+                          device=part.device)
+        torch.distributed.all_gather_into_tensor(out, part)
+        return out
+    parts = [torch.empty_like(part) for _ in range(ws)]
+    torch.distributed.all_gather(parts, part)
+    return torch.cat(parts, 0)
+
+
+def run_lsa_split(args, rank, ws):
+    """One chunk's queries split over the ranks: every rank holds the same
+    (replicated) caches and index, extends the index over the whole chunk,
+    selects and attends its contiguous share of the queries, and the outputs
+    are all-gathered (NCCL) inside the timed step.  Strong scaling: the job is
+    one chunk whatever the rank count."""
+    import long_context_indexing_b200 as lsa
+
+    w = _bench_workload(args)
+    dev = torch.device("cuda")
+    inp = synth.prefill_inputs(w, seed=args.seed, device=dev)      # the same chunk on every rank
+    span = w.p * w.G
+    T_old = w.T - w.nq
+    q0, q1 = _query_slice(w.nq, rank, ws)
+    idx = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16 if w.dtype == "bf16" else lsa.F32)
+    idx.build(inp["latent_K"], (T_old // span) * span)
+    lq = inp["latent_Q"][:, q0:q1].contiguous()
+    Qp = inp["Q"][:, q0:q1].contiguous()
+    work = torch.empty(lsa.lsa_prefill_workspace_bytes(idx, q1 - q0, w.Hq, w.Hkv, w.d, w.R, w.W,
+                                                       w.S), dtype=torch.uint8, device=dev)
+    Op = torch.empty_like(Qp)
+    stream = torch.cuda.current_stream()
+    result = {}
+
+    def step():
+        lsa.lsa_prefill_chunk_queries(idx, inp["latent_K"], lq, Qp, inp["K"], inp["V"], T_old,
+                                      w.T, q0, q1, w.R, w.W, w.S, workspace=work, out=Op)
+        result["O"] = _gather_rows(Op[0], ws)
+
+    for _ in range(args.warmup):
+        step()
+    _barrier(ws)
+    launches0 = lsa.kernel_launches()
+    ms = _max_over_ranks(_events_time(step, args.steps, stream), ws)
+    launches = lsa.kernel_launches() - launches0
+    _barrier(ws)
+    fallbacks = idx.check()
+    line = {"metric": METRIC, "value": round(w.nq / (ms * 1e-3), 2), "unit": "queries/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic (seeded clustered mixture; no model weights or datasets)",
+            "config": dict(_config(w, ws), parallelism="query split of one chunk over %d ranks "
+                           "(replicated caches and index, outputs all-gathered)" % ws),
+            "e2e": None, "gpu_launches": launches, "selection_fallbacks": fallbacks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------------- lsa --
 
 def _bench_workload(args):
@@ -584,6 +660,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-T", type=int, default=None,
                     help="override the decode context length (a multiple of p * block)")
+    ap.add_argument("--split", choices=["chunks", "queries"], default="chunks",
+                    help="several GPUs: every rank runs its own chunk (weak scaling), or one "
+                         "chunk's queries are split over the ranks (strong scaling)")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the decode measurement (prints its object)")
     args = ap.parse_args()
@@ -598,6 +677,8 @@ def main():
                 print(json.dumps(out), flush=True)
         elif args.impl == "reference":
             run_reference(args, rank, ws)
+        elif args.split == "queries":
+            run_lsa_split(args, rank, ws)
         else:
             run_lsa(args, rank, ws)
     finally:

@@ -275,6 +275,26 @@ lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* l
                              int64_t T_new, int Hq, int Hkv, int d, lsa_select_params sp,
                              void* workspace, size_t ws_bytes, void* O, void* stream);
 
+/* lsa_prefill_chunk for a contiguous range of the chunk's queries: rows
+ * q_begin .. q_end - 1 of the chunk, at positions T_old + q_begin ..
+ * T_old + q_end - 1 (this library's own entry, for splitting one chunk's
+ * queries over GPUs; the pages' serving layout splits the KV cache instead,
+ * "Latent Sparse Attention: un indice gerarchico per contesti lunghi",
+ * paragraph on memory).  The index is extended over the whole [T_old, T_new)
+ * exactly as lsa_prefill_chunk does -- the extension is deterministic, so
+ * every caller that runs it on the same keys holds the same index -- and only
+ * the range's queries are selected and attended.  latent_Q [B][n][64], Q and
+ * O [B][n][Hq][d] with n = q_end - q_begin; the workspace is sized by
+ * lsa_prefill_workspace_bytes(idx, n, ...).  Each query's selection and
+ * output are those lsa_prefill_chunk gives it over the whole chunk.
+ * Requires 0 <= q_begin < q_end <= T_new - T_old; fails like
+ * lsa_prefill_chunk otherwise. */
+lsa_status lsa_prefill_chunk_queries(lsa_index* idx, const void* latent_K, const void* latent_Q,
+                                     const void* Q, const void* K, const void* V, int64_t T_old,
+                                     int64_t T_new, int64_t q_begin, int64_t q_end, int Hq,
+                                     int Hkv, int d, lsa_select_params sp, void* workspace,
+                                     size_t ws_bytes, void* O, void* stream);
+
 /* The two halves of lsa_prefill_chunk, for callers that overlap or time them
  * separately (this library's split; the pages describe the chunk as one
  * step).  lsa_prefill_select extends the index over [T_old, T_new) and

@@ -20,7 +20,7 @@ __all__ = [
     "LsaError", "LsaIndex", "lsa_index_bytes", "lsa_build_index", "lsa_select",
     "lsa_sparse_attn", "lsa_prefill_chunk", "lsa_prefill_workspace_bytes",
     "lsa_prefill_partial_slots", "lsa_prefill_select", "lsa_prefill_attend",
-    "lsa_prefill_chunk_host", "set_wait_limit",
+    "lsa_prefill_chunk_host", "lsa_prefill_chunk_queries", "set_wait_limit",
     "lsa_decode_workspace_bytes", "lsa_decode_step", "lsa_select_noalloc", "library_path", "kernel_launches", "F32",
     "BF16",
 ]
@@ -77,6 +77,8 @@ def _declare(lib):
                                     SelectParams, P, SZ, P, P, P, P], I),
         "lsa_decode_workspace_bytes": ([P, I, I, I, SelectParams], SZ),
         "lsa_set_wait_limit": ([I64], I),
+        "lsa_prefill_chunk_queries": ([P, P, P, P, P, P, I64, I64, I64, I64, I, I, I, SelectParams,
+                                       P, SZ, P, P], I),
         "lsa_select_noalloc": ([P, P, P, I64, SelectParams, P, P, I, P], I),
         "lsa_decode_step": ([P, P, P, P, P, P, P, P, P, P, I, I, I, SelectParams, P, SZ, P, P], I),
     }
@@ -316,6 +318,27 @@ def lsa_prefill_chunk(index, latent_K, latent_Q, Q, K, V, T_old, T_new, budget, 
                                   _ptr(V), int(T_old), int(T_new), Hq, Hkv, d,
                                   SelectParams(budget, window, sinks), _ptr(workspace),
                                   workspace.numel(), _ptr(O), _stream(stream)))
+    return O
+
+
+def lsa_prefill_chunk_queries(index, latent_K, latent_Q, Q, K, V, T_old, T_new, q_begin, q_end,
+                              budget, window, sinks, workspace=None, out=None, stream=None):
+    """lsa_prefill_chunk for the chunk's query rows [q_begin, q_end) (positions
+    T_old + q_begin ..); latent_Q, Q and O hold those rows only."""
+    _cuda(latent_K, latent_Q, Q, K, V, out)
+    B, Nq, Hq, d = Q.shape
+    Hkv = K.shape[2]
+    if Nq != q_end - q_begin:
+        raise ValueError("Q holds %d rows, the range %d" % (Nq, q_end - q_begin))
+    if workspace is None:
+        need = lsa_prefill_workspace_bytes(index, Nq, Hq, Hkv, d, budget, window, sinks)
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    O = out if out is not None else torch.empty_like(Q)
+    _check(_lib.lsa_prefill_chunk_queries(index.handle, _ptr(latent_K), _ptr(latent_Q), _ptr(Q),
+                                          _ptr(K), _ptr(V), int(T_old), int(T_new), int(q_begin),
+                                          int(q_end), Hq, Hkv, d,
+                                          SelectParams(budget, window, sinks), _ptr(workspace),
+                                          workspace.numel(), _ptr(O), _stream(stream)))
     return O
 
 

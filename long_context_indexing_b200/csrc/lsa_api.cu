@@ -513,11 +513,10 @@ int64_t lsa_prefill_partial_slots(const lsa_index* idx, int64_t Nq, int Hq, int 
 namespace {
 
 // Checks shared by the prefill entries; fills the layout and the plan view.
-lsa_status prefill_prepare(const lsa_index* idx, int64_t T_old, int64_t T_new, int Hq, int Hkv,
-                           int d, lsa_select_params sp, void* workspace, size_t ws_bytes,
+lsa_status prefill_prepare(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d,
+                           lsa_select_params sp, void* workspace, size_t ws_bytes,
                            PrefillLayout* L, BucketPlan* P)
 {
-    const int64_t Nq = T_new - T_old;
     if (Nq < 1) return fail(LSA_ERR_INVALID_ARG, "empty chunk");
     const int s_max = sp.budget + sp.window + sp.sinks;
     lsa_status s = check_select(idx, sp, s_max);
@@ -560,15 +559,30 @@ lsa_status prefill_prepare(const lsa_index* idx, int64_t T_old, int64_t T_new, i
 
 }  // namespace
 
-lsa_status lsa_prefill_select(lsa_index* idx, const void* latent_K, const void* latent_Q,
-                              int64_t T_old, int64_t T_new, int Hq, int Hkv, int d,
-                              lsa_select_params sp, void* workspace, size_t ws_bytes, void* stream)
+namespace {
+
+// Chunk queries [q0, q1) of positions [T_old, T_new): the query at row r sits
+// at position T_old + q0 + r.
+lsa_status query_range(int64_t T_old, int64_t T_new, int64_t q0, int64_t q1)
+{
+    if (T_old < 0 || T_new <= T_old) return fail(LSA_ERR_INVALID_ARG, "empty chunk");
+    if (q0 < 0 || q1 <= q0 || q1 > T_new - T_old)
+        return fail(LSA_ERR_INVALID_ARG, "query range [%lld, %lld) outside the chunk of %lld",
+                    (long long)q0, (long long)q1, (long long)(T_new - T_old));
+    return LSA_OK;
+}
+
+lsa_status select_part(lsa_index* idx, const void* latent_K, const void* latent_Q, int64_t T_old,
+                       int64_t T_new, int64_t q0, int64_t q1, int Hq, int Hkv, int d,
+                       lsa_select_params sp, void* workspace, size_t ws_bytes, void* stream)
 {
     if (!idx || !latent_K || !latent_Q || !workspace)
         return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    lsa_status s = query_range(T_old, T_new, q0, q1);
+    if (s != LSA_OK) return s;
     PrefillLayout L;
     BucketPlan P;
-    lsa_status s = prefill_prepare(idx, T_old, T_new, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
+    s = prefill_prepare(idx, q1 - q0, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
     if (s != LSA_OK) return s;
     if (!aligned16(latent_Q)) return fail(LSA_ERR_ALIGNMENT, "latent_Q not 16-byte aligned");
     cudaStream_t st = (cudaStream_t)stream;
@@ -576,26 +590,28 @@ lsa_status lsa_prefill_select(lsa_index* idx, const void* latent_K, const void* 
     if (s != LSA_OK) return s;
     char* base = (char*)workspace;
     const int s_max = sp.budget + sp.window + sp.sinks;
-    return run_select(idx, latent_Q, PosSrc{nullptr, T_old}, T_new - T_old, sp,
+    return run_select(idx, latent_Q, PosSrc{nullptr, T_old + q0}, q1 - q0, sp,
                       (int32_t*)(base + L.indices), (int32_t*)(base + L.counts), s_max,
                       base + L.sel, st, L.bucket ? &P : nullptr);
 }
 
-lsa_status lsa_prefill_attend(const lsa_index* idx, const void* Q, const void* K, const void* V,
-                              int64_t T_old, int64_t T_new, int Hq, int Hkv, int d,
-                              lsa_select_params sp, void* workspace, size_t ws_bytes, void* O,
-                              void* stream)
+lsa_status attend_part(const lsa_index* idx, const void* Q, const void* K, const void* V,
+                       int64_t T_old, int64_t T_new, int64_t q0, int64_t q1, int Hq, int Hkv,
+                       int d, lsa_select_params sp, void* workspace, size_t ws_bytes, void* O,
+                       void* stream)
 {
     if (!idx || !Q || !K || !V || !workspace || !O)
         return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    lsa_status s = query_range(T_old, T_new, q0, q1);
+    if (s != LSA_OK) return s;
     PrefillLayout L;
     BucketPlan P;
-    lsa_status s = prefill_prepare(idx, T_old, T_new, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
+    s = prefill_prepare(idx, q1 - q0, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
     if (s != LSA_OK) return s;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
         return fail(LSA_ERR_ALIGNMENT, "Q, K, V and O must be 16-byte aligned");
     cudaStream_t st = (cudaStream_t)stream;
-    const int64_t Nq = T_new - T_old;
+    const int64_t Nq = q1 - q0;
     const int s_max = sp.budget + sp.window + sp.sinks;
     char* base = (char*)workspace;
     const int32_t* indices = (const int32_t*)(base + L.indices);
@@ -604,7 +620,7 @@ lsa_status lsa_prefill_attend(const lsa_index* idx, const void* Q, const void* K
     cudaError_t e;
     if (L.bucket)
         e = launch_bucket_attn(idx->v, idx->n_blk, P, Q, K, V, Nq, Hq, Hkv, d,
-                               PosSrc{nullptr, T_old}, sp.window, sp.sinks, indices, counts,
+                               PosSrc{nullptr, T_old + q0}, sp.window, sp.sinks, indices, counts,
                                s_max, scale, O, st);
     else
         e = launch_attn_status(Q, K, V, idx->v.dtype, idx->v.B, Nq, idx->v.T_cap, Hq, Hkv, d,
@@ -613,25 +629,65 @@ lsa_status lsa_prefill_attend(const lsa_index* idx, const void* Q, const void* K
     return LSA_OK;
 }
 
+lsa_status chunk_part(lsa_index* idx, const void* latent_K, const void* latent_Q, const void* Q,
+                      const void* K, const void* V, int64_t T_old, int64_t T_new, int64_t q0,
+                      int64_t q1, int Hq, int Hkv, int d, lsa_select_params sp, void* workspace,
+                      size_t ws_bytes, void* O, void* stream)
+{
+    if (!idx || !latent_K || !latent_Q || !Q || !K || !V || !workspace || !O)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    lsa_status s = query_range(T_old, T_new, q0, q1);
+    if (s != LSA_OK) return s;
+    PrefillLayout L;
+    BucketPlan P;
+    // every argument check of both halves before the first launch
+    s = prefill_prepare(idx, q1 - q0, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
+    if (s != LSA_OK) return s;
+    if (!aligned16(latent_Q) || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+        return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    s = select_part(idx, latent_K, latent_Q, T_old, T_new, q0, q1, Hq, Hkv, d, sp, workspace,
+                    ws_bytes, stream);
+    if (s != LSA_OK) return s;
+    return attend_part(idx, Q, K, V, T_old, T_new, q0, q1, Hq, Hkv, d, sp, workspace, ws_bytes, O,
+                       stream);
+}
+
+}  // namespace
+
+lsa_status lsa_prefill_select(lsa_index* idx, const void* latent_K, const void* latent_Q,
+                              int64_t T_old, int64_t T_new, int Hq, int Hkv, int d,
+                              lsa_select_params sp, void* workspace, size_t ws_bytes, void* stream)
+{
+    return select_part(idx, latent_K, latent_Q, T_old, T_new, 0, T_new - T_old, Hq, Hkv, d, sp,
+                       workspace, ws_bytes, stream);
+}
+
+lsa_status lsa_prefill_attend(const lsa_index* idx, const void* Q, const void* K, const void* V,
+                              int64_t T_old, int64_t T_new, int Hq, int Hkv, int d,
+                              lsa_select_params sp, void* workspace, size_t ws_bytes, void* O,
+                              void* stream)
+{
+    return attend_part(idx, Q, K, V, T_old, T_new, 0, T_new - T_old, Hq, Hkv, d, sp, workspace,
+                       ws_bytes, O, stream);
+}
+
 lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* latent_Q,
                              const void* Q, const void* K, const void* V, int64_t T_old,
                              int64_t T_new, int Hq, int Hkv, int d, lsa_select_params sp,
                              void* workspace, size_t ws_bytes, void* O, void* stream)
 {
-    if (!idx || !latent_K || !latent_Q || !Q || !K || !V || !workspace || !O)
-        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
-    PrefillLayout L;
-    BucketPlan P;
-    // every argument check of both halves before the first launch
-    lsa_status s = prefill_prepare(idx, T_old, T_new, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
-    if (s != LSA_OK) return s;
-    if (!aligned16(latent_Q) || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
-        return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
-    s = lsa_prefill_select(idx, latent_K, latent_Q, T_old, T_new, Hq, Hkv, d, sp, workspace,
-                           ws_bytes, stream);
-    if (s != LSA_OK) return s;
-    return lsa_prefill_attend(idx, Q, K, V, T_old, T_new, Hq, Hkv, d, sp, workspace, ws_bytes, O,
-                              stream);
+    return chunk_part(idx, latent_K, latent_Q, Q, K, V, T_old, T_new, 0, T_new - T_old, Hq, Hkv,
+                      d, sp, workspace, ws_bytes, O, stream);
+}
+
+lsa_status lsa_prefill_chunk_queries(lsa_index* idx, const void* latent_K, const void* latent_Q,
+                                     const void* Q, const void* K, const void* V, int64_t T_old,
+                                     int64_t T_new, int64_t q_begin, int64_t q_end, int Hq,
+                                     int Hkv, int d, lsa_select_params sp, void* workspace,
+                                     size_t ws_bytes, void* O, void* stream)
+{
+    return chunk_part(idx, latent_K, latent_Q, Q, K, V, T_old, T_new, q_begin, q_end, Hq, Hkv, d,
+                      sp, workspace, ws_bytes, O, stream);
 }
 
 lsa_status lsa_prefill_chunk_host(lsa_index* idx, const void* h_latent_K, const void* h_K,
@@ -647,7 +703,7 @@ lsa_status lsa_prefill_chunk_host(lsa_index* idx, const void* h_latent_K, const 
     if (stream == copy_stream) return fail(LSA_ERR_INVALID_ARG, "copy_stream must differ from stream");
     PrefillLayout L;
     BucketPlan P;
-    lsa_status s = prefill_prepare(idx, T_old, T_new, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
+    lsa_status s = prefill_prepare(idx, T_new - T_old, Hq, Hkv, d, sp, workspace, ws_bytes, &L, &P);
     if (s != LSA_OK) return s;
     if (!aligned16(latent_K) || !aligned16(latent_Q) || !aligned16(Q) || !aligned16(K) ||
         !aligned16(V) || !aligned16(O))

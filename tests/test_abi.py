@@ -146,3 +146,24 @@ def test_wait_hook_without_gpu_fails_cleanly():
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert lsa._lib.lsa_set_wait_limit(0) == 4                           # LSA_ERR_CUDA
+
+
+def test_query_range_entry_argument_checks():
+    # lsa_prefill_chunk_queries refuses an empty or out-of-chunk query range,
+    # a NULL argument and a short workspace before any launch.
+    P = lsa.IndexParams(4, 256, 8, 3)
+    need = lsa._lib.lsa_index_bytes(1, 8192, P, lsa.BF16)
+    h = ctypes.c_void_p()
+    assert lsa._lib.lsa_index_init(ctypes.c_void_p(1 << 20), need, 1, 8192, P, lsa.BF16,
+                                   ctypes.byref(h)) == 0
+    fake = ctypes.c_void_p(1 << 22)
+    S = lsa.SelectParams(512, 64, 4)
+    f = lsa._lib.lsa_prefill_chunk_queries
+    ws = lsa._lib.lsa_prefill_workspace_bytes(h, 32, 8, 2, 64, S)
+    args = [fake] * 6                       # latent_K, latent_Q, Q, K, V (and O below)
+    for q0, q1 in ((10, 10), (-1, 5), (0, 65), (70, 80)):
+        assert f(h, *args[:5], 4096, 4160, q0, q1, 8, 2, 64, S, fake, ws, fake, None) == 1
+        assert b"query range" in lsa._lib.lsa_last_error()
+    assert f(h, None, *args[1:5], 4096, 4160, 0, 32, 8, 2, 64, S, fake, ws, fake, None) == 1
+    assert f(h, *args[:5], 4096, 4160, 0, 32, 8, 2, 64, S, fake, 16, fake, None) == 3
+    lsa._lib.lsa_index_release(h)

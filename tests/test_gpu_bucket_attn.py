@@ -266,3 +266,45 @@ def test_scorer_wait_that_runs_out_reports_a_timeout():
     gpu.check()                          # the status word was cleared by the report
     fb, _ = _run(w, seed=24)
     assert fb == 0
+
+
+@pytest.mark.parametrize("cuts", [(0, 350, 700), (0, 128, 129, 700)])
+def test_query_ranges_equal_the_whole_chunk(cuts):
+    # A chunk that ends inside a block (open-block members are selectable),
+    # split into query ranges with lsa_prefill_chunk_queries: every range
+    # extends the index over the whole chunk, and its rows' selections and
+    # outputs are the whole chunk's, bit for bit.
+    w = _base()
+    T_old = w.T - w.nq
+    inp = synth.prefill_inputs(w, 41, "cpu")
+    dev = {k: v.cuda() for k, v in inp.items()}
+    gpu = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16)
+    gpu.build(dev["latent_K"], T_old)
+    ws = torch.empty(lsa.lsa_prefill_workspace_bytes(gpu, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W, w.S),
+                     dtype=torch.uint8, device="cuda")
+    O = lsa.lsa_prefill_chunk(gpu, dev["latent_K"], dev["latent_Q"], dev["Q"], dev["K"], dev["V"],
+                              T_old, w.T, w.R, w.W, w.S, workspace=ws)
+    g_idx, g_cnt = lsa.prefill_selection_views(ws, w.B, w.nq, w.s_max)
+    g_idx, g_cnt = g_idx.clone(), g_cnt.clone()
+    parts_o, parts_i, parts_c = [], [], []
+    for q0, q1 in zip(cuts[:-1], cuts[1:]):
+        wsp = torch.empty(lsa.lsa_prefill_workspace_bytes(gpu, q1 - q0, w.Hq, w.Hkv, w.d, w.R,
+                                                          w.W, w.S), dtype=torch.uint8,
+                          device="cuda")
+        Op = lsa.lsa_prefill_chunk_queries(gpu, dev["latent_K"],
+                                           dev["latent_Q"][:, q0:q1].contiguous(),
+                                           dev["Q"][:, q0:q1].contiguous(), dev["K"], dev["V"],
+                                           T_old, w.T, q0, q1, w.R, w.W, w.S, workspace=wsp)
+        pi, pc = lsa.prefill_selection_views(wsp, w.B, q1 - q0, w.s_max)
+        parts_o.append(Op)
+        parts_i.append(pi.clone())
+        parts_c.append(pc.clone())
+    torch.cuda.synchronize()
+    assert gpu.check() >= 0
+    assert torch.equal(torch.cat(parts_c, 1), g_cnt)
+    assert torch.equal(torch.cat(parts_i, 1), g_idx)
+    assert torch.equal(torch.cat(parts_o, 1), O)
+    with pytest.raises(lsa.LsaError):
+        lsa.lsa_prefill_chunk_queries(gpu, dev["latent_K"], dev["latent_Q"][:, :10].contiguous(),
+                                      dev["Q"][:, :10].contiguous(), dev["K"], dev["V"], T_old,
+                                      w.T, w.nq - 5, w.nq + 5, w.R, w.W, w.S, workspace=ws)

@@ -74,3 +74,69 @@ def test_reference_arm_under_torchrun_two_ranks():
     j = json.loads(lines[0])
     assert j["impl"] == "reference" and j["n_gpus"] == 2 and j["scaling"] == "weak"
     assert j["value"] > 0 and j["cpu_baseline"]["kind"] == "oracle"
+
+
+def _split_worker(rank, ws, port, q):
+    # One chunk's queries split over two ranks, the oracle standing in for the
+    # GPU on each rank: the gathered rows equal the single-rank chunk.
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(ws), LOCAL_RANK=str(rank), CUDA_VISIBLE_DEVICES="")
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    import oracle
+    import synth
+    r, w = bench._dist(timeout_s=60)
+    wl = synth.workload("tiny", T=2048, nq=64, Hq=4, Hkv=1, d=64, M=16, G=64, k=4, R=200, W=32,
+                        S=4)
+    inp = synth.prefill_inputs(wl, 3, "cpu")                # every rank: the same chunk
+    T_old = wl.T - wl.nq
+    lat = inp["latent_K"][0].numpy()
+    orc = oracle.Index(wl.T, wl.p, wl.G, wl.k, wl.L, rt_bf16=False)
+    orc.extend(lat, 0, wl.T)
+    q0, q1 = bench._query_slice(wl.nq, r, w)
+    pos = T_old + np.arange(q0, q1)
+    sel, cnt, _, _ = oracle.select(orc, inp["latent_Q"][0][q0:q1].numpy(), pos, wl.R, wl.W, wl.S)
+    O, _ = oracle.attend(inp["Q"][0][q0:q1].numpy(), inp["K"][0].numpy(), inp["V"][0].numpy(),
+                         sel, cnt)
+    O_all = bench._gather_rows(torch.from_numpy(O), w)
+    sel_all = bench._gather_rows(torch.from_numpy(sel), w)
+    torch.distributed.destroy_process_group()
+    if r == 0:
+        pos_all = T_old + np.arange(wl.nq)
+        ref_sel, ref_cnt, _, _ = oracle.select(orc, inp["latent_Q"][0].numpy(), pos_all, wl.R,
+                                               wl.W, wl.S)
+        ref_O, _ = oracle.attend(inp["Q"][0].numpy(), inp["K"][0].numpy(), inp["V"][0].numpy(),
+                                 ref_sel, ref_cnt)
+        q.put((bool(np.array_equal(sel_all.numpy(), ref_sel)),
+               bool(np.array_equal(O_all.numpy(), ref_O)), (q0, q1)))
+    else:
+        q.put(None)
+
+
+def test_query_split_over_gloo_matches_the_whole_chunk():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_split_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=240) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    got = [x for x in res if x is not None]
+    assert len(got) == 1
+    same_sel, same_o, rng = got[0]
+    assert same_sel and same_o
+    assert rng == (0, 32)
+
+
+def test_query_slice_ranges():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert [bench._query_slice(32768, r, 4) for r in range(4)] == [
+        (0, 8192), (8192, 16384), (16384, 24576), (24576, 32768)]
+    import pytest
+    with pytest.raises(ValueError):
+        bench._query_slice(10, 0, 3)
