@@ -53,6 +53,9 @@ def _lib():
         lib.orc_select.argtypes = [P, I, P, I64, I64, P, P, P, P, I64, I,
                                    I, I, I, I, I, P, P, P, P]
         lib.orc_select.restype = I
+        lib.orc_tree_select.argtypes = [P, I, P, I64, I64, P, P, P, P, I64, I, I64, P, P, P,
+                                        I, I, I, I, I, I, P, P]
+        lib.orc_tree_select.restype = I
         lib.orc_attend.argtypes = [P, P, P, I64, I64, I, I, I, P, P, I,
                                    ctypes.c_double, P, P]
         lib.orc_attend.restype = I
@@ -223,6 +226,57 @@ def select(index, q, pos, R, W, S, s_max=None):
         _p(index.members), _p(ob), index.n_blocks * index.G, index.G, index.p, R, W, S, s_max,
         _p(out), _p(cnt), _p(mg), _p(nlr)), "select")
     return out, cnt, mg, nlr
+
+
+# --------------------------------------------------------------------------
+# D-LSA Tree [P4 "What it changes": clusters grouped into a hierarchy that a
+# query walks down; P2 multi-level index; P5 Flat vs Tree]
+# --------------------------------------------------------------------------
+
+class Tree:
+    """Level 2 of a two-level D-LSA Tree over one sequence's Flat index.
+
+    READING (the pages give no construction): the closed buckets' fp32
+    centroids are clustered like a block -- spherical k-means (kmeans_block:
+    evenly spaced init, L Lloyd iterations, ties to the lowest id, an empty
+    super-bucket keeps its centroid) -- into n_super super-buckets; each holds
+    the ascending list of its bucket ids (CSR), and its retrieval copy is
+    rounded to bf16 for bf16 indices, as the buckets' is."""
+
+    def __init__(self, index, n_super, L):
+        nb = index.n_buckets
+        if not 1 <= n_super <= nb:
+            raise ValueError("n_super must lie in [1, %d]" % nb)
+        sup, assign, _ = kmeans_block(index.cent[:nb], n_super, L)
+        self.n_super = n_super
+        self.sup = sup
+        self.sup_rt = round_bf16(sup) if index.rt_bf16 else sup.copy()
+        self.assign = assign.astype(np.int32)
+        counts = np.bincount(self.assign, minlength=n_super)
+        self.offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+        self.members = np.argsort(self.assign, kind="stable").astype(np.int32)
+
+
+def tree_select(index, tree, q, pos, branches, R, W, S, s_max=None):
+    """Per query: the `branches` best super-buckets (exact <q, c~2_h>, score
+    desc, lowest id on ties), then the Flat ranking and greedy fill of their
+    buckets only (see select); sinks and window as Flat.
+
+    Returns (indices [nq][s_max] int32, counts [nq] int32)."""
+    q = _f32(q)
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    nq = q.shape[0]
+    if s_max is None:
+        s_max = R + W + S
+    out = np.empty((nq, s_max), np.int32)
+    cnt = np.empty(nq, np.int32)
+    ob = np.ascontiguousarray(index.open_bucket, dtype=np.int32)
+    _check(_lib().orc_tree_select(
+        _p(q), index.dl, _p(pos), nq, index.n_buckets, _p(index.cent_rt), _p(index.offsets),
+        _p(index.members), _p(ob), index.n_blocks * index.G, index.G, tree.n_super,
+        _p(_f32(tree.sup_rt)), _p(tree.offsets), _p(tree.members), int(branches), index.p, R, W,
+        S, s_max, _p(out), _p(cnt)), "tree_select")
+    return out, cnt
 
 
 # --------------------------------------------------------------------------

@@ -467,6 +467,113 @@ int orc_select(const float* q, int dl, const int64_t* pos, int64_t nq, int64_t n
 }
 
 /* ------------------------------------------------------------------------ */
+/* D-LSA Tree retrieval [P4 "What it changes": clusters are grouped into a   */
+/* hierarchy, a query scores a few clusters at each level and walks down;    */
+/* P5 paragraph on Flat vs Tree: a tree search computes less, but a wrong    */
+/* branch can leave useful keys out]                                          */
+/* ------------------------------------------------------------------------ */
+
+/* One query of a two-level tree (READING for the tree's shape: level 2 holds
+ * n_super super-buckets, each a CSR list of bucket ids in ascending order).
+ * The query scores every super-centroid's retrieval copy (exact products,
+ * binary64 sum), walks down the `branches` best (score desc, id asc), and
+ * the buckets of those branches are ranked and filled exactly as Flat ranks
+ * and fills all buckets (orc_select_one): (s desc, g asc), whole buckets
+ * while they fit, the next truncated in ascending position, sinks and window.
+ * Buckets outside the chosen branches are never read. */
+static int orc_tree_select_one(const float* q, int dl, int64_t pos, int64_t n_buckets,
+                               const float* cent_rt, const int32_t* offsets,
+                               const int32_t* members, const int32_t* open_bucket,
+                               int64_t open_j0, int n_open, int64_t n_super,
+                               const float* sup_rt, const int32_t* sup_off,
+                               const int32_t* sup_mem, int branches, int p, int R, int W, int S,
+                               int s_max, orc_rank* rk, orc_rank* rs, int32_t* out,
+                               int32_t* count)
+{
+    for (int64_t h = 0; h < n_super; ++h) {
+        rs[h].s = orc_dot(q, sup_rt + h * dl, dl);
+        rs[h].g = (int32_t)h;
+    }
+    qsort(rs, (size_t)n_super, sizeof(orc_rank), orc_rank_cmp);
+    int64_t nu = 0; /* the chosen branches' buckets */
+    int64_t nb_take = (branches < n_super) ? branches : n_super;
+    for (int64_t r = 0; r < nb_take; ++r) {
+        int32_t h = rs[r].g;
+        for (int32_t x = sup_off[h]; x < sup_off[h + 1]; ++x) {
+            int32_t g = sup_mem[x];
+            if (g < 0 || g >= n_buckets) continue;
+            rk[nu].s = orc_dot(q, cent_rt + (int64_t)g * dl, dl);
+            rk[nu].g = g;
+            ++nu;
+        }
+    }
+    qsort(rk, (size_t)nu, sizeof(orc_rank), orc_rank_cmp);
+
+    int64_t n = 0;
+    int64_t s_end = (S < pos + 1) ? S : pos + 1;
+    for (int64_t t = 0; t < s_end; ++t) out[n++] = (int32_t)t;
+    int64_t rem = R;
+    for (int64_t r = 0; r < nu && rem > 0; ++r) {
+        int32_t g = rk[r].g;
+        int64_t a = orc_avail(g, pos, p, W, S, offsets, members, open_bucket, open_j0, n_open,
+                              NULL, 0);
+        if (a == 0) continue;
+        int64_t take = (a <= rem) ? a : rem;
+        orc_avail(g, pos, p, W, S, offsets, members, open_bucket, open_j0, n_open, out + n, take);
+        n += take;
+        rem -= take;
+    }
+    int64_t w0 = pos - W + 1;
+    if (w0 < s_end) w0 = s_end;
+    for (int64_t t = w0; t <= pos; ++t) out[n++] = (int32_t)t;
+    if (n > s_max) return ORC_EINVAL;
+    for (int64_t x = n; x < s_max; ++x) out[x] = -1;
+    *count = (int32_t)n;
+    return ORC_OK;
+}
+
+/* Tree selection for nq queries of one sequence: the arguments of orc_select
+ * plus the tree (n_super, sup_rt [n_super][dl], sup_off [n_super+1], sup_mem
+ * [sup_off[n_super]]) and the number of branches walked. */
+int orc_tree_select(const float* q, int dl, const int64_t* pos, int64_t nq, int64_t n_buckets,
+                    const float* cent_rt, const int32_t* offsets, const int32_t* members,
+                    const int32_t* open_bucket, int64_t open_j0, int n_open, int64_t n_super,
+                    const float* sup_rt, const int32_t* sup_off, const int32_t* sup_mem,
+                    int branches, int p, int R, int W, int S, int s_max, int32_t* out,
+                    int32_t* count)
+{
+    if (R < 0 || W < 0 || S < 0 || p <= 0 || s_max < 1 || n_buckets < 0 || n_super < 0 ||
+        branches < 0)
+        return ORC_EINVAL;
+    int err = ORC_OK;
+    int64_t n_mem = n_super > 0 ? sup_off[n_super] : 0;
+#pragma omp parallel
+    {
+        orc_rank* rk = (orc_rank*)malloc(sizeof(orc_rank) * (size_t)(n_mem > 0 ? n_mem : 1));
+        orc_rank* rs = (orc_rank*)malloc(sizeof(orc_rank) * (size_t)(n_super > 0 ? n_super : 1));
+        if (!rk || !rs) {
+#pragma omp atomic write
+            err = ORC_ENOMEM;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < nq; ++i) {
+            if (!rk || !rs) continue;
+            int e = orc_tree_select_one(q + i * dl, dl, pos[i], n_buckets, cent_rt, offsets,
+                                        members, open_bucket, open_j0, n_open, n_super, sup_rt,
+                                        sup_off, sup_mem, branches, p, R, W, S, s_max, rk, rs,
+                                        out + i * s_max, count + i);
+            if (e != ORC_OK) {
+#pragma omp atomic write
+                err = e;
+            }
+        }
+        free(rk);
+        free(rs);
+    }
+    return err;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Exact attention over the selected keys [P4 "What it changes": the        */
 /* attention kernel is unchanged; P5 retrieval paragraph]                     */
 /* ------------------------------------------------------------------------ */
