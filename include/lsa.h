@@ -216,6 +216,58 @@ lsa_status lsa_select_noalloc(const lsa_index* idx, const void* latent_Q,
                               int32_t* indices, int32_t* counts, int s_max, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * D-LSA Tree ("Prefrontal's ...", section "What it changes": clusters are
+ * grouped into a hierarchy; a query scores a few clusters at each level, walks
+ * down the tree and only then fetches keys.  "Latent Sparse Attention: un
+ * indice gerarchico per contesti lunghi", paragraph on Flat vs Tree: the tree
+ * computes less, a wrong branch can leave useful keys out.)
+ *
+ * This library's two-level reading: level 2 clusters every sequence's closed
+ * buckets' fp32 centroids into n_super super-buckets exactly as a block's unit
+ * vectors are clustered (init c2_h = c[floor(h * NB / n_super)], lloyd_iters
+ * Lloyd iterations, exact binary64 scores, ties to the lowest id, an empty
+ * super-bucket keeps its centroid); each super-bucket lists its bucket ids in
+ * ascending order, and its retrieval copy is bf16 for bf16 indices.  A query
+ * scores every super-centroid exactly, walks the `branches` best (score desc,
+ * lowest id on ties) and ranks and fills only their buckets, as lsa_select
+ * ranks and fills all of them (same budget, sinks, window, emitted order).
+ * With branches = n_super the selection is lsa_select's.
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of device storage for a tree of n_super super-buckets over idx (0 on
+ * bad arguments). */
+size_t lsa_tree_bytes(const lsa_index* idx, int n_super);
+
+/* Builds the tree over the index's current closed blocks into `tree`
+ * (device, 256-byte aligned, >= lsa_tree_bytes).  Requires at least one
+ * closed block and 1 <= n_super <= closed buckets (and <= 12800).  Rebuild it
+ * after lsa_index_extend: buckets added later belong to no branch. */
+lsa_status lsa_tree_build(const lsa_index* idx, void* tree, size_t bytes, int n_super,
+                          int lloyd_iters, void* stream);
+
+/* Copies the tree to caller DEVICE buffers (any may be NULL): sup
+ * [B][n_super][64] f32 super-centroids, sup_rt [B][n_super][64] retrieval
+ * copy (index dtype), offsets [B][n_super + 1] i32 and members [B][NBK] i32
+ * (bucket ids of super-bucket h at offsets[h] .. offsets[h+1]), NBK being the
+ * index's bucket capacity per sequence. */
+lsa_status lsa_tree_export(const lsa_index* idx, const void* tree, int n_super, float* sup,
+                           void* sup_rt, int32_t* offsets, int32_t* members, void* stream);
+
+/* Workspace bytes for lsa_tree_select on Nq queries per sequence. */
+size_t lsa_tree_select_workspace_bytes(const lsa_index* idx, int64_t Nq, int branches);
+
+/* Tree selection: the arguments of lsa_select plus the tree (built with the
+ * same n_super) and 1 <= branches <= min(n_super, 256).  The candidates of a
+ * query are the chosen branches' buckets; the exact ranking is proved as in
+ * lsa_select, and a query whose proof fails (or whose branches hold more
+ * buckets than the nominator's shared memory) takes an exact fallback over
+ * its chosen branches, counted by lsa_index_check. */
+lsa_status lsa_tree_select(const lsa_index* idx, const void* tree, int n_super, int branches,
+                           const void* latent_Q, const int32_t* positions, int64_t Nq,
+                           lsa_select_params sp, int32_t* indices, int32_t* counts, int s_max,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Exact sparse attention ("Prefrontal's ...", section "What it changes")
  *
  * For query (b, i) and head h with KV head kh = h / (Hq/Hkv):

@@ -20,7 +20,7 @@ __all__ = [
     "LsaError", "LsaIndex", "lsa_index_bytes", "lsa_build_index", "lsa_select",
     "lsa_sparse_attn", "lsa_prefill_chunk", "lsa_prefill_workspace_bytes",
     "lsa_prefill_partial_slots", "lsa_prefill_select", "lsa_prefill_attend",
-    "lsa_prefill_chunk_host", "lsa_prefill_chunk_queries", "set_wait_limit",
+    "lsa_prefill_chunk_host", "lsa_prefill_chunk_queries", "LsaTree", "set_wait_limit",
     "lsa_decode_workspace_bytes", "lsa_decode_step", "lsa_select_noalloc", "library_path", "kernel_launches", "F32",
     "BF16",
 ]
@@ -77,6 +77,11 @@ def _declare(lib):
                                     SelectParams, P, SZ, P, P, P, P], I),
         "lsa_decode_workspace_bytes": ([P, I, I, I, SelectParams], SZ),
         "lsa_set_wait_limit": ([I64], I),
+        "lsa_tree_bytes": ([P, I], SZ),
+        "lsa_tree_build": ([P, P, SZ, I, I, P], I),
+        "lsa_tree_select_workspace_bytes": ([P, I64, I], SZ),
+        "lsa_tree_export": ([P, P, I, P, P, P, P, P], I),
+        "lsa_tree_select": ([P, P, I, I, P, P, I64, SelectParams, P, P, I, P, SZ, P], I),
         "lsa_prefill_chunk_queries": ([P, P, P, P, P, P, I64, I64, I64, I64, I, I, I, SelectParams,
                                        P, SZ, P, P], I),
         "lsa_select_noalloc": ([P, P, P, I64, SelectParams, P, P, I, P], I),
@@ -319,6 +324,61 @@ def lsa_prefill_chunk(index, latent_K, latent_Q, Q, K, V, T_old, T_new, budget, 
                                   SelectParams(budget, window, sinks), _ptr(workspace),
                                   workspace.numel(), _ptr(O), _stream(stream)))
     return O
+
+
+class LsaTree:
+    """Level 2 of a D-LSA Tree over an LsaIndex (C: lsa_tree_build): n_super
+    super-buckets of the index's closed buckets; rebuild after extending the
+    index."""
+
+    def __init__(self, index, n_super, lloyd_iters=3, stream=None):
+        self.index = index
+        self.n_super = int(n_super)
+        n = int(_lib.lsa_tree_bytes(index.handle, self.n_super))
+        if n == 0:
+            raise LsaError(1, "bad tree arguments")
+        self.buffer = torch.empty(n + 256, dtype=torch.uint8, device=index.buffer.device)
+        off = (-self.buffer.data_ptr()) % 256
+        self.view = self.buffer[off:off + n]
+        self.build(lloyd_iters, stream)
+
+    def build(self, lloyd_iters=3, stream=None):
+        _check(_lib.lsa_tree_build(self.index.handle, _ptr(self.view), self.view.numel(),
+                                   self.n_super, int(lloyd_iters), _stream(stream)))
+
+    def export(self, stream=None):
+        """Copies of the tree (C: lsa_tree_export) as torch tensors."""
+        ix = self.index
+        dev = ix.buffer.device
+        rt = torch.bfloat16 if ix.dtype == BF16 else torch.float32
+        out = dict(sup=torch.empty(ix.B, self.n_super, 64, dtype=torch.float32, device=dev),
+                   sup_rt=torch.empty(ix.B, self.n_super, 64, dtype=rt, device=dev),
+                   offsets=torch.empty(ix.B, self.n_super + 1, dtype=torch.int32, device=dev),
+                   members=torch.empty(ix.B, ix.n_buckets_max, dtype=torch.int32, device=dev))
+        _check(_lib.lsa_tree_export(ix.handle, _ptr(self.view), self.n_super, *[
+            _ptr(out[k]) for k in ("sup", "sup_rt", "offsets", "members")], _stream(stream)))
+        return out
+
+    def select(self, latent_Q, positions, branches, budget, window, sinks, s_max=None,
+               workspace=None, stream=None):
+        """Tree selection (C: lsa_tree_select): (indices [B][Nq][s_max], counts [B][Nq])."""
+        _cuda(latent_Q, positions)
+        if positions.dtype != torch.int32:
+            raise TypeError("positions must be int32")
+        B, Nq = latent_Q.shape[0], latent_Q.shape[1]
+        s_max = s_max or (budget + window + sinks)
+        dev = latent_Q.device
+        indices = torch.empty(B, Nq, s_max, dtype=torch.int32, device=dev)
+        counts = torch.empty(B, Nq, dtype=torch.int32, device=dev)
+        need = int(_lib.lsa_tree_select_workspace_bytes(self.index.handle, Nq, int(branches)))
+        if workspace is None or workspace.numel() < need:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        _check(_lib.lsa_tree_select(self.index.handle, _ptr(self.view), self.n_super,
+                                    int(branches), _ptr(latent_Q), _ptr(positions), Nq,
+                                    SelectParams(budget, window, sinks), _ptr(indices),
+                                    _ptr(counts), s_max, _ptr(workspace), workspace.numel(),
+                                    _stream(stream)))
+        return indices, counts
 
 
 def lsa_prefill_chunk_queries(index, latent_K, latent_Q, Q, K, V, T_old, T_new, q_begin, q_end,

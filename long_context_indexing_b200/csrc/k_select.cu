@@ -1503,6 +1503,139 @@ __global__ void __launch_bounds__(DF_THREADS) decode_fill_kernel(IndexView ix, i
 }
 
 // ---------------------------------------------------------------------------
+// D-LSA Tree nomination, one CTA (FILL_THREADS) per query ("Prefrontal's
+// Latent Sparse Attention ...", section "What it changes": the query scores a
+// few clusters at each level and walks down).  1. exact binary64 scores of
+// every super-centroid (retrieval copy), the `branches` best (score desc,
+// lowest id on ties) -- kept per row for the exact fallback; 2. the chosen
+// branches' eligible buckets (the universe) with binary32 approximate scores;
+// 3. the KC largest of them (radix select) are the row's candidate list, tau
+// bounds the rest of the universe (all of it listed: tau = -inf).  A universe
+// larger than the shared-memory area gets an empty list with tau = +inf, so
+// that the fill sends the row to the fallback.  select_fill_kernel then ranks
+// the candidates exactly and fills the budget as Flat does.
+// ---------------------------------------------------------------------------
+constexpr int TREE_MAX_BR = 256;     // branches walked at most
+
+template <typename T>
+__global__ void __launch_bounds__(FILL_THREADS) tree_nominate_kernel(
+    IndexView ix, int64_t n_blk, const T* lq, PosSrc pos, int64_t Nq, int W, SelectWs ws,
+    const T* sup_rt, int64_t NS, int branches, int u_cap)
+{
+    extern __shared__ unsigned char tsm[];
+    double* es2 = reinterpret_cast<double*>(tsm);               // [NS]
+    int32_t* uid = reinterpret_cast<int32_t*>(es2 + NS);        // [u_cap]
+    float* usc = reinterpret_cast<float*>(uid + u_cap);         // [u_cap]
+    __shared__ float q_s[DL];
+    __shared__ int chosen[TREE_MAX_BR];
+    __shared__ int n_u;
+    __shared__ int cand_s[KC];
+    const int64_t b = blockIdx.y, i = blockIdx.x;
+    const int64_t row = b * Nq + i;
+    const int64_t pq = pos.at(b, Nq, i);
+    if (row == 0 && threadIdx.x == 0) *ws.fb_count = 0;
+    if (threadIdx.x == 0) n_u = 0;
+    load_query(q_s, lq, row);
+    __syncthreads();
+    // 1. super-centroids, exact
+    for (int64_t h = threadIdx.x; h < NS; h += FILL_THREADS) {
+        const T* r = sup_rt + (b * NS + h) * DL;
+        double acc = 0.0;
+        for (int d = 0; d < DL; ++d) acc = __fma_rn((double)q_s[d], (double)load_elt(r + d), acc);
+        es2[h] = acc;
+    }
+    __syncthreads();
+    const int nbr = (int)min((int64_t)branches, NS);
+    for (int64_t h = threadIdx.x; h < NS; h += FILL_THREADS) {
+        const double e = es2[h];
+        int r = 0;                             // rank, counted only while it can be < nbr
+        for (int64_t h2 = 0; h2 < NS && r < nbr; ++h2) r += rank_before(es2[h2], (int)h2, e, (int)h);
+        if (r < nbr) {
+            chosen[r] = (int)h;
+            ws.tree_br[row * ws.tree_nbr + r] = (int32_t)h;
+        }
+    }
+    for (int r = nbr + (int)threadIdx.x; r < ws.tree_nbr; r += FILL_THREADS)
+        ws.tree_br[row * ws.tree_nbr + r] = -1;
+    __syncthreads();
+    // 2. the universe: eligible buckets of the chosen branches
+    const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
+    const int32_t* toff = ws.tree_off + b * (NS + 1);
+    const int32_t* tmem = ws.tree_mem + b * ix.NBK;
+    for (int r = 0; r < nbr; ++r) {
+        const int h = chosen[r];
+        for (int32_t x = toff[h] + threadIdx.x; x < toff[h + 1]; x += FILL_THREADS) {
+            const int32_t g = tmem[x];
+            if (g < nb) {
+                const int slot = atomicAdd(&n_u, 1);
+                if (slot < u_cap) uid[slot] = g;
+            }
+        }
+    }
+    __syncthreads();
+    const int nu = n_u;
+    int32_t* cand = ws.lst_g + row * KC;
+    if (nu > u_cap) {                          // too large to rank here: the fallback takes it
+        if (threadIdx.x == 0) {
+            ws.lst_n[row] = 0;
+            ws.lst_tau[row] = INFINITY;
+        }
+        return;
+    }
+    if (nu <= KC) {
+        for (int x = threadIdx.x; x < KC; x += FILL_THREADS) cand[x] = (x < nu) ? uid[x] : -1;
+        if (threadIdx.x == 0) {
+            ws.lst_n[row] = nu;
+            ws.lst_tau[row] = -INFINITY;
+        }
+        return;
+    }
+    // 3. approximate scores of the universe, then its KC best
+    for (int u = threadIdx.x; u < nu; u += FILL_THREADS) {
+        const int64_t g = uid[u];
+        float acc = 0.f;
+        if (ix.dtype == LSA_BF16) {
+            const uint4* r4 = reinterpret_cast<const uint4*>((const __nv_bfloat16*)ix.cent_rt +
+                                                             (b * ix.NBK + g) * DL);
+            uint4 raw[DL / 8];
+#pragma unroll
+            for (int x = 0; x < DL / 8; ++x) raw[x] = __ldg(r4 + x);
+#pragma unroll
+            for (int x = 0; x < DL / 8; ++x) {
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[x]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(h2[e]);
+                    acc = fmaf(q_s[8 * x + 2 * e], f.x, acc);
+                    acc = fmaf(q_s[8 * x + 2 * e + 1], f.y, acc);
+                }
+            }
+        } else {
+            const float4* r4 = reinterpret_cast<const float4*>((const float*)ix.cent_rt +
+                                                               (b * ix.NBK + g) * DL);
+            float4 f[DL / 4];
+#pragma unroll
+            for (int x = 0; x < DL / 4; ++x) f[x] = __ldg(r4 + x);
+#pragma unroll
+            for (int x = 0; x < DL / 4; ++x) {
+                acc = fmaf(q_s[4 * x], f[x].x, acc);
+                acc = fmaf(q_s[4 * x + 1], f[x].y, acc);
+                acc = fmaf(q_s[4 * x + 2], f[x].z, acc);
+                acc = fmaf(q_s[4 * x + 3], f[x].w, acc);
+            }
+        }
+        usc[u] = acc;
+    }
+    __syncthreads();
+    const float tau = radix_top_kc(usc, nu, cand_s);
+    for (int x = threadIdx.x; x < KC; x += FILL_THREADS) cand[x] = uid[cand_s[x]];
+    if (threadIdx.x == 0) {
+        ws.lst_n[row] = KC;
+        ws.lst_tau[row] = tau;
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Exact fallback: persistent CTAs walk the list of flagged queries.  Every
 // eligible bucket gets its exact binary64 score; the fill repeatedly takes the
 // best remaining bucket (score desc, lowest id) until the budget is met.
@@ -1535,7 +1668,23 @@ __global__ void __launch_bounds__(FB_THREADS) select_fallback_kernel(IndexView i
         __syncthreads();
         load_query(q_s, lq, row);
         __syncthreads();
-        for (int64_t g = threadIdx.x; g < nb; g += FB_THREADS) sc[g] = exact_score(ix, b, g, q_s);
+        if (!ws.tree_br) {
+            for (int64_t g = threadIdx.x; g < nb; g += FB_THREADS) sc[g] = exact_score(ix, b, g, q_s);
+        } else {
+            // D-LSA Tree: only the buckets of the row's chosen branches compete
+            for (int64_t g = threadIdx.x; g < nb; g += FB_THREADS) sc[g] = -INFINITY;
+            __syncthreads();
+            const int32_t* toff = ws.tree_off + b * (ws.tree_ns + 1);
+            const int32_t* tmem = ws.tree_mem + b * ix.NBK;
+            for (int r = 0; r < ws.tree_nbr; ++r) {
+                const int h = ws.tree_br[row * ws.tree_nbr + r];
+                if (h < 0) continue;
+                for (int32_t x = toff[h] + threadIdx.x; x < toff[h + 1]; x += FB_THREADS) {
+                    const int32_t g = tmem[x];
+                    if (g < nb) sc[g] = exact_score(ix, b, g, q_s);
+                }
+            }
+        }
         FillCtx f;
         f.ix = ix;
         f.bseq = b;
@@ -1911,9 +2060,9 @@ bool select_uses_tc(const IndexView& ix, int64_t Nq)
 
 // Candidate lists per row: one per tensor-core split, or one of KC from the
 // SIMT nominator.
-static void list_shape(const IndexView& ix, int64_t Nq, int* n_lst, int* cap)
+static void list_shape(const IndexView& ix, int64_t Nq, int* n_lst, int* cap, bool one_list = false)
 {
-    if (select_uses_tc(ix, Nq)) {
+    if (!one_list && select_uses_tc(ix, Nq)) {
         *n_lst = tc_split_plan(ix, Nq).n_split;
         *cap = TC_LIST_CAP;
     } else {
@@ -1923,28 +2072,32 @@ static void list_shape(const IndexView& ix, int64_t Nq, int* n_lst, int* cap)
 }
 
 // Group maxima per row of the tensor-core path (0 otherwise).
-static int64_t n_grp_of(const IndexView& ix, int64_t Nq)
+static int64_t n_grp_of(const IndexView& ix, int64_t Nq, bool one_list = false)
 {
-    return select_uses_tc(ix, Nq) ? tc_split_plan(ix, Nq).n_grp : 0;
+    return (!one_list && select_uses_tc(ix, Nq)) ? tc_split_plan(ix, Nq).n_grp : 0;
 }
 
-size_t select_ws_bytes(const IndexView& ix, int64_t Nq)
+// one_list: a single list of KC candidates per row (SIMT-style nominators:
+// the tree's), whatever the tensor-core scorer would use.
+static size_t ws_bytes_shape(const IndexView& ix, int64_t Nq, bool one_list)
 {
     const size_t rows = (size_t)ix.B * (size_t)Nq;
     int nl, cap;
-    list_shape(ix, Nq, &nl, &cap);
-    const size_t ng = (size_t)n_grp_of(ix, Nq);
+    list_shape(ix, Nq, &nl, &cap, one_list);
+    const size_t ng = (size_t)n_grp_of(ix, Nq, one_list);
     size_t n = al256(rows * nl * cap * 4) + al256(rows * nl * 4) + al256(rows * nl * 4) +
                al256(rows * 4) + al256(4) + al256((size_t)FB_CTAS * (size_t)ix.NBK * 8);
     if (ng) n += al256(rows * ng * 2) + al256(rows * 4);
     return n;
 }
 
-SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
+size_t select_ws_bytes(const IndexView& ix, int64_t Nq) { return ws_bytes_shape(ix, Nq, false); }
+
+static SelectWs carve_shape(void* ws, const IndexView& ix, int64_t Nq, bool one_list)
 {
     const size_t rows = (size_t)ix.B * (size_t)Nq;
     int nl, cap;
-    list_shape(ix, Nq, &nl, &cap);
+    list_shape(ix, Nq, &nl, &cap, one_list);
     char* p = (char*)ws;
     SelectWs w;
     w.n_lst = nl;
@@ -1966,7 +2119,12 @@ SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
     w.dl_n = nullptr;
     w.dl_tau = nullptr;
     w.n_slice = 0;
-    w.n_grp = n_grp_of(ix, Nq);
+    w.tree_br = nullptr;
+    w.tree_off = nullptr;
+    w.tree_mem = nullptr;
+    w.tree_nbr = 0;
+    w.tree_ns = 0;
+    w.n_grp = n_grp_of(ix, Nq, one_list);
     w.gmax = nullptr;
     w.theta = nullptr;
     if (w.n_grp) {
@@ -1981,6 +2139,11 @@ SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
     w.app_slot = nullptr;
     w.app_n = 0;
     return w;
+}
+
+SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq)
+{
+    return carve_shape(ws, ix, Nq, false);
 }
 
 cudaError_t launch_score_lists_tc(const IndexView& ix, int64_t n_blk, const void* latent_Q,
@@ -2072,6 +2235,64 @@ static cudaError_t launch_decode_finish_t(const IndexView& ix, int64_t n_blk, co
                                                                 s_max, indices, counts, ws);
     note_launch();
     return cudaGetLastError();
+}
+
+static int tree_u_cap(const IndexView& ix, int64_t NS, int branches)
+{
+    // room for the chosen branches' buckets: four times the mean branch size
+    // per branch (larger universes take the exact fallback), within what
+    // shared memory holds after the super scores
+    const int64_t mean = (ix.NBK + NS - 1) / NS;
+    int64_t cap = 4 * mean * branches + KC;
+    const int64_t avail = (200 * 1024 - NS * 8) / 8;
+    if (cap > avail) cap = avail;
+    if (cap > ix.NBK) cap = ix.NBK;
+    return (int)(cap < 0 ? 0 : cap);
+}
+
+size_t tree_select_ws_bytes(const IndexView& ix, int64_t Nq, int branches)
+{
+    return ws_bytes_shape(ix, Nq, true) + al256((size_t)ix.B * Nq * branches * 4);
+}
+
+template <typename T>
+static cudaError_t launch_tree_t(const IndexView& ix, int64_t n_blk, const void* tree_buf,
+                                 int64_t NS, int branches, const T* lq, const int32_t* positions,
+                                 int64_t Nq, lsa_select_params sp, int32_t* indices,
+                                 int32_t* counts, int s_max, void* ws_buf, cudaStream_t st)
+{
+    SelectWs ws = carve_shape(ws_buf, ix, Nq, true);
+    ws.tree_br = (int32_t*)((char*)ws_buf + ws_bytes_shape(ix, Nq, true));
+    ws.tree_nbr = branches;
+    ws.tree_ns = NS;
+    const void* sup_rt;
+    tree_select_arrays(ix, tree_buf, NS, &sup_rt, &ws.tree_off, &ws.tree_mem);
+    const int u_cap = tree_u_cap(ix, NS, branches);
+    const size_t smem = (size_t)NS * 8 + (size_t)u_cap * 8;
+    cudaError_t e = ensure_smem_attr((const void*)tree_nominate_kernel<T>, 200 * 1024);
+    if (e != cudaSuccess) return e;
+    const PosSrc pos{positions, 0};
+    tree_nominate_kernel<T><<<dim3((unsigned)Nq, (unsigned)ix.B), FILL_THREADS, smem, st>>>(
+        ix, n_blk, lq, pos, Nq, sp.window, ws, (const T*)sup_rt, NS, branches, u_cap);
+    note_launch();
+    return launch_finish_t(ix, n_blk, lq, pos, Nq, sp, indices, counts, s_max, ws, st);
+}
+
+cudaError_t launch_tree_select(const IndexView& ix, int64_t n_blk, const void* tree_buf,
+                               int64_t NS, int branches, const void* latent_Q,
+                               const int32_t* positions, int64_t Nq, lsa_select_params sp,
+                               int32_t* indices, int32_t* counts, int s_max, void* ws,
+                               cudaStream_t st)
+{
+    if (Nq <= 0) return cudaSuccess;
+    if (branches < 1 || branches > TREE_MAX_BR || NS < 1 || NS * 8 > 100 * 1024 ||
+        tree_u_cap(ix, NS, branches) < (ix.NBK < KC ? ix.NBK : KC))
+        return cudaErrorInvalidValue;
+    if (ix.dtype == LSA_BF16)
+        return launch_tree_t(ix, n_blk, tree_buf, NS, branches, (const __nv_bfloat16*)latent_Q,
+                             positions, Nq, sp, indices, counts, s_max, ws, st);
+    return launch_tree_t(ix, n_blk, tree_buf, NS, branches, (const float*)latent_Q, positions,
+                         Nq, sp, indices, counts, s_max, ws, st);
 }
 
 cudaError_t launch_decode_finish(const IndexView& ix, int64_t n_blk, const void* latent_q,

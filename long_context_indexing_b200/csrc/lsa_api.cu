@@ -471,6 +471,90 @@ lsa_status lsa_select(const lsa_index* idx, const void* latent_Q, const int32_t*
                       (cudaStream_t)stream);
 }
 
+// ---- D-LSA Tree ----
+
+namespace {
+lsa_status check_tree(const lsa_index* idx, int n_super)
+{
+    if (!idx) return fail(LSA_ERR_INVALID_ARG, "NULL index");
+    const int64_t nb = idx->n_blk * idx->v.k;
+    if (idx->n_blk < 1) return fail(LSA_ERR_INVALID_ARG, "the index has no closed block");
+    if (n_super < 1 || n_super > nb)
+        return fail(LSA_ERR_INVALID_ARG, "n_super %d outside [1, %lld]", n_super, (long long)nb);
+    if ((int64_t)n_super * 8 > 100 * 1024)
+        return fail(LSA_ERR_UNSUPPORTED, "n_super %d above the 12800 super-buckets supported",
+                    n_super);
+    return LSA_OK;
+}
+}  // namespace
+
+size_t lsa_tree_bytes(const lsa_index* idx, int n_super)
+{
+    if (!idx || n_super < 1) return 0;
+    return tree_bytes(idx->v, n_super);
+}
+
+lsa_status lsa_tree_build(const lsa_index* idx, void* tree, size_t bytes, int n_super,
+                          int lloyd_iters, void* stream)
+{
+    lsa_status s = check_tree(idx, n_super);
+    if (s != LSA_OK) return s;
+    if (!tree) return fail(LSA_ERR_INVALID_ARG, "NULL tree buffer");
+    if (lloyd_iters < 1) return fail(LSA_ERR_INVALID_ARG, "lloyd_iters < 1");
+    if (((uintptr_t)tree & 255) != 0) return fail(LSA_ERR_ALIGNMENT, "tree buffer not 256-byte aligned");
+    if (bytes < tree_bytes(idx->v, n_super))
+        return fail(LSA_ERR_WORKSPACE, "tree buffer %zu < %zu bytes", bytes,
+                    tree_bytes(idx->v, n_super));
+    cudaError_t e = launch_tree_build(idx->v, idx->n_blk, tree, n_super, lloyd_iters,
+                                      (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tree build");
+    return LSA_OK;
+}
+
+lsa_status lsa_tree_export(const lsa_index* idx, const void* tree, int n_super, float* sup,
+                           void* sup_rt, int32_t* offsets, int32_t* members, void* stream)
+{
+    if (!idx || !tree || n_super < 1) return fail(LSA_ERR_INVALID_ARG, "NULL argument or n_super < 1");
+    cudaError_t e = tree_export(idx->v, tree, n_super, sup, sup_rt, offsets, members,
+                                (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tree export");
+    return LSA_OK;
+}
+
+size_t lsa_tree_select_workspace_bytes(const lsa_index* idx, int64_t Nq, int branches)
+{
+    if (!idx || Nq < 0 || branches < 1) return 0;
+    return tree_select_ws_bytes(idx->v, Nq, branches);
+}
+
+lsa_status lsa_tree_select(const lsa_index* idx, const void* tree, int n_super, int branches,
+                           const void* latent_Q, const int32_t* positions, int64_t Nq,
+                           lsa_select_params sp, int32_t* indices, int32_t* counts, int s_max,
+                           void* workspace, size_t ws_bytes, void* stream)
+{
+    lsa_status s = check_tree(idx, n_super);
+    if (s != LSA_OK) return s;
+    if (!tree || !latent_Q || !positions || !indices || !counts || !workspace)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    if (branches < 1 || branches > 256 || branches > n_super)
+        return fail(LSA_ERR_INVALID_ARG, "branches %d outside [1, min(n_super, 256)]", branches);
+    if (Nq < 0 || Nq > 2147483647LL) return fail(LSA_ERR_INVALID_ARG, "Nq out of range");
+    s = check_select(idx, sp, s_max);
+    if (s != LSA_OK) return s;
+    if (((uintptr_t)tree & 255) != 0) return fail(LSA_ERR_ALIGNMENT, "tree buffer not 256-byte aligned");
+    if (!aligned16(latent_Q) || !aligned16(positions) || !aligned16(indices) ||
+        !aligned16(counts) || !aligned16(workspace))
+        return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    const size_t need = tree_select_ws_bytes(idx->v, Nq, branches);
+    if (ws_bytes < need) return fail(LSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+    if (Nq == 0) return LSA_OK;
+    cudaError_t e = launch_tree_select(idx->v, idx->n_blk, tree, n_super, branches, latent_Q,
+                                       positions, Nq, sp, indices, counts, s_max, workspace,
+                                       (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tree select");
+    return LSA_OK;
+}
+
 lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtype dtype, int64_t B,
                            int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
                            const int32_t* indices, const int32_t* counts, int s_max, float scale,

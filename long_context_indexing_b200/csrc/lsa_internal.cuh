@@ -154,6 +154,14 @@ struct SelectWs {
     int32_t* dl_n;
     float* dl_tau;
     int n_slice;
+    // D-LSA Tree: the rows' chosen branches ([rows][tree_nbr] super-bucket ids)
+    // and the tree's CSR ([B][tree_ns + 1] offsets, [B][NBK] members); when
+    // set, the exact fallback ranks only the chosen branches' buckets.
+    int32_t* tree_br;
+    const int32_t* tree_off;
+    const int32_t* tree_mem;
+    int tree_nbr;
+    int64_t tree_ns;
     int32_t* fb_list;    // [B*Nq]      queries that need the exact fallback
     int32_t* fb_count;   // [1]
     double* fb_scores;   // [FB_CTAS][NBK] scratch of the fallback
@@ -194,6 +202,24 @@ SelectWs select_ws_carve(void* ws, const IndexView& ix, int64_t Nq);
 cudaError_t launch_select(const IndexView& ix, int64_t n_blk, const void* latent_Q, PosSrc pos,
                           int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
                           int s_max, const SelectWs& ws, bool use_tc, cudaStream_t st);
+
+// D-LSA Tree (k_tree.cu): storage bytes, build over the n_blk closed blocks,
+// and the arrays the selection reads.
+size_t tree_bytes(const IndexView& ix, int64_t NS);
+cudaError_t launch_tree_build(const IndexView& ix, int64_t n_blk, void* buf, int64_t NS, int L,
+                              cudaStream_t st);
+void tree_select_arrays(const IndexView& ix, const void* buf, int64_t NS, const void** sup_rt,
+                        const int32_t** off, const int32_t** mem);
+cudaError_t tree_export(const IndexView& ix, const void* buf, int64_t NS, float* sup,
+                        void* sup_rt, int32_t* off, int32_t* mem, cudaStream_t st);
+// Tree selection: workspace bytes and the launch (nominate over the chosen
+// branches, exact fill, exact fallback restricted to the branches).
+size_t tree_select_ws_bytes(const IndexView& ix, int64_t Nq, int branches);
+cudaError_t launch_tree_select(const IndexView& ix, int64_t n_blk, const void* tree_buf,
+                               int64_t NS, int branches, const void* latent_Q,
+                               const int32_t* positions, int64_t Nq, lsa_select_params sp,
+                               int32_t* indices, int32_t* counts, int s_max, void* ws,
+                               cudaStream_t st);
 
 // Decode: exact fill + emission from the slices' sorted lists, then the
 // exact fallback (one query per sequence).
