@@ -337,8 +337,11 @@ lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* l
  * every caller that runs it on the same keys holds the same index -- and only
  * the range's queries are selected and attended.  latent_Q [B][n][64], Q and
  * O [B][n][Hq][d] with n = q_end - q_begin; the workspace is sized by
- * lsa_prefill_workspace_bytes(idx, n, ...).  Each query's selection and
- * output are those lsa_prefill_chunk gives it over the whole chunk.
+ * lsa_prefill_workspace_bytes(idx, n, ...).  Each query's selection is the
+ * one lsa_prefill_chunk gives it over the whole chunk, bit for bit; its output
+ * equals that one up to the order of the softmax sums (a tile of sinks and
+ * windows spans a run of consecutive queries, and a range boundary can cut a
+ * run).
  * Requires 0 <= q_begin < q_end <= T_new - T_old; fails like
  * lsa_prefill_chunk otherwise. */
 lsa_status lsa_prefill_chunk_queries(lsa_index* idx, const void* latent_K, const void* latent_Q,

@@ -272,8 +272,10 @@ def test_scorer_wait_that_runs_out_reports_a_timeout():
 def test_query_ranges_equal_the_whole_chunk(cuts):
     # A chunk that ends inside a block (open-block members are selectable),
     # split into query ranges with lsa_prefill_chunk_queries: every range
-    # extends the index over the whole chunk, and its rows' selections and
-    # outputs are the whole chunk's, bit for bit.
+    # extends the index over the whole chunk; its rows' selections are the
+    # whole chunk's bit for bit, and their outputs equal the whole chunk's up
+    # to summation order (a sinks-and-window tile spans a run of consecutive
+    # queries, so a cut through a run changes its stages): the bf16 bars.
     w = _base()
     T_old = w.T - w.nq
     inp = synth.prefill_inputs(w, 41, "cpu")
@@ -303,7 +305,8 @@ def test_query_ranges_equal_the_whole_chunk(cuts):
     assert gpu.check() >= 0
     assert torch.equal(torch.cat(parts_c, 1), g_cnt)
     assert torch.equal(torch.cat(parts_i, 1), g_idx)
-    assert torch.equal(torch.cat(parts_o, 1), O)
+    err = (torch.cat(parts_o, 1).float() - O.float()).abs()
+    assert err.max().item() <= BF16_MAX and err.mean().item() <= BF16_MEAN
     with pytest.raises(lsa.LsaError):
         lsa.lsa_prefill_chunk_queries(gpu, dev["latent_K"], dev["latent_Q"][:, :10].contiguous(),
                                       dev["Q"][:, :10].contiguous(), dev["K"], dev["V"], T_old,
