@@ -466,6 +466,8 @@ def run_lsa(args, rank, ws):
     _barrier(ws)
     e2e_ms = _max_over_ranks(_events_time(e2e_step, args.steps, stream), ws)
 
+    tree = None if args.tree_super <= 0 else _tree_measure(args, w, inp, idx, T_old, stream)
+
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
@@ -498,9 +500,59 @@ def run_lsa(args, rank, ws):
             "gpu_launches": launches, "clocks": clocks,
             "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "index_build_prefix_s": round(build_s, 3), "selection_fallbacks": fallbacks,
-            "decode": decode}
+            "tree": tree, "decode": decode}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def _tree_measure(args, w, inp, idx, T_old, stream):
+    """D-LSA Tree beside Flat on the chunk's index (covering all T tokens):
+    level-2 build time, tree selection of the chunk's queries against Flat
+    selection (lsa_select) of the same queries, and on a row sample the share
+    of Flat's long-range keys that the tree's walk also keeps."""
+    import long_context_indexing_b200 as lsa
+
+    pos = torch.arange(T_old, w.T, dtype=torch.int32, device="cuda")
+    pos = pos[None].expand(w.B, -1).contiguous()
+    s_max = w.R + w.W + w.S
+    lq = inp["latent_Q"]
+    t_ws = torch.empty(lsa.lsa_tree_select_workspace_bytes(idx, w.nq, args.tree_branches),
+                       dtype=torch.uint8, device="cuda")
+    f_ws = torch.empty(lsa.lsa_select_workspace_bytes(idx, w.nq), dtype=torch.uint8,
+                       device="cuda")
+    tr = lsa.LsaTree(idx, args.tree_super, w.L)
+    build_ms = _events_time(lambda: tr.build(w.L), 3, stream)
+    idx.check()
+    tree_sel = lambda: tr.select(lq, pos, args.tree_branches, w.R, w.W, w.S, s_max, t_ws)
+    flat_sel = lambda: lsa.lsa_select(idx, lq, pos, w.R, w.W, w.S, s_max, f_ws)
+    for _ in range(3):
+        tree_sel()
+        flat_sel()
+    idx.check()
+    t_ms = _events_time(tree_sel, args.steps, stream)
+    fb_tree = idx.check()
+    f_ms = _events_time(flat_sel, args.steps, stream)
+    t_idx, t_cnt = tree_sel()
+    f_idx, f_cnt = flat_sel()
+    rows = _sample_rows(w, 256, "cuda")
+    kept = tot = 0
+    for b in range(w.B):
+        for r in rows.tolist():
+            p = T_old + r
+            lo, hi = w.S, p - w.W                     # long-range key positions
+            fr = f_idx[b, r, :int(f_cnt[b, r])]
+            tr_ = t_idx[b, r, :int(t_cnt[b, r])]
+            fr = fr[(fr >= lo) & (fr <= hi)]
+            tr_ = tr_[(tr_ >= lo) & (tr_ <= hi)]
+            tot += fr.numel()
+            kept += int(torch.isin(fr, tr_).sum())
+    n_buckets = idx.n_buckets_max
+    return {"n_super": args.tree_super, "branches": args.tree_branches, "lloyd_iters": w.L,
+            "index_buckets": n_buckets, "level2_build_ms": round(build_ms, 4),
+            "select_ms": round(t_ms, 4), "flat_select_ms": round(f_ms, 4),
+            "select_fallbacks": fb_tree,
+            "flat_long_range_keys_kept": round(kept / max(tot, 1), 4),
+            "recall_sample": "%d rows (every %d-th) of the chunk" % (len(rows), w.nq // len(rows))}
 
 
 # ------------------------------------------------------------------- decode --
@@ -658,6 +710,10 @@ def main():
     ap.add_argument("--ref-queries", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--tree-super", type=int, default=256,
+                    help="D-LSA Tree beside Flat: super-buckets of level 2 (0: skip)")
+    ap.add_argument("--tree-branches", type=int, default=16,
+                    help="D-LSA Tree beside Flat: super-buckets a query walks")
     ap.add_argument("--decode-T", type=int, default=None,
                     help="override the decode context length (a multiple of p * block)")
     ap.add_argument("--split", choices=["chunks", "queries"], default="chunks",

@@ -18,6 +18,7 @@ import torch
 
 __all__ = [
     "LsaError", "LsaIndex", "lsa_index_bytes", "lsa_build_index", "lsa_select",
+    "lsa_select_workspace_bytes", "lsa_tree_select_workspace_bytes",
     "lsa_sparse_attn", "lsa_prefill_chunk", "lsa_prefill_workspace_bytes",
     "lsa_prefill_partial_slots", "lsa_prefill_select", "lsa_prefill_attend",
     "lsa_prefill_chunk_host", "lsa_prefill_chunk_queries", "LsaTree", "set_wait_limit",
@@ -238,6 +239,16 @@ def lsa_build_index(latent_K, T, p, block, n_buckets, lloyd_iters=3, T_cap=None,
     idx = LsaIndex(B, T_cap or cap, p, block, n_buckets, lloyd_iters, _dtype_code(latent_K),
                    latent_K.device)
     return idx.build(latent_K, T, stream)
+
+
+def lsa_select_workspace_bytes(index, Nq):
+    """Workspace bytes lsa_select needs for Nq queries per sequence."""
+    return int(_lib.lsa_select_workspace_bytes(index.handle, int(Nq)))
+
+
+def lsa_tree_select_workspace_bytes(index, Nq, branches):
+    """Workspace bytes lsa_tree_select needs for Nq queries and `branches`."""
+    return int(_lib.lsa_tree_select_workspace_bytes(index.handle, int(Nq), int(branches)))
 
 
 def lsa_select(index, latent_Q, positions, budget, window, sinks, s_max=None, workspace=None,
