@@ -13,7 +13,7 @@
 //   O += P V     M = 128, N = d, K = 64 keys      (A = P read from TMEM; TMEM,
 //                                                 two accumulators)
 //
-// Warp roles (15 warps):
+// Warp roles (16 warps):
 //   warp 0     planner: claims work items (two ahead) and copies each tile's
 //              description (bucket_tile_records_kernel) and member lists into
 //              shared memory, prefetched to registers one item ahead;
@@ -21,7 +21,9 @@
 //              head (16 keys per warp) with 16-byte cp.async into
 //              128-byte-swizzled planes (the layout the MMA descriptors name);
 //              completion lands on mbarriers;
-//   warp 3     allocates TMEM; lane 0 issues all MMAs and commits;
+//   warp 3     allocates TMEM; lane 0 issues the S MMAs and their commits;
+//   warp 15    lane 0 issues the P V MMAs and their commits (its own thread,
+//              so a P V is never queued behind the issue of later S MMAs);
 //   warp 12    Q loader: the tile's Q rows, as soon as its Q buffer is free;
 //   warps 4-7  softmax: thread = row = TMEM lane; reads its 64 scores of a
 //              stage, masks keys outside its query's ranges, keeps the
@@ -51,15 +53,20 @@ namespace lsa {
 constexpr int TB_M = 128;            // MMA rows: BA_Q queries x 8 query heads
 constexpr int TB_N = 64;             // keys per stage
 constexpr int TB_OPEN_MAX = 2048;    // members of one bucket a tile can hold (block size bound)
-constexpr int TB_SB = 3;             // S buffers in TMEM: S runs up to two stages ahead of P V
+#ifndef LSA_TB_SB
+#define LSA_TB_SB 3
+#endif
+constexpr int TB_SB = LSA_TB_SB;     // S buffers in TMEM: S runs up to TB_SB - 1 stages ahead of P V
 constexpr uint32_t TB_COL_O = TB_SB * 64;   // first TMEM column of the two O accumulators
+static_assert(TB_COL_O + 256 <= 512, "TMEM: S buffers and two O accumulators in 512 columns");
 #ifndef LSA_TB_LOADERS
 #define LSA_TB_LOADERS 4     // K/V loader warps (2 or 4)
 #endif
 constexpr int TB_NL = LSA_TB_LOADERS;
 static_assert(TB_NL == 2 || TB_NL == 4, "K/V loader warps");
 constexpr int TB_KPW = 64 / TB_NL;                // keys of a stage per loader warp
-constexpr int TB_THREADS = 32 * (11 + TB_NL);     // 15 warps with four loaders
+constexpr int TB_PVW = 11 + TB_NL;                // the P V MMA issuer's warp
+constexpr int TB_THREADS = 32 * (12 + TB_NL);     // 16 warps with four loaders
 constexpr uint32_t TB_WAIT = 1u << 22;
 
 // Polls each bounded wait of the tile kernel's roles makes before it gives up
@@ -86,7 +93,7 @@ struct TbCfg {
     static constexpr int OFF_Q = 0;                     // QB buffers
     static constexpr int OFF_KV = OFF_Q + QB * Q_BYTES; // NS stages
     static constexpr int OFF_BAR = OFF_KV + NS * STAGE;
-    static constexpr int NBAR = 25 + 2 * NS;
+    static constexpr int NBAR = 16 + 3 * TB_SB + 2 * NS;
     static constexpr int OFF_ML = OFF_BAR + NBAR * 8;      // [2][128] (max, sum) per row
     static constexpr int OFF_LISTS = OFF_ML + 2 * TB_M * 8;   // then 4 member lists of G ints
     // dynamic shared memory for a block of G pooled groups (+ alignment slack)
@@ -236,14 +243,14 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     uint64_t* info_empty = bars + 2;     // [2]
     uint64_t* q_full = bars + 4;         // [2]
     uint64_t* q_empty = bars + 6;        // [2]
-    uint64_t* s_full = bars + 8;         // [TB_SB]
-    uint64_t* s_empty = bars + 11;       // [TB_SB] (committed after the buffer's P V)
-    uint64_t* p_full = bars + 14;        // [TB_SB]
-    uint64_t* o_full = bars + 17;        // [2] (two O accumulators, by item parity)
-    uint64_t* o_empty = bars + 19;       // [2]
-    uint64_t* ml_full = bars + 21;       // [2]
-    uint64_t* ml_empty = bars + 23;      // [2]
-    uint64_t* kv_full = bars + 25;       // [NS]
+    uint64_t* s_full = bars + 8;                    // [TB_SB]
+    uint64_t* s_empty = s_full + TB_SB;             // [TB_SB] (committed after the buffer's P V)
+    uint64_t* p_full = s_empty + TB_SB;             // [TB_SB]
+    uint64_t* o_full = p_full + TB_SB;              // [2] (two O accumulators, by item parity)
+    uint64_t* o_empty = o_full + 2;                 // [2]
+    uint64_t* ml_full = o_empty + 2;                // [2]
+    uint64_t* ml_empty = ml_full + 2;               // [2]
+    uint64_t* kv_full = ml_empty + 2;               // [NS]
     float2* ml = reinterpret_cast<float2*>(smem + C::OFF_ML);   // [2][TB_M]
     uint64_t* kv_empty = kv_full + NS;
     const int lcap = (a.ix.G + 3) & ~3;  // ints per member list
@@ -256,6 +263,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     __shared__ volatile int abort_flag;
     __shared__ int cnt_s[1];
     __shared__ uint64_t fin_bar;
+    __shared__ uint64_t fin_bar2;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const IndexView& ix = a.ix;
@@ -266,7 +274,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&info_full[i], 1);
-            ptx::mbar_init(&info_empty[i], 10 + TB_NL);   // 4 softmax, 4 epilogue, MMA, K/V loaders, Q loader
+            ptx::mbar_init(&info_empty[i], 11 + TB_NL);   // 4 softmax, 4 epilogue, 2 MMA issuers, K/V loaders, Q loader
             ptx::mbar_init(&o_full[i], 1);
             ptx::mbar_init(&o_empty[i], 4);
             ptx::mbar_init(&ml_full[i], 4);
@@ -284,6 +292,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             ptx::mbar_init(&kv_empty[s], 1);
         }
         ptx::mbar_init(&fin_bar, 1);
+        ptx::mbar_init(&fin_bar2, 1);
         abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -435,7 +444,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
             if (lane == 0) ptx::mbar_arrive(&info_empty[ib]);   // done with ti[ib]
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
-    } else if (warp < 3 || warp >= 13) {
+    } else if (warp < 3 || (warp >= 13 && warp < TB_PVW)) {
         // ============================ loaders ============================
         // Gather every stage's K and V rows of the KV head (tokens from the
         // shared-memory member lists).
@@ -497,34 +506,78 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == 3) {
-        // =========================== MMA issuer ===========================
+        // ========================= S MMA issuer ==========================
+        // S = Q K^T of every stage in order, as soon as the stage's K/V rows
+        // have landed, the item's Q is in and the S buffer's previous P V is
+        // done (so S runs up to TB_SB - 1 stages ahead of P V).
         if (lane == 0) {
             int64_t gs = 0;
-            bool stop = false;
             const uint32_t q_base = ptx::smem_addr(smem + C::OFF_Q);
             const uint32_t kv_base = ptx::smem_addr(smem + C::OFF_KV);
-            // Two cursors over one stream of stages (all items in order). The
-            // issuer polls: a P V MMA goes out as soon as its P is ready; an S
-            // MMA goes out, up to TB_SB - 1 stages ahead of the P V cursor and
-            // across item boundaries, as soon as its inputs have landed.  The S
-            // cursor starts a new item only while it is at most one item ahead
-            // of the P V cursor (item i + 2's description is written only after
-            // item i's epilogue, which needs item i's last P V).
-            int iS = 0, sS = 0, nS = 0;         // S cursor: item, stage, the item's stages
-            int iP = 0, sP = 0;                 // P V cursor
-            int64_t gP = 0;                     // global stage of the P V cursor (gs: S cursor)
-            int nst[2] = {0, 0};                // stages of the (at most two) open items
-            bool s_done = false, item_open = false;
-            uint32_t idle = 0;
-            while (!stop) {
-                if (abort_flag) break;
-                bool progress = false;
-                // ---- P V for the oldest stage whose P is ready ----
-                const int sbP = (int)(gP % TB_SB);
-                if (gP < gs && ptx::mbar_test(&p_full[sbP], (uint32_t)((gP / TB_SB) & 1)) &&
-                    (sP > 0 || ptx::mbar_test(&o_empty[iP & 1], (uint32_t)(((iP >> 1) & 1) ^ 1)))) {
-                    const int ib = iP & 1;
+            for (int i = 0;; ++i) {
+                const int ib = i & 1;
+                const uint32_t iph = (uint32_t)((i >> 1) & 1);
+                if (!wait1(&info_full[ib], iph, 250u)) break;
+                const int nS = ti[ib].n_st;
+                ptx::mbar_arrive(&info_empty[ib]);
+                if (nS < 0) break;
+                const int qb = i % QB;
+                if (!wait1(&q_full[qb], (uint32_t)((i / QB) & 1), 251u)) break;
+                bool stop = false;
+                for (int s = 0; s < nS; ++s, ++gs) {
+                    const int slot = (int)(gs % NS);
+                    const int sb = (int)(gs % TB_SB);
+                    if (!wait1(&kv_full[slot], (uint32_t)((gs / NS) & 1), 252u) ||
+                        !wait1(&s_empty[sb], (uint32_t)(((gs / TB_SB) & 1) ^ 1), 253u)) {
+                        stop = true;
+                        break;
+                    }
+                    tb_fence_after();
+                    ptx::fence_proxy_async();   // the loaders' cp.async rows, to the async proxy
+                    const uint64_t qd = tb_desc(q_base + qb * C::Q_BYTES, 16, 1024);
+                    const uint64_t kd = tb_desc(kv_base + slot * C::STAGE, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < (int)C::KSTEPS; ++kk) {
+                        // k-step kk: plane kk / 4, +32 bytes per step inside the row
+                        const uint64_t qo = (uint64_t)(((kk >> 2) * C::Q_PLANE + (kk & 3) * 32) >> 4);
+                        const uint64_t ko = (uint64_t)(((kk >> 2) * C::KV_PLANE + (kk & 3) * 32) >> 4);
+                        tb_mma(tmem + sb * TB_N, qd + qo, kd + ko, C::IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                    tb_commit(&s_full[sb]);
+                    if (s == nS - 1) tb_commit(&q_empty[qb]);
+                }
+                if (stop) break;
+            }
+            // nothing this thread issued may still run on the tensor cores at exit
+            tb_commit(&fin_bar);
+            ptx::mbar_wait_bounded(&fin_bar, 0, TB_WAIT);
+        }
+    } else if (warp == TB_PVW) {
+        // ======================== P V MMA issuer =========================
+        // O += P V of every stage in order, as soon as its P is in TMEM (and,
+        // for an item's first stage, its O accumulator has been read out).
+        // A thread of its own, so that a P V never waits behind the issue of
+        // later stages' S MMAs.  Its commits release the stage's K/V slot and
+        // S buffer, and after an item's last stage hand O to the epilogue.
+        if (lane == 0) {
+            int64_t gP = 0;
+            const uint32_t kv_base = ptx::smem_addr(smem + C::OFF_KV);
+            for (int i = 0;; ++i) {
+                const int ib = i & 1;
+                const uint32_t iph = (uint32_t)((i >> 1) & 1);
+                if (!wait1(&info_full[ib], iph, 270u)) break;
+                const int n = ti[ib].n_st;
+                ptx::mbar_arrive(&info_empty[ib]);
+                if (n < 0) break;
+                if (!wait1(&o_empty[ib], iph ^ 1u, 271u)) break;
+                bool stop = false;
+                for (int s = 0; s < n; ++s, ++gP) {
+                    const int sbP = (int)(gP % TB_SB);
                     const int slot = (int)(gP % NS);
+                    if (!wait1(&p_full[sbP], (uint32_t)((gP / TB_SB) & 1), 272u)) {
+                        stop = true;
+                        break;
+                    }
                     // the softmax threads' TMEM stores of P are ordered before
                     // their arrivals on p_full
                     tb_fence_after();
@@ -534,71 +587,15 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
 #pragma unroll
                     for (int kk = 0; kk < TB_N / 16; ++kk)   // 16 keys = 8 TMEM columns of P
                         tb_mma_ts(t_o, tmem + sbP * TB_N + kk * 8, vd + (uint64_t)(kk * 128),
-                                  C::IDESC_PV, (sP > 0 || kk > 0) ? 1u : 0u);
+                                  C::IDESC_PV, (s > 0 || kk > 0) ? 1u : 0u);
                     tb_commit(&kv_empty[slot]);
                     tb_commit(&s_empty[sbP]);
-                    if (sP == nst[ib] - 1) tb_commit(&o_full[ib]);
-                    ++gP;
-                    if (++sP == nst[ib]) {
-                        ++iP;
-                        sP = 0;
-                    }
-                    progress = true;
+                    if (s == n - 1) tb_commit(&o_full[ib]);
                 }
-                // ---- the next S, if its inputs are ready ----
-                if (!s_done && gs - gP < TB_SB && (sS > 0 || iS <= iP + 1)) {
-                    const int ib = iS & 1;
-                    const uint32_t iph = (uint32_t)((iS >> 1) & 1);
-                    if (sS == 0 && !item_open && ptx::mbar_test(&info_full[ib], iph)) {
-                        nS = ti[ib].n_st;
-                        ptx::mbar_arrive(&info_empty[ib]);
-                        if (nS < 0) {
-                            s_done = true;
-                        } else {
-                            nst[ib] = nS;
-                            item_open = true;
-                        }
-                        progress = true;
-                    }
-                    const int slot = (int)(gs % NS);
-                    const int sb = (int)(gs % TB_SB);
-                    const int qb = iS % QB;
-                    if (item_open && (sS > 0 || ptx::mbar_test(&q_full[qb], (uint32_t)((iS / QB) & 1))) &&
-                        ptx::mbar_test(&kv_full[slot], (uint32_t)((gs / NS) & 1)) &&
-                        ptx::mbar_test(&s_empty[sb], (uint32_t)(((gs / TB_SB) & 1) ^ 1))) {
-                        tb_fence_after();
-                        ptx::fence_proxy_async();   // the loaders' cp.async rows, to the async proxy
-                        const uint64_t qd = tb_desc(q_base + qb * C::Q_BYTES, 16, 1024);
-                        const uint64_t kd = tb_desc(kv_base + slot * C::STAGE, 16, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < (int)C::KSTEPS; ++kk) {
-                            // k-step kk: plane kk / 4, +32 bytes per step inside the row
-                            const uint64_t qo = (uint64_t)(((kk >> 2) * C::Q_PLANE + (kk & 3) * 32) >> 4);
-                            const uint64_t ko = (uint64_t)(((kk >> 2) * C::KV_PLANE + (kk & 3) * 32) >> 4);
-                            tb_mma(tmem + sb * TB_N, qd + qo, kd + ko, C::IDESC_S, kk > 0 ? 1u : 0u);
-                        }
-                        tb_commit(&s_full[sb]);
-                        if (sS == nS - 1) tb_commit(&q_empty[qb]);
-                        ++gs;
-                        if (++sS == nS) {
-                            ++iS;
-                            sS = 0;
-                            item_open = false;
-                        }
-                        progress = true;
-                    }
-                }
-                if (s_done && gP == gs) break;      // every item's P V is out
-                if (progress) {
-                    idle = 0;
-                } else if (++idle > (wl << 3)) {   // nothing moved for a long time
-                    fail(260u);
-                    break;
-                }
+                if (stop) break;
             }
-            // nothing of this CTA may still run on the tensor cores at exit
-            tb_commit(&fin_bar);
-            ptx::mbar_wait_bounded(&fin_bar, 0, TB_WAIT);
+            tb_commit(&fin_bar2);
+            ptx::mbar_wait_bounded(&fin_bar2, 0, TB_WAIT);
         }
     } else if (warp < 8) {
         // ============================ softmax ============================
