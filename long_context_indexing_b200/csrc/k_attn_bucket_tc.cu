@@ -646,7 +646,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                     };
                     keep = bits(rg.lo0, rg.hi0) | bits(rg.lo1, rg.hi1);
                 }
-                if (keep != ~0ull) {
+                // a row that reads none of the stage's keys takes P = 0 by an
+                // infinite offset instead of masking every score
+                const bool none = keep == 0ull;
+                if (keep != ~0ull && !none) {
 #pragma unroll
                     for (int j = 0; j < TB_N; ++j)
                         if (!((keep >> j) & 1ull)) v[j] = -INFINITY;
@@ -662,7 +665,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                 }
                 const float mraw = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
                                          fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
-                const float mx = mraw * a.scale_log2;   // -inf stays -inf
+                const float mx = none ? -INFINITY : mraw * a.scale_log2;   // -inf stays -inf
                 // Lazy running max: raised only on the item's first stage, from
                 // nothing, or by more than 8 (a factor 2^8), so that O needs
                 // rescaling rarely; P stays <= 2^8.
@@ -677,7 +680,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bucket_attn_tc_kernel(BaArgs a)
                         resc = true;
                     }
                 }
-                const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+                const float mu = none ? INFINITY : ((m_run == -INFINITY) ? 0.f : m_run);
                 uint32_t pk[TB_N / 2];
                 float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
