@@ -1516,9 +1516,10 @@ __global__ void __launch_bounds__(DF_THREADS) decode_fill_kernel(IndexView ix, i
 // the candidates exactly and fills the budget as Flat does.
 // ---------------------------------------------------------------------------
 constexpr int TREE_MAX_BR = 256;     // branches walked at most
+constexpr int TREE_THREADS = 256;
 
 template <typename T>
-__global__ void __launch_bounds__(FILL_THREADS) tree_nominate_kernel(
+__global__ void __launch_bounds__(TREE_THREADS) tree_nominate_kernel(
     IndexView ix, int64_t n_blk, const T* lq, PosSrc pos, int64_t Nq, int W, SelectWs ws,
     const T* sup_rt, int64_t NS, int branches, int u_cap)
 {
@@ -1537,16 +1538,38 @@ __global__ void __launch_bounds__(FILL_THREADS) tree_nominate_kernel(
     if (threadIdx.x == 0) n_u = 0;
     load_query(q_s, lq, row);
     __syncthreads();
-    // 1. super-centroids, exact
-    for (int64_t h = threadIdx.x; h < NS; h += FILL_THREADS) {
-        const T* r = sup_rt + (b * NS + h) * DL;
+    // 1. super-centroids, exact (binary64, ascending dimension; 16-byte loads)
+    for (int64_t h = threadIdx.x; h < NS; h += TREE_THREADS) {
         double acc = 0.0;
-        for (int d = 0; d < DL; ++d) acc = __fma_rn((double)q_s[d], (double)load_elt(r + d), acc);
+        if (ix.dtype == LSA_BF16) {
+            const uint4* r4 = reinterpret_cast<const uint4*>(sup_rt + (b * NS + h) * DL);
+#pragma unroll 2
+            for (int x = 0; x < DL / 8; ++x) {
+                const uint4 raw = __ldg(r4 + x);
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(h2[e]);
+                    acc = __fma_rn((double)q_s[8 * x + 2 * e], (double)f.x, acc);
+                    acc = __fma_rn((double)q_s[8 * x + 2 * e + 1], (double)f.y, acc);
+                }
+            }
+        } else {
+            const float4* r4 = reinterpret_cast<const float4*>(sup_rt + (b * NS + h) * DL);
+#pragma unroll 2
+            for (int x = 0; x < DL / 4; ++x) {
+                const float4 f = __ldg(r4 + x);
+                acc = __fma_rn((double)q_s[4 * x], (double)f.x, acc);
+                acc = __fma_rn((double)q_s[4 * x + 1], (double)f.y, acc);
+                acc = __fma_rn((double)q_s[4 * x + 2], (double)f.z, acc);
+                acc = __fma_rn((double)q_s[4 * x + 3], (double)f.w, acc);
+            }
+        }
         es2[h] = acc;
     }
     __syncthreads();
     const int nbr = (int)min((int64_t)branches, NS);
-    for (int64_t h = threadIdx.x; h < NS; h += FILL_THREADS) {
+    for (int64_t h = threadIdx.x; h < NS; h += TREE_THREADS) {
         const double e = es2[h];
         int r = 0;                             // rank, counted only while it can be < nbr
         for (int64_t h2 = 0; h2 < NS && r < nbr; ++h2) r += rank_before(es2[h2], (int)h2, e, (int)h);
@@ -1555,21 +1578,28 @@ __global__ void __launch_bounds__(FILL_THREADS) tree_nominate_kernel(
             ws.tree_br[row * ws.tree_nbr + r] = (int32_t)h;
         }
     }
-    for (int r = nbr + (int)threadIdx.x; r < ws.tree_nbr; r += FILL_THREADS)
+    for (int r = nbr + (int)threadIdx.x; r < ws.tree_nbr; r += TREE_THREADS)
         ws.tree_br[row * ws.tree_nbr + r] = -1;
     __syncthreads();
     // 2. the universe: eligible buckets of the chosen branches
     const int64_t nb = eligible_buckets(ix, n_blk, pq, W);
     const int32_t* toff = ws.tree_off + b * (NS + 1);
     const int32_t* tmem = ws.tree_mem + b * ix.NBK;
+    // (one shared atomic per warp and chunk: ballot of the eligible members)
+    const int lane = threadIdx.x & 31;
     for (int r = 0; r < nbr; ++r) {
         const int h = chosen[r];
-        for (int32_t x = toff[h] + threadIdx.x; x < toff[h + 1]; x += FILL_THREADS) {
-            const int32_t g = tmem[x];
-            if (g < nb) {
-                const int slot = atomicAdd(&n_u, 1);
-                if (slot < u_cap) uid[slot] = g;
-            }
+        const int32_t x0 = toff[h], x1 = toff[h + 1];
+        for (int32_t xb = x0; xb < x1; xb += TREE_THREADS) {
+            const int32_t x = xb + threadIdx.x;
+            const int32_t g = (x < x1) ? tmem[x] : INT_MAX;
+            const bool take = g < nb;
+            const unsigned bal = __ballot_sync(0xffffffffu, take);
+            int base = 0;
+            if (lane == 0 && bal) base = atomicAdd(&n_u, __popc(bal));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            const int slot = base + __popc(bal & ((1u << lane) - 1u));
+            if (take && slot < u_cap) uid[slot] = g;
         }
     }
     __syncthreads();
@@ -1583,7 +1613,7 @@ __global__ void __launch_bounds__(FILL_THREADS) tree_nominate_kernel(
         return;
     }
     if (nu <= KC) {
-        for (int x = threadIdx.x; x < KC; x += FILL_THREADS) cand[x] = (x < nu) ? uid[x] : -1;
+        for (int x = threadIdx.x; x < KC; x += TREE_THREADS) cand[x] = (x < nu) ? uid[x] : -1;
         if (threadIdx.x == 0) {
             ws.lst_n[row] = nu;
             ws.lst_tau[row] = -INFINITY;
@@ -1591,7 +1621,7 @@ __global__ void __launch_bounds__(FILL_THREADS) tree_nominate_kernel(
         return;
     }
     // 3. approximate scores of the universe, then its KC best
-    for (int u = threadIdx.x; u < nu; u += FILL_THREADS) {
+    for (int u = threadIdx.x; u < nu; u += TREE_THREADS) {
         const int64_t g = uid[u];
         float acc = 0.f;
         if (ix.dtype == LSA_BF16) {
@@ -1628,7 +1658,7 @@ __global__ void __launch_bounds__(FILL_THREADS) tree_nominate_kernel(
     }
     __syncthreads();
     const float tau = radix_top_kc(usc, nu, cand_s);
-    for (int x = threadIdx.x; x < KC; x += FILL_THREADS) cand[x] = uid[cand_s[x]];
+    for (int x = threadIdx.x; x < KC; x += TREE_THREADS) cand[x] = uid[cand_s[x]];
     if (threadIdx.x == 0) {
         ws.lst_n[row] = KC;
         ws.lst_tau[row] = tau;
@@ -2239,11 +2269,11 @@ static cudaError_t launch_decode_finish_t(const IndexView& ix, int64_t n_blk, co
 
 static int tree_u_cap(const IndexView& ix, int64_t NS, int branches)
 {
-    // room for the chosen branches' buckets: four times the mean branch size
+    // room for the chosen branches' buckets: three times the mean branch size
     // per branch (larger universes take the exact fallback), within what
     // shared memory holds after the super scores
     const int64_t mean = (ix.NBK + NS - 1) / NS;
-    int64_t cap = 4 * mean * branches + KC;
+    int64_t cap = 3 * mean * branches + KC;
     const int64_t avail = (200 * 1024 - NS * 8) / 8;
     if (cap > avail) cap = avail;
     if (cap > ix.NBK) cap = ix.NBK;
@@ -2272,7 +2302,7 @@ static cudaError_t launch_tree_t(const IndexView& ix, int64_t n_blk, const void*
     cudaError_t e = ensure_smem_attr((const void*)tree_nominate_kernel<T>, 200 * 1024);
     if (e != cudaSuccess) return e;
     const PosSrc pos{positions, 0};
-    tree_nominate_kernel<T><<<dim3((unsigned)Nq, (unsigned)ix.B), FILL_THREADS, smem, st>>>(
+    tree_nominate_kernel<T><<<dim3((unsigned)Nq, (unsigned)ix.B), TREE_THREADS, smem, st>>>(
         ix, n_blk, lq, pos, Nq, sp.window, ws, (const T*)sup_rt, NS, branches, u_cap);
     note_launch();
     return launch_finish_t(ix, n_blk, lq, pos, Nq, sp, indices, counts, s_max, ws, st);
