@@ -29,13 +29,14 @@
 // with exact binary64 scores and proves the exact ranking against the largest
 // tau, or sends the row to the exact fallback.
 //
-// CTA = 10 warps:
+// CTA = 18 warps:
 //   warp 0     TMA producer: each item's query tile (two buffers), then its
 //              centroid tiles into a TC_STAGES-deep ring (128-byte swizzle);
 //   warp 1     owns 2 x TC_N TMEM columns (two fp32 accumulators) and issues
 //              tcgen05.mma (M = 128, N = TC_N, K = 16, four per tile);
-//   warps 2-9  epilogue: thread = (query row, half of every tile's columns);
-//              tcgen05.ld 32 columns at a time.
+//   warps 2-17 epilogue, four warps per TMEM lane quarter: thread = (query
+//              row, a quarter of every tile's columns, 64 scores); tcgen05.ld
+//              of 32-column pieces, several in flight before one wait.
 // Every mbarrier wait is bounded; after a timeout the CTA records DEV_TIMEOUT
 // in the index status word, the producer and the MMA thread stop, the
 // epilogue runs through its remaining items without waiting (so its named

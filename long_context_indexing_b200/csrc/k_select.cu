@@ -76,10 +76,8 @@ __device__ __forceinline__ void load_query(float* q_s, const T* lq, int64_t row)
 }
 
 // ---------------------------------------------------------------------------
-// Candidate nomination, SIMT: one CTA per query.  Binary32 FMA scores of the
-// eligible buckets into shared memory, then an MSB-first radix select of the
-// KC-th largest score (4 passes of 8 bits).  Candidates: every bucket above
-// that score plus enough of those equal to it.  tau = that score.
+// Helpers of the SIMT nominator (fp32 indices, decode, small chunks) and of
+// the D-LSA Tree walk: approximate scores, exact scores, radix top-KC.
 // ---------------------------------------------------------------------------
 constexpr int SIMT_THREADS = 256;
 constexpr int64_t SIMT_SMEM_MAX = 220 * 1024;
@@ -1503,7 +1501,7 @@ __global__ void __launch_bounds__(DF_THREADS) decode_fill_kernel(IndexView ix, i
 }
 
 // ---------------------------------------------------------------------------
-// D-LSA Tree nomination, one CTA (FILL_THREADS) per query ("Prefrontal's
+// D-LSA Tree nomination, one CTA (TREE_THREADS) per query ("Prefrontal's
 // Latent Sparse Attention ...", section "What it changes": the query scores a
 // few clusters at each level and walks down).  1. exact binary64 scores of
 // every super-centroid (retrieval copy), the `branches` best (score desc,
@@ -1792,9 +1790,10 @@ __global__ void __launch_bounds__(FB_THREADS) select_fallback_kernel(IndexView i
 // centroid.  The two are independent: a pooled group that completes at
 // position pos holds keys >= pos - p + 1, which lie inside the recent window
 // (W >= p - 1), so no selection made at pos can read them.
-// Scores: binary32 FMA over the retrieval copy (16-byte loads, 8 lanes per
-// row), written as fp16 with the fp16 maximum of every 32-score chunk -- the
-// same row the tensor-core scorer writes, which the fill nominates from.
+// Scores: binary32 FMA over the retrieval copy (16-byte loads, lanes over a
+// row's dimensions), then the slice's DEC_M best scores sorted (score desc,
+// lower bucket on ties) with their buckets, and the next score as the bound of
+// everything the slice leaves out -- the lists decode_fill_kernel merges.
 // Append: slice 0 writes the new latent/key/value rows at pos; every slice
 // pools the completed group j = (pos+1)/p - 1 (binary32, left to right; the
 // group's last row comes from the new latent row itself), normalises it
