@@ -265,9 +265,8 @@ cudaError_t launch_attn_combine(const float* part, int ns, int64_t rows, int Hq,
 int attn_head_group(int Hkv);
 
 // Decode: append + approximate scores for one query per sequence, over
-// n_slice CTAs per sequence.  ws.scores / ws.cmax receive the fp16 score row
-// and its 32-score chunk maxima (as the tensor-core scorer writes them);
-// app_score / app_g / app_slot (in ws) the sliced nearest-centroid search.
+// n_slice CTAs per sequence.  ws.dl_* receive every slice's sorted top list
+// and bound; app_score / app_g / app_slot the sliced nearest-centroid search.
 cudaError_t launch_decode_prep(const IndexView& ix, int64_t n_blk, void* latent_K, void* K,
                                void* V, const void* new_latent_k, const void* new_k,
                                const void* new_v, const void* latent_q, const int32_t* pos,
