@@ -467,6 +467,7 @@ def run_lsa(args, rank, ws):
     e2e_ms = _max_over_ranks(_events_time(e2e_step, args.steps, stream), ws)
 
     tree = None if args.tree_super <= 0 else _tree_measure(args, w, inp, idx, T_old, stream)
+    full = None if args.no_full_prefill else _full_prefill(w, inp, work, O, stream)
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -500,7 +501,7 @@ def run_lsa(args, rank, ws):
             "gpu_launches": launches, "clocks": clocks,
             "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "index_build_prefix_s": round(build_s, 3), "selection_fallbacks": fallbacks,
-            "tree": tree, "decode": decode}
+            "tree": tree, "full_prefill": full, "decode": decode}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -553,6 +554,39 @@ def _tree_measure(args, w, inp, idx, T_old, stream):
             "select_fallbacks": fb_tree,
             "flat_long_range_keys_kept": round(kept / max(tot, 1), 4),
             "recall_sample": "%d rows (every %d-th) of the chunk" % (len(rows), w.nq // len(rows))}
+
+
+def _full_prefill(w, inp, work, O, stream):
+    """One layer's whole context prefilled chunk by chunk from position 0
+    (lsa_prefill_chunk over [0, chunk), [chunk, 2 chunk), ...: the index
+    grows by every chunk's blocks, every chunk's queries select and attend).
+    The chunks reuse the bench chunk's latent queries and queries (their
+    content does not change the work); one timed pass, CUDA events."""
+    import long_context_indexing_b200 as lsa
+
+    span = w.p * w.G
+    chunk = w.nq
+    if w.T % chunk or chunk % span:
+        return None
+    idx = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16 if w.dtype == "bf16" else lsa.F32)
+    idx.build(inp["latent_K"], 0)
+    n = w.T // chunk
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    ev[0].record(stream)
+    for c in range(n):
+        lsa.lsa_prefill_chunk(idx, inp["latent_K"], inp["latent_Q"], inp["Q"], inp["K"], inp["V"],
+                              c * chunk, (c + 1) * chunk, w.R, w.W, w.S, workspace=work, out=O)
+        ev[c + 1].record(stream)
+    ev[n].synchronize()
+    per = [ev[c].elapsed_time(ev[c + 1]) for c in range(n)]
+    total = ev[0].elapsed_time(ev[n])
+    fb = idx.check()
+    del idx
+    return {"what": "whole %d-token context of one layer prefilled in %d chunks of %d queries "
+                    "(index built chunk by chunk from position 0)" % (w.T, n, chunk),
+            "total_ms": round(total, 2), "queries_per_s": round(w.T * w.B / (total * 1e-3), 1),
+            "first_chunk_ms": round(per[0], 4), "last_chunk_ms": round(per[-1], 4),
+            "selection_fallbacks": fb}
 
 
 # ------------------------------------------------------------------- decode --
@@ -710,6 +744,8 @@ def main():
     ap.add_argument("--ref-queries", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-full-prefill", action="store_true",
+                    help="skip the whole-context chunk-by-chunk prefill measurement")
     ap.add_argument("--tree-super", type=int, default=256,
                     help="D-LSA Tree beside Flat: super-buckets of level 2 (0: skip)")
     ap.add_argument("--tree-branches", type=int, default=16,

@@ -719,7 +719,16 @@ static bool make_rows64_bf16(CUtensorMap* m, const void* base, uint64_t rows, ui
 
 bool tc_scoring_available() { return true; }
 
-TcSplit tc_split_plan(const IndexView& ix, int64_t Nq)
+// The widest group (2^gl buckets, gl = 2 .. 6) that still leaves a sequence of
+// n buckets at least 4m groups.
+static int tc_group_log2(int64_t n, int m)
+{
+    int gl = 6;
+    while (gl > 2 && (n >> gl) < 4LL * m) --gl;
+    return gl;
+}
+
+TcSplit tc_split_plan(const IndexView& ix, int64_t Nq, int64_t n_blk)
 {
     TcSplit sp;
     sp.n_qt = (Nq + TC_M - 1) / TC_M;
@@ -733,14 +742,20 @@ TcSplit tc_split_plan(const IndexView& ix, int64_t Nq)
     if (sp.n_split < 1) sp.n_split = 1;
     sp.n_items = tiles * sp.n_split;
     // groups of 64 scores (one per epilogue thread and tile), narrower (down
-    // to 4) while a sequence has fewer than 4m groups: with g groups and the
-    // m-th largest maximum as the threshold, scores without structure put
-    // about -g ln(1 - m/g) ~ m (1 + m / 2g) of them above it
+    // to 4) while the sequence's buckets -- those of the blocks closed so far,
+    // not the capacity -- make fewer than 4m groups: with g groups and the m-th
+    // largest maximum as the threshold, scores without structure put about
+    // -g ln(1 - m/g) ~ m (1 + m / 2g) of them above it
     sp.m = TC_TARGET;
-    int gl = 6;
-    while (gl > 2 && (ix.NBK >> gl) < 4LL * sp.m) --gl;
-    sp.gw_log2 = gl;
-    sp.n_grp = (((n_ct * TC_N) >> gl) + 7) / 8 * 8;   // rows of keys start on 16 bytes
+    int64_t nb_now = (n_blk < 0 ? 0 : n_blk) * ix.k;
+    if (nb_now > ix.NBK) nb_now = ix.NBK;
+    sp.gw_log2 = tc_group_log2(nb_now, sp.m);
+    // row stride: the capacity's groups at the capacity's width, and at least
+    // 8m (a narrower width is picked only while the buckets make fewer than
+    // 8m groups at it); rows of keys start on 16 bytes
+    int64_t ng = (n_ct * TC_N) >> tc_group_log2(ix.NBK, sp.m);
+    if (ng < 8LL * sp.m) ng = 8LL * sp.m;
+    sp.n_grp = (ng + 7) / 8 * 8;
     return sp;
 }
 
@@ -755,7 +770,7 @@ cudaError_t launch_score_lists_tc(const IndexView& ix, int64_t n_blk, const void
                                   cudaStream_t st)
 {
     if (ix.dtype != LSA_BF16) return cudaErrorInvalidValue;
-    const TcSplit sp = tc_split_plan(ix, Nq);
+    const TcSplit sp = tc_split_plan(ix, Nq, n_blk);
     if (ws.n_lst != sp.n_split || ws.lst_cap != TC_LIST_CAP || !ws.gmax || !ws.theta ||
         ws.n_grp != sp.n_grp)
         return cudaErrorInvalidValue;

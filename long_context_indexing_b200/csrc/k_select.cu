@@ -2092,7 +2092,7 @@ bool select_uses_tc(const IndexView& ix, int64_t Nq)
 static void list_shape(const IndexView& ix, int64_t Nq, int* n_lst, int* cap, bool one_list = false)
 {
     if (!one_list && select_uses_tc(ix, Nq)) {
-        *n_lst = tc_split_plan(ix, Nq).n_split;
+        *n_lst = tc_split_plan(ix, Nq, 0).n_split;
         *cap = TC_LIST_CAP;
     } else {
         *n_lst = 1;
@@ -2103,7 +2103,7 @@ static void list_shape(const IndexView& ix, int64_t Nq, int* n_lst, int* cap, bo
 // Group maxima per row of the tensor-core path (0 otherwise).
 static int64_t n_grp_of(const IndexView& ix, int64_t Nq, bool one_list = false)
 {
-    return (!one_list && select_uses_tc(ix, Nq)) ? tc_split_plan(ix, Nq).n_grp : 0;
+    return (!one_list && select_uses_tc(ix, Nq)) ? tc_split_plan(ix, Nq, 0).n_grp : 0;
 }
 
 // one_list: a single list of KC candidates per row (SIMT-style nominators:

@@ -187,13 +187,15 @@ constexpr int DEC_MAX_SLICES = 128;
 struct TcSplit {
     int n_split;      // centroid ranges (lists per row)
     int tps;          // centroid tiles of 256 per range
-    int gw_log2;      // group width (columns) of the group maxima, 2 .. 5
+    int gw_log2;      // group width (columns) of the group maxima, 2 .. 6
     int m;            // threshold rank among a row's group maxima
-    int64_t n_grp;    // group maxima per row (all ranges)
+    int64_t n_grp;    // row stride of the group maxima (every width the call may pick)
     int64_t n_qt;     // 128-query tiles per sequence
     int64_t n_items;  // B * n_qt * n_split
 };
-TcSplit tc_split_plan(const IndexView& ix, int64_t Nq);
+// n_blk: closed blocks at the time of the call (the group width follows the
+// buckets that exist; every other field depends on the index capacity only).
+TcSplit tc_split_plan(const IndexView& ix, int64_t Nq, int64_t n_blk);
 // The tensor-core scorer serves bf16 indices and at least one 128-query tile.
 bool select_uses_tc(const IndexView& ix, int64_t Nq);
 size_t select_ws_bytes(const IndexView& ix, int64_t Nq);

@@ -311,3 +311,39 @@ def test_query_ranges_equal_the_whole_chunk(cuts):
         lsa.lsa_prefill_chunk_queries(gpu, dev["latent_K"], dev["latent_Q"][:, :10].contiguous(),
                                       dev["Q"][:, :10].contiguous(), dev["K"], dev["V"], T_old,
                                       w.T, w.nq - 5, w.nq + 5, w.R, w.W, w.S, workspace=ws)
+
+
+def test_whole_context_chunk_by_chunk():
+    # A whole context prefilled in chunks from position 0 (the index grows by
+    # each chunk's blocks): every chunk's selections equal the oracle's, which
+    # extends its index chunk by chunk in the same way, and the outputs are
+    # within the bf16 bars.
+    w = _base(T=4096, nq=4096, R=300, W=40, S=4)
+    chunk = 512                                  # two blocks of 256 tokens
+    inp = synth.prefill_inputs(w, 21, "cpu")
+    dev = {k: v.cuda() for k, v in inp.items()}
+    gpu = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16)
+    gpu.build(dev["latent_K"], 0)
+    ws = torch.empty(lsa.lsa_prefill_workspace_bytes(gpu, chunk, w.Hq, w.Hkv, w.d, w.R, w.W, w.S),
+                     dtype=torch.uint8, device="cuda")
+    lat = inp["latent_K"][0].float().numpy()
+    orc = oracle.Index(w.T, w.p, w.G, w.k, w.L, rt_bf16=True)
+    for t0 in range(0, w.T, chunk):
+        t1 = t0 + chunk
+        O = lsa.lsa_prefill_chunk(gpu, dev["latent_K"], dev["latent_Q"][:, t0:t1].contiguous(),
+                                  dev["Q"][:, t0:t1].contiguous(), dev["K"], dev["V"], t0, t1,
+                                  w.R, w.W, w.S, workspace=ws)
+        torch.cuda.synchronize()
+        assert gpu.check() == 0
+        g_idx, g_cnt = lsa.prefill_selection_views(ws, 1, chunk, w.s_max)
+        orc.extend(lat, t0, t1)
+        pos = np.arange(t0, t1)
+        o_idx, o_cnt, _, _ = oracle.select(orc, inp["latent_Q"][0, t0:t1].float().numpy(), pos,
+                                           w.R, w.W, w.S)
+        assert np.array_equal(g_cnt[0].cpu().numpy(), o_cnt), t0
+        assert np.array_equal(g_idx[0].cpu().numpy(), o_idx), t0
+        O_ref, _ = oracle.attend(inp["Q"][0, t0:t1].float().numpy(), inp["K"][0].float().numpy(),
+                                 inp["V"][0].float().numpy(), o_idx, o_cnt,
+                                 oracle.default_scale(w.d))
+        err = np.abs(O[0].float().cpu().numpy().astype(np.float64) - O_ref)
+        assert err.max() <= BF16_MAX and err.mean() <= BF16_MEAN, (t0, err.max(), err.mean())
