@@ -534,80 +534,118 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_bf16_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Split-KV combine: one warp per (query row, query head).  Lane s holds split
-// s's (max, sum) (32 splits at a time); weights exp2(m_s - M) / L are
-// broadcast by shuffles and every lane accumulates 4 output dimensions with
-// 16-byte loads of each split's partial.
+// Split-KV combine: one CTA (CB_WARPS warps) per (query row, query head), so
+// that every split's partial is in flight at once (the combine is short and
+// latency-bound).  The (max, sum) of every split go to shared memory first:
+// M = the largest max, w_s = exp2(m_s - M), L = sum of w_s * sum_s.  Warp w
+// then accumulates splits w, w + CB_WARPS, ... (lane = 4 output dimensions,
+// 16-byte loads, all of the warp's splits issued before they are summed), the
+// warps' sums meet in shared memory, and O = sum / L.
 // ---------------------------------------------------------------------------
+constexpr int CB_WARPS = 8;
+constexpr int CB_MAX_SPLITS = 128;
+constexpr int CB_PER_WARP = CB_MAX_SPLITS / CB_WARPS;   // splits per warp at most
+
 template <int D>
-__global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restrict__ part, int ns,
-                                                           int64_t n_heads_total, int Hq,
-                                                           __nv_bfloat16* O, float* lse)
+__global__ void __launch_bounds__(32 * CB_WARPS) attn_combine_kernel(const float* __restrict__ part,
+                                                                     int ns, int Hq,
+                                                                     __nv_bfloat16* O, float* lse)
 {
     constexpr int PS = D + 4;
-    const int lane = threadIdx.x & 31;
-    const int64_t wid = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);   // (row, head)
-    if (wid >= n_heads_total) return;
+    __shared__ float w_s[CB_MAX_SPLITS];
+    __shared__ float4 acc_s[CB_WARPS][D / 4];
+    __shared__ float sh_M, sh_L;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t wid = blockIdx.x;                  // (row, head)
     const int64_t row = wid / Hq, h = wid % Hq;
     const float* base = part + (row * ns * Hq + h) * PS;
     const int64_t sstride = (int64_t)Hq * PS;
-    float M = -INFINITY;
-    for (int s0 = 0; s0 < ns; s0 += 32)
-        if (s0 + lane < ns) M = fmaxf(M, __ldcg(base + (s0 + lane) * sstride + D));
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    // every warp's splits, loaded before anything waits on them
     const bool live = lane < D / 4;
-    for (int s0 = 0; s0 < ns; s0 += 32) {
-        float w = 0.f;
-        if (s0 + lane < ns) {
-            const float2 ml = __ldcg(reinterpret_cast<const float2*>(base + (s0 + lane) * sstride + D));
-            w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-            L += ml.y * w;
-        }
-        const int n = min(32, ns - s0);
-        // eight splits' loads in flight at a time
-        for (int j0 = 0; j0 < n; j0 += 8) {
-            float4 v[8];
+    float4 v[CB_PER_WARP];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (live && j0 + u < n)
-                    v[u] = __ldcg(reinterpret_cast<const float4*>(base + (s0 + j0 + u) * sstride) + lane);
-            }
+    for (int u = 0; u < CB_PER_WARP; ++u) {
+        const int sp = warp + CB_WARPS * u;
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (live && sp < ns) v[u] = __ldcg(reinterpret_cast<const float4*>(base + sp * sstride) + lane);
+    }
+    // (max, sum) of every split
+    float m = -INFINITY;
+    for (int sp = threadIdx.x; sp < ns; sp += 32 * CB_WARPS) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(base + sp * sstride + D));
+        w_s[sp] = ml.x;
+        m = fmaxf(m, ml.x);
+    }
+    __shared__ float m_w[CB_WARPS];
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) m_w[warp] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float M = m_w[0];
+        for (int x = 1; x < CB_WARPS; ++x) M = fmaxf(M, m_w[x]);
+        sh_M = M;
+    }
+    __syncthreads();
+    const float M = sh_M;
+    float lsum = 0.f;
+    for (int sp = threadIdx.x; sp < ns; sp += 32 * CB_WARPS) {
+        const float ms = w_s[sp];
+        const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+        w_s[sp] = w;
+        lsum += __ldcg(base + sp * sstride + D + 1) * w;
+    }
+    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+    __syncthreads();                                 // w_s complete; m_w free
+    if (lane == 0) m_w[warp] = lsum;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float wj = __shfl_sync(0xffffffffu, w, (j0 + u) & 31);
-                if (j0 + u < n) {
-                    acc.x += v[u].x * wj;
-                    acc.y += v[u].y * wj;
-                    acc.z += v[u].z * wj;
-                    acc.w += v[u].w * wj;
-                }
-            }
+    for (int u = 0; u < CB_PER_WARP; ++u) {
+        const int sp = warp + CB_WARPS * u;
+        if (sp < ns) {
+            const float w = w_s[sp];
+            acc.x += v[u].x * w;
+            acc.y += v[u].y * w;
+            acc.z += v[u].z * w;
+            acc.w += v[u].w * w;
         }
     }
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (live) {
-        const float inv = 1.f / L;
+    if (live) acc_s[warp][lane] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float L = 0.f;
+        for (int x = 0; x < CB_WARPS; ++x) L += m_w[x];
+        sh_L = L;
+    }
+    __syncthreads();
+    if (warp == 0 && live) {
+        float4 t = acc_s[0][lane];
+#pragma unroll
+        for (int x = 1; x < CB_WARPS; ++x) {
+            const float4 y = acc_s[x][lane];
+            t.x += y.x;
+            t.y += y.y;
+            t.z += y.z;
+            t.w += y.w;
+        }
+        const float inv = 1.f / sh_L;
         __nv_bfloat16* op = O + wid * D + 4 * lane;
-        op[0] = __float2bfloat16_rn(acc.x * inv);
-        op[1] = __float2bfloat16_rn(acc.y * inv);
-        op[2] = __float2bfloat16_rn(acc.z * inv);
-        op[3] = __float2bfloat16_rn(acc.w * inv);
+        op[0] = __float2bfloat16_rn(t.x * inv);
+        op[1] = __float2bfloat16_rn(t.y * inv);
+        op[2] = __float2bfloat16_rn(t.z * inv);
+        op[3] = __float2bfloat16_rn(t.w * inv);
     }
-    if (lane == 0 && lse) lse[wid] = (M + log2f(L)) * 0.69314718055994531f;
+    if (threadIdx.x == 0 && lse) lse[wid] = (M + log2f(sh_L)) * 0.69314718055994531f;
 }
 
 cudaError_t launch_attn_combine(const float* part, int ns, int64_t rows, int Hq, int d, void* O,
                                 float* lse, cudaStream_t st)
 {
-    const int64_t n = rows * Hq;
-    const unsigned grid = (unsigned)((n + 3) / 4);
+    if (ns < 1 || ns > CB_MAX_SPLITS) return cudaErrorInvalidValue;
+    const unsigned grid = (unsigned)(rows * Hq);
     if (d == 128)
-        attn_combine_kernel<128><<<grid, 128, 0, st>>>(part, ns, n, Hq, (__nv_bfloat16*)O, lse);
+        attn_combine_kernel<128><<<grid, 32 * CB_WARPS, 0, st>>>(part, ns, Hq, (__nv_bfloat16*)O, lse);
     else
-        attn_combine_kernel<64><<<grid, 128, 0, st>>>(part, ns, n, Hq, (__nv_bfloat16*)O, lse);
+        attn_combine_kernel<64><<<grid, 32 * CB_WARPS, 0, st>>>(part, ns, Hq, (__nv_bfloat16*)O, lse);
     note_launch();
     return cudaGetLastError();
 }

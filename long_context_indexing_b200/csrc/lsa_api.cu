@@ -226,7 +226,7 @@ DecodeLayout decode_layout(const lsa_index* idx, int Hq, int Hkv, int d, lsa_sel
     // triples
     int64_t ns = ((int64_t)sm_count() * LSA_DEC_SPLIT_MULT + units - 1) / units;
     if (ns < 1) ns = 1;
-    if (ns > 128) ns = 128;   // the combine keeps 2 * heads * ns floats in shared memory
+    if (ns > 128) ns = 128;   // the combine takes at most 128 splits
     int64_t kps = (s_max + ns - 1) / ns;
     kps = ((kps + kt - 1) / kt) * kt;
     ns = (s_max + kps - 1) / kps;
