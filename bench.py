@@ -360,6 +360,97 @@ def run_lsa_split(args, rank, ws):
         print(json.dumps(line), flush=True)
 
 
+def _context_shard(T, span, rank, ws):
+    """Key rows [lo, hi) of `rank`'s shard of a T-token cache: whole blocks of
+    `span` tokens, as even as they come; the last shard also takes a partial
+    block at the end."""
+    nb = T // span
+    lo = (nb * rank // ws) * span
+    hi = T if rank == ws - 1 else (nb * (rank + 1) // ws) * span
+    return lo, hi
+
+
+def _exchange_rows(part, rank, ws):
+    """Every rank's [ws * n][...] tensor cut into ws row blocks; rank j gets
+    block j of every rank, stacked by source rank ([ws][n][...])."""
+    if ws == 1:
+        return part[None]
+    part = part.contiguous()
+    n = part.shape[0] // ws
+    if torch.distributed.get_backend() == "nccl":
+        out = torch.empty_like(part)
+        torch.distributed.all_to_all_single(out, part)
+        return out.view((ws, n) + tuple(part.shape[1:]))
+    parts = [torch.empty_like(part) for _ in range(ws)]
+    torch.distributed.all_gather(parts, part)
+    return torch.stack([p[rank * n:(rank + 1) * n] for p in parts])
+
+
+def run_lsa_context(args, rank, ws):
+    """One chunk with the KV cache in shards of whole blocks over the ranks
+    (the pages' context-parallel layout): every rank holds its shard of K and
+    V, the latent keys and the full index, extends the index and selects for
+    every query of the chunk (the same selection on every rank), attends over
+    the selected keys of its shard (lsa_attend_key_range: output and
+    log-sum-exp per query head), and the partials are exchanged by row blocks
+    (NCCL all-to-all) and merged by LSE weight (lsa_merge_partials) inside the
+    timed step; each rank ends with its row block of the output.  Strong
+    scaling: the job is one chunk whatever the rank count."""
+    import long_context_indexing_b200 as lsa
+
+    w = _bench_workload(args)
+    dev = torch.device("cuda")
+    inp = synth.prefill_inputs(w, seed=args.seed, device=dev)      # the same chunk on every rank
+    span = w.p * w.G
+    T_old = w.T - w.nq
+    lo, hi = _context_shard(w.T, span, rank, ws)
+    Ks = inp["K"][:, lo:hi].contiguous()
+    Vs = inp["V"][:, lo:hi].contiguous()
+    del inp["K"], inp["V"]                                          # a rank keeps its shard only
+    torch.cuda.empty_cache()
+    q0, q1 = _query_slice(w.nq, rank, ws)
+    idx = lsa.LsaIndex(w.B, w.T, w.p, w.G, w.k, w.L, lsa.BF16 if w.dtype == "bf16" else lsa.F32)
+    idx.build(inp["latent_K"], (T_old // span) * span)
+    work = torch.empty(lsa.lsa_prefill_workspace_bytes(idx, w.nq, w.Hq, w.Hkv, w.d, w.R, w.W,
+                                                       w.S), dtype=torch.uint8, device=dev)
+    sel_i, sel_c = lsa.prefill_selection_views(work, w.B, w.nq, w.s_max)
+    Op = torch.empty_like(inp["Q"])
+    Lp = torch.empty(w.B, w.nq, w.Hq, dtype=torch.float32, device=dev)
+    Om = torch.empty((q1 - q0, w.Hq, w.d), dtype=inp["Q"].dtype, device=dev)
+    kr_ws = torch.empty(lsa.lsa_attend_key_range_workspace_bytes(w.B, w.nq, w.s_max),
+                        dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        lsa.lsa_prefill_select(idx, inp["latent_K"], inp["latent_Q"], T_old, w.T, w.Hq, w.Hkv,
+                               w.d, w.R, w.W, w.S, work)
+        lsa.lsa_attend_key_range(inp["Q"], Ks, Vs, sel_i, sel_c, lo, hi, workspace=kr_ws,
+                                 out=Op, lse=Lp)
+        O_parts = _exchange_rows(Op[0], rank, ws)
+        L_parts = _exchange_rows(Lp[0], rank, ws)
+        lsa.lsa_merge_partials(O_parts, L_parts, out=Om)
+
+    for _ in range(args.warmup):
+        step()
+    _barrier(ws)
+    launches0 = lsa.kernel_launches()
+    ms = _max_over_ranks(_events_time(step, args.steps, stream), ws)
+    launches = lsa.kernel_launches() - launches0
+    _barrier(ws)
+    fallbacks = idx.check()
+    line = {"metric": METRIC, "value": round(w.nq / (ms * 1e-3), 2), "unit": "queries/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic (seeded clustered mixture; no model weights or datasets)",
+            "config": dict(_config(w, ws), parallelism="KV cache in %d shards of whole blocks "
+                           "(index replicated; per-shard partials merged by LSE weight after an "
+                           "all-to-all of row blocks)" % ws),
+            "e2e": None, "gpu_launches": launches, "selection_fallbacks": fallbacks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------------- lsa --
 
 def _bench_workload(args):
@@ -752,9 +843,10 @@ def main():
                     help="D-LSA Tree beside Flat: super-buckets a query walks")
     ap.add_argument("--decode-T", type=int, default=None,
                     help="override the decode context length (a multiple of p * block)")
-    ap.add_argument("--split", choices=["chunks", "queries"], default="chunks",
-                    help="several GPUs: every rank runs its own chunk (weak scaling), or one "
-                         "chunk's queries are split over the ranks (strong scaling)")
+    ap.add_argument("--split", choices=["chunks", "queries", "context"], default="chunks",
+                    help="several GPUs: every rank runs its own chunk (weak scaling), one "
+                         "chunk's queries are split over the ranks, or the KV cache is held in "
+                         "shards over the ranks (both strong scaling)")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the decode measurement (prints its object)")
     args = ap.parse_args()
@@ -771,6 +863,8 @@ def main():
             run_reference(args, rank, ws)
         elif args.split == "queries":
             run_lsa_split(args, rank, ws)
+        elif args.split == "context":
+            run_lsa_context(args, rank, ws)
         else:
             run_lsa(args, rank, ws)
     finally:

@@ -283,6 +283,43 @@ lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtyp
                            void* O, float* lse, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * KV cache in shards of whole blocks ("Latent Sparse Attention: un indice
+ * gerarchico per contesti lunghi", paragraph on memory: with context
+ * parallelism every rank keeps its share of the KV cache and a full copy of
+ * the bucket index, so every rank makes the same selection)
+ * ------------------------------------------------------------------------- */
+
+/* Workspace bytes for lsa_attend_key_range (0 on bad sizes). */
+size_t lsa_attend_key_range_workspace_bytes(int64_t B, int64_t Nq, int s_max);
+
+/* Attention of every query over the keys of its selection that lie in
+ * [key_lo, key_hi), read from a shard of the caches:
+ *   K_shard, V_shard [B][key_hi - key_lo][Hkv][d] hold rows key_lo .. key_hi-1
+ *   of the full caches; indices / counts / s_max are the selection in global
+ *   positions (as lsa_select writes it);
+ *   O_part [B][Nq][Hq][d] (dtype) receives the softmax over those keys alone,
+ *   lse_part [B][Nq][Hq] f32 their max + ln(sum) of the scaled logits; a
+ *   (query, head) without a key in the range gets O = 0 and lse = -inf.
+ * The partial results of shards that cover every selected key merge into
+ * lsa_sparse_attn's result with lsa_merge_partials.  Caller-owned device
+ * memory; workspace of lsa_attend_key_range_workspace_bytes(B, Nq, s_max);
+ * all pointers 16-byte aligned; asynchronous on `stream`. */
+lsa_status lsa_attend_key_range(const void* Q, const void* K_shard, const void* V_shard,
+                                lsa_dtype dtype, int64_t B, int64_t Nq, int Hq, int Hkv, int d,
+                                const int32_t* indices, const int32_t* counts, int s_max,
+                                int64_t key_lo, int64_t key_hi, float scale, void* workspace,
+                                size_t ws_bytes, void* O_part, float* lse_part, void* stream);
+
+/* LSE-weighted merge of n_parts (1 .. 32) partial attention results:
+ *   O_parts [n_parts][rows][Hq][d] (dtype), lse_parts [n_parts][rows][Hq] f32;
+ *   O[r][h] = sum_p exp(lse_p - L) O_p[r][h] with L = ln sum_p exp(lse_p)
+ *   (parts with lse = -inf weigh 0; a row no part covers gets 0), lse
+ *   (nullable) [rows][Hq] receives L.  Asynchronous on `stream`. */
+lsa_status lsa_merge_partials(const void* O_parts, const float* lse_parts, lsa_dtype dtype,
+                              int n_parts, int64_t rows, int Hq, int d, void* O, float* lse,
+                              void* stream);
+
+/* ---------------------------------------------------------------------------
  * Fused entries
  * ------------------------------------------------------------------------- */
 

@@ -20,6 +20,7 @@ __all__ = [
     "LsaError", "LsaIndex", "lsa_index_bytes", "lsa_build_index", "lsa_select",
     "lsa_select_workspace_bytes", "lsa_tree_select_workspace_bytes",
     "lsa_sparse_attn", "lsa_prefill_chunk", "lsa_prefill_workspace_bytes",
+    "lsa_attend_key_range", "lsa_attend_key_range_workspace_bytes", "lsa_merge_partials",
     "lsa_prefill_partial_slots", "lsa_prefill_select", "lsa_prefill_attend",
     "lsa_prefill_chunk_host", "lsa_prefill_chunk_queries", "LsaTree", "set_wait_limit",
     "lsa_decode_workspace_bytes", "lsa_decode_step", "lsa_select_noalloc", "library_path", "kernel_launches", "F32",
@@ -68,6 +69,10 @@ def _declare(lib):
         "lsa_select_workspace_bytes": ([P, I64], SZ),
         "lsa_select": ([P, P, P, I64, SelectParams, P, P, I, P, SZ, P], I),
         "lsa_sparse_attn": ([P, P, P, I, I64, I64, I64, I, I, I, P, P, I, F, P, P, P], I),
+        "lsa_attend_key_range_workspace_bytes": ([I64, I64, I], SZ),
+        "lsa_attend_key_range": ([P, P, P, I, I64, I64, I, I, I, P, P, I, I64, I64, F, P, SZ, P,
+                                  P, P], I),
+        "lsa_merge_partials": ([P, P, I, I, I64, I, I, P, P, P], I),
         "lsa_prefill_workspace_bytes": ([P, I64, I, I, I, SelectParams], SZ),
         "lsa_prefill_partial_slots": ([P, I64, I, I, I, SelectParams, SZ], I64),
         "lsa_prefill_chunk": ([P, P, P, P, P, P, I64, I64, I, I, I, SelectParams, P, SZ, P, P],
@@ -300,6 +305,48 @@ def lsa_sparse_attn(Q, K, V, indices, counts, scale=None, return_lse=False, out=
                                 d, _ptr(indices), _ptr(counts), indices.shape[-1], scale, _ptr(O),
                                 _ptr(lse), _stream(stream)))
     return (O, lse) if return_lse else O
+
+
+def lsa_attend_key_range_workspace_bytes(B, Nq, s_max):
+    """Workspace bytes lsa_attend_key_range needs."""
+    return int(_lib.lsa_attend_key_range_workspace_bytes(int(B), int(Nq), int(s_max)))
+
+
+def lsa_attend_key_range(Q, K_shard, V_shard, indices, counts, key_lo, key_hi, scale=None,
+                         workspace=None, out=None, lse=None, stream=None):
+    """Attention over the selected keys in [key_lo, key_hi) (C: lsa_attend_key_range), the
+    caches' rows key_lo .. key_hi-1 in K_shard, V_shard [B][key_hi-key_lo][Hkv][d]: returns
+    (O_part [B][Nq][Hq][d], lse_part [B][Nq][Hq] f32)."""
+    _cuda(Q, K_shard, V_shard, indices, counts, out, lse)
+    B, Nq, Hq, d = Q.shape
+    Hkv = K_shard.shape[2]
+    s_max = indices.shape[-1]
+    if scale is None:
+        scale = float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))
+    O = out if out is not None else torch.empty_like(Q)
+    L = lse if lse is not None else torch.empty(B, Nq, Hq, dtype=torch.float32, device=Q.device)
+    need = int(_lib.lsa_attend_key_range_workspace_bytes(B, Nq, s_max))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+    _check(_lib.lsa_attend_key_range(_ptr(Q), _ptr(K_shard), _ptr(V_shard), _dtype_code(Q), B, Nq,
+                                     Hq, Hkv, d, _ptr(indices), _ptr(counts), s_max, int(key_lo),
+                                     int(key_hi), scale, _ptr(workspace), workspace.numel(),
+                                     _ptr(O), _ptr(L), _stream(stream)))
+    return O, L
+
+
+def lsa_merge_partials(O_parts, lse_parts, out=None, lse=None, stream=None):
+    """LSE-weighted merge (C: lsa_merge_partials) of O_parts [n][rows...][Hq][d] with
+    lse_parts [n][rows...][Hq]; returns O [rows...][Hq][d] (and lse when given)."""
+    _cuda(O_parts, lse_parts, out, lse)
+    n = O_parts.shape[0]
+    Hq, d = O_parts.shape[-2], O_parts.shape[-1]
+    rows = O_parts[0].numel() // (Hq * d)
+    O = out if out is not None else torch.empty(O_parts.shape[1:], dtype=O_parts.dtype,
+                                                device=O_parts.device)
+    _check(_lib.lsa_merge_partials(_ptr(O_parts), _ptr(lse_parts), _dtype_code(O_parts), n, rows,
+                                   Hq, d, _ptr(O), _ptr(lse), _stream(stream)))
+    return O
 
 
 def lsa_prefill_workspace_bytes(index, Nq, Hq, Hkv, d, budget, window, sinks):

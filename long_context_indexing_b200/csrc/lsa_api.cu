@@ -578,6 +578,63 @@ lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtyp
     return LSA_OK;
 }
 
+size_t lsa_attend_key_range_workspace_bytes(int64_t B, int64_t Nq, int s_max)
+{
+    if (B < 1 || Nq < 0 || s_max < 1) return 0;
+    return al256((size_t)B * Nq * s_max * 4) + al256((size_t)B * Nq * 4);
+}
+
+lsa_status lsa_attend_key_range(const void* Q, const void* K_shard, const void* V_shard,
+                                lsa_dtype dtype, int64_t B, int64_t Nq, int Hq, int Hkv, int d,
+                                const int32_t* indices, const int32_t* counts, int s_max,
+                                int64_t key_lo, int64_t key_hi, float scale, void* workspace,
+                                size_t ws_bytes, void* O_part, float* lse_part, void* stream)
+{
+    if (!Q || !K_shard || !V_shard || !indices || !counts || !O_part || !lse_part || !workspace)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
+    if (B < 1 || Nq < 0 || s_max < 1 || key_lo < 0 || key_hi <= key_lo ||
+        key_hi - key_lo > 2147483647LL)
+        return fail(LSA_ERR_INVALID_ARG, "bad sizes or key range");
+    lsa_status sh = check_attn_shape(Hq, Hkv, d, dtype);
+    if (sh != LSA_OK) return sh;
+    if (B * Nq * Hkv > 2147483647LL) return fail(LSA_ERR_UNSUPPORTED, "too many (query, head) pairs");
+    if (!(scale > 0.f)) return fail(LSA_ERR_INVALID_ARG, "scale must be > 0");
+    if (ws_bytes < lsa_attend_key_range_workspace_bytes(B, Nq, s_max))
+        return fail(LSA_ERR_WORKSPACE, "workspace too small");
+    if (!aligned16(Q) || !aligned16(K_shard) || !aligned16(V_shard) || !aligned16(indices) ||
+        !aligned16(counts) || !aligned16(O_part) || !aligned16(lse_part) || !aligned16(workspace))
+        return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    if (Nq == 0) return LSA_OK;
+    const cudaStream_t st = (cudaStream_t)stream;
+    int32_t* loc_idx = (int32_t*)workspace;
+    int32_t* loc_cnt = (int32_t*)((char*)workspace + al256((size_t)B * Nq * s_max * 4));
+    cudaError_t e = launch_range_filter(indices, counts, B * Nq, s_max, key_lo, key_hi, loc_idx,
+                                        loc_cnt, st);
+    if (e == cudaSuccess)
+        e = launch_attn(Q, K_shard, V_shard, dtype, B, Nq, key_hi - key_lo, Hq, Hkv, d, loc_idx,
+                        loc_cnt, s_max, scale, O_part, lse_part, st);
+    if (e == cudaSuccess) e = launch_range_empty(loc_cnt, B * Nq, Hq, d, dtype, O_part, lse_part, st);
+    if (e != cudaSuccess) return cuda_fail(e, "key-range attention");
+    return LSA_OK;
+}
+
+lsa_status lsa_merge_partials(const void* O_parts, const float* lse_parts, lsa_dtype dtype,
+                              int n_parts, int64_t rows, int Hq, int d, void* O, float* lse,
+                              void* stream)
+{
+    if (!O_parts || !lse_parts || !O) return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
+    if (n_parts < 1 || n_parts > 32 || rows < 0 || Hq < 1 || d < 1 || d > 1024)
+        return fail(LSA_ERR_INVALID_ARG, "bad sizes (1 <= n_parts <= 32)");
+    if (!aligned16(O_parts) || !aligned16(lse_parts) || !aligned16(O) || (lse && !aligned16(lse)))
+        return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    cudaError_t e = launch_merge_partials(O_parts, lse_parts, dtype, n_parts, rows, Hq, d, O, lse,
+                                          (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "merge of partials");
+    return LSA_OK;
+}
+
 size_t lsa_prefill_workspace_bytes(const lsa_index* idx, int64_t Nq, int Hq, int Hkv, int d,
                                    lsa_select_params sp)
 {

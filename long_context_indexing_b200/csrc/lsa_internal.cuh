@@ -298,6 +298,18 @@ cudaError_t launch_bucket_attn(const IndexView& ix, int64_t n_blk, const BucketP
 // True when the tensor-core candidate scorer is compiled in.
 bool tc_scoring_available();
 
+// Context parallel (k_cp.cu): a row's selected positions inside [lo, hi) as
+// shard rows; zero output / -inf lse for rows without one; the LSE-weighted
+// merge of n_parts partial results [n_parts][rows][Hq][d].
+cudaError_t launch_range_filter(const int32_t* indices, const int32_t* counts, int64_t rows,
+                                int s_max, int64_t lo, int64_t hi, int32_t* loc_idx,
+                                int32_t* loc_cnt, cudaStream_t st);
+cudaError_t launch_range_empty(const int32_t* loc_cnt, int64_t rows, int Hq, int d, lsa_dtype dt,
+                               void* O, float* lse, cudaStream_t st);
+cudaError_t launch_merge_partials(const void* parts, const float* lse_parts, lsa_dtype dt,
+                                  int n_parts, int64_t rows, int Hq, int d, void* O, float* lse,
+                                  cudaStream_t st);
+
 cudaError_t launch_attn(const void* Q, const void* K, const void* V, lsa_dtype dt, int64_t B,
                         int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
                         const int32_t* indices, const int32_t* counts, int s_max, float scale,

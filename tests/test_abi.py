@@ -167,3 +167,26 @@ def test_query_range_entry_argument_checks():
     assert f(h, None, *args[1:5], 4096, 4160, 0, 32, 8, 2, 64, S, fake, ws, fake, None) == 1
     assert f(h, *args[:5], 4096, 4160, 0, 32, 8, 2, 64, S, fake, 16, fake, None) == 3
     lsa._lib.lsa_index_release(h)
+
+
+def test_context_parallel_entry_argument_checks():
+    # lsa_attend_key_range refuses an empty or negative key range, NULL
+    # arguments, a short workspace and misaligned pointers, and
+    # lsa_merge_partials a part count outside 1 .. 32, before any launch.
+    fake = ctypes.c_void_p(1 << 22)
+    f = lsa._lib.lsa_attend_key_range
+    ws = lsa._lib.lsa_attend_key_range_workspace_bytes(1, 16, 64)
+    assert ws >= 16 * 64 * 4 + 16 * 4
+    assert lsa._lib.lsa_attend_key_range_workspace_bytes(0, 16, 64) == 0
+    base = [fake, fake, fake, lsa.BF16, 1, 16, 8, 2, 64, fake, fake, 64]
+    for lo, hi in ((100, 100), (-1, 50), (50, 10)):
+        assert f(*base, lo, hi, 0.125, fake, ws, fake, fake, None) == 1
+    assert f(None, *base[1:], 0, 256, 0.125, fake, ws, fake, fake, None) == 1
+    assert f(*base, 0, 256, 0.125, fake, ws, fake, None, None) == 1          # lse required
+    assert f(*base, 0, 256, 0.125, fake, 16, fake, fake, None) == 3          # workspace
+    odd = ctypes.c_void_p((1 << 22) + 4)
+    assert f(odd, *base[1:], 0, 256, 0.125, fake, ws, fake, fake, None) == 2  # alignment
+    m = lsa._lib.lsa_merge_partials
+    for n in (0, 33):
+        assert m(fake, fake, lsa.BF16, n, 16, 8, 64, fake, None, None) == 1
+    assert m(None, fake, lsa.BF16, 2, 16, 8, 64, fake, None, None) == 1

@@ -132,6 +132,79 @@ def test_query_split_over_gloo_matches_the_whole_chunk():
     assert rng == (0, 32)
 
 
+def _context_worker(rank, ws, port, q):
+    # The KV cache in two shards of whole blocks, the oracle standing in for
+    # the GPU on each rank: every rank selects for the whole chunk, attends
+    # over the selected keys of its shard (output and log-sum-exp), the
+    # partials are exchanged by row blocks, and the LSE-weighted merge of a
+    # rank's rows equals the single-rank attention of those rows.
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(ws), LOCAL_RANK=str(rank), CUDA_VISIBLE_DEVICES="")
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    import oracle
+    import synth
+    r, w = bench._dist(timeout_s=60)
+    wl = synth.workload("tiny", T=2048, nq=64, Hq=4, Hkv=1, d=64, M=16, G=64, k=4, R=200, W=32,
+                        S=4)
+    inp = synth.prefill_inputs(wl, 5, "cpu")
+    T_old = wl.T - wl.nq
+    orc = oracle.Index(wl.T, wl.p, wl.G, wl.k, wl.L, rt_bf16=False)
+    orc.extend(inp["latent_K"][0].numpy(), 0, wl.T)
+    pos = T_old + np.arange(wl.nq)
+    sel, cnt, _, _ = oracle.select(orc, inp["latent_Q"][0].numpy(), pos, wl.R, wl.W, wl.S)
+    lo, hi = bench._context_shard(wl.T, wl.p * wl.G, r, w)
+    Q, K, V = (inp[k][0].numpy() for k in ("Q", "K", "V"))
+    O_r = np.zeros(Q.shape, np.float32)
+    L_r = np.full(Q.shape[:2], -np.inf, np.float32)
+    loc = np.full(sel.shape, -1, np.int32)
+    lc = np.zeros(cnt.shape, np.int32)
+    for i in range(wl.nq):
+        keep = [t for t in sel[i, :cnt[i]] if lo <= t < hi]
+        loc[i, :len(keep)] = keep
+        lc[i] = len(keep)
+    has = lc > 0
+    if has.any():
+        o, l = oracle.attend(Q[has], K, V, loc[has], lc[has])
+        O_r[has], L_r[has] = o, l
+    O_parts = bench._exchange_rows(torch.from_numpy(O_r), r, w).double().numpy()
+    L_parts = bench._exchange_rows(torch.from_numpy(L_r), r, w).double().numpy()
+    torch.distributed.destroy_process_group()
+    M = L_parts.max(0)
+    wgt = np.exp(L_parts - M)                               # [parts][rows][heads]
+    O_mine = (wgt[..., None] * O_parts).sum(0) / wgt.sum(0)[..., None]
+    q0, q1 = bench._query_slice(wl.nq, r, w)
+    ref_O, _ = oracle.attend(Q[q0:q1], K, V, sel[q0:q1], cnt[q0:q1])
+    q.put((r, (lo, hi), float(np.abs(O_mine - ref_O).max()), bool(np.isinf(L_r).any())))
+
+
+def test_context_split_over_gloo_matches_the_whole_chunk():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_context_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=240) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [x[1] for x in res] == [(0, 1024), (1024, 2048)]
+    for _, _, err, _ in res:
+        assert err < 1e-5
+
+
+def test_context_shards_cover_the_cache():
+    sys.path.insert(0, ROOT)
+    import bench
+    for T, span, ws in ((10485760, 4096, 8), (10485760, 4096, 3), (4096 * 5 + 100, 4096, 2)):
+        got = [bench._context_shard(T, span, r, ws) for r in range(ws)]
+        assert got[0][0] == 0 and got[-1][1] == T
+        for (a, b), (c, _) in zip(got, got[1:]):
+            assert b == c and a < b and b % span == 0
+
+
 def test_query_slice_ranges():
     sys.path.insert(0, ROOT)
     import bench
