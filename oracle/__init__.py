@@ -59,6 +59,9 @@ def _lib():
         lib.orc_attend.argtypes = [P, P, P, I64, I64, I, I, I, P, P, I,
                                    ctypes.c_double, P, P]
         lib.orc_attend.restype = I
+        lib.orc_attend_backward.argtypes = [P, P, P, P, I64, I64, I, I, I, P, P, I,
+                                            ctypes.c_double, P, P, P]
+        lib.orc_attend_backward.restype = I
         lib.orc_num_threads.argtypes = []
         lib.orc_num_threads.restype = I
         lib.orc_set_num_threads.argtypes = [I]
@@ -301,6 +304,29 @@ def attend(Q, K, V, idx, cnt, scale=None):
     _check(_lib().orc_attend(_p(Q), _p(K), _p(V), T, nq, Hq, Hkv, d, _p(idx), _p(cnt),
                              idx.shape[1], float(scale), _p(O), _p(lse)), "attend")
     return O, lse
+
+
+def attend_backward(Q, K, V, dO, idx, cnt, scale=None):
+    """Gradients of attend's output O for an upstream gradient dO [nq][Hq][d]
+    (the selected indices kept from the forward pass): dQ [nq][Hq][d], dK and
+    dV [T][Hkv][d], each summed over every query and head that read the key.
+    p = softmax(scale <q, k_t>) over the query's keys; dV_t += p_t dO,
+    dS_t = p_t (<dO, v_t> - sum_u p_u <dO, v_u>), dQ = scale sum_t dS_t k_t,
+    dK_t += scale dS_t q; binary64 inside (lsa_oracle.c orc_attend_backward)."""
+    Q, K, V, dO = _f32(Q), _f32(K), _f32(V), _f32(dO)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    cnt = np.ascontiguousarray(cnt, dtype=np.int32)
+    nq, Hq, d = Q.shape
+    T, Hkv, _ = K.shape
+    if scale is None:
+        scale = float(np.float32(1.0 / math.sqrt(d)))
+    dQ = np.empty((nq, Hq, d), np.float32)
+    dK = np.empty((T, Hkv, d), np.float32)
+    dV = np.empty((T, Hkv, d), np.float32)
+    _check(_lib().orc_attend_backward(_p(Q), _p(K), _p(V), _p(dO), T, nq, Hq, Hkv, d, _p(idx),
+                                      _p(cnt), idx.shape[1], float(scale), _p(dQ), _p(dK),
+                                      _p(dV)), "attend_backward")
+    return dQ, dK, dV
 
 
 def default_scale(d):

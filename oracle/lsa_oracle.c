@@ -640,3 +640,85 @@ int orc_attend(const float* Q, const float* K, const float* V, int64_t T, int64_
     }
     return err;
 }
+
+/* Gradients of orc_attend's outputs for an upstream gradient dO ("Latent Sparse
+ * Attention: un indice gerarchico per contesti lunghi", paragraph on N-LSA's
+ * memory: the selected indices are kept for the backward pass; the attention
+ * itself is unchanged, so its gradients are those of softmax attention over
+ * the selected keys).  Per query i and head h, with z_t = scale <q, k_t> over
+ * the selected t, p_t = exp(z_t - max) / sum:
+ *   dV_t += p_t dO,   dP_t = <dO, v_t>,   D = sum_t p_t dP_t,
+ *   dS_t = p_t (dP_t - D),   dQ = scale sum_t dS_t k_t,   dK_t += scale dS_t q.
+ * Binary64 throughout, in the order written (queries, heads, keys ascending);
+ * dQ rounded to binary32; dK, dV summed in binary64 over every query and head,
+ * then rounded.  Serial. */
+int orc_attend_backward(const float* Q, const float* K, const float* V, const float* dO,
+                        int64_t T, int64_t nq, int Hq, int Hkv, int d, const int32_t* idx,
+                        const int32_t* count, int s_max, double scale, float* dQ, float* dK,
+                        float* dV)
+{
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || s_max < 1) return ORC_EINVAL;
+    const int grp = Hq / Hkv;
+    double* z = (double*)malloc(sizeof(double) * (size_t)s_max);
+    double* pp = (double*)malloc(sizeof(double) * (size_t)s_max);
+    double* dq = (double*)malloc(sizeof(double) * (size_t)d);
+    double* gk = (double*)calloc((size_t)T * Hkv * d, sizeof(double));
+    double* gv = (double*)calloc((size_t)T * Hkv * d, sizeof(double));
+    int err = (!z || !pp || !dq || !gk || !gv) ? ORC_ENOMEM : ORC_OK;
+    for (int64_t i = 0; i < nq && err == ORC_OK; ++i) {
+        const int32_t* ix = idx + i * s_max;
+        const int n = count[i];
+        if (n < 1 || n > s_max) {
+            err = ORC_EINVAL;
+            break;
+        }
+        for (int x = 0; x < n; ++x)
+            if (ix[x] < 0 || ix[x] >= T) err = ORC_EINVAL;
+        if (err != ORC_OK) break;
+        for (int h = 0; h < Hq; ++h) {
+            const int kh = h / grp;
+            const float* qh = Q + (i * Hq + h) * (int64_t)d;
+            const float* gh = dO + (i * Hq + h) * (int64_t)d;
+            double mx = -INFINITY;
+            for (int x = 0; x < n; ++x) {
+                z[x] = scale * orc_dot(qh, K + ((int64_t)ix[x] * Hkv + kh) * d, d);
+                if (z[x] > mx) mx = z[x];
+            }
+            double den = 0.0;
+            for (int x = 0; x < n; ++x) {
+                pp[x] = exp(z[x] - mx);
+                den = den + pp[x];
+            }
+            for (int x = 0; x < n; ++x) pp[x] = pp[x] / den;
+            // dP_t, kept in z; D
+            double D = 0.0;
+            for (int x = 0; x < n; ++x) {
+                z[x] = orc_dot(gh, V + ((int64_t)ix[x] * Hkv + kh) * d, d);
+                D = D + pp[x] * z[x];
+            }
+            for (int c = 0; c < d; ++c) dq[c] = 0.0;
+            for (int x = 0; x < n; ++x) {
+                const double ds = pp[x] * (z[x] - D);
+                const int64_t row = ((int64_t)ix[x] * Hkv + kh) * d;
+                for (int c = 0; c < d; ++c) {
+                    dq[c] = dq[c] + ds * (double)K[row + c];
+                    gk[row + c] = gk[row + c] + scale * ds * (double)qh[c];
+                    gv[row + c] = gv[row + c] + pp[x] * (double)gh[c];
+                }
+            }
+            float* oq = dQ + (i * Hq + h) * (int64_t)d;
+            for (int c = 0; c < d; ++c) oq[c] = (float)(scale * dq[c]);
+        }
+    }
+    if (err == ORC_OK)
+        for (int64_t x = 0; x < T * Hkv * d; ++x) {
+            dK[x] = (float)gk[x];
+            dV[x] = (float)gv[x];
+        }
+    free(z);
+    free(pp);
+    free(dq);
+    free(gk);
+    free(gv);
+    return err;
+}
