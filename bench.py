@@ -559,6 +559,8 @@ def run_lsa(args, rank, ws):
 
     tree = None if args.tree_super <= 0 else _tree_measure(args, w, inp, idx, T_old, stream)
     full = None if args.no_full_prefill else _full_prefill(w, inp, work, O, stream)
+    bwd = None if args.backward_queries <= 0 else _backward_measure(w, inp, idx, T_old, work,
+                                                                     args.backward_queries, stream)
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -592,7 +594,7 @@ def run_lsa(args, rank, ws):
             "gpu_launches": launches, "clocks": clocks,
             "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "index_build_prefix_s": round(build_s, 3), "selection_fallbacks": fallbacks,
-            "tree": tree, "full_prefill": full, "decode": decode}
+            "tree": tree, "full_prefill": full, "backward": bwd, "decode": decode}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -678,6 +680,38 @@ def _full_prefill(w, inp, work, O, stream):
             "total_ms": round(total, 2), "queries_per_s": round(w.T * w.B / (total * 1e-3), 1),
             "first_chunk_ms": round(per[0], 4), "last_chunk_ms": round(per[-1], 4),
             "selection_fallbacks": fb}
+
+
+def _backward_measure(w, inp, idx, T_old, work, n, stream):
+    """Gradients of the attention over stored selections (lsa_sparse_attn_backward)
+    for n of the chunk's queries (every (nq/n)-th): their selections from a
+    fresh chunk call, the forward's O and lse from lsa_sparse_attn, a random
+    upstream gradient, fp32 dK / dV accumulators over the whole cache.  One
+    timed call after one untimed one, CUDA events."""
+    import long_context_indexing_b200 as lsa
+
+    lsa.lsa_prefill_chunk(idx, inp["latent_K"], inp["latent_Q"], inp["Q"], inp["K"], inp["V"],
+                          T_old, w.T, w.R, w.W, w.S, workspace=work)
+    sel_i, sel_c = lsa.prefill_selection_views(work, w.B, w.nq, w.s_max)
+    rows = _sample_rows(w, n, "cuda")
+    Qs = inp["Q"][:, rows].contiguous()
+    ii = sel_i[:, rows].contiguous()
+    cc = sel_c[:, rows].contiguous()
+    O, lse = lsa.lsa_sparse_attn(Qs, inp["K"], inp["V"], ii, cc, return_lse=True)
+    gen = torch.Generator(device="cuda").manual_seed(0)
+    dO = torch.randn(Qs.shape, generator=gen, device="cuda").to(Qs.dtype)
+    dK = torch.zeros(inp["K"].shape, dtype=torch.float32, device="cuda")
+    dV = torch.zeros_like(dK)
+    lsa.lsa_sparse_attn_backward(Qs, inp["K"], inp["V"], O, lse, dO, ii, cc, dK=dK, dV=dV)
+    ms = _events_time(lambda: lsa.lsa_sparse_attn_backward(Qs, inp["K"], inp["V"], O, lse, dO,
+                                                           ii, cc, dK=dK, dV=dV), 1, stream)
+    keys = int(cc.sum().item())
+    del dK, dV
+    torch.cuda.empty_cache()
+    return {"what": "gradients of the attention over stored selections for %d of the chunk's "
+                    "queries (every %d-th), fp32 dK/dV accumulators" % (len(rows), w.nq // len(rows)),
+            "ms": round(ms, 3), "queries_per_s": round(len(rows) / (ms * 1e-3), 1),
+            "selected_keys": keys}
 
 
 # ------------------------------------------------------------------- decode --
@@ -835,6 +869,8 @@ def main():
     ap.add_argument("--ref-queries", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--backward-queries", type=int, default=512,
+                    help="queries of the chunk whose attention gradients are timed (0: skip)")
     ap.add_argument("--no-full-prefill", action="store_true",
                     help="skip the whole-context chunk-by-chunk prefill measurement")
     ap.add_argument("--tree-super", type=int, default=256,

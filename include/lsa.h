@@ -282,6 +282,25 @@ lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtyp
                            const int32_t* indices, const int32_t* counts, int s_max, float scale,
                            void* O, float* lse, void* stream);
 
+/* Gradients of lsa_sparse_attn over the same stored selection ("Latent Sparse
+ * Attention: un indice gerarchico per contesti lunghi", paragraph on N-LSA's
+ * memory: the selected indices are kept for the backward pass).  Inputs: the
+ * forward's Q, K, V, indices, counts, scale, its output O and lse (as
+ * lsa_sparse_attn returns them), and the upstream gradient dO [B][Nq][Hq][d]
+ * (dtype).  With p_t = exp(scale <q, k_t> - lse):
+ *   D = <dO, O>, dS_t = p_t (<dO, v_t> - D),
+ *   dQ = scale sum_t dS_t k_t          -> dQ [B][Nq][Hq][d] (dtype), written;
+ *   dK_t += scale dS_t q, dV_t += p_t dO -> dK, dV [B][T_cap][Hkv][d] f32,
+ *   ADDED to (zero them first; keys read by several queries receive several
+ *   additions in no fixed order).
+ * Hq/Hkv <= 8, d <= 128; listed indices outside [0, T_cap) are skipped.
+ * Caller-owned device memory, 16-byte aligned; asynchronous on `stream`. */
+lsa_status lsa_sparse_attn_backward(const void* Q, const void* K, const void* V, const void* O,
+                                    const float* lse, const void* dO, lsa_dtype dtype, int64_t B,
+                                    int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
+                                    const int32_t* indices, const int32_t* counts, int s_max,
+                                    float scale, void* dQ, float* dK, float* dV, void* stream);
+
 /* ---------------------------------------------------------------------------
  * KV cache in shards of whole blocks ("Latent Sparse Attention: un indice
  * gerarchico per contesti lunghi", paragraph on memory: with context

@@ -21,6 +21,7 @@ __all__ = [
     "lsa_select_workspace_bytes", "lsa_tree_select_workspace_bytes",
     "lsa_sparse_attn", "lsa_prefill_chunk", "lsa_prefill_workspace_bytes",
     "lsa_attend_key_range", "lsa_attend_key_range_workspace_bytes", "lsa_merge_partials",
+    "lsa_sparse_attn_backward",
     "lsa_prefill_partial_slots", "lsa_prefill_select", "lsa_prefill_attend",
     "lsa_prefill_chunk_host", "lsa_prefill_chunk_queries", "LsaTree", "set_wait_limit",
     "lsa_decode_workspace_bytes", "lsa_decode_step", "lsa_select_noalloc", "library_path", "kernel_launches", "F32",
@@ -69,6 +70,8 @@ def _declare(lib):
         "lsa_select_workspace_bytes": ([P, I64], SZ),
         "lsa_select": ([P, P, P, I64, SelectParams, P, P, I, P, SZ, P], I),
         "lsa_sparse_attn": ([P, P, P, I, I64, I64, I64, I, I, I, P, P, I, F, P, P, P], I),
+        "lsa_sparse_attn_backward": ([P, P, P, P, P, P, I, I64, I64, I64, I, I, I, P, P, I, F,
+                                      P, P, P, P], I),
         "lsa_attend_key_range_workspace_bytes": ([I64, I64, I], SZ),
         "lsa_attend_key_range": ([P, P, P, I, I64, I64, I, I, I, P, P, I, I64, I64, F, P, SZ, P,
                                   P, P], I),
@@ -305,6 +308,27 @@ def lsa_sparse_attn(Q, K, V, indices, counts, scale=None, return_lse=False, out=
                                 d, _ptr(indices), _ptr(counts), indices.shape[-1], scale, _ptr(O),
                                 _ptr(lse), _stream(stream)))
     return (O, lse) if return_lse else O
+
+
+def lsa_sparse_attn_backward(Q, K, V, O, lse, dO, indices, counts, scale=None, dK=None, dV=None,
+                             stream=None):
+    """Gradients of lsa_sparse_attn (C: lsa_sparse_attn_backward): returns (dQ, dK, dV); dK and
+    dV (fp32 [B][T_cap][Hkv][d]) are added to when given, else start from zero."""
+    _cuda(Q, K, V, O, lse, dO, indices, counts, dK, dV)
+    B, Nq, Hq, d = Q.shape
+    T_cap, Hkv = K.shape[1], K.shape[2]
+    if scale is None:
+        scale = float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))
+    dQ = torch.empty_like(Q)
+    if dK is None:
+        dK = torch.zeros(B, T_cap, Hkv, d, dtype=torch.float32, device=Q.device)
+    if dV is None:
+        dV = torch.zeros(B, T_cap, Hkv, d, dtype=torch.float32, device=Q.device)
+    _check(_lib.lsa_sparse_attn_backward(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse), _ptr(dO),
+                                         _dtype_code(Q), B, Nq, T_cap, Hq, Hkv, d, _ptr(indices),
+                                         _ptr(counts), indices.shape[-1], scale, _ptr(dQ),
+                                         _ptr(dK), _ptr(dV), _stream(stream)))
+    return dQ, dK, dV
 
 
 def lsa_attend_key_range_workspace_bytes(B, Nq, s_max):

@@ -578,6 +578,31 @@ lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtyp
     return LSA_OK;
 }
 
+lsa_status lsa_sparse_attn_backward(const void* Q, const void* K, const void* V, const void* O,
+                                    const float* lse, const void* dO, lsa_dtype dtype, int64_t B,
+                                    int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
+                                    const int32_t* indices, const int32_t* counts, int s_max,
+                                    float scale, void* dQ, float* dK, float* dV, void* stream)
+{
+    if (!Q || !K || !V || !O || !lse || !dO || !indices || !counts || !dQ || !dK || !dV)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
+    if (B < 1 || Nq < 0 || T_cap < 1 || T_cap > 2147483647LL || s_max < 1)
+        return fail(LSA_ERR_INVALID_ARG, "bad sizes");
+    if (!attn_backward_supported(Hq, Hkv, d))
+        return fail(LSA_ERR_UNSUPPORTED, "backward needs Hq %% Hkv == 0, Hq/Hkv <= 8, d <= 128");
+    if (B * Nq * Hkv > 2147483647LL) return fail(LSA_ERR_UNSUPPORTED, "too many (query, head) pairs");
+    if (!(scale > 0.f)) return fail(LSA_ERR_INVALID_ARG, "scale must be > 0");
+    const void* ptrs[] = {Q, K, V, O, lse, dO, indices, counts, dQ, dK, dV};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    cudaError_t e = launch_attn_backward(Q, K, V, O, lse, dO, dtype, B, Nq, T_cap, Hq, Hkv, d,
+                                         indices, counts, s_max, scale, dQ, dK, dV, nullptr,
+                                         (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "sparse attention backward");
+    return LSA_OK;
+}
+
 size_t lsa_attend_key_range_workspace_bytes(int64_t B, int64_t Nq, int s_max)
 {
     if (B < 1 || Nq < 0 || s_max < 1) return 0;

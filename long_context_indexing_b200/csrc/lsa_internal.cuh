@@ -298,6 +298,16 @@ cudaError_t launch_bucket_attn(const IndexView& ix, int64_t n_blk, const BucketP
 // True when the tensor-core candidate scorer is compiled in.
 bool tc_scoring_available();
 
+// Gradients of the sparse attention (k_attn_bwd.cu): dQ written, dK and dV
+// (fp32) added to.
+bool attn_backward_supported(int Hq, int Hkv, int d);
+cudaError_t launch_attn_backward(const void* Q, const void* K, const void* V, const void* O,
+                                 const float* lse, const void* dO, lsa_dtype dt, int64_t B,
+                                 int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
+                                 const int32_t* indices, const int32_t* counts, int s_max,
+                                 float scale, void* dQ, float* dK, float* dV, uint32_t* status,
+                                 cudaStream_t st);
+
 // Context parallel (k_cp.cu): a row's selected positions inside [lo, hi) as
 // shard rows; zero output / -inf lse for rows without one; the LSE-weighted
 // merge of n_parts partial results [n_parts][rows][Hq][d].

@@ -190,3 +190,20 @@ def test_context_parallel_entry_argument_checks():
     for n in (0, 33):
         assert m(fake, fake, lsa.BF16, n, 16, 8, 64, fake, None, None) == 1
     assert m(None, fake, lsa.BF16, 2, 16, 8, 64, fake, None, None) == 1
+
+
+def test_backward_entry_argument_checks():
+    # lsa_sparse_attn_backward refuses NULL arguments, unsupported head
+    # shapes and misaligned pointers before any launch.
+    fake = ctypes.c_void_p(1 << 22)
+    f = lsa._lib.lsa_sparse_attn_backward
+    ok = [fake] * 6 + [lsa.BF16, 1, 16, 256, 8, 2, 64, fake, fake, 32, 0.125, fake, fake, fake, None]
+    bad = list(ok)
+    bad[0] = None
+    assert f(*bad) == 1
+    shape = list(ok)
+    shape[10], shape[11] = 16, 1          # 16 query heads per KV head
+    assert f(*shape) == 7                 # LSA_ERR_UNSUPPORTED
+    odd = list(ok)
+    odd[5] = ctypes.c_void_p((1 << 22) + 8)
+    assert f(*odd) == 2
