@@ -561,6 +561,7 @@ def run_lsa(args, rank, ws):
     full = None if args.no_full_prefill else _full_prefill(w, inp, work, O, stream)
     bwd = None if args.backward_queries <= 0 else _backward_measure(w, inp, idx, T_old, work,
                                                                      args.backward_queries, stream)
+    per_key = None if args.no_per_key else _per_key_measure(w, inp, stage_ms, stream)
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -594,7 +595,8 @@ def run_lsa(args, rank, ws):
             "gpu_launches": launches, "clocks": clocks,
             "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "index_build_prefix_s": round(build_s, 3), "selection_fallbacks": fallbacks,
-            "tree": tree, "full_prefill": full, "backward": bwd, "decode": decode}
+            "tree": tree, "full_prefill": full, "backward": bwd, "per_key": per_key,
+            "decode": decode}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -712,6 +714,37 @@ def _backward_measure(w, inp, idx, T_old, work, n, stream):
                     "queries (every %d-th), fp32 dK/dV accumulators" % (len(rows), w.nq // len(rows)),
             "ms": round(ms, 3), "queries_per_s": round(len(rows) / (ms * 1e-3), 1),
             "selected_keys": keys}
+
+
+def _per_key_measure(w, inp, stage_ms, stream):
+    """The brute-force latent per-key indexer (lsa_select_per_key) on the same
+    chunk: every long-range key of each of the chunk's queries scored on the
+    tensor cores (two passes), the exact top-R read, emitted like the bucket
+    selection.  One timed call after one untimed one, CUDA events; compared
+    with the bucket selection and attention stages of the chunk."""
+    import long_context_indexing_b200 as lsa
+
+    pos = inp["positions"].to(torch.int32).contiguous()
+    sel = lsa.lsa_select_per_key(inp["latent_K"], inp["latent_Q"], pos, w.R, w.W, w.S)
+    work = sel[2]
+    fb = lsa.lsa_select_per_key_check(work)
+    ms = _events_time(lambda: lsa.lsa_select_per_key(inp["latent_K"], inp["latent_Q"], pos, w.R,
+                                                     w.W, w.S, workspace=work), 1, stream)
+    fb = max(fb, lsa.lsa_select_per_key_check(work))
+    # scores per pass: every query against its long-range keys [S, pos - W]
+    scored = int((pos.to(torch.int64) - w.W - w.S + 1).clamp(min=0).sum().item())
+    flops = 2 * 2.0 * scored * 64
+    sel_ms, att_ms = stage_ms.get("extend_and_select"), stage_ms.get("attend")
+    del sel, work
+    torch.cuda.empty_cache()
+    return {"what": "brute-force latent per-key indexer over the chunk's %d queries: every "
+                    "long-range key scored on the tensor cores (two passes), exact top-%d by "
+                    "binary64 rescoring, the baseline the bucket selection replaces" % (w.nq, w.R),
+            "ms": round(ms, 3), "queries_per_s": round(w.B * w.nq / (ms * 1e-3), 1),
+            "keys_scored_per_pass": scored, "tensor_tflops_effective": round(flops / ms * 1e-9, 1),
+            "fallbacks": int(fb),
+            "vs_bucket_selection": round(ms / sel_ms, 2) if sel_ms else None,
+            "indexer_share_with_bucket_attention": round(ms / (ms + att_ms), 3) if att_ms else None}
 
 
 # ------------------------------------------------------------------- decode --
@@ -871,6 +904,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--backward-queries", type=int, default=512,
                     help="queries of the chunk whose attention gradients are timed (0: skip)")
+    ap.add_argument("--no-per-key", action="store_true",
+                    help="skip the brute-force per-key indexer measurement")
     ap.add_argument("--no-full-prefill", action="store_true",
                     help="skip the whole-context chunk-by-chunk prefill measurement")
     ap.add_argument("--tree-super", type=int, default=256,

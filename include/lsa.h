@@ -268,6 +268,55 @@ lsa_status lsa_tree_select(const lsa_index* idx, const void* tree, int n_super, 
                            void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Brute-force latent per-key indexer: the baseline that LSA's bucket
+ * retrieval replaces ("Prefrontal's ...", section "What it changes": the
+ * indexer that scores every earlier key for every query, quadratic in the
+ * context and most of a layer's prefill time at 10M tokens; "Latent Sparse
+ * Attention: un indice gerarchico per contesti lunghi", paragraph on the read
+ * budget).  No index is involved: every long-range key of a query is scored.
+ *
+ * For query i of sequence b at p = positions[b][i] (0 <= p < n_keys): the
+ * keys t in [sinks, p - window] are ranked by <latent_Q[b][i], latent_K[b][t]>
+ * (the exact products summed in binary64 in ascending dimension), highest
+ * first, ties to the lower position, and the `budget` first are taken.  The
+ * row is emitted as lsa_select emits it: sinks 0 .. min(sinks, p+1)-1, the
+ * taken keys in ascending position, the window max(p-window+1, n_sinks) .. p,
+ * -1 padded to s_max; counts[b][i] is its length.  A position outside
+ * [0, n_keys) gives an empty row (count 0) and LSA_ERR_INVALID_ARG from
+ * lsa_select_per_key_check.
+ *
+ * Scores come from the tensor cores (bf16 in, fp32 accumulated); the exact
+ * ranking is then proved: a threshold that at least `budget` keys reach,
+ * lowered by twice a bound on the fp32 error, keeps every key of the exact
+ * top set among the candidates, which are ranked by exact binary64 scores.
+ * A query with more than 8192 candidates (scores tied over that many keys)
+ * ranks every eligible key exactly instead (counted by the check).
+ * ------------------------------------------------------------------------- */
+
+/* Workspace bytes for lsa_select_per_key (0 on bad sizes).  About
+ * B*Nq*(2*min(32768, T_cap rounded up to a power of two) + 32 KiB + 12) bytes:
+ * 3.1 GB for 32,768 queries of one 10M-key sequence. */
+size_t lsa_select_per_key_workspace_bytes(int64_t B, int64_t Nq, int64_t T_cap);
+
+/* latent_K [B][T_cap][64] and latent_Q [B][Nq][64] of dtype LSA_BF16 (LSA_F32
+ * returns LSA_ERR_UNSUPPORTED); keys 0 .. n_keys-1 of each sequence are read
+ * (n_keys <= T_cap); positions [B][Nq] int32; sp.budget <= 4096; indices
+ * [B][Nq][s_max] with s_max >= budget + window + sinks; counts [B][Nq].
+ * B*T_cap and B*Nq must stay below 2^31.  The workspace holds the call's
+ * status until the next call on it. */
+lsa_status lsa_select_per_key(const void* latent_K, lsa_dtype dtype, int64_t B, int64_t T_cap,
+                              int64_t n_keys, const void* latent_Q, const int32_t* positions,
+                              int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
+                              int s_max, void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream` and reads the status the last lsa_select_per_key on
+ * this workspace left: LSA_ERR_TIMEOUT (a bounded wait gave up; the outputs
+ * are undefined), LSA_ERR_INVALID_ARG (a position outside [0, n_keys)), else
+ * LSA_OK.  fallbacks (nullable) receives the queries ranked over every
+ * eligible key. */
+lsa_status lsa_select_per_key_check(const void* workspace, int64_t* fallbacks, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Exact sparse attention ("Prefrontal's ...", section "What it changes")
  *
  * For query (b, i) and head h with KV head kh = h / (Hq/Hkv):
@@ -450,10 +499,11 @@ lsa_status lsa_prefill_chunk_host(lsa_index* idx, const void* h_latent_K, const 
  * polls each bounded wait makes before it gives up, in every kernel that waits
  * on a copy or on another warp: the tensor-core centroid scorer (bf16
  * selection with Nq >= 128), the tensor-core attention tiles of bf16 prefill
- * chunks, and the per-query bf16 attention kernel (decode steps, prefill rows
- * attended key by key, lsa_sparse_attn).  A wait that gives up records
- * LSA_ERR_TIMEOUT in the index status word for lsa_index_check (lsa_sparse_attn
- * has no index and no status word), and the kernel still leaves cleanly: its
+ * chunks, the per-query bf16 attention kernel (decode steps, prefill rows
+ * attended key by key, lsa_sparse_attn) and the per-key indexer's scoring
+ * passes.  A wait that gives up records LSA_ERR_TIMEOUT in the index status
+ * word for lsa_index_check (in the workspace for lsa_select_per_key_check;
+ * lsa_sparse_attn has no status word), and the kernel still leaves cleanly: its
  * copies and MMAs in flight are waited for with the default limit, so the
  * context stays usable; the outputs of such a launch are undefined.  polls < 0
  * restores the defaults (about 4 million polls for the tensor-core kernels, 16

@@ -94,6 +94,10 @@ def _declare(lib):
         "lsa_prefill_chunk_queries": ([P, P, P, P, P, P, I64, I64, I64, I64, I, I, I, SelectParams,
                                        P, SZ, P, P], I),
         "lsa_select_noalloc": ([P, P, P, I64, SelectParams, P, P, I, P], I),
+        "lsa_select_per_key_workspace_bytes": ([I64, I64, I64], SZ),
+        "lsa_select_per_key": ([P, I, I64, I64, I64, P, P, I64, SelectParams, P, P, I, P, SZ, P],
+                               I),
+        "lsa_select_per_key_check": ([P, ctypes.POINTER(I64), P], I),
         "lsa_decode_step": ([P, P, P, P, P, P, P, P, P, P, I, I, I, SelectParams, P, SZ, P, P], I),
     }
     for name, (args, res) in sigs.items():
@@ -292,6 +296,47 @@ def lsa_select_noalloc(index, latent_Q, positions, budget, window, sinks, indice
                                    SelectParams(budget, window, sinks), _ptr(indices),
                                    _ptr(counts), indices.shape[-1], _stream(stream)))
     return indices, counts
+
+
+def lsa_select_per_key_workspace_bytes(B, Nq, T_cap):
+    return int(_lib.lsa_select_per_key_workspace_bytes(B, Nq, T_cap))
+
+
+def lsa_select_per_key(latent_K, latent_Q, positions, budget, window, sinks, n_keys=None,
+                       s_max=None, workspace=None, stream=None):
+    """Brute-force per-key indexer over latent_K [B][T_cap][64] (keys
+    0 .. n_keys-1, default T_cap) for latent_Q [B][Nq][64] at positions
+    [B][Nq] (int32).  Returns (indices [B][Nq][s_max] int32, counts [B][Nq]
+    int32, workspace); lsa_select_per_key_check(workspace) reads the call's
+    status and fallback count."""
+    _cuda(latent_K, latent_Q, positions)
+    if positions.dtype != torch.int32:
+        raise TypeError("positions must be int32")
+    B, T_cap = latent_K.shape[0], latent_K.shape[1]
+    Nq = latent_Q.shape[1]
+    n_keys = T_cap if n_keys is None else int(n_keys)
+    s_max = s_max or (budget + window + sinks)
+    dev = latent_Q.device
+    indices = torch.empty(B, Nq, s_max, dtype=torch.int32, device=dev)
+    counts = torch.empty(B, Nq, dtype=torch.int32, device=dev)
+    need = _lib.lsa_select_per_key_workspace_bytes(B, Nq, T_cap)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check(_lib.lsa_select_per_key(_ptr(latent_K), _dtype_code(latent_K), B, T_cap, n_keys,
+                                   _ptr(latent_Q), _ptr(positions), Nq,
+                                   SelectParams(budget, window, sinks), _ptr(indices),
+                                   _ptr(counts), s_max, _ptr(workspace), workspace.numel(),
+                                   _stream(stream)))
+    return indices, counts, workspace
+
+
+def lsa_select_per_key_check(workspace, stream=None):
+    """Status of the last lsa_select_per_key on `workspace` (raises LsaError
+    on a device error); returns the number of queries that took the exact
+    fallback."""
+    fb = ctypes.c_int64(0)
+    _check(_lib.lsa_select_per_key_check(_ptr(workspace), ctypes.byref(fb), _stream(stream)))
+    return fb.value
 
 
 def lsa_sparse_attn(Q, K, V, indices, counts, scale=None, return_lse=False, out=None,

@@ -50,6 +50,7 @@
 #include "ptx.cuh"
 #include "hooks.cuh"
 #include "tmap.cuh"
+#include "tc_common.cuh"
 
 namespace lsa {
 
@@ -77,119 +78,9 @@ constexpr int TC_OFF_MISC = TC_OFF_BAR + TC_NBAR * 8;
 constexpr int TC_MISC_BYTES = TC_M * 4 + TC_EPI_THREADS * 4 + 64;
 constexpr int TC_SMEM = TC_OFF_MISC + TC_MISC_BYTES + 1024;   // + alignment slack
 
-// ---- tcgen05 / TMA wrappers -------------------------------------------------
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(ptx::smem_addr(dst)),
-        "l"((uint64_t)map), "r"(ptx::smem_addr(bar)), "r"(x), "r"(y)
-        : "memory");
-}
-
-__device__ __forceinline__ uint64_t sw128_desc(const void* smem_tile)
-{
-    const uint64_t a = ptx::smem_addr(smem_tile);
-    return ((a >> 4) & 0x3FFFull)   // start address
-           | (1ull << 16)           // leading byte offset (unused for 128B-swizzled K-major)
-           | (64ull << 32)          // stride byte offset: 8 rows x 128 B = 1024 B
-           | (1ull << 46)           // descriptor version (tcgen05)
-           | (2ull << 61);          // 128-byte swizzle
-}
-
 // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both
 // K-major, N = TC_N, M = 128.
-constexpr uint32_t TC_IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_N >> 3) << 17) |
-                              ((uint32_t)(TC_M >> 4) << 24);
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(TC_IDESC), "r"(accumulate));
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     ptx::smem_addr(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v)
-{
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
-        "%29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-}
-
-// Four 32-column loads in flight, one wait: 128 consecutive columns of this
-// thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v)
-{
-    uint32_t r[128];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-            "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-            "%28, %29, %30, %31}, [%32];"
-            : "=r"(r[32 * q + 0]), "=r"(r[32 * q + 1]), "=r"(r[32 * q + 2]), "=r"(r[32 * q + 3]),
-              "=r"(r[32 * q + 4]), "=r"(r[32 * q + 5]), "=r"(r[32 * q + 6]), "=r"(r[32 * q + 7]),
-              "=r"(r[32 * q + 8]), "=r"(r[32 * q + 9]), "=r"(r[32 * q + 10]), "=r"(r[32 * q + 11]),
-              "=r"(r[32 * q + 12]), "=r"(r[32 * q + 13]), "=r"(r[32 * q + 14]), "=r"(r[32 * q + 15]),
-              "=r"(r[32 * q + 16]), "=r"(r[32 * q + 17]), "=r"(r[32 * q + 18]), "=r"(r[32 * q + 19]),
-              "=r"(r[32 * q + 20]), "=r"(r[32 * q + 21]), "=r"(r[32 * q + 22]), "=r"(r[32 * q + 23]),
-              "=r"(r[32 * q + 24]), "=r"(r[32 * q + 25]), "=r"(r[32 * q + 26]), "=r"(r[32 * q + 27]),
-              "=r"(r[32 * q + 28]), "=r"(r[32 * q + 29]), "=r"(r[32 * q + 30]), "=r"(r[32 * q + 31])
-            : "r"(taddr + 32u * q));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int j = 0; j < 128; ++j) v[j] = __uint_as_float(r[j]);
-}
-
-// Two 32-column loads in flight, one wait: 64 consecutive columns of this
-// thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v)
-{
-    uint32_t r[64];
-#pragma unroll
-    for (int q = 0; q < 2; ++q)
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-            "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-            "%28, %29, %30, %31}, [%32];"
-            : "=r"(r[32 * q + 0]), "=r"(r[32 * q + 1]), "=r"(r[32 * q + 2]), "=r"(r[32 * q + 3]),
-              "=r"(r[32 * q + 4]), "=r"(r[32 * q + 5]), "=r"(r[32 * q + 6]), "=r"(r[32 * q + 7]),
-              "=r"(r[32 * q + 8]), "=r"(r[32 * q + 9]), "=r"(r[32 * q + 10]), "=r"(r[32 * q + 11]),
-              "=r"(r[32 * q + 12]), "=r"(r[32 * q + 13]), "=r"(r[32 * q + 14]), "=r"(r[32 * q + 15]),
-              "=r"(r[32 * q + 16]), "=r"(r[32 * q + 17]), "=r"(r[32 * q + 18]), "=r"(r[32 * q + 19]),
-              "=r"(r[32 * q + 20]), "=r"(r[32 * q + 21]), "=r"(r[32 * q + 22]), "=r"(r[32 * q + 23]),
-              "=r"(r[32 * q + 24]), "=r"(r[32 * q + 25]), "=r"(r[32 * q + 26]), "=r"(r[32 * q + 27]),
-              "=r"(r[32 * q + 28]), "=r"(r[32 * q + 29]), "=r"(r[32 * q + 30]), "=r"(r[32 * q + 31])
-            : "r"(taddr + 32u * q));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int j = 0; j < 64; ++j) v[j] = __uint_as_float(r[j]);
-}
+constexpr uint32_t TC_IDESC = tc_idesc_bf16(TC_M, TC_N);
 
 // One of 8 values by a 3-bit index (selects, no indexed registers).
 __device__ __forceinline__ float pick8(const float* v, int e)
@@ -396,7 +287,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(
                     const uint32_t d = tmem + (uint32_t)(buf * TC_N);
 #pragma unroll
                     for (int kk = 0; kk < DL / 16; ++kk)
-                        mma_bf16(d, adesc + 2ull * kk, bdesc + 2ull * kk, kk > 0 ? 1u : 0u);
+                        mma_bf16(d, adesc + 2ull * kk, bdesc + 2ull * kk, TC_IDESC, kk > 0 ? 1u : 0u);
                     mma_commit(&empty[s]);
                     mma_commit(&acc_full[buf]);
                 }
@@ -704,19 +595,6 @@ __global__ void __launch_bounds__(32 * TH_WARPS) score_theta_kernel(IndexView ix
 }
 
 // ---- host side ---------------------------------------------------------------
-static bool make_rows64_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows)
-{
-    TmapEncodeFn enc = tmap_encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)DL, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)DL * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)DL, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 bool tc_scoring_available() { return true; }
 
 // The widest group (2^gl buckets, gl = 2 .. 6) that still leaves a sequence of
@@ -775,8 +653,8 @@ cudaError_t launch_score_lists_tc(const IndexView& ix, int64_t n_blk, const void
         ws.n_grp != sp.n_grp)
         return cudaErrorInvalidValue;
     CUtensorMap tmQ, tmC;
-    if (!make_rows64_bf16(&tmQ, latent_Q, (uint64_t)ix.B * Nq, TC_M) ||
-        !make_rows64_bf16(&tmC, ix.cent_rt, (uint64_t)ix.B * ix.NBK, TC_N))
+    if (!tmap_rows64_bf16(&tmQ, latent_Q, (uint64_t)ix.B * Nq, TC_M) ||
+        !tmap_rows64_bf16(&tmC, ix.cent_rt, (uint64_t)ix.B * ix.NBK, TC_N))
         return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem_attr((const void*)score_tc_kernel<1>, TC_SMEM);
     if (e == cudaSuccess) e = ensure_smem_attr((const void*)score_tc_kernel<2>, TC_SMEM);

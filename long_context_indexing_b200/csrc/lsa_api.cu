@@ -603,6 +603,120 @@ lsa_status lsa_sparse_attn_backward(const void* Q, const void* K, const void* V,
     return LSA_OK;
 }
 
+// ---- brute-force per-key indexer ----------------------------------------------
+namespace {
+
+struct PkLayout {
+    size_t status, colmax, theta, cnt, over, gmax, cand, total;
+};
+
+PkLayout pk_layout(int64_t B, int64_t Nq, int64_t T_cap)
+{
+    const size_t rows = (size_t)B * Nq;
+    const int64_t ng = per_key_groups(T_cap);
+    PkLayout L;
+    size_t o = 0;
+    L.status = o; o += 256;
+    L.colmax = o; o += al256((size_t)B * DL * 4);
+    L.theta = o;  o += al256(rows * 4);
+    L.cnt = o;    o += al256(rows * 4);
+    L.over = o;   o += al256(rows * 4);
+    L.gmax = o;   o += al256(rows * ng * 2);
+    L.cand = o;   o += al256(rows * PK_CAP * 4);
+    L.total = o;
+    return L;
+}
+
+bool pk_sizes_ok(int64_t B, int64_t Nq, int64_t T_cap)
+{
+    return B >= 1 && Nq >= 0 && T_cap >= 1 && T_cap <= 2147483647LL &&
+           B * T_cap <= 2147483647LL && B * Nq <= 2147483647LL;
+}
+
+}  // namespace
+
+size_t lsa_select_per_key_workspace_bytes(int64_t B, int64_t Nq, int64_t T_cap)
+{
+    if (!pk_sizes_ok(B, Nq, T_cap)) return 0;
+    return pk_layout(B, Nq, T_cap).total;
+}
+
+lsa_status lsa_select_per_key(const void* latent_K, lsa_dtype dtype, int64_t B, int64_t T_cap,
+                              int64_t n_keys, const void* latent_Q, const int32_t* positions,
+                              int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
+                              int s_max, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!latent_K || !latent_Q || !positions || !indices || !counts || !workspace)
+        return fail(LSA_ERR_INVALID_ARG, "NULL argument");
+    if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
+    if (dtype != LSA_BF16)
+        return fail(LSA_ERR_UNSUPPORTED, "the per-key indexer scores bf16 latents only");
+    if (!pk_sizes_ok(B, Nq, T_cap) || n_keys < 0 || n_keys > T_cap)
+        return fail(LSA_ERR_INVALID_ARG, "bad sizes (B*T_cap and B*Nq below 2^31, n_keys <= T_cap)");
+    if (sp.budget < 0 || sp.window < 0 || sp.sinks < 0)
+        return fail(LSA_ERR_INVALID_ARG, "budget, window and sinks must be >= 0");
+    if (sp.budget > PK_MAX_R)
+        return fail(LSA_ERR_UNSUPPORTED, "budget %d > %d", sp.budget, PK_MAX_R);
+    if ((int64_t)sp.budget + sp.window + sp.sinks > (int64_t)s_max)
+        return fail(LSA_ERR_INVALID_ARG, "s_max=%d < budget + window + sinks", s_max);
+    if (ws_bytes < lsa_select_per_key_workspace_bytes(B, Nq, T_cap))
+        return fail(LSA_ERR_WORKSPACE, "workspace too small");
+    if (!aligned16(latent_K) || !aligned16(latent_Q) || !aligned16(positions) ||
+        !aligned16(indices) || !aligned16(counts) || !aligned16(workspace))
+        return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    const cudaStream_t st = (cudaStream_t)stream;
+    const PkLayout L = pk_layout(B, Nq, T_cap);
+    char* w = (char*)workspace;
+    cudaError_t e = cudaMemsetAsync(w, 0, L.theta, st);          // status words and colmax
+    if (e != cudaSuccess) return cuda_fail(e, "per-key indexer");
+    if (Nq == 0) return LSA_OK;
+    PerKeyArgs a;
+    a.lat_k = latent_K;
+    a.lat_q = latent_Q;
+    a.pos = positions;
+    a.B = B;
+    a.T_cap = T_cap;
+    a.n_keys = n_keys;
+    a.Nq = Nq;
+    a.R = sp.budget;
+    a.W = sp.window;
+    a.S = sp.sinks;
+    a.indices = indices;
+    a.counts = counts;
+    a.s_max = s_max;
+    PerKeyWs ws;
+    ws.status = (uint32_t*)(w + L.status);
+    ws.colmax = (uint32_t*)(w + L.colmax);
+    ws.theta = (float*)(w + L.theta);
+    ws.cnt = (int32_t*)(w + L.cnt);
+    ws.over = (int32_t*)(w + L.over);
+    ws.gmax = (uint16_t*)(w + L.gmax);
+    ws.cand = (int32_t*)(w + L.cand);
+    ws.ng = per_key_groups(T_cap);
+    e = launch_per_key(a, ws, st);
+    if (e != cudaSuccess) return cuda_fail(e, "per-key indexer");
+    return LSA_OK;
+}
+
+lsa_status lsa_select_per_key_check(const void* workspace, int64_t* fallbacks, void* stream)
+{
+    if (!workspace) return fail(LSA_ERR_INVALID_ARG, "NULL workspace");
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t h[8] = {0};
+    cudaError_t e = cudaMemcpyAsync(h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "per-key check");
+    if (fallbacks) *fallbacks = (int64_t)h[1];
+    switch (h[0]) {
+    case DEV_OK: return LSA_OK;
+    case DEV_BAD_INDEX:
+        return fail(LSA_ERR_INVALID_ARG, "a query position (%d) was outside [0, n_keys)", (int)h[2]);
+    case DEV_TIMEOUT:
+        return fail(LSA_ERR_TIMEOUT, "a bounded wait gave up (site %u)", h[2]);
+    default: return fail(LSA_ERR_INTERNAL, "device status %u (detail %u)", h[0], h[2]);
+    }
+}
+
 size_t lsa_attend_key_range_workspace_bytes(int64_t B, int64_t Nq, int s_max)
 {
     if (B < 1 || Nq < 0 || s_max < 1) return 0;
@@ -934,6 +1048,7 @@ lsa_status lsa_set_wait_limit(int64_t polls)
     cudaError_t e = set_score_wait_polls(polls);
     if (e == cudaSuccess) e = set_tile_wait_polls(polls);
     if (e == cudaSuccess) e = set_attn_wait_polls(polls);
+    if (e == cudaSuccess) e = set_per_key_wait_polls(polls);
     if (e != cudaSuccess) return cuda_fail(e, "wait limit");
     return LSA_OK;
 }

@@ -320,6 +320,35 @@ cudaError_t launch_merge_partials(const void* parts, const float* lse_parts, lsa
                                   int n_parts, int64_t rows, int Hq, int d, void* O, float* lse,
                                   cudaStream_t st);
 
+// Brute-force latent per-key indexer (k_perkey.cu): every long-range key of
+// a query scored on the tensor cores, the best R read.
+constexpr int PK_CAP = 8192;        // candidate list per query row
+constexpr int PK_MAX_R = 4096;      // largest long-range budget
+constexpr int PK_NG_MAX = 32768;    // strided key groups per row (at most)
+struct PerKeyArgs {
+    const void* lat_k;       // bf16 [B][T_cap][64]
+    const void* lat_q;       // bf16 [B][Nq][64]
+    const int32_t* pos;      // [B][Nq]
+    int64_t B, T_cap, n_keys, Nq;
+    int R, W, S;
+    int32_t* indices;        // [B][Nq][s_max]
+    int32_t* counts;         // [B][Nq]
+    int s_max;
+};
+struct PerKeyWs {
+    uint32_t* status;        // [8]: code, fallback rows, detail, overflow rows listed
+    uint32_t* colmax;        // [B][64] max |latent key| per dimension (fp32 bits)
+    float* theta;            // [rows] candidate threshold (-inf: every key, +inf: none)
+    int32_t* cnt;            // [rows] keys appended (may pass PK_CAP)
+    int32_t* over;           // [rows] rows sent to the exact fallback
+    uint16_t* gmax;          // [rows][ng] strided-group maxima (fp16 bits)
+    int32_t* cand;           // [rows][PK_CAP] candidate positions
+    int64_t ng;              // groups per row (power of two, 256 .. PK_NG_MAX)
+};
+int64_t per_key_groups(int64_t T_cap);
+cudaError_t set_per_key_wait_polls(int64_t polls);
+cudaError_t launch_per_key(const PerKeyArgs& a, const PerKeyWs& ws, cudaStream_t st);
+
 cudaError_t launch_attn(const void* Q, const void* K, const void* V, lsa_dtype dt, int64_t B,
                         int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
                         const int32_t* indices, const int32_t* counts, int s_max, float scale,

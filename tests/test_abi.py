@@ -207,3 +207,41 @@ def test_backward_entry_argument_checks():
     odd = list(ok)
     odd[5] = ctypes.c_void_p((1 << 22) + 8)
     assert f(*odd) == 2
+
+
+def test_per_key_entry_argument_checks():
+    # lsa_select_per_key refuses bad arguments before any launch: NULL
+    # pointers, fp32 latents, budgets above 4096, a short s_max or workspace,
+    # misaligned pointers.
+    need = lsa._lib.lsa_select_per_key_workspace_bytes(1, 32768, 10485760)
+    # [rows][32768] fp16 group maxima + [rows][8192] candidates + per-row words
+    assert 32768 * (2 * 32768 + 4 * 8192) < need < 32768 * (2 * 32768 + 4 * 8192 + 64) + (1 << 20)
+    assert lsa._lib.lsa_select_per_key_workspace_bytes(0, 16, 1024) == 0
+    assert lsa._lib.lsa_select_per_key_workspace_bytes(4, 16, 1 << 30) == 0   # B*T_cap >= 2^31
+    fake = ctypes.c_void_p(1 << 22)
+    f = lsa._lib.lsa_select_per_key
+    sp = lsa.SelectParams(256, 64, 4)
+    small = lsa._lib.lsa_select_per_key_workspace_bytes(1, 16, 8192)
+    ok = [fake, lsa.BF16, 1, 8192, 8192, fake, fake, 16, sp, fake, fake, 324, fake, small, None]
+    bad = list(ok)
+    bad[0] = None
+    assert f(*bad) == 1
+    f32 = list(ok)
+    f32[1] = lsa.F32
+    assert f(*f32) == 7                                 # LSA_ERR_UNSUPPORTED
+    big = list(ok)
+    big[8] = lsa.SelectParams(5000, 64, 4)
+    big[11] = 5068
+    assert f(*big) == 7
+    short = list(ok)
+    short[11] = 323                                      # s_max < budget + window + sinks
+    assert f(*short) == 1
+    keys = list(ok)
+    keys[4] = 8193                                       # n_keys > T_cap
+    assert f(*keys) == 1
+    ws = list(ok)
+    ws[13] = small - 1
+    assert f(*ws) == 3                                   # LSA_ERR_WORKSPACE
+    odd = list(ok)
+    odd[6] = ctypes.c_void_p((1 << 22) + 4)
+    assert f(*odd) == 2                                  # LSA_ERR_ALIGNMENT
