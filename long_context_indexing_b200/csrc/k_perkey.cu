@@ -48,9 +48,11 @@
 // warp 0 TMA producer (query tile, key tiles into a 4-deep ring, 128-byte
 // swizzle), warp 1 TMEM owner and MMA issuer (M = 128, N = 256, K = 16, four
 // per tile, two accumulators), warps 2-17 epilogue (thread = query row and 64
-// columns of every tile).  Every mbarrier wait is bounded; a timeout records
-// DEV_TIMEOUT in the status word and the CTA drains and exits as the bucket
-// scorer does.
+// columns of every tile, read from TMEM in 32-column pieces).  Pass 2
+// stages a row's appended keys in shared memory and reserves their place in
+// the row's list with one global atomic per row and item.  Every mbarrier
+// wait is bounded; a timeout records DEV_TIMEOUT in the status word and the
+// CTA drains and exits as the bucket scorer does.
 #include <cuda.h>
 
 #include <cuda_fp16.h>
@@ -65,10 +67,12 @@ namespace lsa {
 
 constexpr int PK_M = 128;
 constexpr int PK_N = 256;                                 // keys per tile
-constexpr int PK_TMEM_COLS = 2 * PK_N;
+constexpr int PK_ACC = 2;                                 // TMEM accumulators
+constexpr int PK_TMEM_COLS = PK_ACC * PK_N;
 constexpr int PK_STAGES = 4;
 constexpr int PK_EPI_WARPS = 16;
 constexpr int PK_COLS = PK_N / 4;                         // columns per epilogue thread
+constexpr int PK_ST = 128;                                // staged appends per row and item
 constexpr int PK_EPI_THREADS = 32 * PK_EPI_WARPS;
 constexpr int PK_THREADS = 64 + PK_EPI_THREADS;
 constexpr uint32_t PK_WAIT = 1u << 22;
@@ -79,10 +83,11 @@ __device__ uint32_t g_pk_wait = PK_WAIT;
 constexpr int PK_Q_BYTES = PK_M * DL * 2;
 constexpr int PK_K_BYTES = PK_N * DL * 2;
 constexpr int PK_OFF_K = 2 * PK_Q_BYTES;
-constexpr int PK_OFF_BAR = PK_OFF_K + PK_STAGES * PK_K_BYTES;
-constexpr int PK_NBAR = 2 + 2 + 2 * PK_STAGES + 2 + 2 + 1;
+constexpr int PK_OFF_ST = PK_OFF_K + PK_STAGES * PK_K_BYTES;     // [PK_M][PK_ST] staged keys
+constexpr int PK_OFF_BAR = PK_OFF_ST + PK_M * PK_ST * 4;
+constexpr int PK_NBAR = 2 + 2 + 2 * PK_STAGES + 2 * PK_ACC + 1;
 constexpr int PK_OFF_MISC = PK_OFF_BAR + PK_NBAR * 8;
-constexpr int PK_SMEM = PK_OFF_MISC + 64 + 1024;          // + alignment slack
+constexpr int PK_SMEM = PK_OFF_MISC + 64 + PK_M * 4 + 1024;      // + staged counts, alignment
 
 // Position of query i of sequence b, or -1 when it lies outside [0, n_keys)
 // (such a row reads nothing and the final kernel reports DEV_BAD_INDEX).
@@ -132,6 +137,37 @@ __device__ __forceinline__ double pk_exact(const double* qd, const __nv_bfloat16
         }
     }
     return s;
+}
+
+// Two keys at once (both rows' loads in flight, the two sums interleaved);
+// each sum is pk_exact's, in the same order.
+__device__ __forceinline__ void pk_exact2(const double* qd, const __nv_bfloat16* ka,
+                                          const __nv_bfloat16* kb, double* sa, double* sb)
+{
+    const uint4* a4 = reinterpret_cast<const uint4*>(ka);
+    const uint4* b4 = reinterpret_cast<const uint4*>(kb);
+    uint4 wa[DL / 8], wb[DL / 8];
+#pragma unroll
+    for (int c = 0; c < DL / 8; ++c) {
+        wa[c] = a4[c];
+        wb[c] = b4[c];
+    }
+    double x = 0.0, y = 0.0;
+#pragma unroll
+    for (int c = 0; c < DL / 8; ++c) {
+        const uint32_t ea[4] = {wa[c].x, wa[c].y, wa[c].z, wa[c].w};
+        const uint32_t eb[4] = {wb[c].x, wb[c].y, wb[c].z, wb[c].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const double q0 = qd[8 * c + 2 * j], q1 = qd[8 * c + 2 * j + 1];
+            x = __dadd_rn(x, __dmul_rn(q0, (double)__uint_as_float(ea[j] << 16)));
+            y = __dadd_rn(y, __dmul_rn(q0, (double)__uint_as_float(eb[j] << 16)));
+            x = __dadd_rn(x, __dmul_rn(q1, (double)__uint_as_float(ea[j] & 0xFFFF0000u)));
+            y = __dadd_rn(y, __dmul_rn(q1, (double)__uint_as_float(eb[j] & 0xFFFF0000u)));
+        }
+    }
+    *sa = x;
+    *sb = y;
 }
 
 // ---------------------------------------------------------------------------
@@ -211,6 +247,12 @@ __device__ __forceinline__ PkItem pk_item(int64_t it, const PerKeyArgs& a, int64
     return r;
 }
 
+// Named barrier of the epilogue warps only.
+__device__ __forceinline__ void pk_epi_sync()
+{
+    asm volatile("bar.sync 1, %0;" ::"n"(PK_EPI_THREADS) : "memory");
+}
+
 template <int PASS>
 __global__ void __launch_bounds__(PK_THREADS, 1) perkey_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, PerKeyArgs a,
@@ -226,12 +268,14 @@ __global__ void __launch_bounds__(PK_THREADS, 1) perkey_tc_kernel(
     uint64_t* q_empty = bars + 2;
     uint64_t* full = bars + 4;
     uint64_t* empty = full + PK_STAGES;
-    uint64_t* acc_full = empty + PK_STAGES;
-    uint64_t* acc_empty = acc_full + 2;
-    uint64_t* fin = acc_empty + 2;
+    uint64_t* acc_full = empty + PK_STAGES;     // [PK_ACC]
+    uint64_t* acc_empty = acc_full + PK_ACC;    // [PK_ACC]
+    uint64_t* fin = acc_empty + PK_ACC;
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + PK_OFF_MISC);
     volatile uint32_t* tmem_slot = misc;
     volatile uint32_t* abort_flag = misc + 1;
+    int32_t* st_buf = reinterpret_cast<int32_t*>(smem + PK_OFF_ST);        // [PK_M][PK_ST]
+    int* st_cnt = reinterpret_cast<int*>(smem + PK_OFF_MISC + 64);          // [PK_M]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t ng = ws.ng;
@@ -239,6 +283,8 @@ __global__ void __launch_bounds__(PK_THREADS, 1) perkey_tc_kernel(
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&q_full[i], 1);
             ptx::mbar_init(&q_empty[i], 1);
+        }
+        for (int i = 0; i < PK_ACC; ++i) {
             ptx::mbar_init(&acc_full[i], 1);
             ptx::mbar_init(&acc_empty[i], PK_EPI_WARPS);
         }
@@ -250,6 +296,7 @@ __global__ void __launch_bounds__(PK_THREADS, 1) perkey_tc_kernel(
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
+    if (threadIdx.x < PK_M) st_cnt[threadIdx.x] = 0;
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          ptx::smem_addr((const void*)tmem_slot)), "n"(PK_TMEM_COLS)
@@ -319,9 +366,9 @@ __global__ void __launch_bounds__(PK_THREADS, 1) perkey_tc_kernel(
             ++qi;
             for (int i = 0; i < I.n_t; ++i, ++gt) {
                 const int s = (int)(gt % PK_STAGES);
-                const int buf = (int)(gt & 1);
+                const int buf = (int)(gt % PK_ACC);
                 if (!waitw(&full[s], (uint32_t)((gt / PK_STAGES) & 1), 6100u) ||
-                    !waitw(&acc_empty[buf], (uint32_t)(((gt >> 1) & 1) ^ 1), 6200u)) {
+                    !waitw(&acc_empty[buf], (uint32_t)(((gt / PK_ACC) & 1) ^ 1), 6200u)) {
                     stop = true;
                     break;
                 }
@@ -351,7 +398,7 @@ __global__ void __launch_bounds__(PK_THREADS, 1) perkey_tc_kernel(
         const int r = 32 * (warp & 3) + lane;             // query row = TMEM lane
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
         const unsigned FULL = 0xffffffffu;
-        int64_t gt = 0;
+        uint32_t gt = 0;                                  // tiles so far (parities only)
         for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
             const PkItem I = pk_item(it, a, ng, n_qt);
             const bool row_valid = I.q0 + r < a.Nq;
@@ -370,20 +417,23 @@ __global__ void __launch_bounds__(PK_THREADS, 1) perkey_tc_kernel(
             }
             const bool go = __all_sync(FULL, *abort_flag == 0);
             for (int i = 0; i < I.n_t; ++i, ++gt) {
-                const int buf = (int)(gt & 1);
-                const bool ok = go && waitw(&acc_full[buf], (uint32_t)((gt >> 1) & 1), 7000u);
+                const int buf = (int)(gt % PK_ACC);
+                const bool ok =
+                    go && waitw(&acc_full[buf], (uint32_t)((gt / PK_ACC) & 1), 7000u);
                 if (!ok) continue;
                 tc_fence_after();
                 const int c0 = (int)(I.gb * PK_N + (int64_t)i * ng) + sl * PK_COLS;   // first key here
                 const uint32_t taddr = tmem + lane_base + (uint32_t)(buf * PK_N + sl * PK_COLS);
                 if (PASS == 1) {
-                    // running maxima of the eligible scores, column by column
+                    // running maxima of the eligible scores, column by column,
+                    // 32 columns at a time
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
+                    for (int h = 0; h < PK_COLS / 32; ++h) {
                         float v[32];
                         __syncwarp();
                         tmem_ld32(taddr + 32u * h, v);
-                        if (h == 1) {
+                        if (h == PK_COLS / 32 - 1) {
+                            // the accumulator is in registers: hand it back
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
@@ -402,6 +452,7 @@ __global__ void __launch_bounds__(PK_THREADS, 1) perkey_tc_kernel(
                     float v[PK_COLS];
                     __syncwarp();
                     tmem_ld64(taddr, v);
+                    // the accumulator is in registers: hand it back before the work
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
@@ -412,12 +463,12 @@ __global__ void __launch_bounds__(PK_THREADS, 1) perkey_tc_kernel(
                         const int e0 = c0 < lo ? lo : c0;
                         const int e1 = (c0 + PK_COLS - 1 < hi) ? c0 + PK_COLS - 1 : hi;
                         if (e1 >= e0) {
-                            const int n = (int)(e1 - e0 + 1), s0 = (int)(e0 - c0);
+                            const int n = e1 - e0 + 1, s0 = e0 - c0;
                             em = (n == 64 ? ~0ull : ((1ull << n) - 1ull)) << s0;
                         }
                     }
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
+                    for (int q = 0; q < PK_COLS / 8; ++q) {
                         const float* w = v + 8 * q;
                         const float mx = fmaxf(fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3])),
                                                fmaxf(fmaxf(w[4], w[5]), fmaxf(w[6], w[7])));
@@ -431,12 +482,23 @@ __global__ void __launch_bounds__(PK_THREADS, 1) perkey_tc_kernel(
                                 bits &= eb;
                             }
                             if (bits) {
-                                int slot = atomicAdd(&ws.cnt[row], __popc(bits));
+                                const int nb = __popc(bits);
+                                int slot = atomicAdd(&st_cnt[r], nb);
+                                // what finds the staging full goes straight to
+                                // the row's list (one reservation per batch)
+                                int g = 0;
+                                if (slot + nb > PK_ST)
+                                    g = atomicAdd(&ws.cnt[row], slot + nb - max(slot, PK_ST));
                                 while (bits) {
                                     const int e = __ffs(bits) - 1;
                                     bits &= bits - 1u;
-                                    if (slot < PK_CAP)
-                                        ws.cand[row * PK_CAP + slot] = (int32_t)(c0 + 8 * q + e);
+                                    const int32_t t = c0 + 8 * q + e;
+                                    if (slot < PK_ST) {
+                                        st_buf[r * PK_ST + slot] = t;
+                                    } else {
+                                        if (g < PK_CAP) ws.cand[row * PK_CAP + g] = t;
+                                        ++g;
+                                    }
                                     ++slot;
                                 }
                             }
@@ -444,6 +506,20 @@ __global__ void __launch_bounds__(PK_THREADS, 1) perkey_tc_kernel(
                     }
                 }
                 __syncwarp();
+            }
+            if (PASS == 2 && I.n_t > 0) {                 // block-uniform
+                // the staged keys of each row go to its list: one reservation
+                pk_epi_sync();
+                if (sl == 0) {
+                    const int n = min(st_cnt[r], PK_ST);
+                    if (n > 0 && row_valid) {
+                        const int base = atomicAdd(&ws.cnt[row], n);
+                        for (int j = 0; j < n && base + j < PK_CAP; ++j)
+                            ws.cand[row * PK_CAP + base + j] = st_buf[r * PK_ST + j];
+                    }
+                    st_cnt[r] = 0;
+                }
+                pk_epi_sync();
             }
             if (PASS == 1 && row_valid) {
                 // the row's 64 group maxima of this block (fp16 bits)
@@ -690,7 +766,7 @@ __global__ void __launch_bounds__(PF_THREADS) perkey_final_kernel(PerKeyArgs a, 
     for (int k = 2; k <= P; k <<= 1) {
         for (int j = k >> 1; j > 0; j >>= 1) {
             for (int x = threadIdx.x; x < P / 2; x += PF_THREADS) {
-                const int lo = 2 * j * (x / j) + (x % j);
+                const int lo = ((x & ~(j - 1)) << 1) | (x & (j - 1));   // j is a power of two
                 const int hi = lo + j;
                 const bool up = (lo & k) == 0;
                 const int32_t u = pos_s[lo], v = pos_s[hi];
@@ -704,8 +780,13 @@ __global__ void __launch_bounds__(PF_THREADS) perkey_final_kernel(PerKeyArgs a, 
     }
     // exact scores as ordered keys
     const __nv_bfloat16* lat = reinterpret_cast<const __nv_bfloat16*>(a.lat_k) + b * a.T_cap * DL;
-    for (int x = threadIdx.x; x < n; x += PF_THREADS)
-        key_s[x] = pk_dkey(pk_exact(q_s, lat + (int64_t)pos_s[x] * DL));
+    for (int x = threadIdx.x; x < n; x += 2 * PF_THREADS) {
+        const int y = x + PF_THREADS;
+        double sx, sy;
+        pk_exact2(q_s, lat + (int64_t)pos_s[x] * DL, lat + (int64_t)pos_s[y < n ? y : x] * DL, &sx, &sy);
+        key_s[x] = pk_dkey(sx);
+        if (y < n) key_s[y] = pk_dkey(sy);
+    }
     __syncthreads();
     // the R-th largest key, and how many equal keys are taken (lowest positions)
     uint64_t cut = 0ull;
