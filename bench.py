@@ -918,6 +918,8 @@ def main():
                     help="several GPUs: every rank runs its own chunk (weak scaling), one "
                          "chunk's queries are split over the ranks, or the KV cache is held in "
                          "shards over the ranks (both strong scaling)")
+    ap.add_argument("--per-key-only", action="store_true",
+                    help="run only the per-key indexer measurement on the workload's chunk")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the decode measurement (prints its object)")
     args = ap.parse_args()
@@ -928,6 +930,12 @@ def main():
         if args.decode_only:
             peaks, src = _peaks()
             out = run_decode(args, peaks, src, ws)
+            if rank == 0:
+                print(json.dumps(out), flush=True)
+        elif args.per_key_only:
+            w = _bench_workload(args)
+            inp = synth.prefill_inputs(w, args.seed, "cuda")
+            out = _per_key_measure(w, inp, {}, torch.cuda.current_stream())
             if rank == 0:
                 print(json.dumps(out), flush=True)
         elif args.impl == "reference":

@@ -11,6 +11,8 @@
 #include <atomic>
 #include <new>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "hooks.cuh"
 #include "lsa_internal.cuh"
 
@@ -37,6 +39,57 @@ lsa_status cuda_fail(cudaError_t e, const char* where)
 }
 
 inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// NVTX range around a public entry (visible to nsys / ncu range filters; a
+// no-op when no tool is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+
+// ---- LSA_DEBUG=1 checks (k_debug.cu) ----
+const char* dbg_kind_name(uint32_t k)
+{
+    switch (k) {
+    case DBG_OFFSETS: return "CSR offsets of a block out of range or decreasing";
+    case DBG_MEMBER: return "a bucket member outside its block";
+    case DBG_ORDER: return "bucket members not ascending";
+    case DBG_ASSIGN: return "a member whose assignment names another bucket";
+    case DBG_OPEN: return "an open-block entry that is no closed bucket";
+    case DBG_COUNT: return "a selection count out of range";
+    case DBG_INDEX: return "a gather index outside [0, T_cap)";
+    case DBG_CAUSAL: return "a selected index after its query's position";
+    case DBG_LAYOUT: return "a selection row not laid out as sinks, long-range keys, window";
+    default: return "unknown";
+    }
+}
+
+lsa_status dbg_result(cudaError_t e, const uint32_t h[4], const char* what)
+{
+    if (e != cudaSuccess) return cuda_fail(e, "debug check");
+    if (h[0] == 0u) return LSA_OK;
+    return fail(LSA_ERR_INTERNAL, "debug check (%s): %s (sequence/row %u, at %u, value %d)", what,
+                dbg_kind_name(h[0]), h[1], h[2], (int)h[3]);
+}
+
+lsa_status dbg_index(const IndexView& v, int64_t n_blk, cudaStream_t st, const char* what)
+{
+    if (!debug_enabled()) return LSA_OK;
+    uint32_t h[4];
+    const cudaError_t e = debug_check_index(v, n_blk, st, h);
+    return dbg_result(e, h, what);
+}
+
+lsa_status dbg_gather(const int32_t* indices, const int32_t* counts, int64_t B, int64_t Nq,
+                      int s_max, int64_t T_cap, PosSrc pos, lsa_select_params sp, int mode,
+                      cudaStream_t st, const char* what)
+{
+    if (!debug_enabled()) return LSA_OK;
+    uint32_t h[4];
+    const cudaError_t e = debug_check_gather(indices, counts, B * Nq, s_max, T_cap, pos, Nq,
+                                             sp.window, sp.sinks, mode, st, h);
+    return dbg_result(e, h, what);
+}
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -110,12 +163,15 @@ lsa_status run_select(const lsa_index* idx, const void* lq, PosSrc pos, int64_t 
     if (!tc && idx->n_blk * idx->v.k > SIMT_MAX_BUCKETS)
         return fail(LSA_ERR_UNSUPPORTED, "%lld buckets exceed the SIMT scorer's %lld",
                     (long long)(idx->n_blk * idx->v.k), (long long)SIMT_MAX_BUCKETS);
+    lsa_status s = dbg_index(idx->v, idx->n_blk, st, "index before selection");
+    if (s != LSA_OK) return s;
     SelectWs w = select_ws_carve(ws, idx->v, Nq);
     if (plan) w.plan = *plan;
     cudaError_t e = launch_select(idx->v, idx->n_blk, lq, pos, Nq, sp, indices, counts, s_max, w,
                                   tc, st);
     if (e != cudaSuccess) return cuda_fail(e, "select");
-    return LSA_OK;
+    return dbg_gather(indices, counts, idx->v.B, Nq, s_max, idx->v.T_cap, pos, sp, DBG_SELECTION,
+                      st, "selection");
 }
 
 // Prefill workspace: selection output and scratch, then (bf16 with a
@@ -354,6 +410,7 @@ int64_t lsa_index_num_blocks(const lsa_index* idx) { return idx ? idx->n_blk : -
 lsa_status lsa_index_extend(lsa_index* idx, const void* latent_K, int64_t T_old, int64_t T_new,
                             void* stream)
 {
+    NvtxRange nv("lsa_index_extend");
     if (!idx || !latent_K) return fail(LSA_ERR_INVALID_ARG, "NULL index or latent_K");
     if (!aligned16(latent_K)) return fail(LSA_ERR_ALIGNMENT, "latent_K not 16-byte aligned");
     const IndexView& v = idx->v;
@@ -385,7 +442,7 @@ lsa_status lsa_index_extend(lsa_index* idx, const void* latent_K, int64_t T_old,
         e = launch_open_assign(v, idx->n_blk, j_end, st);
         if (e != cudaSuccess) return cuda_fail(e, "open assign");
     }
-    return LSA_OK;
+    return dbg_index(v, idx->n_blk, st, "index after extension");
 }
 
 lsa_status lsa_build_index(lsa_index* idx, const void* latent_K, int64_t T, void* stream)
@@ -455,6 +512,7 @@ lsa_status lsa_select(const lsa_index* idx, const void* latent_Q, const int32_t*
                       int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
                       int s_max, void* workspace, size_t ws_bytes, void* stream)
 {
+    NvtxRange nv("lsa_select");
     if (!idx || !latent_Q || !positions || !indices || !counts || !workspace)
         return fail(LSA_ERR_INVALID_ARG, "NULL argument");
     if (Nq < 0 || Nq > 2147483647LL) return fail(LSA_ERR_INVALID_ARG, "Nq out of range");
@@ -497,6 +555,7 @@ size_t lsa_tree_bytes(const lsa_index* idx, int n_super)
 lsa_status lsa_tree_build(const lsa_index* idx, void* tree, size_t bytes, int n_super,
                           int lloyd_iters, void* stream)
 {
+    NvtxRange nv("lsa_tree_build");
     lsa_status s = check_tree(idx, n_super);
     if (s != LSA_OK) return s;
     if (!tree) return fail(LSA_ERR_INVALID_ARG, "NULL tree buffer");
@@ -532,6 +591,7 @@ lsa_status lsa_tree_select(const lsa_index* idx, const void* tree, int n_super, 
                            lsa_select_params sp, int32_t* indices, int32_t* counts, int s_max,
                            void* workspace, size_t ws_bytes, void* stream)
 {
+    NvtxRange nv("lsa_tree_select");
     lsa_status s = check_tree(idx, n_super);
     if (s != LSA_OK) return s;
     if (!tree || !latent_Q || !positions || !indices || !counts || !workspace)
@@ -548,11 +608,14 @@ lsa_status lsa_tree_select(const lsa_index* idx, const void* tree, int n_super, 
     const size_t need = tree_select_ws_bytes(idx->v, Nq, branches);
     if (ws_bytes < need) return fail(LSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
     if (Nq == 0) return LSA_OK;
+    const cudaStream_t st = (cudaStream_t)stream;
+    s = dbg_index(idx->v, idx->n_blk, st, "index before tree selection");
+    if (s != LSA_OK) return s;
     cudaError_t e = launch_tree_select(idx->v, idx->n_blk, tree, n_super, branches, latent_Q,
-                                       positions, Nq, sp, indices, counts, s_max, workspace,
-                                       (cudaStream_t)stream);
+                                       positions, Nq, sp, indices, counts, s_max, workspace, st);
     if (e != cudaSuccess) return cuda_fail(e, "tree select");
-    return LSA_OK;
+    return dbg_gather(indices, counts, idx->v.B, Nq, s_max, idx->v.T_cap, PosSrc{positions, 0},
+                      sp, DBG_SELECTION, st, "tree selection");
 }
 
 lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtype dtype, int64_t B,
@@ -560,6 +623,7 @@ lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtyp
                            const int32_t* indices, const int32_t* counts, int s_max, float scale,
                            void* O, float* lse, void* stream)
 {
+    NvtxRange nv("lsa_sparse_attn");
     if (!Q || !K || !V || !indices || !counts || !O)
         return fail(LSA_ERR_INVALID_ARG, "NULL argument");
     if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
@@ -572,6 +636,10 @@ lsa_status lsa_sparse_attn(const void* Q, const void* K, const void* V, lsa_dtyp
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(indices) ||
         !aligned16(counts) || !aligned16(O) || (lse && !aligned16(lse)))
         return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    lsa_select_params none{0, 0, 0};
+    lsa_status s = dbg_gather(indices, counts, B, Nq, s_max, T_cap, PosSrc{nullptr, 0}, none,
+                              DBG_BOUNDS, (cudaStream_t)stream, "gather indices");
+    if (s != LSA_OK) return s;
     cudaError_t e = launch_attn(Q, K, V, dtype, B, Nq, T_cap, Hq, Hkv, d, indices, counts, s_max,
                                 scale, O, lse, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "sparse attention");
@@ -584,6 +652,7 @@ lsa_status lsa_sparse_attn_backward(const void* Q, const void* K, const void* V,
                                     const int32_t* indices, const int32_t* counts, int s_max,
                                     float scale, void* dQ, float* dK, float* dV, void* stream)
 {
+    NvtxRange nv("lsa_sparse_attn_backward");
     if (!Q || !K || !V || !O || !lse || !dO || !indices || !counts || !dQ || !dK || !dV)
         return fail(LSA_ERR_INVALID_ARG, "NULL argument");
     if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
@@ -596,6 +665,10 @@ lsa_status lsa_sparse_attn_backward(const void* Q, const void* K, const void* V,
     const void* ptrs[] = {Q, K, V, O, lse, dO, indices, counts, dQ, dK, dV};
     for (const void* p : ptrs)
         if (!aligned16(p)) return fail(LSA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    lsa_select_params none{0, 0, 0};
+    lsa_status s = dbg_gather(indices, counts, B, Nq, s_max, T_cap, PosSrc{nullptr, 0}, none,
+                              DBG_BOUNDS, (cudaStream_t)stream, "gather indices");
+    if (s != LSA_OK) return s;
     cudaError_t e = launch_attn_backward(Q, K, V, O, lse, dO, dtype, B, Nq, T_cap, Hq, Hkv, d,
                                          indices, counts, s_max, scale, dQ, dK, dV, nullptr,
                                          (cudaStream_t)stream);
@@ -646,6 +719,7 @@ lsa_status lsa_select_per_key(const void* latent_K, lsa_dtype dtype, int64_t B, 
                               int64_t Nq, lsa_select_params sp, int32_t* indices, int32_t* counts,
                               int s_max, void* workspace, size_t ws_bytes, void* stream)
 {
+    NvtxRange nv("lsa_select_per_key");
     if (!latent_K || !latent_Q || !positions || !indices || !counts || !workspace)
         return fail(LSA_ERR_INVALID_ARG, "NULL argument");
     if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
@@ -695,7 +769,8 @@ lsa_status lsa_select_per_key(const void* latent_K, lsa_dtype dtype, int64_t B, 
     ws.ng = per_key_groups(T_cap);
     e = launch_per_key(a, ws, st);
     if (e != cudaSuccess) return cuda_fail(e, "per-key indexer");
-    return LSA_OK;
+    return dbg_gather(indices, counts, B, Nq, s_max, T_cap, PosSrc{positions, 0}, sp,
+                      DBG_SELECTION_SORTED, st, "per-key selection");
 }
 
 lsa_status lsa_select_per_key_check(const void* workspace, int64_t* fallbacks, void* stream)
@@ -729,6 +804,7 @@ lsa_status lsa_attend_key_range(const void* Q, const void* K_shard, const void* 
                                 int64_t key_lo, int64_t key_hi, float scale, void* workspace,
                                 size_t ws_bytes, void* O_part, float* lse_part, void* stream)
 {
+    NvtxRange nv("lsa_attend_key_range");
     if (!Q || !K_shard || !V_shard || !indices || !counts || !O_part || !lse_part || !workspace)
         return fail(LSA_ERR_INVALID_ARG, "NULL argument");
     if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
@@ -762,6 +838,7 @@ lsa_status lsa_merge_partials(const void* O_parts, const float* lse_parts, lsa_d
                               int n_parts, int64_t rows, int Hq, int d, void* O, float* lse,
                               void* stream)
 {
+    NvtxRange nv("lsa_merge_partials");
     if (!O_parts || !lse_parts || !O) return fail(LSA_ERR_INVALID_ARG, "NULL argument");
     if (dtype != LSA_F32 && dtype != LSA_BF16) return fail(LSA_ERR_INVALID_ARG, "unknown dtype");
     if (n_parts < 1 || n_parts > 32 || rows < 0 || Hq < 1 || d < 1 || d > 1024)
@@ -897,6 +974,9 @@ lsa_status attend_part(const lsa_index* idx, const void* Q, const void* K, const
     const int32_t* indices = (const int32_t*)(base + L.indices);
     const int32_t* counts = (const int32_t*)(base + L.counts);
     const float scale = (float)(1.0 / sqrt((double)d));
+    s = dbg_gather(indices, counts, idx->v.B, Nq, s_max, idx->v.T_cap, PosSrc{nullptr, T_old + q0},
+                   sp, DBG_SELECTION, st, "chunk selection before attention");
+    if (s != LSA_OK) return s;
     cudaError_t e;
     if (L.bucket)
         e = launch_bucket_attn(idx->v, idx->n_blk, P, Q, K, V, Nq, Hq, Hkv, d,
@@ -938,6 +1018,7 @@ lsa_status lsa_prefill_select(lsa_index* idx, const void* latent_K, const void* 
                               int64_t T_old, int64_t T_new, int Hq, int Hkv, int d,
                               lsa_select_params sp, void* workspace, size_t ws_bytes, void* stream)
 {
+    NvtxRange nv("lsa_prefill_select");
     return select_part(idx, latent_K, latent_Q, T_old, T_new, 0, T_new - T_old, Hq, Hkv, d, sp,
                        workspace, ws_bytes, stream);
 }
@@ -947,6 +1028,7 @@ lsa_status lsa_prefill_attend(const lsa_index* idx, const void* Q, const void* K
                               lsa_select_params sp, void* workspace, size_t ws_bytes, void* O,
                               void* stream)
 {
+    NvtxRange nv("lsa_prefill_attend");
     return attend_part(idx, Q, K, V, T_old, T_new, 0, T_new - T_old, Hq, Hkv, d, sp, workspace,
                        ws_bytes, O, stream);
 }
@@ -956,6 +1038,7 @@ lsa_status lsa_prefill_chunk(lsa_index* idx, const void* latent_K, const void* l
                              int64_t T_new, int Hq, int Hkv, int d, lsa_select_params sp,
                              void* workspace, size_t ws_bytes, void* O, void* stream)
 {
+    NvtxRange nv("lsa_prefill_chunk");
     return chunk_part(idx, latent_K, latent_Q, Q, K, V, T_old, T_new, 0, T_new - T_old, Hq, Hkv,
                       d, sp, workspace, ws_bytes, O, stream);
 }
@@ -966,6 +1049,7 @@ lsa_status lsa_prefill_chunk_queries(lsa_index* idx, const void* latent_K, const
                                      int Hkv, int d, lsa_select_params sp, void* workspace,
                                      size_t ws_bytes, void* O, void* stream)
 {
+    NvtxRange nv("lsa_prefill_chunk_queries");
     return chunk_part(idx, latent_K, latent_Q, Q, K, V, T_old, T_new, q_begin, q_end, Hq, Hkv, d,
                       sp, workspace, ws_bytes, O, stream);
 }
@@ -977,6 +1061,7 @@ lsa_status lsa_prefill_chunk_host(lsa_index* idx, const void* h_latent_K, const 
                                   lsa_select_params sp, void* workspace, size_t ws_bytes,
                                   void* O, void* h_O, void* stream, void* copy_stream)
 {
+    NvtxRange nv("lsa_prefill_chunk_host");
     if (!idx || !h_latent_K || !h_K || !h_V || !h_latent_Q || !h_Q || !latent_K || !K || !V ||
         !latent_Q || !Q || !O || !h_O)
         return fail(LSA_ERR_INVALID_ARG, "NULL argument");
@@ -1067,6 +1152,7 @@ lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
                            int Hkv, int d, lsa_select_params sp, void* workspace, size_t ws_bytes,
                            void* O, void* stream)
 {
+    NvtxRange nv("lsa_decode_step");
     if (!idx || !latent_K || !K || !V || !new_latent_k || !new_k || !new_v || !latent_q || !q ||
         !pos || !workspace || !O)
         return fail(LSA_ERR_INVALID_ARG, "NULL argument");
@@ -1111,6 +1197,8 @@ lsa_status lsa_decode_step(lsa_index* idx, void* latent_K, void* K, void* V,
         if (e != cudaSuccess) return cuda_fail(e, "status clear");
         idx->status_clean = true;
     }
+    s = dbg_index(v, idx->n_blk, st, "index before decode step");
+    if (s != LSA_OK) return s;
     cudaError_t e = launch_decode_prep(v, idx->n_blk, latent_K, K, V, new_latent_k, new_k, new_v,
                                        latent_q, pos, Hkv, d, sp.window, w, app_score, app_g,
                                        app_slot, L.n_slice, counter, L.n_hg, st);
@@ -1136,6 +1224,7 @@ lsa_status lsa_select_noalloc(const lsa_index* idx, const void* latent_Q,
                               const int32_t* positions, int64_t Nq, lsa_select_params sp,
                               int32_t* indices, int32_t* counts, int s_max, void* stream)
 {
+    NvtxRange nv("lsa_select_noalloc");
     if (!idx || !latent_Q || !positions || !indices || !counts)
         return fail(LSA_ERR_INVALID_ARG, "NULL argument");
     if (Nq < 0 || Nq > 2147483647LL) return fail(LSA_ERR_INVALID_ARG, "Nq out of range");
@@ -1154,10 +1243,14 @@ lsa_status lsa_select_noalloc(const lsa_index* idx, const void* latent_Q,
         return fail(LSA_ERR_UNSUPPORTED, "%lld buckets exceed the SIMT scorer's %lld",
                     (long long)(idx->n_blk * idx->v.k), (long long)SIMT_MAX_BUCKETS);
     if (Nq == 0) return LSA_OK;
+    const cudaStream_t st = (cudaStream_t)stream;
+    s = dbg_index(idx->v, idx->n_blk, st, "index before selection");
+    if (s != LSA_OK) return s;
     cudaError_t e = noalloc_select(idx->v, idx->n_blk, latent_Q, positions, Nq, sp, indices,
-                                   counts, s_max, tc, (cudaStream_t)stream);
+                                   counts, s_max, tc, st);
     if (e != cudaSuccess) return cuda_fail(e, "select (built-in scratch)");
-    return LSA_OK;
+    return dbg_gather(indices, counts, idx->v.B, Nq, s_max, idx->v.T_cap, PosSrc{positions, 0},
+                      sp, DBG_SELECTION, st, "selection");
 }
 
 }  // extern "C"

@@ -349,6 +349,29 @@ int64_t per_key_groups(int64_t T_cap);
 cudaError_t set_per_key_wait_polls(int64_t polls);
 cudaError_t launch_per_key(const PerKeyArgs& a, const PerKeyWs& ws, cudaStream_t st);
 
+// Checks run when LSA_DEBUG=1 (k_debug.cu).  Each synchronises the stream
+// (it does nothing while the stream is being captured) and returns in out[4]
+// the first violation found: kind (0 = none), sequence or row, place, value.
+enum DbgKind : uint32_t {
+    DBG_OFFSETS = 1,    // a block's CSR offsets out of its range or decreasing
+    DBG_MEMBER = 2,     // a member outside its block
+    DBG_ORDER = 3,      // members not ascending inside a bucket
+    DBG_ASSIGN = 4,     // a member's assignment names another bucket
+    DBG_OPEN = 5,       // an open-block entry that is no closed bucket
+    DBG_COUNT = 6,      // a selection count outside [0, s_max]
+    DBG_INDEX = 7,      // a selected index outside [0, T_cap)
+    DBG_CAUSAL = 8,     // a selected index after the query's position
+    DBG_LAYOUT = 9,     // a selection row not laid out as sinks, long-range keys, window
+};
+// debug_check_gather modes: bounds [0, T_cap) only; a selection row's layout
+// (positions from pos, window W, sinks S); layout with ascending long-range keys.
+enum DbgGather : int { DBG_BOUNDS = 0, DBG_SELECTION = 1, DBG_SELECTION_SORTED = 2 };
+bool debug_enabled();
+cudaError_t debug_check_index(const IndexView& ix, int64_t n_blk, cudaStream_t st, uint32_t out[4]);
+cudaError_t debug_check_gather(const int32_t* indices, const int32_t* counts, int64_t rows,
+                               int s_max, int64_t T_cap, PosSrc pos, int64_t Nq, int W, int S,
+                               int mode, cudaStream_t st, uint32_t out[4]);
+
 cudaError_t launch_attn(const void* Q, const void* K, const void* V, lsa_dtype dt, int64_t B,
                         int64_t Nq, int64_t T_cap, int Hq, int Hkv, int d,
                         const int32_t* indices, const int32_t* counts, int s_max, float scale,
