@@ -446,26 +446,30 @@ constexpr int MERGE_MAX_HEADS = 64;
 __global__ void __launch_bounds__(MERGE_THREADS) bucket_merge_kernel(BucketPlan P, int Hq, int D,
                                                                      __nv_bfloat16* O)
 {
-    __shared__ float w_s[MERGE_MAX_SLOTS * MERGE_MAX_HEADS];   // weights [slot][head], normalised
+    // (max, sum) per [slot][head]; the normalised weight then replaces the max
+    __shared__ float2 ml_s[MERGE_MAX_SLOTS * MERGE_MAX_HEADS];
     const int64_t row = blockIdx.x;
     const int nt = P.row_n[row];
     if (nt < 0) return;                        // gather row: written by the per-query kernel
     const int ns = nt + 1;
     const int64_t base = (int64_t)P.row_base[row] * Hq;   // first (slot, head)
     const float2* ml = P.part_ml + base;
-    // raw weights exp2(m) as pairs first: one pass per head over its slots
+    // every (slot, head) pair of the row in one coalesced pass
+    for (int x = threadIdx.x; x < ns * Hq; x += MERGE_THREADS) ml_s[x] = __ldcg(&ml[x]);
+    __syncthreads();
+    // weights exp2(m - M) * sum: one pass per head over its slots
     for (int h = threadIdx.x; h < Hq; h += MERGE_THREADS) {
         float M = -INFINITY;
-        for (int sl = 0; sl < ns; ++sl) M = fmaxf(M, __ldcg(&ml[(int64_t)sl * Hq + h]).x);
+        for (int sl = 0; sl < ns; ++sl) M = fmaxf(M, ml_s[sl * Hq + h].x);
         float L = 0.f;
         for (int sl = 0; sl < ns; ++sl) {
-            const float2 v = __ldcg(&ml[(int64_t)sl * Hq + h]);
+            const float2 v = ml_s[sl * Hq + h];
             const float wv = (v.x == -INFINITY) ? 0.f : v.y * exp2f(v.x - M);
-            w_s[sl * Hq + h] = wv;
+            ml_s[sl * Hq + h].x = wv;
             L += wv;
         }
         const float inv = 1.f / L;
-        for (int sl = 0; sl < ns; ++sl) w_s[sl * Hq + h] *= inv;
+        for (int sl = 0; sl < ns; ++sl) ml_s[sl * Hq + h].x *= inv;
     }
     __syncthreads();
     const int n8 = Hq * D / 8;                 // 16-byte groups of the row's output
@@ -479,7 +483,7 @@ __global__ void __launch_bounds__(MERGE_THREADS) bucket_merge_kernel(BucketPlan 
 #pragma unroll 4
         for (int sl = 0; sl < ns; ++sl) {
             const uint4 u = __ldcg(reinterpret_cast<const uint4*>(src + (int64_t)sl * Hq * D) + c);
-            const float wv = w_s[sl * Hq + h];
+            const float wv = ml_s[sl * Hq + h].x;
             const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {

@@ -10,6 +10,9 @@ lsa_prefill_chunk exactly as the benchmark calls it.  The oracle then checks
     the kernels rank with exact binary64 scores);
   * the outputs of 1024 rows, four in every 128-query tile of the
     tensor-core scorer, against the bf16 bars.
+Per-key indexer: the whole 10M chunk through lsa_select_per_key as
+bench.py's per_key measurement calls it, no fallback, and six rows spread over
+the chunk row for row against the oracle's per-key indexer.
 Decode: the benchmark's 8 x 1M decode runs once eagerly and is then captured
 in one CUDA graph and replayed twice, as bench.py does (it times the
 replays); every step's selection and output is checked against the oracle on
@@ -136,6 +139,23 @@ def test_full_size_prefill_chunk(name):
         errs.append(np.abs(got.astype(np.float64) - O_ref))
     err = np.concatenate(errs)
     assert err.max() <= BF16_MAX and err.mean() <= BF16_MEAN, (err.max(), err.mean())
+
+
+def test_full_size_per_key_indexer():
+    w = synth.workload("10m")
+    inp = synth.prefill_inputs(w, seed=0, device="cuda")
+    pos = inp["positions"].to(torch.int32).contiguous()
+    g_idx, g_cnt, ws = lsa.lsa_select_per_key(inp["latent_K"], inp["latent_Q"], pos, w.R, w.W,
+                                              w.S)
+    torch.cuda.synchronize()
+    assert lsa.lsa_select_per_key_check(ws) == 0
+    del ws
+    rows = np.array([0, 4099, 12345, 20001, 27777, w.nq - 1])
+    lat = inp["latent_K"][0].double().cpu().numpy()       # binary64 once, not per query
+    lq = inp["latent_Q"][0].float().cpu().numpy()[rows]
+    o_idx, o_cnt = oracle.select_per_key(lat, lq, pos[0].cpu().numpy()[rows], w.R, w.W, w.S)
+    assert np.array_equal(g_cnt[0].cpu().numpy()[rows], o_cnt)
+    assert np.array_equal(g_idx[0].cpu().numpy()[rows], o_idx)
 
 
 def test_full_size_decode_eager_and_graph_replays():
