@@ -4,8 +4,10 @@ lsa_select_per_key must equal oracle.select_per_key row for row (integer
 work with one correct answer: the R best long-range keys by exact binary64
 score, ties to the lower position, emitted with the sinks and the window):
   * contexts where every key is its own strided group and where 4 to 32 keys
-    share one; ragged query counts, positions from 0 to the last key, keys
-    past n_keys left unread, budgets 0, 1 and 4096, window 0;
+    share one; ragged query counts (and fewer than one 128-row tile),
+    positions from 0 to the last key, keys past n_keys left unread, budgets
+    0, 1 and 4096, window 0; positions outside the keys give empty rows and
+    LSA_ERR_INVALID_ARG from the check;
   * tied scores (identical latent keys): rows with more than 8192 candidates
     take the exact fallback (counted), the others rank ties in the final
     kernel, both to the lowest positions;
@@ -71,6 +73,7 @@ def _compare(lat, lq, pos, R, W, S, idx, cnt):
     (50000, 1, 130, 2048, 512, 4, 40000),    # T_cap not a power of two, keys past n_keys
     (20000, 1, 129, 1, 0, 0, None),          # budget 1, no window, no sinks
     (20000, 1, 64, 0, 512, 4, None),         # no long-range budget
+    (12000, 1, 20, 300, 64, 4, None),        # fewer query rows than one 128-row tile
 ])
 def test_per_key_matches_oracle(T, B, nq, R, W, S, n_keys):
     w, mix, lat = _latents(T, B, 64 if T <= 8192 else 1024, T + R)
@@ -82,6 +85,26 @@ def test_per_key_matches_oracle(T, B, nq, R, W, S, n_keys):
     idx, cnt, ws = _run(lat, lq, pos, R, W, S, n_keys=n_keys)
     assert lsa.lsa_select_per_key_check(ws) == 0
     _compare(lat, lq, pos, R, W, S, idx, cnt)
+
+
+def test_per_key_positions_outside_the_keys():
+    # a position at or past n_keys (or negative) reads nothing: its row is
+    # empty and the check reports LSA_ERR_INVALID_ARG; every other row is right
+    T, R, W, S, n_keys = 16384, 256, 64, 4, 12000
+    _, mix, lat = _latents(T, 1, 64, 23)
+    lq = _queries(mix, 140)
+    rng = np.random.default_rng(29)
+    pos = _positions(rng, 1, 140, 0, n_keys, [n_keys - 1, n_keys, T - 1, -5])
+    idx, cnt, ws = _run(lat, lq, pos, R, W, S, n_keys=n_keys)
+    with pytest.raises(lsa.LsaError, match="INVALID_ARG") as e:
+        lsa.lsa_select_per_key_check(ws)
+    assert e.value.code == 1
+    bad = (pos[0] < 0) | (pos[0] >= n_keys)
+    assert bad.sum() == 3 and (cnt[0][bad] == 0).all() and (idx[0][bad] == -1).all()
+    ok = np.nonzero(~bad)[0]
+    o_idx, o_cnt = oracle.select_per_key(lat[0].float().numpy(), lq[0].float().numpy()[ok],
+                                         pos[0][ok], R, W, S, s_max=idx.shape[-1])
+    assert np.array_equal(cnt[0][ok], o_cnt) and np.array_equal(idx[0][ok], o_idx)
 
 
 def test_per_key_ties_take_the_lowest_positions():
