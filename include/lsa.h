@@ -294,7 +294,7 @@ lsa_status lsa_tree_select(const lsa_index* idx, const void* tree, int n_super, 
  * ------------------------------------------------------------------------- */
 
 /* Workspace bytes for lsa_select_per_key (0 on bad sizes).  About
- * B*Nq*(2*min(32768, T_cap rounded up to a power of two) + 32 KiB + 12) bytes:
+ * B*Nq*(2*min(32768, max(256, T_cap rounded up to a power of two)) + 32 KiB + 12) bytes:
  * 3.1 GB for 32,768 queries of one 10M-key sequence. */
 size_t lsa_select_per_key_workspace_bytes(int64_t B, int64_t Nq, int64_t T_cap);
 

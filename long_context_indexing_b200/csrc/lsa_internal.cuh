@@ -343,7 +343,7 @@ struct PerKeyWs {
     int32_t* over;           // [rows] rows sent to the exact fallback
     uint16_t* gmax;          // [rows][ng] strided-group maxima (fp16 bits)
     int32_t* cand;           // [rows][PK_CAP] candidate positions
-    int64_t ng;              // groups per row (power of two, 128 .. PK_NG_MAX)
+    int64_t ng;              // groups per row (power of two, 256 .. PK_NG_MAX)
 };
 int64_t per_key_groups(int64_t T_cap);
 cudaError_t set_per_key_wait_polls(int64_t polls);

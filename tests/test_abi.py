@@ -245,3 +245,25 @@ def test_per_key_entry_argument_checks():
     odd = list(ok)
     odd[6] = ctypes.c_void_p((1 << 22) + 4)
     assert f(*odd) == 2                                  # LSA_ERR_ALIGNMENT
+
+
+def test_per_key_workspace_layout():
+    # rows x (2 B per strided group + 4 B per candidate slot of 8192 + three
+    # 4-byte words), the groups a power of two between 256 (one block of
+    # 256-key columns) and 32768 that covers T_cap, every array 256-byte
+    # aligned, plus the status and per-dimension maxima
+    def groups(T_cap):
+        ng = 256
+        while ng < T_cap and ng < 32768:
+            ng *= 2
+        return ng
+
+    def al(x):
+        return (x + 255) // 256 * 256
+
+    for B, Nq, T_cap in [(1, 1, 100), (1, 300, 5000), (2, 129, 8192), (1, 32768, 10485760),
+                         (3, 7, 40000)]:
+        rows = B * Nq
+        want = (256 + al(B * 64 * 4) + 3 * al(rows * 4) + al(rows * groups(T_cap) * 2)
+                + al(rows * 8192 * 4))
+        assert lsa._lib.lsa_select_per_key_workspace_bytes(B, Nq, T_cap) == want, (B, Nq, T_cap)
