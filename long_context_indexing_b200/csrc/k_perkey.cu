@@ -34,9 +34,10 @@
 //            eligible key scoring >= the threshold: every key of the exact
 //            top R is among them (its approximate score is >= its exact
 //            score - eps >= theta - 2 eps);
-//   final    (perkey_final_kernel, a CTA per row) sorts the candidates by
-//            position, ranks them by exact binary64 scores (radix select of
-//            the R-th largest) and emits the row;
+//   final    (perkey_final_kernel, a CTA per row) ranks the candidates by
+//            exact binary64 scores (radix select of the R-th largest (score,
+//            lower position) pair), sorts the R taken positions and emits the
+//            row;
 //   fallback (perkey_fallback_kernel) rows whose candidates overflowed the
 //            list (scores tied over more than PK_CAP keys) rank every
 //            eligible key exactly, recomputing the scores in each radix pass.
@@ -707,9 +708,13 @@ __global__ void __launch_bounds__(PT_THREADS) perkey_theta_kernel(PerKeyArgs a, 
 }
 
 // ---------------------------------------------------------------------------
-// final: a CTA per row.  Candidates sorted by position (bitonic), ranked by
-// exact scores (8-pass radix select of the R-th largest 64-bit key, ties to
-// the lower position), emitted with the sinks and the window.
+// final: a CTA per row.  The candidates' exact scores as ordered 64-bit keys;
+// the R-th largest (score key, inverted position) pair by radix select -- the
+// pairs are unique, so exactly R are at or above it, ties of the score going
+// to the lower position; the four position passes are skipped when the cut's
+// score is unique.  The R taken positions are compacted, sorted ascending
+// (bitonic over R rounded up to a power of two) and emitted with the sinks
+// and the window.
 // ---------------------------------------------------------------------------
 constexpr int PF_THREADS = 512;
 constexpr int PF_PER = PK_CAP / PF_THREADS;                 // 16 candidates per thread
@@ -728,6 +733,26 @@ __device__ __forceinline__ void pk_emit_edges(const PerKeyArgs& a, int64_t row, 
     for (int64_t x = threadIdx.x; x < n_w; x += blockDim.x) out[n_s + taken + x] = (int32_t)(w0 + x);
     for (int64_t x = n_s + taken + n_w + threadIdx.x; x < a.s_max; x += blockDim.x) out[x] = -1;
     if (threadIdx.x == 0) a.counts[row] = (int32_t)(n_s + taken + n_w);
+}
+
+// Bitonic sort of pos_s[0, P) ascending (P a power of two), whole CTA.
+__device__ __forceinline__ void pk_bitonic(int32_t* pos_s, int P)
+{
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int x = threadIdx.x; x < P / 2; x += PF_THREADS) {
+                const int lo = ((x & ~(j - 1)) << 1) | (x & (j - 1));   // j is a power of two
+                const int hi = lo + j;
+                const bool up = (lo & k) == 0;
+                const int32_t u = pos_s[lo], v = pos_s[hi];
+                if ((u > v) == up) {
+                    pos_s[lo] = v;
+                    pos_s[hi] = u;
+                }
+            }
+            __syncthreads();
+        }
+    }
 }
 
 __global__ void __launch_bounds__(PF_THREADS) perkey_final_kernel(PerKeyArgs a, PerKeyWs ws)
@@ -754,101 +779,97 @@ __global__ void __launch_bounds__(PF_THREADS) perkey_final_kernel(PerKeyArgs a, 
         }
         return;
     }
-    int P = 1;
-    while (P < n) P <<= 1;
     const int32_t* cand = ws.cand + row * PK_CAP;
-    for (int x = threadIdx.x; x < P; x += PF_THREADS) pos_s[x] = (x < n) ? cand[x] : 0x7FFFFFFF;
+    for (int x = threadIdx.x; x < n; x += PF_THREADS) pos_s[x] = cand[x];
     if (threadIdx.x < DL)
         q_s[threadIdx.x] = (double)__bfloat162float(
             reinterpret_cast<const __nv_bfloat16*>(a.lat_q)[row * DL + threadIdx.x]);
     __syncthreads();
-    // bitonic sort of the positions, ascending
-    for (int k = 2; k <= P; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int x = threadIdx.x; x < P / 2; x += PF_THREADS) {
-                const int lo = ((x & ~(j - 1)) << 1) | (x & (j - 1));   // j is a power of two
-                const int hi = lo + j;
-                const bool up = (lo & k) == 0;
-                const int32_t u = pos_s[lo], v = pos_s[hi];
-                if ((u > v) == up) {
-                    pos_s[lo] = v;
-                    pos_s[hi] = u;
-                }
-            }
-            __syncthreads();
+    int taken = n;
+    if (n > a.R) {
+        // exact scores as ordered keys, two rows in flight per thread
+        const __nv_bfloat16* lat =
+            reinterpret_cast<const __nv_bfloat16*>(a.lat_k) + b * a.T_cap * DL;
+        for (int x = threadIdx.x; x < n; x += 2 * PF_THREADS) {
+            const int y = x + PF_THREADS;
+            double sx, sy;
+            pk_exact2(q_s, lat + (int64_t)pos_s[x] * DL, lat + (int64_t)pos_s[y < n ? y : x] * DL,
+                      &sx, &sy);
+            key_s[x] = pk_dkey(sx);
+            if (y < n) key_s[y] = pk_dkey(sy);
         }
-    }
-    // exact scores as ordered keys
-    const __nv_bfloat16* lat = reinterpret_cast<const __nv_bfloat16*>(a.lat_k) + b * a.T_cap * DL;
-    for (int x = threadIdx.x; x < n; x += 2 * PF_THREADS) {
-        const int y = x + PF_THREADS;
-        double sx, sy;
-        pk_exact2(q_s, lat + (int64_t)pos_s[x] * DL, lat + (int64_t)pos_s[y < n ? y : x] * DL, &sx, &sy);
-        key_s[x] = pk_dkey(sx);
-        if (y < n) key_s[y] = pk_dkey(sy);
-    }
-    __syncthreads();
-    // the R-th largest key, and how many equal keys are taken (lowest positions)
-    uint64_t cut = 0ull;
-    uint32_t need = 0u;
-    const bool all = n <= a.R;
-    if (!all) {
-        uint64_t prefix = 0ull, mask = 0ull;
+        __syncthreads();
+        // the R-th largest (key, ~position) pair: 8 passes over the key bytes,
+        // then, unless the cut's key is unique among the rest, 4 over the
+        // inverted position's bytes
+        uint64_t kp = 0ull, km = 0ull;
+        uint32_t ip = 0u, im = 0u;
         uint32_t want = (uint32_t)a.R;
-        for (int pass = 0; pass < 8; ++pass) {
-            const int sh = 56 - 8 * pass;
+        for (int pass = 0; pass < 12; ++pass) {
+            const bool on_key = pass < 8;
+            const int sh = on_key ? 56 - 8 * pass : 24 - 8 * (pass - 8);
             for (int x = threadIdx.x; x < 256; x += PF_THREADS) hist[x] = 0u;
             __syncthreads();
             for (int x = threadIdx.x; x < n; x += PF_THREADS) {
                 const uint64_t k = key_s[x];
-                if ((k & mask) == prefix) atomicAdd(&hist[(k >> sh) & 255u], 1u);
+                if (on_key) {
+                    if ((k & km) == kp) atomicAdd(&hist[(k >> sh) & 255u], 1u);
+                } else if (k == kp) {
+                    const uint32_t v = 0xFFFFFFFFu - (uint32_t)pos_s[x];
+                    if ((v & im) == ip) atomicAdd(&hist[(v >> sh) & 255u], 1u);
+                }
             }
             __syncthreads();
             int bin;
             uint32_t above;
             pk_hist_pick<PF_THREADS>(hist, want, &bin, &above, bc);
-            prefix |= (uint64_t)(uint32_t)bin << sh;
-            mask |= 255ull << sh;
+            const uint32_t in_bin = hist[bin];
             want -= above;
+            if (on_key) {
+                kp |= (uint64_t)(uint32_t)bin << sh;
+                km |= 255ull << sh;
+            } else {
+                ip |= (uint32_t)bin << sh;
+                im |= 255u << sh;
+            }
+            __syncthreads();                   // hist read before the next pass clears it
+            if (pass == 7 && in_bin == want) break;    // every pair with the cut's key is taken
         }
-        cut = prefix;
-        need = want;
-    }
-    // taken flags in position order: thread t owns candidates [PF_PER t, PF_PER t + PF_PER)
-    const int x0 = threadIdx.x * PF_PER;
-    int eq = 0;
-    if (!all) {
+        // compaction of the taken positions (pairs at or above the cut)
+        int32_t mine[PF_PER];
+        uint32_t fl = 0u;
+        int nt = 0;
+        const int x0 = threadIdx.x * PF_PER;
+#pragma unroll
         for (int e = 0; e < PF_PER; ++e) {
             const int x = x0 + e;
-            if (x < n && key_s[x] == cut) ++eq;
-        }
-    }
-    int tot;
-    int eq_before = all ? 0 : pk_block_scan<PF_THREADS>(eq, scan, &tot);
-    uint32_t fl = 0u;
-    int nt = 0;
-    for (int e = 0; e < PF_PER; ++e) {
-        const int x = x0 + e;
-        bool take = false;
-        if (x < n) {
-            if (all) take = true;
-            else {
+            mine[e] = 0;
+            if (x < n) {
                 const uint64_t k = key_s[x];
-                if (k > cut) take = true;
-                else if (k == cut) take = (uint32_t)(eq_before++) < need;
+                const int32_t t = pos_s[x];
+                const bool take = k > kp || (k == kp && (0xFFFFFFFFu - (uint32_t)t) >= ip);
+                mine[e] = t;
+                if (take) {
+                    fl |= 1u << e;
+                    ++nt;
+                }
             }
         }
-        if (take) {
-            fl |= 1u << e;
-            ++nt;
-        }
+        int o = pk_block_scan<PF_THREADS>(nt, scan, &taken);   // syncs before pos_s is rewritten
+#pragma unroll
+        for (int e = 0; e < PF_PER; ++e)
+            if (fl & (1u << e)) pos_s[o++] = mine[e];
+        __syncthreads();
     }
+    // the taken positions ascending, then the row
+    int P = 1;
+    while (P < taken) P <<= 1;
+    for (int x = taken + threadIdx.x; x < P; x += PF_THREADS) pos_s[x] = 0x7FFFFFFF;
+    __syncthreads();
+    pk_bitonic(pos_s, P);
     const int n_s = (int)(p >= 0 ? (p + 1 < a.S ? p + 1 : a.S) : 0);
-    int taken;
-    int o = pk_block_scan<PF_THREADS>(nt, scan, &taken);
     int32_t* out = a.indices + row * (int64_t)a.s_max + n_s;
-    for (int e = 0; e < PF_PER; ++e)
-        if (fl & (1u << e)) out[o++] = pos_s[x0 + e];
+    for (int x = threadIdx.x; x < taken; x += PF_THREADS) out[x] = pos_s[x];
     pk_emit_edges(a, row, p, taken);
 }
 
