@@ -18,8 +18,10 @@
 //             inside [S, pos - W] (and ascending for the per-key indexer).
 // A violation is recorded in a library-owned device word (first one wins:
 // kind, sequence or row, place, value); the host reads it after a stream
-// synchronisation and clears it.  No check traps or faults: a check that
-// finds a bad offset skips the reads it would have guarded.
+// synchronisation and clears it.  The word is one per device: checks that
+// run at the same time on several streams or threads share it, so a debug
+// session serialises its calls.  No check traps or faults: a check that finds
+// a bad offset skips the reads it would have guarded.
 #include "lsa_internal.cuh"
 
 namespace lsa {
