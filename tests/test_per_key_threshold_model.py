@@ -13,7 +13,9 @@ This test checks the claim with numpy, independently of the kernels, on
 approximations pushed to the worst case the bound allows (every top-R key
 scored eps too low, every other key eps too high) and on clustered keys,
 scores beyond fp16's range, scores in its subnormals and tied scores; and that
-on the clustered mixture the kept set stays within the 8192-entry list.
+on the clustered mixture the kept set stays within the 8192-entry list.  In
+the pushed cases one eligible key of large entries and a very low score makes
+eps dominate fp16's rounding, so that both eps of the margin are needed.
 """
 import zlib
 
@@ -59,7 +61,7 @@ def _kept(lat, q, pos, ng, push):
     return keep, top
 
 
-@pytest.mark.parametrize("case", ["mixture", "mixture_push", "large", "tiny", "ties"])
+@pytest.mark.parametrize("case", ["mixture", "mixture_push", "large", "tiny", "ties", "ties_push"])
 def test_kept_keys_hold_the_exact_top_r(case):
     rng = np.random.default_rng(zlib.crc32(case.encode()))
     T, ng = 40000, 4096
@@ -68,9 +70,12 @@ def test_kept_keys_hold_the_exact_top_r(case):
         q = (q * 4.0e5).astype(np.float32)          # group maxima beyond fp16's range
     elif case == "tiny":
         q = (q * 1.0e-5).astype(np.float32)         # group maxima among fp16 subnormals
-    elif case == "ties":
+    elif case in ("ties", "ties_push"):
         lat[:] = lat[:1]                            # every score equal
-    push = case != "mixture"
+    push = case in ("mixture_push", "ties_push")
+    if push:
+        # a key of 50s, scoring far below every other: eps grows ~50x
+        lat[S + 10] = (-50.0 * np.sign(q)).astype(np.float32)
     for pos in (T - 1, T // 2, W + S + R + 5):
         keep, top = _kept(lat, q, pos, ng, push)
         assert keep[top].all(), (case, pos)
