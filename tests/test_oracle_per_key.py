@@ -114,3 +114,17 @@ def test_recall_counts_long_range_keys_only():
     sel = np.array([[0, 1, 10, 30, 50, 95, 96, -1]], np.int32)
     r = oracle.recall(sel, np.array([7]), ref, np.array([7]), np.array([96]), 2, 2)
     assert r[0] == pytest.approx(2 / 3)                      # 10 and 30 of {10, 20, 30}
+
+
+def test_hand_worked_cases():
+    # tests/golden/per_key_hand.json: rows worked by hand from the definition
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "per_key_hand.json")))
+    lat = np.array(g["latent_K"], np.float32)
+    for c in g["cases"]:
+        s_max = c["R"] + c["W"] + c["S"]
+        idx, cnt = oracle.select_per_key(lat, np.array([c["q"]], np.float32), np.array([c["pos"]]),
+                                         c["R"], c["W"], c["S"], s_max=s_max)
+        assert idx[0, :cnt[0]].tolist() == c["row"], c["derivation"]
+        assert np.all(idx[0, cnt[0]:] == -1)
